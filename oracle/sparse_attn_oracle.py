@@ -1,0 +1,264 @@
+"""CPU oracle for block-sparse attention with a cumulative-energy block mask.
+
+TEST INFRASTRUCTURE ONLY. This file is the plain, slow, fp64 statement of what the
+GPU path computes. Only the tests, the package's smoke check and the benchmark's
+CPU-baseline / reference arm may import it; the product path never does. It
+shares no code with the CUDA library (it does not import the package).
+
+What it follows:
+  * SpargeAttn abstract (page "taxoreview ... dblp:344/2858", repeated in the HF
+    Daily Papers listing): a two-stage online filter. Stage 1 predicts the
+    attention map cheaply and skips the matmuls of unimportant regions; stage 2 is
+    an online-softmax-aware filter that skips further matmuls at no extra cost.
+  * "Training-free sparse attention based on cumulative energy filtering"
+    (DynSparse news article, method paragraph): keep tokens until a fixed recall of
+    the attention energy is reached, with a per-row ("dynamic") threshold derived
+    from the cumulative energy instead of a fixed top-k budget or static cut.
+
+Readings where the pages are silent (each is also listed in the design notes):
+  * stage 1 pools Q and K by the mean over blocks of 64 tokens; a ragged last block
+    is averaged over its valid tokens only;
+  * pooled logits use the same softmax scale as the attention;
+  * causal: only key blocks j <= i enter the pooled softmax of query block i;
+  * selection: sort the row of pooled probabilities in descending order (ties:
+    lower block index first), keep the shortest prefix whose running sum reaches
+    tau times the row total;
+  * stage 2: inside the tiled online-softmax loop (64-row query blocks, kept key
+    blocks visited in ascending order), the P.V product of a key block is skipped
+    when every valid row r of the query block has rowmax_r(S_blk) - m_r < lam,
+    with m_r the running max before the block; the block still enters the
+    running max and the running sum l (only P.V is skipped).
+  * a query row that ends with no visible key gets an output of zero.
+
+Arithmetic is fp64 throughout; inputs are the exact values of the bf16 tensors.
+
+Entry points: block_mean_pool, pooled_logits, pooled_softmax,
+cumulative_energy_select, plan, attention_masked, attention_tiled, fwd.
+"""
+from __future__ import annotations
+
+import math
+from typing import Iterable, Optional
+
+import numpy as np
+
+BLOCK = 64
+
+
+def as_f64(x) -> np.ndarray:
+    """Exact fp64 copy of a (possibly bf16 torch) array."""
+    if hasattr(x, "detach"):  # torch tensor, any dtype; bf16 -> fp32 -> fp64 is exact
+        x = x.detach().to("cpu")
+        if str(x.dtype) == "torch.bfloat16":
+            x = x.float()
+        x = x.numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def n_blocks(N: int, block: int = BLOCK) -> int:
+    return -(-N // block)
+
+
+# ---------------------------------------------------------------- stage 1
+
+def block_mean_pool(X: np.ndarray, block: int = BLOCK) -> np.ndarray:
+    """Mean of each block of `block` consecutive tokens: [..., N, d] -> [..., Nb, d].
+
+    Stage 1 of the SpargeAttn abstract ("rapidly ... predict the attention map");
+    the pooling operator is the mean (reading). A ragged tail block divides by its
+    own token count."""
+    N = X.shape[-2]
+    Nb = n_blocks(N, block)
+    out = np.empty(X.shape[:-2] + (Nb, X.shape[-1]), dtype=np.float64)
+    for i in range(Nb):
+        s, e = i * block, min(N, (i + 1) * block)
+        out[..., i, :] = X[..., s:e, :].sum(axis=-2) / (e - s)
+    return out
+
+
+def pooled_logits(Qp: np.ndarray, Kp: np.ndarray, scale: float, causal: bool) -> np.ndarray:
+    """L[i, j] = scale * <Qp_i, Kp_j>; with causal, key blocks after the query block
+    are excluded (-inf)."""
+    L = scale * np.matmul(Qp, np.swapaxes(Kp, -1, -2))
+    if causal:
+        Nb = L.shape[-1]
+        later = np.triu(np.ones((Nb, Nb), dtype=bool), k=1)
+        L = np.where(later, -np.inf, L)
+    return L
+
+
+def pooled_softmax(L: np.ndarray) -> np.ndarray:
+    """Row softmax of the pooled logits: the predicted block attention map."""
+    m = L.max(axis=-1, keepdims=True)
+    e = np.exp(L - m)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def cumulative_energy_select(P: np.ndarray, tau: float):
+    """Per row of the predicted map, keep the fewest blocks whose energy reaches tau.
+
+    DynSparse (cumulative energy filtering): a fixed recall of the attention energy
+    is kept, and the per-row cut-off value (the smallest kept probability) is the
+    dynamic threshold. Steps: sort descending with ties to the lower index (stable
+    sort of -p), running sum c_r, first r with c_r >= tau * c_last, keep that prefix.
+
+    Returns mask (uint8, [..., Nb, Nb]), count (int64 [..., Nb]), idx (int64,
+    ascending kept indices, padded with -1) and, per block in its original
+    position, the row's running sum just before (`c_before`) and after (`c_after`)
+    that block in sorted order, normalised by the row total; these mark the blocks
+    whose fate is decided within rounding of tau.
+    """
+    shape = P.shape
+    rows = P.reshape(-1, shape[-1])
+    Nb = shape[-1]
+    mask = np.zeros(rows.shape, dtype=np.uint8)
+    count = np.zeros(rows.shape[0], dtype=np.int64)
+    idx = np.full(rows.shape, -1, dtype=np.int64)
+    c_before = np.zeros(rows.shape, dtype=np.float64)
+    c_after = np.zeros(rows.shape, dtype=np.float64)
+    for r in range(rows.shape[0]):
+        p = rows[r]
+        order = np.argsort(-p, kind="stable")
+        c = np.cumsum(p[order])
+        total = c[-1]
+        hit = np.nonzero(c >= tau * total)[0]
+        rstar = int(hit[0]) + 1 if hit.size else Nb
+        kept = np.sort(order[:rstar])
+        mask[r, kept] = 1
+        count[r] = rstar
+        idx[r, :rstar] = kept
+        c_after[r, order] = c / total
+        c_before[r, order] = (c - p[order]) / total
+    return (mask.reshape(shape), count.reshape(shape[:-1]), idx.reshape(shape),
+            c_before.reshape(shape), c_after.reshape(shape))
+
+
+def plan(Q, K, tau: float, scale: Optional[float] = None, causal: bool = False,
+         block: int = BLOCK) -> dict:
+    """Stage 1 end to end: pool, pooled logits, pooled softmax, cumulative-energy
+    selection. Q, K: [B, H, N, d]."""
+    Q = as_f64(Q)
+    K = as_f64(K)
+    d = Q.shape[-1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    Qp = block_mean_pool(Q, block)
+    Kp = block_mean_pool(K, block)
+    L = pooled_logits(Qp, Kp, scale, causal)
+    P = pooled_softmax(L)
+    mask, count, idx, cb, ca = cumulative_energy_select(P, tau)
+    return dict(Qp=Qp, Kp=Kp, L=L, P=P, mask=mask, count=count, idx=idx,
+                c_before=cb, c_after=ca)
+
+
+# ---------------------------------------------------------------- stage 2
+
+def _visible(mask_row: np.ndarray, N: int, block: int) -> np.ndarray:
+    """Token-level key visibility of one query block from its block-mask row."""
+    vis = np.repeat(mask_row.astype(bool), block)[:N]
+    return vis
+
+
+def attention_masked(Q, K, V, mask, scale: Optional[float] = None, causal: bool = False,
+                     block: int = BLOCK, qblocks: Optional[Iterable[int]] = None):
+    """Stage-2 output without the lambda filter: for each query token t, softmax
+    attention over the keys of the blocks its query block keeps (and s <= t when
+    causal). Returns O [B, H, N, d] (rows of query blocks not in `qblocks` are NaN)."""
+    Q, K, V = as_f64(Q), as_f64(K), as_f64(V)
+    mask = np.asarray(mask)
+    B, H, N, d = Q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    Nb = n_blocks(N, block)
+    qbs = range(Nb) if qblocks is None else qblocks
+    O = np.full((B, H, N, V.shape[-1]), np.nan)
+    for b in range(B):
+        for h in range(H):
+            for i in qbs:
+                s, e = i * block, min(N, (i + 1) * block)
+                vis = _visible(mask[b, h, i], N, block)
+                S = scale * Q[b, h, s:e] @ K[b, h].T           # [rows, N]
+                allow = np.broadcast_to(vis, S.shape).copy()
+                if causal:
+                    allow &= np.arange(N)[None, :] <= np.arange(s, e)[:, None]
+                S = np.where(allow, S, -np.inf)
+                m = S.max(axis=1, keepdims=True)
+                none = ~np.isfinite(m[:, 0])
+                m[none] = 0.0
+                W = np.exp(S - m)
+                lsum = W.sum(axis=1, keepdims=True)
+                out = (W @ V[b, h]) / np.where(lsum > 0, lsum, 1.0)
+                out[none] = 0.0
+                O[b, h, s:e] = out
+    return O
+
+
+def attention_tiled(Q, K, V, mask, lam: float, scale: Optional[float] = None,
+                    causal: bool = False, block: int = BLOCK,
+                    qblocks: Optional[Iterable[int]] = None, return_stats: bool = False):
+    """Stage 2 with the online-softmax-aware filter, as a literal fp64 run of the
+    tiled loop: per 64-row query block, kept key blocks in ascending order,
+    running max m, running sum l, accumulator O.
+
+    SpargeAttn abstract, second stage: a block whose P.V contribution is
+    negligible under the current running max is skipped at no extra cost. The
+    test is rowmax_r(S_blk) - m_r < lam for every row r of the query block that
+    sees at least one key of the block (m_r before the block, natural-log units
+    of the scaled logits); only P.V is skipped, m and l are still updated.
+    lam = -inf never skips, and then this equals attention_masked."""
+    Q, K, V = as_f64(Q), as_f64(K), as_f64(V)
+    mask = np.asarray(mask)
+    B, H, N, d = Q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    Nb = n_blocks(N, block)
+    qbs = range(Nb) if qblocks is None else qblocks
+    O = np.full((B, H, N, V.shape[-1]), np.nan)
+    kept_pairs = 0
+    skipped_pairs = 0
+    for b in range(B):
+        for h in range(H):
+            for i in qbs:
+                s, e = i * block, min(N, (i + 1) * block)
+                rows = np.arange(s, e)
+                m = np.full(e - s, -np.inf)
+                l = np.zeros(e - s)
+                acc = np.zeros((e - s, V.shape[-1]))
+                for j in np.nonzero(mask[b, h, i])[0]:
+                    ks, ke = j * block, min(N, (j + 1) * block)
+                    S = scale * Q[b, h, s:e] @ K[b, h, ks:ke].T
+                    if causal:
+                        S = np.where(np.arange(ks, ke)[None, :] <= rows[:, None], S, -np.inf)
+                    rmax = S.max(axis=1)
+                    sees = np.isfinite(rmax)
+                    if not sees.any():
+                        continue
+                    kept_pairs += 1
+                    with np.errstate(invalid="ignore"):
+                        diff = rmax - m                      # +inf where m = -inf
+                    skip = bool(np.all(diff[sees] < lam))
+                    m_new = np.maximum(m, rmax)
+                    ref = np.where(np.isfinite(m_new), m_new, 0.0)
+                    alpha = np.where(np.isfinite(m), np.exp(m - ref), 0.0)
+                    Pb = np.exp(S - ref[:, None])
+                    l = l * alpha + Pb.sum(axis=1)
+                    acc = acc * alpha[:, None]
+                    if skip:
+                        skipped_pairs += 1
+                    else:
+                        acc = acc + Pb @ V[b, h, ks:ke]
+                    m = m_new
+                out = acc / np.where(l > 0, l, 1.0)[:, None]
+                out[l <= 0] = 0.0
+                O[b, h, s:e] = out
+    if return_stats:
+        return O, dict(kept_pairs=kept_pairs, pv_skipped=skipped_pairs)
+    return O
+
+
+def fwd(Q, K, V, mask, lam: Optional[float] = None, scale: Optional[float] = None,
+        causal: bool = False, block: int = BLOCK, qblocks=None):
+    """Stage 2: the masked attention, with the lambda filter when lam is finite."""
+    if lam is None or lam == -math.inf:
+        return attention_masked(Q, K, V, mask, scale, causal, block, qblocks)
+    return attention_tiled(Q, K, V, mask, lam, scale, causal, block, qblocks)

@@ -1,0 +1,294 @@
+"""Pins of the CPU oracle to facts outside itself (no GPU).
+
+Each test checks the oracle against something it does not compute itself: a
+closed form, a library routine, brute force on tiny inputs, hand-worked cases, or
+an invariant of the definition; chosen so that a dropped term, a wrong index, a
+transposed operand or a wrong tie rule fails at least one of them.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+from scipy.special import softmax as scipy_softmax
+
+from oracle import sparse_attn_oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ------------------------------------------------------------------ pooling + logits
+
+@pytest.mark.parametrize("N", [1, 63, 64, 65, 200, 256])
+def test_pool_is_block_average_of_token_logits(N):
+    """Bilinearity: scale * <mean Q_blk i, mean K_blk j> equals the mean of the
+    n_i x n_j block of full-resolution scaled logits (ragged tail included)."""
+    r = _rng(N)
+    d = 8
+    Q = r.standard_normal((2, 3, N, d))
+    K = r.standard_normal((2, 3, N, d))
+    scale = 0.37
+    L = orc.pooled_logits(orc.block_mean_pool(Q), orc.block_mean_pool(K), scale, False)
+    S = scale * np.einsum("bhnd,bhmd->bhnm", Q, K)
+    starts = np.arange(0, N, 64)
+    Sr = np.add.reduceat(np.add.reduceat(S, starts, axis=2), starts, axis=3)
+    sizes = np.minimum(starts + 64, N) - starts
+    ref = Sr / (sizes[:, None] * sizes[None, :])
+    np.testing.assert_allclose(L, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_pool_closed_form_row_index():
+    """Rows equal to their token index: block mean = (first + last) / 2, tail too."""
+    N = 150
+    X = np.repeat(np.arange(N, dtype=np.float64)[:, None], 3, axis=1)[None, None]
+    P = orc.block_mean_pool(X)
+    expect = [(0 + 63) / 2, (64 + 127) / 2, (128 + 149) / 2]
+    np.testing.assert_array_equal(P[0, 0, :, 0], expect)
+
+
+def test_causal_pooled_logits_exclude_later_blocks():
+    r = _rng(1)
+    Qp = r.standard_normal((1, 1, 5, 4))
+    L = orc.pooled_logits(Qp, Qp, 1.0, True)
+    assert np.all(np.isneginf(L[0, 0][np.triu_indices(5, 1)]))
+    assert np.all(np.isfinite(L[0, 0][np.tril_indices(5)]))
+
+
+# ------------------------------------------------------------------ softmax
+
+def test_pooled_softmax_matches_library():
+    r = _rng(2)
+    L = 3.0 * r.standard_normal((2, 3, 7, 7))
+    np.testing.assert_allclose(orc.pooled_softmax(L), scipy_softmax(L, axis=-1), rtol=1e-13)
+    Lc = orc.pooled_logits(r.standard_normal((1, 1, 6, 3)), r.standard_normal((1, 1, 6, 3)), 1.0, True)
+    P = orc.pooled_softmax(Lc)
+    np.testing.assert_allclose(P.sum(-1), 1.0, rtol=1e-14)
+    assert np.all(P[0, 0][np.triu_indices(6, 1)] == 0.0)
+
+
+# ------------------------------------------------------------------ selection
+
+def test_select_golden_hand_worked():
+    with open(os.path.join(GOLDEN, "select_cases.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        p = np.array(c["p"], dtype=np.float64)[None]
+        mask, count, idx, cb, ca = orc.cumulative_energy_select(p, c["tau"])
+        assert int(count[0]) == c["count"], c
+        assert list(idx[0, : c["count"]]) == c["idx"], c
+        assert list(np.nonzero(mask[0])[0]) == c["idx"], c
+        assert np.all(idx[0, c["count"]:] == -1)
+        # the running sums in sorted order are the hand-worked ones
+        order = np.argsort(-p[0], kind="stable")
+        np.testing.assert_array_equal(ca[0, order], c["running"])
+
+
+def test_select_end_to_end_constructed_inputs():
+    """Q rows all (1,0); K block j rows all (ln p_j, 0); scale 1: the pooled map of
+    every query block is p exactly, so the plan must keep the hand-worked set
+    {1, 2, 3} at tau = 0.9 for p = (1/16, 8/16, 2/16, 5/16). A ragged last block
+    (8 tokens) must not change that."""
+    p = np.array([1 / 16, 8 / 16, 2 / 16, 5 / 16])
+    for N in (256, 200):
+        Q = np.zeros((1, 1, N, 2)); Q[..., 0] = 1.0
+        K = np.zeros((1, 1, N, 2))
+        for j in range(4):
+            K[0, 0, j * 64:min(N, (j + 1) * 64), 0] = math.log(p[j])
+        out = orc.plan(Q, K, 0.9, scale=1.0)
+        np.testing.assert_allclose(out["P"][0, 0], np.tile(p, (4, 1)), rtol=1e-14)
+        assert np.all(out["mask"][0, 0] == np.array([0, 1, 1, 1]))
+        assert np.all(out["count"][0, 0] == 3)
+
+
+@pytest.mark.parametrize("Nb", [1, 2, 3, 5, 8, 10])
+def test_select_minimal_cardinality_brute_force(Nb):
+    """The kept count equals the smallest size of ANY subset reaching tau of the
+    row total (enumerated), and the kept set has the largest sum among sets of
+    that size."""
+    r = _rng(Nb)
+    for trial in range(25):
+        p = r.dirichlet(np.full(Nb, 0.6))
+        tau = float(r.uniform(0.3, 0.999))
+        mask, count, idx, _, _ = orc.cumulative_energy_select(p[None], tau)
+        best = None
+        best_sum_at_k = {}
+        for k in range(1, Nb + 1):
+            sums = [sum(p[list(s)]) for s in itertools.combinations(range(Nb), k)]
+            best_sum_at_k[k] = max(sums)
+            if best is None and best_sum_at_k[k] >= tau * p.sum() - 1e-15:
+                best = k
+        assert int(count[0]) == best
+        kept_sum = p[mask[0].astype(bool)].sum()
+        assert kept_sum >= tau * p.sum() - 1e-15
+        assert abs(kept_sum - best_sum_at_k[best]) < 1e-12
+
+
+def test_select_invariants_random_rows():
+    r = _rng(7)
+    P = orc.pooled_softmax(2.5 * r.standard_normal((3, 4, 40, 40)))
+    for tau in (0.5, 0.9, 0.95, 0.99):
+        mask, count, idx, cb, ca = orc.cumulative_energy_select(P, tau)
+        kept = mask.astype(bool)
+        e = np.where(kept, P, 0).sum(-1)
+        assert np.all(e >= tau - 1e-12)                       # recall reached
+        smallest = np.where(kept, P, np.inf).min(-1)
+        assert np.all(e - smallest < tau + 1e-12)             # minimal
+        assert np.array_equal(kept.sum(-1), count)
+        # idx ascending, consistent with the mask
+        for flat in range(0, 3 * 4 * 40, 37):
+            b, h, i = np.unravel_index(flat, count.shape)
+            row = idx[b, h, i, : count[b, h, i]]
+            assert np.all(np.diff(row) > 0)
+            assert np.array_equal(row, np.nonzero(mask[b, h, i])[0])
+
+
+def test_select_special_cases():
+    Nb = 12
+    # tau = 1 keeps every block with positive energy
+    r = _rng(3)
+    p = r.dirichlet(np.ones(Nb))
+    mask, count, *_ = orc.cumulative_energy_select(p[None], 1.0)
+    assert count[0] == Nb
+    # one-hot row keeps one block
+    oh = np.zeros(Nb); oh[5] = 1.0
+    mask, count, idx, *_ = orc.cumulative_energy_select(oh[None], 0.9)
+    assert count[0] == 1 and idx[0, 0] == 5
+    # uniform row: tau = (k - 1/2)/Nb keeps k blocks, the lowest indices (ties)
+    u = np.full(Nb, 1.0 / Nb)
+    for k in range(1, Nb + 1):
+        mask, count, idx, *_ = orc.cumulative_energy_select(u[None], (k - 0.5) / Nb)
+        assert count[0] == k
+        assert list(idx[0, :k]) == list(range(k))
+
+
+# ------------------------------------------------------------------ attention
+
+def _sdpa64(Q, K, V, causal, scale):
+    q, k, v = (torch.from_numpy(np.ascontiguousarray(x)) for x in (Q, K, V))
+    return torch.nn.functional.scaled_dot_product_attention(
+        q, k, v, is_causal=causal, scale=scale).numpy()
+
+
+@pytest.mark.parametrize("N,causal", [(64, False), (200, False), (130, True), (256, True), (1, False)])
+def test_full_mask_equals_library_dense_attention(N, causal):
+    """tau = 1 through the whole oracle (plan + fwd, lambda off) reproduces the
+    library's dense fp64 attention."""
+    r = _rng(N)
+    d = 16
+    Q = r.standard_normal((2, 2, N, d))
+    K = r.standard_normal((2, 2, N, d))
+    V = r.standard_normal((2, 2, N, d))
+    scale = 1 / math.sqrt(d)
+    pl = orc.plan(Q, K, 1.0, scale, causal)
+    Nb = orc.n_blocks(N)
+    full = np.ones((Nb, Nb), dtype=np.uint8)
+    if causal:
+        full = np.tril(full)
+    assert np.array_equal(pl["mask"], np.broadcast_to(full, pl["mask"].shape))
+    O = orc.fwd(Q, K, V, pl["mask"], None, scale, causal)
+    np.testing.assert_allclose(O, _sdpa64(Q, K, V, causal, scale), rtol=1e-11, atol=1e-12)
+    O2 = orc.attention_tiled(Q, K, V, pl["mask"], -math.inf, scale, causal)
+    np.testing.assert_allclose(O2, _sdpa64(Q, K, V, causal, scale), rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("N,causal", [(300, False), (257, True)])
+def test_tiled_recurrence_equals_masked_softmax(N, causal):
+    """With lambda = -inf the tiled online-softmax loop equals the direct masked
+    softmax on a random block mask (pins the recurrence: rescale, running sum)."""
+    r = _rng(N + 1)
+    d = 8
+    Q, K, V = (r.standard_normal((1, 2, N, d)) * 2 for _ in range(3))
+    Nb = orc.n_blocks(N)
+    mask = (r.random((1, 2, Nb, Nb)) < 0.5).astype(np.uint8)
+    mask[..., np.arange(Nb), np.arange(Nb)] = 1
+    a = orc.attention_masked(Q, K, V, mask, None, causal)
+    b = orc.attention_tiled(Q, K, V, mask, -math.inf, None, causal)
+    np.testing.assert_allclose(a, b, rtol=1e-11, atol=1e-13)
+
+
+def _two_block_case(first_logit, second_logit):
+    N, d = 128, 2
+    Q = np.zeros((1, 1, N, d)); Q[..., 0] = 1.0
+    K = np.zeros((1, 1, N, d))
+    K[0, 0, :64, 0] = first_logit
+    K[0, 0, 64:, 0] = second_logit
+    V = np.zeros((1, 1, N, d))
+    V[0, 0, :64, 0] = 1.0
+    V[0, 0, 64:, 1] = 1.0
+    mask = np.ones((1, 1, 2, 2), dtype=np.uint8)
+    return Q, K, V, mask
+
+
+def test_lambda_skip_closed_form():
+    """Scores 0 on key block 0 and -20 on key block 1 (visited second). Off or
+    lam = -25: O = (1, e^-20)/(1 + e^-20). lam = -12: P.V of block 1 is skipped
+    but it stays in the running sum: O = (1, 0)/(1 + e^-20)."""
+    Q, K, V, mask = _two_block_case(0.0, -20.0)
+    t = math.exp(-20.0)
+    O_off = orc.fwd(Q, K, V, mask, None, 1.0)
+    O_25, st25 = orc.attention_tiled(Q, K, V, mask, -25.0, 1.0, return_stats=True)
+    O_12, st12 = orc.attention_tiled(Q, K, V, mask, -12.0, 1.0, return_stats=True)
+    np.testing.assert_allclose(O_off[0, 0], np.tile([1 / (1 + t), t / (1 + t)], (128, 1)), rtol=1e-14)
+    np.testing.assert_allclose(O_25, O_off, rtol=1e-14, atol=0)
+    np.testing.assert_allclose(O_12[0, 0], np.tile([1 / (1 + t), 0.0], (128, 1)), rtol=1e-14, atol=0)
+    assert st12 == dict(kept_pairs=4, pv_skipped=2) and st25["pv_skipped"] == 0
+
+
+def test_lambda_first_block_never_skipped_and_order_matters():
+    """Block 0 at -20, block 1 at 0: the low block comes first (running max -inf,
+    never skipped) and block 1 raises the max; nothing is skipped at any lam."""
+    Q, K, V, mask = _two_block_case(-20.0, 0.0)
+    O_off = orc.fwd(Q, K, V, mask, None, 1.0)
+    O_lam, st = orc.attention_tiled(Q, K, V, mask, -1.0, 1.0, return_stats=True)
+    assert st["pv_skipped"] == 0
+    np.testing.assert_allclose(O_lam, O_off, rtol=1e-14)
+
+
+def test_lambda_error_bounded_by_skipped_mass():
+    """Skipping only P.V leaves l unchanged, so per row
+    O_lam - O_off = -(sum of skipped P V) / l, whose size is at most
+    (skipped P mass / l) * max|V|; every skipped entry is below e^lam times the
+    running max's weight (1), and l >= 1. Inputs: key block 0 aligned with
+    every query, the other blocks pure noise, so later blocks fall below lam."""
+    r = _rng(11)
+    N, d = 512, 16
+    u = np.ones(d)
+    Q = 2.0 * u + 0.3 * r.standard_normal((1, 2, N, d))
+    K = r.standard_normal((1, 2, N, d))
+    K[:, :, :64] = 2.0 * u + 0.3 * r.standard_normal((1, 2, 64, d))
+    V = r.standard_normal((1, 2, N, d))
+    Nb = orc.n_blocks(N)
+    mask = np.ones((1, 2, Nb, Nb), dtype=np.uint8)
+    lam = -8.0
+    O_off = orc.attention_masked(Q, K, V, mask)
+    O_lam, st = orc.attention_tiled(Q, K, V, mask, lam, return_stats=True)
+    assert st["pv_skipped"] == 2 * Nb * (Nb - 1)          # every non-aligned block
+    assert np.abs(O_lam - O_off).max() > 0
+    bound = np.abs(V).max() * (Nb - 1) * 64 * math.exp(lam)
+    assert np.abs(O_lam - O_off).max() <= bound
+
+
+def test_row_without_visible_key_is_zero():
+    r = _rng(5)
+    Q, K, V = (r.standard_normal((1, 1, 128, 4)) for _ in range(3))
+    mask = np.zeros((1, 1, 2, 2), dtype=np.uint8)
+    mask[0, 0, 1, 1] = 1
+    O = orc.attention_masked(Q, K, V, mask)
+    assert np.all(O[0, 0, :64] == 0)
+    O2 = orc.attention_tiled(Q, K, V, mask, -5.0)
+    assert np.all(O2[0, 0, :64] == 0)
+    np.testing.assert_allclose(O[0, 0, 64:], O2[0, 0, 64:], rtol=1e-12)
+
+
+def test_bf16_inputs_are_upcast_exactly():
+    x = torch.randn(3, 5).to(torch.bfloat16)
+    y = orc.as_f64(x)
+    assert y.dtype == np.float64
+    assert np.array_equal(y, x.float().numpy().astype(np.float64))
