@@ -1,0 +1,380 @@
+#!/usr/bin/env python
+"""Benchmark of the block-sparse attention path (stage 1 plan + stage 2 forward).
+
+One step = sparse_attn_plan + sparse_attn_fwd over one batch of resident bf16
+Q/K/V of the chosen workload (default: the small DiT-layer shape, B=1 H=24 N=4096
+d=128, tau=0.95, lambda=-12). Prints ONE JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload small|tiny|wan|hunyuan|lm]
+                    [--tau T] [--lam L|off] [--impl ours|reference]
+
+Multi-GPU: the path has no exchange step; N ranks run N independent replicas of
+the same workload (weak scaling), timed on the device, max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from free_block_sparse_mean_b200 import workloads as wl  # noqa: E402
+
+METRIC = "sparse attn ms/call & dense-equiv TFLOPS at τ; sparsity %; % of BF16 peak"
+UNIT = "TFLOP/s dense-equivalent"
+L2_BYTES = 126 * 1024 * 1024
+FLUSH_BYTES = 512 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="small", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--tau", type=float, default=0.95)
+    ap.add_argument("--lam", default="-12")
+    ap.add_argument("--centroid-weight", type=float, default=None)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def lam_value(s):
+    return None if s in ("off", "none", "None", "-inf") else float(s)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def dense_flops(w):
+    if w.causal:
+        return 2.0 * w.B * w.H * w.N * (w.N + 1) * w.D
+    return 4.0 * w.B * w.H * w.N * w.N * w.D
+
+
+# --------------------------------------------------------------------------- dist
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=timedelta(seconds=120))
+        pg = dist
+    return world, rank, local, pg
+
+
+def reduce_max(pg, x: float, device) -> float:
+    if pg is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(pg, device=None):
+    if pg is not None:
+        if device is not None and device.type == "cuda":
+            pg.barrier(device_ids=[device.index])
+        else:
+            pg.barrier()
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"sa_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+            os.remove(self.path)
+        except Exception:
+            return None
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = max(float(r[2]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        loaded = [x for x in sm if x > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- CPU oracle timing
+def time_oracle(w, tau, lam, budget_s, seed):
+    """The oracle as it stands (fp64 NumPy) on a bounded sample of the workload:
+    whole heads (plan + forward) until the time budget is used, at least one."""
+    from oracle import sparse_attn_oracle as orc
+    try:
+        import threadpoolctl
+        cores = max(v.get("num_threads", 1) for v in threadpoolctl.threadpool_info()) or os.cpu_count()
+    except Exception:
+        cores = os.cpu_count()
+    per_head_dense = dense_flops(w) / (w.B * w.H)
+    if w.N > 8192:
+        qblocks = list(range(0, -(-w.N // 64), max(1, (-(-w.N // 64)) // 16)))[:16]
+    else:
+        qblocks = None
+    t_total = 0.0
+    flops = 0.0
+    heads = 0
+    for h in range(w.H):
+        q, k, v = wl.generate(w, seed=seed, device="cpu", heads=[h])
+        t0 = time.perf_counter()
+        p = orc.plan(q, k, tau, None, w.causal)
+        orc.fwd(q, k, v, p["mask"], lam, None, w.causal, qblocks=qblocks)
+        dt = time.perf_counter() - t0
+        t_total += dt
+        nb = -(-w.N // 64)
+        frac = 1.0 if qblocks is None else len(qblocks) / nb
+        # attention part scales with the sampled query blocks; plan is whole-head
+        flops += per_head_dense * frac
+        heads += 1
+        if t_total >= budget_s:
+            break
+    sample = (f"{heads} of {w.H} heads, full plan"
+              + ("" if qblocks is None else f", forward on {len(qblocks)} of {-(-w.N // 64)} query blocks"))
+    return flops / t_total / 1e12, t_total, cores, sample
+
+
+# --------------------------------------------------------------------------- main arms
+def run_reference(args, w, world, rank, pg):
+    lam = lam_value(args.lam)
+    if rank != 0:
+        return
+    per_step = []
+    vals = []
+    budget = max(2.0, min(args.cpu_seconds, 240.0 / max(1, args.steps + args.warmup)))
+    for i in range(args.warmup + args.steps):
+        v, t, cores, sample = time_oracle(w, args.tau, lam, budget, args.seed)
+        if i >= args.warmup:
+            per_step.append(t)
+            vals.append(v)
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.median(per_step),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_dict(w, args, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(w, args, world):
+    return {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.D} block=64 "
+                        f"{'causal' if w.causal else 'non-causal'}",
+            "tau": args.tau, "lambda": lam_value(args.lam), "seq_len": w.N, "heads": w.H, "head_dim": w.D,
+            "global_batch": w.B * world, "parallelism": f"replicas{world}",
+            "l2": "flushed between timed steps" if 3 * w.B * w.H * w.N * w.D * 2 < 2 * L2_BYTES
+            else "inputs larger than L2 (flushed too)",
+            "centroid_weight": args.centroid_weight}
+
+
+def run_ours(args, w, world, rank, local, pg):
+    import free_block_sparse_mean_b200 as sa
+    if not torch.cuda.is_available():
+        raise RuntimeError("no CUDA device: the benchmark needs a B200")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    lam = lam_value(args.lam)
+    q, k, v = wl.generate(w, seed=args.seed, device=dev, centroid_weight=args.centroid_weight)
+    torch.cuda.synchronize()
+    B, H, N, D = w.B, w.H, w.N, w.D
+    Nb = -(-N // 64)
+    # buffers reused by every step (resident, allocated once)
+    plan = sa.sparse_attn_plan(q, k, args.tau, None, w.causal, with_idx=False)
+    ws = torch.empty(sa.sparse_attn_plan_workspace_size(B, H, N, D), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False)
+        sa.sparse_attn_fwd(q, k, v, plan, lam, out=out)
+
+    # stats (outside timing): kept pairs, skipped P.V, algorithmic FLOPs of the forward
+    stats = torch.zeros(4, dtype=torch.int64, device=dev)
+    sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False)
+    sa.sparse_attn_fwd(q, k, v, plan, lam, out=out, stats=stats)
+    torch.cuda.synchronize()
+    st = [int(x) for x in stats.cpu()]
+    n_tok = torch.full((Nb,), 64, dtype=torch.float64, device=dev)
+    n_tok[-1] = N - 64 * (Nb - 1)
+    m = plan.mask.to(torch.float64)
+    if w.causal:
+        m = m * torch.tril(torch.ones(Nb, Nb, dtype=torch.float64, device=dev))
+    pair_tokens = float(torch.einsum("bhij,i,j->", m, n_tok, n_tok))   # sum over kept pairs n_i n_j
+    kept_pairs = float(m.sum())
+    total_pairs = B * H * (Nb * (Nb + 1) / 2 if w.causal else Nb * Nb)
+    skipped = st[1]
+    avg_pair_tokens = pair_tokens / max(kept_pairs, 1)
+    exec_flops = 2.0 * D * pair_tokens + 2.0 * D * avg_pair_tokens * (kept_pairs - skipped)
+    dflops = dense_flops(w)
+
+    # dense reference time of our own kernel (full mask), for the predictor budget
+    full = torch.ones((B, H, Nb, Nb), dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        sa.sparse_attn_fwd(q, k, v, full, None, out=out, causal=w.causal)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flush.zero_()
+    e0.record(stream)
+    sa.sparse_attn_fwd(q, k, v, full, None, out=out, causal=w.causal)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dense_ms = e0.elapsed_time(e1)
+    del full
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    barrier(pg, dev)
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        flush.zero_()                       # L2 flush, outside the timed events
+        a, b, c = ev[i]
+        a.record(stream)
+        sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False)
+        b.record(stream)
+        sa.sparse_attn_fwd(q, k, v, plan, lam, out=out)
+        c.record(stream)
+    torch.cuda.synchronize()
+    barrier(pg, dev)
+    clocks = sampler.stop()
+    plan_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    fwd_ms = [b.elapsed_time(c) for _, b, c in ev]
+    step_ms_local = sum(p + f for p, f in zip(plan_ms, fwd_ms)) / args.steps
+    step_ms = reduce_max(pg, step_ms_local, dev)
+    value = world * dflops / (step_ms * 1e-3) / 1e12
+    fwd_avg = statistics.mean(fwd_ms)
+    plan_avg = statistics.mean(plan_ms)
+
+    # end to end through the public API from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+        for _ in range(2):
+            sa.sparse_attention(qh, kh, vh, args.tau, lam, None, w.causal, device=dev)
+        torch.cuda.synchronize()
+        barrier(pg, dev)
+        t = []
+        for _ in range(max(3, min(args.steps, 10))):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            o_host = sa.sparse_attention(qh, kh, vh, args.tau, lam, None, w.causal, device=dev)
+            b.record(stream)
+            torch.cuda.synchronize()
+            t.append(a.elapsed_time(b))
+        e2e_ms = reduce_max(pg, statistics.mean(t), dev)
+        e2e = {"value": world * dflops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "ms_per_call": e2e_ms,
+               "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": o_host.numel() * 2}
+        del qh, kh, vh
+
+    pk, pk_kind = peaks()
+    peak_t = float(pk["bf16_tflops"])
+    achieved = exec_flops / (fwd_avg * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded cluster-centroid generator)",
+        "config": config_dict(w, args, world),
+        "plan_ms": plan_avg, "fwd_ms": fwd_avg, "dense_fwd_ms": dense_ms,
+        "sparsity_pct": 100.0 * (1.0 - kept_pairs / total_pairs),
+        "lambda_skip_pct": 100.0 * skipped / max(kept_pairs, 1),
+        "executed_tflops": achieved, "pct_of_bf16_peak_executed": 100.0 * achieved / peak_t,
+        "predictor_pct_of_dense": 100.0 * plan_avg / dense_ms,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": achieved / peak_t, "traffic": None,
+                     "kernel": "fwd_kernel<128,3> (sparse_attn_fwd)",
+                     "peak_source": f"{pk_kind} bf16_tflops (burst)"},
+        "e2e": e2e, "gpu_launches": 4 * args.steps, "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu:
+        v_cpu, t_cpu, cores, sample = time_oracle(w, args.tau, lam, args.cpu_seconds, args.seed)
+        line["cpu_baseline"] = {"value": v_cpu, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": sample, "seconds": t_cpu}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    w = wl.WORKLOADS[args.workload]
+    world, rank, local, pg = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, w, world, rank, pg)
+        else:
+            run_ours(args, w, world, rank, local, pg)
+    finally:
+        if pg is not None:
+            pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,181 @@
+"""B200 (sm_100a) block-sparse attention: cumulative-energy block mask + sparse forward.
+
+Thin binding over the C ABI (include/sparse_attn.h): every call below only checks
+and marshals torch tensors into pointers and sizes, then calls the library, which
+runs all the work in its CUDA kernels on the tensors' device and the current
+torch stream. PyTorch provides device memory and streams, nothing else.
+
+    plan = sparse_attn_plan(q, k, tau=0.95)            # stage 1: block mask
+    o = sparse_attn_fwd(q, k, v, plan, lam=-12.0)      # stage 2: sparse attention
+
+q, k, v: bf16 CUDA tensors [B, H, N, d], contiguous, d in {64, 128}.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import SaShape, SparseAttnError
+
+BLOCK = 64
+
+__all__ = ["Plan", "sparse_attn_plan", "sparse_attn_fwd", "sparse_attention",
+           "sparse_attn_plan_workspace_size", "sparse_attn_num_tiles", "sparse_attn_device_error",
+           "SparseAttnError", "BLOCK"]
+
+
+def _shape(q: torch.Tensor) -> SaShape:
+    B, H, N, d = q.shape
+    return SaShape(B, H, N, d, BLOCK)
+
+
+def _check_qkv(*ts: torch.Tensor):
+    q = ts[0]
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must be CUDA tensors")
+        if t.dtype != torch.bfloat16:
+            raise ValueError("tensors must be bf16")
+        if t.dim() != 4 or t.shape != q.shape:
+            raise ValueError("q, k, v must share the shape [B, H, N, d]")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous [B, H, N, d]")
+        if t.device != q.device:
+            raise ValueError("tensors must be on one device")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _call(name: str, status: int):
+    if status != _lib.SA_OK:
+        raise SparseAttnError(name, status, _lib.load())
+
+
+@dataclass
+class Plan:
+    """Output of sparse_attn_plan (all on the inputs' device).
+
+    mask  uint8 [B, H, Nb, Nb]  1 = kept key block
+    count int32 [B, H, Nb]      kept blocks per query block
+    idx   int32 [B, H, Nb, Nb]  ascending kept blocks in the first count entries
+                                of each row (rest of the row undefined), or None
+    work  int32 [num_tiles]     tile order for sparse_attn_fwd, or None
+    """
+    mask: torch.Tensor
+    count: torch.Tensor
+    idx: Optional[torch.Tensor]
+    work: Optional[torch.Tensor]
+    tau: float
+    causal: bool
+
+
+def sparse_attn_plan_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(_lib.load().sparse_attn_plan_workspace_size(SaShape(B, H, N, d, BLOCK)))
+
+
+def sparse_attn_num_tiles(B: int, H: int, N: int, d: int) -> int:
+    return int(_lib.load().sparse_attn_num_tiles(SaShape(B, H, N, d, BLOCK)))
+
+
+def sparse_attn_plan(q: torch.Tensor, k: torch.Tensor, tau: float, scale: Optional[float] = None,
+                     causal: bool = False, *, with_idx: bool = True, with_work: bool = True,
+                     out: Optional[Plan] = None, workspace: Optional[torch.Tensor] = None) -> Plan:
+    """Stage 1: cumulative-energy block mask from mean-pooled q and k."""
+    lib = _lib.load()
+    _check_qkv(q, k)
+    B, H, N, d = q.shape
+    Nb = -(-N // BLOCK)
+    s = _shape(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dev = q.device
+    if out is None:
+        out = Plan(
+            mask=torch.empty((B, H, Nb, Nb), dtype=torch.uint8, device=dev),
+            count=torch.empty((B, H, Nb), dtype=torch.int32, device=dev),
+            idx=torch.empty((B, H, Nb, Nb), dtype=torch.int32, device=dev) if with_idx else None,
+            work=torch.empty((max(1, lib.sparse_attn_num_tiles(s)),), dtype=torch.int32, device=dev)
+            if with_work else None,
+            tau=float(tau), causal=bool(causal))
+    else:
+        out.tau, out.causal = float(tau), bool(causal)
+    ws_bytes = int(lib.sparse_attn_plan_workspace_size(s))
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty((max(ws_bytes, 256),), dtype=torch.uint8, device=dev)
+    st = lib.sparse_attn_plan(_ptr(q), _ptr(k), s, float(tau), float(scale), int(bool(causal)),
+                              _ptr(out.mask), _ptr(out.count), _ptr(out.idx), _ptr(out.work),
+                              _ptr(workspace), ws_bytes, _stream(dev))
+    _call("sparse_attn_plan", st)
+    return out
+
+
+def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan, lam: Optional[float] = None,
+                    scale: Optional[float] = None, causal: Optional[bool] = None, *,
+                    out: Optional[torch.Tensor] = None, stats: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Stage 2: attention over the kept blocks with the lambda P.V filter.
+
+    `plan` is a Plan or a uint8 mask [B, H, Nb, Nb]. lam=None turns the filter off.
+    `stats`, if given, is an int64 CUDA tensor of 4 entries (see the C header)."""
+    lib = _lib.load()
+    _check_qkv(q, k, v)
+    B, H, N, d = q.shape
+    Nb = -(-N // BLOCK)
+    if isinstance(plan, Plan):
+        mask, work = plan.mask, plan.work
+        if causal is None:
+            causal = plan.causal
+    else:
+        mask, work = plan, None
+    causal = bool(causal)
+    if mask.dtype != torch.uint8 or tuple(mask.shape) != (B, H, Nb, Nb) or not mask.is_contiguous() \
+            or mask.device != q.device:
+        raise ValueError("mask must be a contiguous uint8 tensor [B, H, Nb, Nb] on q's device")
+    if work is not None and (work.dtype != torch.int32 or work.device != q.device):
+        raise ValueError("work must be int32 on q's device")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    lam_f = -math.inf if lam is None else float(lam)
+    if out is None:
+        out = torch.empty_like(q)
+    if stats is not None and (stats.dtype != torch.int64 or stats.numel() < 4 or stats.device != q.device):
+        raise ValueError("stats must be an int64 tensor of >= 4 entries on q's device")
+    st = lib.sparse_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _shape(q), _ptr(mask), _ptr(work), lam_f,
+                             float(scale), int(causal), _ptr(out), _ptr(stats), _stream(q.device))
+    _call("sparse_attn_fwd", st)
+    return out
+
+
+def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float,
+                     lam: Optional[float] = None, scale: Optional[float] = None, causal: bool = False,
+                     device="cuda") -> torch.Tensor:
+    """End to end from host tensors: copy q, k, v to the GPU, plan + forward, copy O back.
+
+    Host inputs should be pinned for overlap; the result is a host bf16 tensor."""
+    dev = torch.device(device)
+    qd = q.to(dev, non_blocking=True)
+    kd = k.to(dev, non_blocking=True)
+    vd = v.to(dev, non_blocking=True)
+    plan = sparse_attn_plan(qd, kd, tau, scale, causal, with_idx=False)
+    od = sparse_attn_fwd(qd, kd, vd, plan, lam, scale, causal)
+    return od.to("cpu")
+
+
+def sparse_attn_device_error(device=None) -> int:
+    """Read and clear the device error word (0 = no device-side check fired)."""
+    lib = _lib.load()
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    code = ctypes.c_int32(0)
+    with torch.cuda.device(dev):
+        _call("sparse_attn_device_error", lib.sparse_attn_device_error(_stream(dev), ctypes.byref(code)))
+    return int(code.value)

@@ -1,0 +1,77 @@
+"""ctypes loader for the C ABI in include/sparse_attn.h (libsparse_attn.so).
+
+No fallback: if the library is missing the import of the calls fails loudly."""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsparse_attn.so")
+
+SA_OK = 0
+STATUS_NAMES = {
+    0: "SA_OK",
+    1: "SA_ERR_INVALID_ARG",
+    2: "SA_ERR_UNSUPPORTED",
+    3: "SA_ERR_WORKSPACE",
+    4: "SA_ERR_CUDA",
+    5: "SA_ERR_DEVICE_CHECK",
+}
+
+# Every symbol include/sparse_attn.h declares.
+EXPORTS = (
+    "sparse_attn_plan_workspace_size",
+    "sparse_attn_num_tiles",
+    "sparse_attn_plan",
+    "sparse_attn_fwd",
+    "sparse_attn_status_string",
+    "sparse_attn_device_error",
+)
+
+
+class SaShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32),
+                ("d", ctypes.c_int32), ("block", ctypes.c_int32)]
+
+
+class SparseAttnError(RuntimeError):
+    def __init__(self, call: str, status: int, lib=None):
+        msg = STATUS_NAMES.get(status, f"status {status}")
+        if lib is not None:
+            try:
+                msg = lib.sparse_attn_status_string(status).decode()
+            except Exception:  # pragma: no cover - message only
+                pass
+        super().__init__(f"{call} failed: {msg}")
+        self.status = status
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load the shared library once and declare the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(
+            f"CUDA library not built: {path} is missing (run __graft_entry__.build() or "
+            "python -m free_block_sparse_mean_b200.build)")
+    lib = ctypes.CDLL(path)
+    vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    lib.sparse_attn_plan_workspace_size.argtypes = [SaShape]
+    lib.sparse_attn_plan_workspace_size.restype = sz
+    lib.sparse_attn_num_tiles.argtypes = [SaShape]
+    lib.sparse_attn_num_tiles.restype = ctypes.c_int64
+    lib.sparse_attn_plan.argtypes = [vp, vp, SaShape, f32, f32, i32, vp, vp, vp, vp, vp, sz, vp]
+    lib.sparse_attn_plan.restype = i32
+    lib.sparse_attn_fwd.argtypes = [vp, vp, vp, SaShape, vp, vp, f32, f32, i32, vp, vp, vp]
+    lib.sparse_attn_fwd.restype = i32
+    lib.sparse_attn_status_string.argtypes = [i32]
+    lib.sparse_attn_status_string.restype = ctypes.c_char_p
+    lib.sparse_attn_device_error.argtypes = [vp, ctypes.POINTER(i32)]
+    lib.sparse_attn_device_error.restype = i32
+    _lib = lib
+    return lib

@@ -1,0 +1,281 @@
+// Stage 1 kernels: block mean pooling, pooled scores + cumulative-energy
+// selection, and the per-head tile order.
+//
+// Stage 1 of the two-stage filter in the SpargeAttn abstract predicts the
+// attention map cheaply; the kept set per query block is the one the DynSparse
+// article ("Training-free sparse attention based on cumulative energy
+// filtering") describes: a fixed recall of attention energy, i.e. a per-row
+// threshold derived from the cumulative energy.
+#pragma once
+
+#include "sa_device.cuh"
+
+namespace sa {
+
+// ----------------------------------------------------------------------------
+// Pool: Xp[bh, i, :] = mean of X[bh, 64 i : min(N, 64 i + 64), :], fp32.
+// One CTA per (block, head) and per tensor (blockIdx.y: 0 = Q, 1 = K). Each
+// thread loads 16-byte vectors (8 bf16) of a row; D/8 threads cover a row, so a
+// warp reads whole rows contiguously. Partial sums meet in shared memory.
+// HBM-bound: it is the one full pass over Q and K on the predictor side.
+template <int D>
+__global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ Q,
+                                                   const __nv_bfloat16* __restrict__ K,
+                                                   float* __restrict__ Qp, float* __restrict__ Kp,
+                                                   int N, int Nb) {
+  constexpr int LPR = D / 8;          // threads per row
+  constexpr int RPP = 256 / LPR;      // rows per pass
+  __shared__ float part[RPP][D];
+  const long long g = blockIdx.x;     // (bh, i) flattened
+  const long long bh = g / Nb;
+  const int i = static_cast<int>(g - bh * Nb);
+  const __nv_bfloat16* src = (blockIdx.y == 0 ? Q : K) + (bh * N + static_cast<long long>(i) * kBlock) * D;
+  float* dst = (blockIdx.y == 0 ? Qp : Kp) + g * D;
+  const int rows = min(kBlock, N - i * kBlock);
+  const int r0 = threadIdx.x / LPR;
+  const int c8 = (threadIdx.x % LPR) * 8;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+  for (int p = 0; p < kBlock / RPP; ++p) {
+    const int r = r0 + p * RPP;
+    if (r < rows) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(src + static_cast<long long>(r) * D + c8));
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h[e]);
+        acc[2 * e] += f.x;
+        acc[2 * e + 1] += f.y;
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) part[r0][c8 + e] = acc[e];
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float s = 0.f;
+#pragma unroll
+    for (int r = 0; r < RPP; ++r) s += part[r][threadIdx.x];
+    dst[threadIdx.x] = s / static_cast<float>(rows);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Pooled scores + selection. One CTA = R query blocks of one head.
+//
+// Phase 1 (CUDA-core fp32 GEMM, the pooled scores must stay fp32 to keep the
+// kept set stable near tau): thread t owns key blocks c = 2t, 2t+1 of each
+// 512-wide pass and all R rows; the R pooled query rows sit in shared memory
+// (transposed, read as broadcast float4), Kp rows stream from L2 in 32-byte
+// pieces. Scores go to shared memory: L[r][j] = scale * <Qp_r, Kp_j>, -inf for
+// causal j > i.
+//
+// Phase 2 (one warp per row): e_j = exp(L_j - max), T = tau * sum e. The kept set
+// is {j : e_j > e*} plus the lowest-index ties at e* needed to reach T, where
+// e* is the largest value with sum_{e_j >= e*} e_j >= T. e* is found by bisection
+// on the IEEE bit pattern of e (monotone for non-negative floats); every probe
+// sums in the same order as the total, so the probe at 0 equals the total
+// exactly. This is the sorted-prefix rule without sorting.
+template <int D, int R>
+__global__ void __launch_bounds__(256) score_select_kernel(const float* __restrict__ Qp,
+                                                           const float* __restrict__ Kp, int Nb,
+                                                           float scale, int causal, float tau,
+                                                           uint8_t* __restrict__ mask,
+                                                           int* __restrict__ count,
+                                                           int* __restrict__ idx) {
+  static_assert(R % 4 == 0 && R <= 16, "R rows per CTA");
+  constexpr int QS = R + 4;  // padded row stride of the transposed query tile
+  extern __shared__ __align__(16) float sm[];
+  float* qT = sm;                          // [D][QS]
+  float* L = sm + D * QS;                  // [R][ldL]
+  const int ldL = (Nb + 3) & ~3;
+  const long long bh = blockIdx.y;
+  const int i0 = blockIdx.x * R;
+  const float* qp = Qp + bh * Nb * D;
+  const float* kp = Kp + bh * Nb * D;
+
+  for (int e = threadIdx.x; e < R * D; e += blockDim.x) {
+    const int r = e / D, k = e % D;
+    qT[k * QS + r] = (i0 + r < Nb) ? qp[static_cast<long long>(i0 + r) * D + k] : 0.f;
+  }
+  __syncthreads();
+
+  // ---------------- phase 1: scores
+  for (int cb = 0; cb < Nb; cb += 512) {
+    const int c0 = cb + 2 * threadIdx.x;
+    float acc0[R], acc1[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc0[r] = acc1[r] = 0.f;
+    if (c0 < Nb) {
+      const bool has1 = c0 + 1 < Nb;
+      const float4* k0 = reinterpret_cast<const float4*>(kp + static_cast<long long>(c0) * D);
+      const float4* k1 = reinterpret_cast<const float4*>(kp + static_cast<long long>(has1 ? c0 + 1 : c0) * D);
+#pragma unroll 2
+      for (int k = 0; k < D; k += 8) {
+        float4 a[2], b[2];
+        a[0] = __ldg(k0 + k / 4);
+        a[1] = __ldg(k0 + k / 4 + 1);
+        b[0] = __ldg(k1 + k / 4);
+        b[1] = __ldg(k1 + k / 4 + 1);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const float av = reinterpret_cast<const float*>(a)[kk];
+          const float bv = reinterpret_cast<const float*>(b)[kk];
+          const float4* qrow = reinterpret_cast<const float4*>(qT + (k + kk) * QS);
+#pragma unroll
+          for (int r4 = 0; r4 < R / 4; ++r4) {
+            const float4 q = qrow[r4];
+            acc0[4 * r4 + 0] = fmaf(q.x, av, acc0[4 * r4 + 0]);
+            acc0[4 * r4 + 1] = fmaf(q.y, av, acc0[4 * r4 + 1]);
+            acc0[4 * r4 + 2] = fmaf(q.z, av, acc0[4 * r4 + 2]);
+            acc0[4 * r4 + 3] = fmaf(q.w, av, acc0[4 * r4 + 3]);
+            acc1[4 * r4 + 0] = fmaf(q.x, bv, acc1[4 * r4 + 0]);
+            acc1[4 * r4 + 1] = fmaf(q.y, bv, acc1[4 * r4 + 1]);
+            acc1[4 * r4 + 2] = fmaf(q.z, bv, acc1[4 * r4 + 2]);
+            acc1[4 * r4 + 3] = fmaf(q.w, bv, acc1[4 * r4 + 3]);
+          }
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int i = i0 + r;
+        float v0 = acc0[r] * scale, v1 = acc1[r] * scale;
+        if (causal) {
+          if (c0 > i) v0 = -INFINITY;
+          if (c0 + 1 > i) v1 = -INFINITY;
+        }
+        if (has1) {
+          *reinterpret_cast<float2*>(L + r * ldL + c0) = make_float2(v0, v1);
+        } else {
+          L[r * ldL + c0] = v0;
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---------------- phase 2: selection, one warp per row
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned FULL = 0xffffffffu;
+  const float LOG2E = 1.4426950408889634f;
+  for (int r = warp; r < R; r += 8) {
+    const int i = i0 + r;
+    if (i >= Nb) break;
+    float* row = L + r * ldL;
+    float m = -INFINITY;
+    for (int j = lane; j < Nb; j += 32) m = fmaxf(m, row[j]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
+    // e_j in place; the row max maps to exactly 1.
+    float tot = 0.f;
+    uint32_t kmax = 0;
+    for (int j = lane; j < Nb; j += 32) {
+      const float e = ex2((row[j] - m) * LOG2E);
+      row[j] = e;
+      tot += e;
+      kmax = max(kmax, __float_as_uint(e));
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      tot += __shfl_xor_sync(FULL, tot, o);
+      kmax = max(kmax, __shfl_xor_sync(FULL, kmax, o));
+    }
+    __syncwarp();
+    uint32_t K;          // key (bit pattern) of the cut-off value e*
+    int need_ties;       // how many ties at e* are kept (lowest indices first)
+    if (tau >= 1.f) {
+      K = 1u;            // every block with e_j > 0 (finite score) is kept
+      need_ties = 0x7fffffff;
+    } else {
+      const float T = tau * tot;
+      uint32_t lo = 0u, hi = kmax + 1u;   // S(lo) >= T > S(hi)
+      while (hi - lo > 1u) {
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        float s = 0.f;
+        for (int j = lane; j < Nb; j += 32) {
+          const float e = row[j];
+          s += (__float_as_uint(e) >= mid) ? e : 0.f;
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(FULL, s, o);
+        if (s >= T) lo = mid; else hi = mid;
+      }
+      K = lo;
+      float sgt = 0.f;
+      int nties = 0;
+      for (int j = lane; j < Nb; j += 32) {
+        const uint32_t kj = __float_as_uint(row[j]);
+        sgt += (kj > K) ? row[j] : 0.f;
+        nties += (kj == K);
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        sgt += __shfl_xor_sync(FULL, sgt, o);
+        nties += __shfl_xor_sync(FULL, nties, o);
+      }
+      const float eK = __uint_as_float(K);
+      float acc = sgt;
+      need_ties = 0;
+      do {
+        acc += eK;
+        ++need_ties;
+      } while (acc < T && need_ties < nties);
+    }
+    // emit mask, ascending idx, count
+    uint8_t* mrow = mask + (bh * Nb + i) * static_cast<long long>(Nb);
+    int* irow = idx ? idx + (bh * Nb + i) * static_cast<long long>(Nb) : nullptr;
+    int kept = 0, ties_seen = 0;
+    for (int jb = 0; jb < Nb; jb += 32) {
+      const int j = jb + lane;
+      uint32_t kj = 0u;
+      if (j < Nb) kj = __float_as_uint(row[j]);
+      const bool tie = (j < Nb) && (kj == K);
+      const unsigned tb = __ballot_sync(FULL, tie);
+      const int my_tie_rank = ties_seen + __popc(tb & ((1u << lane) - 1u));
+      const bool keep = (j < Nb) && (kj > K || (tie && my_tie_rank < need_ties));
+      ties_seen += __popc(tb);
+      const unsigned kb = __ballot_sync(FULL, keep);
+      if (j < Nb) mrow[j] = keep ? 1 : 0;
+      if (irow && keep) irow[kept + __popc(kb & ((1u << lane) - 1u))] = j;
+      kept += __popc(kb);
+    }
+    if (lane == 0) count[bh * Nb + i] = kept;
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Tile order: for each head, a counting sort of its Tq query tiles by decreasing
+// cost = count[2t] + count[2t+1]. Heads stay in ascending order so that the
+// tiles running at the same time share one head's K/V in L2.
+__global__ void __launch_bounds__(1024) tile_order_kernel(const int* __restrict__ count, int Nb, int Tq,
+                                                          int* __restrict__ work) {
+  extern __shared__ int hist[];  // [2*Nb + 1]
+  const int nbins = 2 * Nb + 1;
+  const long long bh = blockIdx.x;
+  const int* cnt = count + bh * Nb;
+  for (int c = threadIdx.x; c < nbins; c += blockDim.x) hist[c] = 0;
+  __syncthreads();
+  for (int t = threadIdx.x; t < Tq; t += blockDim.x) {
+    const int c = cnt[2 * t] + ((2 * t + 1 < Nb) ? cnt[2 * t + 1] : 0);
+    atomicAdd(&hist[min(max(c, 0), nbins - 1)], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {  // exclusive scan from the top bin down (nbins <= 8193)
+    int run = 0;
+    for (int c = nbins - 1; c >= 0; --c) {
+      const int h = hist[c];
+      hist[c] = run;
+      run += h;
+    }
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < Tq; t += blockDim.x) {
+    const int c = cnt[2 * t] + ((2 * t + 1 < Nb) ? cnt[2 * t + 1] : 0);
+    const int pos = atomicAdd(&hist[min(max(c, 0), nbins - 1)], 1);
+    work[bh * Tq + pos] = static_cast<int>(bh * Tq + t);
+  }
+}
+
+}  // namespace sa

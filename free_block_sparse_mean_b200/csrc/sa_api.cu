@@ -1,0 +1,209 @@
+// C ABI of the block-sparse attention library: argument checks, workspace
+// layout, TMA descriptors and launches. The kernels are in plan_kernels.cuh and
+// fwd_kernel.cuh; everything is compiled as this one translation unit.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/sparse_attn.h"
+#include "fwd_kernel.cuh"
+#include "plan_kernels.cuh"
+
+namespace {
+
+constexpr int kFwdStages = 3;
+
+inline int64_t num_blocks(const sa_shape& s) { return (static_cast<int64_t>(s.N) + 63) / 64; }
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+sa_status check_shape(const sa_shape& s) {
+  if (s.B < 1 || s.H < 1 || s.N < 1) return SA_ERR_INVALID_ARG;
+  if (s.block != 64) return SA_ERR_UNSUPPORTED;
+  if (s.d != 64 && s.d != 128) return SA_ERR_UNSUPPORTED;
+  if (num_blocks(s) > sa::kMaxNb) return SA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(s.B) * s.H > 65535) return SA_ERR_UNSUPPORTED;
+  return SA_OK;
+}
+
+size_t pooled_bytes(const sa_shape& s) {
+  return align_up(static_cast<size_t>(s.B) * s.H * num_blocks(s) * s.d * sizeof(float), 256);
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [B*H, N, d] bf16 viewed as a 3-D tensor {d, N, B*H}; box {64, rows, 1}, 128B swizzle.
+// Rows past N of a head read as zero (out-of-bounds fill), never the next head.
+bool make_map(CUtensorMap* map, const void* ptr, const sa_shape& s, int box_rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(s.d), static_cast<cuuint64_t>(s.N),
+                        static_cast<cuuint64_t>(s.B) * s.H};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(s.d) * 2, static_cast<cuuint64_t>(s.N) * s.d * 2};
+  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <typename F>
+sa_status set_smem(F* kernel, int bytes) {
+  // Per device: the attribute belongs to the current context.
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lk(mu);
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return SA_ERR_CUDA;
+  return SA_OK;
+}
+
+template <int D>
+sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau, float scale, int causal,
+                      uint8_t* mask, int32_t* count, int32_t* idx, int32_t* work, void* ws, cudaStream_t st) {
+  const int Nb = static_cast<int>(num_blocks(s));
+  const long long BH = static_cast<long long>(s.B) * s.H;
+  float* Qp = static_cast<float*>(ws);
+  float* Kp = reinterpret_cast<float*>(static_cast<char*>(ws) + pooled_bytes(s));
+  sa::pool_kernel<D><<<dim3(static_cast<unsigned>(BH * Nb), 2), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Qp, Kp, s.N, Nb);
+  if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+
+  const int ldL = (Nb + 3) & ~3;
+  if (Nb <= 3000) {
+    constexpr int R = 16;
+    const int smem = (D * (R + 4) + R * ldL) * static_cast<int>(sizeof(float));
+    if (set_smem(sa::score_select_kernel<D, R>, smem) != SA_OK) return SA_ERR_CUDA;
+    sa::score_select_kernel<D, R><<<dim3((Nb + R - 1) / R, static_cast<unsigned>(BH)), 256, smem, st>>>(
+        Qp, Kp, Nb, scale, causal, tau, mask, count, idx);
+  } else {
+    constexpr int R = 8;
+    const int smem = (D * (R + 4) + R * ldL) * static_cast<int>(sizeof(float));
+    if (set_smem(sa::score_select_kernel<D, R>, smem) != SA_OK) return SA_ERR_CUDA;
+    sa::score_select_kernel<D, R><<<dim3((Nb + R - 1) / R, static_cast<unsigned>(BH)), 256, smem, st>>>(
+        Qp, Kp, Nb, scale, causal, tau, mask, count, idx);
+  }
+  if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+
+  if (work) {
+    const int Tq = (Nb + 1) / 2;
+    const int smem = (2 * Nb + 1) * static_cast<int>(sizeof(int));
+    sa::tile_order_kernel<<<static_cast<unsigned>(BH), 1024, smem, st>>>(count, Nb, Tq, work);
+    if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+  }
+  return SA_OK;
+}
+
+template <int D>
+sa_status launch_fwd(const sa_shape& s, const void* Q, const void* K, const void* V, const uint8_t* mask,
+                     const int32_t* work, float lambda, float scale, int causal, void* O, int64_t* stats,
+                     cudaStream_t st) {
+  using Cfg = sa::FwdCfg<D, kFwdStages>;
+  const int Nb = static_cast<int>(num_blocks(s));
+  const int Tq = (Nb + 1) / 2;
+  const long long tiles = static_cast<long long>(s.B) * s.H * Tq;
+  if (tiles > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, Q, s, 128) || !make_map(&mk, K, s, 64) || !make_map(&mv, V, s, 64)) return SA_ERR_CUDA;
+  if (stats && cudaMemsetAsync(stats, 0, 4 * sizeof(int64_t), st) != cudaSuccess) return SA_ERR_CUDA;
+  auto kern = sa::fwd_kernel<D, kFwdStages>;
+  if (set_smem(kern, Cfg::kSmemBytes) != SA_OK) return SA_ERR_CUDA;
+  const float LOG2E = 1.4426950408889634f;
+  const int lam_on = std::isinf(lambda) && lambda < 0 ? 0 : 1;
+  kern<<<static_cast<unsigned>(tiles), 256, Cfg::kSmemBytes, st>>>(
+      mq, mk, mv, mask, work, static_cast<__nv_bfloat16*>(O), s.N, Nb, Tq, tiles, scale * LOG2E,
+      lam_on ? lambda * LOG2E : 0.f, lam_on, causal, reinterpret_cast<unsigned long long*>(stats));
+  if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+  return SA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sparse_attn_plan_workspace_size(sa_shape s) {
+  if (check_shape(s) != SA_OK) return 0;
+  return 2 * pooled_bytes(s);
+}
+
+int64_t sparse_attn_num_tiles(sa_shape s) {
+  if (check_shape(s) != SA_OK) return 0;
+  return static_cast<int64_t>(s.B) * s.H * ((num_blocks(s) + 1) / 2);
+}
+
+sa_status sparse_attn_plan(const void* Q, const void* K, sa_shape s, float tau, float scale, int32_t causal,
+                           uint8_t* mask, int32_t* count, int32_t* idx, int32_t* work, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  if (!Q || !K || !mask || !count) return SA_ERR_INVALID_ARG;
+  const sa_status sh = check_shape(s);
+  if (sh != SA_OK) return sh;
+  if (!(tau > 0.f && tau <= 1.f)) return SA_ERR_INVALID_ARG;  // also rejects NaN
+  if (!(std::isfinite(scale) && scale > 0.f)) return SA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K)) return SA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < sparse_attn_plan_workspace_size(s))
+    return SA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s.d == 64) return launch_plan<64>(s, Q, K, tau, scale, causal != 0, mask, count, idx, work, workspace, st);
+  return launch_plan<128>(s, Q, K, tau, scale, causal != 0, mask, count, idx, work, workspace, st);
+}
+
+sa_status sparse_attn_fwd(const void* Q, const void* K, const void* V, sa_shape s, const uint8_t* mask,
+                          const int32_t* work, float lambda, float scale, int32_t causal, void* O,
+                          int64_t* stats, void* stream) {
+  if (!Q || !K || !V || !mask || !O) return SA_ERR_INVALID_ARG;
+  const sa_status sh = check_shape(s);
+  if (sh != SA_OK) return sh;
+  if (std::isnan(lambda) || (std::isinf(lambda) && lambda > 0)) return SA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return SA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SA_ERR_INVALID_ARG;
+  if (stats && (reinterpret_cast<uintptr_t>(stats) & 7u) != 0) return SA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s.d == 64) return launch_fwd<64>(s, Q, K, V, mask, work, lambda, scale, causal != 0, O, stats, st);
+  return launch_fwd<128>(s, Q, K, V, mask, work, lambda, scale, causal != 0, O, stats, st);
+}
+
+const char* sparse_attn_status_string(sa_status st) {
+  switch (st) {
+    case SA_OK: return "SA_OK";
+    case SA_ERR_INVALID_ARG: return "SA_ERR_INVALID_ARG: null pointer, bad size or value, or misaligned pointer";
+    case SA_ERR_UNSUPPORTED: return "SA_ERR_UNSUPPORTED: d must be 64 or 128, block 64, Nb <= 4096, B*H <= 65535";
+    case SA_ERR_WORKSPACE: return "SA_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case SA_ERR_CUDA: return "SA_ERR_CUDA: a CUDA call or kernel launch failed";
+    case SA_ERR_DEVICE_CHECK: return "SA_ERR_DEVICE_CHECK: a device-side check fired";
+  }
+  return "unknown sa_status";
+}
+
+sa_status sparse_attn_device_error(void* stream, int32_t* code) {
+  if (!code) return SA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, sa::g_dev_error, sizeof(v), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return SA_ERR_CUDA;
+  if (cudaMemcpyToSymbolAsync(sa::g_dev_error, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, st) !=
+      cudaSuccess)
+    return SA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SA_ERR_CUDA;
+  *code = static_cast<int32_t>(v);
+  return SA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,133 @@
+/*
+ * sparse_attn.h — C ABI of the B200 (sm_100a) block-sparse attention library.
+ *
+ * Two calls make up the path:
+ *
+ *   sparse_attn_plan  — stage 1 of the two-stage filter in the SpargeAttn abstract
+ *                       ("rapidly and accurately predict the attention map"):
+ *                       mean-pool Q and K over 64-token blocks, softmax of the
+ *                       pooled scores, and per query block keep the fewest key
+ *                       blocks whose cumulative attention energy reaches tau —
+ *                       the per-row dynamic threshold of the DynSparse article
+ *                       ("Training-free sparse attention based on cumulative
+ *                       energy filtering", method paragraph).
+ *   sparse_attn_fwd   — stage 2: FlashAttention-style forward over the kept
+ *                       blocks only, plus the online-softmax-aware filter of the
+ *                       SpargeAttn abstract (second stage): skip P.V of a block
+ *                       whose rows all satisfy rowmax(S_blk) - running_max < lambda.
+ *
+ * Conventions shared by every call:
+ *   - Q, K, V, O are bf16, row-major [B, H, N, d] (d contiguous), device memory,
+ *     16-byte aligned. d is 64 or 128. block must be 64.
+ *   - Nb = ceil(N / 64) blocks per head; the last block may be ragged.
+ *   - A query tile is 128 rows = query blocks (2t, 2t+1) of one (b, h);
+ *     Tq = ceil(Nb / 2) tiles per head, B*H*Tq tiles in all.
+ *   - All pointers are owned by the caller. The library allocates no memory and
+ *     keeps no state across calls except one device-side error word per GPU.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Every call is asynchronous on that stream; results are ready when it is.
+ *   - Argument errors are detected on the host before anything is launched and
+ *     return a status; nothing is written then. A failed launch returns
+ *     SA_ERR_CUDA. Device-side checks (a wait that timed out, an index out of
+ *     range) never trap: the kernel stops its tile, records a code in the
+ *     device error word and returns; read it with sparse_attn_device_error.
+ */
+#ifndef SPARSE_ATTN_H
+#define SPARSE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SA_OK = 0,
+  SA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, tau outside (0,1], NaN, misaligned pointer */
+  SA_ERR_UNSUPPORTED = 2,  /* d not in {64,128}, block != 64, Nb > 4096, B*H > 65535 */
+  SA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than sparse_attn_plan_workspace_size */
+  SA_ERR_CUDA = 4,         /* a CUDA runtime/driver call or a launch failed */
+  SA_ERR_DEVICE_CHECK = 5  /* the device error word was set (see sparse_attn_device_error) */
+} sa_status;
+
+typedef struct {
+  int32_t B;     /* batch */
+  int32_t H;     /* heads */
+  int32_t N;     /* tokens per head, >= 1 */
+  int32_t d;     /* head dim, 64 or 128 */
+  int32_t block; /* mask block size, must be 64 */
+} sa_shape;
+
+/* Bytes of device workspace sparse_attn_plan needs for shape s (pooled Q and K,
+ * fp32 [B,H,Nb,d] each, 256-byte aligned). 0 if the shape is invalid. */
+size_t sparse_attn_plan_workspace_size(sa_shape s);
+
+/* Number of 128-row query tiles, B*H*ceil(Nb/2): the length of `work`. 0 if the
+ * shape is invalid. */
+int64_t sparse_attn_num_tiles(sa_shape s);
+
+/* Stage 1: block mask from mean-pooled Q and K.
+ *
+ *   Q, K      device bf16 [B,H,N,d]
+ *   tau       recall threshold in (0, 1]: per query block i, the kept set is the
+ *             shortest prefix of key blocks sorted by pooled probability
+ *             (descending, ties to the lower index) whose sum reaches tau times
+ *             the row sum. tau = 1 keeps every block with a finite pooled score.
+ *   scale     softmax scale of the pooled scores (use the attention's, 1/sqrt(d))
+ *   causal    nonzero: key block j > i is excluded from row i's softmax
+ *   mask      out, device uint8 [B,H,Nb,Nb]: 1 = kept
+ *   count     out, device int32 [B,H,Nb]: kept blocks per query block (>= 1)
+ *   idx       out, device int32 [B,H,Nb,Nb] or NULL: kept key blocks in ascending
+ *             order in the first count[..] entries of each row; the rest of the
+ *             row is left untouched
+ *   work      out, device int32 [sparse_attn_num_tiles(s)] or NULL: a permutation
+ *             of query-tile ids (tile = (b*H + h)*Tq + t) grouped by head in
+ *             ascending (b,h) order, and within a head ordered by decreasing
+ *             count[2t] + count[2t+1] (order among equal counts unspecified);
+ *             sparse_attn_fwd runs tiles in this order
+ *   workspace device scratch of at least sparse_attn_plan_workspace_size(s) bytes,
+ *             256-byte aligned; its contents on entry do not matter
+ */
+sa_status sparse_attn_plan(const void* Q, const void* K, sa_shape s, float tau, float scale,
+                           int32_t causal, uint8_t* mask, int32_t* count, int32_t* idx,
+                           int32_t* work, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Stage 2: sparse attention over the kept blocks, with the lambda P.V filter.
+ *
+ *   Q, K, V   device bf16 [B,H,N,d]
+ *   mask      device uint8 [B,H,Nb,Nb] (nonzero = kept), e.g. from sparse_attn_plan;
+ *             with causal, entries j > i are ignored
+ *   work      device int32 [num_tiles] tile order from sparse_attn_plan, or NULL for
+ *             the natural order. Entries must be a permutation of [0, num_tiles).
+ *   lambda    threshold in natural-log units of the scaled scores. For each query
+ *             block and kept key block (ascending order), the block's P.V is skipped
+ *             when every row that sees a key of the block has
+ *             rowmax(S_blk) - m < lambda (m = running max before the block); the
+ *             block still updates the running max and the softmax denominator.
+ *             -INFINITY turns the filter off. NaN is rejected.
+ *   scale     softmax scale (1/sqrt(d) for standard attention), finite, > 0
+ *   causal    nonzero: key token s is visible to query token t only if s <= t
+ *   O         out, device bf16 [B,H,N,d]. A row with no visible key is written as 0.
+ *   stats     device int64[4] or NULL; zeroed, then filled with: kept (query block,
+ *             key block) pairs visited, pairs whose P.V was skipped by lambda,
+ *             128x64 score tiles computed, 128x64 P.V tiles computed
+ */
+sa_status sparse_attn_fwd(const void* Q, const void* K, const void* V, sa_shape s,
+                          const uint8_t* mask, const int32_t* work, float lambda, float scale,
+                          int32_t causal, void* O, int64_t* stats, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* sparse_attn_status_string(sa_status st);
+
+/* Reads the device error word of the current GPU (after synchronising `stream`),
+ * stores it in *code (0 = no device-side check fired; bit 0 = a pipeline wait
+ * timed out, bit 1 = an index was out of range) and clears it. Returns SA_OK, or
+ * SA_ERR_CUDA if the copy failed. */
+sa_status sparse_attn_device_error(void* stream, int32_t* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_ATTN_H */

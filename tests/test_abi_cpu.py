@@ -1,0 +1,108 @@
+"""The C-ABI library loads without a GPU, exports every symbol its header declares,
+and rejects bad arguments on the host (no device work is launched)."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+from free_block_sparse_mean_b200 import _lib
+from free_block_sparse_mean_b200._lib import SaShape
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sparse_attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from free_block_sparse_mean_b200 import build
+    build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sparse_attn_\w+)\s*\(", src)))
+
+
+def test_header_matches_binding_list():
+    assert declared_functions() == sorted(_lib.EXPORTS)
+
+
+def test_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        s = lib.sparse_attn_status_string(code).decode()
+        assert s.startswith(_lib.STATUS_NAMES[code])
+    assert lib.sparse_attn_status_string(99).decode() == "unknown sa_status"
+
+
+def test_workspace_and_tiles(lib):
+    s = SaShape(1, 40, 75600, 128, 64)
+    Nb = math.ceil(75600 / 64)
+    pooled = 1 * 40 * Nb * 128 * 4
+    pooled = (pooled + 255) // 256 * 256
+    assert lib.sparse_attn_plan_workspace_size(s) == 2 * pooled
+    assert lib.sparse_attn_num_tiles(s) == 40 * ((Nb + 1) // 2)
+    assert lib.sparse_attn_num_tiles(SaShape(2, 3, 1, 64, 64)) == 6
+    for bad in (SaShape(1, 1, 64, 96, 64), SaShape(1, 1, 64, 128, 32), SaShape(0, 1, 64, 128, 64),
+                SaShape(1, 1, 0, 128, 64), SaShape(1, 1, 64 * 4097, 128, 64)):
+        assert lib.sparse_attn_plan_workspace_size(bad) == 0
+        assert lib.sparse_attn_num_tiles(bad) == 0
+
+
+FAKE = ctypes.c_void_p(0x10000)       # never dereferenced: checks fail before any launch
+FAKE_ODD = ctypes.c_void_p(0x10008)
+
+
+def _plan(lib, Q=FAKE, K=FAKE, s=SaShape(1, 2, 128, 128, 64), tau=0.9, scale=0.1, mask=FAKE, count=FAKE,
+          ws=FAKE, ws_bytes=1 << 30):
+    return lib.sparse_attn_plan(Q, K, s, tau, scale, 0, mask, count, None, None, ws, ws_bytes, None)
+
+
+def test_plan_argument_errors(lib):
+    E = _lib
+    assert _plan(lib, Q=None) == 1
+    assert _plan(lib, mask=None) == 1
+    assert _plan(lib, count=None) == 1
+    assert _plan(lib, tau=0.0) == 1
+    assert _plan(lib, tau=1.5) == 1
+    assert _plan(lib, tau=float("nan")) == 1
+    assert _plan(lib, scale=float("inf")) == 1
+    assert _plan(lib, scale=-1.0) == 1
+    assert _plan(lib, Q=FAKE_ODD) == 1
+    assert _plan(lib, s=SaShape(1, 2, 128, 96, 64)) == 2
+    assert _plan(lib, s=SaShape(1, 2, 128, 128, 128)) == 2
+    assert _plan(lib, s=SaShape(1, 1, 64 * 5000, 128, 64)) == 2
+    assert _plan(lib, s=SaShape(1, 2, 0, 128, 64)) == 1
+    assert _plan(lib, ws=None) == 3
+    assert _plan(lib, ws_bytes=10) == 3
+    assert _plan(lib, ws=ctypes.c_void_p(0x10010)) == 3     # not 256-byte aligned
+
+
+def _fwd(lib, Q=FAKE, K=FAKE, V=FAKE, s=SaShape(1, 2, 128, 128, 64), mask=FAKE, lam=-math.inf, scale=0.1,
+         O=FAKE, stats=None):
+    return lib.sparse_attn_fwd(Q, K, V, s, mask, None, lam, scale, 0, O, stats, None)
+
+
+def test_fwd_argument_errors(lib):
+    assert _fwd(lib, V=None) == 1
+    assert _fwd(lib, mask=None) == 1
+    assert _fwd(lib, O=None) == 1
+    assert _fwd(lib, lam=float("nan")) == 1
+    assert _fwd(lib, lam=float("inf")) == 1
+    assert _fwd(lib, scale=0.0) == 1
+    assert _fwd(lib, O=FAKE_ODD) == 1
+    assert _fwd(lib, stats=ctypes.c_void_p(0x10004)) == 1
+    assert _fwd(lib, s=SaShape(1, 2, 128, 32, 64)) == 2
+    assert _fwd(lib, s=SaShape(70000, 1, 128, 128, 64)) == 2
+
+
+def test_device_error_needs_output_pointer(lib):
+    assert lib.sparse_attn_device_error(None, None) == 1

@@ -1,0 +1,167 @@
+"""CUDA path (through the C ABI) against the CPU oracle, element by element.
+
+Masks: exact except blocks whose cumulative energy lies within 1e-4 of tau.
+Outputs: oracle run with the GPU's own mask, max-abs <= 2e-2 and relative
+Frobenius <= 1e-2 (bf16 inputs, fp32 accumulation)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import sparse_attn_oracle as orc
+from tests.helpers import (assert_output_close, check_plan_consistency, compare_masks,
+                           output_errors, to_np)
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import free_block_sparse_mean_b200 as sa
+    from free_block_sparse_mean_b200 import workloads as wl
+
+
+def _dev():
+    return torch.device("cuda:0")
+
+
+def _no_device_error():
+    assert sa.sparse_attn_device_error() == 0
+
+
+def _plan_and_check(q, k, tau, causal, scale=None):
+    p = sa.sparse_attn_plan(q, k, tau, scale, causal)
+    torch.cuda.synchronize()
+    mask, count, idx = to_np(p.mask), to_np(p.count), to_np(p.idx)
+    check_plan_consistency(mask, count, idx)
+    op = orc.plan(q.cpu(), k.cpu(), tau, scale, causal)
+    rows, excused = compare_masks(mask, op, tau)
+    total_rows = mask.shape[0] * mask.shape[1] * mask.shape[2]
+    assert rows <= max(2, total_rows // 200), f"{rows} of {total_rows} rows differ"
+    return p, mask, op
+
+
+def _work_ok(p, B, H, Nb):
+    Tq = (Nb + 1) // 2
+    work = to_np(p.work).astype(np.int64)
+    assert sorted(work.tolist()) == list(range(B * H * Tq))
+    count = to_np(p.count).reshape(B * H, Nb)
+    cost = np.zeros((B * H, Tq), dtype=np.int64)
+    cost += count[:, 0::2]
+    cost[:, : count[:, 1::2].shape[1]] += count[:, 1::2]
+    for bh in range(B * H):
+        seg = work[bh * Tq:(bh + 1) * Tq]
+        assert np.all(seg // Tq == bh)                   # grouped by head, in order
+        c = cost[bh, seg - bh * Tq]
+        assert np.all(np.diff(c) <= 0)                   # decreasing cost
+
+
+SHAPES = [
+    # B, H, N, d, causal, tau
+    (1, 1, 1, 64, False, 0.9),
+    (1, 2, 63, 128, False, 0.9),
+    (1, 2, 64, 64, True, 0.95),
+    (2, 1, 65, 128, False, 0.5),
+    (1, 2, 200, 128, True, 0.9),
+    (1, 3, 1000, 64, False, 0.95),
+    (2, 2, 1024, 128, True, 0.99),
+    (1, 2, 1500, 128, False, 1.0),
+    (1, 1, 4160, 128, False, 0.8),
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,causal,tau", SHAPES)
+def test_plan_and_fwd_random(B, H, N, d, causal, tau):
+    q, k, v = wl.random_qkv(B, H, N, d, seed=N + d, device=_dev(), scale_qk=2.0)
+    p, mask, op = _plan_and_check(q, k, tau, causal)
+    _work_ok(p, B, H, -(-N // 64))
+    o = sa.sparse_attn_fwd(q, k, v, p)
+    torch.cuda.synchronize()
+    ref = orc.fwd(q.cpu(), k.cpu(), v.cpu(), mask, None, None, causal)
+    assert_output_close(to_np(o), ref, f"fwd B{B} H{H} N{N} d{d} causal{causal}")
+    _no_device_error()
+
+
+@pytest.mark.parametrize("N,d,causal", [(64, 128, False), (300, 64, True), (1088, 128, False),
+                                        (777, 128, True)])
+def test_fwd_full_mask_is_dense(N, d, causal):
+    q, k, v = wl.random_qkv(1, 2, N, d, seed=7, device=_dev())
+    Nb = -(-N // 64)
+    mask = torch.ones((1, 2, Nb, Nb), dtype=torch.uint8, device=_dev())
+    o = sa.sparse_attn_fwd(q, k, v, mask, None, None, causal)
+    torch.cuda.synchronize()
+    ref = orc.attention_masked(q.cpu(), k.cpu(), v.cpu(), np.ones((1, 2, Nb, Nb), np.uint8), None, causal)
+    assert_output_close(to_np(o), ref, "dense")
+
+
+@pytest.mark.parametrize("N,d,causal,density", [(640, 128, False, 0.3), (1000, 64, False, 0.5),
+                                                (900, 128, True, 0.4), (130, 128, False, 0.0)])
+def test_fwd_random_mask(N, d, causal, density):
+    """Arbitrary masks, including rows with no kept block (output 0)."""
+    q, k, v = wl.random_qkv(1, 3, N, d, seed=11, device=_dev())
+    Nb = -(-N // 64)
+    g = torch.Generator().manual_seed(3)
+    m = (torch.rand((1, 3, Nb, Nb), generator=g) < density).to(torch.uint8)
+    o = sa.sparse_attn_fwd(q, k, v, m.to(_dev()), None, None, causal)
+    torch.cuda.synchronize()
+    ref = orc.attention_masked(q.cpu(), k.cpu(), v.cpu(), m.numpy(), None, causal)
+    assert_output_close(to_np(o), ref, "random mask")
+    _no_device_error()
+
+
+@pytest.mark.parametrize("lam", [-12.0, -6.0, -3.0])
+def test_fwd_lambda_skip(lam):
+    """Key block 0 aligned with all queries, the rest weaker: later blocks fall
+    below lambda; GPU skips must give the oracle's tiled-loop output."""
+    N, d = 1024, 128
+    q, k, v = wl.random_qkv(1, 2, N, d, seed=5, device=_dev())
+    u = torch.ones(d, device=_dev())
+    q = (q.float() * 0.3 + u).to(torch.bfloat16)
+    k = k.float()
+    k[:, :, :64] = k[:, :, :64] * 0.3 + u
+    k = k.to(torch.bfloat16)
+    Nb = N // 64
+    mask = torch.ones((1, 2, Nb, Nb), dtype=torch.uint8, device=_dev())
+    stats = torch.zeros(4, dtype=torch.int64, device=_dev())
+    o = sa.sparse_attn_fwd(q, k, v, mask, lam, stats=stats)
+    torch.cuda.synchronize()
+    ref, st = orc.attention_tiled(q.cpu(), k.cpu(), v.cpu(), to_np(mask).astype(np.uint8), lam,
+                                  return_stats=True)
+    assert_output_close(to_np(o), ref, f"lambda={lam}")
+    s = to_np(stats)
+    assert s[0] == st["kept_pairs"]
+    assert abs(int(s[1]) - st["pv_skipped"]) <= max(2, st["pv_skipped"] // 100)
+
+
+@pytest.mark.parametrize("tau,lam", [(0.9, None), (0.95, -12.0), (0.99, -12.0)])
+def test_small_workload(tau, lam):
+    """The small DiT-layer shape (H=24, d=128, N=4096), all heads."""
+    w = wl.WORKLOADS["small"]
+    q, k, v = wl.generate(w, seed=0, device=_dev())
+    p, mask, op = _plan_and_check(q, k, tau, False)
+    o = sa.sparse_attn_fwd(q, k, v, p, lam)
+    torch.cuda.synchronize()
+    ref = orc.fwd(q.cpu(), k.cpu(), v.cpu(), mask, lam)
+    assert_output_close(to_np(o), ref, f"small tau={tau} lam={lam}")
+    _no_device_error()
+
+
+def test_tiny_workload_and_sparse_vs_dense():
+    w = wl.WORKLOADS["tiny"]
+    q, k, v = wl.generate(w, seed=0, device=_dev())
+    p, mask, op = _plan_and_check(q, k, 0.95, False)
+    o = sa.sparse_attn_fwd(q, k, v, p)
+    torch.cuda.synchronize()
+    ref = orc.fwd(q.cpu(), k.cpu(), v.cpu(), mask)
+    assert_output_close(to_np(o), ref, "tiny")
+    dense = orc.attention_masked(q.cpu(), k.cpu(), v.cpu(), np.ones_like(mask))
+    max_abs, rel = output_errors(to_np(o), dense)
+    print(f"tiny sparse-vs-dense: max_abs={max_abs:.3e} rel_fro={rel:.3e} "
+          f"density={mask.mean():.3f}")
+
+
+def test_repeatable_masks():
+    q, k, _ = wl.random_qkv(1, 4, 3000, 128, seed=2, device=_dev(), scale_qk=2.0)
+    a = sa.sparse_attn_plan(q, k, 0.9)
+    b = sa.sparse_attn_plan(q, k, 0.9)
+    torch.cuda.synchronize()
+    assert torch.equal(a.mask, b.mask) and torch.equal(a.count, b.count)
