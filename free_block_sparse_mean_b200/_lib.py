@@ -27,6 +27,7 @@ EXPORTS = (
     "sparse_attn_fwd",
     "sparse_attn_status_string",
     "sparse_attn_device_error",
+    "sparse_attn_plan_noalloc",
 )
 
 
@@ -73,5 +74,7 @@ def load(path: str = LIB_PATH):
     lib.sparse_attn_status_string.restype = ctypes.c_char_p
     lib.sparse_attn_device_error.argtypes = [vp, ctypes.POINTER(i32)]
     lib.sparse_attn_device_error.restype = i32
+    lib.sparse_attn_plan_noalloc.argtypes = [vp, vp, SaShape, f32, f32, i32, vp, vp, vp, vp, vp]
+    lib.sparse_attn_plan_noalloc.restype = i32
     _lib = lib
     return lib

@@ -1,4 +1,4 @@
-"""Build libsparse_attn.so in-tree for sm_100a with nvcc (one translation unit).
+"""Build libsparse_attn.so in-tree for sm_100a with nvcc.
 
     python -m free_block_sparse_mean_b200.build
 """
@@ -11,7 +11,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SRC = os.path.join(HERE, "csrc", "sa_api.cu")
+SRCS = [os.path.join(HERE, "csrc", "sa_api.cu"), os.path.join(HERE, "csrc", "sa_noalloc.cu")]
 OUT = os.path.join(HERE, "libsparse_attn.so")
 DEPS = [os.path.join(HERE, "csrc", f) for f in os.listdir(os.path.join(HERE, "csrc"))] + \
        [os.path.join(ROOT, "include", "sparse_attn.h")]
@@ -41,7 +41,7 @@ def up_to_date() -> bool:
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return OUT
-    cmd = [nvcc(), *NVCC_FLAGS, "-o", OUT + ".tmp", SRC]
+    cmd = [nvcc(), *NVCC_FLAGS, "-o", OUT + ".tmp", *SRCS]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd))

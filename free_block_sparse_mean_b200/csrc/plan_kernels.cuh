@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(256) score_select_kernel(const float* __restri
 // Tile order: for each head, a counting sort of its Tq query tiles by decreasing
 // cost = count[2t] + count[2t+1]. Heads stay in ascending order so that the
 // tiles running at the same time share one head's K/V in L2.
-__global__ void __launch_bounds__(1024) tile_order_kernel(const int* __restrict__ count, int Nb, int Tq,
+static __global__ void __launch_bounds__(1024) tile_order_kernel(const int* __restrict__ count, int Nb, int Tq,
                                                           int* __restrict__ work) {
   extern __shared__ int hist[];  // [2*Nb + 1]
   const int nbins = 2 * Nb + 1;

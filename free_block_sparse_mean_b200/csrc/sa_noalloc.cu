@@ -1,0 +1,126 @@
+// sparse_attn_plan_noalloc: the plan call for callers that cannot allocate device
+// memory.
+//
+// Some hosts cannot give this library a workspace. Examples: an inference
+// runtime that reserves its whole device-memory budget at start-up and hands
+// out nothing afterwards; a plugin whose host process owns the allocator and
+// gives the plugin none; a latency-critical path where a cudaMalloc, which can
+// synchronise the device or fail once memory is fragmented, is not acceptable.
+// This entry point needs no workspace: the pooled Q and K live in a fixed
+// array of device memory that is part of the loaded library.
+//
+// Scratch: kNoAllocScratchBytes = 32 MiB, a file-scope __device__ array. Every
+// GPU that loads the library holds it until the process exits. The pooled
+// tensors take 2 * B*H*ceil(N/64)*d*4 bytes (each 256-byte aligned), so a call
+// fits when B*H*ceil(N/64)*d <= 4,194,304 values per tensor (for example H=24,
+// d=128 up to N = 87,360). Larger calls are rejected with SA_ERR_WORKSPACE
+// before anything runs.
+//
+// Every call shares the one array, and the array keeps the last call's
+// contents. The kernels write every scratch byte they later read, so nothing
+// has to start at zero. Calls whose work overlaps on the GPU (on two streams,
+// or from two host threads) race on the array and give wrong masks: order them
+// on one stream or otherwise serialise them.
+//
+// The first call on each device looks up the array's device address with
+// cudaGetSymbolAddress (in host code the array's name is only a host-side
+// stand-in, not a device address) and caches it for that device; make that
+// first call before any stream capture on the device.
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/sparse_attn.h"
+#include "plan_kernels.cuh"
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+constexpr int kMaxDevices = 64;
+
+__device__ __align__(256) unsigned char g_plan_scratch[kNoAllocScratchBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+size_t pooled_bytes_noalloc(const sa_shape& s) {
+  const size_t nb = (static_cast<size_t>(s.N) + 63) / 64;
+  const size_t b = static_cast<size_t>(s.B) * s.H * nb * s.d * sizeof(float);
+  return (b + 255) / 256 * 256;
+}
+
+// Device address of the scratch array on the current device (set up once per device).
+sa_status scratch_for_current_device(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_plan_scratch) != cudaSuccess || p == nullptr) return SA_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return SA_OK;
+}
+
+template <int D>
+sa_status launch_plan_noalloc(const sa_shape& s, const void* Q, const void* K, float tau, float scale,
+                              int causal, uint8_t* mask, int32_t* count, int32_t* idx, int32_t* work,
+                              void* scratch, cudaStream_t st) {
+  const int Nb = static_cast<int>((static_cast<int64_t>(s.N) + 63) / 64);
+  const long long BH = static_cast<long long>(s.B) * s.H;
+  float* Qp = static_cast<float*>(scratch);
+  float* Kp = reinterpret_cast<float*>(static_cast<char*>(scratch) + pooled_bytes_noalloc(s));
+  sa::pool_kernel<D><<<dim3(static_cast<unsigned>(BH * Nb), 2), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Qp, Kp, s.N, Nb);
+  if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+  const int ldL = (Nb + 3) & ~3;
+  if (Nb <= 3000) {
+    constexpr int R = 16;
+    const int smem = (D * (R + 4) + R * ldL) * static_cast<int>(sizeof(float));
+    if (cudaFuncSetAttribute(sa::score_select_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return SA_ERR_CUDA;
+    sa::score_select_kernel<D, R><<<dim3((Nb + R - 1) / R, static_cast<unsigned>(BH)), 256, smem, st>>>(
+        Qp, Kp, Nb, scale, causal, tau, mask, count, idx);
+  } else {
+    constexpr int R = 8;
+    const int smem = (D * (R + 4) + R * ldL) * static_cast<int>(sizeof(float));
+    if (cudaFuncSetAttribute(sa::score_select_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return SA_ERR_CUDA;
+    sa::score_select_kernel<D, R><<<dim3((Nb + R - 1) / R, static_cast<unsigned>(BH)), 256, smem, st>>>(
+        Qp, Kp, Nb, scale, causal, tau, mask, count, idx);
+  }
+  if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+  if (work) {
+    const int Tq = (Nb + 1) / 2;
+    const int smem = (2 * Nb + 1) * static_cast<int>(sizeof(int));
+    sa::tile_order_kernel<<<static_cast<unsigned>(BH), 1024, smem, st>>>(count, Nb, Tq, work);
+    if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+  }
+  return SA_OK;
+}
+
+}  // namespace
+
+extern "C" sa_status sparse_attn_plan_noalloc(const void* Q, const void* K, sa_shape s, float tau, float scale,
+                                              int32_t causal, uint8_t* mask, int32_t* count, int32_t* idx,
+                                              int32_t* work, void* stream) {
+  if (!Q || !K || !mask || !count) return SA_ERR_INVALID_ARG;
+  if (s.B < 1 || s.H < 1 || s.N < 1) return SA_ERR_INVALID_ARG;
+  if (s.block != 64 || (s.d != 64 && s.d != 128)) return SA_ERR_UNSUPPORTED;
+  if ((static_cast<int64_t>(s.N) + 63) / 64 > sa::kMaxNb) return SA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(s.B) * s.H > 65535) return SA_ERR_UNSUPPORTED;
+  if (!(tau > 0.f && tau <= 1.f)) return SA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return SA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(Q) & 15u) || (reinterpret_cast<uintptr_t>(K) & 15u)) return SA_ERR_INVALID_ARG;
+  if (2 * pooled_bytes_noalloc(s) > kNoAllocScratchBytes) return SA_ERR_WORKSPACE;  // beyond the fixed scratch
+  void* scratch = nullptr;
+  const sa_status got = scratch_for_current_device(&scratch);
+  if (got != SA_OK) return got;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s.d == 64)
+    return launch_plan_noalloc<64>(s, Q, K, tau, scale, causal != 0, mask, count, idx, work, scratch, st);
+  return launch_plan_noalloc<128>(s, Q, K, tau, scale, causal != 0, mask, count, idx, work, scratch, st);
+}

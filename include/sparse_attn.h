@@ -117,6 +117,24 @@ sa_status sparse_attn_fwd(const void* Q, const void* K, const void* V, sa_shape 
                           const uint8_t* mask, const int32_t* work, float lambda, float scale,
                           int32_t causal, void* O, int64_t* stats, void* stream);
 
+/* sparse_attn_plan without a workspace, for callers that cannot allocate device
+ * memory (a runtime that reserves its whole memory budget up front, a plugin
+ * whose host owns the allocator, a latency-critical path that must not call
+ * cudaMalloc). The paper has no counterpart: this is a deployment variant.
+ *
+ * Same arguments, outputs and errors as sparse_attn_plan, minus the workspace.
+ * The pooled Q and K go to a fixed 32 MiB device array inside the library, held
+ * by every GPU that loads the library until the process exits; the call fits when
+ * B*H*ceil(N/64)*d <= 4,194,304 and returns SA_ERR_WORKSPACE (nothing launched)
+ * otherwise. It calls no allocator. The first call on a device looks up the
+ * array's device address and caches it; make that first call before any stream
+ * capture on the device. All calls share the array (it keeps the last call's
+ * contents, and nothing in it needs to start at zero), so calls that overlap on
+ * the GPU race: keep them ordered on one stream. */
+sa_status sparse_attn_plan_noalloc(const void* Q, const void* K, sa_shape s, float tau, float scale,
+                                   int32_t causal, uint8_t* mask, int32_t* count, int32_t* idx,
+                                   int32_t* work, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* sparse_attn_status_string(sa_status st);
 
