@@ -14,8 +14,6 @@
 
 namespace {
 
-constexpr int kFwdStages = 3;
-
 inline int64_t num_blocks(const sa_shape& s) { return (static_cast<int64_t>(s.N) + 63) / 64; }
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -115,7 +113,7 @@ template <int D>
 sa_status launch_fwd(const sa_shape& s, const void* Q, const void* K, const void* V, const uint8_t* mask,
                      const int32_t* work, float lambda, float scale, int causal, void* O, int64_t* stats,
                      cudaStream_t st) {
-  using Cfg = sa::FwdCfg<D, kFwdStages>;
+  using Cfg = sa::FwdCfg<D>;
   const int Nb = static_cast<int>(num_blocks(s));
   const int Tq = (Nb + 1) / 2;
   const long long tiles = static_cast<long long>(s.B) * s.H * Tq;
@@ -123,7 +121,7 @@ sa_status launch_fwd(const sa_shape& s, const void* Q, const void* K, const void
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, Q, s, 128) || !make_map(&mk, K, s, 64) || !make_map(&mv, V, s, 64)) return SA_ERR_CUDA;
   if (stats && cudaMemsetAsync(stats, 0, 4 * sizeof(int64_t), st) != cudaSuccess) return SA_ERR_CUDA;
-  auto kern = sa::fwd_kernel<D, kFwdStages>;
+  auto kern = sa::fwd_kernel<D>;
   if (set_smem(kern, Cfg::kSmemBytes) != SA_OK) return SA_ERR_CUDA;
   const float LOG2E = 1.4426950408889634f;
   const int lam_on = std::isinf(lambda) && lambda < 0 ? 0 : 1;
