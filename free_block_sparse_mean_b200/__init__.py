@@ -70,7 +70,8 @@ class Plan:
     count int32 [B, H, Nb]      kept blocks per query block
     idx   int32 [B, H, Nb, Nb]  ascending kept blocks in the first count entries
                                 of each row (rest of the row undefined), or None
-    work  int32 [num_tiles]     tile order for sparse_attn_fwd, or None
+    work  int32 [2*num_tiles]   query-block pairs in execution order for sparse_attn_fwd
+                                (global ids (b*H+h)*Nb+i, second -1 if absent), or None
     """
     mask: torch.Tensor
     count: torch.Tensor
@@ -105,7 +106,7 @@ def sparse_attn_plan(q: torch.Tensor, k: torch.Tensor, tau: float, scale: Option
             mask=torch.empty((B, H, Nb, Nb), dtype=torch.uint8, device=dev),
             count=torch.empty((B, H, Nb), dtype=torch.int32, device=dev),
             idx=torch.empty((B, H, Nb, Nb), dtype=torch.int32, device=dev) if with_idx else None,
-            work=torch.empty((max(1, lib.sparse_attn_num_tiles(s)),), dtype=torch.int32, device=dev)
+            work=torch.empty((max(2, 2 * lib.sparse_attn_num_tiles(s)),), dtype=torch.int32, device=dev)
             if with_work else None,
             tau=float(tau), causal=bool(causal))
     else:

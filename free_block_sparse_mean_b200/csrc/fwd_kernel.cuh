@@ -6,10 +6,11 @@
 // filter skips more P.V products at no extra cost. The DynSparse article places
 // the selection inside the FlashAttention operator; this kernel is that operator.
 //
-// One CTA = one 128-row query tile = query blocks (2t, 2t+1) of one head. The
-// tile walks the ascending union of the two blocks' kept key blocks; the half
-// that did not keep a block sees it fully masked, so each 64-row query block
-// gets exactly its own mask. Per key block j (64 keys):
+// One CTA = one 128-row query tile = two 64-row query blocks (qa, qb) of one head,
+// paired by the plan so that their kept sets overlap (natural pairs (2t, 2t+1)
+// without a plan order). The tile walks the ascending union of the two blocks'
+// kept key blocks; the half that did not keep a block sees it fully masked, so
+// each 64-row query block gets exactly its own mask. Per key block j (64 keys):
 //   S = Q K_j^T     128x64 fp32 into TMEM (tcgen05.mma, Q and K_j TMA'd into
 //                   128B-swizzled shared memory, both K-major)
 //   softmax warps   read S from TMEM (thread = row), row max, lambda vote per
@@ -73,8 +74,8 @@ __global__ void __launch_bounds__(256, 2)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const uint8_t* __restrict__ mask,
                const int* __restrict__ work, __nv_bfloat16* __restrict__ O, int N, int Nb, int Tq,
-               long long num_tiles, float scale_log2, float lam_log2, int lam_on, int causal,
-               unsigned long long* __restrict__ stats) {
+               long long num_tiles, long long num_qblocks, float scale_log2, float lam_log2, int lam_on,
+               int causal, unsigned long long* __restrict__ stats) {
   using C = FwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -102,14 +103,23 @@ __global__ void __launch_bounds__(256, 2)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (blockIdx.x >= num_tiles) return;
-  const long long tile = work ? static_cast<long long>(work[blockIdx.x]) : static_cast<long long>(blockIdx.x);
-  if (tile < 0 || tile >= num_tiles) {  // corrupt work list: record and skip this CTA
-    if (threadIdx.x == 0) atomicOr(&g_dev_error, DEVERR_RANGE);
+  long long ga, gb;  // global query-block ids (b*H + h)*Nb + i of the two halves
+  if (work) {
+    ga = work[2 * static_cast<long long>(blockIdx.x)];
+    gb = work[2 * static_cast<long long>(blockIdx.x) + 1];
+  } else {
+    const long long bh0 = blockIdx.x / Tq;
+    const int t = static_cast<int>(blockIdx.x - bh0 * Tq);
+    ga = bh0 * Nb + 2 * t;
+    gb = (2 * t + 1 < Nb) ? ga + 1 : -1;
+  }
+  if (ga < 0 || ga >= num_qblocks || gb < -1 || gb >= num_qblocks || (gb >= 0 && gb / Nb != ga / Nb)) {
+    if (threadIdx.x == 0) atomicOr(&g_dev_error, DEVERR_RANGE);  // corrupt work list: skip
     return;
   }
-  const long long bh = tile / Tq;
-  const int t = static_cast<int>(tile - bh * Tq);
-  const int qb0 = 2 * t, qb1 = 2 * t + 1;
+  const long long bh = ga / Nb;
+  const int qb0 = static_cast<int>(ga - bh * Nb);              // query block of rows 0..63
+  const int qb1 = gb >= 0 ? static_cast<int>(gb - bh * Nb) : -1;  // rows 64..127 (-1: none)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STK; ++s) {
@@ -141,8 +151,8 @@ __global__ void __launch_bounds__(256, 2)
     // Ascending union of the kept lists of query blocks qb0 and qb1, one keep bit
     // per half; with causal, key blocks after a half's query block are dropped.
     const uint8_t* m0 = mask + (bh * Nb + qb0) * static_cast<long long>(Nb);
-    const uint8_t* m1 = (qb1 < Nb) ? m0 + Nb : nullptr;
-    const int jend = causal ? min(Nb, qb1 + 1) : Nb;
+    const uint8_t* m1 = (qb1 >= 0) ? mask + (bh * Nb + qb1) * static_cast<long long>(Nb) : nullptr;
+    const int jend = causal ? min(Nb, max(qb0, qb1) + 1) : Nb;
     int n = 0;
     for (int jb = 0; jb < jend; jb += 128) {
       uint32_t a[4], b[4];
@@ -195,10 +205,15 @@ __global__ void __launch_bounds__(256, 2)
   } else if (warp == 3) {
     // ------------------------------------------------------------ Q + V producer
     if (lane == 0 && n > 0) {
-      mbar_expect_tx(q_full, C::kQBytes);
+      // Q rows of the two query blocks into rows 0..63 / 64..127 of the tile
+      mbar_expect_tx(q_full, (qb1 >= 0 ? 2 : 1) * C::kKVBytes);
 #pragma unroll
-      for (int c = 0; c < C::kChunks; ++c)
-        tma_load_3d(sQ + c * C::kQChunkBytes, &tmQ, c * 64, t * 128, static_cast<int>(bh), q_full);
+      for (int c = 0; c < C::kChunks; ++c) {
+        tma_load_3d(sQ + c * C::kQChunkBytes, &tmQ, c * 64, qb0 * kBlock, static_cast<int>(bh), q_full);
+        if (qb1 >= 0)
+          tma_load_3d(sQ + c * C::kQChunkBytes + C::kKVChunkBytes, &tmQ, c * 64, qb1 * kBlock,
+                      static_cast<int>(bh), q_full);
+      }
       int k = 0;
       for (; k < n; ++k) {
         const int s = k % C::STV;
@@ -275,8 +290,9 @@ __global__ void __launch_bounds__(256, 2)
     const int wq = warp & 3;
     const int row = wq * 32 + lane;              // tile row == TMEM lane
     const int half = wq >> 1;                    // warps 4,5 -> query block qb0; 6,7 -> qb1
-    const long long qrow = static_cast<long long>(t) * 128 + row;
-    const bool valid = qrow < N;
+    const int myqb = half ? qb1 : qb0;
+    const long long qrow = static_cast<long long>(myqb) * kBlock + (row & (kBlock - 1));
+    const bool valid = myqb >= 0 && qrow < N;
     const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
     const unsigned FULL = 0xffffffffu;
     float m_true = -INFINITY, m_ref = -INFINITY, l = 0.f;

@@ -8,6 +8,8 @@
 // threshold derived from the cumulative energy.
 #pragma once
 
+#include <climits>
+
 #include "sa_device.cuh"
 
 namespace sa {
@@ -246,36 +248,196 @@ __global__ void __launch_bounds__(256) score_select_kernel(const float* __restri
 }
 
 // ----------------------------------------------------------------------------
-// Tile order: for each head, a counting sort of its Tq query tiles by decreasing
-// cost = count[2t] + count[2t+1]. Heads stay in ascending order so that the
-// tiles running at the same time share one head's K/V in L2.
-static __global__ void __launch_bounds__(1024) tile_order_kernel(const int* __restrict__ count, int Nb, int Tq,
-                                                          int* __restrict__ work) {
-  extern __shared__ int hist[];  // [2*Nb + 1]
-  const int nbins = 2 * Nb + 1;
-  const long long bh = blockIdx.x;
-  const int* cnt = count + bh * Nb;
-  for (int c = threadIdx.x; c < nbins; c += blockDim.x) hist[c] = 0;
-  __syncthreads();
-  for (int t = threadIdx.x; t < Tq; t += blockDim.x) {
-    const int c = cnt[2 * t] + ((2 * t + 1 < Nb) ? cnt[2 * t + 1] : 0);
-    atomicAdd(&hist[min(max(c, 0), nbins - 1)], 1);
+// Query-tile pairing and order. A 128-row query tile holds two 64-row query
+// blocks of one head and walks the union of their kept lists, so its cost is the
+// union size. Adjacent blocks of a video raster often keep disjoint key blocks
+// (their partners are in the neighbouring frame), so the pairs are chosen from
+// the masks: query blocks are sorted by two MinHash signatures of their kept
+// sets (equal sets sort together), then each block, in that order, takes as
+// partner the unused block among the next 32 whose kept set matches best
+// (overlap minus symmetric difference), else the next unused block. The pairs of
+// a head are then ordered by decreasing union size (longest first). Above
+// kPairGreedyMaxNb blocks per head the bitsets no longer fit in shared memory and
+// consecutive blocks of the sorted order are paired directly.
+// Output: work[2*r], work[2*r+1] = global query-block ids (bh*Nb + i) of the r-th
+// tile (second -1 if the head has an odd block count), heads in ascending order.
+constexpr int kPairGreedyMaxNb = 1024;
+constexpr int kPairWindow = 32;
+
+static __device__ __forceinline__ uint32_t mix32(uint32_t x) {
+  // MurmurHash3's 32-bit finaliser (a published bijective mixer).
+  x ^= x >> 16;
+  x *= 0x85ebca6bu;
+  x ^= x >> 13;
+  x *= 0xc2b2ae35u;
+  x ^= x >> 16;
+  return x;
+}
+
+// In-place ascending bitonic sort of n64 (a power of two) 64-bit keys in shared memory.
+static __device__ void block_bitonic_sort(unsigned long long* keys, int n64) {
+  for (int k = 2; k <= n64; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int t = threadIdx.x; t < n64 / 2; t += blockDim.x) {
+        const int lo = 2 * j * (t / j) + (t % j);
+        const int hi = lo + j;
+        const bool up = ((lo & k) == 0);
+        const unsigned long long a = keys[lo], b = keys[hi];
+        if ((a > b) == up) {
+          keys[lo] = b;
+          keys[hi] = a;
+        }
+      }
+      __syncthreads();
+    }
   }
+}
+
+static __global__ void __launch_bounds__(1024) pair_order_kernel(const uint8_t* __restrict__ mask,
+                                                                 const int* __restrict__ count, int Nb,
+                                                                 int Tq, int* __restrict__ work) {
+  extern __shared__ __align__(16) unsigned char psm[];
+  const int P = 1 << (32 - __clz(max(Nb, 2) - 1));   // next power of two >= Nb
+  const int P2 = 1 << (32 - __clz(max(Tq, 2) - 1));
+  const bool greedy = Nb <= kPairGreedyMaxNb;
+  const int W = (Nb + 31) / 32;                       // bitset words per row
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(psm);       // [P]
+  unsigned long long* keys2 = keys + P;                                          // [P2]
+  int* pa = reinterpret_cast<int*>(keys2 + P2);                                  // [Tq]
+  int* pb = pa + Tq;                                                             // [Tq]
+  int* order = pb + Tq;                                                          // [Nb]
+  int* used = order + Nb;                                                        // [Nb]
+  uint32_t* bits = reinterpret_cast<uint32_t*>(used + Nb);                      // [Nb][W] (greedy only)
+  const long long bh = blockIdx.x;
+  const uint8_t* m = mask + bh * static_cast<long long>(Nb) * Nb;
+  const int* cnt = count + bh * Nb;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  const unsigned FULL = 0xffffffffu;
+
+  // 1. signatures (and bitsets) of every query block's kept set
+  for (int i = warp; i < Nb; i += nwarps) {
+    uint32_t s1 = 0xffffffffu, s2 = 0xffffffffu;
+    const uint8_t* row = m + static_cast<long long>(i) * Nb;
+    for (int jb = 0; jb < Nb; jb += 32) {
+      const int j = jb + lane;
+      const bool kept = (j < Nb) && row[j] != 0;
+      if (kept) {
+        s1 = min(s1, mix32(static_cast<uint32_t>(j) ^ 0x9e3779b9u));
+        s2 = min(s2, mix32(static_cast<uint32_t>(j) + 0x7f4a7c15u));
+      }
+      const unsigned bal = __ballot_sync(FULL, kept);
+      if (greedy && lane == 0) bits[i * W + jb / 32] = bal;
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      s1 = min(s1, __shfl_xor_sync(FULL, s1, o));
+      s2 = min(s2, __shfl_xor_sync(FULL, s2, o));
+    }
+    if (lane == 0)
+      keys[i] = (static_cast<unsigned long long>(s1) << 32) | (static_cast<unsigned long long>(s2 & 0xffffu) << 16) |
+                static_cast<unsigned long long>(i);
+  }
+  for (int i = Nb + threadIdx.x; i < P; i += blockDim.x) keys[i] = ~0ull;
+  for (int i = threadIdx.x; i < Nb; i += blockDim.x) used[i] = 0;
   __syncthreads();
-  if (threadIdx.x == 0) {  // exclusive scan from the top bin down (nbins <= 8193)
-    int run = 0;
-    for (int c = nbins - 1; c >= 0; --c) {
-      const int h = hist[c];
-      hist[c] = run;
-      run += h;
+  block_bitonic_sort(keys, P);
+  for (int i = threadIdx.x; i < Nb; i += blockDim.x) order[i] = static_cast<int>(keys[i] & 0xffffu);
+  __syncthreads();
+
+  // 2. pairs and their costs (union sizes, or count sums without bitsets)
+  if (greedy) {
+    if (warp == 0) {
+      int np = 0;
+      for (int pos = 0; pos < Nb; ++pos) {
+        const int i = order[pos];
+        if (used[i]) continue;   // same value in every lane
+        __syncwarp();
+        if (lane == 0) used[i] = 1;
+        __syncwarp();
+        const int cpos = pos + 1 + lane;
+        const int c = (cpos < Nb && lane < kPairWindow) ? order[cpos] : -1;
+        int score = INT_MIN, uni = 0;
+        if (c >= 0 && !used[c]) {
+          int ov = 0, sd = 0;
+          for (int w = 0; w < W; ++w) {
+            const uint32_t a = bits[i * W + w], b = bits[c * W + w];
+            ov += __popc(a & b);
+            sd += __popc(a ^ b);
+            uni += __popc(a | b);
+          }
+          score = ov - sd;
+        }
+        // warp argmax, ties to the lowest lane
+        int best = score, bl = lane;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+          const int os = __shfl_xor_sync(FULL, best, o), ol = __shfl_xor_sync(FULL, bl, o);
+          if (os > best || (os == best && ol < bl)) {
+            best = os;
+            bl = ol;
+          }
+        }
+        int partner = __shfl_sync(FULL, c, bl);
+        int ucost = __shfl_sync(FULL, uni, bl);
+        if (best == INT_MIN) {   // nothing unused in the window: next unused block in order
+          partner = -1;
+          for (int q = pos + 1 + kPairWindow; q < Nb; q += 32) {
+            const int cc = (q + lane < Nb) ? order[q + lane] : -1;
+            const unsigned fr = __ballot_sync(FULL, cc >= 0 && !used[cc]);
+            if (fr) {
+              partner = __shfl_sync(FULL, cc, __ffs(fr) - 1);
+              break;
+            }
+          }
+          ucost = 0;
+          if (partner >= 0)
+            for (int w = lane; w < W; w += 32) ucost += __popc(bits[i * W + w] | bits[partner * W + w]);
+          else
+            for (int w = lane; w < W; w += 32) ucost += __popc(bits[i * W + w]);
+#pragma unroll
+          for (int o = 16; o; o >>= 1) ucost += __shfl_xor_sync(FULL, ucost, o);
+        }
+        if (lane == 0) {
+          if (partner >= 0) used[partner] = 1;
+          pa[np] = i;
+          pb[np] = partner;
+          keys2[np] = (static_cast<unsigned long long>(0xffffffu - static_cast<uint32_t>(ucost)) << 32) |
+                      static_cast<unsigned long long>(np);
+        }
+        __syncwarp();
+        ++np;
+      }
+    }
+  } else {
+    for (int p = threadIdx.x; p < Tq; p += blockDim.x) {
+      const int a = order[2 * p], b = (2 * p + 1 < Nb) ? order[2 * p + 1] : -1;
+      pa[p] = a;
+      pb[p] = b;
+      const int c = cnt[a] + (b >= 0 ? cnt[b] : 0);
+      keys2[p] = (static_cast<unsigned long long>(0xffffffu - static_cast<uint32_t>(c)) << 32) |
+                 static_cast<unsigned long long>(p);
     }
   }
   __syncthreads();
-  for (int t = threadIdx.x; t < Tq; t += blockDim.x) {
-    const int c = cnt[2 * t] + ((2 * t + 1 < Nb) ? cnt[2 * t + 1] : 0);
-    const int pos = atomicAdd(&hist[min(max(c, 0), nbins - 1)], 1);
-    work[bh * Tq + pos] = static_cast<int>(bh * Tq + t);
+  for (int p = Tq + threadIdx.x; p < P2; p += blockDim.x) keys2[p] = ~0ull;
+  __syncthreads();
+  // 3. longest first, then write the global query-block ids
+  block_bitonic_sort(keys2, P2);
+  for (int r = threadIdx.x; r < Tq; r += blockDim.x) {
+    const int p = static_cast<int>(keys2[r] & 0xffffffffu);
+    const int a = pa[p], b = pb[p];
+    work[2 * (bh * Tq + r)] = static_cast<int>(bh * Nb + a);
+    work[2 * (bh * Tq + r) + 1] = b >= 0 ? static_cast<int>(bh * Nb + b) : -1;
   }
+}
+
+// Shared memory of pair_order_kernel for Nb blocks per head.
+inline int pair_order_smem_bytes(int Nb) {
+  auto p2 = [](int x) { int p = 2; while (p < x) p <<= 1; return p; };
+  const int Tq = (Nb + 1) / 2;
+  int bytes = (p2(Nb) + p2(Tq)) * 8 + (2 * Tq + 2 * Nb) * 4;
+  if (Nb <= kPairGreedyMaxNb) bytes += Nb * ((Nb + 31) / 32) * 4;
+  return bytes;
 }
 
 }  // namespace sa

@@ -102,8 +102,9 @@ sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau
 
   if (work) {
     const int Tq = (Nb + 1) / 2;
-    const int smem = (2 * Nb + 1) * static_cast<int>(sizeof(int));
-    sa::tile_order_kernel<<<static_cast<unsigned>(BH), 1024, smem, st>>>(count, Nb, Tq, work);
+    const int smem = sa::pair_order_smem_bytes(Nb);
+    if (set_smem(sa::pair_order_kernel, smem) != SA_OK) return SA_ERR_CUDA;
+    sa::pair_order_kernel<<<static_cast<unsigned>(BH), 1024, smem, st>>>(mask, count, Nb, Tq, work);
     if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   }
   return SA_OK;
@@ -119,14 +120,15 @@ sa_status launch_fwd(const sa_shape& s, const void* Q, const void* K, const void
   const long long tiles = static_cast<long long>(s.B) * s.H * Tq;
   if (tiles > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, Q, s, 128) || !make_map(&mk, K, s, 64) || !make_map(&mv, V, s, 64)) return SA_ERR_CUDA;
+  if (!make_map(&mq, Q, s, 64) || !make_map(&mk, K, s, 64) || !make_map(&mv, V, s, 64)) return SA_ERR_CUDA;
   if (stats && cudaMemsetAsync(stats, 0, 4 * sizeof(int64_t), st) != cudaSuccess) return SA_ERR_CUDA;
   auto kern = sa::fwd_kernel<D>;
   if (set_smem(kern, Cfg::kSmemBytes) != SA_OK) return SA_ERR_CUDA;
   const float LOG2E = 1.4426950408889634f;
   const int lam_on = std::isinf(lambda) && lambda < 0 ? 0 : 1;
   kern<<<static_cast<unsigned>(tiles), 256, Cfg::kSmemBytes, st>>>(
-      mq, mk, mv, mask, work, static_cast<__nv_bfloat16*>(O), s.N, Nb, Tq, tiles, scale * LOG2E,
+      mq, mk, mv, mask, work, static_cast<__nv_bfloat16*>(O), s.N, Nb, Tq, tiles,
+      static_cast<long long>(s.B) * s.H * Nb, scale * LOG2E,
       lam_on ? lambda * LOG2E : 0.f, lam_on, causal, reinterpret_cast<unsigned long long*>(stats));
   if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   return SA_OK;

@@ -95,8 +95,11 @@ sa_status launch_plan_noalloc(const sa_shape& s, const void* Q, const void* K, f
   if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   if (work) {
     const int Tq = (Nb + 1) / 2;
-    const int smem = (2 * Nb + 1) * static_cast<int>(sizeof(int));
-    sa::tile_order_kernel<<<static_cast<unsigned>(BH), 1024, smem, st>>>(count, Nb, Tq, work);
+    const int smem = sa::pair_order_smem_bytes(Nb);
+    if (cudaFuncSetAttribute(sa::pair_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return SA_ERR_CUDA;
+    sa::pair_order_kernel<<<static_cast<unsigned>(BH), 1024, smem, st>>>(mask, count, Nb, Tq, work);
     if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   }
   return SA_OK;

@@ -20,8 +20,9 @@
  *   - Q, K, V, O are bf16, row-major [B, H, N, d] (d contiguous), device memory,
  *     16-byte aligned. d is 64 or 128. block must be 64.
  *   - Nb = ceil(N / 64) blocks per head; the last block may be ragged.
- *   - A query tile is 128 rows = query blocks (2t, 2t+1) of one (b, h);
- *     Tq = ceil(Nb / 2) tiles per head, B*H*Tq tiles in all.
+ *   - A query tile is 128 rows = two 64-row query blocks of one (b, h), paired by
+ *     sparse_attn_plan (or (2t, 2t+1) without a plan order); Tq = ceil(Nb / 2)
+ *     tiles per head, B*H*Tq tiles in all.
  *   - All pointers are owned by the caller. The library allocates no memory and
  *     keeps no state across calls except one device-side error word per GPU.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
@@ -63,8 +64,8 @@ typedef struct {
  * fp32 [B,H,Nb,d] each, 256-byte aligned). 0 if the shape is invalid. */
 size_t sparse_attn_plan_workspace_size(sa_shape s);
 
-/* Number of 128-row query tiles, B*H*ceil(Nb/2): the length of `work`. 0 if the
- * shape is invalid. */
+/* Number of 128-row query tiles, B*H*ceil(Nb/2); `work` holds two entries per
+ * tile. 0 if the shape is invalid. */
 int64_t sparse_attn_num_tiles(sa_shape s);
 
 /* Stage 1: block mask from mean-pooled Q and K.
@@ -81,11 +82,16 @@ int64_t sparse_attn_num_tiles(sa_shape s);
  *   idx       out, device int32 [B,H,Nb,Nb] or NULL: kept key blocks in ascending
  *             order in the first count[..] entries of each row; the rest of the
  *             row is left untouched
- *   work      out, device int32 [sparse_attn_num_tiles(s)] or NULL: a permutation
- *             of query-tile ids (tile = (b*H + h)*Tq + t) grouped by head in
- *             ascending (b,h) order, and within a head ordered by decreasing
- *             count[2t] + count[2t+1] (order among equal counts unspecified);
- *             sparse_attn_fwd runs tiles in this order
+ *   work      out, device int32 [2 * sparse_attn_num_tiles(s)] or NULL: the query
+ *             tiles in execution order, two global query-block ids per tile
+ *             ((b*H + h)*Nb + i; the second is -1 when a head has an odd block
+ *             count). Every query block appears exactly once; heads come in
+ *             ascending (b,h) order. Within a head, blocks are paired so that the
+ *             two kept sets overlap (sorted by two MinHash signatures of the kept
+ *             set, then each block takes the best-matching unused block among the
+ *             next 32, for Nb <= 1024; consecutive blocks of that order above),
+ *             and tiles are ordered by decreasing union size (longest first).
+ *             Deterministic for a given mask.
  *   workspace device scratch of at least sparse_attn_plan_workspace_size(s) bytes,
  *             256-byte aligned; its contents on entry do not matter
  */
@@ -98,8 +104,11 @@ sa_status sparse_attn_plan(const void* Q, const void* K, sa_shape s, float tau, 
  *   Q, K, V   device bf16 [B,H,N,d]
  *   mask      device uint8 [B,H,Nb,Nb] (nonzero = kept), e.g. from sparse_attn_plan;
  *             with causal, entries j > i are ignored
- *   work      device int32 [num_tiles] tile order from sparse_attn_plan, or NULL for
- *             the natural order. Entries must be a permutation of [0, num_tiles).
+ *   work      device int32 [2 * num_tiles]: query-block pairs from sparse_attn_plan, or
+ *             NULL for the natural pairs (2t, 2t+1) of each head. Each entry must be
+ *             a global query-block id < B*H*Nb (or -1 as the second of a pair), both
+ *             of a pair in one head, every block exactly once; a tile whose entry is
+ *             out of range is skipped and sets the device error word.
  *   lambda    threshold in natural-log units of the scaled scores. For each query
  *             block and kept key block (ascending order), the block's P.V is skipped
  *             when every row that sees a key of the block has

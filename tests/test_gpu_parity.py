@@ -41,18 +41,37 @@ def _plan_and_check(q, k, tau, causal, scale=None):
 
 
 def _work_ok(p, B, H, Nb):
+    """work lists every query block once, in pairs of one head, heads in order,
+    and within a head the pairs' union sizes do not increase."""
     Tq = (Nb + 1) // 2
-    work = to_np(p.work).astype(np.int64)
-    assert sorted(work.tolist()) == list(range(B * H * Tq))
-    count = to_np(p.count).reshape(B * H, Nb)
-    cost = np.zeros((B * H, Tq), dtype=np.int64)
-    cost += count[:, 0::2]
-    cost[:, : count[:, 1::2].shape[1]] += count[:, 1::2]
+    work = to_np(p.work).astype(np.int64)[: 2 * B * H * Tq].reshape(B * H, Tq, 2)
+    mask = to_np(p.mask).reshape(B * H, Nb, Nb).astype(bool)
     for bh in range(B * H):
-        seg = work[bh * Tq:(bh + 1) * Tq]
-        assert np.all(seg // Tq == bh)                   # grouped by head, in order
-        c = cost[bh, seg - bh * Tq]
-        assert np.all(np.diff(c) <= 0)                   # decreasing cost
+        a, b = work[bh, :, 0], work[bh, :, 1]
+        assert np.all(a // Nb == bh) and np.all((b == -1) | (b // Nb == bh))
+        ids = np.concatenate([a, b[b >= 0]]) - bh * Nb
+        assert sorted(ids.tolist()) == list(range(Nb))
+        assert (b == -1).sum() == Nb % 2
+        uni = [(mask[bh, x - bh * Nb] | (mask[bh, y - bh * Nb] if y >= 0 else False)).sum()
+               for x, y in zip(a, b)]
+        if Nb <= 1024:
+            assert np.all(np.diff(uni) <= 0)
+
+
+def test_pairing_reduces_union_on_small_workload():
+    """On the video raster the plan's pairs must cost fewer union entries than
+    the natural adjacent pairs (2t, 2t+1)."""
+    w = wl.WORKLOADS["small"]
+    q, k, _ = wl.generate(w, seed=0, device=_dev())
+    p = sa.sparse_attn_plan(q, k, 0.95)
+    torch.cuda.synchronize()
+    _work_ok(p, 1, w.H, 64)
+    m = to_np(p.mask).reshape(w.H, 64, 64).astype(bool)
+    work = to_np(p.work).astype(np.int64).reshape(w.H, 32, 2)
+    paired = sum((m[h, x % 64] | m[h, y % 64]).sum() for h in range(w.H) for x, y in work[h])
+    natural = sum((m[h, 2 * t] | m[h, 2 * t + 1]).sum() for h in range(w.H) for t in range(32))
+    print(f"union entries: plan pairs {paired}, natural pairs {natural}, kept pairs {m.sum()}")
+    assert paired < 0.8 * natural
 
 
 SHAPES = [
