@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--heads", type=int, default=None,
                     help="run only the first H heads of the workload (profiling captures)")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense (full-mask) reference timing")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch plan and forward directly instead of replaying CUDA graphs")
     return ap.parse_args()
 
 
@@ -287,10 +289,29 @@ def run_ours(args, w, world, rank, local, pg):
         dense_ms = e0.elapsed_time(e1)
         del full
 
+    def run_plan():
+        sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False)
+
+    def run_fwd():
+        sa.sparse_attn_fwd(q, k, v, plan, lam, out=out)
+
     for _ in range(args.warmup):
         flush.zero_()
         step()
     torch.cuda.synchronize()
+    if not args.no_graph:
+        # Each stage is one CUDA graph (its kernels only), so the timed steps replay
+        # two launches instead of paying host launch overhead per kernel.
+        g_plan, g_fwd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_plan):
+            run_plan()
+        with torch.cuda.graph(g_fwd):
+            run_fwd()
+        g_plan.replay()
+        g_fwd.replay()
+        torch.cuda.synchronize()
+        run_plan, run_fwd = g_plan.replay, g_fwd.replay
+        stream = torch.cuda.current_stream(dev)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     sampler = ClockSampler(local)
@@ -302,9 +323,9 @@ def run_ours(args, w, world, rank, local, pg):
         flush.zero_()                       # L2 flush, outside the timed events
         a, b, c = ev[i]
         a.record(stream)
-        sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False)
+        run_plan()
         b.record(stream)
-        sa.sparse_attn_fwd(q, k, v, plan, lam, out=out)
+        run_fwd()
         c.record(stream)
     torch.cuda.synchronize()
     barrier(pg, dev)
@@ -357,7 +378,7 @@ def run_ours(args, w, world, rank, local, pg):
                      "frac": achieved / peak_t, "traffic": None,
                      "kernel": "fwd_kernel<128,3> (sparse_attn_fwd)",
                      "peak_source": f"{pk_kind} bf16_tflops (burst)"},
-        "e2e": e2e, "gpu_launches": 4 * args.steps, "clocks": clocks,
+        "e2e": e2e, "gpu_launches": 4 * args.steps, "cuda_graphs": not args.no_graph, "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu:
         v_cpu, t_cpu, cores, sample = time_oracle(w, args.tau, lam, args.cpu_seconds, args.seed)

@@ -18,7 +18,8 @@
 //                   first 32 columns of the same TMEM buffer
 //   O += P V_j      128xD fp32 in TMEM; A operand (P) read from TMEM, B (V_j)
 //                   from shared memory as an MN-major operand
-// Roles (256 threads): warp 0 loads K, warp 3 loads V and Q (TMA), warp 1 issues
+// Roles (256 threads): warp 0 loads K, warp 3 loads V and Q (TMA; K and V as one
+// 4-D box per 64-row block, since TMA issue cost is per instruction), warp 1 issues
 // the MMAs (one thread) and owns TMEM, warp 2 builds the union list, warps 4..7
 // run the softmax, the O correction and the epilogue. S is double-buffered in
 // TMEM: S(k+1) is on the tensor cores while the softmax works on S(k), and
@@ -194,10 +195,7 @@ __global__ void __launch_bounds__(256, 2)
         if (!mbar_wait(&kempty[s], (static_cast<uint32_t>(k / C::STK) & 1u) ^ 1u, abort_flag)) break;
         const int j = static_cast<int>(lst[k] & kListJMask);
         mbar_expect_tx(&kfull[s], C::kKVBytes);
-#pragma unroll
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(sK + s * C::kKVBytes + c * C::kKVChunkBytes, &tmK, c * 64, j * kBlock,
-                      static_cast<int>(bh), &kfull[s]);
+        tma_load_4d(sK + s * C::kKVBytes, &tmK, 0, j * kBlock, 0, static_cast<int>(bh), &kfull[s]);
       }
       for (int kk = max(0, k - C::STK); kk < k; ++kk)  // let issued loads land before exit
         mbar_wait_drain(&kfull[kk % C::STK], static_cast<uint32_t>(kk / C::STK) & 1u);
@@ -220,10 +218,7 @@ __global__ void __launch_bounds__(256, 2)
         if (!mbar_wait(&vempty[s], (static_cast<uint32_t>(k / C::STV) & 1u) ^ 1u, abort_flag)) break;
         const int j = static_cast<int>(lst[k] & kListJMask);
         mbar_expect_tx(&vfull[s], C::kKVBytes);
-#pragma unroll
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(sV + s * C::kKVBytes + c * C::kKVChunkBytes, &tmV, c * 64, j * kBlock,
-                      static_cast<int>(bh), &vfull[s]);
+        tma_load_4d(sV + s * C::kKVBytes, &tmV, 0, j * kBlock, 0, static_cast<int>(bh), &vfull[s]);
       }
       mbar_wait_drain(q_full, 0u);
       for (int kk = max(0, k - C::STV); kk < k; ++kk)

@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 //
 // Phase 1 (CUDA-core fp32 GEMM, the pooled scores must stay fp32 to keep the
 // kept set stable near tau): thread t owns key blocks c = 2t, 2t+1 of each
-// 512-wide pass and all R rows; the R pooled query rows sit in shared memory
+// 2*NT-wide pass and all R rows; the R pooled query rows sit in shared memory
 // (transposed, read as broadcast float4), Kp rows stream from L2 in 32-byte
 // pieces. Scores go to shared memory: L[r][j] = scale * <Qp_r, Kp_j>, -inf for
 // causal j > i.
@@ -80,14 +80,15 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 // on the IEEE bit pattern of e (monotone for non-negative floats); every probe
 // sums in the same order as the total, so the probe at 0 equals the total
 // exactly. This is the sorted-prefix rule without sorting.
-template <int D, int R>
-__global__ void __launch_bounds__(256) score_select_kernel(const float* __restrict__ Qp,
+template <int D, int R, int NT>
+__global__ void __launch_bounds__(NT) score_select_kernel(const float* __restrict__ Qp,
                                                            const float* __restrict__ Kp, int Nb,
                                                            float scale, int causal, float tau,
                                                            uint8_t* __restrict__ mask,
                                                            int* __restrict__ count,
                                                            int* __restrict__ idx) {
-  static_assert(R % 4 == 0 && R <= 16, "R rows per CTA");
+  static_assert(R % 4 == 0 && R <= 16 && NT % 32 == 0, "R rows per CTA, NT threads");
+  constexpr int kCols = 2 * NT;  // key blocks per pass of phase 1
   constexpr int QS = R + 4;  // padded row stride of the transposed query tile
   extern __shared__ __align__(16) float sm[];
   float* qT = sm;                          // [D][QS]
@@ -105,7 +106,7 @@ __global__ void __launch_bounds__(256) score_select_kernel(const float* __restri
   __syncthreads();
 
   // ---------------- phase 1: scores
-  for (int cb = 0; cb < Nb; cb += 512) {
+  for (int cb = 0; cb < Nb; cb += kCols) {
     const int c0 = cb + 2 * threadIdx.x;
     float acc0[R], acc1[R];
 #pragma unroll
@@ -162,7 +163,7 @@ __global__ void __launch_bounds__(256) score_select_kernel(const float* __restri
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned FULL = 0xffffffffu;
   const float LOG2E = 1.4426950408889634f;
-  for (int r = warp; r < R; r += 8) {
+  for (int r = warp; r < R; r += NT / 32) {
     const int i = i0 + r;
     if (i >= Nb) break;
     float* row = L + r * ldL;

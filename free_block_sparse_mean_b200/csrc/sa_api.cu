@@ -63,6 +63,25 @@ bool make_map(CUtensorMap* map, const void* ptr, const sa_shape& s, int box_rows
   return r == CUDA_SUCCESS;
 }
 
+// [B*H, N, d] bf16 viewed as a 4-D tensor {64 elements, N rows, d/64 chunks, B*H}
+// (row stride 2d bytes, chunk stride 128 bytes): one box {64, 64, d/64, 1} is a
+// whole 64-row block, landing in shared memory as [chunk][row][128 B] with the
+// 128B swizzle, one TMA instruction per block. Rows past N of a head read as zero
+// (out-of-bounds fill), never the next head.
+bool make_block_map(CUtensorMap* map, const void* ptr, const sa_shape& s) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {64u, static_cast<cuuint64_t>(s.N), static_cast<cuuint64_t>(s.d / 64),
+                        static_cast<cuuint64_t>(s.B) * s.H};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(s.d) * 2, 128u, static_cast<cuuint64_t>(s.N) * s.d * 2};
+  cuuint32_t box[4] = {64u, 64u, static_cast<cuuint32_t>(s.d / 64), 1u};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <typename F>
 sa_status set_smem(F* kernel, int bytes) {
   // Per device: the attribute belongs to the current context.
@@ -85,26 +104,30 @@ sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau
   if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
 
   const int ldL = (Nb + 3) & ~3;
-  if (Nb <= 3000) {
-    constexpr int R = 16;
+  // Small heads: 4 query blocks per CTA so the grid still fills the GPU.
+  auto launch_ss = [&](auto kern, int R, int NT) -> sa_status {
     const int smem = (D * (R + 4) + R * ldL) * static_cast<int>(sizeof(float));
-    if (set_smem(sa::score_select_kernel<D, R>, smem) != SA_OK) return SA_ERR_CUDA;
-    sa::score_select_kernel<D, R><<<dim3((Nb + R - 1) / R, static_cast<unsigned>(BH)), 256, smem, st>>>(
-        Qp, Kp, Nb, scale, causal, tau, mask, count, idx);
-  } else {
-    constexpr int R = 8;
-    const int smem = (D * (R + 4) + R * ldL) * static_cast<int>(sizeof(float));
-    if (set_smem(sa::score_select_kernel<D, R>, smem) != SA_OK) return SA_ERR_CUDA;
-    sa::score_select_kernel<D, R><<<dim3((Nb + R - 1) / R, static_cast<unsigned>(BH)), 256, smem, st>>>(
-        Qp, Kp, Nb, scale, causal, tau, mask, count, idx);
-  }
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return SA_ERR_CUDA;
+    kern<<<dim3((Nb + R - 1) / R, static_cast<unsigned>(BH)), NT, smem, st>>>(Qp, Kp, Nb, scale, causal, tau,
+                                                                               mask, count, idx);
+    return SA_OK;
+  };
+  sa_status ls;
+  if (Nb <= 256)
+    ls = launch_ss(sa::score_select_kernel<D, 4, 128>, 4, 128);
+  else if (Nb <= 3000)
+    ls = launch_ss(sa::score_select_kernel<D, 16, 256>, 16, 256);
+  else
+    ls = launch_ss(sa::score_select_kernel<D, 8, 256>, 8, 256);
+  if (ls != SA_OK) return ls;
   if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
 
   if (work) {
     const int Tq = (Nb + 1) / 2;
     const int smem = sa::pair_order_smem_bytes(Nb);
     if (set_smem(sa::pair_order_kernel, smem) != SA_OK) return SA_ERR_CUDA;
-    sa::pair_order_kernel<<<static_cast<unsigned>(BH), 1024, smem, st>>>(mask, count, Nb, Tq, work);
+    sa::pair_order_kernel<<<static_cast<unsigned>(BH), Nb <= 512 ? 256 : 1024, smem, st>>>(mask, count, Nb, Tq, work);
     if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   }
   return SA_OK;
@@ -120,7 +143,7 @@ sa_status launch_fwd(const sa_shape& s, const void* Q, const void* K, const void
   const long long tiles = static_cast<long long>(s.B) * s.H * Tq;
   if (tiles > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, Q, s, 64) || !make_map(&mk, K, s, 64) || !make_map(&mv, V, s, 64)) return SA_ERR_CUDA;
+  if (!make_map(&mq, Q, s, 64) || !make_block_map(&mk, K, s) || !make_block_map(&mv, V, s)) return SA_ERR_CUDA;
   if (stats && cudaMemsetAsync(stats, 0, 4 * sizeof(int64_t), st) != cudaSuccess) return SA_ERR_CUDA;
   auto kern = sa::fwd_kernel<D>;
   if (set_smem(kern, Cfg::kSmemBytes) != SA_OK) return SA_ERR_CUDA;

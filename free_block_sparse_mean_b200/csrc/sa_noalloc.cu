@@ -75,23 +75,23 @@ sa_status launch_plan_noalloc(const sa_shape& s, const void* Q, const void* K, f
       static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Qp, Kp, s.N, Nb);
   if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   const int ldL = (Nb + 3) & ~3;
-  if (Nb <= 3000) {
-    constexpr int R = 16;
+  // Small heads: 4 query blocks per CTA so the grid still fills the GPU.
+  auto launch_ss = [&](auto kern, int R, int NT) -> sa_status {
     const int smem = (D * (R + 4) + R * ldL) * static_cast<int>(sizeof(float));
-    if (cudaFuncSetAttribute(sa::score_select_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return SA_ERR_CUDA;
-    sa::score_select_kernel<D, R><<<dim3((Nb + R - 1) / R, static_cast<unsigned>(BH)), 256, smem, st>>>(
-        Qp, Kp, Nb, scale, causal, tau, mask, count, idx);
-  } else {
-    constexpr int R = 8;
-    const int smem = (D * (R + 4) + R * ldL) * static_cast<int>(sizeof(float));
-    if (cudaFuncSetAttribute(sa::score_select_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
-      return SA_ERR_CUDA;
-    sa::score_select_kernel<D, R><<<dim3((Nb + R - 1) / R, static_cast<unsigned>(BH)), 256, smem, st>>>(
-        Qp, Kp, Nb, scale, causal, tau, mask, count, idx);
-  }
+    kern<<<dim3((Nb + R - 1) / R, static_cast<unsigned>(BH)), NT, smem, st>>>(Qp, Kp, Nb, scale, causal, tau,
+                                                                               mask, count, idx);
+    return SA_OK;
+  };
+  sa_status ls;
+  if (Nb <= 256)
+    ls = launch_ss(sa::score_select_kernel<D, 4, 128>, 4, 128);
+  else if (Nb <= 3000)
+    ls = launch_ss(sa::score_select_kernel<D, 16, 256>, 16, 256);
+  else
+    ls = launch_ss(sa::score_select_kernel<D, 8, 256>, 8, 256);
+  if (ls != SA_OK) return ls;
   if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   if (work) {
     const int Tq = (Nb + 1) / 2;
@@ -99,7 +99,7 @@ sa_status launch_plan_noalloc(const sa_shape& s, const void* Q, const void* K, f
     if (cudaFuncSetAttribute(sa::pair_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
       return SA_ERR_CUDA;
-    sa::pair_order_kernel<<<static_cast<unsigned>(BH), 1024, smem, st>>>(mask, count, Nb, Tq, work);
+    sa::pair_order_kernel<<<static_cast<unsigned>(BH), Nb <= 512 ? 256 : 1024, smem, st>>>(mask, count, Nb, Tq, work);
     if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   }
   return SA_OK;
