@@ -1,0 +1,62 @@
+"""Parity at the full workload sizes, in the launch configuration the benchmark
+times (plan with the tile order, forward over the plan's pairs).
+
+Masks: every head (every 4th for the extra centroid weights) against the
+oracle's plan (exact outside the 1e-4 band).
+Outputs: the oracle run with the GPU's own mask on sampled query blocks (the
+first, the last, which is the ragged tail when N % 64 != 0, and seeded random
+ones) of a few heads; each query block's output is independent given the mask,
+so the sampled rows are exact comparisons."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import sparse_attn_oracle as orc
+from tests.helpers import assert_output_close, check_plan_consistency, compare_masks, to_np
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+if torch.cuda.is_available():
+    import free_block_sparse_mean_b200 as sa
+    from free_block_sparse_mean_b200 import workloads as wl
+
+CASES = [
+    # workload, tau, lambda, centroid weight, heads whose outputs are sampled, mask-head stride
+    ("wan", 0.95, None, None, (0, 23), 1),
+    ("hunyuan", 0.95, -12.0, None, (0, 17), 1),
+    ("hunyuan", 0.90, -12.0, 3.0, (5,), 4),
+    ("hunyuan", 0.90, -12.0, 0.5, (9,), 4),
+    ("lm", 0.95, None, None, (0, 31), 1),
+]
+
+
+@pytest.mark.parametrize("name,tau,lam,cw,out_heads,stride", CASES)
+def test_full_size_masks_and_sampled_outputs(name, tau, lam, cw, out_heads, stride):
+    dev = torch.device("cuda:0")
+    w = wl.WORKLOADS[name]
+    q, k, v = wl.generate(w, seed=0, device=dev, centroid_weight=cw)
+    plan = sa.sparse_attn_plan(q, k, tau, None, w.causal)
+    out = sa.sparse_attn_fwd(q, k, v, plan, lam)
+    torch.cuda.synchronize()
+    assert sa.sparse_attn_device_error() == 0
+    Nb = -(-w.N // 64)
+    mask = to_np(plan.mask)
+    check_plan_consistency(mask[0, :2], to_np(plan.count)[0, :2], to_np(plan.idx)[0, :2])
+    rows_diff = excused = 0
+    heads = range(0, w.H, stride)
+    for h in heads:
+        qh, kh = q[:, h:h + 1].cpu(), k[:, h:h + 1].cpu()
+        op = orc.plan(qh, kh, tau, None, w.causal)
+        r, e = compare_masks(mask[:, h:h + 1], op, tau)
+        rows_diff += r
+        excused += e
+    print(f"{name} tau={tau} cw={cw}: rows differing {rows_diff} of {len(heads) * Nb}, excused blocks {excused}, "
+          f"density {mask.mean():.3f}")
+    assert rows_diff <= max(2, (len(heads) * Nb) // 500)
+    rng = np.random.default_rng(7)
+    for h in out_heads:
+        qbs = sorted({0, Nb - 1, *rng.choice(Nb, size=4, replace=False).tolist()})
+        qh, kh, vh = (x[:, h:h + 1].cpu() for x in (q, k, v))
+        ref = orc.fwd(qh, kh, vh, mask[:, h:h + 1], lam, None, w.causal, qblocks=qbs)
+        got = to_np(out[:, h:h + 1])
+        assert_output_close(got, ref, f"{name} head {h} query blocks {qbs}")
