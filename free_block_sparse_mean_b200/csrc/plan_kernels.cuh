@@ -14,6 +14,36 @@
 
 namespace sa {
 
+// Byte offsets of the plan workspace: pooled Q and K (fp32 [B,H,Nb,d]), then per
+// query block a 64-bit MinHash sort key and the kept set as a bitset of W words.
+struct PlanWorkspace {
+  size_t qp, kp, sig, bits, total;
+  int W;
+};
+inline PlanWorkspace plan_workspace(long long BH, int Nb, int D) {
+  auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+  PlanWorkspace w;
+  w.W = (Nb + 31) / 32;
+  const size_t pooled = al(static_cast<size_t>(BH) * Nb * D * sizeof(float));
+  w.qp = 0;
+  w.kp = pooled;
+  w.sig = 2 * pooled;
+  w.bits = w.sig + al(static_cast<size_t>(BH) * Nb * sizeof(unsigned long long));
+  w.total = w.bits + al(static_cast<size_t>(BH) * Nb * w.W * sizeof(uint32_t));
+  return w;
+}
+
+// MurmurHash3's 32-bit finaliser (a published bijective mixer): MinHash of kept sets.
+static __device__ __forceinline__ uint32_t mix32(uint32_t x) {
+  // MurmurHash3's 32-bit finaliser (a published bijective mixer).
+  x ^= x >> 16;
+  x *= 0x85ebca6bu;
+  x ^= x >> 13;
+  x *= 0xc2b2ae35u;
+  x ^= x >> 16;
+  return x;
+}
+
 // ----------------------------------------------------------------------------
 // Pool: Xp[bh, i, :] = mean of X[bh, 64 i : min(N, 64 i + 64), :], fp32.
 // One CTA per (block, head) and per tensor (blockIdx.y: 0 = Q, 1 = K). Each
@@ -86,7 +116,9 @@ __global__ void __launch_bounds__(NT) score_select_kernel(const float* __restric
                                                            float scale, int causal, float tau,
                                                            uint8_t* __restrict__ mask,
                                                            int* __restrict__ count,
-                                                           int* __restrict__ idx) {
+                                                           int* __restrict__ idx,
+                                                           unsigned long long* __restrict__ sig,
+                                                           uint32_t* __restrict__ bits) {
   static_assert(R % 4 == 0 && R <= 16 && NT % 32 == 0, "R rows per CTA, NT threads");
   constexpr int kCols = 2 * NT;  // key blocks per pass of phase 1
   constexpr int QS = R + 4;  // padded row stride of the transposed query tile
@@ -229,6 +261,8 @@ __global__ void __launch_bounds__(NT) score_select_kernel(const float* __restric
     // emit mask, ascending idx, count
     uint8_t* mrow = mask + (bh * Nb + i) * static_cast<long long>(Nb);
     int* irow = idx ? idx + (bh * Nb + i) * static_cast<long long>(Nb) : nullptr;
+    uint32_t* brow = bits ? bits + (bh * Nb + i) * static_cast<long long>((Nb + 31) / 32) : nullptr;
+    uint32_t s1 = 0xffffffffu, s2 = 0xffffffffu;  // MinHash signatures of the kept set
     int kept = 0, ties_seen = 0;
     for (int jb = 0; jb < Nb; jb += 32) {
       const int j = jb + lane;
@@ -242,9 +276,26 @@ __global__ void __launch_bounds__(NT) score_select_kernel(const float* __restric
       const unsigned kb = __ballot_sync(FULL, keep);
       if (j < Nb) mrow[j] = keep ? 1 : 0;
       if (irow && keep) irow[kept + __popc(kb & ((1u << lane) - 1u))] = j;
+      if (brow && lane == 0) brow[jb >> 5] = kb;
+      if (keep) {
+        s1 = min(s1, mix32(static_cast<uint32_t>(j) ^ 0x9e3779b9u));
+        s2 = min(s2, mix32(static_cast<uint32_t>(j) + 0x7f4a7c15u));
+      }
       kept += __popc(kb);
     }
-    if (lane == 0) count[bh * Nb + i] = kept;
+    if (sig) {
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        s1 = min(s1, __shfl_xor_sync(FULL, s1, o));
+        s2 = min(s2, __shfl_xor_sync(FULL, s2, o));
+      }
+    }
+    if (lane == 0) {
+      count[bh * Nb + i] = kept;
+      if (sig)
+        sig[bh * Nb + i] = (static_cast<unsigned long long>(s1) << 32) |
+                           (static_cast<unsigned long long>(s2 & 0xffffu) << 16) | static_cast<unsigned long long>(i);
+    }
   }
 }
 
@@ -265,15 +316,6 @@ __global__ void __launch_bounds__(NT) score_select_kernel(const float* __restric
 constexpr int kPairGreedyMaxNb = 1024;
 constexpr int kPairWindow = 32;
 
-static __device__ __forceinline__ uint32_t mix32(uint32_t x) {
-  // MurmurHash3's 32-bit finaliser (a published bijective mixer).
-  x ^= x >> 16;
-  x *= 0x85ebca6bu;
-  x ^= x >> 13;
-  x *= 0xc2b2ae35u;
-  x ^= x >> 16;
-  return x;
-}
 
 // In-place ascending bitonic sort of n64 (a power of two) 64-bit keys in shared memory.
 static __device__ void block_bitonic_sort(unsigned long long* keys, int n64) {
@@ -294,7 +336,8 @@ static __device__ void block_bitonic_sort(unsigned long long* keys, int n64) {
   }
 }
 
-static __global__ void __launch_bounds__(1024) pair_order_kernel(const uint8_t* __restrict__ mask,
+static __global__ void __launch_bounds__(1024) pair_order_kernel(const unsigned long long* __restrict__ sig,
+                                                                 const uint32_t* __restrict__ bits_g,
                                                                  const int* __restrict__ count, int Nb,
                                                                  int Tq, int* __restrict__ work) {
   extern __shared__ __align__(16) unsigned char psm[];
@@ -310,36 +353,20 @@ static __global__ void __launch_bounds__(1024) pair_order_kernel(const uint8_t* 
   int* used = order + Nb;                                                        // [Nb]
   uint32_t* bits = reinterpret_cast<uint32_t*>(used + Nb);                      // [Nb][W] (greedy only)
   const long long bh = blockIdx.x;
-  const uint8_t* m = mask + bh * static_cast<long long>(Nb) * Nb;
   const int* cnt = count + bh * Nb;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned FULL = 0xffffffffu;
 
-  // 1. signatures (and bitsets) of every query block's kept set
-  for (int i = warp; i < Nb; i += nwarps) {
-    uint32_t s1 = 0xffffffffu, s2 = 0xffffffffu;
-    const uint8_t* row = m + static_cast<long long>(i) * Nb;
-    for (int jb = 0; jb < Nb; jb += 32) {
-      const int j = jb + lane;
-      const bool kept = (j < Nb) && row[j] != 0;
-      if (kept) {
-        s1 = min(s1, mix32(static_cast<uint32_t>(j) ^ 0x9e3779b9u));
-        s2 = min(s2, mix32(static_cast<uint32_t>(j) + 0x7f4a7c15u));
-      }
-      const unsigned bal = __ballot_sync(FULL, kept);
-      if (greedy && lane == 0) bits[i * W + jb / 32] = bal;
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-      s1 = min(s1, __shfl_xor_sync(FULL, s1, o));
-      s2 = min(s2, __shfl_xor_sync(FULL, s2, o));
-    }
-    if (lane == 0)
-      keys[i] = (static_cast<unsigned long long>(s1) << 32) | (static_cast<unsigned long long>(s2 & 0xffffu) << 16) |
-                static_cast<unsigned long long>(i);
+  // 1. MinHash keys (from the selection kernel), bitsets into shared memory
+  for (int i = threadIdx.x; i < Nb; i += blockDim.x) {
+    keys[i] = sig[bh * Nb + i];
+    used[i] = 0;
   }
   for (int i = Nb + threadIdx.x; i < P; i += blockDim.x) keys[i] = ~0ull;
-  for (int i = threadIdx.x; i < Nb; i += blockDim.x) used[i] = 0;
+  if (greedy) {
+    const uint32_t* src = bits_g + bh * static_cast<long long>(Nb) * W;
+    for (int x = threadIdx.x; x < Nb * W; x += blockDim.x) bits[x] = src[x];
+  }
   __syncthreads();
   block_bitonic_sort(keys, P);
   for (int i = threadIdx.x; i < Nb; i += blockDim.x) order[i] = static_cast<int>(keys[i] & 0xffffu);

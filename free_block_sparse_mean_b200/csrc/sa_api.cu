@@ -29,9 +29,6 @@ sa_status check_shape(const sa_shape& s) {
   return SA_OK;
 }
 
-size_t pooled_bytes(const sa_shape& s) {
-  return align_up(static_cast<size_t>(s.B) * s.H * num_blocks(s) * s.d * sizeof(float), 256);
-}
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
@@ -97,8 +94,12 @@ sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau
                       uint8_t* mask, int32_t* count, int32_t* idx, int32_t* work, void* ws, cudaStream_t st) {
   const int Nb = static_cast<int>(num_blocks(s));
   const long long BH = static_cast<long long>(s.B) * s.H;
-  float* Qp = static_cast<float*>(ws);
-  float* Kp = reinterpret_cast<float*>(static_cast<char*>(ws) + pooled_bytes(s));
+  const sa::PlanWorkspace L = sa::plan_workspace(BH, Nb, D);
+  char* wsb = static_cast<char*>(ws);
+  float* Qp = reinterpret_cast<float*>(wsb + L.qp);
+  float* Kp = reinterpret_cast<float*>(wsb + L.kp);
+  unsigned long long* sig = reinterpret_cast<unsigned long long*>(wsb + L.sig);
+  uint32_t* bits = reinterpret_cast<uint32_t*>(wsb + L.bits);
   sa::pool_kernel<D><<<dim3(static_cast<unsigned>(BH * Nb), 2), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Qp, Kp, s.N, Nb);
   if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
@@ -110,7 +111,7 @@ sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return SA_ERR_CUDA;
     kern<<<dim3((Nb + R - 1) / R, static_cast<unsigned>(BH)), NT, smem, st>>>(Qp, Kp, Nb, scale, causal, tau,
-                                                                               mask, count, idx);
+                                                                               mask, count, idx, sig, bits);
     return SA_OK;
   };
   sa_status ls;
@@ -127,7 +128,7 @@ sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau
     const int Tq = (Nb + 1) / 2;
     const int smem = sa::pair_order_smem_bytes(Nb);
     if (set_smem(sa::pair_order_kernel, smem) != SA_OK) return SA_ERR_CUDA;
-    sa::pair_order_kernel<<<static_cast<unsigned>(BH), Nb <= 512 ? 256 : 1024, smem, st>>>(mask, count, Nb, Tq, work);
+    sa::pair_order_kernel<<<static_cast<unsigned>(BH), Nb <= 512 ? 256 : 1024, smem, st>>>(sig, bits, count, Nb, Tq, work);
     if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   }
   return SA_OK;
@@ -163,7 +164,7 @@ extern "C" {
 
 size_t sparse_attn_plan_workspace_size(sa_shape s) {
   if (check_shape(s) != SA_OK) return 0;
-  return 2 * pooled_bytes(s);
+  return sa::plan_workspace(static_cast<long long>(s.B) * s.H, static_cast<int>(num_blocks(s)), s.d).total;
 }
 
 int64_t sparse_attn_num_tiles(sa_shape s) {

@@ -10,11 +10,12 @@
 // array of device memory that is part of the loaded library.
 //
 // Scratch: kNoAllocScratchBytes = 32 MiB, a file-scope __device__ array. Every
-// GPU that loads the library holds it until the process exits. The pooled
-// tensors take 2 * B*H*ceil(N/64)*d*4 bytes (each 256-byte aligned), so a call
-// fits when B*H*ceil(N/64)*d <= 4,194,304 values per tensor (for example H=24,
-// d=128 up to N = 87,360). Larger calls are rejected with SA_ERR_WORKSPACE
-// before anything runs.
+// GPU that loads the library holds it until the process exits. A call needs the
+// same bytes as sparse_attn_plan_workspace_size: the pooled Q and K
+// (2 * B*H*ceil(N/64)*d*4 bytes) plus, per query block, an 8-byte sort key and a
+// ceil(Nb/32)-word bitset of its kept set (for example H=24, d=128 fits up to
+// N = 75,776). Larger calls are rejected with SA_ERR_WORKSPACE before
+// anything runs.
 //
 // Every call shares the one array, and the array keeps the last call's
 // contents. The kernels write every scratch byte they later read, so nothing
@@ -43,11 +44,6 @@ __device__ __align__(256) unsigned char g_plan_scratch[kNoAllocScratchBytes];
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 
-size_t pooled_bytes_noalloc(const sa_shape& s) {
-  const size_t nb = (static_cast<size_t>(s.N) + 63) / 64;
-  const size_t b = static_cast<size_t>(s.B) * s.H * nb * s.d * sizeof(float);
-  return (b + 255) / 256 * 256;
-}
 
 // Device address of the scratch array on the current device (set up once per device).
 sa_status scratch_for_current_device(void** out) {
@@ -69,8 +65,12 @@ sa_status launch_plan_noalloc(const sa_shape& s, const void* Q, const void* K, f
                               void* scratch, cudaStream_t st) {
   const int Nb = static_cast<int>((static_cast<int64_t>(s.N) + 63) / 64);
   const long long BH = static_cast<long long>(s.B) * s.H;
-  float* Qp = static_cast<float*>(scratch);
-  float* Kp = reinterpret_cast<float*>(static_cast<char*>(scratch) + pooled_bytes_noalloc(s));
+  const sa::PlanWorkspace L = sa::plan_workspace(BH, Nb, D);
+  char* wsb = static_cast<char*>(scratch);
+  float* Qp = reinterpret_cast<float*>(wsb + L.qp);
+  float* Kp = reinterpret_cast<float*>(wsb + L.kp);
+  unsigned long long* sig = reinterpret_cast<unsigned long long*>(wsb + L.sig);
+  uint32_t* bits = reinterpret_cast<uint32_t*>(wsb + L.bits);
   sa::pool_kernel<D><<<dim3(static_cast<unsigned>(BH * Nb), 2), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Qp, Kp, s.N, Nb);
   if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
@@ -81,7 +81,7 @@ sa_status launch_plan_noalloc(const sa_shape& s, const void* Q, const void* K, f
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return SA_ERR_CUDA;
     kern<<<dim3((Nb + R - 1) / R, static_cast<unsigned>(BH)), NT, smem, st>>>(Qp, Kp, Nb, scale, causal, tau,
-                                                                               mask, count, idx);
+                                                                               mask, count, idx, sig, bits);
     return SA_OK;
   };
   sa_status ls;
@@ -99,7 +99,7 @@ sa_status launch_plan_noalloc(const sa_shape& s, const void* Q, const void* K, f
     if (cudaFuncSetAttribute(sa::pair_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
       return SA_ERR_CUDA;
-    sa::pair_order_kernel<<<static_cast<unsigned>(BH), Nb <= 512 ? 256 : 1024, smem, st>>>(mask, count, Nb, Tq, work);
+    sa::pair_order_kernel<<<static_cast<unsigned>(BH), Nb <= 512 ? 256 : 1024, smem, st>>>(sig, bits, count, Nb, Tq, work);
     if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   }
   return SA_OK;
@@ -118,7 +118,9 @@ extern "C" sa_status sparse_attn_plan_noalloc(const void* Q, const void* K, sa_s
   if (!(tau > 0.f && tau <= 1.f)) return SA_ERR_INVALID_ARG;
   if (!(std::isfinite(scale) && scale > 0.f)) return SA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(Q) & 15u) || (reinterpret_cast<uintptr_t>(K) & 15u)) return SA_ERR_INVALID_ARG;
-  if (2 * pooled_bytes_noalloc(s) > kNoAllocScratchBytes) return SA_ERR_WORKSPACE;  // beyond the fixed scratch
+  const sa::PlanWorkspace need = sa::plan_workspace(static_cast<long long>(s.B) * s.H,
+                                                    static_cast<int>((static_cast<int64_t>(s.N) + 63) / 64), s.d);
+  if (need.total > kNoAllocScratchBytes) return SA_ERR_WORKSPACE;  // beyond the fixed scratch
   void* scratch = nullptr;
   const sa_status got = scratch_for_current_device(&scratch);
   if (got != SA_OK) return got;

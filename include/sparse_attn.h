@@ -60,8 +60,9 @@ typedef struct {
   int32_t block; /* mask block size, must be 64 */
 } sa_shape;
 
-/* Bytes of device workspace sparse_attn_plan needs for shape s (pooled Q and K,
- * fp32 [B,H,Nb,d] each, 256-byte aligned). 0 if the shape is invalid. */
+/* Bytes of device workspace sparse_attn_plan needs for shape s: pooled Q and K
+ * (fp32 [B,H,Nb,d] each), an 8-byte sort key and a ceil(Nb/32)-word kept-set
+ * bitset per query block, each region 256-byte aligned. 0 if the shape is invalid. */
 size_t sparse_attn_plan_workspace_size(sa_shape s);
 
 /* Number of 128-row query tiles, B*H*ceil(Nb/2); `work` holds two entries per
@@ -132,10 +133,11 @@ sa_status sparse_attn_fwd(const void* Q, const void* K, const void* V, sa_shape 
  * cudaMalloc). The paper has no counterpart: this is a deployment variant.
  *
  * Same arguments, outputs and errors as sparse_attn_plan, minus the workspace.
- * The pooled Q and K go to a fixed 32 MiB device array inside the library, held
- * by every GPU that loads the library until the process exits; the call fits when
- * B*H*ceil(N/64)*d <= 4,194,304 and returns SA_ERR_WORKSPACE (nothing launched)
- * otherwise. It calls no allocator. The first call on a device looks up the
+ * Its scratch (the same bytes sparse_attn_plan_workspace_size reports) goes to a
+ * fixed 32 MiB device array inside the library, held by every GPU that loads the
+ * library until the process exits; the call fits when that size is <= 32 MiB
+ * (e.g. H=24, d=128 up to N = 75,776) and returns SA_ERR_WORKSPACE (nothing
+ * launched) otherwise. It calls no allocator. The first call on a device looks up the
  * array's device address and caches it; make that first call before any stream
  * capture on the device. All calls share the array (it keeps the last call's
  * contents, and nothing in it needs to start at zero), so calls that overlap on

@@ -67,6 +67,6 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     dev = torch.device("cuda:0")
     q = torch.zeros((1, 1, 64, 128), dtype=torch.bfloat16, device=dev)
     out = _outputs(1, 1, 1, 1, dev)
-    big = SaShape(1, 40, 75600, 128, 64)     # 40*1182*128 pooled values per tensor > 4,194,304
+    big = SaShape(1, 40, 75600, 128, 64)     # needs about 50 MB of scratch > 32 MiB
     st = lib.sparse_attn_plan_noalloc(_p(q), _p(q), big, 0.9, 0.1, 0, *(_p(t) for t in out), None)
     assert st == 3                          # SA_ERR_WORKSPACE, nothing launched
