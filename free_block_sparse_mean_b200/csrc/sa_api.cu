@@ -16,7 +16,6 @@ namespace {
 
 inline int64_t num_blocks(const sa_shape& s) { return (static_cast<int64_t>(s.N) + 63) / 64; }
 
-inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
