@@ -72,6 +72,27 @@ def peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def measured_traffic(w, tau, lam):
+    """DRAM bytes per launch of the forward kernel from the committed ncu capture,
+    or None if the kernel source changed since (or the workload differs)."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "fwd_kernel_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    h = hashlib.sha256()
+    for src in d.get("sources", []):
+        with open(os.path.join(ROOT, src), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != d.get("source_sha256"):
+        return None
+    key = f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.D} tau={tau:g} lambda={lam if lam is not None else 'off'}"
+    key = key.replace("lambda=-12.0", "lambda=-12")
+    ent = d.get("traffic_bytes_per_launch", {}).get(key)
+    return None if ent is None else float(ent["total"])
+
+
 def dense_flops(w):
     if w.causal:
         return 2.0 * w.B * w.H * w.N * (w.N + 1) * w.D
@@ -375,7 +396,7 @@ def run_ours(args, w, world, rank, local, pg):
         "executed_tflops": achieved, "pct_of_bf16_peak_executed": 100.0 * achieved / peak_t,
         "predictor_pct_of_dense": None if dense_ms is None else 100.0 * plan_avg / dense_ms,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
-                     "frac": achieved / peak_t, "traffic": None,
+                     "frac": achieved / peak_t, "traffic": measured_traffic(w, args.tau, lam),
                      "kernel": "fwd_kernel<128,3> (sparse_attn_fwd)",
                      "peak_source": f"{pk_kind} bf16_tflops (burst)"},
         "e2e": e2e, "gpu_launches": 4 * args.steps, "cuda_graphs": not args.no_graph, "clocks": clocks,
