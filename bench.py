@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--heads", type=int, default=None,
                     help="run only the first H heads of the workload (profiling captures)")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense (full-mask) reference timing")
+    ap.add_argument("--sweep", action="store_true",
+                    help="one JSON line per configured (workload, tau, lambda, centroid weight); kernel timing only")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch plan and forward directly instead of replaying CUDA graphs")
     return ap.parse_args()
@@ -254,6 +256,13 @@ def config_dict(w, args, world):
             "centroid_weight": args.centroid_weight}
 
 
+def check_device(sa, where):
+    """A bounded wait that ran out or a range check makes every number void."""
+    code = sa.sparse_attn_device_error()
+    if code:
+        raise RuntimeError(f"device-side check fired during {where}: error word {code}")
+
+
 def run_ours(args, w, world, rank, local, pg):
     import free_block_sparse_mean_b200 as sa
     if not torch.cuda.is_available():
@@ -281,6 +290,7 @@ def run_ours(args, w, world, rank, local, pg):
     sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False)
     sa.sparse_attn_fwd(q, k, v, plan, lam, out=out, stats=stats)
     torch.cuda.synchronize()
+    check_device(sa, "the stats pass")
     st = [int(x) for x in stats.cpu()]
     n_tok = torch.full((Nb,), 64, dtype=torch.float64, device=dev)
     n_tok[-1] = N - 64 * (Nb - 1)
@@ -308,6 +318,7 @@ def run_ours(args, w, world, rank, local, pg):
         e1.record(stream)
         torch.cuda.synchronize()
         dense_ms = e0.elapsed_time(e1)
+        check_device(sa, "the dense (full-mask) reference")
         del full
 
     def run_plan():
@@ -351,6 +362,7 @@ def run_ours(args, w, world, rank, local, pg):
     torch.cuda.synchronize()
     barrier(pg, dev)
     clocks = sampler.stop()
+    check_device(sa, "the timed steps")
     plan_ms = [a.elapsed_time(b) for a, b, _ in ev]
     fwd_ms = [b.elapsed_time(c) for _, b, c in ev]
     step_ms_local = sum(p + f for p, f in zip(plan_ms, fwd_ms)) / args.steps
@@ -376,6 +388,7 @@ def run_ours(args, w, world, rank, local, pg):
             b.record(stream)
             torch.cuda.synchronize()
             t.append(a.elapsed_time(b))
+        check_device(sa, "the end-to-end calls")
         e2e_ms = reduce_max(pg, statistics.mean(t), dev)
         e2e = {"value": world * dflops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                "ms_per_call": e2e_ms,
@@ -397,7 +410,7 @@ def run_ours(args, w, world, rank, local, pg):
         "predictor_pct_of_dense": None if dense_ms is None else 100.0 * plan_avg / dense_ms,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": achieved / peak_t, "traffic": measured_traffic(w, args.tau, lam),
-                     "kernel": "fwd_kernel<128,3> (sparse_attn_fwd)",
+                     "kernel": f"fwd_kernel<{D}> (sparse_attn_fwd)",
                      "peak_source": f"{pk_kind} bf16_tflops (burst)"},
         "e2e": e2e, "gpu_launches": 4 * args.steps, "cuda_graphs": not args.no_graph, "clocks": clocks,
     }
@@ -409,8 +422,26 @@ def run_ours(args, w, world, rank, local, pg):
         print(json.dumps(line), flush=True)
 
 
+def sweep(args):
+    """Every configured point of every workload (one GPU, kernel timing only)."""
+    base = dict(vars(args))
+    for name, w in wl.WORKLOADS.items():
+        cws = w.centroid_weights or (None,)
+        for tau in w.taus:
+            for lam in w.lams:
+                for cw in cws:
+                    a = argparse.Namespace(**base)
+                    a.workload, a.tau, a.lam, a.centroid_weight = name, tau, "off" if lam is None else str(lam), cw
+                    a.no_e2e, a.no_cpu, a.steps, a.warmup = True, True, min(args.steps, 5), 3
+                    run_ours(a, w, 1, 0, 0, None)
+                    torch.cuda.empty_cache()
+
+
 def main():
     args = parse()
+    if args.sweep:
+        sweep(args)
+        return
     w = wl.WORKLOADS[args.workload]
     if args.heads:
         w = w.with_(H=min(args.heads, w.H))

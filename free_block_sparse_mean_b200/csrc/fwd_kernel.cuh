@@ -31,9 +31,15 @@
 // max grows by more than 2^8), which leaves O/l unchanged and makes the O
 // correction rare; the softmax waits for the previous P.V only when it has to
 // correct O. The lambda test uses the exact running max.
-// An mbarrier wait by parity is only sound when the waiter is at most one phase
-// behind; the barriers below are laid out so that every wait satisfies that
-// (double-buffered P.V completion, a single-phase barrier for the epilogue).
+// An mbarrier wait by parity is only sound when the barrier is at most one phase
+// ahead of, and at most one phase short of, the phase waited for; otherwise the
+// parity aliases and the wait returns early or never. The barriers below are laid
+// out so that every wait satisfies that. P(k) ready and P(k).V finished are
+// double-buffered by k parity: S(k+1) is already in TMEM when the MMA thread
+// waits for P(k), so the softmax can publish P(k) and P(k+1) before that thread
+// looks, and one barrier would then be two phases ahead; entry k+2 cannot be
+// published before S(k+2) is issued, which comes after that wait. The epilogue
+// waits on a single-phase barrier.
 #pragma once
 
 #include "sa_device.cuh"
@@ -90,10 +96,10 @@ __global__ void __launch_bounds__(256, 2)
   uint64_t* vempty = vfull + C::STV;           // [STV] V stage consumed by P.V MMA
   uint64_t* q_full = vempty + C::STV;          // Q tile loaded
   uint64_t* s_full = q_full + 1;               // [2] S buffer written by MMA
-  uint64_t* p_full = q_full + 3;               // P(k) in TMEM and O corrected (4 warp arrivals)
-  uint64_t* pv_done = q_full + 4;              // [2] by k parity: P(k).V finished
-  uint64_t* vote_bar = q_full + 6;             // lambda vote of the 4 softmax warps
-  uint64_t* drain = q_full + 7;                // every MMA of the tile finished (single phase)
+  uint64_t* p_full = q_full + 3;               // [2] by k parity: P(k) in TMEM and O corrected (4 warp arrivals)
+  uint64_t* pv_done = q_full + 5;              // [2] by k parity: P(k).V finished
+  uint64_t* vote_bar = q_full + 7;             // lambda vote of the 4 softmax warps
+  uint64_t* drain = q_full + 8;                // every MMA of the tile finished (single phase)
   int* misc = reinterpret_cast<int*>(base + C::oMisc);
   volatile int* abort_flag = misc + 0;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(misc + 1);
@@ -134,7 +140,8 @@ __global__ void __launch_bounds__(256, 2)
     mbar_init(q_full, 1);
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
-    mbar_init(p_full, 4);
+    mbar_init(&p_full[0], 4);
+    mbar_init(&p_full[1], 4);
     mbar_init(&pv_done[0], 1);
     mbar_init(&pv_done[1], 1);
     mbar_init(vote_bar, 4);
@@ -252,7 +259,7 @@ __global__ void __launch_bounds__(256, 2)
       uint32_t o_init = 0;
       unsigned long long pv_tiles = 0;
       for (int k = 0; ok && k < n; ++k) {
-        if (!mbar_wait(p_full, static_cast<uint32_t>(k) & 1u, abort_flag)) break;
+        if (!mbar_wait(&p_full[k & 1], static_cast<uint32_t>(k >> 1) & 1u, abort_flag)) break;
         const int s = k % C::STV;
         if (!mbar_wait(&vfull[s], static_cast<uint32_t>(k / C::STV) & 1u, abort_flag)) break;
         tc_fence_after();
@@ -401,7 +408,7 @@ __global__ void __launch_bounds__(256, 2)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[k & 1]);
     }
     // ------------------------------------------------------------ epilogue
     if (alive && n > 0) {

@@ -60,3 +60,26 @@ def test_full_size_masks_and_sampled_outputs(name, tau, lam, cw, out_heads, stri
         ref = orc.fwd(qh, kh, vh, mask[:, h:h + 1], lam, None, w.causal, qblocks=qbs)
         got = to_np(out[:, h:h + 1])
         assert_output_close(got, ref, f"{name} head {h} query blocks {qbs}")
+
+
+def test_full_mask_natural_pairs_repeated():
+    """Full mask over every key block, tiles in natural order (no plan), on the
+    peaked HunyuanVideo data (centroid weight 3): long union lists with S(k+1)
+    already resident while P(k) is published, repeated so a barrier-phase race
+    would show as a device-side timeout. Sampled rows against the oracle."""
+    dev = torch.device("cuda:0")
+    w = wl.WORKLOADS["hunyuan"]
+    q, k, v = wl.generate(w, seed=0, device=dev, centroid_weight=3.0)
+    Nb = -(-w.N // 64)
+    full = torch.ones((w.B, w.H, Nb, Nb), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+    for _ in range(3):
+        sa.sparse_attn_fwd(q, k, v, full, None, out=out, causal=w.causal)
+        torch.cuda.synchronize()
+        assert sa.sparse_attn_device_error() == 0
+    h = 11
+    qbs = [0, 777, Nb - 1]
+    qh, kh, vh = (x[:, h:h + 1].cpu() for x in (q, k, v))
+    ones = np.ones((1, 1, Nb, Nb), dtype=np.uint8)
+    ref = orc.fwd(qh, kh, vh, ones, None, None, w.causal, qblocks=qbs)
+    assert_output_close(to_np(out[:, h:h + 1]), ref, f"full mask head {h} query blocks {qbs}")
