@@ -14,32 +14,40 @@
 //   S = Q K_j^T     128x64 fp32 into TMEM (tcgen05.mma, Q and K_j TMA'd into
 //                   128B-swizzled shared memory, both K-major)
 //   softmax warps   read S from TMEM (thread = row), row max, lambda vote per
-//                   64-row half, exp2, row sum; P (bf16) written back into the
-//                   first 32 columns of the same TMEM buffer
+//                   64-row half, exp2, row sum; P (bf16) written to TMEM
 //   O += P V_j      128xD fp32 in TMEM; A operand (P) read from TMEM, B (V_j)
 //                   from shared memory as an MN-major operand
-// Roles (256 threads): warp 0 loads K, warp 3 loads V and Q (TMA; K and V as one
-// 4-D box per 64-row block, since TMA issue cost is per instruction), warp 1 issues
-// the MMAs (one thread) and owns TMEM, warp 2 builds the union list, warps 4..7
-// run the softmax, the O correction and the epilogue. S is double-buffered in
-// TMEM: S(k+1) is on the tensor cores while the softmax works on S(k), and
-// S(k+2) reuses S(k)'s buffer after P(k).V has been issued (tcgen05 MMAs of one
-// thread run in issue order). Two CTAs fit on an SM (about 105 KB of shared
-// memory and 256 TMEM columns each), so one CTA's softmax overlaps the other's
-// MMAs.
+//
+// Roles (192 threads): warp 0 builds the union list, then one of its threads loads
+// Q, K and V (TMA; K and V as one 4-D box per 64-row block, since TMA issue cost
+// is per instruction); warp 1 owns TMEM and one of its threads issues the MMAs;
+// warps 2..5 run the softmax (thread = row; warp w reaches TMEM lanes 32*(w%4) ..
+// 32*(w%4)+31), the O correction and the epilogue.
+//
+// TMEM (256 columns): S [0,64), P double buffer [64,96) and [96,128), O [128,
+// 128+D). S is released as soon as the softmax warps hold S(k) in registers, so
+// S(k+1) runs on the tensor cores while the softmax works on S(k); P(k) goes to
+// buffer k&1, whose previous reader P(k-2).V has finished by the time S(k) is
+// complete (the MMAs of one thread run in issue order). Two CTAs fit on an SM
+// (about 106 KB of shared memory and 256 TMEM columns each), so one CTA's softmax
+// also overlaps the other's MMAs.
+//
 // The running max used for the exponentials is raised lazily (only when a row's
 // max grows by more than 2^8), which leaves O/l unchanged and makes the O
-// correction rare; the softmax waits for the previous P.V only when it has to
-// correct O. The lambda test uses the exact running max.
+// correction rare. The exponentials are computed against the current reference
+// while the block's row max is still being reduced, and redone in the rare case
+// of a raise. The lambda test uses the exact running max. P(k) is stored before
+// the lambda vote of the other warp of the half is read; a half that skips then
+// overwrites its P(k) with zeros.
+//
 // An mbarrier wait by parity is only sound when the barrier is at most one phase
 // ahead of, and at most one phase short of, the phase waited for; otherwise the
-// parity aliases and the wait returns early or never. The barriers below are laid
-// out so that every wait satisfies that. P(k) ready and P(k).V finished are
-// double-buffered by k parity: S(k+1) is already in TMEM when the MMA thread
-// waits for P(k), so the softmax can publish P(k) and P(k+1) before that thread
-// looks, and one barrier would then be two phases ahead; entry k+2 cannot be
-// published before S(k+2) is issued, which comes after that wait. The epilogue
-// waits on a single-phase barrier.
+// parity aliases and the wait returns early or never. Every wait below satisfies
+// that: S(k+1) is issued only after all softmax warps released S(k); P(k+2) can be
+// published only after S(k+2), which the MMA thread issues after it has waited for
+// P(k); P.V completions are double-buffered like P. The lambda votes carry the
+// entry index as a tag, and a vote slot is reused for entry k+2 only after every
+// softmax warp has released S(k+1), which each does after reading entry k's vote.
 #pragma once
 
 #include "sa_device.cuh"
@@ -49,6 +57,7 @@ namespace sa {
 template <int D>
 struct FwdCfg {
   static constexpr int kRows = 128;                    // query rows per tile
+  static constexpr int kThreads = 192;                 // 2 role warps + 4 softmax warps
   static constexpr int kChunks = D / 64;               // 128-byte (64 x bf16) column chunks
   static constexpr int STK = (D == 64) ? 4 : 2;        // K ring stages
   static constexpr int STV = (D == 64) ? 4 : 2;        // V ring stages
@@ -61,12 +70,12 @@ struct FwdCfg {
   static constexpr int oK = oQ + kQBytes;
   static constexpr int oV = oK + STK * kKVBytes;
   static constexpr int oBar = oV + STV * kKVBytes;     // mbarriers
-  static constexpr int kNumBars = 2 * STK + 2 * STV + 9;
-  static constexpr int oMisc = oBar + kNumBars * 8;    // small words
-  static constexpr int oList = oMisc + 64;
+  static constexpr int kNumBars = 2 * STK + 2 * STV + 8;
+  static constexpr int oMisc = oBar + kNumBars * 8;    // small words (256 bytes)
+  static constexpr int oList = oMisc + 256;
   static constexpr int kSmemBytes = oList + kMaxNb * 2 + 1024;  // + alignment slack
-  // TMEM columns: two S/P buffers and the O accumulator
-  static constexpr uint32_t kColS0 = 0, kColS1 = 64, kColO = 128;
+  // TMEM columns: S, two P buffers (bf16 pairs), the O accumulator
+  static constexpr uint32_t kColS = 0, kColP0 = 64, kColP1 = 96, kColO = 128;
   static constexpr uint32_t kTmemCols = 256;
   static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, false);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
@@ -76,8 +85,31 @@ struct FwdCfg {
 constexpr uint32_t kListJMask = 0x0FFFu;
 constexpr uint32_t kListLo = 1u << 14, kListHi = 1u << 15;
 
+// p = 2^(s * scale_log2 - mref) for the 64 columns of one row; P as bf16 pairs
+// and the fp32 sum of the p. Scale-subtract and sums on fp32 pairs.
+__device__ __forceinline__ float softmax_exp64(const float (&s)[64], float scale_log2, float mref,
+                                               uint32_t (&pk)[32]) {
+  const uint64_t sc2 = f2pack(scale_log2, scale_log2), nm2 = f2pack(-mref, -mref);
+  uint64_t acc0 = f2pack(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+  for (int c = 0; c < 64; c += 2) {
+    float x0, x1;
+    f2unpack(ffma2(f2pack(s[c], s[c + 1]), sc2, nm2), x0, x1);
+    const float p0 = ex2(x0), p1 = ex2(x1);
+    if ((c >> 1) & 1)
+      acc1 = fadd2(acc1, f2pack(p0, p1));
+    else
+      acc0 = fadd2(acc0, f2pack(p0, p1));
+    pk[c >> 1] = pack_bf16x2(p0, p1);
+  }
+  float r0, r1, r2, r3;
+  f2unpack(acc0, r0, r1);
+  f2unpack(acc1, r2, r3);
+  return (r0 + r1) + (r2 + r3);
+}
+
 template <int D>
-__global__ void __launch_bounds__(256, 2)
+__global__ void __launch_bounds__(192, 2)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const uint8_t* __restrict__ mask,
                const int* __restrict__ work, __nv_bfloat16* __restrict__ O, int N, int Nb, int Tq,
@@ -95,17 +127,17 @@ __global__ void __launch_bounds__(256, 2)
   uint64_t* vfull = kempty + C::STK;           // [STV] V stage loaded
   uint64_t* vempty = vfull + C::STV;           // [STV] V stage consumed by P.V MMA
   uint64_t* q_full = vempty + C::STV;          // Q tile loaded
-  uint64_t* s_full = q_full + 1;               // [2] S buffer written by MMA
-  uint64_t* p_full = q_full + 3;               // [2] by k parity: P(k) in TMEM and O corrected (4 warp arrivals)
+  uint64_t* s_full = q_full + 1;               // S(k) written by the MMA (phase k)
+  uint64_t* s_free = q_full + 2;               // S(k) read by all 4 softmax warps (phase k)
+  uint64_t* p_full = q_full + 3;               // [2] by k parity: P(k) in TMEM and O corrected (4 warps)
   uint64_t* pv_done = q_full + 5;              // [2] by k parity: P(k).V finished
-  uint64_t* vote_bar = q_full + 7;             // lambda vote of the 4 softmax warps
-  uint64_t* drain = q_full + 8;                // every MMA of the tile finished (single phase)
+  uint64_t* drain = q_full + 7;                // every MMA of the tile finished (single phase)
   int* misc = reinterpret_cast<int*>(base + C::oMisc);
   volatile int* abort_flag = misc + 0;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(misc + 1);
   int* list_n = misc + 2;
-  volatile int* pv_need = misc + 4;            // [2] by k parity: issue P.V for entry k
-  volatile int* votes = misc + 8;              // [2][4] by k parity, per softmax warp
+  volatile int* contrib = misc + 4;            // [2 parity][2 halves]: the half's P.V is needed
+  volatile int* votes = misc + 8;              // [2 parity][4 softmax warps]: (k << 1) | pass
   uint16_t* lst = reinterpret_cast<uint16_t*>(base + C::oList);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -138,24 +170,26 @@ __global__ void __launch_bounds__(256, 2)
       mbar_init(&vempty[s], 1);
     }
     mbar_init(q_full, 1);
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 4);
     mbar_init(&p_full[0], 4);
     mbar_init(&p_full[1], 4);
     mbar_init(&pv_done[0], 1);
     mbar_init(&pv_done[1], 1);
-    mbar_init(vote_bar, 4);
     mbar_init(drain, 1);
     *abort_flag = 0;
+    for (int x = 8; x < 16; ++x) misc[x] = -1;   // vote tags -1: no entry yet
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmQ);
-    tma_prefetch_desc(&tmK);
-    tma_prefetch_desc(&tmV);
+  if (warp == 1) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+    }
+    tmem_alloc(tmem_holder, C::kTmemCols);
   }
-  if (warp == 1) tmem_alloc(tmem_holder, C::kTmemCols);
-  if (warp == 2) {
+  if (warp == 0) {
     // Ascending union of the kept lists of query blocks qb0 and qb1, one keep bit
     // per half; with causal, key blocks after a half's query block are dropped.
     const uint8_t* m0 = mask + (bh * Nb + qb0) * static_cast<long long>(Nb);
@@ -194,21 +228,9 @@ __global__ void __launch_bounds__(256, 2)
   const int n = *list_n;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ K producer
-    if (lane == 0 && n > 0) {
-      int k = 0;
-      for (; k < n; ++k) {
-        const int s = k % C::STK;
-        if (!mbar_wait(&kempty[s], (static_cast<uint32_t>(k / C::STK) & 1u) ^ 1u, abort_flag)) break;
-        const int j = static_cast<int>(lst[k] & kListJMask);
-        mbar_expect_tx(&kfull[s], C::kKVBytes);
-        tma_load_4d(sK + s * C::kKVBytes, &tmK, 0, j * kBlock, 0, static_cast<int>(bh), &kfull[s]);
-      }
-      for (int kk = max(0, k - C::STK); kk < k; ++kk)  // let issued loads land before exit
-        mbar_wait_drain(&kfull[kk % C::STK], static_cast<uint32_t>(kk / C::STK) & 1u);
-    }
-  } else if (warp == 3) {
-    // ------------------------------------------------------------ Q + V producer
+    // ------------------------------------------------------------ Q, K, V producer
+    // Loads in the order the MMAs need them: Q, K(0), then K(k+1) before V(k)
+    // (S(k+1) is issued before P(k).V).
     if (lane == 0 && n > 0) {
       // Q rows of the two query blocks into rows 0..63 / 64..127 of the tile
       mbar_expect_tx(q_full, (qb1 >= 0 ? 2 : 1) * C::kKVBytes);
@@ -219,16 +241,32 @@ __global__ void __launch_bounds__(256, 2)
           tma_load_3d(sQ + c * C::kQChunkBytes + C::kKVChunkBytes, &tmQ, c * 64, qb1 * kBlock,
                       static_cast<int>(bh), q_full);
       }
-      int k = 0;
-      for (; k < n; ++k) {
+      auto load_k = [&](int k) -> bool {
+        const int s = k % C::STK;
+        if (!mbar_wait(&kempty[s], (static_cast<uint32_t>(k / C::STK) & 1u) ^ 1u, abort_flag)) return false;
+        const int j = static_cast<int>(lst[k] & kListJMask);
+        mbar_expect_tx(&kfull[s], C::kKVBytes);
+        tma_load_4d(sK + s * C::kKVBytes, &tmK, 0, j * kBlock, 0, static_cast<int>(bh), &kfull[s]);
+        return true;
+      };
+      int nk = load_k(0) ? 1 : 0, nv = 0;         // loads issued
+      for (int k = 0; nk > k && k < n; ++k) {
+        if (k + 1 < n) {
+          if (!load_k(k + 1)) break;
+          ++nk;
+        }
         const int s = k % C::STV;
         if (!mbar_wait(&vempty[s], (static_cast<uint32_t>(k / C::STV) & 1u) ^ 1u, abort_flag)) break;
         const int j = static_cast<int>(lst[k] & kListJMask);
         mbar_expect_tx(&vfull[s], C::kKVBytes);
         tma_load_4d(sV + s * C::kKVBytes, &tmV, 0, j * kBlock, 0, static_cast<int>(bh), &vfull[s]);
+        ++nv;
       }
+      // let issued loads land before exit
       mbar_wait_drain(q_full, 0u);
-      for (int kk = max(0, k - C::STV); kk < k; ++kk)
+      for (int kk = max(0, nk - C::STK); kk < nk; ++kk)
+        mbar_wait_drain(&kfull[kk % C::STK], static_cast<uint32_t>(kk / C::STK) & 1u);
+      for (int kk = max(0, nv - C::STV); kk < nv; ++kk)
         mbar_wait_drain(&vfull[kk % C::STV], static_cast<uint32_t>(kk / C::STV) & 1u);
     }
   } else if (warp == 1) {
@@ -237,12 +275,12 @@ __global__ void __launch_bounds__(256, 2)
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
       bool ok = mbar_wait(q_full, 0u, abort_flag);
       tc_fence_after();
-      // S(k) = Q K_k^T into S buffer k&1 (its previous P has been consumed).
+      // S(k) = Q K_k^T into the S columns (the softmax warps have released S(k-1)).
       auto issue_S = [&](int k) -> bool {
         const int s = k % C::STK;
         if (!mbar_wait(&kfull[s], static_cast<uint32_t>(k / C::STK) & 1u, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t dS = tmem_base + ((k & 1) ? C::kColS1 : C::kColS0);
+        const uint32_t dS = tmem_base + C::kColS;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk & 3) * 32;  // 16 bf16 = 32 bytes inside the swizzle atom
@@ -250,22 +288,26 @@ __global__ void __launch_bounds__(256, 2)
           const uint64_t bd = sdesc_sw128(sKa + s * C::kKVBytes + (kk >> 2) * C::kKVChunkBytes + off, 16, 1024);
           tc_mma_ss(dS, ad, bd, C::kIdescS, kk > 0 ? 1u : 0u);
         }
-        tc_commit(&s_full[k & 1]);
+        tc_commit(s_full);
         tc_commit(&kempty[s]);
         return true;
       };
       if (ok) ok = issue_S(0);
-      if (ok && n > 1) ok = issue_S(1);
       uint32_t o_init = 0;
       unsigned long long pv_tiles = 0;
       for (int k = 0; ok && k < n; ++k) {
+        if (k + 1 < n) {
+          if (!mbar_wait(s_free, static_cast<uint32_t>(k) & 1u, abort_flag)) break;
+          tc_fence_after();
+          if (!issue_S(k + 1)) break;
+        }
         if (!mbar_wait(&p_full[k & 1], static_cast<uint32_t>(k >> 1) & 1u, abort_flag)) break;
         const int s = k % C::STV;
         if (!mbar_wait(&vfull[s], static_cast<uint32_t>(k / C::STV) & 1u, abort_flag)) break;
         tc_fence_after();
-        if (pv_need[k & 1]) {
+        if (contrib[(k & 1) * 2] | contrib[(k & 1) * 2 + 1]) {
           const uint32_t dO = tmem_base + C::kColO;
-          const uint32_t aP = tmem_base + ((k & 1) ? C::kColS1 : C::kColS0);
+          const uint32_t aP = tmem_base + ((k & 1) ? C::kColP1 : C::kColP0);
 #pragma unroll
           for (int kk = 0; kk < kBlock / 16; ++kk) {
             const uint64_t bd = sdesc_sw128(sVa + s * C::kKVBytes + kk * 16 * 128, C::kKVChunkBytes, 1024);
@@ -276,7 +318,6 @@ __global__ void __launch_bounds__(256, 2)
         }
         tc_commit(&pv_done[k & 1]);
         tc_commit(&vempty[s]);
-        if (k + 2 < n && !issue_S(k + 2)) break;
       }
       // Drain: every MMA this thread issued has finished (bounded); the softmax
       // warps wait on the same single-phase barrier before reading O.
@@ -287,129 +328,156 @@ __global__ void __launch_bounds__(256, 2)
         atomicAdd(&stats[3], pv_tiles);
       }
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 2) {
     // ------------------------------------------------------------ softmax warps
-    const int wq = warp & 3;
+    const int wq = warp & 3;                     // TMEM lane quadrant: rows 32*wq .. 32*wq+31
     const int row = wq * 32 + lane;              // tile row == TMEM lane
-    const int half = wq >> 1;                    // warps 4,5 -> query block qb0; 6,7 -> qb1
+    const int half = wq >> 1;                    // quadrants 0,1 -> query block qb0; 2,3 -> qb1
     const int myqb = half ? qb1 : qb0;
     const long long qrow = static_cast<long long>(myqb) * kBlock + (row & (kBlock - 1));
     const bool valid = myqb >= 0 && qrow < N;
     const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t s_addr = tmem_base + lane_bits + C::kColS;
+    const uint32_t o_addr = tmem_base + lane_bits + C::kColO;
+    const bool writer = (wq & 1) == 0 && lane == 0;   // one per half: contrib, stats
     const unsigned FULL = 0xffffffffu;
     float m_true = -INFINITY, m_ref = -INFINITY, l = 0.f;
     unsigned long long kept_pairs = 0, skipped_pairs = 0;
     bool alive = true;
-    for (int k = 0; k < n; ++k) {
+    // S(k) is loaded from TMEM one entry ahead: the load of S(k+1) is issued while
+    // the store of P(k) is still in flight.
+    float s[64];
+    if (n > 0) {
+      if (warp_wait(s_full, 0u, abort_flag)) {
+        tc_fence_after();
+        tmem_ld32(s_addr, *reinterpret_cast<float(*)[32]>(&s[0]));
+        tmem_ld32(s_addr + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
+      } else {
+        alive = false;
+      }
+    }
+    for (int k = 0; alive && k < n; ++k) {
       const uint32_t e = lst[k];
       const int j = static_cast<int>(e & kListJMask);
       const bool keep_lo = (e & kListLo) != 0u, keep_hi = (e & kListHi) != 0u;
       const bool keep = half ? keep_hi : keep_lo;
-      const uint32_t sbuf = tmem_base + lane_bits + ((k & 1) ? C::kColS1 : C::kColS0);
-      if (!warp_wait(&s_full[k & 1], static_cast<uint32_t>(k >> 1) & 1u, abort_flag)) { alive = false; break; }
-      tc_fence_after();
       const int kbase = j * kBlock;
       // visible columns of this row in the block: c < ncol (tail, causal diagonal)
       int ncol = (keep && valid) ? min(kBlock, N - kbase) : 0;
       if (causal) ncol = min(ncol, static_cast<int>(max(qrow - kbase + 1, 0LL)));
       const bool warp_none = __all_sync(FULL, ncol == 0);
       const bool warp_full = __all_sync(FULL, ncol == kBlock);
+      tmem_wait_ld();                             // S(k) is in s[]
+      pin32(*reinterpret_cast<float(*)[32]>(&s[0]));
+      pin32(*reinterpret_cast<float(*)[32]>(&s[32]));
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);         // S may now be overwritten by S(k+1)
       uint32_t pk[32];                            // P as packed bf16 pairs
-      float rmax = -INFINITY, rsum = 0.f;
-      bool raise = false;
-      float alpha = 1.f;
-      if (warp_none) {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = 0u;
-      } else {
-        float s[64];
-        tmem_ld32(sbuf, *reinterpret_cast<float(*)[32]>(&s[0]));
-        tmem_ld32(sbuf + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
-        tmem_wait_ld();
+      float rmax = -INFINITY, psum = 0.f;
+      if (!warp_none) {
         if (!warp_full) {
 #pragma unroll
           for (int c = 0; c < 64; ++c) s[c] = (c < ncol) ? s[c] : -INFINITY;
         }
         float mx[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) mx[c] = fmaxf(s[c], s[c + 8]);
+        for (int u = 0; u < 8; ++u) mx[u] = fmax3(s[u], s[u + 8], s[u + 16]);
 #pragma unroll
-        for (int c = 16; c < 64; c += 8) {
+        for (int c = 24; c < 56; c += 16) {
 #pragma unroll
-          for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], s[c + u]);
+          for (int u = 0; u < 8; ++u) mx[u] = fmax3(mx[u], s[c + u], s[c + 8 + u]);
         }
-        rmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-        rmax *= scale_log2;                       // -inf stays -inf (scale > 0)
-        const float m_new = fmaxf(m_true, rmax);
-        raise = m_new > m_ref + 8.f;              // also true for the first finite max
-        if (raise) {
-          alpha = ex2(m_ref - m_new);             // 0 when m_ref = -inf
-          m_ref = m_new;
-        }
-        const float mref = (m_ref == -INFINITY) ? 0.f : m_ref;
-        float sm[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float p0 = ex2(fmaf(s[c], scale_log2, -mref));
-          const float p1 = ex2(fmaf(s[c + 1], scale_log2, -mref));
-          sm[(c >> 1) & 3] += p0 + p1;
-          pk[c >> 1] = pack_bf16x2(p0, p1);
-        }
-        rsum = (sm[0] + sm[1]) + (sm[2] + sm[3]);
+        for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], s[56 + u]);
+        rmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
+               scale_log2;                        // -inf stays -inf (scale > 0)
+        // exponentials against the current reference, independent of the max above
+        psum = softmax_exp64(s, scale_log2, (m_ref == -INFINITY) ? 0.f : m_ref, pk);
       }
-      // lambda vote: a half skips P.V when all its rows that see the block pass
-      bool half_skip = false, skip_lo = false, skip_hi = false;
+      bool wpass = true;
       if (lam_on) {
+        // this warp's lambda vote, posted before the store of P(k)
         const bool pass = !(rmax > -INFINITY) || (rmax - m_true < lam_log2);
-        const bool wpass = __all_sync(FULL, pass);
-        if (lane == 0) {
-          votes[(k & 1) * 4 + wq] = wpass ? 1 : 0;
-          mbar_arrive(vote_bar);
-        }
-        if (!warp_wait(vote_bar, static_cast<uint32_t>(k) & 1u, abort_flag)) { alive = false; break; }
-        skip_lo = votes[(k & 1) * 4 + 0] && votes[(k & 1) * 4 + 1];
-        skip_hi = votes[(k & 1) * 4 + 2] && votes[(k & 1) * 4 + 3];
-        half_skip = half ? skip_hi : skip_lo;
+        wpass = __all_sync(FULL, pass);
+        if (lane == 0) votes[(k & 1) * 4 + wq] = (k << 1) | (wpass ? 1 : 0);
       }
-      m_true = fmaxf(m_true, rmax);
-      l = l * alpha + rsum;
-      if (half_skip) {
+      const float m_new = fmaxf(m_true, rmax);
+      const bool raise = m_new > m_ref + 8.f;    // also true for the first finite max
+      float alpha = 1.f;
+      if (raise) {
+        alpha = ex2(m_ref - m_new);               // 0 when m_ref = -inf
+        m_ref = m_new;
+      }
+      const bool any_raise = __any_sync(FULL, raise);
+      if (any_raise && !warp_none)
+        psum = softmax_exp64(s, scale_log2, (m_ref == -INFINITY) ? 0.f : m_ref, pk);
+      if (warp_none) {
 #pragma unroll
         for (int c = 0; c < 32; ++c) pk[c] = 0u;
       }
-      tmem_st32u(sbuf, pk);                       // P(k) over the first 32 columns of S(k)
-      // O correction for rows whose reference max was raised (after P(k-1).V).
-      // pv_done is double-buffered: S(k), already waited for, was issued after
-      // P(k-2).V, so pv_done[(k-1)&1] is at most one phase short of entry k-1.
-      if (k > 0 && __any_sync(FULL, raise)) {
+      m_true = m_new;
+      l = l * alpha + psum;
+      // P(k) into buffer k&1 (its previous reader, P(k-2).V, finished before S(k))
+      const uint32_t p_addr = tmem_base + lane_bits + ((k & 1) ? C::kColP1 : C::kColP0);
+      tmem_st32u(p_addr, pk);
+      // O correction for rows whose reference max was raised (after P(k-1).V);
+      // pv_done[(k-1)&1] is at most one phase short of entry k-1 (P(k-3).V finished
+      // before S(k-1)).
+      if (k > 0 && any_raise) {
         if (!warp_wait(&pv_done[(k - 1) & 1], static_cast<uint32_t>((k - 1) >> 1) & 1u, abort_flag)) {
           alive = false;
           break;
         }
         tc_fence_after();
-#pragma unroll
+#pragma unroll 1
         for (int cc = 0; cc < D; cc += 32) {
           float o[32];
-          tmem_ld32(tmem_base + lane_bits + C::kColO + cc, o);
+          tmem_ld32(o_addr + cc, o);
           tmem_wait_ld();
+          pin32(o);
 #pragma unroll
           for (int x = 0; x < 32; ++x) o[x] *= alpha;
-          tmem_st32(tmem_base + lane_bits + C::kColO + cc, o);
+          tmem_st32(o_addr + cc, o);
         }
       }
+      // lambda: the half skips P.V when both of its warps pass; a skipping half
+      // replaces its P(k) with zeros
+      bool half_skip = false;
+      if (lam_on) {
+        int pv = 0;
+        if (lane == 0) pv = spin_tag(&votes[(k & 1) * 4 + (wq ^ 1)], k, abort_flag);
+        pv = __shfl_sync(FULL, pv, 0);
+        if (pv < 0) { alive = false; break; }
+        half_skip = wpass && (pv & 1);
+        if (half_skip && !warp_none) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) pk[c] = 0u;
+          tmem_wait_st();
+          tmem_st32u(p_addr, pk);
+        }
+      }
+      // prefetch S(k+1) while P(k) is being stored
+      if (k + 1 < n) {
+        if (!warp_wait(s_full, static_cast<uint32_t>(k + 1) & 1u, abort_flag)) {
+          alive = false;
+          break;
+        }
+        tc_fence_after();
+        tmem_ld32(s_addr, *reinterpret_cast<float(*)[32]>(&s[0]));
+        tmem_ld32(s_addr + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
+      }
       tmem_wait_st();
-      if (threadIdx.x == 128) {
-        const bool contrib_lo = keep_lo && !skip_lo, contrib_hi = keep_hi && !skip_hi;
-        pv_need[k & 1] = (contrib_lo || contrib_hi) ? 1 : 0;
-        kept_pairs += static_cast<unsigned long long>(keep_lo) + static_cast<unsigned long long>(keep_hi);
-        skipped_pairs += static_cast<unsigned long long>(keep_lo && skip_lo) +
-                         static_cast<unsigned long long>(keep_hi && skip_hi);
+      if (writer) {
+        contrib[(k & 1) * 2 + half] = (keep && !half_skip) ? 1 : 0;
+        kept_pairs += keep ? 1ull : 0ull;
+        skipped_pairs += (keep && half_skip) ? 1ull : 0ull;
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[k & 1]);
     }
+    tmem_wait_ld();                               // no TMEM load left in flight
     // ------------------------------------------------------------ epilogue
     if (alive && n > 0) {
       if (warp_wait(drain, 0u, abort_flag)) {
@@ -419,8 +487,9 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
         for (int cc = 0; cc < D; cc += 32) {
           float o[32];
-          tmem_ld32(tmem_base + lane_bits + C::kColO + cc, o);
+          tmem_ld32(o_addr + cc, o);
           tmem_wait_ld();
+          pin32(o);
           if (valid) {
 #pragma unroll
             for (int x = 0; x < 32; x += 8) {
@@ -438,7 +507,7 @@ __global__ void __launch_bounds__(256, 2)
       __nv_bfloat16* orow = O + (bh * N + qrow) * static_cast<long long>(D);
       for (int x = 0; x < D; x += 8) *reinterpret_cast<uint4*>(orow + x) = make_uint4(0u, 0u, 0u, 0u);
     }
-    if (threadIdx.x == 128 && stats) {
+    if (writer && stats) {
       atomicAdd(&stats[0], kept_pairs);
       atomicAdd(&stats[1], skipped_pairs);
     }

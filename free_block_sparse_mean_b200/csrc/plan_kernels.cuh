@@ -315,6 +315,13 @@ __global__ void __launch_bounds__(NT) score_select_kernel(const float* __restric
 // tile (second -1 if the head has an odd block count), heads in ascending order.
 constexpr int kPairGreedyMaxNb = 1024;
 constexpr int kPairWindow = 32;
+// Heads per interleaved group of the tile order: as many as have their K and V
+// together within half of L2 (64 MB), at least one.
+inline int order_group_heads(long long BH, int N, int D) {
+  const long long kv_bytes = 2ll * N * D * 2;
+  const long long g = (64ll << 20) / kv_bytes;
+  return static_cast<int>(g < 1 ? 1 : (g > BH ? BH : g));
+}
 
 
 // In-place ascending bitonic sort of n64 (a power of two) 64-bit keys in shared memory.
@@ -336,10 +343,15 @@ static __device__ void block_bitonic_sort(unsigned long long* keys, int n64) {
   }
 }
 
+// Heads are laid out in groups of G consecutive heads (the last group may be
+// smaller); within a group, tile rank r of the group's u-th head goes to position
+// group_start + r * group_size + u. The CTAs running at one time then take the
+// longest tiles of every head of the group first, while the group's K and V
+// (chosen by the host to fit in L2) stay resident.
 static __global__ void __launch_bounds__(1024) pair_order_kernel(const unsigned long long* __restrict__ sig,
                                                                  const uint32_t* __restrict__ bits_g,
                                                                  const int* __restrict__ count, int Nb,
-                                                                 int Tq, int* __restrict__ work) {
+                                                                 int Tq, int G, int* __restrict__ work) {
   extern __shared__ __align__(16) unsigned char psm[];
   const int P = 1 << (32 - __clz(max(Nb, 2) - 1));   // next power of two >= Nb
   const int P2 = 1 << (32 - __clz(max(Tq, 2) - 1));
@@ -451,11 +463,15 @@ static __global__ void __launch_bounds__(1024) pair_order_kernel(const unsigned 
   __syncthreads();
   // 3. longest first, then write the global query-block ids
   block_bitonic_sort(keys2, P2);
+  const long long g0 = (bh / G) * G;                                  // first head of the group
+  const long long gsize = min(static_cast<long long>(G), static_cast<long long>(gridDim.x) - g0);
+  const long long u = bh - g0;
   for (int r = threadIdx.x; r < Tq; r += blockDim.x) {
     const int p = static_cast<int>(keys2[r] & 0xffffffffu);
     const int a = pa[p], b = pb[p];
-    work[2 * (bh * Tq + r)] = static_cast<int>(bh * Nb + a);
-    work[2 * (bh * Tq + r) + 1] = b >= 0 ? static_cast<int>(bh * Nb + b) : -1;
+    const long long pos = g0 * Tq + static_cast<long long>(r) * gsize + u;
+    work[2 * pos] = static_cast<int>(bh * Nb + a);
+    work[2 * pos + 1] = b >= 0 ? static_cast<int>(bh * Nb + b) : -1;
   }
 }
 

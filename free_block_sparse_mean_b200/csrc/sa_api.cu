@@ -127,7 +127,9 @@ sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau
     const int Tq = (Nb + 1) / 2;
     const int smem = sa::pair_order_smem_bytes(Nb);
     if (set_smem(sa::pair_order_kernel, smem) != SA_OK) return SA_ERR_CUDA;
-    sa::pair_order_kernel<<<static_cast<unsigned>(BH), Nb <= 512 ? 256 : 1024, smem, st>>>(sig, bits, count, Nb, Tq, work);
+    const int G = sa::order_group_heads(BH, s.N, D);
+    sa::pair_order_kernel<<<static_cast<unsigned>(BH), Nb <= 512 ? 256 : 1024, smem, st>>>(sig, bits, count, Nb, Tq,
+                                                                                          G, work);
     if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   }
   return SA_OK;
@@ -149,7 +151,7 @@ sa_status launch_fwd(const sa_shape& s, const void* Q, const void* K, const void
   if (set_smem(kern, Cfg::kSmemBytes) != SA_OK) return SA_ERR_CUDA;
   const float LOG2E = 1.4426950408889634f;
   const int lam_on = std::isinf(lambda) && lambda < 0 ? 0 : 1;
-  kern<<<static_cast<unsigned>(tiles), 256, Cfg::kSmemBytes, st>>>(
+  kern<<<static_cast<unsigned>(tiles), Cfg::kThreads, Cfg::kSmemBytes, st>>>(
       mq, mk, mv, mask, work, static_cast<__nv_bfloat16*>(O), s.N, Nb, Tq, tiles,
       static_cast<long long>(s.B) * s.H * Nb, scale * LOG2E,
       lam_on ? lambda * LOG2E : 0.f, lam_on, causal, reinterpret_cast<unsigned long long*>(stats));

@@ -59,11 +59,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Waits for the phase with the given parity to complete. Gives up (returns false)
-// when *abort is set by another role or after kWaitTimeoutNs, in which case it
-// sets *abort and records DEVERR_TIMEOUT.
-static __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Slow path of mbar_wait: polls until the phase with the given parity completes.
+// Gives up (returns false) when *abort is set by another role or after
+// kWaitTimeoutNs, in which case it sets *abort and records DEVERR_TIMEOUT.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort) {
   const unsigned long long t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -76,6 +75,38 @@ static __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, vo
       }
     }
   }
+}
+// Waits for the phase with the given parity to complete (bounded, see
+// mbar_wait_slow). The common case, a phase already complete or completing
+// within try_wait's own suspend window, stays inline.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort);
+}
+
+// Slow path of spin_tag: polls a shared-memory word until its tag (value >> 1)
+// equals `tag`; bounded like mbar_wait_slow. Returns the word, or -1 on abort.
+static __device__ __noinline__ int spin_tag_slow(volatile int* word, int tag, volatile int* abort) {
+  const unsigned long long t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    const int v = *word;
+    if ((v >> 1) == tag) return v;
+    if ((it & 63u) == 0u) {
+      if (*abort) return -1;
+      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+        *abort = 1;
+        atomicOr(&g_dev_error, DEVERR_TIMEOUT);
+        return -1;
+      }
+    }
+  }
+}
+// Reads a tagged shared-memory word ((tag << 1) | bit) written by another warp
+// once its tag matches; -1 if the wait was abandoned.
+__device__ __forceinline__ int spin_tag(volatile int* word, int tag, volatile int* abort) {
+  const int v = *word;
+  if ((v >> 1) == tag) return v;
+  return spin_tag_slow(word, tag, abort);
 }
 
 // Bounded wait that ignores the abort flag: used to drain copies and MMAs still
@@ -182,6 +213,16 @@ __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[3
       : "memory");
 }
 
+// tcgen05.st of 16 packed 32-bit values to this warp's lanes.
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 layout (version 1).
 // Address and both byte offsets are stored >> 4.
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
@@ -252,6 +293,63 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipe, for x <= 8 (larger x is not supported). Range reduction
+// x = j + f with j = round(x) and f in [-1/2, 1/2] (Cody and Waite's scheme: the
+// 1.5 * 2^23 addition rounds x to an integer that lands in the low mantissa
+// bits of t), then 2^f from a degree-3 polynomial whose coefficients minimise the
+// maximum relative error on [-1/2, 1/2] (fitted for this library with the Remez
+// exchange algorithm; 7.5e-5 in fp32 Horner form), and j is added to the exponent
+// field. x is clamped at -126 first, so tiny results (and x = -inf) come out as a
+// positive value below 2^-125 instead of 0.
+constexpr float kExp2C0 = 0.99992805719375610f;
+constexpr float kExp2C1 = 0.69326096773147583f;
+constexpr float kExp2C2 = 0.24261112511157990f;
+constexpr float kExp2C3 = 0.05517166852951050f;
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.f);
+  const float t = x + 12582912.f;
+  const float f = x - (t - 12582912.f);
+  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): one instruction for two lanes of
+// work, which halves the issue slots of the softmax's scale-subtract and sums.
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// Orders every later use of v after the preceding tcgen05.wait::ld: the values of
+// an asynchronous TMEM load may only be read once that wait has returned.
+__device__ __forceinline__ void pin32(float (&v)[32]) {
+  asm volatile(""
+               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]), "+f"(v[7]),
+                 "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]), "+f"(v[14]),
+                 "+f"(v[15]), "+f"(v[16]), "+f"(v[17]), "+f"(v[18]), "+f"(v[19]), "+f"(v[20]), "+f"(v[21]),
+                 "+f"(v[22]), "+f"(v[23]), "+f"(v[24]), "+f"(v[25]), "+f"(v[26]), "+f"(v[27]), "+f"(v[28]),
+                 "+f"(v[29]), "+f"(v[30]), "+f"(v[31]));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

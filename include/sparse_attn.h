@@ -86,13 +86,17 @@ int64_t sparse_attn_num_tiles(sa_shape s);
  *   work      out, device int32 [2 * sparse_attn_num_tiles(s)] or NULL: the query
  *             tiles in execution order, two global query-block ids per tile
  *             ((b*H + h)*Nb + i; the second is -1 when a head has an odd block
- *             count). Every query block appears exactly once; heads come in
- *             ascending (b,h) order. Within a head, blocks are paired so that the
- *             two kept sets overlap (sorted by two MinHash signatures of the kept
- *             set, then each block takes the best-matching unused block among the
- *             next 32, for Nb <= 1024; consecutive blocks of that order above),
- *             and tiles are ordered by decreasing union size (longest first).
- *             Deterministic for a given mask.
+ *             count). Every query block appears exactly once. Within a head,
+ *             blocks are paired so that the two kept sets overlap (sorted by two
+ *             MinHash signatures of the kept set, then each block takes the
+ *             best-matching unused block among the next 32, for Nb <= 1024;
+ *             consecutive blocks of that order above), and the head's tiles are
+ *             ranked by decreasing union size (longest first). Heads are taken in
+ *             ascending (b,h) order in groups of G consecutive heads, G being the
+ *             most heads whose K and V together fit in 64 MB (at least 1); within a
+ *             group the tiles are interleaved by rank (rank 0 of every head of the
+ *             group, then rank 1, ...), so the longest tiles of all of the group's
+ *             heads start first. Deterministic for a given mask.
  *   workspace device scratch of at least sparse_attn_plan_workspace_size(s) bytes,
  *             256-byte aligned; its contents on entry do not matter
  */

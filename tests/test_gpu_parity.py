@@ -41,21 +41,31 @@ def _plan_and_check(q, k, tau, causal, scale=None):
 
 
 def _work_ok(p, B, H, Nb):
-    """work lists every query block once, in pairs of one head, heads in order,
-    and within a head the pairs' union sizes do not increase."""
+    """work lists every query block once, in pairs of one head; heads come in
+    groups of consecutive heads whose tiles are interleaved by rank, and within a
+    head the pairs' union sizes do not increase."""
     Tq = (Nb + 1) // 2
-    work = to_np(p.work).astype(np.int64)[: 2 * B * H * Tq].reshape(B * H, Tq, 2)
+    work = to_np(p.work).astype(np.int64)[: 2 * B * H * Tq].reshape(B * H * Tq, 2)
     mask = to_np(p.mask).reshape(B * H, Nb, Nb).astype(bool)
+    a, b = work[:, 0], work[:, 1]
+    head = a // Nb
+    assert np.all((b == -1) | (b // Nb == head))
     for bh in range(B * H):
-        a, b = work[bh, :, 0], work[bh, :, 1]
-        assert np.all(a // Nb == bh) and np.all((b == -1) | (b // Nb == bh))
-        ids = np.concatenate([a, b[b >= 0]]) - bh * Nb
+        sel = np.nonzero(head == bh)[0]
+        assert len(sel) == Tq
+        ids = np.concatenate([a[sel], b[sel][b[sel] >= 0]]) - bh * Nb
         assert sorted(ids.tolist()) == list(range(Nb))
-        assert (b == -1).sum() == Nb % 2
+        assert (b[sel] == -1).sum() == Nb % 2
         uni = [(mask[bh, x - bh * Nb] | (mask[bh, y - bh * Nb] if y >= 0 else False)).sum()
-               for x, y in zip(a, b)]
+               for x, y in zip(a[sel], b[sel])]
         if Nb <= 1024:
             assert np.all(np.diff(uni) <= 0)
+    # each head's tiles fill one contiguous group of positions with the other heads of its group
+    first = np.array([np.nonzero(head == bh)[0].min() for bh in range(B * H)])
+    last = np.array([np.nonzero(head == bh)[0].max() for bh in range(B * H)])
+    assert np.all(np.diff(first) > 0)
+    for bh in range(1, B * H):
+        assert first[bh] > last[bh - 1] or first[bh] == first[bh - 1] + 1
 
 
 def test_pairing_reduces_union_on_small_workload():
@@ -67,8 +77,8 @@ def test_pairing_reduces_union_on_small_workload():
     torch.cuda.synchronize()
     _work_ok(p, 1, w.H, 64)
     m = to_np(p.mask).reshape(w.H, 64, 64).astype(bool)
-    work = to_np(p.work).astype(np.int64).reshape(w.H, 32, 2)
-    paired = sum((m[h, x % 64] | m[h, y % 64]).sum() for h in range(w.H) for x, y in work[h])
+    work = to_np(p.work).astype(np.int64).reshape(w.H * 32, 2)
+    paired = sum((m[x // 64, x % 64] | m[y // 64, y % 64]).sum() for x, y in work)
     natural = sum((m[h, 2 * t] | m[h, 2 * t + 1]).sum() for h in range(w.H) for t in range(32))
     print(f"union entries: plan pairs {paired}, natural pairs {natural}, kept pairs {m.sum()}")
     assert paired < 0.8 * natural
