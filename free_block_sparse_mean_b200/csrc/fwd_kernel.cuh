@@ -34,11 +34,9 @@
 //
 // The running max used for the exponentials is raised lazily (only when a row's
 // max grows by more than 2^8), which leaves O/l unchanged and makes the O
-// correction rare. The exponentials are computed against the current reference
-// while the block's row max is still being reduced, and redone in the rare case
-// of a raise. The lambda test uses the exact running max. P(k) is stored before
-// the lambda vote of the other warp of the half is read; a half that skips then
-// overwrites its P(k) with zeros.
+// correction rare. The lambda test uses the exact running max. Each warp posts its
+// lambda vote right after the row max and reads the other warp's vote of the half
+// after its exponentials, so the exchange rarely waits.
 //
 // An mbarrier wait by parity is only sound when the barrier is at most one phase
 // ahead of, and at most one phase short of, the phase waited for; otherwise the
@@ -392,12 +390,11 @@ __global__ void __launch_bounds__(192, 2)
         for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], s[56 + u]);
         rmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
                scale_log2;                        // -inf stays -inf (scale > 0)
-        // exponentials against the current reference, independent of the max above
-        psum = softmax_exp64(s, scale_log2, (m_ref == -INFINITY) ? 0.f : m_ref, pk);
       }
       bool wpass = true;
       if (lam_on) {
-        // this warp's lambda vote, posted before the store of P(k)
+        // this warp's lambda vote, posted before the exponentials so that the other
+        // warp of the half finds it when it needs it
         const bool pass = !(rmax > -INFINITY) || (rmax - m_true < lam_log2);
         wpass = __all_sync(FULL, pass);
         if (lane == 0) votes[(k & 1) * 4 + wq] = (k << 1) | (wpass ? 1 : 0);
@@ -410,17 +407,31 @@ __global__ void __launch_bounds__(192, 2)
         m_ref = m_new;
       }
       const bool any_raise = __any_sync(FULL, raise);
-      if (any_raise && !warp_none)
-        psum = softmax_exp64(s, scale_log2, (m_ref == -INFINITY) ? 0.f : m_ref, pk);
+      float mref = (m_ref == -INFINITY) ? 0.f : m_ref;
+      asm volatile("" : "+f"(mref) :: "memory");  // the exponentials after the vote is posted
       if (warp_none) {
 #pragma unroll
         for (int c = 0; c < 32; ++c) pk[c] = 0u;
+      } else {
+        psum = softmax_exp64(s, scale_log2, mref, pk);
       }
       m_true = m_new;
       l = l * alpha + psum;
+      // lambda: the half skips P.V when both of its warps pass; its P(k) is zero
+      bool half_skip = false;
+      if (lam_on) {
+        int pv = 0;
+        if (lane == 0) pv = spin_tag(&votes[(k & 1) * 4 + (wq ^ 1)], k, abort_flag);
+        pv = __shfl_sync(FULL, pv, 0);
+        if (pv < 0) { alive = false; break; }
+        half_skip = wpass && (pv & 1);
+        if (half_skip) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) pk[c] = 0u;
+        }
+      }
       // P(k) into buffer k&1 (its previous reader, P(k-2).V, finished before S(k))
-      const uint32_t p_addr = tmem_base + lane_bits + ((k & 1) ? C::kColP1 : C::kColP0);
-      tmem_st32u(p_addr, pk);
+      tmem_st32u(tmem_base + lane_bits + ((k & 1) ? C::kColP1 : C::kColP0), pk);
       // O correction for rows whose reference max was raised (after P(k-1).V);
       // pv_done[(k-1)&1] is at most one phase short of entry k-1 (P(k-3).V finished
       // before S(k-1)).
@@ -439,22 +450,6 @@ __global__ void __launch_bounds__(192, 2)
 #pragma unroll
           for (int x = 0; x < 32; ++x) o[x] *= alpha;
           tmem_st32(o_addr + cc, o);
-        }
-      }
-      // lambda: the half skips P.V when both of its warps pass; a skipping half
-      // replaces its P(k) with zeros
-      bool half_skip = false;
-      if (lam_on) {
-        int pv = 0;
-        if (lane == 0) pv = spin_tag(&votes[(k & 1) * 4 + (wq ^ 1)], k, abort_flag);
-        pv = __shfl_sync(FULL, pv, 0);
-        if (pv < 0) { alive = false; break; }
-        half_skip = wpass && (pv & 1);
-        if (half_skip && !warp_none) {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) pk[c] = 0u;
-          tmem_wait_st();
-          tmem_st32u(p_addr, pk);
         }
       }
       // prefetch S(k+1) while P(k) is being stored
