@@ -304,17 +304,21 @@ __global__ void __launch_bounds__(NT) score_select_kernel(const float* __restric
 // blocks of one head and walks the union of their kept lists, so its cost is the
 // union size. Adjacent blocks of a video raster often keep disjoint key blocks
 // (their partners are in the neighbouring frame), so the pairs are chosen from
-// the masks: query blocks are sorted by two MinHash signatures of their kept
-// sets (equal sets sort together), then each block, in that order, takes as
-// partner the unused block among the next 32 whose kept set matches best
-// (overlap minus symmetric difference), else the next unused block. The pairs of
-// a head are then ordered by decreasing union size (longest first). Above
-// kPairGreedyMaxNb blocks per head the bitsets no longer fit in shared memory and
-// consecutive blocks of the sorted order are paired directly.
+// the masks. Query blocks are sorted by two MinHash signatures of their kept sets
+// (equal sets sort together). Then, in rounds, every unpaired block picks the
+// unpaired block within kPairWindow places of it in that order whose kept set
+// matches best (overlap minus symmetric difference; ties to the nearer, then the
+// earlier block), and blocks that pick each other are paired; after
+// kPairRounds rounds, or a round without a new pair, the rest are paired in
+// order. Every block of a head is examined at once, so a round costs one pass.
+// The pairs of a head are then ordered by decreasing union size (longest first).
+// Above kPairMatchMaxNb blocks per head the bitsets no longer fit in shared
+// memory and consecutive blocks of the sorted order are paired directly.
 // Output: work[2*r], work[2*r+1] = global query-block ids (bh*Nb + i) of the r-th
-// tile (second -1 if the head has an odd block count), heads in ascending order.
-constexpr int kPairGreedyMaxNb = 1024;
-constexpr int kPairWindow = 32;
+// tile (second -1 if the head has an odd block count).
+constexpr int kPairMatchMaxNb = 1024;
+constexpr int kPairWindow = 16;
+constexpr int kPairRounds = 6;
 // Heads per interleaved group of the tile order: as many as have their K and V
 // together within half of L2 (64 MB), at least one.
 inline int order_group_heads(long long BH, int N, int D) {
@@ -343,6 +347,36 @@ static __device__ void block_bitonic_sort(unsigned long long* keys, int n64) {
   }
 }
 
+// Exclusive prefix sum of v over the threads of the block (any multiple of 32
+// threads up to 1024); every thread must call it. *total receives the sum.
+// sbuf: 33 ints of shared memory.
+static __device__ int block_exclusive_scan(int v, int* sbuf, int* total) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sbuf[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = (lane < nw) ? sbuf[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < nw) sbuf[lane] = w;            // inclusive warp totals
+    if (lane == 31) sbuf[32] = w;
+  }
+  __syncthreads();
+  const int excl = x - v + (warp > 0 ? sbuf[warp - 1] : 0);
+  *total = sbuf[32];
+  __syncthreads();                            // sbuf may be reused right after
+  return excl;
+}
+
 // Heads are laid out in groups of G consecutive heads (the last group may be
 // smaller); within a group, tile rank r of the group's u-th head goes to position
 // group_start + r * group_size + u. The CTAs running at one time then take the
@@ -355,105 +389,128 @@ static __global__ void __launch_bounds__(1024) pair_order_kernel(const unsigned 
   extern __shared__ __align__(16) unsigned char psm[];
   const int P = 1 << (32 - __clz(max(Nb, 2) - 1));   // next power of two >= Nb
   const int P2 = 1 << (32 - __clz(max(Tq, 2) - 1));
-  const bool greedy = Nb <= kPairGreedyMaxNb;
+  const bool match = Nb <= kPairMatchMaxNb;
   const int W = (Nb + 31) / 32;                       // bitset words per row
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(psm);       // [P]
   unsigned long long* keys2 = keys + P;                                          // [P2]
   int* pa = reinterpret_cast<int*>(keys2 + P2);                                  // [Tq]
   int* pb = pa + Tq;                                                             // [Tq]
-  int* order = pb + Tq;                                                          // [Nb]
-  int* used = order + Nb;                                                        // [Nb]
-  uint32_t* bits = reinterpret_cast<uint32_t*>(used + Nb);                      // [Nb][W] (greedy only)
+  int* order = pb + Tq;                                                          // [Nb] position -> block
+  int* alive = order + Nb;                                                       // [Nb] unpaired positions, ascending
+  int* best = alive + Nb;                                                        // [Nb] pick of a position
+  int* partner = best + Nb;                                                      // [Nb] -1 while unpaired
+  int* sbuf = partner + Nb;                                                      // [34] scan scratch
+  uint32_t* bitsT = reinterpret_cast<uint32_t*>(sbuf + 34);                     // [W][Nb] by position (match only)
   const long long bh = blockIdx.x;
   const int* cnt = count + bh * Nb;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const unsigned FULL = 0xffffffffu;
 
-  // 1. MinHash keys (from the selection kernel), bitsets into shared memory
+  // 1. MinHash keys (from the selection kernel); sort
   for (int i = threadIdx.x; i < Nb; i += blockDim.x) {
     keys[i] = sig[bh * Nb + i];
-    used[i] = 0;
+    partner[i] = -1;
   }
   for (int i = Nb + threadIdx.x; i < P; i += blockDim.x) keys[i] = ~0ull;
-  if (greedy) {
-    const uint32_t* src = bits_g + bh * static_cast<long long>(Nb) * W;
-    for (int x = threadIdx.x; x < Nb * W; x += blockDim.x) bits[x] = src[x];
-  }
   __syncthreads();
   block_bitonic_sort(keys, P);
-  for (int i = threadIdx.x; i < Nb; i += blockDim.x) order[i] = static_cast<int>(keys[i] & 0xffffu);
+  for (int p = threadIdx.x; p < Nb; p += blockDim.x) {
+    order[p] = static_cast<int>(keys[p] & 0xffffu);
+    alive[p] = p;
+  }
   __syncthreads();
 
-  // 2. pairs and their costs (union sizes, or count sums without bitsets)
-  if (greedy) {
-    if (warp == 0) {
-      int np = 0;
-      for (int pos = 0; pos < Nb; ++pos) {
-        const int i = order[pos];
-        if (used[i]) continue;   // same value in every lane
-        __syncwarp();
-        if (lane == 0) used[i] = 1;
-        __syncwarp();
-        const int cpos = pos + 1 + lane;
-        const int c = (cpos < Nb && lane < kPairWindow) ? order[cpos] : -1;
-        int score = INT_MIN, uni = 0;
-        if (c >= 0 && !used[c]) {
-          int ov = 0, sd = 0;
-          for (int w = 0; w < W; ++w) {
-            const uint32_t a = bits[i * W + w], b = bits[c * W + w];
-            ov += __popc(a & b);
-            sd += __popc(a ^ b);
-            uni += __popc(a | b);
-          }
-          score = ov - sd;
-        }
-        // warp argmax, ties to the lowest lane
-        int best = score, bl = lane;
+  // 2. pairs (as sorted positions in pa/pb) and their costs (union sizes, or count
+  //    sums without bitsets)
+  if (match) {
+    // kept-set bitsets, word-major by sorted position: neighbouring candidates are
+    // neighbouring addresses
+    const uint32_t* src = bits_g + bh * static_cast<long long>(Nb) * W;
+    for (int x = threadIdx.x; x < Nb * W; x += blockDim.x) {
+      const int p = x / W, w = x - p * W;
+      bitsT[w * Nb + p] = src[static_cast<long long>(order[p]) * W + w];
+    }
+    __syncthreads();
+    // one thread per alive position (the launch gives at least Nb threads)
+    int na = Nb;
+    constexpr int NC = 2 * kPairWindow + 1;
+    for (int round = 0; round < kPairRounds; ++round) {
+      const int t = threadIdx.x;
+      if (t < na) {
+        const int me = alive[t];
+        const int qlo = t - kPairWindow;
+        int sc[NC];                               // overlap minus symmetric difference
 #pragma unroll
-        for (int o = 16; o; o >>= 1) {
-          const int os = __shfl_xor_sync(FULL, best, o), ol = __shfl_xor_sync(FULL, bl, o);
-          if (os > best || (os == best && ol < bl)) {
-            best = os;
-            bl = ol;
-          }
-        }
-        int partner = __shfl_sync(FULL, c, bl);
-        int ucost = __shfl_sync(FULL, uni, bl);
-        if (best == INT_MIN) {   // nothing unused in the window: next unused block in order
-          partner = -1;
-          for (int q = pos + 1 + kPairWindow; q < Nb; q += 32) {
-            const int cc = (q + lane < Nb) ? order[q + lane] : -1;
-            const unsigned fr = __ballot_sync(FULL, cc >= 0 && !used[cc]);
-            if (fr) {
-              partner = __shfl_sync(FULL, cc, __ffs(fr) - 1);
-              break;
-            }
-          }
-          ucost = 0;
-          if (partner >= 0)
-            for (int w = lane; w < W; w += 32) ucost += __popc(bits[i * W + w] | bits[partner * W + w]);
-          else
-            for (int w = lane; w < W; w += 32) ucost += __popc(bits[i * W + w]);
+        for (int d = 0; d < NC; ++d) sc[d] = 0;
+        for (int w = 0; w < W; ++w) {
+          const uint32_t* row = bitsT + w * Nb;
+          const uint32_t x = row[me];
 #pragma unroll
-          for (int o = 16; o; o >>= 1) ucost += __shfl_xor_sync(FULL, ucost, o);
+          for (int d = 0; d < NC; ++d) {
+            const int q = qlo + d;
+            const uint32_t y = (q >= 0 && q < na) ? row[alive[q]] : 0u;
+            sc[d] += __popc(x & y) - __popc(x ^ y);
+          }
         }
-        if (lane == 0) {
-          if (partner >= 0) used[partner] = 1;
-          pa[np] = i;
-          pb[np] = partner;
-          keys2[np] = (static_cast<unsigned long long>(0xffffffu - static_cast<uint32_t>(ucost)) << 32) |
-                      static_cast<unsigned long long>(np);
+        // best score; ties to the nearer, then the earlier candidate
+        int bs = INT_MIN, bd = INT_MAX, bp = -1;
+#pragma unroll
+        for (int d = 0; d < NC; ++d) {
+          const int q = qlo + d, dist = abs(d - kPairWindow);
+          if (q >= 0 && q < na && d != kPairWindow && (sc[d] > bs || (sc[d] == bs && dist < bd))) {
+            bs = sc[d];
+            bd = dist;
+            bp = alive[q];
+          }
         }
-        __syncwarp();
-        ++np;
+        best[me] = bp;
       }
+      __syncthreads();
+      if (t < na) {
+        const int me = alive[t], c = best[me];
+        if (c >= 0 && best[c] == me) partner[me] = c;
+      }
+      __syncthreads();
+      const int me = (t < na) ? alive[t] : -1;
+      const bool stay = me >= 0 && partner[me] < 0;
+      int nna = 0;
+      const int at = block_exclusive_scan(stay ? 1 : 0, sbuf, &nna);
+      if (stay) alive[at] = me;
+      __syncthreads();
+      if (nna == na) break;
+      na = nna;
+    }
+    // matched pairs, numbered by the position of their earlier block, then the
+    // unpaired blocks two by two in order
+    int nm = 0;
+    for (int p0 = 0; p0 < Nb; p0 += blockDim.x) {
+      const int p = p0 + threadIdx.x;
+      const int c = (p < Nb) ? partner[p] : -1;
+      const bool first = c > p;
+      int tot = 0;
+      const int j = nm + block_exclusive_scan(first ? 1 : 0, sbuf, &tot);
+      if (first) {
+        pa[j] = p;
+        pb[j] = c;
+      }
+      nm += tot;
+    }
+    for (int q = 2 * threadIdx.x; q < na; q += 2 * blockDim.x) {
+      pa[nm + q / 2] = alive[q];
+      pb[nm + q / 2] = (q + 1 < na) ? alive[q + 1] : -1;
+    }
+    __syncthreads();
+    for (int p = threadIdx.x; p < Tq; p += blockDim.x) {
+      const int a = pa[p], b = pb[p];
+      int c = 0;
+      for (int w = 0; w < W; ++w) c += __popc(bitsT[w * Nb + a] | (b >= 0 ? bitsT[w * Nb + b] : 0u));
+      keys2[p] = (static_cast<unsigned long long>(0xffffffu - static_cast<uint32_t>(c)) << 32) |
+                 static_cast<unsigned long long>(p);
     }
   } else {
     for (int p = threadIdx.x; p < Tq; p += blockDim.x) {
-      const int a = order[2 * p], b = (2 * p + 1 < Nb) ? order[2 * p + 1] : -1;
+      const int a = 2 * p, b = (2 * p + 1 < Nb) ? 2 * p + 1 : -1;
       pa[p] = a;
       pb[p] = b;
-      const int c = cnt[a] + (b >= 0 ? cnt[b] : 0);
+      const int c = cnt[order[a]] + (b >= 0 ? cnt[order[b]] : 0);
       keys2[p] = (static_cast<unsigned long long>(0xffffffu - static_cast<uint32_t>(c)) << 32) |
                  static_cast<unsigned long long>(p);
     }
@@ -468,7 +525,7 @@ static __global__ void __launch_bounds__(1024) pair_order_kernel(const unsigned 
   const long long u = bh - g0;
   for (int r = threadIdx.x; r < Tq; r += blockDim.x) {
     const int p = static_cast<int>(keys2[r] & 0xffffffffu);
-    const int a = pa[p], b = pb[p];
+    const int a = order[pa[p]], b = pb[p] >= 0 ? order[pb[p]] : -1;
     const long long pos = g0 * Tq + static_cast<long long>(r) * gsize + u;
     work[2 * pos] = static_cast<int>(bh * Nb + a);
     work[2 * pos + 1] = b >= 0 ? static_cast<int>(bh * Nb + b) : -1;
@@ -479,9 +536,15 @@ static __global__ void __launch_bounds__(1024) pair_order_kernel(const unsigned 
 inline int pair_order_smem_bytes(int Nb) {
   auto p2 = [](int x) { int p = 2; while (p < x) p <<= 1; return p; };
   const int Tq = (Nb + 1) / 2;
-  int bytes = (p2(Nb) + p2(Tq)) * 8 + (2 * Tq + 2 * Nb) * 4;
-  if (Nb <= kPairGreedyMaxNb) bytes += Nb * ((Nb + 31) / 32) * 4;
+  int bytes = (p2(Nb) + p2(Tq)) * 8 + (2 * Tq + 4 * Nb + 34) * 4;
+  if (Nb <= kPairMatchMaxNb) bytes += Nb * ((Nb + 31) / 32) * 4;
   return bytes;
+}
+
+// Threads of pair_order_kernel: one per query block when pairs are matched.
+inline int pair_order_threads(int Nb) {
+  if (Nb <= kPairMatchMaxNb) return Nb <= 64 ? 64 : ((Nb + 31) / 32) * 32;
+  return 1024;
 }
 
 }  // namespace sa

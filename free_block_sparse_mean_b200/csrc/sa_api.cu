@@ -128,7 +128,7 @@ sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau
     const int smem = sa::pair_order_smem_bytes(Nb);
     if (set_smem(sa::pair_order_kernel, smem) != SA_OK) return SA_ERR_CUDA;
     const int G = sa::order_group_heads(BH, s.N, D);
-    sa::pair_order_kernel<<<static_cast<unsigned>(BH), Nb <= 512 ? 256 : 1024, smem, st>>>(sig, bits, count, Nb, Tq,
+    sa::pair_order_kernel<<<static_cast<unsigned>(BH), sa::pair_order_threads(Nb), smem, st>>>(sig, bits, count, Nb, Tq,
                                                                                           G, work);
     if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   }

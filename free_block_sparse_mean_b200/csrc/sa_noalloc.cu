@@ -99,7 +99,7 @@ sa_status launch_plan_noalloc(const sa_shape& s, const void* Q, const void* K, f
     if (cudaFuncSetAttribute(sa::pair_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
       return SA_ERR_CUDA;
-    sa::pair_order_kernel<<<static_cast<unsigned>(BH), Nb <= 512 ? 256 : 1024, smem, st>>>(
+    sa::pair_order_kernel<<<static_cast<unsigned>(BH), sa::pair_order_threads(Nb), smem, st>>>(
         sig, bits, count, Nb, Tq, sa::order_group_heads(BH, s.N, D), work);
     if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   }
