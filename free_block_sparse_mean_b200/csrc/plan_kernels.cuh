@@ -429,39 +429,41 @@ static __global__ void __launch_bounds__(1024) pair_order_kernel(const unsigned 
       bitsT[w * Nb + p] = src[static_cast<long long>(order[p]) * W + w];
     }
     __syncthreads();
-    // one thread per alive position (the launch gives at least Nb threads)
+    // one warp per alive position, one lane per candidate (the 16 alive positions
+    // on each side); the launch gives at least Nb threads, so t < Nb covers the
+    // alive list in the mutual-pick step
     int na = Nb;
-    constexpr int NC = 2 * kPairWindow + 1;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
     for (int round = 0; round < kPairRounds; ++round) {
       const int t = threadIdx.x;
-      if (t < na) {
-        const int me = alive[t];
-        const int qlo = t - kPairWindow;
-        int sc[NC];                               // overlap minus symmetric difference
-#pragma unroll
-        for (int d = 0; d < NC; ++d) sc[d] = 0;
-        for (int w = 0; w < W; ++w) {
-          const uint32_t* row = bitsT + w * Nb;
-          const uint32_t x = row[me];
-#pragma unroll
-          for (int d = 0; d < NC; ++d) {
-            const int q = qlo + d;
-            const uint32_t y = (q >= 0 && q < na) ? row[alive[q]] : 0u;
-            sc[d] += __popc(x & y) - __popc(x ^ y);
+      for (int a = warp; a < na; a += nwarps) {
+        const int me = alive[a];
+        const int d = lane < kPairWindow ? lane - kPairWindow : lane - kPairWindow + 1;   // -16..-1, 1..16
+        const int q = a + d;
+        const bool ok = q >= 0 && q < na;
+        const int cpos = ok ? alive[q] : -1;
+        int sc = INT_MIN;
+        if (ok) {
+          sc = 0;
+          for (int w = 0; w < W; ++w) {
+            const uint32_t x = bitsT[w * Nb + me], y = bitsT[w * Nb + cpos];
+            sc += __popc(x & y) - __popc(x ^ y);
           }
         }
-        // best score; ties to the nearer, then the earlier candidate
-        int bs = INT_MIN, bd = INT_MAX, bp = -1;
+        // warp argmax of (score, -distance, -offset): ties to the nearer, then the earlier
+        int bs = sc, bd = abs(d), bdd = d, bp = cpos;
 #pragma unroll
-        for (int d = 0; d < NC; ++d) {
-          const int q = qlo + d, dist = abs(d - kPairWindow);
-          if (q >= 0 && q < na && d != kPairWindow && (sc[d] > bs || (sc[d] == bs && dist < bd))) {
-            bs = sc[d];
-            bd = dist;
-            bp = alive[q];
+        for (int o = 16; o; o >>= 1) {
+          const int os = __shfl_xor_sync(0xffffffffu, bs, o), od = __shfl_xor_sync(0xffffffffu, bd, o);
+          const int odd = __shfl_xor_sync(0xffffffffu, bdd, o), op = __shfl_xor_sync(0xffffffffu, bp, o);
+          if (os > bs || (os == bs && (od < bd || (od == bd && odd < bdd)))) {
+            bs = os;
+            bd = od;
+            bdd = odd;
+            bp = op;
           }
         }
-        best[me] = bp;
+        if (lane == 0) best[me] = (bs == INT_MIN) ? -1 : bp;
       }
       __syncthreads();
       if (t < na) {
@@ -541,10 +543,8 @@ inline int pair_order_smem_bytes(int Nb) {
   return bytes;
 }
 
-// Threads of pair_order_kernel: one per query block when pairs are matched.
-inline int pair_order_threads(int Nb) {
-  if (Nb <= kPairMatchMaxNb) return Nb <= 64 ? 64 : ((Nb + 31) / 32) * 32;
-  return 1024;
-}
+// Threads of pair_order_kernel: a warp per query block in the matching rounds,
+// and at least one thread per block of the alive list.
+inline int pair_order_threads(int /*Nb*/) { return 1024; }
 
 }  // namespace sa
