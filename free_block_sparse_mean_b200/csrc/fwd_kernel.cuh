@@ -18,17 +18,20 @@
 //   O += P V_j      128xD fp32 in TMEM; A operand (P) read from TMEM, B (V_j)
 //                   from shared memory as an MN-major operand
 //
-// Roles (192 threads): warp 0 builds the union list, then one of its threads loads
-// Q, K and V (TMA; K and V as one 4-D box per 64-row block, since TMA issue cost
-// is per instruction); warp 1 owns TMEM and one of its threads issues the MMAs;
-// warps 2..5 run the softmax (thread = row; warp w reaches TMEM lanes 32*(w%4) ..
-// 32*(w%4)+31), the O correction and the epilogue.
+// Roles (192 threads): warp 0 builds the union list, then one of its threads
+// loads V and issues the P.V MMAs; warp 1 owns TMEM and one of its threads loads
+// Q and K and issues the S MMAs (TMA, K and V as one 4-D box per 64-row block,
+// since TMA issue cost is per instruction); warps 2..5 run the softmax (thread =
+// row; warp w reaches TMEM lanes 32*(w%4) .. 32*(w%4)+31), the O correction and
+// the epilogue. The issue of a tcgen05.mma that accumulates into the result of
+// the previous one waits for it, so S and P.V get a thread each: S(k+1) is issued
+// as soon as S(k) is released, whatever P(k-1).V is doing.
 //
 // TMEM (256 columns): S [0,64), P double buffer [64,96) and [96,128), O [128,
 // 128+D). S is released as soon as the softmax warps hold S(k) in registers, so
 // S(k+1) runs on the tensor cores while the softmax works on S(k); P(k) goes to
-// buffer k&1, whose previous reader P(k-2).V has finished by the time S(k) is
-// complete (the MMAs of one thread run in issue order). Two CTAs fit on an SM
+// buffer k&1 once its previous reader, P(k-2).V, has finished (a wait that has
+// normally long passed). Two CTAs fit on an SM
 // (about 106 KB of shared memory and 256 TMEM columns each), so one CTA's softmax
 // also overlaps the other's MMAs.
 //
@@ -41,9 +44,12 @@
 // An mbarrier wait by parity is only sound when the barrier is at most one phase
 // ahead of, and at most one phase short of, the phase waited for; otherwise the
 // parity aliases and the wait returns early or never. Every wait below satisfies
-// that: S(k+1) is issued only after all softmax warps released S(k); P(k+2) can be
-// published only after S(k+2), which the MMA thread issues after it has waited for
-// P(k); P.V completions are double-buffered like P. The lambda votes carry the
+// that: S(k+1) is issued only after all softmax warps released S(k); P(k+2) is
+// published only after the softmax warps have seen P(k).V finish, so the P.V
+// thread has waited for P(k) by then; the P.V completions are double-buffered like
+// P, and the softmax waits on them for P(k-2) (and, to correct O, P(k-1)) after
+// having waited for P(k-4) (P(k-3)) before. A K or V stage is refilled only after
+// the MMA that read it has completed. The lambda votes carry the
 // entry index as a tag, and a vote slot is reused for entry k+2 only after every
 // softmax warp has released S(k+1), which each does after reading entry k's vote.
 #pragma once
@@ -129,7 +135,7 @@ __global__ void __launch_bounds__(192, 2)
   uint64_t* s_free = q_full + 2;               // S(k) read by all 4 softmax warps (phase k)
   uint64_t* p_full = q_full + 3;               // [2] by k parity: P(k) in TMEM and O corrected (4 warps)
   uint64_t* pv_done = q_full + 5;              // [2] by k parity: P(k).V finished
-  uint64_t* drain = q_full + 7;                // every MMA of the tile finished (single phase)
+  uint64_t* drain = q_full + 7;                // every MMA of the tile finished (single phase, 2 issuers)
   int* misc = reinterpret_cast<int*>(base + C::oMisc);
   volatile int* abort_flag = misc + 0;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(misc + 1);
@@ -174,7 +180,7 @@ __global__ void __launch_bounds__(192, 2)
     mbar_init(&p_full[1], 4);
     mbar_init(&pv_done[0], 1);
     mbar_init(&pv_done[1], 1);
-    mbar_init(drain, 1);
+    mbar_init(drain, 2);
     *abort_flag = 0;
     for (int x = 8; x < 16; ++x) misc[x] = -1;   // vote tags -1: no entry yet
     fence_mbar_init();
@@ -226,79 +232,20 @@ __global__ void __launch_bounds__(192, 2)
   const int n = *list_n;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ Q, K, V producer
-    // Loads in the order the MMAs need them: Q, K(0), then K(k+1) before V(k)
-    // (S(k+1) is issued before P(k).V).
+    // ------------------------------------------------------------ V producer, P.V issuer
     if (lane == 0 && n > 0) {
-      // Q rows of the two query blocks into rows 0..63 / 64..127 of the tile
-      mbar_expect_tx(q_full, (qb1 >= 0 ? 2 : 1) * C::kKVBytes);
-#pragma unroll
-      for (int c = 0; c < C::kChunks; ++c) {
-        tma_load_3d(sQ + c * C::kQChunkBytes, &tmQ, c * 64, qb0 * kBlock, static_cast<int>(bh), q_full);
-        if (qb1 >= 0)
-          tma_load_3d(sQ + c * C::kQChunkBytes + C::kKVChunkBytes, &tmQ, c * 64, qb1 * kBlock,
-                      static_cast<int>(bh), q_full);
-      }
-      auto load_k = [&](int k) -> bool {
-        const int s = k % C::STK;
-        if (!mbar_wait(&kempty[s], (static_cast<uint32_t>(k / C::STK) & 1u) ^ 1u, abort_flag)) return false;
-        const int j = static_cast<int>(lst[k] & kListJMask);
-        mbar_expect_tx(&kfull[s], C::kKVBytes);
-        tma_load_4d(sK + s * C::kKVBytes, &tmK, 0, j * kBlock, 0, static_cast<int>(bh), &kfull[s]);
-        return true;
-      };
-      int nk = load_k(0) ? 1 : 0, nv = 0;         // loads issued
-      for (int k = 0; nk > k && k < n; ++k) {
-        if (k + 1 < n) {
-          if (!load_k(k + 1)) break;
-          ++nk;
-        }
+      const uint32_t sVa = smem_u32(sV);
+      auto load_v = [&](int k) {
         const int s = k % C::STV;
-        if (!mbar_wait(&vempty[s], (static_cast<uint32_t>(k / C::STV) & 1u) ^ 1u, abort_flag)) break;
         const int j = static_cast<int>(lst[k] & kListJMask);
         mbar_expect_tx(&vfull[s], C::kKVBytes);
         tma_load_4d(sV + s * C::kKVBytes, &tmV, 0, j * kBlock, 0, static_cast<int>(bh), &vfull[s]);
-        ++nv;
-      }
-      // let issued loads land before exit
-      mbar_wait_drain(q_full, 0u);
-      for (int kk = max(0, nk - C::STK); kk < nk; ++kk)
-        mbar_wait_drain(&kfull[kk % C::STK], static_cast<uint32_t>(kk / C::STK) & 1u);
-      for (int kk = max(0, nv - C::STV); kk < nv; ++kk)
-        mbar_wait_drain(&vfull[kk % C::STV], static_cast<uint32_t>(kk / C::STV) & 1u);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n > 0) {
-      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-      bool ok = mbar_wait(q_full, 0u, abort_flag);
-      tc_fence_after();
-      // S(k) = Q K_k^T into the S columns (the softmax warps have released S(k-1)).
-      auto issue_S = [&](int k) -> bool {
-        const int s = k % C::STK;
-        if (!mbar_wait(&kfull[s], static_cast<uint32_t>(k / C::STK) & 1u, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t dS = tmem_base + C::kColS;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk & 3) * 32;  // 16 bf16 = 32 bytes inside the swizzle atom
-          const uint64_t ad = sdesc_sw128(sQa + (kk >> 2) * C::kQChunkBytes + off, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sKa + s * C::kKVBytes + (kk >> 2) * C::kKVChunkBytes + off, 16, 1024);
-          tc_mma_ss(dS, ad, bd, C::kIdescS, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(s_full);
-        tc_commit(&kempty[s]);
-        return true;
       };
-      if (ok) ok = issue_S(0);
+      int nv = 0;                                 // V loads issued
+      for (; nv < C::STV && nv < n; ++nv) load_v(nv);
       uint32_t o_init = 0;
       unsigned long long pv_tiles = 0;
-      for (int k = 0; ok && k < n; ++k) {
-        if (k + 1 < n) {
-          if (!mbar_wait(s_free, static_cast<uint32_t>(k) & 1u, abort_flag)) break;
-          tc_fence_after();
-          if (!issue_S(k + 1)) break;
-        }
+      for (int k = 0; k < n; ++k) {
         if (!mbar_wait(&p_full[k & 1], static_cast<uint32_t>(k >> 1) & 1u, abort_flag)) break;
         const int s = k % C::STV;
         if (!mbar_wait(&vfull[s], static_cast<uint32_t>(k / C::STV) & 1u, abort_flag)) break;
@@ -316,15 +263,72 @@ __global__ void __launch_bounds__(192, 2)
         }
         tc_commit(&pv_done[k & 1]);
         tc_commit(&vempty[s]);
+        // refill this stage with V(k+STV) once P(k).V has read it
+        if (k + C::STV < n) {
+          if (!mbar_wait(&vempty[s], static_cast<uint32_t>(k / C::STV) & 1u, abort_flag)) break;
+          load_v(k + C::STV);
+          ++nv;
+        }
       }
-      // Drain: every MMA this thread issued has finished (bounded); the softmax
-      // warps wait on the same single-phase barrier before reading O.
+      // Drain: every MMA this thread issued has finished and its loads have landed
+      // (bounded); the softmax warps wait on the same barrier before reading O.
       tc_commit(drain);
       mbar_wait_drain(drain, 0u);
-      if (stats) {
-        atomicAdd(&stats[2], static_cast<unsigned long long>(n));
-        atomicAdd(&stats[3], pv_tiles);
+      for (int kk = max(0, nv - C::STV); kk < nv; ++kk)
+        mbar_wait_drain(&vfull[kk % C::STV], static_cast<uint32_t>(kk / C::STV) & 1u);
+      if (stats) atomicAdd(&stats[3], pv_tiles);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ Q, K producer, S issuer
+    if (lane == 0 && n > 0) {
+      // Q rows of the two query blocks into rows 0..63 / 64..127 of the tile
+      mbar_expect_tx(q_full, (qb1 >= 0 ? 2 : 1) * C::kKVBytes);
+#pragma unroll
+      for (int c = 0; c < C::kChunks; ++c) {
+        tma_load_3d(sQ + c * C::kQChunkBytes, &tmQ, c * 64, qb0 * kBlock, static_cast<int>(bh), q_full);
+        if (qb1 >= 0)
+          tma_load_3d(sQ + c * C::kQChunkBytes + C::kKVChunkBytes, &tmQ, c * 64, qb1 * kBlock,
+                      static_cast<int>(bh), q_full);
       }
+      auto load_k = [&](int k) {
+        const int s = k % C::STK;
+        const int j = static_cast<int>(lst[k] & kListJMask);
+        mbar_expect_tx(&kfull[s], C::kKVBytes);
+        tma_load_4d(sK + s * C::kKVBytes, &tmK, 0, j * kBlock, 0, static_cast<int>(bh), &kfull[s]);
+      };
+      int nk = 0;                                 // K loads issued
+      for (; nk < C::STK && nk < n; ++nk) load_k(nk);
+      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK);
+      bool ok = mbar_wait(q_full, 0u, abort_flag);
+      // S(k) = Q K_k^T into the S columns, once the softmax warps released S(k-1)
+      for (int k = 0; ok && k < n; ++k) {
+        if (k > 0 && !mbar_wait(s_free, static_cast<uint32_t>(k - 1) & 1u, abort_flag)) break;
+        const int s = k % C::STK;
+        if (!mbar_wait(&kfull[s], static_cast<uint32_t>(k / C::STK) & 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t dS = tmem_base + C::kColS;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk & 3) * 32;  // 16 bf16 = 32 bytes inside the swizzle atom
+          const uint64_t ad = sdesc_sw128(sQa + (kk >> 2) * C::kQChunkBytes + off, 16, 1024);
+          const uint64_t bd = sdesc_sw128(sKa + s * C::kKVBytes + (kk >> 2) * C::kKVChunkBytes + off, 16, 1024);
+          tc_mma_ss(dS, ad, bd, C::kIdescS, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(s_full);
+        tc_commit(&kempty[s]);
+        // refill this stage with K(k+STK) once S(k) has read it
+        if (k + C::STK < n) {
+          if (!mbar_wait(&kempty[s], static_cast<uint32_t>(k / C::STK) & 1u, abort_flag)) break;
+          load_k(k + C::STK);
+          ++nk;
+        }
+      }
+      tc_commit(drain);
+      mbar_wait_drain(drain, 0u);
+      mbar_wait_drain(q_full, 0u);
+      for (int kk = max(0, nk - C::STK); kk < nk; ++kk)
+        mbar_wait_drain(&kfull[kk % C::STK], static_cast<uint32_t>(kk / C::STK) & 1u);
+      if (stats) atomicAdd(&stats[2], static_cast<unsigned long long>(n));
     }
   } else if (warp >= 2) {
     // ------------------------------------------------------------ softmax warps
@@ -430,11 +434,18 @@ __global__ void __launch_bounds__(192, 2)
           for (int c = 0; c < 32; ++c) pk[c] = 0u;
         }
       }
-      // P(k) into buffer k&1 (its previous reader, P(k-2).V, finished before S(k))
+      // P(k) into buffer k&1 once its previous reader, P(k-2).V, has finished
+      if (k >= 2) {
+        if (!warp_wait(&pv_done[k & 1], static_cast<uint32_t>((k - 2) >> 1) & 1u, abort_flag)) {
+          alive = false;
+          break;
+        }
+        tc_fence_after();
+      }
       tmem_st32u(tmem_base + lane_bits + ((k & 1) ? C::kColP1 : C::kColP0), pk);
       // O correction for rows whose reference max was raised (after P(k-1).V);
-      // pv_done[(k-1)&1] is at most one phase short of entry k-1 (P(k-3).V finished
-      // before S(k-1)).
+      // pv_done[(k-1)&1] is at most one phase short of entry k-1 (this warp waited
+      // for P(k-3).V before storing P(k-1)).
       if (k > 0 && any_raise) {
         if (!warp_wait(&pv_done[(k - 1) & 1], static_cast<uint32_t>((k - 1) >> 1) & 1u, abort_flag)) {
           alive = false;
