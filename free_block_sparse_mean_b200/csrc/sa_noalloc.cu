@@ -74,10 +74,10 @@ sa_status launch_plan_noalloc(const sa_shape& s, const void* Q, const void* K, f
   sa::pool_kernel<D><<<dim3(static_cast<unsigned>(BH * Nb), 2), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Qp, Kp, s.N, Nb);
   if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
-  const int ldL = (Nb + 3) & ~3;
   // Small heads: 4 query blocks per CTA so the grid still fills the GPU.
   auto launch_ss = [&](auto kern, int R, int NT) -> sa_status {
-    const int smem = (D * (R + 4) + R * ldL) * static_cast<int>(sizeof(float));
+    const int smem = R == 4 ? sa::score_select_smem_bytes<D, 4>(Nb)
+                            : (R == 8 ? sa::score_select_smem_bytes<D, 8>(Nb) : sa::score_select_smem_bytes<D, 16>(Nb));
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return SA_ERR_CUDA;
     kern<<<dim3((Nb + R - 1) / R, static_cast<unsigned>(BH)), NT, smem, st>>>(Qp, Kp, Nb, scale, causal, tau,
