@@ -15,7 +15,7 @@ from __future__ import annotations
 import ctypes
 import math
 from dataclasses import dataclass
-from typing import Optional
+from typing import Optional, Union
 
 import torch
 
@@ -26,6 +26,7 @@ BLOCK = 64
 
 __all__ = ["Plan", "sparse_attn_plan", "sparse_attn_fwd", "sparse_attention",
            "sparse_attn_plan_workspace_size", "sparse_attn_num_tiles", "sparse_attn_device_error",
+           "sparse_attn_selftest_wait_timeout",
            "SparseAttnError", "BLOCK"]
 
 
@@ -77,7 +78,7 @@ class Plan:
     count: torch.Tensor
     idx: Optional[torch.Tensor]
     work: Optional[torch.Tensor]
-    tau: float
+    tau: Union[float, torch.Tensor]   # one threshold, or one per (batch, head)
     causal: bool
 
 
@@ -89,10 +90,13 @@ def sparse_attn_num_tiles(B: int, H: int, N: int, d: int) -> int:
     return int(_lib.load().sparse_attn_num_tiles(SaShape(B, H, N, d, BLOCK)))
 
 
-def sparse_attn_plan(q: torch.Tensor, k: torch.Tensor, tau: float, scale: Optional[float] = None,
+def sparse_attn_plan(q: torch.Tensor, k: torch.Tensor, tau, scale: Optional[float] = None,
                      causal: bool = False, *, with_idx: bool = True, with_work: bool = True,
                      out: Optional[Plan] = None, workspace: Optional[torch.Tensor] = None) -> Plan:
-    """Stage 1: cumulative-energy block mask from mean-pooled q and k."""
+    """Stage 1: cumulative-energy block mask from mean-pooled q and k.
+
+    tau is one recall threshold for every head (a float), or one per head: a float32
+    CUDA tensor of shape [B, H] or [H] on q's device (sparse_attn_plan_heads)."""
     lib = _lib.load()
     _check_qkv(q, k)
     B, H, N, d = q.shape
@@ -108,12 +112,25 @@ def sparse_attn_plan(q: torch.Tensor, k: torch.Tensor, tau: float, scale: Option
             idx=torch.empty((B, H, Nb, Nb), dtype=torch.int32, device=dev) if with_idx else None,
             work=torch.empty((max(2, 2 * lib.sparse_attn_num_tiles(s)),), dtype=torch.int32, device=dev)
             if with_work else None,
-            tau=float(tau), causal=bool(causal))
+            tau=tau if isinstance(tau, torch.Tensor) else float(tau), causal=bool(causal))
     else:
-        out.tau, out.causal = float(tau), bool(causal)
+        out.tau, out.causal = (tau if isinstance(tau, torch.Tensor) else float(tau)), bool(causal)
     ws_bytes = int(lib.sparse_attn_plan_workspace_size(s))
     if workspace is None or workspace.numel() < ws_bytes:
         workspace = torch.empty((max(ws_bytes, 256),), dtype=torch.uint8, device=dev)
+    if isinstance(tau, torch.Tensor):
+        if tau.dtype != torch.float32 or tau.device != dev:
+            raise ValueError("a per-head tau must be a float32 tensor on q's device")
+        if tuple(tau.shape) == (H,):
+            tau = tau.unsqueeze(0).expand(B, H)
+        if tuple(tau.shape) != (B, H):
+            raise ValueError("a per-head tau must have shape [B, H] or [H]")
+        tau = tau.contiguous()
+        st = lib.sparse_attn_plan_heads(_ptr(q), _ptr(k), s, _ptr(tau), float(scale), int(bool(causal)),
+                                        _ptr(out.mask), _ptr(out.count), _ptr(out.idx), _ptr(out.work),
+                                        _ptr(workspace), ws_bytes, _stream(dev))
+        _call("sparse_attn_plan_heads", st)
+        return out
     st = lib.sparse_attn_plan(_ptr(q), _ptr(k), s, float(tau), float(scale), int(bool(causal)),
                               _ptr(out.mask), _ptr(out.count), _ptr(out.idx), _ptr(out.work),
                               _ptr(workspace), ws_bytes, _stream(dev))
@@ -180,3 +197,14 @@ def sparse_attn_device_error(device=None) -> int:
     with torch.cuda.device(dev):
         _call("sparse_attn_device_error", lib.sparse_attn_device_error(_stream(dev), ctypes.byref(code)))
     return int(code.value)
+
+
+def sparse_attn_selftest_wait_timeout(limit_us: int, device=None) -> None:
+    """Launch the library's failure-path diagnostic on the current stream: one warp
+    waits on a barrier that nothing completes, gives up after limit_us
+    microseconds and records a timeout in the device error word (read it with
+    sparse_attn_device_error). The kernel returns normally."""
+    lib = _lib.load()
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        _call("sparse_attn_selftest_wait_timeout", lib.sparse_attn_selftest_wait_timeout(int(limit_us), _stream(dev)))

@@ -24,10 +24,12 @@ EXPORTS = (
     "sparse_attn_plan_workspace_size",
     "sparse_attn_num_tiles",
     "sparse_attn_plan",
+    "sparse_attn_plan_heads",
     "sparse_attn_fwd",
     "sparse_attn_status_string",
     "sparse_attn_device_error",
     "sparse_attn_plan_noalloc",
+    "sparse_attn_selftest_wait_timeout",
 )
 
 
@@ -68,6 +70,8 @@ def load(path: str = LIB_PATH):
     lib.sparse_attn_num_tiles.restype = ctypes.c_int64
     lib.sparse_attn_plan.argtypes = [vp, vp, SaShape, f32, f32, i32, vp, vp, vp, vp, vp, sz, vp]
     lib.sparse_attn_plan.restype = i32
+    lib.sparse_attn_plan_heads.argtypes = [vp, vp, SaShape, vp, f32, i32, vp, vp, vp, vp, vp, sz, vp]
+    lib.sparse_attn_plan_heads.restype = i32
     lib.sparse_attn_fwd.argtypes = [vp, vp, vp, SaShape, vp, vp, f32, f32, i32, vp, vp, vp]
     lib.sparse_attn_fwd.restype = i32
     lib.sparse_attn_status_string.argtypes = [i32]
@@ -76,5 +80,7 @@ def load(path: str = LIB_PATH):
     lib.sparse_attn_device_error.restype = i32
     lib.sparse_attn_plan_noalloc.argtypes = [vp, vp, SaShape, f32, f32, i32, vp, vp, vp, vp, vp]
     lib.sparse_attn_plan_noalloc.restype = i32
+    lib.sparse_attn_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp]
+    lib.sparse_attn_selftest_wait_timeout.restype = i32
     _lib = lib
     return lib

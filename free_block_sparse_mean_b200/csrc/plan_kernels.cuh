@@ -95,7 +95,8 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 }
 
 // ----------------------------------------------------------------------------
-// Pooled scores + selection. One CTA = R query blocks of one head.
+// Pooled scores + selection. One CTA = R query blocks of one head. tau is the
+// recall threshold of every head, or tau_bh[b*H + h] per head when tau_bh is given.
 //
 // Phase 1 (CUDA-core fp32 GEMM, the pooled scores must stay fp32 to keep the
 // kept set stable near tau): thread t owns key blocks c = 2t, 2t+1 of each
@@ -123,6 +124,7 @@ template <int D, int R, int NT>
 __global__ void __launch_bounds__(NT) score_select_kernel(const float* __restrict__ Qp,
                                                            const float* __restrict__ Kp, int Nb,
                                                            float scale, int causal, float tau,
+                                                           const float* __restrict__ tau_bh,
                                                            uint8_t* __restrict__ mask,
                                                            int* __restrict__ count,
                                                            int* __restrict__ idx,
@@ -250,6 +252,15 @@ __global__ void __launch_bounds__(NT) score_select_kernel(const float* __restric
   __syncthreads();
 
   // ---------------- phase 2: selection, one warp per row
+  // the head's own tau when one is given per (b, h); an invalid one (not in (0, 1])
+  // is recorded in the device error word and the head keeps every block
+  if (tau_bh) {
+    tau = tau_bh[bh];
+    if (!(tau > 0.f && tau <= 1.f)) {
+      if (threadIdx.x == 0) atomicOr(&g_dev_error, DEVERR_VALUE);
+      tau = 1.f;
+    }
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned FULL = 0xffffffffu;
   const float LOG2E = 1.4426950408889634f;

@@ -89,8 +89,9 @@ sa_status set_smem(F* kernel, int bytes) {
 }
 
 template <int D>
-sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau, float scale, int causal,
-                      uint8_t* mask, int32_t* count, int32_t* idx, int32_t* work, void* ws, cudaStream_t st) {
+sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau, const float* tau_bh,
+                      float scale, int causal, uint8_t* mask, int32_t* count, int32_t* idx, int32_t* work,
+                      void* ws, cudaStream_t st) {
   const int Nb = static_cast<int>(num_blocks(s));
   const long long BH = static_cast<long long>(s.B) * s.H;
   const sa::PlanWorkspace L = sa::plan_workspace(BH, Nb, D);
@@ -110,7 +111,7 @@ sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return SA_ERR_CUDA;
     kern<<<dim3((Nb + R - 1) / R, static_cast<unsigned>(BH)), NT, smem, st>>>(Qp, Kp, Nb, scale, causal, tau,
-                                                                               mask, count, idx, sig, bits);
+                                                                               tau_bh, mask, count, idx, sig, bits);
     return SA_OK;
   };
   sa_status ls;
@@ -161,6 +162,25 @@ sa_status launch_fwd(const sa_shape& s, const void* Q, const void* K, const void
 
 }  // namespace
 
+namespace sa {
+// Exercises the device-side failure path: one warp waits on an mbarrier whose
+// phase nothing completes, through the same bounded wait the pipelines use, with
+// a short limit. The wait gives up, records DEVERR_TIMEOUT in the error word and
+// the kernel returns normally.
+__global__ void __launch_bounds__(32) wait_timeout_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) mbar_wait_slow(&bar, 0u, &abort_flag, limit_ns);   // nothing arrives
+  __syncwarp();
+}
+}  // namespace sa
+
 extern "C" {
 
 size_t sparse_attn_plan_workspace_size(sa_shape s) {
@@ -186,8 +206,26 @@ sa_status sparse_attn_plan(const void* Q, const void* K, sa_shape s, float tau, 
       workspace_bytes < sparse_attn_plan_workspace_size(s))
     return SA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (s.d == 64) return launch_plan<64>(s, Q, K, tau, scale, causal != 0, mask, count, idx, work, workspace, st);
-  return launch_plan<128>(s, Q, K, tau, scale, causal != 0, mask, count, idx, work, workspace, st);
+  if (s.d == 64)
+    return launch_plan<64>(s, Q, K, tau, nullptr, scale, causal != 0, mask, count, idx, work, workspace, st);
+  return launch_plan<128>(s, Q, K, tau, nullptr, scale, causal != 0, mask, count, idx, work, workspace, st);
+}
+
+sa_status sparse_attn_plan_heads(const void* Q, const void* K, sa_shape s, const float* tau, float scale,
+                                 int32_t causal, uint8_t* mask, int32_t* count, int32_t* idx, int32_t* work,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  if (!Q || !K || !tau || !mask || !count) return SA_ERR_INVALID_ARG;
+  const sa_status sh = check_shape(s);
+  if (sh != SA_OK) return sh;
+  if (!(std::isfinite(scale) && scale > 0.f)) return SA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || (reinterpret_cast<uintptr_t>(tau) & 3u) != 0) return SA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < sparse_attn_plan_workspace_size(s))
+    return SA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s.d == 64)
+    return launch_plan<64>(s, Q, K, 1.f, tau, scale, causal != 0, mask, count, idx, work, workspace, st);
+  return launch_plan<128>(s, Q, K, 1.f, tau, scale, causal != 0, mask, count, idx, work, workspace, st);
 }
 
 sa_status sparse_attn_fwd(const void* Q, const void* K, const void* V, sa_shape s, const uint8_t* mask,
@@ -215,6 +253,14 @@ const char* sparse_attn_status_string(sa_status st) {
     case SA_ERR_DEVICE_CHECK: return "SA_ERR_DEVICE_CHECK: a device-side check fired";
   }
   return "unknown sa_status";
+}
+
+sa_status sparse_attn_selftest_wait_timeout(uint32_t limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 4000000) return SA_ERR_INVALID_ARG;
+  sa::wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<unsigned long long>(limit_us) * 1000ull);
+  if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+  return SA_OK;
 }
 
 sa_status sparse_attn_device_error(void* stream, int32_t* code) {

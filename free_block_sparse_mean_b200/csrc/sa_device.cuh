@@ -17,7 +17,7 @@ constexpr int kMaxNb = 4096;  // largest supported number of blocks per head
 // Device error word (one per GPU that loads the library). Kernels OR codes into
 // it instead of trapping; the host reads and clears it. All kernels live in one
 // translation unit, so this definition is the only one.
-enum : unsigned { DEVERR_TIMEOUT = 1u, DEVERR_RANGE = 2u };
+enum : unsigned { DEVERR_TIMEOUT = 1u, DEVERR_RANGE = 2u, DEVERR_VALUE = 4u };
 static __device__ unsigned int g_dev_error;
 
 // A single pipeline wait never legitimately takes this long.
@@ -60,15 +60,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Slow path of mbar_wait: polls until the phase with the given parity completes.
-// Gives up (returns false) when *abort is set by another role or after
-// kWaitTimeoutNs, in which case it sets *abort and records DEVERR_TIMEOUT.
-static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// Gives up (returns false) when *abort is set by another role or after limit_ns
+// (kWaitTimeoutNs unless given), in which case it sets *abort and records
+// DEVERR_TIMEOUT.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                   unsigned long long limit_ns = kWaitTimeoutNs) {
   const unsigned long long t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0u) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort = 1;
         atomicOr(&g_dev_error, DEVERR_TIMEOUT);
         return false;

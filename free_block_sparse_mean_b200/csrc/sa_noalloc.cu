@@ -81,7 +81,7 @@ sa_status launch_plan_noalloc(const sa_shape& s, const void* Q, const void* K, f
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return SA_ERR_CUDA;
     kern<<<dim3((Nb + R - 1) / R, static_cast<unsigned>(BH)), NT, smem, st>>>(Qp, Kp, Nb, scale, causal, tau,
-                                                                               mask, count, idx, sig, bits);
+                                                                               nullptr, mask, count, idx, sig, bits);
     return SA_OK;
   };
   sa_status ls;

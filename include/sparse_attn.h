@@ -104,6 +104,19 @@ sa_status sparse_attn_plan(const void* Q, const void* K, sa_shape s, float tau, 
                            int32_t causal, uint8_t* mask, int32_t* count, int32_t* idx,
                            int32_t* work, void* workspace, size_t workspace_bytes, void* stream);
 
+/* sparse_attn_plan with one recall threshold per head: head (b, h) keeps, per
+ * query block, the shortest prefix of its sorted pooled probabilities reaching
+ * tau[b*H + h] times the row sum. This is the per-head, per-call threshold of an
+ * SNR-guided sparsity schedule (iCATS abstract: the sparsity follows the
+ * denoising timestep). tau is a DEVICE array of B*H floats, 4-byte aligned, read
+ * on the stream. A value outside (0, 1] (NaN included) cannot be checked on the
+ * host: that head then keeps every block with a finite score (as tau = 1), and
+ * bit 2 of the device error word is set. All other arguments, outputs and
+ * errors are those of sparse_attn_plan. */
+sa_status sparse_attn_plan_heads(const void* Q, const void* K, sa_shape s, const float* tau, float scale,
+                                 int32_t causal, uint8_t* mask, int32_t* count, int32_t* idx,
+                                 int32_t* work, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Stage 2: sparse attention over the kept blocks, with the lambda P.V filter.
  *
  *   Q, K, V   device bf16 [B,H,N,d]
@@ -150,13 +163,25 @@ sa_status sparse_attn_plan_noalloc(const void* Q, const void* K, sa_shape s, flo
                                    int32_t causal, uint8_t* mask, int32_t* count, int32_t* idx,
                                    int32_t* work, void* stream);
 
+/* Diagnostic of the device-side failure path (no counterpart in the paper; it
+ * tests this library's own safeguards). Launches one warp on `stream` that
+ * waits on a barrier nothing completes, through the bounded wait every pipeline
+ * of this library uses, with a limit of limit_us microseconds instead of the
+ * usual 4 s. The wait gives up, records bit 0 (a wait timed out) in the device
+ * error word and the kernel returns normally, so the context stays usable; read
+ * the word with sparse_attn_device_error. limit_us must be in [1, 4000000],
+ * else SA_ERR_INVALID_ARG and nothing is launched. A failed launch returns
+ * SA_ERR_CUDA. */
+sa_status sparse_attn_selftest_wait_timeout(uint32_t limit_us, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* sparse_attn_status_string(sa_status st);
 
 /* Reads the device error word of the current GPU (after synchronising `stream`),
  * stores it in *code (0 = no device-side check fired; bit 0 = a pipeline wait
- * timed out, bit 1 = an index was out of range) and clears it. Returns SA_OK, or
- * SA_ERR_CUDA if the copy failed. */
+ * timed out, bit 1 = an index was out of range, bit 2 = a value read from
+ * device memory was invalid, e.g. a per-head tau outside (0, 1]) and clears
+ * it. Returns SA_OK, or SA_ERR_CUDA if the copy failed. */
 sa_status sparse_attn_device_error(void* stream, int32_t* code);
 
 #ifdef __cplusplus

@@ -94,8 +94,12 @@ def pooled_softmax(L: np.ndarray) -> np.ndarray:
     return e / e.sum(axis=-1, keepdims=True)
 
 
-def cumulative_energy_select(P: np.ndarray, tau: float):
+def cumulative_energy_select(P: np.ndarray, tau):
     """Per row of the predicted map, keep the fewest blocks whose energy reaches tau.
+
+    tau is a scalar, or one value per (batch, head) (an array broadcastable to
+    P.shape[:-2], e.g. [B, H] or [H]): every row of a head uses its head's tau,
+    the per-head recall threshold of an SNR-guided schedule (iCATS abstract).
 
     DynSparse (cumulative energy filtering): a fixed recall of the attention energy
     is kept, and the per-row cut-off value (the smallest kept probability) is the
@@ -116,12 +120,13 @@ def cumulative_energy_select(P: np.ndarray, tau: float):
     idx = np.full(rows.shape, -1, dtype=np.int64)
     c_before = np.zeros(rows.shape, dtype=np.float64)
     c_after = np.zeros(rows.shape, dtype=np.float64)
+    tau_rows = np.broadcast_to(np.asarray(tau, dtype=np.float64)[..., None], shape[:-1]).reshape(-1)
     for r in range(rows.shape[0]):
         p = rows[r]
         order = np.argsort(-p, kind="stable")
         c = np.cumsum(p[order])
         total = c[-1]
-        hit = np.nonzero(c >= tau * total)[0]
+        hit = np.nonzero(c >= tau_rows[r] * total)[0]
         rstar = int(hit[0]) + 1 if hit.size else Nb
         kept = np.sort(order[:rstar])
         mask[r, kept] = 1
@@ -133,10 +138,10 @@ def cumulative_energy_select(P: np.ndarray, tau: float):
             c_before.reshape(shape), c_after.reshape(shape))
 
 
-def plan(Q, K, tau: float, scale: Optional[float] = None, causal: bool = False,
+def plan(Q, K, tau, scale: Optional[float] = None, causal: bool = False,
          block: int = BLOCK) -> dict:
     """Stage 1 end to end: pool, pooled logits, pooled softmax, cumulative-energy
-    selection. Q, K: [B, H, N, d]."""
+    selection. Q, K: [B, H, N, d]; tau a scalar or one value per (batch, head)."""
     Q = as_f64(Q)
     K = as_f64(K)
     d = Q.shape[-1]

@@ -107,3 +107,25 @@ def test_fwd_argument_errors(lib):
 
 def test_device_error_needs_output_pointer(lib):
     assert lib.sparse_attn_device_error(None, None) == 1
+
+
+def test_selftest_rejects_bad_limits(lib):
+    # checked on the host: nothing is launched
+    assert lib.sparse_attn_selftest_wait_timeout(0, None) == 1
+    assert lib.sparse_attn_selftest_wait_timeout(4000001, None) == 1
+
+
+def test_plan_heads_rejects_bad_arguments(lib):
+    s = SaShape(1, 2, 128, 128, 64)
+    fake = ctypes.c_void_p(256)       # never dereferenced: the checks run first
+    ws = int(lib.sparse_attn_plan_workspace_size(s))
+    # no tau array
+    assert lib.sparse_attn_plan_heads(fake, fake, s, None, 0.1, 0, fake, fake, None, None, fake, ws, None) == 1
+    # misaligned tau array
+    assert lib.sparse_attn_plan_heads(fake, fake, s, ctypes.c_void_p(258), 0.1, 0, fake, fake, None, None,
+                                      fake, ws, None) == 1
+    # bad scale, bad shape, missing workspace
+    assert lib.sparse_attn_plan_heads(fake, fake, s, fake, 0.0, 0, fake, fake, None, None, fake, ws, None) == 1
+    assert lib.sparse_attn_plan_heads(fake, fake, SaShape(1, 2, 128, 96, 64), fake, 0.1, 0, fake, fake, None,
+                                      None, fake, ws, None) == 2
+    assert lib.sparse_attn_plan_heads(fake, fake, s, fake, 0.1, 0, fake, fake, None, None, None, ws, None) == 3

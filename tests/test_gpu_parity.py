@@ -194,3 +194,38 @@ def test_repeatable_masks():
     b = sa.sparse_attn_plan(q, k, 0.9)
     torch.cuda.synchronize()
     assert torch.equal(a.mask, b.mask) and torch.equal(a.count, b.count)
+
+
+def test_per_head_tau_matches_oracle_and_flags_invalid_values():
+    """sparse_attn_plan_heads: every head keeps its own tau's set (small DiT
+    workload, tau from 0.85 to 0.99 over the heads), and a value outside (0, 1]
+    keeps every block of its head and sets bit 2 of the device error word."""
+    w = wl.WORKLOADS["small"]
+    q, k, _ = wl.generate(w, seed=0, device=_dev())
+    taus = torch.linspace(0.85, 0.99, w.H, dtype=torch.float32, device=_dev())
+    p = sa.sparse_attn_plan(q, k, taus)
+    torch.cuda.synchronize()
+    _no_device_error()
+    mask, count, idx = to_np(p.mask), to_np(p.count), to_np(p.idx)
+    check_plan_consistency(mask, count, idx)
+    _work_ok(p, 1, w.H, 64)
+    tau_np = taus.cpu().numpy().astype(np.float64)
+    op = orc.plan(q.cpu(), k.cpu(), tau_np[None, :])
+    rows = 0
+    for h in range(w.H):
+        oh = {key: op[key][:, h:h + 1] for key in ("mask", "P", "c_before", "c_after")}
+        r, _ = compare_masks(mask[:, h:h + 1], oh, float(tau_np[h]))
+        rows += r
+    assert rows <= max(2, (w.H * 64) // 200)
+    counts = count.reshape(w.H, 64).mean(-1)
+    assert counts[-1] > counts[0]                      # a higher tau keeps more
+
+    bad = taus.clone()
+    bad[3] = 1.5
+    bad[7] = float("nan")
+    p2 = sa.sparse_attn_plan(q, k, bad)
+    torch.cuda.synchronize()
+    assert sa.sparse_attn_device_error() == 4
+    m2 = to_np(p2.mask)
+    assert np.all(m2[0, 3] == 1) and np.all(m2[0, 7] == 1)
+    assert np.array_equal(m2[0, 4], mask[0, 4])

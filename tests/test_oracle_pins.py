@@ -168,6 +168,33 @@ def test_select_special_cases():
         assert list(idx[0, :k]) == list(range(k))
 
 
+def test_select_per_head_tau():
+    """One tau per (batch, head) applies to every row of that head: each row's kept
+    count is the smallest size of any subset reaching its head's tau (brute force),
+    the kept energy reaches it, tau = 1 keeps every block, and an [H] tau
+    broadcasts over the batch."""
+    r = _rng(11)
+    B, H, Nb = 2, 3, 8
+    P = orc.pooled_softmax(2.0 * r.standard_normal((B, H, Nb, Nb)))
+    taus = np.array([[1.0, 0.5, 0.9], [0.7, 0.99, 0.3]])
+    mask, count, idx, cb, ca = orc.cumulative_energy_select(P, taus)
+    for b in range(B):
+        for h in range(H):
+            t = taus[b, h]
+            for i in range(Nb):
+                p = P[b, h, i]
+                k_min = next(k for k in range(1, Nb + 1)
+                             if max(sum(p[list(c)]) for c in itertools.combinations(range(Nb), k))
+                             >= t * p.sum() - 1e-15)
+                assert count[b, h, i] == k_min
+                assert p[mask[b, h, i].astype(bool)].sum() >= t * p.sum() - 1e-15
+            if t == 1.0:
+                assert np.all(mask[b, h] == 1)
+    m_h, c_h, *_ = orc.cumulative_energy_select(P, taus[0])
+    m_bh, c_bh, *_ = orc.cumulative_energy_select(P, np.broadcast_to(taus[0], (B, H)))
+    assert np.array_equal(m_h, m_bh) and np.array_equal(c_h, c_bh)
+
+
 # ------------------------------------------------------------------ attention
 
 def _sdpa64(Q, K, V, causal, scale):
