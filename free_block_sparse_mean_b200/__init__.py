@@ -174,19 +174,61 @@ def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan, lam
     return out
 
 
-def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float,
+def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau,
                      lam: Optional[float] = None, scale: Optional[float] = None, causal: bool = False,
-                     device="cuda") -> torch.Tensor:
+                     device="cuda", out: Optional[torch.Tensor] = None, chunks: Optional[int] = None) -> torch.Tensor:
     """End to end from host tensors: copy q, k, v to the GPU, plan + forward, copy O back.
 
-    Host inputs should be pinned for overlap; the result is a host bf16 tensor."""
+    Host inputs should be pinned, so the copies are asynchronous DMA. The result is
+    a host bf16 tensor in pinned memory (`out` if given, else one from torch's
+    caching pinned allocator), ready when this returns.
+
+    Heads are independent, so the call is pipelined over `chunks` groups of heads
+    (default: up to 4): group g's host-to-device copy, its plan + forward and its
+    device-to-host copy run on three streams, so the copies of one group overlap
+    the work of the others in both directions of the link. tau may be one value or
+    a per-head float32 tensor ([B, H] or [H]) on `device`."""
     dev = torch.device(device)
-    qd = q.to(dev, non_blocking=True)
-    kd = k.to(dev, non_blocking=True)
-    vd = v.to(dev, non_blocking=True)
-    plan = sparse_attn_plan(qd, kd, tau, scale, causal, with_idx=False)
-    od = sparse_attn_fwd(qd, kd, vd, plan, lam, scale, causal)
-    return od.to("cpu")
+    if q.shape != k.shape or q.shape != v.shape or q.dim() != 4:
+        raise ValueError("q, k, v must share the shape [B, H, N, d]")
+    B, H, N, d = q.shape
+    BH = B * H
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    elif out.shape != q.shape or out.dtype != q.dtype or out.device.type != "cpu":
+        raise ValueError("out must be a host bf16 tensor of q's shape")
+    if isinstance(tau, torch.Tensor):
+        tau = (tau.unsqueeze(0).expand(B, H) if tau.dim() == 1 else tau).reshape(BH)
+    nch = max(1, min(BH, chunks if chunks is not None else 4))
+    bounds = [BH * c // nch for c in range(nch + 1)]
+    flat = [x.reshape(BH, N, d) for x in (q, k, v, out)]
+    qd, kd, vd, od = (torch.empty((BH, N, d), dtype=q.dtype, device=dev) for _ in range(4))
+    main = torch.cuda.current_stream(dev)
+    h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    h2d.wait_stream(main)
+    d2h.wait_stream(main)
+    for c in range(nch):
+        lo, hi = bounds[c], bounds[c + 1]
+        if hi == lo:
+            continue
+        with torch.cuda.stream(h2d):
+            for dst, src in zip((qd, kd, vd), flat[:3]):
+                dst[lo:hi].copy_(src[lo:hi], non_blocking=True)
+            ready = torch.cuda.Event()
+            ready.record(h2d)
+        main.wait_event(ready)
+        view = lambda x: x[lo:hi].view(1, hi - lo, N, d)
+        t = tau[lo:hi].view(1, hi - lo) if isinstance(tau, torch.Tensor) else tau
+        plan = sparse_attn_plan(view(qd), view(kd), t, scale, causal, with_idx=False)
+        sparse_attn_fwd(view(qd), view(kd), view(vd), plan, lam, scale, causal, out=view(od))
+        done = torch.cuda.Event()
+        done.record(main)
+        d2h.wait_event(done)
+        with torch.cuda.stream(d2h):
+            flat[3][lo:hi].copy_(od[lo:hi], non_blocking=True)
+    main.wait_stream(d2h)
+    main.synchronize()
+    return out
 
 
 def sparse_attn_device_error(device=None) -> int:

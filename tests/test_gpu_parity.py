@@ -229,3 +229,23 @@ def test_per_head_tau_matches_oracle_and_flags_invalid_values():
     m2 = to_np(p2.mask)
     assert np.all(m2[0, 3] == 1) and np.all(m2[0, 7] == 1)
     assert np.array_equal(m2[0, 4], mask[0, 4])
+
+
+def test_end_to_end_from_pinned_host_buffers():
+    """sparse_attention (host in, host out, pipelined over head groups) returns
+    exactly what the device-side plan + forward return, for any number of groups
+    and for a per-head tau: heads are independent, so grouping changes nothing."""
+    w = wl.WORKLOADS["small"].with_(H=6)
+    q, k, v = wl.generate(w, seed=3, device=_dev())
+    ref = sa.sparse_attn_fwd(q, k, v, sa.sparse_attn_plan(q, k, 0.95), -12.0)
+    taus = torch.linspace(0.9, 0.97, w.H, dtype=torch.float32, device=_dev())
+    ref_t = sa.sparse_attn_fwd(q, k, v, sa.sparse_attn_plan(q, k, taus), -12.0)
+    torch.cuda.synchronize()
+    qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+    for chunks in (1, 4, 6):
+        o = sa.sparse_attention(qh, kh, vh, 0.95, -12.0, chunks=chunks)
+        assert o.device.type == "cpu" and o.is_pinned()
+        assert torch.equal(o, ref.cpu()), f"chunks={chunks}"
+    o_t = sa.sparse_attention(qh, kh, vh, taus, -12.0, chunks=4)
+    assert torch.equal(o_t, ref_t.cpu())
+    _no_device_error()
