@@ -94,6 +94,147 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   }
 }
 
+// Selection of one row by one warp (phase 2 of the score kernels): e_j = exp(L_j -
+// max) in place of the scores, the cut-off e* by an IEEE bit-pattern search (a
+// bisection, or 8-way with kEightWay), then the mask row, the ascending kept list,
+// count[bh*Nb + i], the MinHash sort key of the kept set (*sig_out) and its bitset
+// (brow, ceil(Nb/32) words) for the pairing. sig_out and brow may be null.
+template <bool kEightWay>
+static __device__ __forceinline__ void select_row(float* row, int Nb, int i, long long bh, float tau, int lane,
+                                                  uint8_t* __restrict__ mask, int* __restrict__ count,
+                                                  int* __restrict__ idx, unsigned long long* sig_out,
+                                                  uint32_t* brow) {
+  const unsigned FULL = 0xffffffffu;
+  const float LOG2E = 1.4426950408889634f;
+  float m = -INFINITY;
+  for (int j = lane; j < Nb; j += 32) m = fmaxf(m, row[j]);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
+  // e_j in place; the row max maps to exactly 1.
+  float tot = 0.f;
+  uint32_t kmax = 0;
+  for (int j = lane; j < Nb; j += 32) {
+    const float e = ex2((row[j] - m) * LOG2E);
+    row[j] = e;
+    tot += e;
+    kmax = max(kmax, __float_as_uint(e));
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    tot += __shfl_xor_sync(FULL, tot, o);
+    kmax = max(kmax, __shfl_xor_sync(FULL, kmax, o));
+  }
+  __syncwarp();
+  uint32_t K;          // key (bit pattern) of the cut-off value e*
+  int need_ties;       // how many ties at e* are kept (lowest indices first)
+  if (tau >= 1.f) {
+    K = 1u;            // every block with e_j > 0 (finite score) is kept
+    need_ties = 0x7fffffff;
+  } else {
+    const float T = tau * tot;
+    uint32_t lo = 0u, hi = kmax + 1u;   // S(lo) >= T > S(hi)
+    while (hi - lo > 1u) {
+      if constexpr (kEightWay) {
+        // 7 probes split [lo, hi) into 8 parts; the last one is above lo once hi - lo >= 2
+        const uint32_t span = hi - lo;
+        uint32_t pr[7];
+        float ps[7];
+#pragma unroll
+        for (int t = 0; t < 7; ++t) {
+          pr[t] = lo + static_cast<uint32_t>((static_cast<unsigned long long>(span) * (t + 1)) >> 3);
+          ps[t] = 0.f;
+        }
+        for (int j = lane; j < Nb; j += 32) {
+          const float e = row[j];
+          const uint32_t u = __float_as_uint(e);
+#pragma unroll
+          for (int t = 0; t < 7; ++t) ps[t] += (u >= pr[t]) ? e : 0.f;
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+#pragma unroll
+          for (int t = 0; t < 7; ++t) ps[t] += __shfl_xor_sync(FULL, ps[t], o);
+        }
+        uint32_t nlo = lo, nhi = hi;
+#pragma unroll
+        for (int t = 0; t < 7; ++t) {
+          if (ps[t] >= T) nlo = max(nlo, pr[t]);
+          else nhi = min(nhi, pr[t]);
+        }
+        lo = nlo;
+        hi = nhi;
+      } else {
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        float s = 0.f;
+        for (int j = lane; j < Nb; j += 32) {
+          const float e = row[j];
+          s += (__float_as_uint(e) >= mid) ? e : 0.f;
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(FULL, s, o);
+        if (s >= T) lo = mid; else hi = mid;
+      }
+    }
+    K = lo;
+    float sgt = 0.f;
+    int nties = 0;
+    for (int j = lane; j < Nb; j += 32) {
+      const uint32_t kj = __float_as_uint(row[j]);
+      sgt += (kj > K) ? row[j] : 0.f;
+      nties += (kj == K);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      sgt += __shfl_xor_sync(FULL, sgt, o);
+      nties += __shfl_xor_sync(FULL, nties, o);
+    }
+    const float eK = __uint_as_float(K);
+    float acc = sgt;
+    need_ties = 0;
+    do {
+      acc += eK;
+      ++need_ties;
+    } while (acc < T && need_ties < nties);
+  }
+  // emit mask, ascending idx, count
+  uint8_t* mrow = mask + (bh * Nb + i) * static_cast<long long>(Nb);
+  int* irow = idx ? idx + (bh * Nb + i) * static_cast<long long>(Nb) : nullptr;
+  uint32_t s1 = 0xffffffffu, s2 = 0xffffffffu;  // MinHash signatures of the kept set
+  int kept = 0, ties_seen = 0;
+  for (int jb = 0; jb < Nb; jb += 32) {
+    const int j = jb + lane;
+    uint32_t kj = 0u;
+    if (j < Nb) kj = __float_as_uint(row[j]);
+    const bool tie = (j < Nb) && (kj == K);
+    const unsigned tb = __ballot_sync(FULL, tie);
+    const int my_tie_rank = ties_seen + __popc(tb & ((1u << lane) - 1u));
+    const bool keep = (j < Nb) && (kj > K || (tie && my_tie_rank < need_ties));
+    ties_seen += __popc(tb);
+    const unsigned kb = __ballot_sync(FULL, keep);
+    if (j < Nb) mrow[j] = keep ? 1 : 0;
+    if (irow && keep) irow[kept + __popc(kb & ((1u << lane) - 1u))] = j;
+    if (brow && lane == 0) brow[jb >> 5] = kb;
+    if (keep) {
+      s1 = min(s1, mix32(static_cast<uint32_t>(j) ^ 0x9e3779b9u));
+      s2 = min(s2, mix32(static_cast<uint32_t>(j) + 0x7f4a7c15u));
+    }
+    kept += __popc(kb);
+  }
+  if (sig_out) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      s1 = min(s1, __shfl_xor_sync(FULL, s1, o));
+      s2 = min(s2, __shfl_xor_sync(FULL, s2, o));
+    }
+  }
+  if (lane == 0) {
+    count[bh * Nb + i] = kept;
+    if (sig_out)
+      *sig_out = (static_cast<unsigned long long>(s1) << 32) | (static_cast<unsigned long long>(s2 & 0xffffu) << 16) |
+                 static_cast<unsigned long long>(i);
+  }
+}
+
 // ----------------------------------------------------------------------------
 // Pooled scores + selection. One CTA = R query blocks of one head. tau is the
 // recall threshold of every head, or tau_bh[b*H + h] per head when tau_bh is given.
@@ -262,140 +403,11 @@ __global__ void __launch_bounds__(NT) score_select_kernel(const float* __restric
     }
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const unsigned FULL = 0xffffffffu;
-  const float LOG2E = 1.4426950408889634f;
   for (int r = warp; r < R; r += NT / 32) {
     const int i = i0 + r;
     if (i >= Nb) break;
-    float* row = L + r * ldL;
-    float m = -INFINITY;
-    for (int j = lane; j < Nb; j += 32) m = fmaxf(m, row[j]);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
-    // e_j in place; the row max maps to exactly 1.
-    float tot = 0.f;
-    uint32_t kmax = 0;
-    for (int j = lane; j < Nb; j += 32) {
-      const float e = ex2((row[j] - m) * LOG2E);
-      row[j] = e;
-      tot += e;
-      kmax = max(kmax, __float_as_uint(e));
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-      tot += __shfl_xor_sync(FULL, tot, o);
-      kmax = max(kmax, __shfl_xor_sync(FULL, kmax, o));
-    }
-    __syncwarp();
-    uint32_t K;          // key (bit pattern) of the cut-off value e*
-    int need_ties;       // how many ties at e* are kept (lowest indices first)
-    if (tau >= 1.f) {
-      K = 1u;            // every block with e_j > 0 (finite score) is kept
-      need_ties = 0x7fffffff;
-    } else {
-      const float T = tau * tot;
-      uint32_t lo = 0u, hi = kmax + 1u;   // S(lo) >= T > S(hi)
-      while (hi - lo > 1u) {
-        if constexpr (kSmall) {
-          // 7 probes split [lo, hi) into 8 parts; the last one is above lo once hi - lo >= 2
-          const uint32_t span = hi - lo;
-          uint32_t pr[7];
-          float ps[7];
-#pragma unroll
-          for (int t = 0; t < 7; ++t) {
-            pr[t] = lo + static_cast<uint32_t>((static_cast<unsigned long long>(span) * (t + 1)) >> 3);
-            ps[t] = 0.f;
-          }
-          for (int j = lane; j < Nb; j += 32) {
-            const float e = row[j];
-            const uint32_t u = __float_as_uint(e);
-#pragma unroll
-            for (int t = 0; t < 7; ++t) ps[t] += (u >= pr[t]) ? e : 0.f;
-          }
-#pragma unroll
-          for (int o = 16; o; o >>= 1) {
-#pragma unroll
-            for (int t = 0; t < 7; ++t) ps[t] += __shfl_xor_sync(FULL, ps[t], o);
-          }
-          uint32_t nlo = lo, nhi = hi;
-#pragma unroll
-          for (int t = 0; t < 7; ++t) {
-            if (ps[t] >= T) nlo = max(nlo, pr[t]);
-            else nhi = min(nhi, pr[t]);
-          }
-          lo = nlo;
-          hi = nhi;
-        } else {
-          const uint32_t mid = lo + ((hi - lo) >> 1);
-          float s = 0.f;
-          for (int j = lane; j < Nb; j += 32) {
-            const float e = row[j];
-            s += (__float_as_uint(e) >= mid) ? e : 0.f;
-          }
-#pragma unroll
-          for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(FULL, s, o);
-          if (s >= T) lo = mid; else hi = mid;
-        }
-      }
-      K = lo;
-      float sgt = 0.f;
-      int nties = 0;
-      for (int j = lane; j < Nb; j += 32) {
-        const uint32_t kj = __float_as_uint(row[j]);
-        sgt += (kj > K) ? row[j] : 0.f;
-        nties += (kj == K);
-      }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) {
-        sgt += __shfl_xor_sync(FULL, sgt, o);
-        nties += __shfl_xor_sync(FULL, nties, o);
-      }
-      const float eK = __uint_as_float(K);
-      float acc = sgt;
-      need_ties = 0;
-      do {
-        acc += eK;
-        ++need_ties;
-      } while (acc < T && need_ties < nties);
-    }
-    // emit mask, ascending idx, count
-    uint8_t* mrow = mask + (bh * Nb + i) * static_cast<long long>(Nb);
-    int* irow = idx ? idx + (bh * Nb + i) * static_cast<long long>(Nb) : nullptr;
-    uint32_t* brow = bits ? bits + (bh * Nb + i) * static_cast<long long>((Nb + 31) / 32) : nullptr;
-    uint32_t s1 = 0xffffffffu, s2 = 0xffffffffu;  // MinHash signatures of the kept set
-    int kept = 0, ties_seen = 0;
-    for (int jb = 0; jb < Nb; jb += 32) {
-      const int j = jb + lane;
-      uint32_t kj = 0u;
-      if (j < Nb) kj = __float_as_uint(row[j]);
-      const bool tie = (j < Nb) && (kj == K);
-      const unsigned tb = __ballot_sync(FULL, tie);
-      const int my_tie_rank = ties_seen + __popc(tb & ((1u << lane) - 1u));
-      const bool keep = (j < Nb) && (kj > K || (tie && my_tie_rank < need_ties));
-      ties_seen += __popc(tb);
-      const unsigned kb = __ballot_sync(FULL, keep);
-      if (j < Nb) mrow[j] = keep ? 1 : 0;
-      if (irow && keep) irow[kept + __popc(kb & ((1u << lane) - 1u))] = j;
-      if (brow && lane == 0) brow[jb >> 5] = kb;
-      if (keep) {
-        s1 = min(s1, mix32(static_cast<uint32_t>(j) ^ 0x9e3779b9u));
-        s2 = min(s2, mix32(static_cast<uint32_t>(j) + 0x7f4a7c15u));
-      }
-      kept += __popc(kb);
-    }
-    if (sig) {
-#pragma unroll
-      for (int o = 16; o; o >>= 1) {
-        s1 = min(s1, __shfl_xor_sync(FULL, s1, o));
-        s2 = min(s2, __shfl_xor_sync(FULL, s2, o));
-      }
-    }
-    if (lane == 0) {
-      count[bh * Nb + i] = kept;
-      if (sig)
-        sig[bh * Nb + i] = (static_cast<unsigned long long>(s1) << 32) |
-                           (static_cast<unsigned long long>(s2 & 0xffffu) << 16) | static_cast<unsigned long long>(i);
-    }
+    select_row<kSmall>(L + r * ldL, Nb, i, bh, tau, lane, mask, count, idx, sig ? sig + bh * Nb + i : nullptr,
+                       bits ? bits + (bh * Nb + i) * static_cast<long long>((Nb + 31) / 32) : nullptr);
   }
 }
 
@@ -491,17 +503,19 @@ static __device__ int block_exclusive_scan(int v, int* sbuf, int* total) {
 // group_start + r * group_size + u. The CTAs running at one time then take the
 // longest tiles of every head of the group first, while the group's K and V
 // (chosen by the host to fit in L2) stay resident.
-static __global__ void __launch_bounds__(1024) pair_order_kernel(const unsigned long long* __restrict__ sig,
-                                                                 const uint32_t* __restrict__ bits_g,
-                                                                 const int* __restrict__ count, int Nb,
-                                                                 int Tq, int G, int* __restrict__ work) {
-  extern __shared__ __align__(16) unsigned char psm[];
+// Pairs and orders the query blocks of head bh (see above); called by every
+// thread of the CTA. keys: shared memory for P 64-bit keys whose first Nb entries
+// hold the blocks' MinHash sort keys; bits_rows: the kept-set bitsets, row-major
+// [Nb][ceil(Nb/32)], in global or shared memory; psm: the rest of the shared
+// memory (pair_order_smem_bytes minus the keys). BH heads in all.
+static __device__ void pair_and_order(unsigned long long* keys, const uint32_t* bits_rows,
+                                      const int* __restrict__ count, int Nb, int Tq, int G, long long bh,
+                                      long long BH, int* __restrict__ work, unsigned char* psm) {
   const int P = 1 << (32 - __clz(max(Nb, 2) - 1));   // next power of two >= Nb
   const int P2 = 1 << (32 - __clz(max(Tq, 2) - 1));
   const bool match = Nb <= kPairMatchMaxNb;
   const int W = (Nb + 31) / 32;                       // bitset words per row
-  unsigned long long* keys = reinterpret_cast<unsigned long long*>(psm);       // [P]
-  unsigned long long* keys2 = keys + P;                                          // [P2]
+  unsigned long long* keys2 = reinterpret_cast<unsigned long long*>(psm);      // [P2]
   int* pa = reinterpret_cast<int*>(keys2 + P2);                                  // [Tq]
   int* pb = pa + Tq;                                                             // [Tq]
   int* order = pb + Tq;                                                          // [Nb] position -> block
@@ -510,14 +524,10 @@ static __global__ void __launch_bounds__(1024) pair_order_kernel(const unsigned 
   int* partner = best + Nb;                                                      // [Nb] -1 while unpaired
   int* sbuf = partner + Nb;                                                      // [34] scan scratch
   uint32_t* bitsT = reinterpret_cast<uint32_t*>(sbuf + 34);                     // [W][Nb] by position (match only)
-  const long long bh = blockIdx.x;
   const int* cnt = count + bh * Nb;
 
-  // 1. MinHash keys (from the selection kernel); sort
-  for (int i = threadIdx.x; i < Nb; i += blockDim.x) {
-    keys[i] = sig[bh * Nb + i];
-    partner[i] = -1;
-  }
+  // 1. sort the MinHash keys
+  for (int i = threadIdx.x; i < Nb; i += blockDim.x) partner[i] = -1;
   for (int i = Nb + threadIdx.x; i < P; i += blockDim.x) keys[i] = ~0ull;
   __syncthreads();
   block_bitonic_sort(keys, P);
@@ -532,10 +542,9 @@ static __global__ void __launch_bounds__(1024) pair_order_kernel(const unsigned 
   if (match) {
     // kept-set bitsets, word-major by sorted position: neighbouring candidates are
     // neighbouring addresses
-    const uint32_t* src = bits_g + bh * static_cast<long long>(Nb) * W;
     for (int x = threadIdx.x; x < Nb * W; x += blockDim.x) {
       const int p = x / W, w = x - p * W;
-      bitsT[w * Nb + p] = src[static_cast<long long>(order[p]) * W + w];
+      bitsT[w * Nb + p] = bits_rows[static_cast<long long>(order[p]) * W + w];
     }
     __syncthreads();
     // one warp per alive position, one lane per candidate (the 16 alive positions
@@ -632,7 +641,7 @@ static __global__ void __launch_bounds__(1024) pair_order_kernel(const unsigned 
   // 3. longest first, then write the global query-block ids
   block_bitonic_sort(keys2, P2);
   const long long g0 = (bh / G) * G;                                  // first head of the group
-  const long long gsize = min(static_cast<long long>(G), static_cast<long long>(gridDim.x) - g0);
+  const long long gsize = min(static_cast<long long>(G), BH - g0);
   const long long u = bh - g0;
   for (int r = threadIdx.x; r < Tq; r += blockDim.x) {
     const int p = static_cast<int>(keys2[r] & 0xffffffffu);
@@ -641,6 +650,20 @@ static __global__ void __launch_bounds__(1024) pair_order_kernel(const unsigned 
     work[2 * pos] = static_cast<int>(bh * Nb + a);
     work[2 * pos + 1] = b >= 0 ? static_cast<int>(bh * Nb + b) : -1;
   }
+}
+
+// One CTA per head: MinHash keys and bitsets from the selection kernel.
+static __global__ void __launch_bounds__(1024) pair_order_kernel(const unsigned long long* __restrict__ sig,
+                                                                 const uint32_t* __restrict__ bits_g,
+                                                                 const int* __restrict__ count, int Nb,
+                                                                 int Tq, int G, int* __restrict__ work) {
+  extern __shared__ __align__(16) unsigned char psm[];
+  const int P = 1 << (32 - __clz(max(Nb, 2) - 1));
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(psm);
+  const long long bh = blockIdx.x;
+  for (int i = threadIdx.x; i < Nb; i += blockDim.x) keys[i] = sig[bh * Nb + i];
+  pair_and_order(keys, bits_g + bh * static_cast<long long>(Nb) * ((Nb + 31) / 32), count, Nb, Tq, G, bh,
+                 gridDim.x, work, psm + P * sizeof(unsigned long long));
 }
 
 // Shared memory of pair_order_kernel for Nb blocks per head.
