@@ -375,9 +375,11 @@ def run_ours(args, w, world, rank, local, pg):
     e2e = None
     if not args.no_e2e:
         qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
-        for _ in range(2):
-            sa.sparse_attention(qh, kh, vh, args.tau, lam, None, w.causal, device=dev)
-        torch.cuda.synchronize()
+        # warm-up calls exactly like the timed ones, so that the caching pinned
+        # allocator holds the output blocks the timed calls cycle through
+        for _ in range(max(3, args.warmup)):
+            o_host = sa.sparse_attention(qh, kh, vh, args.tau, lam, None, w.causal, device=dev)
+            torch.cuda.synchronize()
         barrier(pg, dev)
         t = []
         for _ in range(max(3, min(args.steps, 10))):

@@ -174,6 +174,18 @@ def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan, lam
     return out
 
 
+_COPY_STREAMS = {}
+
+
+def _copy_streams(dev: torch.device):
+    """The two copy streams of `sparse_attention` on a device (host-to-device and
+    device-to-host), created once per device and reused by every call."""
+    idx = dev.index if dev.index is not None else torch.cuda.current_device()
+    if idx not in _COPY_STREAMS:
+        _COPY_STREAMS[idx] = (torch.cuda.Stream(idx), torch.cuda.Stream(idx))
+    return _COPY_STREAMS[idx]
+
+
 def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau,
                      lam: Optional[float] = None, scale: Optional[float] = None, causal: bool = False,
                      device="cuda", out: Optional[torch.Tensor] = None, chunks: Optional[int] = None) -> torch.Tensor:
@@ -204,7 +216,7 @@ def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau,
     flat = [x.reshape(BH, N, d) for x in (q, k, v, out)]
     qd, kd, vd, od = (torch.empty((BH, N, d), dtype=q.dtype, device=dev) for _ in range(4))
     main = torch.cuda.current_stream(dev)
-    h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    h2d, d2h = _copy_streams(dev)
     h2d.wait_stream(main)
     d2h.wait_stream(main)
     for c in range(nch):
