@@ -20,7 +20,7 @@
 //
 // Roles (192 threads): warp 0 builds the union list, then one of its threads
 // loads V and issues the P.V MMAs; warp 1 owns TMEM and one of its threads loads
-// Q and K and issues the S MMAs (TMA, K and V as one 4-D box per 64-row block,
+// Q (at once, while the list is built) and K and issues the S MMAs (TMA, K and V as one 4-D box per 64-row block,
 // since TMA issue cost is per instruction); warps 2..5 run the softmax (thread =
 // row; warp w reaches TMEM lanes 32*(w%4) .. 32*(w%4)+31), the O correction and
 // the epilogue. The issue of a tcgen05.mma that accumulates into the result of
@@ -173,7 +173,6 @@ __global__ void __launch_bounds__(192, 2)
       mbar_init(&vfull[s], 1);
       mbar_init(&vempty[s], 1);
     }
-    mbar_init(q_full, 1);
     mbar_init(s_full, 1);
     mbar_init(s_free, 4);
     mbar_init(&p_full[0], 4);
@@ -190,7 +189,20 @@ __global__ void __launch_bounds__(192, 2)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
+      // Q rows of the two query blocks into rows 0..63 / 64..127 of the tile, issued
+      // now so that the load overlaps warp 0's build of the union list
+      mbar_init(q_full, 1);
+      fence_mbar_init();
+      mbar_expect_tx(q_full, (qb1 >= 0 ? 2 : 1) * C::kKVBytes);
+#pragma unroll
+      for (int c = 0; c < C::kChunks; ++c) {
+        tma_load_3d(sQ + c * C::kQChunkBytes, &tmQ, c * 64, qb0 * kBlock, static_cast<int>(bh), q_full);
+        if (qb1 >= 0)
+          tma_load_3d(sQ + c * C::kQChunkBytes + C::kKVChunkBytes, &tmQ, c * 64, qb1 * kBlock,
+                      static_cast<int>(bh), q_full);
+      }
     }
+    __syncwarp();
     tmem_alloc(tmem_holder, C::kTmemCols);
   }
   if (warp == 0) {
@@ -281,15 +293,6 @@ __global__ void __launch_bounds__(192, 2)
   } else if (warp == 1) {
     // ------------------------------------------------------------ Q, K producer, S issuer
     if (lane == 0 && n > 0) {
-      // Q rows of the two query blocks into rows 0..63 / 64..127 of the tile
-      mbar_expect_tx(q_full, (qb1 >= 0 ? 2 : 1) * C::kKVBytes);
-#pragma unroll
-      for (int c = 0; c < C::kChunks; ++c) {
-        tma_load_3d(sQ + c * C::kQChunkBytes, &tmQ, c * 64, qb0 * kBlock, static_cast<int>(bh), q_full);
-        if (qb1 >= 0)
-          tma_load_3d(sQ + c * C::kQChunkBytes + C::kKVChunkBytes, &tmQ, c * 64, qb1 * kBlock,
-                      static_cast<int>(bh), q_full);
-      }
       auto load_k = [&](int k) {
         const int s = k % C::STK;
         const int j = static_cast<int>(lst[k] & kListJMask);
@@ -329,6 +332,8 @@ __global__ void __launch_bounds__(192, 2)
       for (int kk = max(0, nk - C::STK); kk < nk; ++kk)
         mbar_wait_drain(&kfull[kk % C::STK], static_cast<uint32_t>(kk / C::STK) & 1u);
       if (stats) atomicAdd(&stats[2], static_cast<unsigned long long>(n));
+    } else if (lane == 0) {
+      mbar_wait_drain(q_full, 0u);                // no entry: the Q load still lands first
     }
   } else if (warp >= 2) {
     // ------------------------------------------------------------ softmax warps
