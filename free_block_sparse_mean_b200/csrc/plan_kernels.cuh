@@ -94,6 +94,131 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   }
 }
 
+// Ascending bitonic sort of 64 64-bit keys held two per lane by one warp: lane l
+// holds elements 2l (v[0]) and 2l+1 (v[1]). Stages with partner distance 1 stay in
+// the lane; longer ones exchange with lane l ^ (distance / 2).
+static __device__ __forceinline__ void warp_bitonic_sort64(unsigned long long (&v)[2], int lane) {
+#pragma unroll
+  for (int k = 2; k <= 64; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j == 1) {
+        const bool up = ((2 * lane) & k) == 0;
+        const unsigned long long a = v[0], b = v[1];
+        v[0] = up ? min(a, b) : max(a, b);
+        v[1] = up ? max(a, b) : min(a, b);
+      } else {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int i = 2 * lane + h;
+          const unsigned long long o = __shfl_xor_sync(0xffffffffu, v[h], j >> 1);
+          const bool up = (i & k) == 0, lower = (i & j) == 0;
+          v[h] = (lower == up) ? min(v[h], o) : max(v[h], o);
+        }
+      }
+    }
+  }
+}
+
+// In-place ascending sort of n64 <= 64 (a power of two) 64-bit keys in shared
+// memory by one warp (the caller synchronises afterwards).
+static __device__ void warp_sort_keys(unsigned long long* keys, int n64, int lane) {
+  unsigned long long v[2];
+  v[0] = (2 * lane < n64) ? keys[2 * lane] : ~0ull;
+  v[1] = (2 * lane + 1 < n64) ? keys[2 * lane + 1] : ~0ull;
+  warp_bitonic_sort64(v, lane);
+  if (2 * lane < n64) keys[2 * lane] = v[0];
+  if (2 * lane + 1 < n64) keys[2 * lane + 1] = v[1];
+}
+
+// Selection of one row of at most 64 blocks by one warp, the sorted-prefix rule
+// itself: e_j = exp(L_j - max) sorted descending (ties: lower j first), prefix sums
+// in that order, and the kept set is the shortest prefix whose sum reaches tau times
+// the total (every e_j > 0 when tau >= 1). Same outputs as select_row.
+static __device__ __forceinline__ void select_row_sorted64(const float* row, int Nb, int i, long long bh,
+                                                           float tau, int lane, uint8_t* __restrict__ mask,
+                                                           int* __restrict__ count, int* __restrict__ idx,
+                                                           unsigned long long* sig_out, uint32_t* brow) {
+  const unsigned FULL = 0xffffffffu;
+  const float LOG2E = 1.4426950408889634f;
+  const int j0 = 2 * lane, j1 = 2 * lane + 1;
+  const float x0 = (j0 < Nb) ? row[j0] : -INFINITY, x1 = (j1 < Nb) ? row[j1] : -INFINITY;
+  float m = fmaxf(x0, x1);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
+  // keys sorted ascending = e descending, then j ascending: ~((e bits << 32) | (0xffff - j))
+  auto key = [&](float x, int j) -> unsigned long long {
+    const float e = (j < Nb) ? ex2((x - m) * LOG2E) : 0.f;
+    return ~((static_cast<unsigned long long>(__float_as_uint(e)) << 32) | static_cast<uint32_t>(0xffff - j));
+  };
+  unsigned long long v[2] = {key(x0, j0), key(x1, j1)};
+  warp_bitonic_sort64(v, lane);
+  // sorted positions 2*lane, 2*lane+1: their e and block index
+  const unsigned long long u0 = ~v[0], u1 = ~v[1];
+  const float e0 = __uint_as_float(static_cast<uint32_t>(u0 >> 32));
+  const float e1 = __uint_as_float(static_cast<uint32_t>(u1 >> 32));
+  const int s0 = 0xffff - static_cast<int>(u0 & 0xffffu), s1 = 0xffff - static_cast<int>(u1 & 0xffffu);
+  // inclusive prefix sums in sorted order
+  const float pair = e0 + e1;
+  float inc = pair;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float y = __shfl_up_sync(FULL, inc, o);
+    if (lane >= o) inc += y;
+  }
+  const float c1 = inc, c0 = inc - pair + e0;
+  const float total = __shfl_sync(FULL, inc, 31);
+  bool k0, k1;
+  if (tau >= 1.f) {
+    k0 = e0 > 0.f;
+    k1 = e1 > 0.f;
+  } else {
+    const float T = tau * total;
+    const unsigned b0 = __ballot_sync(FULL, c0 >= T), b1 = __ballot_sync(FULL, c1 >= T);
+    const int r0 = b0 ? 2 * (__ffs(b0) - 1) : 1 << 30, r1 = b1 ? 2 * (__ffs(b1) - 1) + 1 : 1 << 30;
+    const int rstar = min(r0, r1);                  // last kept sorted position
+    k0 = 2 * lane <= rstar;
+    k1 = 2 * lane + 1 <= rstar;
+  }
+  unsigned long long kept = (k0 ? 1ull << s0 : 0ull) | (k1 ? 1ull << s1 : 0ull);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) kept |= __shfl_xor_sync(FULL, kept, o);
+  // emit mask, ascending idx, count, MinHash key and bitset
+  uint8_t* mrow = mask + (bh * Nb + i) * static_cast<long long>(Nb);
+  int* irow = idx ? idx + (bh * Nb + i) * static_cast<long long>(Nb) : nullptr;
+  uint32_t h1 = 0xffffffffu, h2 = 0xffffffffu;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int j = 32 * half + lane;
+    if (j < Nb) {
+      const bool keep = (kept >> j) & 1ull;
+      mrow[j] = keep ? 1 : 0;
+      if (keep) {
+        if (irow) irow[__popcll(kept & ((1ull << j) - 1ull))] = j;
+        h1 = min(h1, mix32(static_cast<uint32_t>(j) ^ 0x9e3779b9u));
+        h2 = min(h2, mix32(static_cast<uint32_t>(j) + 0x7f4a7c15u));
+      }
+    }
+  }
+  if (sig_out) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      h1 = min(h1, __shfl_xor_sync(FULL, h1, o));
+      h2 = min(h2, __shfl_xor_sync(FULL, h2, o));
+    }
+  }
+  if (lane == 0) {
+    count[bh * Nb + i] = __popcll(kept);
+    if (brow) {
+      brow[0] = static_cast<uint32_t>(kept);
+      if (Nb > 32) brow[1] = static_cast<uint32_t>(kept >> 32);
+    }
+    if (sig_out)
+      *sig_out = (static_cast<unsigned long long>(h1) << 32) | (static_cast<unsigned long long>(h2 & 0xffffu) << 16) |
+                 static_cast<unsigned long long>(i);
+  }
+}
+
 // Selection of one row by one warp (phase 2 of the score kernels): e_j = exp(L_j -
 // max) in place of the scores, the cut-off e* by an IEEE bit-pattern search (a
 // bisection, or 8-way with kEightWay), then the mask row, the ascending kept list,
@@ -406,8 +531,12 @@ __global__ void __launch_bounds__(NT) score_select_kernel(const float* __restric
   for (int r = warp; r < R; r += NT / 32) {
     const int i = i0 + r;
     if (i >= Nb) break;
-    select_row<kSmall>(L + r * ldL, Nb, i, bh, tau, lane, mask, count, idx, sig ? sig + bh * Nb + i : nullptr,
-                       bits ? bits + (bh * Nb + i) * static_cast<long long>((Nb + 31) / 32) : nullptr);
+    uint32_t* brow = bits ? bits + (bh * Nb + i) * static_cast<long long>((Nb + 31) / 32) : nullptr;
+    unsigned long long* srow = sig ? sig + bh * Nb + i : nullptr;
+    if (kSmall && Nb <= 64)
+      select_row_sorted64(L + r * ldL, Nb, i, bh, tau, lane, mask, count, idx, srow, brow);
+    else
+      select_row<kSmall>(L + r * ldL, Nb, i, bh, tau, lane, mask, count, idx, srow, brow);
   }
 }
 
@@ -530,7 +659,12 @@ static __device__ void pair_and_order(unsigned long long* keys, const uint32_t* 
   for (int i = threadIdx.x; i < Nb; i += blockDim.x) partner[i] = -1;
   for (int i = Nb + threadIdx.x; i < P; i += blockDim.x) keys[i] = ~0ull;
   __syncthreads();
-  block_bitonic_sort(keys, P);
+  if (P <= 64) {
+    if (threadIdx.x < 32) warp_sort_keys(keys, P, threadIdx.x);
+    __syncthreads();
+  } else {
+    block_bitonic_sort(keys, P);
+  }
   for (int p = threadIdx.x; p < Nb; p += blockDim.x) {
     order[p] = static_cast<int>(keys[p] & 0xffffu);
     alive[p] = p;
@@ -639,7 +773,12 @@ static __device__ void pair_and_order(unsigned long long* keys, const uint32_t* 
   for (int p = Tq + threadIdx.x; p < P2; p += blockDim.x) keys2[p] = ~0ull;
   __syncthreads();
   // 3. longest first, then write the global query-block ids
-  block_bitonic_sort(keys2, P2);
+  if (P2 <= 64) {
+    if (threadIdx.x < 32) warp_sort_keys(keys2, P2, threadIdx.x);
+    __syncthreads();
+  } else {
+    block_bitonic_sort(keys2, P2);
+  }
   const long long g0 = (bh / G) * G;                                  // first head of the group
   const long long gsize = min(static_cast<long long>(G), BH - g0);
   const long long u = bh - g0;
