@@ -599,7 +599,9 @@ static __device__ void block_bitonic_sort(unsigned long long* keys, int n64) {
 
 // Exclusive prefix sum of v over the threads of the block (any multiple of 32
 // threads up to 1024); every thread must call it. *total receives the sum.
-// sbuf: 33 ints of shared memory.
+// sbuf: 33 ints of shared memory. Without kTrailingSync the caller must pass a
+// __syncthreads before sbuf is written again.
+template <bool kTrailingSync = true>
 static __device__ int block_exclusive_scan(int v, int* sbuf, int* total) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   int x = v;
@@ -623,7 +625,7 @@ static __device__ int block_exclusive_scan(int v, int* sbuf, int* total) {
   __syncthreads();
   const int excl = x - v + (warp > 0 ? sbuf[warp - 1] : 0);
   *total = sbuf[32];
-  __syncthreads();                            // sbuf may be reused right after
+  if (kTrailingSync) __syncthreads();         // sbuf may be reused right after
   return excl;
 }
 
@@ -702,31 +704,29 @@ static __device__ void pair_and_order(unsigned long long* keys, const uint32_t* 
             sc += __popc(x & y) - __popc(x ^ y);
           }
         }
-        // warp argmax of (score, -distance, -offset): ties to the nearer, then the earlier
-        int bs = sc, bd = abs(d), bdd = d, bp = cpos;
+        // warp argmax of (score, -distance, -offset): ties to the nearer, then the
+        // earlier. One 64-bit key per lane (score + 4096 in the high word, distinct
+        // offsets below it, the candidate in the low bits); 0 = no candidate.
+        unsigned long long kb = 0ull;
+        if (ok)
+          kb = (static_cast<unsigned long long>(sc + 4096) << 32) |
+               (static_cast<unsigned long long>(16 - abs(d)) << 24) |
+               (static_cast<unsigned long long>(16 - d) << 16) | static_cast<unsigned long long>(cpos);
 #pragma unroll
-        for (int o = 16; o; o >>= 1) {
-          const int os = __shfl_xor_sync(0xffffffffu, bs, o), od = __shfl_xor_sync(0xffffffffu, bd, o);
-          const int odd = __shfl_xor_sync(0xffffffffu, bdd, o), op = __shfl_xor_sync(0xffffffffu, bp, o);
-          if (os > bs || (os == bs && (od < bd || (od == bd && odd < bdd)))) {
-            bs = os;
-            bd = od;
-            bdd = odd;
-            bp = op;
-          }
-        }
-        if (lane == 0) best[me] = (bs == INT_MIN) ? -1 : bp;
+        for (int o = 16; o; o >>= 1) kb = max(kb, __shfl_xor_sync(0xffffffffu, kb, o));
+        if (lane == 0) best[me] = kb ? static_cast<int>(kb & 0xffffu) : -1;
       }
       __syncthreads();
-      if (t < na) {
-        const int me = alive[t], c = best[me];
+      // mutual picks pair up; thread t alone reads and writes partner[alive[t]]
+      const int me = (t < na) ? alive[t] : -1;
+      if (me >= 0) {
+        const int c = best[me];
         if (c >= 0 && best[c] == me) partner[me] = c;
       }
-      __syncthreads();
-      const int me = (t < na) ? alive[t] : -1;
       const bool stay = me >= 0 && partner[me] < 0;
       int nna = 0;
-      const int at = block_exclusive_scan(stay ? 1 : 0, sbuf, &nna);
+      // no trailing barrier: sbuf is next written after this round's last barrier
+      const int at = block_exclusive_scan<false>(stay ? 1 : 0, sbuf, &nna);
       if (stay) alive[at] = me;
       __syncthreads();
       if (nna == na) break;
