@@ -69,18 +69,23 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  // every load of the thread first (all in flight at once), then the sums
+  constexpr int kPasses = kBlock / RPP;
+  uint4 u[kPasses];
 #pragma unroll
-  for (int p = 0; p < kBlock / RPP; ++p) {
+  for (int p = 0; p < kPasses; ++p) {
     const int r = r0 + p * RPP;
-    if (r < rows) {
-      const uint4 u = __ldg(reinterpret_cast<const uint4*>(src + static_cast<long long>(r) * D + c8));
-      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+    u[p] = (r < rows) ? __ldg(reinterpret_cast<const uint4*>(src + static_cast<long long>(r) * D + c8))
+                      : make_uint4(0u, 0u, 0u, 0u);
+  }
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(h[e]);
-        acc[2 * e] += f.x;
-        acc[2 * e + 1] += f.y;
-      }
+  for (int p = 0; p < kPasses; ++p) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u[p]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h[e]);
+      acc[2 * e] += f.x;
+      acc[2 * e + 1] += f.y;
     }
   }
 #pragma unroll
