@@ -32,8 +32,17 @@ Readings where the pages are silent (each is also listed in the design notes):
 
 Arithmetic is fp64 throughout; inputs are the exact values of the bf16 tensors.
 
+Quantized QK^T (SpargeAttn is "sparse and quantized"; the pages give no scheme,
+so this is a design, stated here and pinned by the tests): Q and K are quantized
+per (batch, head, 64-token block) to FP8 E4M3 with one scale per block,
+s = max|x| / 448 (448 = largest finite E4M3 value), codes = nearest E4M3 value
+of x * (448 / max|x|) computed in fp32 (the kernel's precision for this integer
+decision), ties to even, saturating. The scores are then the dequantized
+(code * s) products; V, P and the rest of the attention are unchanged.
+
 Entry points: block_mean_pool, pooled_logits, pooled_softmax,
-cumulative_energy_select, plan, attention_masked, attention_tiled, fwd.
+cumulative_energy_select, plan, attention_masked, attention_tiled, fwd,
+round_e4m3, quantize_blocks_e4m3, fwd_fp8qk.
 """
 from __future__ import annotations
 
@@ -267,3 +276,58 @@ def fwd(Q, K, V, mask, lam: Optional[float] = None, scale: Optional[float] = Non
     if lam is None or lam == -math.inf:
         return attention_masked(Q, K, V, mask, scale, causal, block, qblocks)
     return attention_tiled(Q, K, V, mask, lam, scale, causal, block, qblocks)
+
+
+# ----------------------------------------------------------------------------
+# FP8 E4M3 quantization of Q and K (see the module docstring)
+E4M3_MAX = 448.0
+
+
+def round_e4m3(x) -> np.ndarray:
+    """Nearest FP8 E4M3 value of x (fp64 result), ties to even, saturating at
+    +-448. E4M3: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits, no
+    infinities. In the binade [2^e, 2^(e+1)) (e >= -6) the representable values are
+    spaced 2^(e-3); below 2^-6 the subnormals are spaced 2^-9 as well."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    _, ex = np.frexp(np.maximum(a, 2.0 ** -6))      # a = m * 2^ex with m in [0.5, 1)
+    step = np.ldexp(1.0, ex - 1 - 3)
+    r = np.minimum(np.round(a / step) * step, E4M3_MAX)   # np.round: half to even
+    return np.copysign(r, x)
+
+
+def quantize_blocks_e4m3(X, block: int = BLOCK):
+    """Per (batch, head, block of 64 tokens) E4M3 quantization of X [B, H, N, d]:
+    amax = max |x| over the block, scale = amax / 448 and codes =
+    round_e4m3(x * (448 / amax)), both in fp32 (scale 1 and codes 0 for an
+    all-zero block). Returns (codes as fp64 values [B, H, N, d], scales fp64
+    [B, H, Nb]); code * scale is the dequantized value."""
+    X32 = np.asarray(as_f64(X), dtype=np.float32)
+    B, H, N, d = X32.shape
+    nb = n_blocks(N, block)
+    codes = np.zeros((B, H, N, d))
+    scales = np.ones((B, H, nb))
+    for i in range(nb):
+        sl = slice(i * block, min(N, (i + 1) * block))
+        amax = np.abs(X32[:, :, sl, :]).max(axis=(2, 3))
+        pos = amax > 0
+        inv = np.where(pos, np.float32(E4M3_MAX) / np.where(pos, amax, np.float32(1)), np.float32(0))
+        inv = inv.astype(np.float32)
+        y = (X32[:, :, sl, :] * inv[:, :, None, None]).astype(np.float32)
+        codes[:, :, sl, :] = round_e4m3(y)
+        scales[:, :, i] = np.where(pos, (amax / np.float32(E4M3_MAX)).astype(np.float32), 1.0)
+    return codes, scales
+
+
+def fwd_fp8qk(Q, K, V, mask, lam: Optional[float] = None, scale: Optional[float] = None,
+              causal: bool = False, block: int = BLOCK, qblocks=None):
+    """Stage 2 with quantized scores: fwd on the dequantized Q and K (codes times
+    their block scale), V as given. The mask comes from the unquantized plan."""
+    cq, sq = quantize_blocks_e4m3(Q, block)
+    ck, sk = quantize_blocks_e4m3(K, block)
+    N = cq.shape[2]
+    tok = np.minimum(np.arange(N) // block, sq.shape[2] - 1)
+    Qd = cq * sq[:, :, tok][..., None]
+    Kd = ck * sk[:, :, tok][..., None]
+    return fwd(Qd, Kd, V, mask, lam, scale, causal, block, qblocks)
+

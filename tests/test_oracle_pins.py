@@ -319,3 +319,60 @@ def test_bf16_inputs_are_upcast_exactly():
     y = orc.as_f64(x)
     assert y.dtype == np.float64
     assert np.array_equal(y, x.float().numpy().astype(np.float64))
+
+
+# ---------------------------------------------------------------- FP8 E4M3 quantization
+def test_round_e4m3_matches_the_format_and_torch():
+    """Hand values from the E4M3 definition (3 mantissa bits, ties to even,
+    subnormal spacing 2^-9, largest 448, saturating), then torch's own
+    float8_e4m3fn cast on 200k values spread over every binade."""
+    hand = {0.3: 0.3125, 1.0625: 1.0, 1.1875: 1.25, 2.0 ** -10: 0.0, 3 * 2.0 ** -10: 2.0 ** -8,
+            2.0 ** -9: 2.0 ** -9, 0.875 * 2.0 ** -6: 0.875 * 2.0 ** -6, 240.0: 240.0, 232.0: 224.0,
+            448.0: 448.0, 460.0: 448.0, 1.0e4: 448.0, -0.3: -0.3125, 0.0: 0.0}
+    for x, want in hand.items():
+        assert orc.round_e4m3(x) == want, x
+    r = _rng(11)
+    x = np.sign(r.standard_normal(200000)) * np.exp2(r.uniform(-14.0, 8.85, 200000))   # |x| < 462
+    t = torch.tensor(x, dtype=torch.float64).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(orc.round_e4m3(x), t)
+
+
+def test_quantize_blocks_e4m3_scales_and_error_bound():
+    r = _rng(12)
+    X = r.standard_normal((1, 2, 200, 16)) * np.array([1.0, 30.0])[None, :, None, None]
+    X[0, 1, 64:128] = 0.0                                    # an all-zero block
+    codes, scales = orc.quantize_blocks_e4m3(X)
+    assert scales.shape == (1, 2, 4)
+    assert scales[0, 1, 1] == 1.0 and np.all(codes[0, 1, 64:128] == 0)
+    for h in range(2):
+        for i in range(4):
+            blk = slice(64 * i, min(200, 64 * i + 64))
+            c = codes[0, h, blk]
+            if scales[0, h, i] != 1.0 or np.any(c):
+                assert np.abs(c).max() == 448.0                  # the block's absmax maps to 448
+            assert np.array_equal(c, orc.round_e4m3(c))          # every code is an E4M3 value
+            deq = c * scales[0, h, i]
+            err = np.abs(deq - X[0, h, blk])
+            # half a step of the code's binade (relative 2^-4), or of the subnormal spacing
+            bound = np.maximum(np.abs(X[0, h, blk]) * 2.0 ** -4, scales[0, h, i] * 2.0 ** -10) * 1.0001
+            assert np.all(err <= bound)
+
+
+def test_fwd_fp8qk_is_fwd_when_q_and_k_are_representable():
+    """Inputs that are E4M3 values times a power of two, each block holding a 448,
+    quantize exactly, so the quantized forward equals the plain one; on generic
+    inputs it stays within the quantization error."""
+    r = _rng(13)
+    grid = orc.round_e4m3(r.uniform(-448, 448, (1, 2, 192, 8)))
+    grid[:, :, ::64, 0] = 448.0
+    Q, K = grid * 2.0 ** -7, orc.round_e4m3(r.uniform(-448, 448, (1, 2, 192, 8)))
+    K[:, :, ::64, 0] = 448.0
+    K = K * 2.0 ** -8
+    V = r.standard_normal((1, 2, 192, 8))
+    mask = (r.uniform(size=(1, 2, 3, 3)) < 0.7).astype(np.uint8)
+    mask[..., 0, 0] = 1
+    for lam in (None, -2.0):
+        np.testing.assert_array_equal(orc.fwd_fp8qk(Q, K, V, mask, lam), orc.fwd(Q, K, V, mask, lam))
+    Qg, Kg = r.standard_normal((1, 2, 192, 8)), r.standard_normal((1, 2, 192, 8))
+    a, b = orc.fwd_fp8qk(Qg, Kg, V, mask), orc.fwd(Qg, Kg, V, mask)
+    assert 0 < np.abs(a - b).max() < 0.1
