@@ -73,6 +73,8 @@ class Plan:
                                 of each row (rest of the row undefined), or None
     work  int32 [2*num_tiles]   query-block pairs in execution order for sparse_attn_fwd
                                 (global ids (b*H+h)*Nb+i, second -1 if absent), or None
+    q8, k8          uint8 [B, H, N, d]  FP8 E4M3 codes of q and k (quantize=True), else None
+    qscale, kscale  float32 [B, H, Nb]  their per-block scales (quantize=True), else None
     """
     mask: torch.Tensor
     count: torch.Tensor
@@ -80,6 +82,10 @@ class Plan:
     work: Optional[torch.Tensor]
     tau: Union[float, torch.Tensor]   # one threshold, or one per (batch, head)
     causal: bool
+    q8: Optional[torch.Tensor] = None
+    k8: Optional[torch.Tensor] = None
+    qscale: Optional[torch.Tensor] = None
+    kscale: Optional[torch.Tensor] = None
 
 
 def sparse_attn_plan_workspace_size(B: int, H: int, N: int, d: int) -> int:
@@ -92,11 +98,14 @@ def sparse_attn_num_tiles(B: int, H: int, N: int, d: int) -> int:
 
 def sparse_attn_plan(q: torch.Tensor, k: torch.Tensor, tau, scale: Optional[float] = None,
                      causal: bool = False, *, with_idx: bool = True, with_work: bool = True,
-                     out: Optional[Plan] = None, workspace: Optional[torch.Tensor] = None) -> Plan:
+                     out: Optional[Plan] = None, workspace: Optional[torch.Tensor] = None,
+                     quantize: bool = False) -> Plan:
     """Stage 1: cumulative-energy block mask from mean-pooled q and k.
 
     tau is one recall threshold for every head (a float), or one per head: a float32
-    CUDA tensor of shape [B, H] or [H] on q's device (sparse_attn_plan_heads)."""
+    CUDA tensor of shape [B, H] or [H] on q's device (sparse_attn_plan_heads).
+    quantize=True (one tau, d = 128) also writes FP8 E4M3 copies of q and k with
+    per-block scales (sparse_attn_plan_q8) for sparse_attn_fwd(..., qk_fp8=True)."""
     lib = _lib.load()
     _check_qkv(q, k)
     B, H, N, d = q.shape
@@ -115,9 +124,23 @@ def sparse_attn_plan(q: torch.Tensor, k: torch.Tensor, tau, scale: Optional[floa
             tau=tau if isinstance(tau, torch.Tensor) else float(tau), causal=bool(causal))
     else:
         out.tau, out.causal = (tau if isinstance(tau, torch.Tensor) else float(tau)), bool(causal)
+    if quantize and out.q8 is None:
+        out.q8 = torch.empty((B, H, N, d), dtype=torch.uint8, device=dev)
+        out.k8 = torch.empty((B, H, N, d), dtype=torch.uint8, device=dev)
+        out.qscale = torch.empty((B, H, Nb), dtype=torch.float32, device=dev)
+        out.kscale = torch.empty((B, H, Nb), dtype=torch.float32, device=dev)
     ws_bytes = int(lib.sparse_attn_plan_workspace_size(s))
     if workspace is None or workspace.numel() < ws_bytes:
         workspace = torch.empty((max(ws_bytes, 256),), dtype=torch.uint8, device=dev)
+    if quantize:
+        if isinstance(tau, torch.Tensor):
+            raise ValueError("quantize=True takes one tau for every head")
+        st = lib.sparse_attn_plan_q8(_ptr(q), _ptr(k), s, float(tau), float(scale), int(bool(causal)),
+                                     _ptr(out.mask), _ptr(out.count), _ptr(out.idx), _ptr(out.work),
+                                     _ptr(out.q8), _ptr(out.k8), _ptr(out.qscale), _ptr(out.kscale),
+                                     _ptr(workspace), ws_bytes, _stream(dev))
+        _call("sparse_attn_plan_q8", st)
+        return out
     if isinstance(tau, torch.Tensor):
         if tau.dtype != torch.float32 or tau.device != dev:
             raise ValueError("a per-head tau must be a float32 tensor on q's device")
@@ -140,11 +163,14 @@ def sparse_attn_plan(q: torch.Tensor, k: torch.Tensor, tau, scale: Optional[floa
 
 def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan, lam: Optional[float] = None,
                     scale: Optional[float] = None, causal: Optional[bool] = None, *,
-                    out: Optional[torch.Tensor] = None, stats: Optional[torch.Tensor] = None) -> torch.Tensor:
+                    out: Optional[torch.Tensor] = None, stats: Optional[torch.Tensor] = None,
+                    qk_fp8: bool = False) -> torch.Tensor:
     """Stage 2: attention over the kept blocks with the lambda P.V filter.
 
     `plan` is a Plan or a uint8 mask [B, H, Nb, Nb]. lam=None turns the filter off.
-    `stats`, if given, is an int64 CUDA tensor of 4 entries (see the C header)."""
+    `stats`, if given, is an int64 CUDA tensor of 4 entries (see the C header).
+    qk_fp8=True takes the scores on the plan's FP8 copies of q and k
+    (sparse_attn_fwd_q8; the plan must come from sparse_attn_plan(quantize=True))."""
     lib = _lib.load()
     _check_qkv(q, k, v)
     B, H, N, d = q.shape
@@ -168,6 +194,14 @@ def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan, lam
         out = torch.empty_like(q)
     if stats is not None and (stats.dtype != torch.int64 or stats.numel() < 4 or stats.device != q.device):
         raise ValueError("stats must be an int64 tensor of >= 4 entries on q's device")
+    if qk_fp8:
+        if not isinstance(plan, Plan) or plan.q8 is None:
+            raise ValueError("qk_fp8=True needs a plan made with quantize=True")
+        st = lib.sparse_attn_fwd_q8(_ptr(plan.q8), _ptr(plan.k8), _ptr(plan.qscale), _ptr(plan.kscale), _ptr(v),
+                                    _shape(q), _ptr(mask), _ptr(work), lam_f, float(scale), int(causal),
+                                    _ptr(out), _ptr(stats), _stream(q.device))
+        _call("sparse_attn_fwd_q8", st)
+        return out
     st = lib.sparse_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _shape(q), _ptr(mask), _ptr(work), lam_f,
                              float(scale), int(causal), _ptr(out), _ptr(stats), _stream(q.device))
     _call("sparse_attn_fwd", st)

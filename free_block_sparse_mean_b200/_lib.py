@@ -29,6 +29,8 @@ EXPORTS = (
     "sparse_attn_status_string",
     "sparse_attn_device_error",
     "sparse_attn_plan_noalloc",
+    "sparse_attn_plan_q8",
+    "sparse_attn_fwd_q8",
     "sparse_attn_selftest_wait_timeout",
 )
 
@@ -80,6 +82,10 @@ def load(path: str = LIB_PATH):
     lib.sparse_attn_device_error.restype = i32
     lib.sparse_attn_plan_noalloc.argtypes = [vp, vp, SaShape, f32, f32, i32, vp, vp, vp, vp, vp]
     lib.sparse_attn_plan_noalloc.restype = i32
+    lib.sparse_attn_plan_q8.argtypes = [vp, vp, SaShape, f32, f32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.sparse_attn_plan_q8.restype = i32
+    lib.sparse_attn_fwd_q8.argtypes = [vp, vp, vp, vp, vp, SaShape, vp, vp, f32, f32, i32, vp, vp, vp]
+    lib.sparse_attn_fwd_q8.restype = i32
     lib.sparse_attn_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp]
     lib.sparse_attn_selftest_wait_timeout.restype = i32
     _lib = lib

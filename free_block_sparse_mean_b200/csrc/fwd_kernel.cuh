@@ -58,30 +58,38 @@
 
 namespace sa {
 
-template <int D>
+// kF8: Q and K arrive as FP8 E4M3 codes with one scale per 64-token block
+// (d = 128 only); S = Q K^T runs as tcgen05.mma kind::f8f6f4 and the two block
+// scales join the softmax scale. V, P and O are as in the bf16 kernel.
+template <int D, bool kF8 = false>
 struct FwdCfg {
+  static_assert(!kF8 || D == 128, "the FP8-score kernel is for d = 128");
   static constexpr int kRows = 128;                    // query rows per tile
   static constexpr int kThreads = 192;                 // 2 role warps + 4 softmax warps
-  static constexpr int kChunks = D / 64;               // 128-byte (64 x bf16) column chunks
-  static constexpr int STK = (D == 64) ? 4 : 2;        // K ring stages
+  static constexpr int kChunks = D / 64;               // 128-byte (64 x bf16) column chunks of V
+  static constexpr int kQKChunks = kF8 ? 1 : kChunks;  // 128-byte column chunks of a Q or K row
+  static constexpr int STK = (D == 64 || kF8) ? 4 : 2; // K ring stages
   static constexpr int STV = (D == 64) ? 4 : 2;        // V ring stages
   static constexpr int kQChunkBytes = kRows * 128;     // 16 KB
   static constexpr int kKVChunkBytes = kBlock * 128;   // 8 KB
-  static constexpr int kQBytes = kChunks * kQChunkBytes;
-  static constexpr int kKVBytes = kChunks * kKVChunkBytes;
+  static constexpr int kQBytes = kQKChunks * kQChunkBytes;
+  static constexpr int kKBytes = kQKChunks * kKVChunkBytes;   // one K stage (also one query block of Q)
+  static constexpr int kKVBytes = kChunks * kKVChunkBytes;    // one V stage
+  static constexpr int kSSteps = kF8 ? D / 32 : D / 16;       // K-steps of one S MMA group
   // shared-memory layout (offsets from a 1024-aligned base)
   static constexpr int oQ = 0;
   static constexpr int oK = oQ + kQBytes;
-  static constexpr int oV = oK + STK * kKVBytes;
+  static constexpr int oV = oK + STK * kKBytes;
   static constexpr int oBar = oV + STV * kKVBytes;     // mbarriers
   static constexpr int kNumBars = 2 * STK + 2 * STV + 8;
   static constexpr int oMisc = oBar + kNumBars * 8;    // small words (256 bytes)
   static constexpr int oList = oMisc + 256;
-  static constexpr int kSmemBytes = oList + kMaxNb * 2 + 1024;  // + alignment slack
+  static constexpr int oListScale = oList + kMaxNb * 2;                      // kF8: K block scale per entry
+  static constexpr int kSmemBytes = oListScale + (kF8 ? kMaxNb * 4 : 0) + 1024;  // + alignment slack
   // TMEM columns: S, two P buffers (bf16 pairs), the O accumulator
   static constexpr uint32_t kColS = 0, kColP0 = 64, kColP1 = 96, kColO = 128;
   static constexpr uint32_t kTmemCols = 256;
-  static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, false);
+  static constexpr uint32_t kIdescS = kF8 ? idesc_e4m3_f32(128, 64) : idesc_bf16_f32(128, 64, false);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
 };
 
@@ -112,14 +120,15 @@ __device__ __forceinline__ float softmax_exp64(const float (&s)[64], float scale
   return (r0 + r1) + (r2 + r3);
 }
 
-template <int D>
+template <int D, bool kF8>
 __global__ void __launch_bounds__(192, 2)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const uint8_t* __restrict__ mask,
                const int* __restrict__ work, __nv_bfloat16* __restrict__ O, int N, int Nb, int Tq,
                long long num_tiles, long long num_qblocks, float scale_log2, float lam_log2, int lam_on,
-               int causal, unsigned long long* __restrict__ stats) {
-  using C = FwdCfg<D>;
+               int causal, unsigned long long* __restrict__ stats, const float* __restrict__ qscale,
+               const float* __restrict__ kscale) {
+  using C = FwdCfg<D, kF8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base + C::oQ;
@@ -143,6 +152,7 @@ __global__ void __launch_bounds__(192, 2)
   volatile int* contrib = misc + 4;            // [2 parity][2 halves]: the half's P.V is needed
   volatile int* votes = misc + 8;              // [2 parity][4 softmax warps]: (k << 1) | pass
   uint16_t* lst = reinterpret_cast<uint16_t*>(base + C::oList);
+  float* lsk = reinterpret_cast<float*>(base + C::oListScale);   // kF8: K block scale of each entry
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (blockIdx.x >= num_tiles) return;
@@ -193,9 +203,9 @@ __global__ void __launch_bounds__(192, 2)
       // now so that the load overlaps warp 0's build of the union list
       mbar_init(q_full, 1);
       fence_mbar_init();
-      mbar_expect_tx(q_full, (qb1 >= 0 ? 2 : 1) * C::kKVBytes);
+      mbar_expect_tx(q_full, (qb1 >= 0 ? 2 : 1) * C::kKBytes);
 #pragma unroll
-      for (int c = 0; c < C::kChunks; ++c) {
+      for (int c = 0; c < C::kQKChunks; ++c) {
         tma_load_3d(sQ + c * C::kQChunkBytes, &tmQ, c * 64, qb0 * kBlock, static_cast<int>(bh), q_full);
         if (qb1 >= 0)
           tma_load_3d(sQ + c * C::kQChunkBytes + C::kKVChunkBytes, &tmQ, c * 64, qb1 * kBlock,
@@ -236,6 +246,10 @@ __global__ void __launch_bounds__(192, 2)
       }
     }
     if (lane == 0) *list_n = n;
+    if constexpr (kF8) {
+      __syncwarp();
+      for (int e = lane; e < n; e += 32) lsk[e] = kscale[bh * Nb + (lst[e] & kListJMask)];
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -296,8 +310,11 @@ __global__ void __launch_bounds__(192, 2)
       auto load_k = [&](int k) {
         const int s = k % C::STK;
         const int j = static_cast<int>(lst[k] & kListJMask);
-        mbar_expect_tx(&kfull[s], C::kKVBytes);
-        tma_load_4d(sK + s * C::kKVBytes, &tmK, 0, j * kBlock, 0, static_cast<int>(bh), &kfull[s]);
+        mbar_expect_tx(&kfull[s], C::kKBytes);
+        if constexpr (kF8)
+          tma_load_3d(sK + s * C::kKBytes, &tmK, 0, j * kBlock, static_cast<int>(bh), &kfull[s]);
+        else
+          tma_load_4d(sK + s * C::kKBytes, &tmK, 0, j * kBlock, 0, static_cast<int>(bh), &kfull[s]);
       };
       int nk = 0;                                 // K loads issued
       for (; nk < C::STK && nk < n; ++nk) load_k(nk);
@@ -311,11 +328,14 @@ __global__ void __launch_bounds__(192, 2)
         tc_fence_after();
         const uint32_t dS = tmem_base + C::kColS;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk & 3) * 32;  // 16 bf16 = 32 bytes inside the swizzle atom
+        for (int kk = 0; kk < C::kSSteps; ++kk) {
+          const uint32_t off = (kk & 3) * 32;  // 16 bf16 or 32 e4m3 = 32 bytes inside the swizzle atom
           const uint64_t ad = sdesc_sw128(sQa + (kk >> 2) * C::kQChunkBytes + off, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sKa + s * C::kKVBytes + (kk >> 2) * C::kKVChunkBytes + off, 16, 1024);
-          tc_mma_ss(dS, ad, bd, C::kIdescS, kk > 0 ? 1u : 0u);
+          const uint64_t bd = sdesc_sw128(sKa + s * C::kKBytes + (kk >> 2) * C::kKVChunkBytes + off, 16, 1024);
+          if constexpr (kF8)
+            tc_mma_ss_f8(dS, ad, bd, C::kIdescS, kk > 0 ? 1u : 0u);
+          else
+            tc_mma_ss(dS, ad, bd, C::kIdescS, kk > 0 ? 1u : 0u);
         }
         tc_commit(s_full);
         tc_commit(&kempty[s]);
@@ -347,6 +367,8 @@ __global__ void __launch_bounds__(192, 2)
     const uint32_t s_addr = tmem_base + lane_bits + C::kColS;
     const uint32_t o_addr = tmem_base + lane_bits + C::kColO;
     const bool writer = (wq & 1) == 0 && lane == 0;   // one per half: contrib, stats
+    // kF8: the scores are codes; this row's query-block scale joins the softmax scale
+    const float sqh = kF8 ? (myqb >= 0 ? qscale[bh * Nb + myqb] : 1.f) : 1.f;
     const unsigned FULL = 0xffffffffu;
     float m_true = -INFINITY, m_ref = -INFINITY, l = 0.f;
     unsigned long long kept_pairs = 0, skipped_pairs = 0;
@@ -374,6 +396,7 @@ __global__ void __launch_bounds__(192, 2)
       if (causal) ncol = min(ncol, static_cast<int>(max(qrow - kbase + 1, 0LL)));
       const bool warp_none = __all_sync(FULL, ncol == 0);
       const bool warp_full = __all_sync(FULL, ncol == kBlock);
+      const float sc = kF8 ? scale_log2 * sqh * lsk[k] : scale_log2;   // log2-domain scale of S(k)
       tmem_wait_ld();                             // S(k) is in s[]
       pin32(*reinterpret_cast<float(*)[32]>(&s[0]));
       pin32(*reinterpret_cast<float(*)[32]>(&s[32]));
@@ -398,7 +421,7 @@ __global__ void __launch_bounds__(192, 2)
 #pragma unroll
         for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], s[56 + u]);
         rmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
-               scale_log2;                        // -inf stays -inf (scale > 0)
+               sc;                                // -inf stays -inf (sc > 0)
       }
       bool wpass = true;
       if (lam_on) {
@@ -422,7 +445,7 @@ __global__ void __launch_bounds__(192, 2)
 #pragma unroll
         for (int c = 0; c < 32; ++c) pk[c] = 0u;
       } else {
-        psum = softmax_exp64(s, scale_log2, mref, pk);
+        psum = softmax_exp64(s, sc, mref, pk);
       }
       m_true = m_new;
       l = l * alpha + psum;

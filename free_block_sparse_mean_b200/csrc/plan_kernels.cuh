@@ -10,6 +10,8 @@
 
 #include <climits>
 
+#include <cuda_fp8.h>
+
 #include "sa_device.cuh"
 
 namespace sa {
@@ -50,14 +52,22 @@ static __device__ __forceinline__ uint32_t mix32(uint32_t x) {
 // thread loads 16-byte vectors (8 bf16) of a row; D/8 threads cover a row, so a
 // warp reads whole rows contiguously. Partial sums meet in shared memory.
 // HBM-bound: it is the one full pass over Q and K on the predictor side.
+// With Q8 (and K8, qs, ks) given, the same pass also quantizes the block to FP8
+// E4M3 for the quantized-score forward: scale = amax / 448 over the block, codes =
+// x * (448 / amax) rounded to nearest even and saturated (scale 1, codes 0 for an
+// all-zero block), [B,H,N,d] bytes and [B,H,Nb] fp32 scales.
 template <int D>
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ Q,
                                                    const __nv_bfloat16* __restrict__ K,
                                                    float* __restrict__ Qp, float* __restrict__ Kp,
-                                                   int N, int Nb) {
+                                                   int N, int Nb, uint8_t* __restrict__ Q8 = nullptr,
+                                                   uint8_t* __restrict__ K8 = nullptr,
+                                                   float* __restrict__ qs = nullptr,
+                                                   float* __restrict__ ks = nullptr) {
   constexpr int LPR = D / 8;          // threads per row
   constexpr int RPP = 256 / LPR;      // rows per pass
   __shared__ float part[RPP][D];
+  __shared__ float wmax[8];
   const long long g = blockIdx.x;     // (bh, i) flattened
   const long long bh = g / Nb;
   const int i = static_cast<int>(g - bh * Nb);
@@ -90,12 +100,51 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   }
 #pragma unroll
   for (int e = 0; e < 8; ++e) part[r0][c8 + e] = acc[e];
+  uint8_t* q8 = (Q8 == nullptr) ? nullptr : (blockIdx.y == 0 ? Q8 : K8);
+  float amax = 0.f;
+  if (q8) {
+    // largest |x| of the block (tail rows loaded as zeros)
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p) {
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u[p]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h[e]);
+        amax = fmax3(amax, fabsf(f.x), fabsf(f.y));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = amax;
+  }
   __syncthreads();
   if (threadIdx.x < D) {
     float s = 0.f;
 #pragma unroll
     for (int r = 0; r < RPP; ++r) s += part[r][threadIdx.x];
     dst[threadIdx.x] = s / static_cast<float>(rows);
+  }
+  if (q8) {
+    amax = fmax3(fmax3(wmax[0], wmax[1], wmax[2]), fmax3(wmax[3], wmax[4], wmax[5]), fmaxf(wmax[6], wmax[7]));
+    const float inv = amax > 0.f ? 448.f / amax : 0.f;
+    if (threadIdx.x == 0) (blockIdx.y == 0 ? qs : ks)[g] = amax > 0.f ? amax / 448.f : 1.f;
+    uint8_t* dst8 = q8 + (bh * N + static_cast<long long>(i) * kBlock) * D;
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p) {
+      const int r = r0 + p * RPP;
+      if (r < rows) {
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u[p]);
+        uint32_t w[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float2 f0 = __bfloat1622float2(h[2 * e]), f1 = __bfloat1622float2(h[2 * e + 1]);
+          const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(f0.x * inv, f0.y * inv), __NV_SATFINITE, __NV_E4M3);
+          const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(f1.x * inv, f1.y * inv), __NV_SATFINITE, __NV_E4M3);
+          w[e] = lo | (hi << 16);
+        }
+        *reinterpret_cast<uint2*>(dst8 + static_cast<long long>(r) * D + c8) = make_uint2(w[0], w[1]);
+      }
+    }
   }
 }
 

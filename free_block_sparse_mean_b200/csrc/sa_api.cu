@@ -78,6 +78,22 @@ bool make_block_map(CUtensorMap* map, const void* ptr, const sa_shape& s) {
   return r == CUDA_SUCCESS;
 }
 
+// FP8 codes [B*H, N, d] (d bytes per row) as a 3-D tensor {d, N, B*H}; box
+// {d = 128, 64 rows, 1}, 128B swizzle: one load per 64-row block.
+bool make_map8(CUtensorMap* map, const void* ptr, const sa_shape& s) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(s.d), static_cast<cuuint64_t>(s.N),
+                        static_cast<cuuint64_t>(s.B) * s.H};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(s.d), static_cast<cuuint64_t>(s.N) * s.d};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(s.d), 64u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <typename F>
 sa_status set_smem(F* kernel, int bytes) {
   // Per device: the attribute belongs to the current context.
@@ -91,7 +107,8 @@ sa_status set_smem(F* kernel, int bytes) {
 template <int D>
 sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau, const float* tau_bh,
                       float scale, int causal, uint8_t* mask, int32_t* count, int32_t* idx, int32_t* work,
-                      void* ws, cudaStream_t st) {
+                      void* ws, cudaStream_t st, uint8_t* Q8 = nullptr, uint8_t* K8 = nullptr,
+                      float* qscale = nullptr, float* kscale = nullptr) {
   const int Nb = static_cast<int>(num_blocks(s));
   const long long BH = static_cast<long long>(s.B) * s.H;
   const sa::PlanWorkspace L = sa::plan_workspace(BH, Nb, D);
@@ -101,7 +118,8 @@ sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau
   unsigned long long* sig = reinterpret_cast<unsigned long long*>(wsb + L.sig);
   uint32_t* bits = reinterpret_cast<uint32_t*>(wsb + L.bits);
   sa::pool_kernel<D><<<dim3(static_cast<unsigned>(BH * Nb), 2), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Qp, Kp, s.N, Nb);
+      static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Qp, Kp, s.N, Nb, Q8, K8, qscale,
+      kscale);
   if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
 
   // Small heads: 4 query blocks per CTA so the grid still fills the GPU.
@@ -136,26 +154,32 @@ sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau
   return SA_OK;
 }
 
-template <int D>
+template <int D, bool kF8 = false>
 sa_status launch_fwd(const sa_shape& s, const void* Q, const void* K, const void* V, const uint8_t* mask,
                      const int32_t* work, float lambda, float scale, int causal, void* O, int64_t* stats,
-                     cudaStream_t st) {
-  using Cfg = sa::FwdCfg<D>;
+                     cudaStream_t st, const float* qscale = nullptr, const float* kscale = nullptr) {
+  using Cfg = sa::FwdCfg<D, kF8>;
   const int Nb = static_cast<int>(num_blocks(s));
   const int Tq = (Nb + 1) / 2;
   const long long tiles = static_cast<long long>(s.B) * s.H * Tq;
   if (tiles > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, Q, s, 64) || !make_block_map(&mk, K, s) || !make_block_map(&mv, V, s)) return SA_ERR_CUDA;
+  if (kF8) {
+    if (!make_map8(&mq, Q, s) || !make_map8(&mk, K, s)) return SA_ERR_CUDA;
+  } else {
+    if (!make_map(&mq, Q, s, 64) || !make_block_map(&mk, K, s)) return SA_ERR_CUDA;
+  }
+  if (!make_block_map(&mv, V, s)) return SA_ERR_CUDA;
   if (stats && cudaMemsetAsync(stats, 0, 4 * sizeof(int64_t), st) != cudaSuccess) return SA_ERR_CUDA;
-  auto kern = sa::fwd_kernel<D>;
+  auto kern = sa::fwd_kernel<D, kF8>;
   if (set_smem(kern, Cfg::kSmemBytes) != SA_OK) return SA_ERR_CUDA;
   const float LOG2E = 1.4426950408889634f;
   const int lam_on = std::isinf(lambda) && lambda < 0 ? 0 : 1;
   kern<<<static_cast<unsigned>(tiles), Cfg::kThreads, Cfg::kSmemBytes, st>>>(
       mq, mk, mv, mask, work, static_cast<__nv_bfloat16*>(O), s.N, Nb, Tq, tiles,
       static_cast<long long>(s.B) * s.H * Nb, scale * LOG2E,
-      lam_on ? lambda * LOG2E : 0.f, lam_on, causal, reinterpret_cast<unsigned long long*>(stats));
+      lam_on ? lambda * LOG2E : 0.f, lam_on, causal, reinterpret_cast<unsigned long long*>(stats), qscale,
+      kscale);
   if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   return SA_OK;
 }
@@ -253,6 +277,44 @@ const char* sparse_attn_status_string(sa_status st) {
     case SA_ERR_DEVICE_CHECK: return "SA_ERR_DEVICE_CHECK: a device-side check fired";
   }
   return "unknown sa_status";
+}
+
+sa_status sparse_attn_plan_q8(const void* Q, const void* K, sa_shape s, float tau, float scale, int32_t causal,
+                              uint8_t* mask, int32_t* count, int32_t* idx, int32_t* work, void* Q8, void* K8,
+                              float* qscale, float* kscale, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  if (!Q || !K || !mask || !count || !Q8 || !K8 || !qscale || !kscale) return SA_ERR_INVALID_ARG;
+  const sa_status sh = check_shape(s);
+  if (sh != SA_OK) return sh;
+  if (s.d != 128) return SA_ERR_UNSUPPORTED;
+  if (!(tau > 0.f && tau <= 1.f)) return SA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return SA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(Q8) || !aligned16(K8) ||
+      (reinterpret_cast<uintptr_t>(qscale) & 3u) != 0 || (reinterpret_cast<uintptr_t>(kscale) & 3u) != 0)
+    return SA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < sparse_attn_plan_workspace_size(s))
+    return SA_ERR_WORKSPACE;
+  return launch_plan<128>(s, Q, K, tau, nullptr, scale, causal != 0, mask, count, idx, work, workspace,
+                          static_cast<cudaStream_t>(stream), static_cast<uint8_t*>(Q8), static_cast<uint8_t*>(K8),
+                          qscale, kscale);
+}
+
+sa_status sparse_attn_fwd_q8(const void* Q8, const void* K8, const float* qscale, const float* kscale,
+                             const void* V, sa_shape s, const uint8_t* mask, const int32_t* work, float lambda,
+                             float scale, int32_t causal, void* O, int64_t* stats, void* stream) {
+  if (!Q8 || !K8 || !qscale || !kscale || !V || !mask || !O) return SA_ERR_INVALID_ARG;
+  const sa_status sh = check_shape(s);
+  if (sh != SA_OK) return sh;
+  if (s.d != 128) return SA_ERR_UNSUPPORTED;
+  if (std::isnan(lambda) || (std::isinf(lambda) && lambda > 0)) return SA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return SA_ERR_INVALID_ARG;
+  if (!aligned16(Q8) || !aligned16(K8) || !aligned16(V) || !aligned16(O) ||
+      (reinterpret_cast<uintptr_t>(qscale) & 3u) != 0 || (reinterpret_cast<uintptr_t>(kscale) & 3u) != 0)
+    return SA_ERR_INVALID_ARG;
+  if (stats && (reinterpret_cast<uintptr_t>(stats) & 7u) != 0) return SA_ERR_INVALID_ARG;
+  return launch_fwd<128, true>(s, Q8, K8, V, mask, work, lambda, scale, causal != 0, O, stats,
+                               static_cast<cudaStream_t>(stream), qscale, kscale);
 }
 
 sa_status sparse_attn_selftest_wait_timeout(uint32_t limit_us, void* stream) {

@@ -144,6 +144,33 @@ sa_status sparse_attn_fwd(const void* Q, const void* K, const void* V, sa_shape 
                           const uint8_t* mask, const int32_t* work, float lambda, float scale,
                           int32_t causal, void* O, int64_t* stats, void* stream);
 
+/* Quantized scores (SpargeAttn: "sparse and quantized"; the quantization scheme
+ * is this library's own, the pages give none). sparse_attn_plan that also writes
+ * FP8 E4M3 copies of Q and K from the same pass over them:
+ *
+ *   Q8, K8          out, device uint8 [B,H,N,d] (16-byte aligned): E4M3 codes
+ *   qscale, kscale  out, device float [B,H,Nb]: one scale per 64-token block
+ *
+ * For each (b, h, block) of Q and of K: amax = max |x| over the block, scale =
+ * amax / 448 and code = x * (448 / amax) rounded to the nearest E4M3 value (ties
+ * to even, saturating at 448), both in fp32; an all-zero block gets scale 1 and
+ * codes 0. code * scale is the dequantized value. d must be 128, else
+ * SA_ERR_UNSUPPORTED. Other arguments, outputs and errors: as sparse_attn_plan. */
+sa_status sparse_attn_plan_q8(const void* Q, const void* K, sa_shape s, float tau, float scale,
+                              int32_t causal, uint8_t* mask, int32_t* count, int32_t* idx,
+                              int32_t* work, void* Q8, void* K8, float* qscale, float* kscale,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* sparse_attn_fwd with the scores taken on the FP8 codes of sparse_attn_plan_q8:
+ * S = (Q8 K8^T) * qscale[query block] * kscale[key block] by tcgen05.mma
+ * kind::f8f6f4 (fp32 accumulate); the softmax, the lambda filter, P.V (bf16 P, bf16
+ * V) and O are those of sparse_attn_fwd. d must be 128. Other arguments and
+ * errors: as sparse_attn_fwd. */
+sa_status sparse_attn_fwd_q8(const void* Q8, const void* K8, const float* qscale, const float* kscale,
+                             const void* V, sa_shape s, const uint8_t* mask, const int32_t* work,
+                             float lambda, float scale, int32_t causal, void* O, int64_t* stats,
+                             void* stream);
+
 /* sparse_attn_plan without a workspace, for callers that cannot allocate device
  * memory (a runtime that reserves its whole memory budget up front, a plugin
  * whose host owns the allocator, a latency-critical path that must not call

@@ -105,6 +105,25 @@ def test_fwd_argument_errors(lib):
     assert _fwd(lib, s=SaShape(70000, 1, 128, 128, 64)) == 2
 
 
+def test_q8_entry_points_reject_bad_arguments(lib):
+    s, s64 = SaShape(1, 2, 128, 128, 64), SaShape(1, 2, 128, 64, 64)
+    ws = ctypes.c_void_p(0x100000)
+
+    def plan(s=s, Q8=FAKE, qs=FAKE, tau=0.9):
+        return lib.sparse_attn_plan_q8(FAKE, FAKE, s, tau, 0.1, 0, FAKE, FAKE, None, None, Q8, FAKE, qs, FAKE,
+                                       ws, 1 << 30, None)
+
+    def fwd(s=s, K8=FAKE, ks=FAKE, lam=-math.inf):
+        return lib.sparse_attn_fwd_q8(FAKE, K8, FAKE, ks, FAKE, s, FAKE, None, lam, 0.1, 0, FAKE, None, None)
+
+    assert plan(Q8=None) == 1 and plan(qs=None) == 1
+    assert plan(qs=ctypes.c_void_p(0x10002)) == 1                    # scales must be 4-byte aligned
+    assert plan(Q8=FAKE_ODD) == 1 and plan(tau=1.5) == 1
+    assert plan(s=s64) == 2                                         # d = 128 only
+    assert fwd(K8=None) == 1 and fwd(ks=None) == 1 and fwd(lam=float("nan")) == 1
+    assert fwd(s=s64) == 2
+
+
 def test_device_error_needs_output_pointer(lib):
     assert lib.sparse_attn_device_error(None, None) == 1
 
