@@ -14,6 +14,7 @@ the same workload (weak scaling), timed on the device, max over ranks.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -56,6 +57,8 @@ def parse():
     ap.add_argument("--no-dense", action="store_true", help="skip the dense (full-mask) reference timing")
     ap.add_argument("--sweep", action="store_true",
                     help="one JSON line per configured (workload, tau, lambda, centroid weight); kernel timing only")
+    ap.add_argument("--qk", default="bf16", choices=["bf16", "fp8"],
+                    help="score operands: bf16 Q and K, or their FP8 E4M3 per-block codes (P.V stays bf16)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch plan and forward directly instead of replaying CUDA graphs")
     return ap.parse_args()
@@ -74,7 +77,7 @@ def peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def measured_traffic(w, tau, lam):
+def measured_traffic(w, tau, lam, qk="bf16"):
     """DRAM bytes per launch of the forward kernel from the committed ncu capture,
     or None if the kernel source changed since (or the workload differs)."""
     import hashlib
@@ -90,7 +93,7 @@ def measured_traffic(w, tau, lam):
     if h.hexdigest() != d.get("source_sha256"):
         return None
     key = f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.D} tau={tau:g} lambda={lam if lam is not None else 'off'}"
-    key = key.replace("lambda=-12.0", "lambda=-12")
+    key = key.replace("lambda=-12.0", "lambda=-12") + ("" if qk == "bf16" else f" qk={qk}")
     ent = d.get("traffic_bytes_per_launch", {}).get(key)
     return None if ent is None else float(ent["total"])
 
@@ -250,6 +253,7 @@ def config_dict(w, args, world):
     return {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.D} block=64 "
                         f"{'causal' if w.causal else 'non-causal'}",
             "tau": args.tau, "lambda": lam_value(args.lam), "seq_len": w.N, "heads": w.H, "head_dim": w.D,
+            "qk": getattr(args, "qk", "bf16"),
             "global_batch": w.B * world, "parallelism": f"replicas{world}",
             "l2": "flushed between timed steps" if 3 * w.B * w.H * w.N * w.D * 2 < 2 * L2_BYTES
             else "inputs larger than L2 (flushed too)",
@@ -275,20 +279,21 @@ def run_ours(args, w, world, rank, local, pg):
     B, H, N, D = w.B, w.H, w.N, w.D
     Nb = -(-N // 64)
     # buffers reused by every step (resident, allocated once)
-    plan = sa.sparse_attn_plan(q, k, args.tau, None, w.causal, with_idx=False)
+    q8 = args.qk == "fp8"
+    plan = sa.sparse_attn_plan(q, k, args.tau, None, w.causal, with_idx=False, quantize=q8)
     ws = torch.empty(sa.sparse_attn_plan_workspace_size(B, H, N, D), dtype=torch.uint8, device=dev)
     out = torch.empty_like(q)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False)
-        sa.sparse_attn_fwd(q, k, v, plan, lam, out=out)
+        sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False, quantize=q8)
+        sa.sparse_attn_fwd(q, k, v, plan, lam, out=out, qk_fp8=q8)
 
     # stats (outside timing): kept pairs, skipped P.V, algorithmic FLOPs of the forward
     stats = torch.zeros(4, dtype=torch.int64, device=dev)
-    sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False)
-    sa.sparse_attn_fwd(q, k, v, plan, lam, out=out, stats=stats)
+    sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False, quantize=q8)
+    sa.sparse_attn_fwd(q, k, v, plan, lam, out=out, stats=stats, qk_fp8=q8)
     torch.cuda.synchronize()
     check_device(sa, "the stats pass")
     st = [int(x) for x in stats.cpu()]
@@ -309,12 +314,14 @@ def run_ours(args, w, world, rank, local, pg):
     dense_ms = None
     if not args.no_dense:
         full = torch.ones((B, H, Nb, Nb), dtype=torch.uint8, device=dev)
+        if q8:   # the same score operands, every block kept
+            full = dataclasses.replace(plan, mask=full, work=None)
         for _ in range(2):
-            sa.sparse_attn_fwd(q, k, v, full, None, out=out, causal=w.causal)
+            sa.sparse_attn_fwd(q, k, v, full, None, out=out, causal=w.causal, qk_fp8=q8)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         flush.zero_()
         e0.record(stream)
-        sa.sparse_attn_fwd(q, k, v, full, None, out=out, causal=w.causal)
+        sa.sparse_attn_fwd(q, k, v, full, None, out=out, causal=w.causal, qk_fp8=q8)
         e1.record(stream)
         torch.cuda.synchronize()
         dense_ms = e0.elapsed_time(e1)
@@ -322,10 +329,10 @@ def run_ours(args, w, world, rank, local, pg):
         del full
 
     def run_plan():
-        sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False)
+        sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False, quantize=q8)
 
     def run_fwd():
-        sa.sparse_attn_fwd(q, k, v, plan, lam, out=out)
+        sa.sparse_attn_fwd(q, k, v, plan, lam, out=out, qk_fp8=q8)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -378,7 +385,7 @@ def run_ours(args, w, world, rank, local, pg):
         # warm-up calls exactly like the timed ones, so that the caching pinned
         # allocator holds the output blocks the timed calls cycle through
         for _ in range(max(3, args.warmup)):
-            o_host = sa.sparse_attention(qh, kh, vh, args.tau, lam, None, w.causal, device=dev)
+            o_host = sa.sparse_attention(qh, kh, vh, args.tau, lam, None, w.causal, device=dev, qk_fp8=q8)
             torch.cuda.synchronize()
         barrier(pg, dev)
         t = []
@@ -386,7 +393,7 @@ def run_ours(args, w, world, rank, local, pg):
             flush.zero_()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            o_host = sa.sparse_attention(qh, kh, vh, args.tau, lam, None, w.causal, device=dev)
+            o_host = sa.sparse_attention(qh, kh, vh, args.tau, lam, None, w.causal, device=dev, qk_fp8=q8)
             b.record(stream)
             torch.cuda.synchronize()
             t.append(a.elapsed_time(b))
@@ -399,11 +406,20 @@ def run_ours(args, w, world, rank, local, pg):
 
     pk, pk_kind = peaks()
     peak_t = float(pk["bf16_tflops"])
+    peak_source = f"{pk_kind} bf16_tflops (burst)"
+    if q8:
+        # QK^T on FP8 at twice the bf16 peak (the nominal fp8 : bf16 ratio), P.V at the
+        # bf16 peak: the peak of this mix is the FLOPs over the time each part needs
+        s_flops = 2.0 * D * pair_tokens
+        peak_t = exec_flops / (s_flops / (2.0 * peak_t) + (exec_flops - s_flops) / peak_t)
+        peak_source = (f"{pk_kind} bf16_tflops (burst) for P.V, x2 (nominal fp8:bf16) for QK^T, "
+                       "combined over the executed FLOPs")
     achieved = exec_flops / (fwd_avg * 1e-3) / 1e12
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded cluster-centroid generator)",
+        "vs_baseline": None, "dtype": "fp8 e4m3 QK^T, bf16 P.V" if q8 else "bf16",
+        "data": "synthetic (seeded cluster-centroid generator)",
         "config": config_dict(w, args, world),
         "plan_ms": plan_avg, "fwd_ms": fwd_avg, "dense_fwd_ms": dense_ms,
         "sparsity_pct": 100.0 * (1.0 - kept_pairs / total_pairs),
@@ -411,9 +427,10 @@ def run_ours(args, w, world, rank, local, pg):
         "executed_tflops": achieved, "pct_of_bf16_peak_executed": 100.0 * achieved / peak_t,
         "predictor_pct_of_dense": None if dense_ms is None else 100.0 * plan_avg / dense_ms,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
-                     "frac": achieved / peak_t, "traffic": measured_traffic(w, args.tau, lam),
-                     "kernel": f"fwd_kernel<{D}> (sparse_attn_fwd)",
-                     "peak_source": f"{pk_kind} bf16_tflops (burst)"},
+                     "frac": achieved / peak_t, "traffic": measured_traffic(w, args.tau, lam, args.qk),
+                     "kernel": f"fwd_kernel<{D}, fp8 scores> (sparse_attn_fwd_q8)" if q8
+                     else f"fwd_kernel<{D}> (sparse_attn_fwd)",
+                     "peak_source": peak_source},
         "e2e": e2e, "gpu_launches": 4 * args.steps, "cuda_graphs": not args.no_graph, "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -428,6 +445,8 @@ def sweep(args):
     """Every configured point of every workload (one GPU, kernel timing only)."""
     base = dict(vars(args))
     for name, w in wl.WORKLOADS.items():
+        if args.qk == "fp8" and w.D != 128:
+            continue                                  # FP8 scores are for d = 128
         cws = w.centroid_weights or (None,)
         for tau in w.taus:
             for lam in w.lams:

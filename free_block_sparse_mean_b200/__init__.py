@@ -222,7 +222,8 @@ def _copy_streams(dev: torch.device):
 
 def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau,
                      lam: Optional[float] = None, scale: Optional[float] = None, causal: bool = False,
-                     device="cuda", out: Optional[torch.Tensor] = None, chunks: Optional[int] = None) -> torch.Tensor:
+                     device="cuda", out: Optional[torch.Tensor] = None, chunks: Optional[int] = None,
+                     qk_fp8: bool = False) -> torch.Tensor:
     """End to end from host tensors: copy q, k, v to the GPU, plan + forward, copy O back.
 
     Host inputs should be pinned, so the copies are asynchronous DMA. The result is
@@ -233,7 +234,8 @@ def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau,
     (default: up to 4): group g's host-to-device copy, its plan + forward and its
     device-to-host copy run on three streams, so the copies of one group overlap
     the work of the others in both directions of the link. tau may be one value or
-    a per-head float32 tensor ([B, H] or [H]) on `device`."""
+    a per-head float32 tensor ([B, H] or [H]) on `device`. qk_fp8=True takes the
+    scores on FP8 copies of q and k (see sparse_attn_plan's quantize)."""
     dev = torch.device(device)
     if q.shape != k.shape or q.shape != v.shape or q.dim() != 4:
         raise ValueError("q, k, v must share the shape [B, H, N, d]")
@@ -265,8 +267,8 @@ def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau,
         main.wait_event(ready)
         view = lambda x: x[lo:hi].view(1, hi - lo, N, d)
         t = tau[lo:hi].view(1, hi - lo) if isinstance(tau, torch.Tensor) else tau
-        plan = sparse_attn_plan(view(qd), view(kd), t, scale, causal, with_idx=False)
-        sparse_attn_fwd(view(qd), view(kd), view(vd), plan, lam, scale, causal, out=view(od))
+        plan = sparse_attn_plan(view(qd), view(kd), t, scale, causal, with_idx=False, quantize=qk_fp8)
+        sparse_attn_fwd(view(qd), view(kd), view(vd), plan, lam, scale, causal, out=view(od), qk_fp8=qk_fp8)
         done = torch.cuda.Event()
         done.record(main)
         d2h.wait_event(done)
