@@ -83,3 +83,30 @@ def test_full_mask_natural_pairs_repeated():
     ones = np.ones((1, 1, Nb, Nb), dtype=np.uint8)
     ref = orc.fwd(qh, kh, vh, ones, None, None, w.causal, qblocks=qbs)
     assert_output_close(to_np(out[:, h:h + 1]), ref, f"full mask head {h} query blocks {qbs}")
+
+
+@pytest.mark.parametrize("name,tau,lam,out_heads", [("hunyuan", 0.95, -12.0, (3,)), ("wan", 0.95, None, (7,))])
+def test_full_size_fp8_scores(name, tau, lam, out_heads):
+    """The quantized-score variant at full size: the codes and scales of sampled
+    heads byte for byte against the oracle's quantizer, and sampled query blocks of
+    the forward on the codes against the oracle on the dequantized Q and K."""
+    dev = torch.device("cuda:0")
+    w = wl.WORKLOADS[name]
+    q, k, v = wl.generate(w, seed=0, device=dev)
+    plan = sa.sparse_attn_plan(q, k, tau, None, w.causal, quantize=True)
+    out = sa.sparse_attn_fwd(q, k, v, plan, lam, qk_fp8=True)
+    torch.cuda.synchronize()
+    assert sa.sparse_attn_device_error() == 0
+    Nb = -(-w.N // 64)
+    mask = to_np(plan.mask)
+    rng = np.random.default_rng(11)
+    for h in out_heads:
+        qh, kh, vh = (x[:, h:h + 1].cpu() for x in (q, k, v))
+        for x, x8, sc in ((qh, plan.q8, plan.qscale), (kh, plan.k8, plan.kscale)):
+            codes, scales = orc.quantize_blocks_e4m3(x)
+            want = torch.tensor(codes, dtype=torch.float32).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+            np.testing.assert_array_equal(to_np(x8[:, h:h + 1]), want)
+            np.testing.assert_array_equal(to_np(sc[:, h:h + 1]).astype(np.float64), scales)
+        qbs = sorted({0, Nb - 1, *rng.choice(Nb, size=4, replace=False).tolist()})
+        ref = orc.fwd_fp8qk(qh, kh, vh, mask[:, h:h + 1], lam, None, w.causal, qblocks=qbs)
+        assert_output_close(to_np(out[:, h:h + 1]), ref, f"fp8 {name} head {h} query blocks {qbs}")
