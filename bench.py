@@ -415,6 +415,13 @@ def run_ours(args, w, world, rank, local, pg):
         peak_source = (f"{pk_kind} bf16_tflops (burst) for P.V, x2 (nominal fp8:bf16) for QK^T, "
                        "combined over the executed FLOPs")
     achieved = exec_flops / (fwd_avg * 1e-3) / 1e12
+    # predictor: compulsory bytes (Q and K read once; mask and counts written; with
+    # FP8 scores also the codes and scales) over the plan time, against the HBM copy peak
+    pred_bytes = 2.0 * B * H * N * D * 2 + B * H * Nb * Nb + 4.0 * B * H * Nb
+    if q8:
+        pred_bytes += 2.0 * B * H * N * D + 8.0 * B * H * Nb
+    hbm = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    pred_gbs = pred_bytes / (plan_avg * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
@@ -426,6 +433,8 @@ def run_ours(args, w, world, rank, local, pg):
         "lambda_skip_pct": 100.0 * skipped / max(kept_pairs, 1),
         "executed_tflops": achieved, "pct_of_bf16_peak_executed": 100.0 * achieved / peak_t,
         "predictor_pct_of_dense": None if dense_ms is None else 100.0 * plan_avg / dense_ms,
+        "predictor": {"bound": "hbm", "achieved": pred_gbs, "peak": hbm, "unit": "GB/s", "frac": pred_gbs / hbm,
+                      "bytes": pred_bytes, "peak_source": f"{pk_kind} hbm_gbs"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": achieved / peak_t, "traffic": measured_traffic(w, args.tau, lam, args.qk),
                      "kernel": f"fwd_kernel<{D}, fp8 scores> (sparse_attn_fwd_q8)" if q8
