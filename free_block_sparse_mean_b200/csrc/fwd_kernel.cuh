@@ -51,7 +51,8 @@
 // having waited for P(k-4) (P(k-3)) before. A K or V stage is refilled only after
 // the MMA that read it has completed. The lambda votes carry the
 // entry index as a tag, and a vote slot is reused for entry k+2 only after every
-// softmax warp has released S(k+1), which each does after reading entry k's vote.
+// softmax warp has released S(k+1), which each does after reading entry k's vote
+// (a warp whose own rows do not all pass cannot skip and does not read it).
 #pragma once
 
 #include "sa_device.cuh"
@@ -451,12 +452,12 @@ __global__ void __launch_bounds__(192, 2)
       l = l * alpha + psum;
       // lambda: the half skips P.V when both of its warps pass; its P(k) is zero
       bool half_skip = false;
-      if (lam_on) {
+      if (lam_on && wpass) {                      // a warp that does not pass never skips
         int pv = 0;
         if (lane == 0) pv = spin_tag(&votes[(k & 1) * 4 + (wq ^ 1)], k, abort_flag);
         pv = __shfl_sync(FULL, pv, 0);
         if (pv < 0) { alive = false; break; }
-        half_skip = wpass && (pv & 1);
+        half_skip = (pv & 1) != 0;
         if (half_skip) {
 #pragma unroll
           for (int c = 0; c < 32; ++c) pk[c] = 0u;
