@@ -54,7 +54,7 @@ def test_fp8_score_forward_matches_the_oracle(case, lam):
         w = wl.WORKLOADS["lm"].with_(H=2, N=2048)
         q, k, v = wl.generate(w, seed=3, device=_dev())
     else:
-        q, k, v = wl.random_qkv(1, 3, 1000, 128, seed=10, device=_dev(), scale_qk=2.0)
+        q, k, v = wl.random_qkv(2, 3, 1000, 128, seed=10, device=_dev(), scale_qk=2.0)   # B = 2, ragged tail
     p = sa.sparse_attn_plan(q, k, 0.95, None, causal, quantize=True)
     st8 = torch.zeros(4, dtype=torch.int64, device=_dev())
     st = torch.zeros(4, dtype=torch.int64, device=_dev())
