@@ -29,6 +29,12 @@ Readings where the pages are silent (each is also listed in the design notes):
     with m_r the running max before the block; the block still enters the
     running max and the running sum l (only P.V is skipped).
   * a query row that ends with no visible key gets an output of zero.
+  * in-operator cumulative-energy filter (the DynSparse step placed inside the
+    FlashAttention operator; an alternative to the lambda test): the same tiled
+    loop, but a key block's P.V is skipped when, for every row of the query block
+    that sees it, the energy skipped so far plus the block's own energy stays
+    within (1 - recall) of the running sum l including the block; l is the
+    cumulative energy the operator already keeps, the threshold moves with it.
 
 Arithmetic is fp64 throughout; inputs are the exact values of the bf16 tensors.
 
@@ -41,8 +47,8 @@ decision), ties to even, saturating. The scores are then the dequantized
 (code * s) products; V, P and the rest of the attention are unchanged.
 
 Entry points: block_mean_pool, pooled_logits, pooled_softmax,
-cumulative_energy_select, plan, attention_masked, attention_tiled, fwd,
-round_e4m3, quantize_blocks_e4m3, fwd_fp8qk.
+cumulative_energy_select, plan, attention_masked, attention_tiled,
+attention_recall, fwd, round_e4m3, quantize_blocks_e4m3, fwd_fp8qk.
 """
 from __future__ import annotations
 
@@ -267,6 +273,93 @@ def attention_tiled(Q, K, V, mask, lam: float, scale: Optional[float] = None,
                 O[b, h, s:e] = out
     if return_stats:
         return O, dict(kept_pairs=kept_pairs, pv_skipped=skipped_pairs)
+    return O
+
+
+def attention_recall(Q, K, V, mask, recall: float, scale: Optional[float] = None,
+                     causal: bool = False, block: int = BLOCK,
+                     qblocks: Optional[Iterable[int]] = None, return_stats: bool = False):
+    """Stage 2 with the in-operator cumulative-energy filter, as a literal fp64 run
+    of the tiled loop (64-row query blocks, kept key blocks in ascending order).
+
+    DynSparse article: a fixed recall of the attention energy is enough for
+    accuracy, and the threshold is a dynamic one derived from the cumulative
+    energy of the selected tokens, which the FlashAttention operator already holds
+    (its running sum l). Reading: per row r, l_r is the energy seen so far and
+    sk_r the part of it whose P.V was skipped, both relative to the running max.
+    For key block j with row energies e_r = sum_c exp(S_rc - m'_r), the block's
+    P.V is skipped when every row r of the query block that sees a key of the
+    block has sk_r * alpha_r + e_r <= (1 - recall) * (l_r * alpha_r + e_r)
+    (alpha_r = exp(m_r - m'_r) rescales the old sums to the new max). l always
+    takes e_r; sk takes it only when the block is skipped. By induction
+    sk_r <= (1 - recall) * l_r after every block, so each row keeps at least the
+    fraction `recall` of the energy of the blocks it visits.
+
+    With return_stats, also returns dict(kept_pairs, pv_skipped, decisions,
+    recall_rows): decisions is a list of (b, h, i, j, skipped, margin) where
+    margin = min over the seeing rows of ((1 - recall) * l' - (sk * alpha + e)) / l'
+    (the decision is "skip" iff margin >= 0), and recall_rows [B, H, N] is
+    1 - sk / l per row at the end (NaN for rows not computed)."""
+    Q, K, V = as_f64(Q), as_f64(K), as_f64(V)
+    mask = np.asarray(mask)
+    B, H, N, d = Q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    Nb = n_blocks(N, block)
+    qbs = range(Nb) if qblocks is None else qblocks
+    O = np.full((B, H, N, V.shape[-1]), np.nan)
+    rec_rows = np.full((B, H, N), np.nan)
+    kept_pairs = 0
+    skipped_pairs = 0
+    decisions = []
+    budget = 1.0 - recall
+    for b in range(B):
+        for h in range(H):
+            for i in qbs:
+                s, e = i * block, min(N, (i + 1) * block)
+                rows = np.arange(s, e)
+                m = np.full(e - s, -np.inf)
+                l = np.zeros(e - s)
+                sk = np.zeros(e - s)
+                acc = np.zeros((e - s, V.shape[-1]))
+                for j in np.nonzero(mask[b, h, i])[0]:
+                    ks, ke = j * block, min(N, (j + 1) * block)
+                    S = scale * Q[b, h, s:e] @ K[b, h, ks:ke].T
+                    if causal:
+                        S = np.where(np.arange(ks, ke)[None, :] <= rows[:, None], S, -np.inf)
+                    rmax = S.max(axis=1)
+                    sees = np.isfinite(rmax)
+                    if not sees.any():
+                        continue
+                    kept_pairs += 1
+                    m_new = np.maximum(m, rmax)
+                    ref = np.where(np.isfinite(m_new), m_new, 0.0)
+                    alpha = np.where(np.isfinite(m), np.exp(m - ref), 0.0)
+                    Pb = np.exp(S - ref[:, None])
+                    en = Pb.sum(axis=1)
+                    l_new = l * alpha + en
+                    sk_try = sk * alpha + en
+                    room = budget * l_new - sk_try
+                    margin = float(np.min(room[sees] / l_new[sees]))
+                    skip = bool(np.all(room[sees] >= 0.0))
+                    decisions.append((b, h, i, int(j), skip, margin))
+                    l = l_new
+                    acc = acc * alpha[:, None]
+                    if skip:
+                        skipped_pairs += 1
+                        sk = sk_try
+                    else:
+                        sk = sk * alpha
+                        acc = acc + Pb @ V[b, h, ks:ke]
+                    m = m_new
+                out = acc / np.where(l > 0, l, 1.0)[:, None]
+                out[l <= 0] = 0.0
+                O[b, h, s:e] = out
+                with np.errstate(invalid="ignore", divide="ignore"):
+                    rec_rows[b, h, s:e] = np.where(l > 0, 1.0 - sk / np.where(l > 0, l, 1.0), 1.0)
+    if return_stats:
+        return O, dict(kept_pairs=kept_pairs, pv_skipped=skipped_pairs, decisions=decisions,
+                       recall_rows=rec_rows)
     return O
 
 

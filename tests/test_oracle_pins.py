@@ -302,6 +302,171 @@ def test_lambda_error_bounded_by_skipped_mass():
     assert np.abs(O_lam - O_off).max() <= bound
 
 
+# ---------------------------------------------------------------- in-operator recall filter
+@pytest.mark.parametrize("c,recall,skipped", [(5.0, 0.99, True), (5.0, 0.995, False),
+                                               (1.0, 0.7, True), (1.0, 0.75, False)])
+def test_recall_skip_closed_form(c, recall, skipped):
+    """Scores 0 on key block 0 and -c on key block 1 (visited second); t = e^-c.
+    Block 1 carries the energy fraction t / (1 + t) of the row, so it is skipped
+    exactly when t / (1 + t) <= 1 - recall: recall <= 1 / (1 + t), which is 0.99331
+    for c = 5 and 0.7311 for c = 1 (where 1 - recall = 0.3 lies between
+    t / (1 + t) = 0.269 and t = 0.368: the block's own energy counts in the sum).
+    Skipped: O = (1, 0) / (1 + t) (l keeps the block); kept: O = (1, t) / (1 + t)."""
+    Q, K, V, mask = _two_block_case(0.0, -c)
+    t = math.exp(-c)
+    O, st = orc.attention_recall(Q, K, V, mask, recall, 1.0, return_stats=True)
+    want = [1 / (1 + t), 0.0 if skipped else t / (1 + t)]
+    np.testing.assert_allclose(O[0, 0], np.tile(want, (128, 1)), rtol=1e-14, atol=0)
+    assert st["kept_pairs"] == 4 and st["pv_skipped"] == (2 if skipped else 0)
+    np.testing.assert_allclose(st["recall_rows"][0, 0], 1 / (1 + t) if skipped else 1.0, rtol=1e-14)
+
+
+def test_recall_first_block_never_skipped_and_old_sums_rescaled():
+    """Block 0 at -20 then block 1 at 0: block 0 comes first (nothing to compare
+    with) and block 1 holds almost all of the energy once the old sum is rescaled
+    to the new max (e^-20 * 64 against 64), so nothing is skipped even at
+    recall = 0.5. Without the rescale the first block's sum would hide block 1."""
+    Q, K, V, mask = _two_block_case(-20.0, 0.0)
+    O_off = orc.fwd(Q, K, V, mask, None, 1.0)
+    O, st = orc.attention_recall(Q, K, V, mask, 0.5, 1.0, return_stats=True)
+    assert st["pv_skipped"] == 0
+    np.testing.assert_allclose(O, O_off, rtol=1e-14)
+
+
+def test_recall_sums_rescaled_when_the_max_rises():
+    """Four key blocks with scores 0, -5, 3, -2 (t = e^-5), recall 0.99, visited in
+    that order. Block 1 holds t / (1 + t) = 0.0067 <= 0.01 of the energy: skipped.
+    Block 2 raises the max by 3 and holds most of the energy: kept. Block 3 (e^-5
+    against the new max): skipped-so-far t e^-3 plus its own t is 0.00707, within
+    0.01 of the sum e^-3 (1 + t) + 1 + t = 1.0568: skipped. Had the skipped sum
+    not been rescaled to the new max (t + t = 0.0135) it would be kept.
+    O = (e^-3, 0, 1, 0) / (e^-3 + e^-8 + 1 + e^-5)."""
+    N, d = 256, 4
+    Q = np.zeros((1, 1, N, d)); Q[..., 0] = 1.0
+    K = np.zeros((1, 1, N, d))
+    V = np.zeros((1, 1, N, d))
+    for j, sc in enumerate([0.0, -5.0, 3.0, -2.0]):
+        K[0, 0, 64 * j:64 * j + 64, 0] = sc
+        V[0, 0, 64 * j:64 * j + 64, j] = 1.0
+    mask = np.ones((1, 1, 4, 4), dtype=np.uint8)
+    O, st = orc.attention_recall(Q, K, V, mask, 0.99, 1.0, return_stats=True)
+    z = math.exp(-3) + math.exp(-8) + 1 + math.exp(-5)
+    np.testing.assert_allclose(O[0, 0], np.tile([math.exp(-3) / z, 0, 1 / z, 0], (N, 1)), rtol=1e-13, atol=0)
+    assert [x[4] for x in st["decisions"][:4]] == [False, True, False, True]
+    np.testing.assert_allclose(st["recall_rows"][0, 0], (math.exp(-3) + 1) / z, rtol=1e-13)
+
+
+def test_recall_block_that_raises_the_max_can_be_skipped():
+    """Recall 0.95; key block 0 at score 0, block 1 at -5 (t = e^-5), block 2 one
+    key at +1 and 63 at -50. Block 1: t / (1 + t) <= 0.05, skipped. Block 2 raises
+    the max by 1 but holds one key's worth of energy: against the new max the
+    skipped sum is 64 t e^-1 = 0.1586, plus its own 1 gives 1.1586 <= 0.05 *
+    (64 (1 + t) e^-1 + 1) = 1.2351: skipped (the skipped sum unrescaled, 1.4312,
+    would keep it). O = (64 e^-1, 0, 0) / (64 e^-1 + 64 e^-6 + 1 + 63 e^-51)."""
+    N, d = 192, 3
+    Q = np.zeros((1, 1, N, d)); Q[..., 0] = 1.0
+    K = np.zeros((1, 1, N, d))
+    V = np.zeros((1, 1, N, d))
+    K[0, 0, 64:128, 0] = -5.0
+    K[0, 0, 128:, 0] = -50.0
+    K[0, 0, 128, 0] = 1.0
+    for j in range(3):
+        V[0, 0, 64 * j:64 * j + 64, j] = 1.0
+    mask = np.ones((1, 1, 3, 3), dtype=np.uint8)
+    O, st = orc.attention_recall(Q, K, V, mask, 0.95, 1.0, return_stats=True)
+    z = 64 * math.exp(-1) + 64 * math.exp(-6) + 1 + 63 * math.exp(-51)
+    np.testing.assert_allclose(O[0, 0], np.tile([64 * math.exp(-1) / z, 0, 0], (N, 1)), rtol=1e-13, atol=0)
+    assert [x[4] for x in st["decisions"][:3]] == [False, True, True]
+
+
+def _recall_case(seed, N, d, causal, aligned=0):
+    """Key block `aligned` aligned with every query, the rest noise of varied
+    strength per block, a random block mask with the diagonal and the aligned
+    block kept. With aligned > 0 the running max rises midway through the row."""
+    r = _rng(seed)
+    u = np.ones(d)
+    Nb = orc.n_blocks(N)
+    Q = 1.5 * u + 0.5 * r.standard_normal((1, 2, N, d))
+    K = r.standard_normal((1, 2, N, d))
+    K *= np.repeat(r.uniform(0.05, 1.5, size=(1, 2, Nb, 1)), 64, axis=2)[:, :, :N]
+    a = slice(64 * aligned, 64 * aligned + 64)
+    K[:, :, a] = 1.5 * u + 0.5 * r.standard_normal((1, 2, 64, d))
+    V = r.standard_normal((1, 2, N, d))
+    mask = (r.random((1, 2, Nb, Nb)) < 0.6).astype(np.uint8)
+    mask[..., np.arange(Nb), np.arange(Nb)] = 1
+    mask[..., aligned] = 1
+    return Q, K, V, mask
+
+
+@pytest.mark.parametrize("N,causal,recall,aligned", [(512, False, 0.99, 0), (449, True, 0.95, 0),
+                                                     (320, False, 0.9, 0), (640, False, 0.97, 5),
+                                                     (577, True, 0.9, 3)])
+def test_recall_decisions_and_output_brute_force(N, causal, recall, aligned):
+    """Brute force without a running max: every row's block energies are taken
+    against one fixed reference (the row's largest visible score), and the sums
+    of earlier blocks are plain sums. Block j of query block i is skipped iff for
+    every row that sees it, skipped-so-far + E_j <= (1 - recall) * (seen-so-far
+    + E_j). The output is the unskipped blocks' weighted V over the energy of all
+    visited blocks. The oracle's decisions and output must agree."""
+    d = 16
+    Q, K, V, mask = _recall_case(N + int(causal), N, d, causal, aligned)
+    scale = 1.0 / math.sqrt(d)
+    O, st = orc.attention_recall(Q, K, V, mask, recall, None, causal, return_stats=True)
+    dec = {(b, h, i, j): (sk, mg) for b, h, i, j, sk, mg in st["decisions"]}
+    Nb = orc.n_blocks(N)
+    n_skip = 0
+    for h in range(2):
+        for i in range(Nb):
+            s, e = i * 64, min(N, i * 64 + 64)
+            S = scale * Q[0, h, s:e] @ K[0, h].T
+            vis = np.repeat(mask[0, h, i].astype(bool), 64)[:N][None, :].repeat(e - s, 0)
+            if causal:
+                vis &= np.arange(N)[None, :] <= np.arange(s, e)[:, None]
+            S = np.where(vis, S, -np.inf)
+            M = S.max(axis=1)
+            W = np.exp(S - M[:, None])
+            seen = np.zeros(e - s)
+            skipped = np.zeros(e - s)
+            num = np.zeros((e - s, d))
+            for j in np.nonzero(mask[0, h, i])[0]:
+                cols = slice(j * 64, min(N, j * 64 + 64))
+                sees = vis[:, cols].any(axis=1)
+                if not sees.any():
+                    continue
+                E = W[:, cols].sum(axis=1)
+                ok = skipped + E <= (1 - recall) * (seen + E)
+                skip = bool(ok[sees].all())
+                got, margin = dec[(0, h, i, int(j))]
+                if abs(margin) > 1e-9:
+                    assert got == skip, (h, i, j)
+                skip = got
+                seen += E
+                if skip:
+                    skipped += E
+                    n_skip += 1
+                else:
+                    num += W[:, cols] @ V[0, h, cols]
+            np.testing.assert_allclose(O[0, h, s:e], num / seen[:, None], rtol=1e-10, atol=1e-12)
+            assert np.all(skipped <= (1 - recall) * seen * (1 + 1e-12))
+    assert n_skip == st["pv_skipped"] and n_skip > 0
+    assert np.all(st["recall_rows"][np.isfinite(st["recall_rows"])] >= recall - 1e-12)
+
+
+@pytest.mark.parametrize("recall", [0.9, 0.99])
+def test_recall_error_bounded_by_budget(recall):
+    """The skipped blocks stay in l, so per row O_recall - O_off = -(skipped
+    weighted V) / l, at most (skipped energy / l) * max|V| <= (1 - recall) * max|V|
+    in every element; recall = 1 skips nothing and is the masked attention."""
+    Q, K, V, mask = _recall_case(3, 384, 8, False)
+    O_off = orc.attention_masked(Q, K, V, mask)
+    O, st = orc.attention_recall(Q, K, V, mask, recall, return_stats=True)
+    assert st["pv_skipped"] > 0
+    assert np.abs(O - O_off).max() <= (1 - recall) * np.abs(V).max() * (1 + 1e-12)
+    O1, st1 = orc.attention_recall(Q, K, V, mask, 1.0, return_stats=True)
+    assert st1["pv_skipped"] == 0
+    np.testing.assert_allclose(O1, O_off, rtol=1e-11, atol=1e-13)
+
+
 def test_row_without_visible_key_is_zero():
     r = _rng(5)
     Q, K, V = (r.standard_normal((1, 1, 128, 4)) for _ in range(3))
