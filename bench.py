@@ -6,7 +6,7 @@ Q/K/V of the chosen workload (default: the small DiT-layer shape, B=1 H=24 N=409
 d=128, tau=0.95, lambda=-12). Prints ONE JSON line on rank 0.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload small|tiny|wan|hunyuan|lm]
-                    [--tau T] [--lam L|off] [--impl ours|reference]
+                    [--tau T] [--lam L|off] [--recall R] [--impl ours|reference]
 
 Multi-GPU: the path has no exchange step; N ranks run N independent replicas of
 the same workload (weak scaling), timed on the device, max over ranks.
@@ -59,6 +59,9 @@ def parse():
                     help="one JSON line per configured (workload, tau, lambda, centroid weight); kernel timing only")
     ap.add_argument("--qk", default="bf16", choices=["bf16", "fp8"],
                     help="score operands: bf16 Q and K, or their FP8 E4M3 per-block codes (P.V stays bf16)")
+    ap.add_argument("--recall", type=float, default=None,
+                    help="P.V filter: the cumulative-energy test keeping this recall per row "
+                         "(sparse_attn_fwd_recall) instead of the lambda test")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch plan and forward directly instead of replaying CUDA graphs")
     return ap.parse_args()
@@ -77,7 +80,7 @@ def peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def measured_traffic(w, tau, lam, qk="bf16"):
+def measured_traffic(w, tau, lam, qk="bf16", recall=None):
     """DRAM bytes per launch of the forward kernel from the committed ncu capture,
     or None if the kernel source changed since (or the workload differs)."""
     import hashlib
@@ -94,6 +97,8 @@ def measured_traffic(w, tau, lam, qk="bf16"):
         return None
     key = f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.D} tau={tau:g} lambda={lam if lam is not None else 'off'}"
     key = key.replace("lambda=-12.0", "lambda=-12") + ("" if qk == "bf16" else f" qk={qk}")
+    if recall is not None:
+        key = key.split(" lambda=")[0] + f" recall={recall:g}"
     ent = d.get("traffic_bytes_per_launch", {}).get(key)
     return None if ent is None else float(ent["total"])
 
@@ -187,7 +192,7 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- CPU oracle timing
-def time_oracle(w, tau, lam, budget_s, seed):
+def time_oracle(w, tau, lam, budget_s, seed, recall=None):
     """The oracle as it stands (fp64 NumPy) on a bounded sample of the workload:
     whole heads (plan + forward) until the time budget is used, at least one."""
     from oracle import sparse_attn_oracle as orc
@@ -208,7 +213,10 @@ def time_oracle(w, tau, lam, budget_s, seed):
         q, k, v = wl.generate(w, seed=seed, device="cpu", heads=[h])
         t0 = time.perf_counter()
         p = orc.plan(q, k, tau, None, w.causal)
-        orc.fwd(q, k, v, p["mask"], lam, None, w.causal, qblocks=qblocks)
+        if recall is not None:
+            orc.attention_recall(q, k, v, p["mask"], recall, None, w.causal, qblocks=qblocks)
+        else:
+            orc.fwd(q, k, v, p["mask"], lam, None, w.causal, qblocks=qblocks)
         dt = time.perf_counter() - t0
         t_total += dt
         nb = -(-w.N // 64)
@@ -232,7 +240,7 @@ def run_reference(args, w, world, rank, pg):
     vals = []
     budget = max(2.0, min(args.cpu_seconds, 240.0 / max(1, args.steps + args.warmup)))
     for i in range(args.warmup + args.steps):
-        v, t, cores, sample = time_oracle(w, args.tau, lam, budget, args.seed)
+        v, t, cores, sample = time_oracle(w, args.tau, lam, budget, args.seed, args.recall)
         if i >= args.warmup:
             per_step.append(t)
             vals.append(v)
@@ -252,7 +260,9 @@ def run_reference(args, w, world, rank, pg):
 def config_dict(w, args, world):
     return {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.D} block=64 "
                         f"{'causal' if w.causal else 'non-causal'}",
-            "tau": args.tau, "lambda": lam_value(args.lam), "seq_len": w.N, "heads": w.H, "head_dim": w.D,
+            "tau": args.tau, "lambda": None if getattr(args, "recall", None) is not None else lam_value(args.lam),
+            "pv_filter": "recall" if getattr(args, "recall", None) is not None else "lambda",
+            "recall": getattr(args, "recall", None), "seq_len": w.N, "heads": w.H, "head_dim": w.D,
             "qk": getattr(args, "qk", "bf16"),
             "global_batch": w.B * world, "parallelism": f"replicas{world}",
             "l2": "flushed between timed steps" if 3 * w.B * w.H * w.N * w.D * 2 < 2 * L2_BYTES
@@ -273,13 +283,16 @@ def run_ours(args, w, world, rank, local, pg):
         raise RuntimeError("no CUDA device: the benchmark needs a B200")
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    lam = lam_value(args.lam)
+    rec = args.recall
+    lam = None if rec is not None else lam_value(args.lam)   # the recall test replaces lambda
     q, k, v = wl.generate(w, seed=args.seed, device=dev, centroid_weight=args.centroid_weight)
     torch.cuda.synchronize()
     B, H, N, D = w.B, w.H, w.N, w.D
     Nb = -(-N // 64)
     # buffers reused by every step (resident, allocated once)
     q8 = args.qk == "fp8"
+    if q8 and rec is not None:
+        raise SystemExit("--recall runs on bf16 scores: drop --qk fp8")
     plan = sa.sparse_attn_plan(q, k, args.tau, None, w.causal, with_idx=False, quantize=q8)
     ws = torch.empty(sa.sparse_attn_plan_workspace_size(B, H, N, D), dtype=torch.uint8, device=dev)
     out = torch.empty_like(q)
@@ -288,12 +301,12 @@ def run_ours(args, w, world, rank, local, pg):
 
     def step():
         sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False, quantize=q8)
-        sa.sparse_attn_fwd(q, k, v, plan, lam, out=out, qk_fp8=q8)
+        sa.sparse_attn_fwd(q, k, v, plan, lam, out=out, qk_fp8=q8, recall=rec)
 
     # stats (outside timing): kept pairs, skipped P.V, algorithmic FLOPs of the forward
     stats = torch.zeros(4, dtype=torch.int64, device=dev)
     sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False, quantize=q8)
-    sa.sparse_attn_fwd(q, k, v, plan, lam, out=out, stats=stats, qk_fp8=q8)
+    sa.sparse_attn_fwd(q, k, v, plan, lam, out=out, stats=stats, qk_fp8=q8, recall=rec)
     torch.cuda.synchronize()
     check_device(sa, "the stats pass")
     st = [int(x) for x in stats.cpu()]
@@ -332,7 +345,7 @@ def run_ours(args, w, world, rank, local, pg):
         sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False, quantize=q8)
 
     def run_fwd():
-        sa.sparse_attn_fwd(q, k, v, plan, lam, out=out, qk_fp8=q8)
+        sa.sparse_attn_fwd(q, k, v, plan, lam, out=out, qk_fp8=q8, recall=rec)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -385,7 +398,8 @@ def run_ours(args, w, world, rank, local, pg):
         # warm-up calls exactly like the timed ones, so that the caching pinned
         # allocator holds the output blocks the timed calls cycle through
         for _ in range(max(3, args.warmup)):
-            o_host = sa.sparse_attention(qh, kh, vh, args.tau, lam, None, w.causal, device=dev, qk_fp8=q8)
+            o_host = sa.sparse_attention(qh, kh, vh, args.tau, lam, None, w.causal, device=dev, qk_fp8=q8,
+                                             recall=rec)
             torch.cuda.synchronize()
         barrier(pg, dev)
         t = []
@@ -393,7 +407,8 @@ def run_ours(args, w, world, rank, local, pg):
             flush.zero_()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            o_host = sa.sparse_attention(qh, kh, vh, args.tau, lam, None, w.causal, device=dev, qk_fp8=q8)
+            o_host = sa.sparse_attention(qh, kh, vh, args.tau, lam, None, w.causal, device=dev, qk_fp8=q8,
+                                             recall=rec)
             b.record(stream)
             torch.cuda.synchronize()
             t.append(a.elapsed_time(b))
@@ -430,20 +445,21 @@ def run_ours(args, w, world, rank, local, pg):
         "config": config_dict(w, args, world),
         "plan_ms": plan_avg, "fwd_ms": fwd_avg, "dense_fwd_ms": dense_ms,
         "sparsity_pct": 100.0 * (1.0 - kept_pairs / total_pairs),
-        "lambda_skip_pct": 100.0 * skipped / max(kept_pairs, 1),
+        "lambda_skip_pct" if rec is None else "recall_skip_pct": 100.0 * skipped / max(kept_pairs, 1),
         "executed_tflops": achieved, "pct_of_bf16_peak_executed": 100.0 * achieved / peak_t,
         "predictor_pct_of_dense": None if dense_ms is None else 100.0 * plan_avg / dense_ms,
         "predictor": {"bound": "hbm", "achieved": pred_gbs, "peak": hbm, "unit": "GB/s", "frac": pred_gbs / hbm,
                       "bytes": pred_bytes, "peak_source": f"{pk_kind} hbm_gbs"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
-                     "frac": achieved / peak_t, "traffic": measured_traffic(w, args.tau, lam, args.qk),
+                     "frac": achieved / peak_t, "traffic": measured_traffic(w, args.tau, lam, args.qk, rec),
                      "kernel": f"fwd_kernel<{D}, fp8 scores> (sparse_attn_fwd_q8)" if q8
-                     else f"fwd_kernel<{D}> (sparse_attn_fwd)",
+                     else (f"fwd_kernel<{D}, recall filter> (sparse_attn_fwd_recall)" if rec is not None
+                           else f"fwd_kernel<{D}> (sparse_attn_fwd)"),
                      "peak_source": peak_source},
         "e2e": e2e, "gpu_launches": 4 * args.steps, "cuda_graphs": not args.no_graph, "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu:
-        v_cpu, t_cpu, cores, sample = time_oracle(w, args.tau, lam, args.cpu_seconds, args.seed)
+        v_cpu, t_cpu, cores, sample = time_oracle(w, args.tau, lam, args.cpu_seconds, args.seed, rec)
         line["cpu_baseline"] = {"value": v_cpu, "unit": UNIT, "cores": cores, "kind": "oracle",
                                 "sample": sample, "seconds": t_cpu}
     if rank == 0:

@@ -24,7 +24,7 @@ from ._lib import SaShape, SparseAttnError
 
 BLOCK = 64
 
-__all__ = ["Plan", "sparse_attn_plan", "sparse_attn_fwd", "sparse_attention",
+__all__ = ["Plan", "sparse_attn_plan", "sparse_attn_fwd", "sparse_attn_fwd_recall", "sparse_attention",
            "sparse_attn_plan_workspace_size", "sparse_attn_num_tiles", "sparse_attn_device_error",
            "sparse_attn_selftest_wait_timeout",
            "SparseAttnError", "BLOCK"]
@@ -164,13 +164,16 @@ def sparse_attn_plan(q: torch.Tensor, k: torch.Tensor, tau, scale: Optional[floa
 def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan, lam: Optional[float] = None,
                     scale: Optional[float] = None, causal: Optional[bool] = None, *,
                     out: Optional[torch.Tensor] = None, stats: Optional[torch.Tensor] = None,
-                    qk_fp8: bool = False) -> torch.Tensor:
+                    qk_fp8: bool = False, recall: Optional[float] = None) -> torch.Tensor:
     """Stage 2: attention over the kept blocks with the lambda P.V filter.
 
     `plan` is a Plan or a uint8 mask [B, H, Nb, Nb]. lam=None turns the filter off.
     `stats`, if given, is an int64 CUDA tensor of 4 entries (see the C header).
     qk_fp8=True takes the scores on the plan's FP8 copies of q and k
-    (sparse_attn_fwd_q8; the plan must come from sparse_attn_plan(quantize=True))."""
+    (sparse_attn_fwd_q8; the plan must come from sparse_attn_plan(quantize=True)).
+    recall=rho (in (0, 1]) replaces the lambda test by the cumulative-energy test
+    of sparse_attn_fwd_recall: every row keeps at least the fraction rho of the
+    softmax energy of the blocks it visits; lam must then be None."""
     lib = _lib.load()
     _check_qkv(q, k, v)
     B, H, N, d = q.shape
@@ -194,6 +197,15 @@ def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan, lam
         out = torch.empty_like(q)
     if stats is not None and (stats.dtype != torch.int64 or stats.numel() < 4 or stats.device != q.device):
         raise ValueError("stats must be an int64 tensor of >= 4 entries on q's device")
+    if recall is not None:
+        if lam is not None or qk_fp8:
+            raise ValueError("recall replaces the lambda filter and takes bf16 scores: "
+                             "pass lam=None and qk_fp8=False with it")
+        st = lib.sparse_attn_fwd_recall(_ptr(q), _ptr(k), _ptr(v), _shape(q), _ptr(mask), _ptr(work),
+                                        float(recall), float(scale), int(causal), _ptr(out), _ptr(stats),
+                                        _stream(q.device))
+        _call("sparse_attn_fwd_recall", st)
+        return out
     if qk_fp8:
         if not isinstance(plan, Plan) or plan.q8 is None:
             raise ValueError("qk_fp8=True needs a plan made with quantize=True")
@@ -206,6 +218,15 @@ def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan, lam
                              float(scale), int(causal), _ptr(out), _ptr(stats), _stream(q.device))
     _call("sparse_attn_fwd", st)
     return out
+
+
+def sparse_attn_fwd_recall(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan, recall: float,
+                           scale: Optional[float] = None, causal: Optional[bool] = None, *,
+                           out: Optional[torch.Tensor] = None,
+                           stats: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Stage 2 with the cumulative-energy P.V filter (the C call of the same name):
+    sparse_attn_fwd(q, k, v, plan, None, scale, causal, recall=recall, ...)."""
+    return sparse_attn_fwd(q, k, v, plan, None, scale, causal, out=out, stats=stats, recall=recall)
 
 
 _COPY_STREAMS = {}
@@ -223,7 +244,7 @@ def _copy_streams(dev: torch.device):
 def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau,
                      lam: Optional[float] = None, scale: Optional[float] = None, causal: bool = False,
                      device="cuda", out: Optional[torch.Tensor] = None, chunks: Optional[int] = None,
-                     qk_fp8: bool = False) -> torch.Tensor:
+                     qk_fp8: bool = False, recall: Optional[float] = None) -> torch.Tensor:
     """End to end from host tensors: copy q, k, v to the GPU, plan + forward, copy O back.
 
     Host inputs should be pinned, so the copies are asynchronous DMA. The result is
@@ -235,7 +256,8 @@ def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau,
     device-to-host copy run on three streams, so the copies of one group overlap
     the work of the others in both directions of the link. tau may be one value or
     a per-head float32 tensor ([B, H] or [H]) on `device`. qk_fp8=True takes the
-    scores on FP8 copies of q and k (see sparse_attn_plan's quantize)."""
+    scores on FP8 copies of q and k (see sparse_attn_plan's quantize); recall
+    selects the cumulative-energy P.V filter instead of lambda (see sparse_attn_fwd)."""
     dev = torch.device(device)
     if q.shape != k.shape or q.shape != v.shape or q.dim() != 4:
         raise ValueError("q, k, v must share the shape [B, H, N, d]")
@@ -268,7 +290,8 @@ def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau,
         view = lambda x: x[lo:hi].view(1, hi - lo, N, d)
         t = tau[lo:hi].view(1, hi - lo) if isinstance(tau, torch.Tensor) else tau
         plan = sparse_attn_plan(view(qd), view(kd), t, scale, causal, with_idx=False, quantize=qk_fp8)
-        sparse_attn_fwd(view(qd), view(kd), view(vd), plan, lam, scale, causal, out=view(od), qk_fp8=qk_fp8)
+        sparse_attn_fwd(view(qd), view(kd), view(vd), plan, lam, scale, causal, out=view(od), qk_fp8=qk_fp8,
+                        recall=recall)
         done = torch.cuda.Event()
         done.record(main)
         d2h.wait_event(done)

@@ -31,6 +31,7 @@ EXPORTS = (
     "sparse_attn_plan_noalloc",
     "sparse_attn_plan_q8",
     "sparse_attn_fwd_q8",
+    "sparse_attn_fwd_recall",
     "sparse_attn_selftest_wait_timeout",
 )
 
@@ -86,6 +87,8 @@ def load(path: str = LIB_PATH):
     lib.sparse_attn_plan_q8.restype = i32
     lib.sparse_attn_fwd_q8.argtypes = [vp, vp, vp, vp, vp, SaShape, vp, vp, f32, f32, i32, vp, vp, vp]
     lib.sparse_attn_fwd_q8.restype = i32
+    lib.sparse_attn_fwd_recall.argtypes = [vp, vp, vp, SaShape, vp, vp, f32, f32, i32, vp, vp, vp]
+    lib.sparse_attn_fwd_recall.restype = i32
     lib.sparse_attn_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp]
     lib.sparse_attn_selftest_wait_timeout.restype = i32
     _lib = lib

@@ -53,6 +53,8 @@
 // entry index as a tag, and a vote slot is reused for entry k+2 only after every
 // softmax warp has released S(k+1), which each does after reading entry k's vote
 // (a warp whose own rows do not all pass cannot skip and does not read it).
+// The recall filter (kRecall, below) uses the same slots, posting its vote after
+// the exponentials instead; the argument is unchanged.
 #pragma once
 
 #include "sa_device.cuh"
@@ -121,14 +123,23 @@ __device__ __forceinline__ float softmax_exp64(const float (&s)[64], float scale
   return (r0 + r1) + (r2 + r3);
 }
 
-template <int D, bool kF8>
+// kRecall: the P.V filter is the cumulative-energy (recall) test instead of the
+// lambda test. Each row keeps, beside its running sum l (the energy of the keys
+// it has seen, relative to the reference max), the part sk of l whose P.V was
+// skipped. A half skips P.V of entry k when each of its rows that sees a key of
+// the block has sk*alpha + e <= budget * (l*alpha + e), e = the row's sum of P(k)
+// and budget = 1 - recall; then sk takes e. So sk <= budget * l throughout and
+// every row keeps at least the fraction `recall` of the energy it has seen. The
+// vote needs e, so it is posted after the exponentials; the exchange is the
+// lambda vote's.
+template <int D, bool kF8, bool kRecall = false>
 __global__ void __launch_bounds__(192, 2)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const uint8_t* __restrict__ mask,
                const int* __restrict__ work, __nv_bfloat16* __restrict__ O, int N, int Nb, int Tq,
                long long num_tiles, long long num_qblocks, float scale_log2, float lam_log2, int lam_on,
-               int causal, unsigned long long* __restrict__ stats, const float* __restrict__ qscale,
-               const float* __restrict__ kscale) {
+               float budget, int causal, unsigned long long* __restrict__ stats,
+               const float* __restrict__ qscale, const float* __restrict__ kscale) {
   using C = FwdCfg<D, kF8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -372,6 +383,7 @@ __global__ void __launch_bounds__(192, 2)
     const float sqh = kF8 ? (myqb >= 0 ? qscale[bh * Nb + myqb] : 1.f) : 1.f;
     const unsigned FULL = 0xffffffffu;
     float m_true = -INFINITY, m_ref = -INFINITY, l = 0.f;
+    float sk = 0.f;                              // kRecall: skipped part of l
     unsigned long long kept_pairs = 0, skipped_pairs = 0;
     bool alive = true;
     // S(k) is loaded from TMEM one entry ahead: the load of S(k+1) is issued while
@@ -425,7 +437,7 @@ __global__ void __launch_bounds__(192, 2)
                sc;                                // -inf stays -inf (sc > 0)
       }
       bool wpass = true;
-      if (lam_on) {
+      if (!kRecall && lam_on) {
         // this warp's lambda vote, posted before the exponentials so that the other
         // warp of the half finds it when it needs it
         const bool pass = !(rmax > -INFINITY) || (rmax - m_true < lam_log2);
@@ -450,7 +462,15 @@ __global__ void __launch_bounds__(192, 2)
       }
       m_true = m_new;
       l = l * alpha + psum;
-      // lambda: the half skips P.V when both of its warps pass; its P(k) is zero
+      float sk_try = 0.f;
+      if (kRecall) {
+        // this warp's recall vote (rows that see no key of the block have no say)
+        sk_try = sk * alpha + psum;
+        const bool pass = ncol == 0 || sk_try <= budget * l;
+        wpass = __all_sync(FULL, pass);
+        if (lane == 0) votes[(k & 1) * 4 + wq] = (k << 1) | (wpass ? 1 : 0);
+      }
+      // the half skips P.V when both of its warps pass; its P(k) is zero
       bool half_skip = false;
       if (lam_on && wpass) {                      // a warp that does not pass never skips
         int pv = 0;
@@ -463,6 +483,7 @@ __global__ void __launch_bounds__(192, 2)
           for (int c = 0; c < 32; ++c) pk[c] = 0u;
         }
       }
+      if (kRecall) sk = half_skip ? sk_try : sk * alpha;
       // P(k) into buffer k&1 once its previous reader, P(k-2).V, has finished
       if (k >= 2) {
         if (!warp_wait(&pv_done[k & 1], static_cast<uint32_t>((k - 2) >> 1) & 1u, abort_flag)) {

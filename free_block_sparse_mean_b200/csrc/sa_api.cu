@@ -154,10 +154,12 @@ sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau
   return SA_OK;
 }
 
-template <int D, bool kF8 = false>
+// kRecall: the P.V filter is the recall test with budget = 1 - recall (lambda unused).
+template <int D, bool kF8 = false, bool kRecall = false>
 sa_status launch_fwd(const sa_shape& s, const void* Q, const void* K, const void* V, const uint8_t* mask,
                      const int32_t* work, float lambda, float scale, int causal, void* O, int64_t* stats,
-                     cudaStream_t st, const float* qscale = nullptr, const float* kscale = nullptr) {
+                     cudaStream_t st, const float* qscale = nullptr, const float* kscale = nullptr,
+                     float budget = 0.f) {
   using Cfg = sa::FwdCfg<D, kF8>;
   const int Nb = static_cast<int>(num_blocks(s));
   const int Tq = (Nb + 1) / 2;
@@ -171,15 +173,15 @@ sa_status launch_fwd(const sa_shape& s, const void* Q, const void* K, const void
   }
   if (!make_block_map(&mv, V, s)) return SA_ERR_CUDA;
   if (stats && cudaMemsetAsync(stats, 0, 4 * sizeof(int64_t), st) != cudaSuccess) return SA_ERR_CUDA;
-  auto kern = sa::fwd_kernel<D, kF8>;
+  auto kern = sa::fwd_kernel<D, kF8, kRecall>;
   if (set_smem(kern, Cfg::kSmemBytes) != SA_OK) return SA_ERR_CUDA;
   const float LOG2E = 1.4426950408889634f;
-  const int lam_on = std::isinf(lambda) && lambda < 0 ? 0 : 1;
+  const int lam_on = kRecall ? 1 : (std::isinf(lambda) && lambda < 0 ? 0 : 1);
   kern<<<static_cast<unsigned>(tiles), Cfg::kThreads, Cfg::kSmemBytes, st>>>(
       mq, mk, mv, mask, work, static_cast<__nv_bfloat16*>(O), s.N, Nb, Tq, tiles,
       static_cast<long long>(s.B) * s.H * Nb, scale * LOG2E,
-      lam_on ? lambda * LOG2E : 0.f, lam_on, causal, reinterpret_cast<unsigned long long*>(stats), qscale,
-      kscale);
+      (lam_on && !kRecall) ? lambda * LOG2E : 0.f, lam_on, budget, causal,
+      reinterpret_cast<unsigned long long*>(stats), qscale, kscale);
   if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   return SA_OK;
 }
@@ -265,6 +267,25 @@ sa_status sparse_attn_fwd(const void* Q, const void* K, const void* V, sa_shape 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (s.d == 64) return launch_fwd<64>(s, Q, K, V, mask, work, lambda, scale, causal != 0, O, stats, st);
   return launch_fwd<128>(s, Q, K, V, mask, work, lambda, scale, causal != 0, O, stats, st);
+}
+
+sa_status sparse_attn_fwd_recall(const void* Q, const void* K, const void* V, sa_shape s, const uint8_t* mask,
+                                 const int32_t* work, float recall, float scale, int32_t causal, void* O,
+                                 int64_t* stats, void* stream) {
+  if (!Q || !K || !V || !mask || !O) return SA_ERR_INVALID_ARG;
+  const sa_status sh = check_shape(s);
+  if (sh != SA_OK) return sh;
+  if (!(recall > 0.f && recall <= 1.f)) return SA_ERR_INVALID_ARG;  // also rejects NaN
+  if (!(std::isfinite(scale) && scale > 0.f)) return SA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SA_ERR_INVALID_ARG;
+  if (stats && (reinterpret_cast<uintptr_t>(stats) & 7u) != 0) return SA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const float budget = 1.f - recall;
+  if (s.d == 64)
+    return launch_fwd<64, false, true>(s, Q, K, V, mask, work, 0.f, scale, causal != 0, O, stats, st, nullptr,
+                                       nullptr, budget);
+  return launch_fwd<128, false, true>(s, Q, K, V, mask, work, 0.f, scale, causal != 0, O, stats, st, nullptr,
+                                      nullptr, budget);
 }
 
 const char* sparse_attn_status_string(sa_status st) {

@@ -144,6 +144,29 @@ sa_status sparse_attn_fwd(const void* Q, const void* K, const void* V, sa_shape 
                           const uint8_t* mask, const int32_t* work, float lambda, float scale,
                           int32_t causal, void* O, int64_t* stats, void* stream);
 
+/* Stage 2 with the in-operator cumulative-energy P.V filter instead of the lambda
+ * test (DynSparse article: keep a fixed recall of the attention energy, with a
+ * threshold that follows the cumulative energy the FlashAttention operator
+ * already holds; the formula below is this library's reading of it).
+ *
+ *   recall    in (0, 1]. Per row r, l_r is the running softmax sum (the energy of
+ *             the keys seen so far) and sk_r the part of it whose P.V was skipped,
+ *             both relative to the running max. For each query block and kept key
+ *             block (ascending order), with e_r the block's energy in row r and
+ *             alpha_r the rescale to the new running max, the block's P.V is
+ *             skipped when every row that sees a key of the block has
+ *             sk_r*alpha_r + e_r <= (1 - recall) * (l_r*alpha_r + e_r); the
+ *             block always enters l, and enters sk only when skipped. Every row
+ *             then keeps at least the fraction `recall` of the energy of the
+ *             blocks it visits. recall = 1 skips only blocks of zero energy.
+ *             NaN or a value outside (0, 1] is rejected.
+ *   stats     as sparse_attn_fwd; entry 1 counts the pairs skipped by this test.
+ *
+ * All other arguments, outputs and errors are those of sparse_attn_fwd. */
+sa_status sparse_attn_fwd_recall(const void* Q, const void* K, const void* V, sa_shape s,
+                                 const uint8_t* mask, const int32_t* work, float recall, float scale,
+                                 int32_t causal, void* O, int64_t* stats, void* stream);
+
 /* Quantized scores (SpargeAttn: "sparse and quantized"; the quantization scheme
  * is this library's own, the pages give none). sparse_attn_plan that also writes
  * FP8 E4M3 copies of Q and K from the same pass over them:

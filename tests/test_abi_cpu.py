@@ -124,6 +124,20 @@ def test_q8_entry_points_reject_bad_arguments(lib):
     assert fwd(s=s64) == 2
 
 
+def test_recall_forward_rejects_bad_arguments(lib):
+    s = SaShape(1, 2, 128, 128, 64)
+
+    def fwd(s=s, K=FAKE, O=FAKE, recall=0.95, stats=None):
+        return lib.sparse_attn_fwd_recall(FAKE, K, FAKE, s, FAKE, None, recall, 0.1, 0, O, stats, None)
+
+    assert fwd(K=None) == 1 and fwd(O=None) == 1
+    for bad in (0.0, -0.5, 1.0001, float("nan"), float("inf")):
+        assert fwd(recall=bad) == 1, bad
+    assert fwd(stats=ctypes.c_void_p(0x10004)) == 1                 # stats must be 8-byte aligned
+    assert fwd(K=FAKE_ODD) == 1
+    assert fwd(s=SaShape(1, 2, 128, 96, 64)) == 2                   # d in {64, 128}
+
+
 def test_device_error_needs_output_pointer(lib):
     assert lib.sparse_attn_device_error(None, None) == 1
 
