@@ -46,9 +46,28 @@ of x * (448 / max|x|) computed in fp32 (the kernel's precision for this integer
 decision), ties to even, saturating. The scores are then the dequantized
 (code * s) products; V, P and the rest of the attention are unchanged.
 
+Clustered variant (iCATS abstract: clustering of query and key tokens "based on
+query-key dot-product interactions", reformulated "as a simple quadratic form";
+the abstract gives no formula, so this is a reading, pinned by the tests):
+  * replacing a query q by a centroid c changes its dot products with every key
+    k by (q - c).k, and the sum of their squares over the keys is the quadratic
+    form (q - c)^T G_K (q - c) with G_K = sum_k k k^T, the keys' Gram matrix; the
+    queries are clustered by k-means under that distance, the keys likewise
+    under G_Q = sum_q q q^T;
+  * ceil(N/64) clusters per side, initialised to the 64-token block means (so
+    zero iterations is the plain block pooling); Lloyd iterations assign each
+    token to the nearest centroid (ties: lowest cluster index) and move each
+    centroid to the mean of its tokens (a cluster left empty keeps its centroid);
+  * tokens are then reordered by cluster (stable: ascending token index within a
+    cluster) and the clusters packed back to back, so the tail of one cluster
+    shares a 64-token block with the head of the next instead of being padded
+    ("tail merging"); the plan and the forward run on the reordered Q, K, V and
+    the output rows are put back in token order. Non-causal only.
+
 Entry points: block_mean_pool, pooled_logits, pooled_softmax,
 cumulative_energy_select, plan, attention_masked, attention_tiled,
-attention_recall, fwd, round_e4m3, quantize_blocks_e4m3, fwd_fp8qk.
+attention_recall, fwd, round_e4m3, quantize_blocks_e4m3, fwd_fp8qk, gram, interaction_distance,
+kmeans_interaction, cluster_permutation, clustered_attention.
 """
 from __future__ import annotations
 
@@ -424,3 +443,88 @@ def fwd_fp8qk(Q, K, V, mask, lam: Optional[float] = None, scale: Optional[float]
     Kd = ck * sk[:, :, tok][..., None]
     return fwd(Qd, Kd, V, mask, lam, scale, causal, block, qblocks)
 
+
+
+# ----------------------------------------------------------------------------
+# Clustering by query-key interaction (see the module docstring)
+
+def gram(Y) -> np.ndarray:
+    """Gram matrix sum_t y_t y_t^T of the tokens of Y [..., N, d]: [..., d, d]."""
+    Y = as_f64(Y)
+    return np.swapaxes(Y, -1, -2) @ Y
+
+
+def interaction_distance(X, C, G) -> np.ndarray:
+    """(x - c)^T G (x - c) for every token x of X [..., N, d] and centroid c of
+    C [..., M, d] under G [..., d, d]: [..., N, M]. Expanded as
+    x^T G x - 2 x^T G c + c^T G c (the tests check it against the sum over the
+    other side's tokens of ((x - c).y)^2)."""
+    X, C, G = as_f64(X), as_f64(C), as_f64(G)
+    XG = X @ G
+    xx = np.sum(XG * X, axis=-1)[..., :, None]
+    cc = np.sum((C @ G) * C, axis=-1)[..., None, :]
+    return xx - 2.0 * XG @ np.swapaxes(C, -1, -2) + cc
+
+
+def kmeans_interaction(X, Y, iters: int, block: int = BLOCK):
+    """k-means of the tokens of X [B, H, N, d] under the metric G = gram(Y) of the
+    other side, per (batch, head): ceil(N/block) clusters, initialised to the
+    block means, `iters` Lloyd iterations. Returns (assign int64 [B, H, N],
+    centroids [B, H, C, d], objective list of length iters + 1: the sum over the
+    tokens of the distance to their centroid, after the initial assignment to
+    the blocks and after each iteration)."""
+    X, Y = as_f64(X), as_f64(Y)
+    B, H, N, d = X.shape
+    nc = n_blocks(N, block)
+    G = gram(Y)
+    cent = block_mean_pool(X, block)
+    assign = np.broadcast_to(np.arange(N) // block, (B, H, N)).copy()
+
+    def objective(a, c):
+        dist = interaction_distance(X, c, G)
+        return float(np.take_along_axis(dist, a[..., None], axis=-1).sum())
+
+    obj = [objective(assign, cent)]
+    for _ in range(iters):
+        dist = interaction_distance(X, cent, G)
+        assign = np.argmin(dist, axis=-1)                  # first minimum: lowest index
+        new = cent.copy()
+        for b in range(B):
+            for h in range(H):
+                for c in range(nc):
+                    members = assign[b, h] == c
+                    if members.any():
+                        new[b, h, c] = X[b, h, members].mean(axis=0)
+        cent = new
+        obj.append(objective(assign, cent))
+    return assign, cent, obj
+
+
+def cluster_permutation(assign) -> np.ndarray:
+    """perm[..., p] = the token at position p once the tokens are ordered by
+    cluster, ascending token index within a cluster (a stable sort)."""
+    return np.argsort(np.asarray(assign), axis=-1, kind="stable")
+
+
+def clustered_attention(Q, K, V, tau, lam: Optional[float] = None, iters: int = 2,
+                        scale: Optional[float] = None, block: int = BLOCK, perms=None):
+    """Plan + forward on tokens reordered by interaction clustering, output in
+    token order. Queries are clustered under gram(K), keys under gram(Q); K and V
+    share the key order. `perms` = (perm_q, perm_k) replaces the clustering (for
+    checking an output against a given ordering). Returns (O [B, H, N, d], dict
+    with perm_q, perm_k, the plan on the reordered tokens)."""
+    Q, K, V = as_f64(Q), as_f64(K), as_f64(V)
+    if perms is None:
+        aq, _, _ = kmeans_interaction(Q, K, iters, block)
+        ak, _, _ = kmeans_interaction(K, Q, iters, block)
+        pq, pk = cluster_permutation(aq), cluster_permutation(ak)
+    else:
+        pq, pk = (np.asarray(p, dtype=np.int64) for p in perms)
+    Qs = np.take_along_axis(Q, pq[..., None], axis=2)
+    Ks = np.take_along_axis(K, pk[..., None], axis=2)
+    Vs = np.take_along_axis(V, pk[..., None], axis=2)
+    p = plan(Qs, Ks, tau, scale, False, block)
+    Os = fwd(Qs, Ks, Vs, p["mask"], lam, scale, False, block)
+    O = np.empty_like(Os)
+    np.put_along_axis(O, pq[..., None], Os, axis=2)
+    return O, dict(perm_q=pq, perm_k=pk, plan=p)

@@ -541,3 +541,119 @@ def test_fwd_fp8qk_is_fwd_when_q_and_k_are_representable():
     Qg, Kg = r.standard_normal((1, 2, 192, 8)), r.standard_normal((1, 2, 192, 8))
     a, b = orc.fwd_fp8qk(Qg, Kg, V, mask), orc.fwd(Qg, Kg, V, mask)
     assert 0 < np.abs(a - b).max() < 0.1
+
+
+# ---------------------------------------------------------------- interaction clustering
+def test_interaction_distance_is_the_summed_squared_score_change():
+    """Replacing x by c changes its score with every token y of the other side by
+    (x - c).y; the quadratic form under the other side's Gram matrix is the sum
+    of the squares of those changes (brute force over y)."""
+    r = _rng(21)
+    X, C, Y = r.standard_normal((1, 1, 7, 5)), r.standard_normal((1, 1, 3, 5)), r.standard_normal((1, 1, 11, 5))
+    D = orc.interaction_distance(X, C, orc.gram(Y))
+    for n in range(7):
+        for m in range(3):
+            brute = sum(float(np.dot(X[0, 0, n] - C[0, 0, m], Y[0, 0, t])) ** 2 for t in range(11))
+            assert D[0, 0, n, m] == pytest.approx(brute, rel=1e-12)
+
+
+def test_kmeans_metric_comes_from_the_other_side():
+    """Keys all along e1 (G_K = 64 e1 e1^T): a query differing from a centroid
+    only in e2 is at distance 0 from it, whatever the Euclidean distance. Query
+    block 0 holds x = (0, 10) and 63 copies of (0, 0); block 1 holds (0.9, 10)
+    x 64. Under the key metric x joins block 0's cluster (distance 0 against
+    0.81 * 64 to the other); under the Euclidean or the query-side metric it
+    would join block 1's."""
+    d = 2
+    Q = np.zeros((1, 1, 128, d))
+    Q[0, 0, 0] = [0.0, 10.0]
+    Q[0, 0, 64:] = [0.9, 10.0]
+    K = np.zeros((1, 1, 128, d)); K[..., 0] = 1.0
+    a, c, _ = orc.kmeans_interaction(Q, K, 1)
+    assert a[0, 0, 0] == 0 and np.all(a[0, 0, 1:64] == 0) and np.all(a[0, 0, 64:] == 1)
+    a_wrong, _, _ = orc.kmeans_interaction(Q, Q, 1)       # query-side metric
+    assert a_wrong[0, 0, 0] == 1
+
+
+def test_kmeans_separates_two_interleaved_groups_in_one_iteration():
+    """Tokens equal to a or b (a - b not in the null space of G): block 0 holds 48
+    a and 16 b, block 1 16 a and 48 b, interleaved. The initial centroids are
+    (3a + b)/4 and (a + 3b)/4, so one iteration sends every a to cluster 0 and
+    every b to cluster 1, and the centroids become a and b exactly. The order puts
+    the a tokens first, each group in token order."""
+    r = _rng(5)
+    d = 6
+    a_vec, b_vec = r.standard_normal(d), r.standard_normal(d)
+    is_a = np.zeros(128, dtype=bool)
+    is_a[np.arange(0, 64)[np.arange(64) % 4 != 3]] = True      # 48 of block 0
+    is_a[64 + np.arange(0, 64, 4)] = True                       # 16 of block 1
+    X = np.where(is_a[:, None], a_vec, b_vec)[None, None]
+    Y = r.standard_normal((1, 1, 128, d))
+    a, c, obj = orc.kmeans_interaction(X, Y, 1)
+    np.testing.assert_array_equal(a[0, 0], np.where(is_a, 0, 1))
+    np.testing.assert_allclose(c[0, 0], np.stack([a_vec, b_vec]), rtol=1e-14, atol=1e-14)
+    perm = orc.cluster_permutation(a)[0, 0]
+    np.testing.assert_array_equal(perm, np.concatenate([np.nonzero(is_a)[0], np.nonzero(~is_a)[0]]))
+    assert obj[1] == pytest.approx(0.0, abs=1e-9) and obj[0] > 0
+
+
+@pytest.mark.parametrize("N", [300, 256])
+def test_kmeans_objective_never_increases(N):
+    """Lloyd iterations under a positive semi-definite metric: the assignment step
+    and the mean step (the minimiser of the cluster's summed quadratic form) can
+    only lower the objective."""
+    r = _rng(N)
+    X, Y = r.standard_normal((1, 2, N, 8)) + np.linspace(0, 3, N)[None, None, :, None], r.standard_normal((1, 2, N, 8))
+    _, _, obj = orc.kmeans_interaction(X, Y, 5)
+    assert all(b <= a * (1 + 1e-12) for a, b in zip(obj, obj[1:]))
+    assert obj[-1] < obj[0]
+
+
+def test_zero_iterations_is_block_pooling():
+    r = _rng(8)
+    Q, K, V = (r.standard_normal((1, 2, 200, 8)) for _ in range(3))
+    a, c, _ = orc.kmeans_interaction(Q, K, 0)
+    np.testing.assert_array_equal(a[0, 1], np.arange(200) // 64)
+    np.testing.assert_allclose(c, orc.block_mean_pool(Q), rtol=0, atol=0)
+    O, info = orc.clustered_attention(Q, K, V, 0.9, None, 0)
+    p = orc.plan(Q, K, 0.9)
+    np.testing.assert_allclose(O, orc.fwd(Q, K, V, p["mask"]), rtol=1e-13, atol=1e-14)
+
+
+@pytest.mark.parametrize("iters", [1, 3])
+def test_clustered_attention_with_every_block_kept_is_dense(iters):
+    """Attention is invariant under a common reordering of K and V, and reordering
+    the queries only moves the output rows: with tau = 1 every block is kept, so
+    the clustered path must give dense attention in token order (pins the
+    gathers and the scatter back)."""
+    r = _rng(30 + iters)
+    N, d = 320, 8
+    Q = r.standard_normal((1, 2, N, d)) + np.sin(np.arange(N) / 7.0)[None, None, :, None]
+    K, V = r.standard_normal((1, 2, N, d)), r.standard_normal((1, 2, N, d))
+    O, info = orc.clustered_attention(Q, K, V, 1.0, None, iters)
+    assert not np.array_equal(info["perm_q"][0, 0], np.arange(N))      # the order did change
+    np.testing.assert_allclose(O, _sdpa64(Q, K, V, False, 1.0 / math.sqrt(d)), rtol=1e-11, atol=1e-12)
+
+
+def test_clustered_attention_uses_each_side_under_the_others_metric():
+    """The set-up of test_kmeans_metric_comes_from_the_other_side on each side in
+    turn. Side A: token 0 = (0, 10), tokens 1..63 = 0, tokens 64..127 = (0.9, 10);
+    side B: every token (1, 0). Clustered under side B's metric, side A keeps
+    the identity order (token 0 stays with block 0); under its own metric token 0
+    would move to the second cluster. Side B's tokens are all equal, so its order
+    is the identity too (ties go to the first cluster). Checked with A as the
+    queries and with A as the keys."""
+    A = np.zeros((1, 1, 128, 2))
+    A[0, 0, 0] = [0.0, 10.0]
+    A[0, 0, 64:] = [0.9, 10.0]
+    Bside = np.zeros((1, 1, 128, 2)); Bside[..., 0] = 1.0
+    V = _rng(2).standard_normal((1, 1, 128, 2))
+    ident = np.arange(128)
+    _, info = orc.clustered_attention(A, Bside, V, 0.9, None, 1)
+    np.testing.assert_array_equal(info["perm_q"][0, 0], ident)
+    np.testing.assert_array_equal(info["perm_k"][0, 0], ident)
+    _, info = orc.clustered_attention(Bside, A, V, 0.9, None, 1)
+    np.testing.assert_array_equal(info["perm_k"][0, 0], ident)
+    np.testing.assert_array_equal(info["perm_q"][0, 0], ident)
+    moved = orc.cluster_permutation(orc.kmeans_interaction(A, A, 1)[0])[0, 0]
+    assert moved[63] == 0                                     # own metric: token 0 leaves block 0
