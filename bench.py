@@ -62,6 +62,9 @@ def parse():
     ap.add_argument("--recall", type=float, default=None,
                     help="P.V filter: the cumulative-energy test keeping this recall per row "
                          "(sparse_attn_fwd_recall) instead of the lambda test")
+    ap.add_argument("--cluster-iters", type=int, default=None,
+                    help="reorder the tokens by interaction clustering (this many k-means iterations) "
+                         "before the plan, and the output back after the forward (non-causal workloads)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch plan and forward directly instead of replaying CUDA graphs")
     return ap.parse_args()
@@ -192,7 +195,7 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- CPU oracle timing
-def time_oracle(w, tau, lam, budget_s, seed, recall=None):
+def time_oracle(w, tau, lam, budget_s, seed, recall=None, cluster_iters=None):
     """The oracle as it stands (fp64 NumPy) on a bounded sample of the workload:
     whole heads (plan + forward) until the time budget is used, at least one."""
     from oracle import sparse_attn_oracle as orc
@@ -212,6 +215,14 @@ def time_oracle(w, tau, lam, budget_s, seed, recall=None):
     for h in range(w.H):
         q, k, v = wl.generate(w, seed=seed, device="cpu", heads=[h])
         t0 = time.perf_counter()
+        if cluster_iters is not None:      # clustering, plan and forward of whole heads
+            orc.clustered_attention(q, k, v, tau, lam, cluster_iters)
+            t_total += time.perf_counter() - t0
+            flops += per_head_dense
+            heads += 1
+            if t_total >= budget_s:
+                break
+            continue
         p = orc.plan(q, k, tau, None, w.causal)
         if recall is not None:
             orc.attention_recall(q, k, v, p["mask"], recall, None, w.causal, qblocks=qblocks)
@@ -226,6 +237,8 @@ def time_oracle(w, tau, lam, budget_s, seed, recall=None):
         heads += 1
         if t_total >= budget_s:
             break
+    if cluster_iters is not None:
+        return flops / t_total / 1e12, t_total, cores, f"{heads} of {w.H} heads, clustering + plan + forward"
     sample = (f"{heads} of {w.H} heads, full plan"
               + ("" if qblocks is None else f", forward on {len(qblocks)} of {-(-w.N // 64)} query blocks"))
     return flops / t_total / 1e12, t_total, cores, sample
@@ -240,7 +253,7 @@ def run_reference(args, w, world, rank, pg):
     vals = []
     budget = max(2.0, min(args.cpu_seconds, 240.0 / max(1, args.steps + args.warmup)))
     for i in range(args.warmup + args.steps):
-        v, t, cores, sample = time_oracle(w, args.tau, lam, budget, args.seed, args.recall)
+        v, t, cores, sample = time_oracle(w, args.tau, lam, budget, args.seed, args.recall, args.cluster_iters)
         if i >= args.warmup:
             per_step.append(t)
             vals.append(v)
@@ -264,6 +277,7 @@ def config_dict(w, args, world):
             "pv_filter": "recall" if getattr(args, "recall", None) is not None else "lambda",
             "recall": getattr(args, "recall", None), "seq_len": w.N, "heads": w.H, "head_dim": w.D,
             "qk": getattr(args, "qk", "bf16"),
+            "cluster_iters": getattr(args, "cluster_iters", None),
             "global_batch": w.B * world, "parallelism": f"replicas{world}",
             "l2": "flushed between timed steps" if 3 * w.B * w.H * w.N * w.D * 2 < 2 * L2_BYTES
             else "inputs larger than L2 (flushed too)",
@@ -293,20 +307,54 @@ def run_ours(args, w, world, rank, local, pg):
     q8 = args.qk == "fp8"
     if q8 and rec is not None:
         raise SystemExit("--recall runs on bf16 scores: drop --qk fp8")
+    cl = args.cluster_iters
+    if cl is not None and (q8 or w.causal):
+        raise SystemExit("--cluster-iters needs bf16 scores and a non-causal workload")
     plan = sa.sparse_attn_plan(q, k, args.tau, None, w.causal, with_idx=False, quantize=q8)
     ws = torch.empty(sa.sparse_attn_plan_workspace_size(B, H, N, D), dtype=torch.uint8, device=dev)
     out = torch.empty_like(q)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    if cl is not None:
+        # the clustered path: both orders, the reordered q, k, v, then the plan on them;
+        # the forward on the reordered tensors and its rows put back in token order
+        ws_c = torch.empty(sa.sparse_attn_cluster_workspace_size(B, H, N, D), dtype=torch.uint8, device=dev)
+        cq = sa.Clustering(perm=torch.empty((B, H, N), dtype=torch.int32, device=dev))
+        ck = sa.Clustering(perm=torch.empty((B, H, N), dtype=torch.int32, device=dev))
+        qs, ks, vs, os_ = (torch.empty_like(q) for _ in range(4))
+
+        def run_plan():
+            sa.sparse_attn_cluster(q, k, cl, out=cq, workspace=ws_c)
+            sa.sparse_attn_cluster(k, q, cl, out=ck, workspace=ws_c)
+            sa.sparse_attn_permute_rows(q, cq.perm, out=qs)
+            sa.sparse_attn_permute_rows(k, ck.perm, out=ks)
+            sa.sparse_attn_permute_rows(v, ck.perm, out=vs)
+            sa.sparse_attn_plan(qs, ks, args.tau, None, False, out=plan, workspace=ws, with_idx=False)
+
+        def run_fwd(stats=None):
+            sa.sparse_attn_fwd(qs, ks, vs, plan, lam, out=os_, stats=stats, recall=rec)
+            sa.sparse_attn_permute_rows(os_, cq.perm, inverse=True, out=out)
+        # kernels per step: per clustering 4 + 5 per iteration (+2 with none), 3 row moves,
+        # 3 plan kernels, the forward, the move back
+        launches_per_step = 2 * (4 + 5 * cl + (2 if cl == 0 else 0)) + 3 + 3 + 1 + 1
+    else:
+        def run_plan():
+            sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False,
+                                quantize=q8)
+
+        def run_fwd(stats=None):
+            sa.sparse_attn_fwd(q, k, v, plan, lam, out=out, stats=stats, qk_fp8=q8, recall=rec)
+        launches_per_step = 4
+
     def step():
-        sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False, quantize=q8)
-        sa.sparse_attn_fwd(q, k, v, plan, lam, out=out, qk_fp8=q8, recall=rec)
+        run_plan()
+        run_fwd()
 
     # stats (outside timing): kept pairs, skipped P.V, algorithmic FLOPs of the forward
     stats = torch.zeros(4, dtype=torch.int64, device=dev)
-    sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False, quantize=q8)
-    sa.sparse_attn_fwd(q, k, v, plan, lam, out=out, stats=stats, qk_fp8=q8, recall=rec)
+    run_plan()
+    run_fwd(stats)
     torch.cuda.synchronize()
     check_device(sa, "the stats pass")
     st = [int(x) for x in stats.cpu()]
@@ -340,12 +388,6 @@ def run_ours(args, w, world, rank, local, pg):
         dense_ms = e0.elapsed_time(e1)
         check_device(sa, "the dense (full-mask) reference")
         del full
-
-    def run_plan():
-        sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False, quantize=q8)
-
-    def run_fwd():
-        sa.sparse_attn_fwd(q, k, v, plan, lam, out=out, qk_fp8=q8, recall=rec)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -393,7 +435,7 @@ def run_ours(args, w, world, rank, local, pg):
 
     # end to end through the public API from pinned host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and cl is None:
         qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
         # warm-up calls exactly like the timed ones, so that the caching pinned
         # allocator holds the output blocks the timed calls cycle through
@@ -451,15 +493,15 @@ def run_ours(args, w, world, rank, local, pg):
         "predictor": {"bound": "hbm", "achieved": pred_gbs, "peak": hbm, "unit": "GB/s", "frac": pred_gbs / hbm,
                       "bytes": pred_bytes, "peak_source": f"{pk_kind} hbm_gbs"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
-                     "frac": achieved / peak_t, "traffic": measured_traffic(w, args.tau, lam, args.qk, rec),
+                     "frac": achieved / peak_t, "traffic": None if cl is not None else measured_traffic(w, args.tau, lam, args.qk, rec),
                      "kernel": f"fwd_kernel<{D}, fp8 scores> (sparse_attn_fwd_q8)" if q8
                      else (f"fwd_kernel<{D}, recall filter> (sparse_attn_fwd_recall)" if rec is not None
                            else f"fwd_kernel<{D}> (sparse_attn_fwd)"),
                      "peak_source": peak_source},
-        "e2e": e2e, "gpu_launches": 4 * args.steps, "cuda_graphs": not args.no_graph, "clocks": clocks,
+        "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "cuda_graphs": not args.no_graph, "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu:
-        v_cpu, t_cpu, cores, sample = time_oracle(w, args.tau, lam, args.cpu_seconds, args.seed, rec)
+        v_cpu, t_cpu, cores, sample = time_oracle(w, args.tau, lam, args.cpu_seconds, args.seed, rec, cl)
         line["cpu_baseline"] = {"value": v_cpu, "unit": UNIT, "cores": cores, "kind": "oracle",
                                 "sample": sample, "seconds": t_cpu}
     if rank == 0:

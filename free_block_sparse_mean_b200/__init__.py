@@ -25,6 +25,8 @@ from ._lib import SaShape, SparseAttnError
 BLOCK = 64
 
 __all__ = ["Plan", "sparse_attn_plan", "sparse_attn_fwd", "sparse_attn_fwd_recall", "sparse_attention",
+           "Clustering", "sparse_attn_cluster", "sparse_attn_cluster_workspace_size", "sparse_attn_permute_rows",
+           "sparse_attention_clustered",
            "sparse_attn_plan_workspace_size", "sparse_attn_num_tiles", "sparse_attn_device_error",
            "sparse_attn_selftest_wait_timeout",
            "SparseAttnError", "BLOCK"]
@@ -227,6 +229,82 @@ def sparse_attn_fwd_recall(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, pl
     """Stage 2 with the cumulative-energy P.V filter (the C call of the same name):
     sparse_attn_fwd(q, k, v, plan, None, scale, causal, recall=recall, ...)."""
     return sparse_attn_fwd(q, k, v, plan, None, scale, causal, out=out, stats=stats, recall=recall)
+
+
+@dataclass
+class Clustering:
+    """Output of sparse_attn_cluster (on the inputs' device).
+
+    perm      int32 [B, H, N]     perm[b, h, p] = the token at position p in cluster order
+    assign    int32 [B, H, N]     each token's cluster, or None
+    centroids fp32 [B, H, C, d]   the final cluster means (C = ceil(N/64)), or None
+    """
+    perm: torch.Tensor
+    assign: Optional[torch.Tensor] = None
+    centroids: Optional[torch.Tensor] = None
+
+
+def sparse_attn_cluster_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(_lib.load().sparse_attn_cluster_workspace_size(SaShape(B, H, N, d, BLOCK)))
+
+
+def sparse_attn_cluster(x: torch.Tensor, y: torch.Tensor, iters: int = 2, *, with_assign: bool = True,
+                        with_centroids: bool = False, out: Optional[Clustering] = None,
+                        workspace: Optional[torch.Tensor] = None) -> Clustering:
+    """Interaction clustering of x's tokens under the Gram metric of y (the C call
+    of the same name): queries are clustered with y = k, keys with y = q."""
+    lib = _lib.load()
+    _check_qkv(x, y)
+    B, H, N, d = x.shape
+    C = -(-N // BLOCK)
+    dev = x.device
+    if out is None:
+        out = Clustering(
+            perm=torch.empty((B, H, N), dtype=torch.int32, device=dev),
+            assign=torch.empty((B, H, N), dtype=torch.int32, device=dev) if with_assign else None,
+            centroids=torch.empty((B, H, C, d), dtype=torch.float32, device=dev) if with_centroids else None)
+    if workspace is None:
+        workspace = torch.empty(sparse_attn_cluster_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+    st = lib.sparse_attn_cluster(_ptr(x), _ptr(y), _shape(x), int(iters), _ptr(out.assign), _ptr(out.perm),
+                                 _ptr(out.centroids), _ptr(workspace), workspace.numel(), _stream(dev))
+    _call("sparse_attn_cluster", st)
+    return out
+
+
+def sparse_attn_permute_rows(src: torch.Tensor, perm: torch.Tensor, inverse: bool = False, *,
+                             out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Rows of src [B, H, N, d] moved by perm [B, H, N] (int32): gathered
+    (out[b, h, p] = src[b, h, perm[b, h, p]]) or, with inverse, scattered."""
+    lib = _lib.load()
+    _check_qkv(src)
+    if perm.dtype != torch.int32 or tuple(perm.shape) != tuple(src.shape[:3]) or perm.device != src.device \
+            or not perm.is_contiguous():
+        raise ValueError("perm must be a contiguous int32 tensor [B, H, N] on src's device")
+    if out is None:
+        out = torch.empty_like(src)
+    st = lib.sparse_attn_permute_rows(_ptr(src), _ptr(perm), _shape(src), int(bool(inverse)), _ptr(out),
+                                      _stream(src.device))
+    _call("sparse_attn_permute_rows", st)
+    return out
+
+
+def sparse_attention_clustered(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau, lam: Optional[float] = None,
+                               iters: int = 2, scale: Optional[float] = None, *,
+                               recall: Optional[float] = None):
+    """Plan + forward on tokens reordered by interaction clustering (non-causal):
+    queries clustered under k's Gram metric, keys under q's; q, k, v reordered,
+    sparse_attn_plan and sparse_attn_fwd on the reordered tensors, and the output
+    rows put back in token order. Returns (o, info) with info = dict(cq, ck, plan)."""
+    _check_qkv(q, k, v)
+    cq = sparse_attn_cluster(q, k, iters, with_assign=False)
+    ck = sparse_attn_cluster(k, q, iters, with_assign=False)
+    qs = sparse_attn_permute_rows(q, cq.perm)
+    ks = sparse_attn_permute_rows(k, ck.perm)
+    vs = sparse_attn_permute_rows(v, ck.perm)
+    plan = sparse_attn_plan(qs, ks, tau, scale, False)
+    os_ = sparse_attn_fwd(qs, ks, vs, plan, lam, scale, False, recall=recall)
+    o = sparse_attn_permute_rows(os_, cq.perm, inverse=True)
+    return o, dict(cq=cq, ck=ck, plan=plan)
 
 
 _COPY_STREAMS = {}

@@ -32,6 +32,9 @@ EXPORTS = (
     "sparse_attn_plan_q8",
     "sparse_attn_fwd_q8",
     "sparse_attn_fwd_recall",
+    "sparse_attn_cluster_workspace_size",
+    "sparse_attn_cluster",
+    "sparse_attn_permute_rows",
     "sparse_attn_selftest_wait_timeout",
 )
 
@@ -89,6 +92,12 @@ def load(path: str = LIB_PATH):
     lib.sparse_attn_fwd_q8.restype = i32
     lib.sparse_attn_fwd_recall.argtypes = [vp, vp, vp, SaShape, vp, vp, f32, f32, i32, vp, vp, vp]
     lib.sparse_attn_fwd_recall.restype = i32
+    lib.sparse_attn_cluster_workspace_size.argtypes = [SaShape]
+    lib.sparse_attn_cluster_workspace_size.restype = sz
+    lib.sparse_attn_cluster.argtypes = [vp, vp, SaShape, i32, vp, vp, vp, vp, sz, vp]
+    lib.sparse_attn_cluster.restype = i32
+    lib.sparse_attn_permute_rows.argtypes = [vp, vp, SaShape, i32, vp, vp]
+    lib.sparse_attn_permute_rows.restype = i32
     lib.sparse_attn_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp]
     lib.sparse_attn_selftest_wait_timeout.restype = i32
     _lib = lib

@@ -11,6 +11,7 @@
 #include "../../include/sparse_attn.h"
 #include "fwd_kernel.cuh"
 #include "plan_kernels.cuh"
+#include "cluster_kernels.cuh"
 
 namespace {
 
@@ -186,6 +187,57 @@ sa_status launch_fwd(const sa_shape& s, const void* Q, const void* K, const void
   return SA_OK;
 }
 
+// Interaction clustering of X under the Gram metric of Y (see cluster_kernels.cuh).
+template <int D>
+sa_status launch_cluster(const sa_shape& s, const void* X, const void* Y, int iters, int32_t* assign_out,
+                         int32_t* perm, float* cent_out, void* ws, cudaStream_t st) {
+  const int N = s.N;
+  const long long BH = static_cast<long long>(s.B) * s.H;
+  const sa::ClusterWorkspace L = sa::cluster_workspace(BH, N, D);
+  const int C = L.C;
+  char* wsb = static_cast<char*>(ws);
+  float* gpart = reinterpret_cast<float*>(wsb + L.gpart);
+  float* G = reinterpret_cast<float*>(wsb + L.gram);
+  float* cent = reinterpret_cast<float*>(wsb + L.cent);
+  float* W = reinterpret_cast<float*>(wsb + L.w);
+  float* bvec = reinterpret_cast<float*>(wsb + L.b);
+  int* cnt = reinterpret_cast<int*>(wsb + L.cnt);
+  int* off = reinterpret_cast<int*>(wsb + L.off);
+  int* assign = assign_out ? assign_out : reinterpret_cast<int*>(wsb + L.assign);
+  const auto* x = static_cast<const __nv_bfloat16*>(X);
+  const auto* y = static_cast<const __nv_bfloat16*>(Y);
+  const unsigned by = static_cast<unsigned>(BH);
+  sa::gram_partial_kernel<D><<<dim3(L.splits, by), 256, 0, st>>>(y, gpart, N, L.splits, L.chunk);
+  sa::gram_reduce_kernel<D><<<dim3(D * D / 256, by), 256, 0, st>>>(gpart, G, L.splits);
+  // the block means (the pooling kernel, queries half only) and every token in its block
+  sa::pool_kernel<D><<<dim3(static_cast<unsigned>(BH * C), 1), 256, 0, st>>>(x, x, cent, nullptr, N, C);
+  const long long total = BH * N;
+  sa::cluster_init_assign_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(assign, cnt, N, C,
+                                                                                               total);
+  if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+  constexpr int kAssignSmem = sa::cluster_assign_smem_bytes<D>();
+  if (set_smem(sa::cluster_assign_kernel<D>, kAssignSmem) != SA_OK) return SA_ERR_CUDA;
+  const dim3 order_grid((C + sa::kOrderClusters - 1) / sa::kOrderClusters, by);
+  const dim3 cent_grid((C + 7) / 8, by);
+  for (int it = 0; it < iters; ++it) {
+    sa::cluster_prep_kernel<D><<<dim3((C + 15) / 16, by), D, 0, st>>>(G, cent, W, bvec, cnt, C);
+    sa::cluster_assign_kernel<D><<<dim3((N + 63) / 64, by), 256, kAssignSmem, st>>>(x, W, bvec, assign, cnt, N, C);
+    sa::cluster_offsets_kernel<<<by, 1024, 0, st>>>(cnt, off, C);
+    sa::cluster_order_kernel<<<order_grid, 256, 0, st>>>(assign, off, perm, N, C);
+    sa::cluster_centroid_kernel<D><<<cent_grid, 256, 0, st>>>(x, perm, off, cnt, cent, N, C);
+    if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+  }
+  if (iters == 0) {   // the plain blocks: identity order, block means from the pooling kernel
+    sa::cluster_offsets_kernel<<<by, 1024, 0, st>>>(cnt, off, C);
+    sa::cluster_order_kernel<<<order_grid, 256, 0, st>>>(assign, off, perm, N, C);
+  }
+  if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+  if (cent_out && cudaMemcpyAsync(cent_out, cent, static_cast<size_t>(BH) * C * D * sizeof(float),
+                                  cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return SA_ERR_CUDA;
+  return SA_OK;
+}
+
 }  // namespace
 
 namespace sa {
@@ -286,6 +338,50 @@ sa_status sparse_attn_fwd_recall(const void* Q, const void* K, const void* V, sa
                                        nullptr, budget);
   return launch_fwd<128, false, true>(s, Q, K, V, mask, work, 0.f, scale, causal != 0, O, stats, st, nullptr,
                                       nullptr, budget);
+}
+
+size_t sparse_attn_cluster_workspace_size(sa_shape s) {
+  if (check_shape(s) != SA_OK) return 0;
+  return sa::cluster_workspace(static_cast<long long>(s.B) * s.H, s.N, s.d).total;
+}
+
+sa_status sparse_attn_cluster(const void* X, const void* Y, sa_shape s, int32_t iters, int32_t* assign,
+                              int32_t* perm, float* centroids, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  if (!X || !Y || !perm) return SA_ERR_INVALID_ARG;
+  const sa_status sh = check_shape(s);
+  if (sh != SA_OK) return sh;
+  if (iters < 0 || iters > 64) return SA_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Y) || (reinterpret_cast<uintptr_t>(perm) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(assign) & 3u) != 0 || (reinterpret_cast<uintptr_t>(centroids) & 3u) != 0)
+    return SA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < sparse_attn_cluster_workspace_size(s))
+    return SA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s.d == 64) return launch_cluster<64>(s, X, Y, iters, assign, perm, centroids, workspace, st);
+  return launch_cluster<128>(s, X, Y, iters, assign, perm, centroids, workspace, st);
+}
+
+sa_status sparse_attn_permute_rows(const void* src, const int32_t* perm, sa_shape s, int32_t inverse, void* dst,
+                                   void* stream) {
+  if (!src || !perm || !dst || src == dst) return SA_ERR_INVALID_ARG;
+  const sa_status sh = check_shape(s);
+  if (sh != SA_OK) return sh;
+  if (!aligned16(src) || !aligned16(dst) || (reinterpret_cast<uintptr_t>(perm) & 3u) != 0)
+    return SA_ERR_INVALID_ARG;
+  const long long rows = static_cast<long long>(s.B) * s.H * s.N;
+  const long long threads = rows * (s.d / 8);
+  const unsigned grid = static_cast<unsigned>((threads + 255) / 256);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const auto* x = static_cast<const __nv_bfloat16*>(src);
+  auto* y = static_cast<__nv_bfloat16*>(dst);
+  if (s.d == 64)
+    sa::permute_rows_kernel<64><<<grid, 256, 0, st>>>(x, perm, y, s.N, rows, inverse != 0);
+  else
+    sa::permute_rows_kernel<128><<<grid, 256, 0, st>>>(x, perm, y, s.N, rows, inverse != 0);
+  if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+  return SA_OK;
 }
 
 const char* sparse_attn_status_string(sa_status st) {

@@ -194,6 +194,44 @@ sa_status sparse_attn_fwd_q8(const void* Q8, const void* K8, const float* qscale
                              float lambda, float scale, int32_t causal, void* O, int64_t* stats,
                              void* stream);
 
+/* Interaction clustering (iCATS abstract: query and key tokens clustered by
+ * their dot-product interaction, the objective written as a quadratic form; the
+ * formula is this library's reading of it). Replacing a token x of X by a
+ * centroid c changes its score with every token y of Y by (x - c).y; the sum of
+ * the squares is (x - c)^T G (x - c), G = sum_y y y^T. Per (b, h): k-means of
+ * X's tokens under that distance, C = ceil(N/64) clusters initialised to the
+ * 64-token block means, `iters` Lloyd iterations (assign each token to the
+ * nearest centroid, fp32, ties to the lowest cluster index; move each centroid
+ * to the mean of its tokens, an empty cluster keeping its centroid). Then the
+ * tokens are ordered by cluster, in token order within a cluster, clusters
+ * packed back to back (no padding: a cluster's tail shares a block with the
+ * next one's head).
+ *
+ *   X, Y       device bf16 [B,H,N,d]: the side to cluster and the other side
+ *              (queries are clustered with Y = K, keys with Y = Q)
+ *   iters      0..64; 0 leaves every token in its block (perm = identity)
+ *   assign     out, device int32 [B,H,N] or NULL: each token's cluster
+ *   perm       out, device int32 [B,H,N]: perm[b,h,p] = the token at position p
+ *   centroids  out, device fp32 [B,H,C,d] or NULL: the means of the final clusters
+ *   workspace  device scratch of sparse_attn_cluster_workspace_size(s) bytes,
+ *              256-byte aligned
+ * Errors: as sparse_attn_plan (misaligned or NULL X, Y or perm, iters outside
+ * 0..64: SA_ERR_INVALID_ARG; workspace: SA_ERR_WORKSPACE). A token whose every
+ * distance is NaN goes to cluster 0 and sets bit 2 of the device error word. */
+size_t sparse_attn_cluster_workspace_size(sa_shape s);
+sa_status sparse_attn_cluster(const void* X, const void* Y, sa_shape s, int32_t iters, int32_t* assign,
+                              int32_t* perm, float* centroids, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/* Moves the rows of a bf16 [B,H,N,d] tensor by a per-head permutation (e.g.
+ * sparse_attn_cluster's perm): inverse = 0 gathers dst[b,h,p] = src[b,h,perm[p]],
+ * inverse != 0 scatters dst[b,h,perm[p]] = src[b,h,p]. src and dst must differ,
+ * 16-byte aligned; perm 4-byte aligned and, per head, a permutation of 0..N-1
+ * (an entry outside 0..N-1 moves nothing and sets bit 1 of the device error
+ * word). */
+sa_status sparse_attn_permute_rows(const void* src, const int32_t* perm, sa_shape s, int32_t inverse, void* dst,
+                                   void* stream);
+
 /* sparse_attn_plan without a workspace, for callers that cannot allocate device
  * memory (a runtime that reserves its whole memory budget up front, a plugin
  * whose host owns the allocator, a latency-critical path that must not call

@@ -138,6 +138,28 @@ def test_recall_forward_rejects_bad_arguments(lib):
     assert fwd(s=SaShape(1, 2, 128, 96, 64)) == 2                   # d in {64, 128}
 
 
+def test_cluster_entry_points_reject_bad_arguments(lib):
+    s = SaShape(1, 2, 1000, 128, 64)
+    ws_need = int(lib.sparse_attn_cluster_workspace_size(s))
+    assert ws_need > 0 and lib.sparse_attn_cluster_workspace_size(SaShape(1, 2, 1000, 96, 64)) == 0
+    ws = ctypes.c_void_p(0x100000)
+
+    def cl(X=FAKE, perm=FAKE, iters=2, ws=ws, nbytes=ws_need, s=s):
+        return lib.sparse_attn_cluster(X, FAKE, s, iters, None, perm, None, ws, nbytes, None)
+
+    assert cl(X=None) == 1 and cl(perm=None) == 1 and cl(X=FAKE_ODD) == 1
+    assert cl(iters=-1) == 1 and cl(iters=65) == 1
+    assert cl(ws=None) == 3 and cl(nbytes=ws_need - 1) == 3 and cl(ws=ctypes.c_void_p(0x100010)) == 3
+    assert cl(s=SaShape(1, 2, 1000, 96, 64)) == 2
+
+    def pr(src=FAKE, dst=ctypes.c_void_p(0x20000), perm=FAKE, s=s):
+        return lib.sparse_attn_permute_rows(src, perm, s, 0, dst, None)
+
+    assert pr(src=None) == 1 and pr(perm=None) == 1 and pr(dst=FAKE) == 1     # dst must differ from src
+    assert pr(src=FAKE_ODD) == 1 and pr(perm=ctypes.c_void_p(0x10002)) == 1
+    assert pr(s=SaShape(1, 2, 1000, 128, 32)) == 2
+
+
 def test_device_error_needs_output_pointer(lib):
     assert lib.sparse_attn_device_error(None, None) == 1
 
