@@ -241,6 +241,8 @@ sa_status launch_cluster(const sa_shape& s, const void* X, const void* Y, int it
 }  // namespace
 
 namespace sa {
+cudaError_t take_noalloc_device_error(cudaStream_t st, unsigned int* out);   // sa_noalloc.cu
+
 // Exercises the device-side failure path: one warp waits on an mbarrier whose
 // phase nothing completes, through the same bounded wait the pipelines use, with
 // a short limit. The wait gives up, records DEVERR_TIMEOUT in the error word and
@@ -452,7 +454,9 @@ sa_status sparse_attn_device_error(void* stream, int32_t* code) {
       cudaSuccess)
     return SA_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return SA_ERR_CUDA;
-  *code = static_cast<int32_t>(v);
+  unsigned int w = 0;   // the other translation unit's word (see sa_noalloc.cu)
+  if (sa::take_noalloc_device_error(st, &w) != cudaSuccess) return SA_ERR_CUDA;
+  *code = static_cast<int32_t>(v | w);
   return SA_OK;
 }
 

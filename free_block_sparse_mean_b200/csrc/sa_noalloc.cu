@@ -108,6 +108,21 @@ sa_status launch_plan_noalloc(const sa_shape& s, const void* Q, const void* K, f
 
 }  // namespace
 
+namespace sa {
+// Reads and clears this translation unit's copy of the device error word. The
+// plan kernels are templates instantiated here and in the main translation unit;
+// a launch may run either unit's copy, and each copy reports into its own unit's
+// word, so sparse_attn_device_error reads both.
+cudaError_t take_noalloc_device_error(cudaStream_t st, unsigned int* out) {
+  unsigned int zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_dev_error, sizeof(*out), 0, cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return e;
+  e = cudaMemcpyToSymbolAsync(g_dev_error, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return e;
+  return cudaStreamSynchronize(st);
+}
+}  // namespace sa
+
 extern "C" sa_status sparse_attn_plan_noalloc(const void* Q, const void* K, sa_shape s, float tau, float scale,
                                               int32_t causal, uint8_t* mask, int32_t* count, int32_t* idx,
                                               int32_t* work, void* stream) {
