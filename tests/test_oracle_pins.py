@@ -657,3 +657,17 @@ def test_clustered_attention_uses_each_side_under_the_others_metric():
     np.testing.assert_array_equal(info["perm_q"][0, 0], ident)
     moved = orc.cluster_permutation(orc.kmeans_interaction(A, A, 1)[0])[0, 0]
     assert moved[63] == 0                                     # own metric: token 0 leaves block 0
+
+
+def test_kmeans_heads_are_independent():
+    """Each (batch, head) is clustered on its own: a [2, 2] batch gives what the
+    four heads give one by one (pins the per-head Gram matrix and indexing)."""
+    r = _rng(17)
+    X = r.standard_normal((2, 2, 150, 6)) + np.linspace(0, 2, 150)[None, None, :, None]
+    Y = r.standard_normal((2, 2, 150, 6)) * np.array([0.5, 1.0, 1.5, 2.0]).reshape(2, 2, 1, 1)
+    a, c, _ = orc.kmeans_interaction(X, Y, 2)
+    for b in range(2):
+        for h in range(2):
+            a1, c1, _ = orc.kmeans_interaction(X[b:b + 1, h:h + 1], Y[b:b + 1, h:h + 1], 2)
+            np.testing.assert_array_equal(a[b, h], a1[0, 0])
+            np.testing.assert_allclose(c[b, h], c1[0, 0], rtol=1e-13, atol=1e-13)
