@@ -234,7 +234,8 @@ def attention_masked(Q, K, V, mask, scale: Optional[float] = None, causal: bool 
 
 def attention_tiled(Q, K, V, mask, lam: float, scale: Optional[float] = None,
                     causal: bool = False, block: int = BLOCK,
-                    qblocks: Optional[Iterable[int]] = None, return_stats: bool = False):
+                    qblocks: Optional[Iterable[int]] = None, return_stats: bool = False,
+                    forced=None):
     """Stage 2 with the online-softmax-aware filter, as a literal fp64 run of the
     tiled loop: per 64-row query block, kept key blocks in ascending order,
     running max m, running sum l, accumulator O.
@@ -244,7 +245,18 @@ def attention_tiled(Q, K, V, mask, lam: float, scale: Optional[float] = None,
     test is rowmax_r(S_blk) - m_r < lam for every row r of the query block that
     sees at least one key of the block (m_r before the block, natural-log units
     of the scaled logits); only P.V is skipped, m and l are still updated.
-    lam = -inf never skips, and then this equals attention_masked."""
+    lam = -inf never skips, and then this equals attention_masked.
+
+    forced [B, H, Nb, Nb] (0/1), if given, replaces the test: the pair (i, j) is
+    skipped iff forced[b, h, i, j] is nonzero (a replay of decisions recorded
+    elsewhere; the test is still evaluated and reported). The filter's reading
+    allows a decision taken in lower precision to flip only where the test's
+    margin is within rounding of zero, which the caller checks on the margins.
+
+    With return_stats, also returns dict(kept_pairs, pv_skipped, decisions): a
+    list of (b, h, i, j, own_skip, margin) with margin = lam - max over the
+    seeing rows of (rowmax - m) (the test says "skip" iff margin > 0; +inf for a
+    row's first block, which is never skipped, is reported as -inf)."""
     Q, K, V = as_f64(Q), as_f64(K), as_f64(V)
     mask = np.asarray(mask)
     B, H, N, d = Q.shape
@@ -255,6 +267,7 @@ def attention_tiled(Q, K, V, mask, lam: float, scale: Optional[float] = None,
     O = np.full((B, H, N, V.shape[-1]), np.nan)
     kept_pairs = 0
     skipped_pairs = 0
+    decisions = []
     for b in range(B):
         for h in range(H):
             for i in qbs:
@@ -275,7 +288,9 @@ def attention_tiled(Q, K, V, mask, lam: float, scale: Optional[float] = None,
                     kept_pairs += 1
                     with np.errstate(invalid="ignore"):
                         diff = rmax - m                      # +inf where m = -inf
-                    skip = bool(np.all(diff[sees] < lam))
+                    own = bool(np.all(diff[sees] < lam))
+                    decisions.append((b, h, i, int(j), own, float(lam - diff[sees].max())))
+                    skip = own if forced is None else bool(forced[b, h, i, j])
                     m_new = np.maximum(m, rmax)
                     ref = np.where(np.isfinite(m_new), m_new, 0.0)
                     alpha = np.where(np.isfinite(m), np.exp(m - ref), 0.0)
@@ -291,13 +306,14 @@ def attention_tiled(Q, K, V, mask, lam: float, scale: Optional[float] = None,
                 out[l <= 0] = 0.0
                 O[b, h, s:e] = out
     if return_stats:
-        return O, dict(kept_pairs=kept_pairs, pv_skipped=skipped_pairs)
+        return O, dict(kept_pairs=kept_pairs, pv_skipped=skipped_pairs, decisions=decisions)
     return O
 
 
 def attention_recall(Q, K, V, mask, recall: float, scale: Optional[float] = None,
                      causal: bool = False, block: int = BLOCK,
-                     qblocks: Optional[Iterable[int]] = None, return_stats: bool = False):
+                     qblocks: Optional[Iterable[int]] = None, return_stats: bool = False,
+                     forced=None):
     """Stage 2 with the in-operator cumulative-energy filter, as a literal fp64 run
     of the tiled loop (64-row query blocks, kept key blocks in ascending order).
 
@@ -318,7 +334,12 @@ def attention_recall(Q, K, V, mask, recall: float, scale: Optional[float] = None
     recall_rows): decisions is a list of (b, h, i, j, skipped, margin) where
     margin = min over the seeing rows of ((1 - recall) * l' - (sk * alpha + e)) / l'
     (the decision is "skip" iff margin >= 0), and recall_rows [B, H, N] is
-    1 - sk / l per row at the end (NaN for rows not computed)."""
+    1 - sk / l per row at the end (NaN for rows not computed).
+
+    forced [B, H, Nb, Nb] (0/1), if given, replaces the test as in
+    attention_tiled: pair (i, j) is skipped iff forced[b, h, i, j] is nonzero, and
+    sk, l and the output follow that decision; `decisions` still reports the
+    test's own verdict and margin for each pair."""
     Q, K, V = as_f64(Q), as_f64(K), as_f64(V)
     mask = np.asarray(mask)
     B, H, N, d = Q.shape
@@ -360,8 +381,9 @@ def attention_recall(Q, K, V, mask, recall: float, scale: Optional[float] = None
                     sk_try = sk * alpha + en
                     room = budget * l_new - sk_try
                     margin = float(np.min(room[sees] / l_new[sees]))
-                    skip = bool(np.all(room[sees] >= 0.0))
-                    decisions.append((b, h, i, int(j), skip, margin))
+                    own = bool(np.all(room[sees] >= 0.0))
+                    decisions.append((b, h, i, int(j), own, margin))
+                    skip = own if forced is None else bool(forced[b, h, i, j])
                     l = l_new
                     acc = acc * alpha[:, None]
                     if skip:
@@ -383,11 +405,12 @@ def attention_recall(Q, K, V, mask, recall: float, scale: Optional[float] = None
 
 
 def fwd(Q, K, V, mask, lam: Optional[float] = None, scale: Optional[float] = None,
-        causal: bool = False, block: int = BLOCK, qblocks=None):
-    """Stage 2: the masked attention, with the lambda filter when lam is finite."""
+        causal: bool = False, block: int = BLOCK, qblocks=None, forced=None):
+    """Stage 2: the masked attention, with the lambda filter when lam is finite
+    (forced: a replay of recorded filter decisions, see attention_tiled)."""
     if lam is None or lam == -math.inf:
         return attention_masked(Q, K, V, mask, scale, causal, block, qblocks)
-    return attention_tiled(Q, K, V, mask, lam, scale, causal, block, qblocks)
+    return attention_tiled(Q, K, V, mask, lam, scale, causal, block, qblocks, forced=forced)
 
 
 # ----------------------------------------------------------------------------

@@ -265,7 +265,12 @@ def test_lambda_skip_closed_form():
     np.testing.assert_allclose(O_off[0, 0], np.tile([1 / (1 + t), t / (1 + t)], (128, 1)), rtol=1e-14)
     np.testing.assert_allclose(O_25, O_off, rtol=1e-14, atol=0)
     np.testing.assert_allclose(O_12[0, 0], np.tile([1 / (1 + t), 0.0], (128, 1)), rtol=1e-14, atol=0)
-    assert st12 == dict(kept_pairs=4, pv_skipped=2) and st25["pv_skipped"] == 0
+    assert (st12["kept_pairs"], st12["pv_skipped"]) == (4, 2) and st25["pv_skipped"] == 0
+    # margins: lam - (rowmax - m) of the second block is -12 + 20 = 8 (skip); the
+    # first block of a row is never skipped (margin -inf)
+    margins = sorted(mg for *_, mg in st12["decisions"])
+    assert margins[:2] == [-math.inf, -math.inf]
+    np.testing.assert_allclose(margins[2:], [8.0, 8.0], rtol=1e-14)
 
 
 def test_lambda_first_block_never_skipped_and_order_matters():
@@ -671,3 +676,62 @@ def test_kmeans_heads_are_independent():
             a1, c1, _ = orc.kmeans_interaction(X[b:b + 1, h:h + 1], Y[b:b + 1, h:h + 1], 2)
             np.testing.assert_array_equal(a[b, h], a1[0, 0])
             np.testing.assert_allclose(c[b, h], c1[0, 0], rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------- replay of recorded decisions
+def _brute_force_replay(Q, K, V, mask, decide, causal):
+    """Reference-free output of the tiled loop under given skip decisions: per
+    row, block energies against one fixed reference (the row's largest visible
+    score); the output is the unskipped blocks' weighted V over the energy of
+    every visited block (a skipped block stays in the sum, only P.V is dropped)."""
+    B, H, N, d = Q.shape
+    scale = 1.0 / math.sqrt(d)
+    Nb = orc.n_blocks(N)
+    O = np.zeros_like(V)
+    for b in range(B):
+        for h in range(H):
+            for i in range(Nb):
+                s, e = i * 64, min(N, i * 64 + 64)
+                S = scale * Q[b, h, s:e] @ K[b, h].T
+                vis = np.repeat(mask[b, h, i].astype(bool), 64)[:N][None, :].repeat(e - s, 0)
+                if causal:
+                    vis &= np.arange(N)[None, :] <= np.arange(s, e)[:, None]
+                S = np.where(vis, S, -np.inf)
+                M = S.max(axis=1)
+                W = np.exp(S - M[:, None])
+                num = np.zeros((e - s, V.shape[-1]))
+                for j in np.nonzero(mask[b, h, i])[0]:
+                    cols = slice(j * 64, min(N, j * 64 + 64))
+                    if not vis[:, cols].any() or decide[b, h, i, j]:
+                        continue
+                    num += W[:, cols] @ V[b, h, cols]
+                O[b, h, s:e] = num / W.sum(axis=1)[:, None]
+    return O
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_forced_decisions_replay_brute_force(causal):
+    """Any decision map, replayed by either filter's loop, gives the brute-force
+    output for those decisions (the filter's own test plays no part); replaying
+    the loop's own decisions reproduces its unforced output exactly; and each
+    reported own decision agrees with the sign of its margin."""
+    N, d = 449, 16
+    Q, K, V, mask = _recall_case(N + int(causal), N, d, causal, 2)
+    Nb = orc.n_blocks(N)
+    r = _rng(23)
+    forced = (r.random(mask.shape) < 0.4).astype(np.uint8)
+    want = _brute_force_replay(Q, K, V, mask, forced, causal)
+    got_l = orc.attention_tiled(Q, K, V, mask, -3.0, None, causal, forced=forced)
+    got_r = orc.attention_recall(Q, K, V, mask, 0.9, None, causal, forced=forced)
+    np.testing.assert_allclose(got_l, want, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(got_r, want, rtol=1e-10, atol=1e-12)
+    for fn, arg, strict in ((orc.attention_tiled, -3.0, True), (orc.attention_recall, 0.9, False)):
+        O, st = fn(Q, K, V, mask, arg, None, causal, return_stats=True)
+        own = np.zeros(mask.shape, dtype=np.uint8)
+        for b, h, i, j, sk, mg in st["decisions"]:
+            own[b, h, i, j] = sk
+            assert sk == ((mg > 0) if strict else (mg >= 0))
+        assert own.sum() == st["pv_skipped"] > 0
+        np.testing.assert_array_equal(fn(Q, K, V, mask, arg, None, causal, forced=own), O)
+        np.testing.assert_allclose(O, _brute_force_replay(Q, K, V, mask, own, causal), rtol=1e-10, atol=1e-12)
+    assert Nb > 4
