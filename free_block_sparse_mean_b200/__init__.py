@@ -28,6 +28,7 @@ __all__ = ["Plan", "sparse_attn_plan", "sparse_attn_fwd", "sparse_attn_fwd_recal
            "Clustering", "sparse_attn_cluster", "sparse_attn_cluster_workspace_size", "sparse_attn_permute_rows",
            "sparse_attention_clustered",
            "sparse_attn_plan_workspace_size", "sparse_attn_num_tiles", "sparse_attn_device_error",
+           "sparse_attn_host_workspace_size",
            "sparse_attn_selftest_wait_timeout",
            "SparseAttnError", "BLOCK"]
 
@@ -98,8 +99,13 @@ def sparse_attn_num_tiles(B: int, H: int, N: int, d: int) -> int:
     return int(_lib.load().sparse_attn_num_tiles(SaShape(B, H, N, d, BLOCK)))
 
 
+def sparse_attn_host_workspace_size(B: int, H: int, N: int, d: int, chunks: int = 4, qk_fp8: bool = False) -> int:
+    return int(_lib.load().sparse_attn_host_workspace_size(SaShape(B, H, N, d, BLOCK), int(chunks),
+                                                           _lib.SA_HOST_FP8_SCORES if qk_fp8 else 0))
+
+
 def sparse_attn_plan(q: torch.Tensor, k: torch.Tensor, tau, scale: Optional[float] = None,
-                     causal: bool = False, *, with_idx: bool = True, with_work: bool = True,
+                     causal: bool = False, *, with_idx: bool = False, with_work: bool = True,
                      out: Optional[Plan] = None, workspace: Optional[torch.Tensor] = None,
                      quantize: bool = False) -> Plan:
     """Stage 1: cumulative-energy block mask from mean-pooled q and k.
@@ -107,7 +113,10 @@ def sparse_attn_plan(q: torch.Tensor, k: torch.Tensor, tau, scale: Optional[floa
     tau is one recall threshold for every head (a float), or one per head: a float32
     CUDA tensor of shape [B, H] or [H] on q's device (sparse_attn_plan_heads).
     quantize=True (one tau, d = 128) also writes FP8 E4M3 copies of q and k with
-    per-block scales (sparse_attn_plan_q8) for sparse_attn_fwd(..., qk_fp8=True)."""
+    per-block scales (sparse_attn_plan_q8) for sparse_attn_fwd(..., qk_fp8=True).
+    with_idx=True also writes the ascending kept lists (an int32 [B, H, Nb, Nb]
+    tensor: 4 bytes per block pair, 331 MB on the 118,800-token video shape); the
+    forward does not read them, so they are off by default."""
     lib = _lib.load()
     _check_qkv(q, k)
     B, H, N, d = q.shape
@@ -166,7 +175,8 @@ def sparse_attn_plan(q: torch.Tensor, k: torch.Tensor, tau, scale: Optional[floa
 def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan, lam: Optional[float] = None,
                     scale: Optional[float] = None, causal: Optional[bool] = None, *,
                     out: Optional[torch.Tensor] = None, stats: Optional[torch.Tensor] = None,
-                    qk_fp8: bool = False, recall: Optional[float] = None) -> torch.Tensor:
+                    qk_fp8: bool = False, recall: Optional[float] = None,
+                    decisions: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Stage 2: attention over the kept blocks with the lambda P.V filter.
 
     `plan` is a Plan or a uint8 mask [B, H, Nb, Nb]. lam=None turns the filter off.
@@ -175,7 +185,10 @@ def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan, lam
     (sparse_attn_fwd_q8; the plan must come from sparse_attn_plan(quantize=True)).
     recall=rho (in (0, 1]) replaces the lambda test by the cumulative-energy test
     of sparse_attn_fwd_recall: every row keeps at least the fraction rho of the
-    softmax energy of the blocks it visits; lam must then be None."""
+    softmax energy of the blocks it visits; lam must then be None.
+    decisions, if given (uint8 [B, H, Nb, Nb] on q's device, bf16 scores), receives
+    the filter's per-pair decisions (sparse_attn_fwd_decisions): 1 where a visited
+    pair's P.V was skipped, 0 where it was computed; other entries are untouched."""
     lib = _lib.load()
     _check_qkv(q, k, v)
     B, H, N, d = q.shape
@@ -199,6 +212,20 @@ def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan, lam
         out = torch.empty_like(q)
     if stats is not None and (stats.dtype != torch.int64 or stats.numel() < 4 or stats.device != q.device):
         raise ValueError("stats must be an int64 tensor of >= 4 entries on q's device")
+    if decisions is not None:
+        if qk_fp8:
+            raise ValueError("decisions are recorded by the bf16-score forward")
+        if decisions.dtype != torch.uint8 or tuple(decisions.shape) != (B, H, Nb, Nb) \
+                or not decisions.is_contiguous() or decisions.device != q.device:
+            raise ValueError("decisions must be a contiguous uint8 tensor [B, H, Nb, Nb] on q's device")
+        if recall is not None and lam is not None:
+            raise ValueError("recall replaces the lambda filter: pass lam=None with it")
+        filt, val = (_lib.SA_FILTER_RECALL, float(recall)) if recall is not None else (_lib.SA_FILTER_LAMBDA, lam_f)
+        st = lib.sparse_attn_fwd_decisions(_ptr(q), _ptr(k), _ptr(v), _shape(q), _ptr(mask), _ptr(work), filt, val,
+                                           float(scale), int(causal), _ptr(out), _ptr(stats), _ptr(decisions),
+                                           _stream(q.device))
+        _call("sparse_attn_fwd_decisions", st)
+        return out
     if recall is not None:
         if lam is not None or qk_fp8:
             raise ValueError("recall replaces the lambda filter and takes bf16 scores: "
@@ -322,8 +349,10 @@ def _copy_streams(dev: torch.device):
 def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau,
                      lam: Optional[float] = None, scale: Optional[float] = None, causal: bool = False,
                      device="cuda", out: Optional[torch.Tensor] = None, chunks: Optional[int] = None,
-                     qk_fp8: bool = False, recall: Optional[float] = None) -> torch.Tensor:
-    """End to end from host tensors: copy q, k, v to the GPU, plan + forward, copy O back.
+                     qk_fp8: bool = False, recall: Optional[float] = None,
+                     workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """End to end from host tensors (the C call sparse_attn_host): copy q, k, v to
+    the GPU, plan + forward, copy O back.
 
     Host inputs should be pinned, so the copies are asynchronous DMA. The result is
     a host bf16 tensor in pinned memory (`out` if given, else one from torch's
@@ -333,50 +362,63 @@ def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau,
     (default: up to 4): group g's host-to-device copy, its plan + forward and its
     device-to-host copy run on three streams, so the copies of one group overlap
     the work of the others in both directions of the link. tau may be one value or
-    a per-head float32 tensor ([B, H] or [H]) on `device`. qk_fp8=True takes the
-    scores on FP8 copies of q and k (see sparse_attn_plan's quantize); recall
-    selects the cumulative-energy P.V filter instead of lambda (see sparse_attn_fwd)."""
+    a per-head float32 tensor ([B, H] or [H]) on `device`; qk_fp8=True takes the scores on FP8 copies of q and k (see
+    sparse_attn_plan's quantize); recall selects the cumulative-energy P.V filter
+    instead of lambda (see sparse_attn_fwd). The device workspace is allocated
+    here unless given (sparse_attn_host_workspace_size bytes).
+
+    After the call the device error word is read: a device-side check that fired
+    (a bounded wait that gave up, a range check) raises SparseAttnError with
+    SA_ERR_DEVICE_CHECK, since O is then undefined for the affected rows."""
+    lib = _lib.load()
     dev = torch.device(device)
     if q.shape != k.shape or q.shape != v.shape or q.dim() != 4:
         raise ValueError("q, k, v must share the shape [B, H, N, d]")
+    for t in (q, k, v):
+        if t.device.type != "cpu" or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous host bf16 tensors")
+    if recall is not None and (lam is not None or qk_fp8):
+        raise ValueError("recall replaces the lambda filter and takes bf16 scores")
     B, H, N, d = q.shape
-    BH = B * H
     if out is None:
         out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
-    elif out.shape != q.shape or out.dtype != q.dtype or out.device.type != "cpu":
-        raise ValueError("out must be a host bf16 tensor of q's shape")
+    elif out.shape != q.shape or out.dtype != q.dtype or out.device.type != "cpu" or not out.is_contiguous():
+        raise ValueError("out must be a contiguous host bf16 tensor of q's shape")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    nch = max(1, min(B * H, chunks if chunks is not None else 4))
+    flags = _lib.SA_HOST_FP8_SCORES if qk_fp8 else 0
+    s = _shape(q)
+    ws_bytes = int(lib.sparse_attn_host_workspace_size(s, nch, flags))
+    if ws_bytes == 0:
+        raise ValueError("unsupported shape for sparse_attention")
+    if workspace is None or workspace.numel() < ws_bytes or workspace.device != dev:
+        workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
+    tau_heads = None
     if isinstance(tau, torch.Tensor):
-        tau = (tau.unsqueeze(0).expand(B, H) if tau.dim() == 1 else tau).reshape(BH)
-    nch = max(1, min(BH, chunks if chunks is not None else 4))
-    bounds = [BH * c // nch for c in range(nch + 1)]
-    flat = [x.reshape(BH, N, d) for x in (q, k, v, out)]
-    qd, kd, vd, od = (torch.empty((BH, N, d), dtype=q.dtype, device=dev) for _ in range(4))
+        if tau.dtype != torch.float32 or tau.device != dev:
+            raise ValueError("a per-head tau must be a float32 tensor on `device`")
+        if tuple(tau.shape) == (H,):
+            tau = tau.unsqueeze(0).expand(B, H)
+        if tuple(tau.shape) != (B, H):
+            raise ValueError("a per-head tau must have shape [B, H] or [H]")
+        tau_heads = tau.contiguous()
+        tau = 1.0
+    filt, val = (_lib.SA_FILTER_RECALL, float(recall)) if recall is not None else \
+        (_lib.SA_FILTER_LAMBDA, -math.inf if lam is None else float(lam))
     main = torch.cuda.current_stream(dev)
     h2d, d2h = _copy_streams(dev)
-    h2d.wait_stream(main)
-    d2h.wait_stream(main)
-    for c in range(nch):
-        lo, hi = bounds[c], bounds[c + 1]
-        if hi == lo:
-            continue
-        with torch.cuda.stream(h2d):
-            for dst, src in zip((qd, kd, vd), flat[:3]):
-                dst[lo:hi].copy_(src[lo:hi], non_blocking=True)
-            ready = torch.cuda.Event()
-            ready.record(h2d)
-        main.wait_event(ready)
-        view = lambda x: x[lo:hi].view(1, hi - lo, N, d)
-        t = tau[lo:hi].view(1, hi - lo) if isinstance(tau, torch.Tensor) else tau
-        plan = sparse_attn_plan(view(qd), view(kd), t, scale, causal, with_idx=False, quantize=qk_fp8)
-        sparse_attn_fwd(view(qd), view(kd), view(vd), plan, lam, scale, causal, out=view(od), qk_fp8=qk_fp8,
-                        recall=recall)
-        done = torch.cuda.Event()
-        done.record(main)
-        d2h.wait_event(done)
-        with torch.cuda.stream(d2h):
-            flat[3][lo:hi].copy_(od[lo:hi], non_blocking=True)
-    main.wait_stream(d2h)
-    main.synchronize()
+    with torch.cuda.device(dev):
+        st = lib.sparse_attn_host(_ptr(q), _ptr(k), _ptr(v), s, float(tau), _ptr(tau_heads), filt, val, float(scale),
+                                  int(bool(causal)), flags, _ptr(out), _ptr(workspace), ws_bytes, nch,
+                                  ctypes.c_void_p(main.cuda_stream), ctypes.c_void_p(h2d.cuda_stream),
+                                  ctypes.c_void_p(d2h.cuda_stream))
+        _call("sparse_attn_host", st)
+        main.synchronize()
+        code = ctypes.c_int32(0)
+        _call("sparse_attn_device_error", lib.sparse_attn_device_error(_stream(dev), ctypes.byref(code)))
+    if code.value:
+        raise SparseAttnError(f"sparse_attention (device error word {code.value})", _lib.SA_ERR_DEVICE_CHECK, lib)
     return out
 
 

@@ -10,6 +10,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsparse_attn.so")
 
 SA_OK = 0
+SA_ERR_DEVICE_CHECK = 5
+SA_FILTER_LAMBDA = 0
+SA_FILTER_RECALL = 1
+SA_HOST_FP8_SCORES = 1
 STATUS_NAMES = {
     0: "SA_OK",
     1: "SA_ERR_INVALID_ARG",
@@ -32,6 +36,9 @@ EXPORTS = (
     "sparse_attn_plan_q8",
     "sparse_attn_fwd_q8",
     "sparse_attn_fwd_recall",
+    "sparse_attn_fwd_decisions",
+    "sparse_attn_host_workspace_size",
+    "sparse_attn_host",
     "sparse_attn_cluster_workspace_size",
     "sparse_attn_cluster",
     "sparse_attn_permute_rows",
@@ -92,6 +99,12 @@ def load(path: str = LIB_PATH):
     lib.sparse_attn_fwd_q8.restype = i32
     lib.sparse_attn_fwd_recall.argtypes = [vp, vp, vp, SaShape, vp, vp, f32, f32, i32, vp, vp, vp]
     lib.sparse_attn_fwd_recall.restype = i32
+    lib.sparse_attn_fwd_decisions.argtypes = [vp, vp, vp, SaShape, vp, vp, i32, f32, f32, i32, vp, vp, vp, vp]
+    lib.sparse_attn_fwd_decisions.restype = i32
+    lib.sparse_attn_host_workspace_size.argtypes = [SaShape, i32, i32]
+    lib.sparse_attn_host_workspace_size.restype = sz
+    lib.sparse_attn_host.argtypes = [vp, vp, vp, SaShape, f32, vp, i32, f32, f32, i32, i32, vp, vp, sz, i32, vp, vp, vp]
+    lib.sparse_attn_host.restype = i32
     lib.sparse_attn_cluster_workspace_size.argtypes = [SaShape]
     lib.sparse_attn_cluster_workspace_size.restype = sz
     lib.sparse_attn_cluster.argtypes = [vp, vp, SaShape, i32, vp, vp, vp, vp, sz, vp]

@@ -10,7 +10,7 @@
 // c^T G c - 2 x . (G c). So each Lloyd iteration is: w_c = G c and b_c = c . w_c
 // per centroid (cluster_prep_kernel), an argmin over all centroids per token
 // (cluster_assign_kernel, a register-tiled fp32 product of the tokens with the
-// w_c), and the mean of each cluster's tokens (cluster_members_kernel). The
+// w_c), and the mean of each cluster's tokens (cluster_centroid_kernel). The
 // clusters start at the 64-token block means (the pooling kernel), so zero
 // iterations reproduce the plain blocks.
 //

@@ -2,8 +2,8 @@
 // with the online-softmax-aware P.V skip.
 //
 // Stage 2 of the SpargeAttn abstract: the attention is computed only on the kept
-// blocks ("skip of some matrix multiplications"), and an online-softmax-aware
-// filter skips more P.V products at no extra cost. The DynSparse article places
+// blocks (stage 1 drops the matmuls of the blocks it predicts unimportant), and an
+// online-softmax-aware filter skips more P.V products at no extra cost. The DynSparse article places
 // the selection inside the FlashAttention operator; this kernel is that operator.
 //
 // One CTA = one 128-row query tile = two 64-row query blocks (qa, qb) of one head,
@@ -132,6 +132,8 @@ __device__ __forceinline__ float softmax_exp64(const float (&s)[64], float scale
 // every row keeps at least the fraction `recall` of the energy it has seen. The
 // vote needs e, so it is posted after the exponentials; the exchange is the
 // lambda vote's.
+// decisions (optional, [B,H,Nb,Nb] bytes): for every (query block, kept key
+// block) pair the tile visits, 1 if the filter skipped its P.V, else 0.
 template <int D, bool kF8, bool kRecall = false>
 __global__ void __launch_bounds__(192, 2)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -139,7 +141,8 @@ __global__ void __launch_bounds__(192, 2)
                const int* __restrict__ work, __nv_bfloat16* __restrict__ O, int N, int Nb, int Tq,
                long long num_tiles, long long num_qblocks, float scale_log2, float lam_log2, int lam_on,
                float budget, int causal, unsigned long long* __restrict__ stats,
-               const float* __restrict__ qscale, const float* __restrict__ kscale) {
+               const float* __restrict__ qscale, const float* __restrict__ kscale,
+               uint8_t* __restrict__ decisions) {
   using C = FwdCfg<D, kF8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -528,6 +531,7 @@ __global__ void __launch_bounds__(192, 2)
         contrib[(k & 1) * 2 + half] = (keep && !half_skip) ? 1 : 0;
         kept_pairs += keep ? 1ull : 0ull;
         skipped_pairs += (keep && half_skip) ? 1ull : 0ull;
+        if (decisions && keep) decisions[(bh * Nb + myqb) * static_cast<long long>(Nb) + j] = half_skip ? 1 : 0;
       }
       tc_fence_before();
       __syncwarp();

@@ -1,16 +1,20 @@
 // C ABI of the block-sparse attention library: argument checks, workspace
-// layout, TMA descriptors and launches. The kernels are in plan_kernels.cuh and
-// fwd_kernel.cuh; everything is compiled as this one translation unit.
+// layout, TMA descriptors and launches. The kernels are in plan_kernels.cuh,
+// fwd_kernel.cuh and cluster_kernels.cuh; the stage-1 launch sequence is in
+// plan_launch.cuh, shared with the allocation-free entry point (sa_noalloc.cu,
+// the library's second translation unit).
 #include <cudaTypedefs.h>
 
 #include <cmath>
 #include <cstdint>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
 #include "../../include/sparse_attn.h"
 #include "fwd_kernel.cuh"
 #include "plan_kernels.cuh"
+#include "plan_launch.cuh"
 #include "cluster_kernels.cuh"
 
 namespace {
@@ -95,72 +99,12 @@ bool make_map8(CUtensorMap* map, const void* ptr, const sa_shape& s) {
   return r == CUDA_SUCCESS;
 }
 
-template <typename F>
-sa_status set_smem(F* kernel, int bytes) {
-  // Per device: the attribute belongs to the current context.
-  static std::mutex mu;
-  std::lock_guard<std::mutex> lk(mu);
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
-    return SA_ERR_CUDA;
-  return SA_OK;
-}
-
-template <int D>
-sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau, const float* tau_bh,
-                      float scale, int causal, uint8_t* mask, int32_t* count, int32_t* idx, int32_t* work,
-                      void* ws, cudaStream_t st, uint8_t* Q8 = nullptr, uint8_t* K8 = nullptr,
-                      float* qscale = nullptr, float* kscale = nullptr) {
-  const int Nb = static_cast<int>(num_blocks(s));
-  const long long BH = static_cast<long long>(s.B) * s.H;
-  const sa::PlanWorkspace L = sa::plan_workspace(BH, Nb, D);
-  char* wsb = static_cast<char*>(ws);
-  float* Qp = reinterpret_cast<float*>(wsb + L.qp);
-  float* Kp = reinterpret_cast<float*>(wsb + L.kp);
-  unsigned long long* sig = reinterpret_cast<unsigned long long*>(wsb + L.sig);
-  uint32_t* bits = reinterpret_cast<uint32_t*>(wsb + L.bits);
-  sa::pool_kernel<D><<<dim3(static_cast<unsigned>(BH * Nb), 2), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Qp, Kp, s.N, Nb, Q8, K8, qscale,
-      kscale);
-  if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
-
-  // Small heads: 4 query blocks per CTA so the grid still fills the GPU.
-  auto launch_ss = [&](auto kern, int R, int NT) -> sa_status {
-    const int smem = R == 4 ? sa::score_select_smem_bytes<D, 4>(Nb)
-                            : (R == 8 ? sa::score_select_smem_bytes<D, 8>(Nb) : sa::score_select_smem_bytes<D, 16>(Nb));
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return SA_ERR_CUDA;
-    kern<<<dim3((Nb + R - 1) / R, static_cast<unsigned>(BH)), NT, smem, st>>>(Qp, Kp, Nb, scale, causal, tau,
-                                                                               tau_bh, mask, count, idx, sig, bits);
-    return SA_OK;
-  };
-  sa_status ls;
-  if (Nb <= 256)
-    ls = launch_ss(sa::score_select_kernel<D, 4, 128>, 4, 128);
-  else if (Nb <= 3000)
-    ls = launch_ss(sa::score_select_kernel<D, 16, 256>, 16, 256);
-  else
-    ls = launch_ss(sa::score_select_kernel<D, 8, 256>, 8, 256);
-  if (ls != SA_OK) return ls;
-  if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
-
-  if (work) {
-    const int Tq = (Nb + 1) / 2;
-    const int smem = sa::pair_order_smem_bytes(Nb);
-    if (set_smem(sa::pair_order_kernel, smem) != SA_OK) return SA_ERR_CUDA;
-    const int G = sa::order_group_heads(BH, s.N, D);
-    sa::pair_order_kernel<<<static_cast<unsigned>(BH), sa::pair_order_threads(Nb), smem, st>>>(sig, bits, count, Nb, Tq,
-                                                                                          G, work);
-    if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
-  }
-  return SA_OK;
-}
-
 // kRecall: the P.V filter is the recall test with budget = 1 - recall (lambda unused).
 template <int D, bool kF8 = false, bool kRecall = false>
 sa_status launch_fwd(const sa_shape& s, const void* Q, const void* K, const void* V, const uint8_t* mask,
                      const int32_t* work, float lambda, float scale, int causal, void* O, int64_t* stats,
                      cudaStream_t st, const float* qscale = nullptr, const float* kscale = nullptr,
-                     float budget = 0.f) {
+                     float budget = 0.f, uint8_t* decisions = nullptr) {
   using Cfg = sa::FwdCfg<D, kF8>;
   const int Nb = static_cast<int>(num_blocks(s));
   const int Tq = (Nb + 1) / 2;
@@ -175,14 +119,14 @@ sa_status launch_fwd(const sa_shape& s, const void* Q, const void* K, const void
   if (!make_block_map(&mv, V, s)) return SA_ERR_CUDA;
   if (stats && cudaMemsetAsync(stats, 0, 4 * sizeof(int64_t), st) != cudaSuccess) return SA_ERR_CUDA;
   auto kern = sa::fwd_kernel<D, kF8, kRecall>;
-  if (set_smem(kern, Cfg::kSmemBytes) != SA_OK) return SA_ERR_CUDA;
+  if (sa::set_smem(kern, Cfg::kSmemBytes) != SA_OK) return SA_ERR_CUDA;
   const float LOG2E = 1.4426950408889634f;
   const int lam_on = kRecall ? 1 : (std::isinf(lambda) && lambda < 0 ? 0 : 1);
   kern<<<static_cast<unsigned>(tiles), Cfg::kThreads, Cfg::kSmemBytes, st>>>(
       mq, mk, mv, mask, work, static_cast<__nv_bfloat16*>(O), s.N, Nb, Tq, tiles,
       static_cast<long long>(s.B) * s.H * Nb, scale * LOG2E,
       (lam_on && !kRecall) ? lambda * LOG2E : 0.f, lam_on, budget, causal,
-      reinterpret_cast<unsigned long long*>(stats), qscale, kscale);
+      reinterpret_cast<unsigned long long*>(stats), qscale, kscale, decisions);
   if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   return SA_OK;
 }
@@ -216,7 +160,7 @@ sa_status launch_cluster(const sa_shape& s, const void* X, const void* Y, int it
                                                                                                total);
   if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   constexpr int kAssignSmem = sa::cluster_assign_smem_bytes<D>();
-  if (set_smem(sa::cluster_assign_kernel<D>, kAssignSmem) != SA_OK) return SA_ERR_CUDA;
+  if (sa::set_smem(sa::cluster_assign_kernel<D>, kAssignSmem) != SA_OK) return SA_ERR_CUDA;
   const dim3 order_grid((C + sa::kOrderClusters - 1) / sa::kOrderClusters, by);
   const dim3 cent_grid((C + 7) / 8, by);
   for (int it = 0; it < iters; ++it) {
@@ -287,8 +231,8 @@ sa_status sparse_attn_plan(const void* Q, const void* K, sa_shape s, float tau, 
     return SA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (s.d == 64)
-    return launch_plan<64>(s, Q, K, tau, nullptr, scale, causal != 0, mask, count, idx, work, workspace, st);
-  return launch_plan<128>(s, Q, K, tau, nullptr, scale, causal != 0, mask, count, idx, work, workspace, st);
+    return sa::launch_plan<64>(s, Q, K, tau, nullptr, scale, causal != 0, mask, count, idx, work, workspace, st);
+  return sa::launch_plan<128>(s, Q, K, tau, nullptr, scale, causal != 0, mask, count, idx, work, workspace, st);
 }
 
 sa_status sparse_attn_plan_heads(const void* Q, const void* K, sa_shape s, const float* tau, float scale,
@@ -304,8 +248,8 @@ sa_status sparse_attn_plan_heads(const void* Q, const void* K, sa_shape s, const
     return SA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (s.d == 64)
-    return launch_plan<64>(s, Q, K, 1.f, tau, scale, causal != 0, mask, count, idx, work, workspace, st);
-  return launch_plan<128>(s, Q, K, 1.f, tau, scale, causal != 0, mask, count, idx, work, workspace, st);
+    return sa::launch_plan<64>(s, Q, K, 1.f, tau, scale, causal != 0, mask, count, idx, work, workspace, st);
+  return sa::launch_plan<128>(s, Q, K, 1.f, tau, scale, causal != 0, mask, count, idx, work, workspace, st);
 }
 
 sa_status sparse_attn_fwd(const void* Q, const void* K, const void* V, sa_shape s, const uint8_t* mask,
@@ -340,6 +284,197 @@ sa_status sparse_attn_fwd_recall(const void* Q, const void* K, const void* V, sa
                                        nullptr, budget);
   return launch_fwd<128, false, true>(s, Q, K, V, mask, work, 0.f, scale, causal != 0, O, stats, st, nullptr,
                                       nullptr, budget);
+}
+
+sa_status sparse_attn_fwd_decisions(const void* Q, const void* K, const void* V, sa_shape s,
+                                    const uint8_t* mask, const int32_t* work, int32_t filter, float value,
+                                    float scale, int32_t causal, void* O, int64_t* stats, uint8_t* decisions,
+                                    void* stream) {
+  if (!Q || !K || !V || !mask || !O || !decisions) return SA_ERR_INVALID_ARG;
+  const sa_status sh = check_shape(s);
+  if (sh != SA_OK) return sh;
+  if (filter == SA_FILTER_LAMBDA) {
+    if (std::isnan(value) || (std::isinf(value) && value > 0)) return SA_ERR_INVALID_ARG;
+  } else if (filter == SA_FILTER_RECALL) {
+    if (!(value > 0.f && value <= 1.f)) return SA_ERR_INVALID_ARG;
+  } else {
+    return SA_ERR_INVALID_ARG;
+  }
+  if (!(std::isfinite(scale) && scale > 0.f)) return SA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SA_ERR_INVALID_ARG;
+  if (stats && (reinterpret_cast<uintptr_t>(stats) & 7u) != 0) return SA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool c = causal != 0;
+  if (filter == SA_FILTER_RECALL) {
+    const float budget = 1.f - value;
+    if (s.d == 64)
+      return launch_fwd<64, false, true>(s, Q, K, V, mask, work, 0.f, scale, c, O, stats, st, nullptr, nullptr,
+                                         budget, decisions);
+    return launch_fwd<128, false, true>(s, Q, K, V, mask, work, 0.f, scale, c, O, stats, st, nullptr, nullptr,
+                                        budget, decisions);
+  }
+  if (s.d == 64)
+    return launch_fwd<64>(s, Q, K, V, mask, work, value, scale, c, O, stats, st, nullptr, nullptr, 0.f, decisions);
+  return launch_fwd<128>(s, Q, K, V, mask, work, value, scale, c, O, stats, st, nullptr, nullptr, 0.f, decisions);
+}
+
+// ---------------------------------------------------------------- host-buffer call
+namespace {
+// Device workspace of sparse_attn_host: Q, K, V, O copies, mask, count, work, the
+// plan scratch of the largest head group, and with FP8 scores their codes and scales.
+struct HostWorkspace {
+  size_t q, k, v, o, mask, count, work, plan, q8, k8, qs, ks, total;
+};
+HostWorkspace host_workspace(const sa_shape& s, int chunks, bool fp8) {
+  auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+  const size_t BH = static_cast<size_t>(s.B) * s.H;
+  const size_t Nb = static_cast<size_t>(num_blocks(s)), Tq = (Nb + 1) / 2;
+  const size_t act = BH * s.N * s.d * 2;
+  const long long group = (static_cast<long long>(BH) + chunks - 1) / chunks;
+  HostWorkspace w{};
+  size_t o = 0;
+  w.q = o; o += al(act);
+  w.k = o; o += al(act);
+  w.v = o; o += al(act);
+  w.o = o; o += al(act);
+  w.mask = o; o += al(BH * Nb * Nb);
+  w.count = o; o += al(BH * Nb * 4);
+  w.work = o; o += al(2 * BH * Tq * 4);
+  w.plan = o; o += al(sa::plan_workspace(group, static_cast<int>(Nb), s.d).total);
+  if (fp8) {
+    w.q8 = o; o += al(act / 2);
+    w.k8 = o; o += al(act / 2);
+    w.qs = o; o += al(BH * Nb * 4);
+    w.ks = o; o += al(BH * Nb * 4);
+  }
+  w.total = o;
+  return w;
+}
+}  // namespace
+
+size_t sparse_attn_host_workspace_size(sa_shape s, int32_t chunks, int32_t flags) {
+  if (check_shape(s) != SA_OK || chunks < 1) return 0;
+  const long long BH = static_cast<long long>(s.B) * s.H;
+  return host_workspace(s, static_cast<int>(std::min<long long>(chunks, BH)), (flags & SA_HOST_FP8_SCORES) != 0)
+      .total;
+}
+
+sa_status sparse_attn_host(const void* Qh, const void* Kh, const void* Vh, sa_shape s, float tau,
+                           const float* tau_heads, int32_t filter, float value, float scale, int32_t causal,
+                           int32_t flags, void* Oh, void* workspace,
+                           size_t workspace_bytes, int32_t chunks, void* stream, void* copy_in_stream,
+                           void* copy_out_stream) {
+  if (!Qh || !Kh || !Vh || !Oh) return SA_ERR_INVALID_ARG;
+  const sa_status sh = check_shape(s);
+  if (sh != SA_OK) return sh;
+  const bool fp8 = (flags & SA_HOST_FP8_SCORES) != 0;
+  if ((flags & ~SA_HOST_FP8_SCORES) != 0 || chunks < 1) return SA_ERR_INVALID_ARG;
+  if (tau_heads ? (reinterpret_cast<uintptr_t>(tau_heads) & 3u) != 0 : !(tau > 0.f && tau <= 1.f))
+    return SA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return SA_ERR_INVALID_ARG;
+  if (filter == SA_FILTER_LAMBDA) {
+    if (std::isnan(value) || (std::isinf(value) && value > 0)) return SA_ERR_INVALID_ARG;
+  } else if (filter == SA_FILTER_RECALL) {
+    if (!(value > 0.f && value <= 1.f) || fp8) return SA_ERR_INVALID_ARG;
+  } else {
+    return SA_ERR_INVALID_ARG;
+  }
+  if (fp8 && s.d != 128) return SA_ERR_UNSUPPORTED;
+  const long long BH = static_cast<long long>(s.B) * s.H;
+  const int nch = static_cast<int>(std::min<long long>(chunks, BH));
+  const HostWorkspace L = host_workspace(s, nch, fp8);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < L.total)
+    return SA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaStream_t cin = copy_in_stream ? static_cast<cudaStream_t>(copy_in_stream) : st;
+  cudaStream_t cout = copy_out_stream ? static_cast<cudaStream_t>(copy_out_stream) : st;
+  char* ws = static_cast<char*>(workspace);
+  const int Nb = static_cast<int>(num_blocks(s)), Tq = (Nb + 1) / 2;
+  const size_t row_bytes = static_cast<size_t>(s.N) * s.d * 2;   // one head of Q, K, V or O
+
+  // Events order the three streams; each is released at the end of the call
+  // (the runtime keeps it alive until its recorded work has completed).
+  cudaEvent_t start = nullptr, finish = nullptr;
+  cudaEvent_t ev[2 * 64] = {};
+  const int nev = 2 * std::min(nch, 64);
+  sa_status rc = SA_OK;
+  auto ok = [&](cudaError_t e) {
+    if (e != cudaSuccess && rc == SA_OK) rc = SA_ERR_CUDA;
+    return e == cudaSuccess;
+  };
+  if (!ok(cudaEventCreateWithFlags(&start, cudaEventDisableTiming)) ||
+      !ok(cudaEventCreateWithFlags(&finish, cudaEventDisableTiming)))
+    goto done;
+  for (int i = 0; i < nev; ++i)
+    if (!ok(cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming))) goto done;
+  // the copies may only overwrite the workspace once earlier work on `stream` is done
+  if (!ok(cudaEventRecord(start, st)) || !ok(cudaStreamWaitEvent(cin, start, 0)) ||
+      !ok(cudaStreamWaitEvent(cout, start, 0)))
+    goto done;
+  for (int c = 0; c < nch && rc == SA_OK; ++c) {
+    const long long lo = BH * c / nch, hi = BH * (c + 1) / nch;
+    if (hi == lo) continue;
+    cudaEvent_t in_ready = ev[2 * (c % 64)], out_ready = ev[2 * (c % 64) + 1];
+    const size_t off = static_cast<size_t>(lo) * row_bytes, bytes = static_cast<size_t>(hi - lo) * row_bytes;
+    if (!ok(cudaMemcpyAsync(ws + L.q + off, static_cast<const char*>(Qh) + off, bytes, cudaMemcpyHostToDevice, cin)) ||
+        !ok(cudaMemcpyAsync(ws + L.k + off, static_cast<const char*>(Kh) + off, bytes, cudaMemcpyHostToDevice, cin)) ||
+        !ok(cudaMemcpyAsync(ws + L.v + off, static_cast<const char*>(Vh) + off, bytes, cudaMemcpyHostToDevice, cin)) ||
+        !ok(cudaEventRecord(in_ready, cin)) || !ok(cudaStreamWaitEvent(st, in_ready, 0)))
+      break;
+    const sa_shape g{1, static_cast<int32_t>(hi - lo), s.N, s.d, 64};
+    const void* q = ws + L.q + off;
+    const void* k = ws + L.k + off;
+    const void* v = ws + L.v + off;
+    void* o = ws + L.o + off;
+    uint8_t* mask = reinterpret_cast<uint8_t*>(ws + L.mask) + static_cast<size_t>(lo) * Nb * Nb;
+    int32_t* count = reinterpret_cast<int32_t*>(ws + L.count) + static_cast<size_t>(lo) * Nb;
+    int32_t* work = reinterpret_cast<int32_t*>(ws + L.work) + static_cast<size_t>(2) * lo * Tq;
+    void* pws = ws + L.plan;
+    const float* tg = tau_heads ? tau_heads + lo : nullptr;   // this group's per-head thresholds
+    sa_status r;
+    if (fp8) {
+      uint8_t* q8 = reinterpret_cast<uint8_t*>(ws + L.q8) + off / 2;
+      uint8_t* k8 = reinterpret_cast<uint8_t*>(ws + L.k8) + off / 2;
+      float* qs = reinterpret_cast<float*>(ws + L.qs) + static_cast<size_t>(lo) * Nb;
+      float* ks = reinterpret_cast<float*>(ws + L.ks) + static_cast<size_t>(lo) * Nb;
+      r = sa::launch_plan<128>(g, q, k, tau, tg, scale, causal != 0, mask, count, nullptr, work, pws, st, q8, k8,
+                               qs, ks);
+      if (r == SA_OK)
+        r = launch_fwd<128, true>(g, q8, k8, v, mask, work, value, scale, causal != 0, o, nullptr, st, qs, ks);
+    } else {
+      r = s.d == 64 ? sa::launch_plan<64>(g, q, k, tau, tg, scale, causal != 0, mask, count, nullptr, work, pws, st)
+                    : sa::launch_plan<128>(g, q, k, tau, tg, scale, causal != 0, mask, count, nullptr, work, pws,
+                                           st);
+      if (r == SA_OK) {
+        if (filter == SA_FILTER_RECALL)
+          r = s.d == 64 ? launch_fwd<64, false, true>(g, q, k, v, mask, work, 0.f, scale, causal != 0, o, nullptr,
+                                                      st, nullptr, nullptr, 1.f - value)
+                        : launch_fwd<128, false, true>(g, q, k, v, mask, work, 0.f, scale, causal != 0, o, nullptr,
+                                                       st, nullptr, nullptr, 1.f - value);
+        else
+          r = s.d == 64 ? launch_fwd<64>(g, q, k, v, mask, work, value, scale, causal != 0, o, nullptr, st)
+                        : launch_fwd<128>(g, q, k, v, mask, work, value, scale, causal != 0, o, nullptr, st);
+      }
+    }
+    if (r != SA_OK) {
+      rc = r;
+      break;
+    }
+    if (!ok(cudaEventRecord(out_ready, st)) || !ok(cudaStreamWaitEvent(cout, out_ready, 0)) ||
+        !ok(cudaMemcpyAsync(static_cast<char*>(Oh) + off, ws + L.o + off, bytes, cudaMemcpyDeviceToHost, cout)))
+      break;
+  }
+  // `stream` completes only once the last copy back has
+  if (rc == SA_OK) {
+    ok(cudaEventRecord(finish, cout));
+    ok(cudaStreamWaitEvent(st, finish, 0));
+  }
+done:
+  for (int i = 0; i < nev; ++i)
+    if (ev[i]) cudaEventDestroy(ev[i]);
+  if (start) cudaEventDestroy(start);
+  if (finish) cudaEventDestroy(finish);
+  return rc;
 }
 
 size_t sparse_attn_cluster_workspace_size(sa_shape s) {
@@ -414,7 +549,7 @@ sa_status sparse_attn_plan_q8(const void* Q, const void* K, sa_shape s, float ta
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
       workspace_bytes < sparse_attn_plan_workspace_size(s))
     return SA_ERR_WORKSPACE;
-  return launch_plan<128>(s, Q, K, tau, nullptr, scale, causal != 0, mask, count, idx, work, workspace,
+  return sa::launch_plan<128>(s, Q, K, tau, nullptr, scale, causal != 0, mask, count, idx, work, workspace,
                           static_cast<cudaStream_t>(stream), static_cast<uint8_t*>(Q8), static_cast<uint8_t*>(K8),
                           qscale, kscale);
 }

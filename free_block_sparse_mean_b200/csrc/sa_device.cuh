@@ -14,9 +14,11 @@ namespace sa {
 constexpr int kBlock = 64;    // tokens per mask block
 constexpr int kMaxNb = 4096;  // largest supported number of blocks per head
 
-// Device error word (one per GPU that loads the library). Kernels OR codes into
-// it instead of trapping; the host reads and clears it. All kernels live in one
-// translation unit, so this definition is the only one.
+// Device error word. Kernels OR codes into it instead of trapping; the host reads
+// and clears it. The definition is static, so each translation unit that
+// includes this header has its own copy on every GPU (the library has two:
+// sa_api.cu and sa_noalloc.cu); sparse_attn_device_error reads, clears and ORs
+// both.
 enum : unsigned { DEVERR_TIMEOUT = 1u, DEVERR_RANGE = 2u, DEVERR_VALUE = 4u };
 static __device__ unsigned int g_dev_error;
 

@@ -23,16 +23,18 @@
 // or from two host threads) race on the array and give wrong masks: order them
 // on one stream or otherwise serialise them.
 //
-// The first call on each device looks up the array's device address with
-// cudaGetSymbolAddress (in host code the array's name is only a host-side
-// stand-in, not a device address) and caches it for that device; make that
-// first call before any stream capture on the device.
+// Each call made outside stream capture looks up the array's device address on
+// the current device with cudaGetSymbolAddress (in host code the array's name is
+// only a host-side stand-in, not a device address) and remembers it for that
+// device; a call made while its stream is being captured uses the remembered
+// address. So make the first call on a device before any stream capture on it
+// (a first call inside a capture returns SA_ERR_CUDA).
 #include <cmath>
 #include <cstdint>
 #include <mutex>
 
 #include "../../include/sparse_attn.h"
-#include "plan_kernels.cuh"
+#include "plan_launch.cuh"
 
 namespace {
 
@@ -44,65 +46,25 @@ __device__ __align__(256) unsigned char g_plan_scratch[kNoAllocScratchBytes];
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 
-
-// Device address of the scratch array on the current device (set up once per device).
-sa_status scratch_for_current_device(void** out) {
+// Device address of the scratch array on the current device. A call made outside
+// stream capture looks the address up again (cheap), so a context that was torn
+// down and re-created, e.g. after cudaDeviceReset, gets the array's new address;
+// a call made while `st` is being captured uses the address cached by the last
+// call outside capture, since a lookup could load the module inside the capture.
+sa_status scratch_for_current_device(cudaStream_t st, void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SA_ERR_CUDA;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return SA_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_plan_scratch) != cudaSuccess || p == nullptr) return SA_ERR_CUDA;
     g_scratch_ptr[dev] = p;
+  } else if (!g_scratch_ptr[dev]) {
+    return SA_ERR_CUDA;   // first call on this device inside a capture: no address yet
   }
   *out = g_scratch_ptr[dev];
-  return SA_OK;
-}
-
-template <int D>
-sa_status launch_plan_noalloc(const sa_shape& s, const void* Q, const void* K, float tau, float scale,
-                              int causal, uint8_t* mask, int32_t* count, int32_t* idx, int32_t* work,
-                              void* scratch, cudaStream_t st) {
-  const int Nb = static_cast<int>((static_cast<int64_t>(s.N) + 63) / 64);
-  const long long BH = static_cast<long long>(s.B) * s.H;
-  const sa::PlanWorkspace L = sa::plan_workspace(BH, Nb, D);
-  char* wsb = static_cast<char*>(scratch);
-  float* Qp = reinterpret_cast<float*>(wsb + L.qp);
-  float* Kp = reinterpret_cast<float*>(wsb + L.kp);
-  unsigned long long* sig = reinterpret_cast<unsigned long long*>(wsb + L.sig);
-  uint32_t* bits = reinterpret_cast<uint32_t*>(wsb + L.bits);
-  sa::pool_kernel<D><<<dim3(static_cast<unsigned>(BH * Nb), 2), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Qp, Kp, s.N, Nb);
-  if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
-  // Small heads: 4 query blocks per CTA so the grid still fills the GPU.
-  auto launch_ss = [&](auto kern, int R, int NT) -> sa_status {
-    const int smem = R == 4 ? sa::score_select_smem_bytes<D, 4>(Nb)
-                            : (R == 8 ? sa::score_select_smem_bytes<D, 8>(Nb) : sa::score_select_smem_bytes<D, 16>(Nb));
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return SA_ERR_CUDA;
-    kern<<<dim3((Nb + R - 1) / R, static_cast<unsigned>(BH)), NT, smem, st>>>(Qp, Kp, Nb, scale, causal, tau,
-                                                                               nullptr, mask, count, idx, sig, bits);
-    return SA_OK;
-  };
-  sa_status ls;
-  if (Nb <= 256)
-    ls = launch_ss(sa::score_select_kernel<D, 4, 128>, 4, 128);
-  else if (Nb <= 3000)
-    ls = launch_ss(sa::score_select_kernel<D, 16, 256>, 16, 256);
-  else
-    ls = launch_ss(sa::score_select_kernel<D, 8, 256>, 8, 256);
-  if (ls != SA_OK) return ls;
-  if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
-  if (work) {
-    const int Tq = (Nb + 1) / 2;
-    const int smem = sa::pair_order_smem_bytes(Nb);
-    if (cudaFuncSetAttribute(sa::pair_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
-      return SA_ERR_CUDA;
-    sa::pair_order_kernel<<<static_cast<unsigned>(BH), sa::pair_order_threads(Nb), smem, st>>>(
-        sig, bits, count, Nb, Tq, sa::order_group_heads(BH, s.N, D), work);
-    if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
-  }
   return SA_OK;
 }
 
@@ -138,10 +100,10 @@ extern "C" sa_status sparse_attn_plan_noalloc(const void* Q, const void* K, sa_s
                                                     static_cast<int>((static_cast<int64_t>(s.N) + 63) / 64), s.d);
   if (need.total > kNoAllocScratchBytes) return SA_ERR_WORKSPACE;  // beyond the fixed scratch
   void* scratch = nullptr;
-  const sa_status got = scratch_for_current_device(&scratch);
-  if (got != SA_OK) return got;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const sa_status got = scratch_for_current_device(st, &scratch);
+  if (got != SA_OK) return got;
   if (s.d == 64)
-    return launch_plan_noalloc<64>(s, Q, K, tau, scale, causal != 0, mask, count, idx, work, scratch, st);
-  return launch_plan_noalloc<128>(s, Q, K, tau, scale, causal != 0, mask, count, idx, work, scratch, st);
+    return sa::launch_plan<64>(s, Q, K, tau, nullptr, scale, causal != 0, mask, count, idx, work, scratch, st);
+  return sa::launch_plan<128>(s, Q, K, tau, nullptr, scale, causal != 0, mask, count, idx, work, scratch, st);
 }

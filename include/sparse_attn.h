@@ -139,6 +139,12 @@ sa_status sparse_attn_plan_heads(const void* Q, const void* K, sa_shape s, const
  *   stats     device int64[4] or NULL; zeroed, then filled with: kept (query block,
  *             key block) pairs visited, pairs whose P.V was skipped by lambda,
  *             128x64 score tiles computed, 128x64 P.V tiles computed
+ *
+ * If a bounded device wait gives up (a pipeline stalled for seconds; this does
+ * not happen in a healthy run), the tile stops, records the timeout in the
+ * device error word and leaves its rows of O unwritten: O is undefined for
+ * those rows. A caller that needs to know checks sparse_attn_device_error after
+ * the stream has finished.
  */
 sa_status sparse_attn_fwd(const void* Q, const void* K, const void* V, sa_shape s,
                           const uint8_t* mask, const int32_t* work, float lambda, float scale,
@@ -166,6 +172,74 @@ sa_status sparse_attn_fwd(const void* Q, const void* K, const void* V, sa_shape 
 sa_status sparse_attn_fwd_recall(const void* Q, const void* K, const void* V, sa_shape s,
                                  const uint8_t* mask, const int32_t* work, float recall, float scale,
                                  int32_t causal, void* O, int64_t* stats, void* stream);
+
+/* P.V filter selectors of sparse_attn_fwd_decisions. */
+typedef enum {
+  SA_FILTER_LAMBDA = 0,  /* the lambda test of sparse_attn_fwd; value = lambda (-INFINITY = off) */
+  SA_FILTER_RECALL = 1   /* the cumulative-energy test of sparse_attn_fwd_recall; value = recall */
+} sa_filter;
+
+/* Stage 2 that also records the P.V filter's decisions, for verification: the
+ * filters decide in fp32 on the GPU, so a decision may flip against an fp64
+ * re-computation where the test's margin is within rounding of zero; with the
+ * decisions recorded, a checker can replay exactly the skips the kernel took.
+ * The same kernels, tile order and arithmetic as sparse_attn_fwd (filter =
+ * SA_FILTER_LAMBDA) or sparse_attn_fwd_recall (SA_FILTER_RECALL); the only
+ * extra work is one byte written per visited pair.
+ *
+ *   filter     SA_FILTER_LAMBDA or SA_FILTER_RECALL (else SA_ERR_INVALID_ARG)
+ *   value      lambda or recall, checked as by the call it selects
+ *   decisions  out, device uint8 [B,H,Nb,Nb], not NULL: for every query block i
+ *              and kept, visible key block j the kernel visits, 1 if the pair's
+ *              P.V was skipped, else 0. Entries of other pairs are not written
+ *              (fill the buffer first if they are read).
+ *
+ * All other arguments, outputs and errors are those of sparse_attn_fwd. */
+sa_status sparse_attn_fwd_decisions(const void* Q, const void* K, const void* V, sa_shape s,
+                                    const uint8_t* mask, const int32_t* work, int32_t filter, float value,
+                                    float scale, int32_t causal, void* O, int64_t* stats, uint8_t* decisions,
+                                    void* stream);
+
+/* End to end from host buffers: copy Q, K, V to the device, sparse_attn_plan +
+ * the forward, copy O back, all on the caller's streams. The B*H heads are
+ * independent, so the call pipelines them over `chunks` consecutive groups of
+ * heads: group g's host-to-device copy runs on copy_in_stream, its plan and
+ * forward on `stream`, and its device-to-host copy on copy_out_stream, so the
+ * copies of one group overlap the work of the others in both directions of the
+ * host link.
+ *
+ *   Qh, Kh, Vh  host bf16 [B,H,N,d]; pinned (page-locked) memory makes the copies
+ *               asynchronous DMA, pageable memory works but serialises them
+ *   tau         one recall threshold for every head, as sparse_attn_plan
+ *   tau_heads   NULL, or a DEVICE array of B*H thresholds (4-byte aligned) that
+ *               replaces tau, as sparse_attn_plan_heads (tau is then ignored)
+ *   filter, value  the P.V filter, as sparse_attn_fwd_decisions (SA_FILTER_RECALL
+ *               cannot be combined with SA_HOST_FP8_SCORES)
+ *   scale, causal  as sparse_attn_fwd
+ *   flags       0, or SA_HOST_FP8_SCORES: scores on FP8 codes of Q and K
+ *               (sparse_attn_plan_q8 + sparse_attn_fwd_q8; d must be 128)
+ *   Oh          out, host bf16 [B,H,N,d]; complete once `stream` is
+ *   workspace   device memory of at least sparse_attn_host_workspace_size(s,
+ *               chunks, flags) bytes, 256-byte aligned: the device copies of Q, K,
+ *               V, O, the plan's outputs and scratch. The call waits (on the
+ *               device) for earlier work on `stream` before overwriting it.
+ *   chunks      number of head groups, >= 1 (values above B*H act as B*H)
+ *   stream      the compute stream; when it completes, so has everything the call
+ *               enqueued, the last copy back included
+ *   copy_in_stream, copy_out_stream  streams for the two copy directions, or NULL
+ *               to put that direction on `stream` (no overlap)
+ *
+ * The call enqueues and returns; synchronise `stream` before reading Oh, then
+ * check sparse_attn_device_error if device-side failures matter (see
+ * sparse_attn_fwd). Errors: those of sparse_attn_plan and sparse_attn_fwd, and
+ * SA_ERR_WORKSPACE for a missing, misaligned or short workspace. */
+#define SA_HOST_FP8_SCORES 1
+size_t sparse_attn_host_workspace_size(sa_shape s, int32_t chunks, int32_t flags);
+sa_status sparse_attn_host(const void* Qh, const void* Kh, const void* Vh, sa_shape s, float tau,
+                           const float* tau_heads, int32_t filter, float value, float scale,
+                           int32_t causal, int32_t flags,
+                           void* Oh, void* workspace, size_t workspace_bytes, int32_t chunks,
+                           void* stream, void* copy_in_stream, void* copy_out_stream);
 
 /* Quantized scores (SpargeAttn: "sparse and quantized"; the quantization scheme
  * is this library's own, the pages give none). sparse_attn_plan that also writes

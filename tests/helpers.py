@@ -78,3 +78,37 @@ def assert_output_close(gpu_o: np.ndarray, ref_o: np.ndarray, what: str = ""):
     max_abs, rel = output_errors(gpu_o, ref_o)
     assert max_abs <= MAX_ABS and rel <= REL_FRO, f"{what}: max_abs={max_abs:.3e} rel_fro={rel:.3e}"
     return max_abs, rel
+
+
+LAM_BORDER = 1e-3     # |lam - (rowmax - m)| below this (natural-log units): fp32 may flip the lambda test
+RECALL_BORDER = 1e-4  # |((1 - recall) l - sk alpha - e) / l| below this: fp32 may flip the recall test
+
+
+def check_filter_replay(q, k, v, mask, gpu_out, gpu_dec, *, lam=None, recall=None, causal=False,
+                        qblocks=None, what=""):
+    """The GPU's P.V filter decisions replayed by the oracle's tiled loop.
+
+    gpu_dec: the kernel's decision map (uint8 [B, H, Nb, Nb], zero-filled before
+    the call). The oracle runs the same loop with those decisions forced, so its
+    output must match the GPU's at the output tolerance on every computed row;
+    and at every visited pair its own test must agree with the GPU's decision
+    unless the test's margin is within the fp32 border of zero. Returns
+    (oracle stats, flipped decisions)."""
+    from oracle import sparse_attn_oracle as orc
+    dec = np.asarray(gpu_dec).astype(np.uint8)
+    assert not np.any(dec & (np.asarray(mask) == 0)), "decision recorded for a pair that is not kept"
+    if recall is not None:
+        ref, st = orc.attention_recall(q, k, v, mask, recall, None, causal, qblocks=qblocks, return_stats=True,
+                                       forced=dec)
+        border = RECALL_BORDER
+    else:
+        ref, st = orc.attention_tiled(q, k, v, mask, lam, None, causal, qblocks=qblocks, return_stats=True,
+                                      forced=dec)
+        border = LAM_BORDER
+    assert_output_close(to_np(gpu_out) if isinstance(gpu_out, torch.Tensor) else gpu_out, ref, what)
+    flips = 0
+    for b, h, i, j, own, margin in st["decisions"]:
+        if bool(dec[b, h, i, j]) != own:
+            assert abs(margin) < border, f"{what}: pair {(b, h, i, j)} decided {dec[b, h, i, j]}, margin {margin}"
+            flips += 1
+    return st, flips

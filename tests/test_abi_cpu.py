@@ -184,3 +184,40 @@ def test_plan_heads_rejects_bad_arguments(lib):
     assert lib.sparse_attn_plan_heads(fake, fake, SaShape(1, 2, 128, 96, 64), fake, 0.1, 0, fake, fake, None,
                                       None, fake, ws, None) == 2
     assert lib.sparse_attn_plan_heads(fake, fake, s, fake, 0.1, 0, fake, fake, None, None, None, ws, None) == 3
+
+
+def test_decisions_forward_rejects_bad_arguments(lib):
+    s = SaShape(1, 2, 128, 128, 64)
+
+    def fwd(s=s, filt=0, value=-12.0, dec=FAKE, O=FAKE):
+        return lib.sparse_attn_fwd_decisions(FAKE, FAKE, FAKE, s, FAKE, None, filt, value, 0.1, 0, O, None, dec,
+                                             None)
+
+    assert fwd(dec=None) == 1 and fwd(O=None) == 1
+    assert fwd(filt=2) == 1 and fwd(filt=-1) == 1                   # unknown filter
+    assert fwd(value=float("nan")) == 1 and fwd(value=float("inf")) == 1
+    assert fwd(filt=1, value=0.0) == 1 and fwd(filt=1, value=1.5) == 1
+    assert fwd(s=SaShape(1, 2, 128, 96, 64)) == 2
+
+
+def test_host_call_rejects_bad_arguments(lib):
+    s = SaShape(1, 2, 128, 128, 64)
+    need = lib.sparse_attn_host_workspace_size(s, 2, 0)
+    assert need > 4 * 2 * 128 * 128 * 2                              # the four device copies at least
+    assert lib.sparse_attn_host_workspace_size(s, 0, 0) == 0         # chunks >= 1
+    assert lib.sparse_attn_host_workspace_size(s, 2, 1) > need       # FP8 codes and scales on top
+    ws = ctypes.c_void_p(0x100000)
+
+    def call(s=s, Qh=FAKE, tau=0.9, tau_heads=None, filt=0, value=-12.0, flags=0, ws=ws, nbytes=need, chunks=2):
+        return lib.sparse_attn_host(Qh, FAKE, FAKE, s, tau, tau_heads, filt, value, 0.1, 0, flags, FAKE, ws,
+                                    nbytes, chunks, None, None, None)
+
+    assert call(Qh=None) == 1
+    assert call(tau=0.0) == 1 and call(tau=float("nan")) == 1
+    assert call(tau_heads=ctypes.c_void_p(0x10002)) == 1             # per-head taus must be 4-byte aligned
+    assert call(filt=3) == 1 and call(value=float("nan")) == 1
+    assert call(filt=1, value=0.9, flags=1) == 1                     # recall with FP8 scores: not combined
+    assert call(flags=4) == 1 and call(chunks=0) == 1
+    assert call(flags=1, s=SaShape(1, 2, 128, 64, 64)) == 2           # FP8 scores: d = 128
+    assert call(ws=None) == 3 and call(nbytes=need - 1) == 3
+    assert call(ws=ctypes.c_void_p(0x100010)) == 3                   # workspace 256-byte aligned

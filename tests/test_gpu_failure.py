@@ -40,3 +40,24 @@ def test_bounded_wait_times_out_and_context_survives():
     mask = to_np(plan.mask)
     ref = orc.fwd(q.cpu(), k.cpu(), v.cpu(), mask, -12.0)
     assert_output_close(to_np(o), ref, "tiny workload after the timeout diagnostic")
+
+
+def test_public_host_call_raises_on_a_device_error():
+    """sparse_attention reads the device error word after its work: a fired check
+    (here the timeout diagnostic's, left in the word before the call) raises
+    SparseAttnError with SA_ERR_DEVICE_CHECK instead of returning a silent
+    result; the word is cleared by that read, and the next call succeeds."""
+    dev = torch.device("cuda:0")
+    w = wl.WORKLOADS["tiny"]
+    q, k, v = wl.generate(w, seed=0, device=dev)
+    qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+    torch.cuda.synchronize()
+    assert sa.sparse_attn_device_error() == 0
+    sa.sparse_attn_selftest_wait_timeout(50_000)       # records a timeout, returns normally
+    with pytest.raises(sa.SparseAttnError) as ei:
+        sa.sparse_attention(qh, kh, vh, 0.95, -12.0)
+    assert ei.value.status == 5                        # SA_ERR_DEVICE_CHECK
+    o = sa.sparse_attention(qh, kh, vh, 0.95, -12.0)
+    ref = sa.sparse_attn_fwd(q, k, v, sa.sparse_attn_plan(q, k, 0.95), -12.0)
+    torch.cuda.synchronize()
+    assert torch.equal(o, ref.cpu())

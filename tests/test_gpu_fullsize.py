@@ -3,16 +3,18 @@ times (plan with the tile order, forward over the plan's pairs).
 
 Masks: every head (every 4th for the extra centroid weights) against the
 oracle's plan (exact outside the 1e-4 band).
-Outputs: the oracle run with the GPU's own mask on sampled query blocks (the
-first, the last, which is the ragged tail when N % 64 != 0, and seeded random
-ones) of a few heads; each query block's output is independent given the mask,
-so the sampled rows are exact comparisons."""
+Outputs: the oracle run with the GPU's own mask on 64 seeded query blocks plus
+the first and the last (the ragged tail when N % 64 != 0) of the sampled heads;
+each query block's output is independent given the mask, so the sampled rows
+are exact comparisons. With lambda the oracle replays the GPU's recorded skip
+decisions, and each decision is checked against the oracle's own test."""
 import numpy as np
 import pytest
 import torch
 
 from oracle import sparse_attn_oracle as orc
-from tests.helpers import assert_output_close, check_plan_consistency, compare_masks, to_np
+from tests.helpers import (assert_output_close, check_filter_replay, check_plan_consistency, compare_masks,
+                           output_errors, to_np)
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -20,14 +22,24 @@ if torch.cuda.is_available():
     import free_block_sparse_mean_b200 as sa
     from free_block_sparse_mean_b200 import workloads as wl
 
+SAMPLED_QBLOCKS = 64
+
 CASES = [
     # workload, tau, lambda, centroid weight, heads whose outputs are sampled, mask-head stride
     ("wan", 0.95, None, None, (0, 23), 1),
-    ("hunyuan", 0.95, -12.0, None, (0, 17), 1),
-    ("hunyuan", 0.90, -12.0, 3.0, (5,), 4),
     ("hunyuan", 0.90, -12.0, 0.5, (9,), 4),
+    ("hunyuan", 0.90, -12.0, 1.5, (2,), 4),
+    ("hunyuan", 0.90, -12.0, 3.0, (5,), 4),
+    ("hunyuan", 0.95, -12.0, 0.5, (7,), 4),
+    ("hunyuan", 0.95, -12.0, 1.5, (0, 17), 1),
+    ("hunyuan", 0.95, -12.0, 3.0, (21,), 4),
     ("lm", 0.95, None, None, (0, 31), 1),
 ]
+
+
+def sampled_qblocks(Nb, seed):
+    rng = np.random.default_rng(seed)
+    return sorted({0, Nb - 1, *rng.choice(Nb, size=min(Nb, SAMPLED_QBLOCKS), replace=False).tolist()})
 
 
 @pytest.mark.parametrize("name,tau,lam,cw,out_heads,stride", CASES)
@@ -35,13 +47,15 @@ def test_full_size_masks_and_sampled_outputs(name, tau, lam, cw, out_heads, stri
     dev = torch.device("cuda:0")
     w = wl.WORKLOADS[name]
     q, k, v = wl.generate(w, seed=0, device=dev, centroid_weight=cw)
-    plan = sa.sparse_attn_plan(q, k, tau, None, w.causal)
-    out = sa.sparse_attn_fwd(q, k, v, plan, lam)
+    Nb = -(-w.N // 64)
+    plan = sa.sparse_attn_plan(q, k, tau, None, w.causal, with_idx=True)
+    dec = torch.zeros((w.B, w.H, Nb, Nb), dtype=torch.uint8, device=dev)
+    out = sa.sparse_attn_fwd(q, k, v, plan, lam, decisions=dec)
     torch.cuda.synchronize()
     assert sa.sparse_attn_device_error() == 0
-    Nb = -(-w.N // 64)
     mask = to_np(plan.mask)
     check_plan_consistency(mask[0, :2], to_np(plan.count)[0, :2], to_np(plan.idx)[0, :2])
+    del plan
     rows_diff = excused = 0
     heads = range(0, w.H, stride)
     for h in heads:
@@ -53,13 +67,23 @@ def test_full_size_masks_and_sampled_outputs(name, tau, lam, cw, out_heads, stri
     print(f"{name} tau={tau} cw={cw}: rows differing {rows_diff} of {len(heads) * Nb}, excused blocks {excused}, "
           f"density {mask.mean():.3f}")
     assert rows_diff <= max(2, (len(heads) * Nb) // 500)
-    rng = np.random.default_rng(7)
+    dec_np = to_np(dec) if lam is not None else None
     for h in out_heads:
-        qbs = sorted({0, Nb - 1, *rng.choice(Nb, size=4, replace=False).tolist()})
+        qbs = sampled_qblocks(Nb, 7 + h)
         qh, kh, vh = (x[:, h:h + 1].cpu() for x in (q, k, v))
-        ref = orc.fwd(qh, kh, vh, mask[:, h:h + 1], lam, None, w.causal, qblocks=qbs)
         got = to_np(out[:, h:h + 1])
-        assert_output_close(got, ref, f"{name} head {h} query blocks {qbs}")
+        if lam is None:
+            ref = orc.fwd(qh, kh, vh, mask[:, h:h + 1], None, None, w.causal, qblocks=qbs)
+            assert_output_close(got, ref, f"{name} head {h}, {len(qbs)} query blocks")
+        else:
+            _, flips = check_filter_replay(qh, kh, vh, mask[:, h:h + 1], got, dec_np[:, h:h + 1], lam=lam,
+                                           causal=w.causal, qblocks=qbs,
+                                           what=f"{name} cw={cw} head {h}, {len(qbs)} query blocks")
+            print(f"  head {h}: {flips} lambda decisions flipped within the border")
+        dense = orc.attention_masked(qh, kh, vh, np.ones((1, 1, Nb, Nb), np.uint8), None, w.causal,
+                                     qblocks=qbs[:8])
+        ma, rel = output_errors(got, dense)
+        print(f"  head {h}: sparse-vs-dense on 8 query blocks max_abs={ma:.3e} rel_fro={rel:.3e}")
 
 
 def test_full_mask_natural_pairs_repeated():

@@ -10,8 +10,8 @@ import pytest
 import torch
 
 from oracle import sparse_attn_oracle as orc
-from tests.helpers import (assert_output_close, check_plan_consistency, compare_masks,
-                           output_errors, to_np)
+from tests.helpers import (assert_output_close, check_filter_replay, check_plan_consistency,
+                           compare_masks, output_errors, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -29,7 +29,7 @@ def _no_device_error():
 
 
 def _plan_and_check(q, k, tau, causal, scale=None):
-    p = sa.sparse_attn_plan(q, k, tau, scale, causal)
+    p = sa.sparse_attn_plan(q, k, tau, scale, causal, with_idx=True)
     torch.cuda.synchronize()
     mask, count, idx = to_np(p.mask), to_np(p.count), to_np(p.idx)
     check_plan_consistency(mask, count, idx)
@@ -140,7 +140,10 @@ def test_fwd_random_mask(N, d, causal, density):
 @pytest.mark.parametrize("lam", [-12.0, -6.0, -3.0])
 def test_fwd_lambda_skip(lam):
     """Key block 0 aligned with all queries, the rest weaker: later blocks fall
-    below lambda; GPU skips must give the oracle's tiled-loop output."""
+    below lambda. The oracle's tiled loop must give the GPU's output both on its
+    own decisions (up to fp32 flips) and, exactly at the tolerance, when it
+    replays the GPU's recorded decisions; each GPU decision must agree with the
+    oracle's test unless that test's margin is within the fp32 border."""
     N, d = 1024, 128
     q, k, v = wl.random_qkv(1, 2, N, d, seed=5, device=_dev())
     u = torch.ones(d, device=_dev())
@@ -151,27 +154,65 @@ def test_fwd_lambda_skip(lam):
     Nb = N // 64
     mask = torch.ones((1, 2, Nb, Nb), dtype=torch.uint8, device=_dev())
     stats = torch.zeros(4, dtype=torch.int64, device=_dev())
-    o = sa.sparse_attn_fwd(q, k, v, mask, lam, stats=stats)
+    dec = torch.zeros((1, 2, Nb, Nb), dtype=torch.uint8, device=_dev())
+    o = sa.sparse_attn_fwd(q, k, v, mask, lam, stats=stats, decisions=dec)
     torch.cuda.synchronize()
+    _no_device_error()
     ref, st = orc.attention_tiled(q.cpu(), k.cpu(), v.cpu(), to_np(mask).astype(np.uint8), lam,
                                   return_stats=True)
     assert_output_close(to_np(o), ref, f"lambda={lam}")
+    st_r, flips = check_filter_replay(q.cpu(), k.cpu(), v.cpu(), to_np(mask).astype(np.uint8), o, to_np(dec),
+                                      lam=lam, what=f"lambda={lam} replay")
     s = to_np(stats)
-    assert s[0] == st["kept_pairs"]
-    assert abs(int(s[1]) - st["pv_skipped"]) <= max(2, st["pv_skipped"] // 100)
+    assert s[0] == st["kept_pairs"] == st_r["kept_pairs"]
+    assert s[1] == int(to_np(dec).sum())
+    assert abs(int(s[1]) - st["pv_skipped"]) <= flips
 
 
-@pytest.mark.parametrize("tau,lam", [(0.9, None), (0.95, -12.0), (0.99, -12.0)])
+def test_fwd_lambda_plain_call_equals_recorded():
+    """sparse_attn_fwd and sparse_attn_fwd_decisions run the same kernel: the
+    outputs and the counts are bit-identical."""
+    w = wl.WORKLOADS["small"].with_(H=4)
+    q, k, v = wl.generate(w, seed=2, device=_dev())
+    p = sa.sparse_attn_plan(q, k, 0.95)
+    s1 = torch.zeros(4, dtype=torch.int64, device=_dev())
+    s2 = torch.zeros(4, dtype=torch.int64, device=_dev())
+    dec = torch.zeros((1, 4, 64, 64), dtype=torch.uint8, device=_dev())
+    a = sa.sparse_attn_fwd(q, k, v, p, -12.0, stats=s1)
+    b = sa.sparse_attn_fwd(q, k, v, p, -12.0, stats=s2, decisions=dec)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and torch.equal(s1, s2)
+    assert int(dec.sum()) == int(s2[1]) > 0
+
+
+SMALL_POINTS = [(tau, lam) for tau in (0.90, 0.95, 0.99) for lam in (None, -12.0)]
+
+
+@pytest.mark.parametrize("tau,lam", SMALL_POINTS)
 def test_small_workload(tau, lam):
-    """The small DiT-layer shape (H=24, d=128, N=4096), all heads."""
+    """The small DiT-layer shape (H=24, d=128, N=4096), all heads, at every
+    configured (tau, lambda) point: masks against the oracle's plan, outputs
+    against the oracle on the GPU's mask (with lambda: replaying the GPU's
+    recorded decisions, every decision checked against the oracle's test)."""
     w = wl.WORKLOADS["small"]
     q, k, v = wl.generate(w, seed=0, device=_dev())
     p, mask, op = _plan_and_check(q, k, tau, False)
-    o = sa.sparse_attn_fwd(q, k, v, p, lam)
+    dec = torch.zeros((1, w.H, 64, 64), dtype=torch.uint8, device=_dev())
+    o = sa.sparse_attn_fwd(q, k, v, p, lam, decisions=dec)
     torch.cuda.synchronize()
-    ref = orc.fwd(q.cpu(), k.cpu(), v.cpu(), mask, lam)
-    assert_output_close(to_np(o), ref, f"small tau={tau} lam={lam}")
     _no_device_error()
+    if lam is None:
+        ref = orc.fwd(q.cpu(), k.cpu(), v.cpu(), mask, lam)
+        assert_output_close(to_np(o), ref, f"small tau={tau} lam={lam}")
+        assert int(dec.sum()) == 0
+    else:
+        _, flips = check_filter_replay(q.cpu(), k.cpu(), v.cpu(), mask, o, to_np(dec), lam=lam,
+                                       what=f"small tau={tau} lam={lam}")
+        print(f"small tau={tau} lam={lam}: {int(dec.sum())} skipped, {flips} flips within the border")
+    dense = orc.attention_masked(q[:, :2].cpu(), k[:, :2].cpu(), v[:, :2].cpu(), np.ones_like(mask[:, :2]))
+    max_abs, rel = output_errors(to_np(o[:, :2]), dense)
+    print(f"small tau={tau} lam={lam}: sparse-vs-dense (heads 0-1) max_abs={max_abs:.3e} rel_fro={rel:.3e}, "
+          f"density={mask.mean():.3f}")
 
 
 def test_tiny_workload_and_sparse_vs_dense():
@@ -203,7 +244,7 @@ def test_per_head_tau_matches_oracle_and_flags_invalid_values():
     w = wl.WORKLOADS["small"]
     q, k, _ = wl.generate(w, seed=0, device=_dev())
     taus = torch.linspace(0.85, 0.99, w.H, dtype=torch.float32, device=_dev())
-    p = sa.sparse_attn_plan(q, k, taus)
+    p = sa.sparse_attn_plan(q, k, taus, with_idx=True)
     torch.cuda.synchronize()
     _no_device_error()
     mask, count, idx = to_np(p.mask), to_np(p.count), to_np(p.idx)
@@ -232,20 +273,57 @@ def test_per_head_tau_matches_oracle_and_flags_invalid_values():
 
 
 def test_end_to_end_from_pinned_host_buffers():
-    """sparse_attention (host in, host out, pipelined over head groups) returns
-    exactly what the device-side plan + forward return, for any number of groups
-    and for a per-head tau: heads are independent, so grouping changes nothing."""
+    """sparse_attention (the C call sparse_attn_host: host in, host out, pipelined
+    over head groups on three streams) returns exactly what the device-side plan +
+    forward return, for any number of groups, for a per-head tau, for the recall
+    filter and for FP8 scores: heads are independent, so grouping changes nothing."""
     w = wl.WORKLOADS["small"].with_(H=6)
     q, k, v = wl.generate(w, seed=3, device=_dev())
     ref = sa.sparse_attn_fwd(q, k, v, sa.sparse_attn_plan(q, k, 0.95), -12.0)
     taus = torch.linspace(0.9, 0.97, w.H, dtype=torch.float32, device=_dev())
     ref_t = sa.sparse_attn_fwd(q, k, v, sa.sparse_attn_plan(q, k, taus), -12.0)
+    ref_r = sa.sparse_attn_fwd(q, k, v, sa.sparse_attn_plan(q, k, 0.9), recall=0.95)
+    p8 = sa.sparse_attn_plan(q, k, 0.95, quantize=True)
+    ref_8 = sa.sparse_attn_fwd(q, k, v, p8, -12.0, qk_fp8=True)
     torch.cuda.synchronize()
     qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
     for chunks in (1, 4, 6):
         o = sa.sparse_attention(qh, kh, vh, 0.95, -12.0, chunks=chunks)
         assert o.device.type == "cpu" and o.is_pinned()
         assert torch.equal(o, ref.cpu()), f"chunks={chunks}"
-    o_t = sa.sparse_attention(qh, kh, vh, taus, -12.0, chunks=4)
-    assert torch.equal(o_t, ref_t.cpu())
+    assert torch.equal(sa.sparse_attention(qh, kh, vh, taus, -12.0, chunks=4), ref_t.cpu())
+    assert torch.equal(sa.sparse_attention(qh, kh, vh, 0.9, recall=0.95, chunks=3), ref_r.cpu())
+    assert torch.equal(sa.sparse_attention(qh, kh, vh, 0.95, -12.0, chunks=2, qk_fp8=True), ref_8.cpu())
     _no_device_error()
+
+
+def test_host_call_through_the_c_abi_on_one_stream():
+    """sparse_attn_host called directly, both copy directions on the compute
+    stream (NULL copy streams), pageable input buffers: same output."""
+    import ctypes
+    from free_block_sparse_mean_b200 import _lib
+    lib = _lib.load()
+    w = wl.WORKLOADS["small"].with_(H=3)
+    q, k, v = wl.generate(w, seed=4, device=_dev())
+    ref = sa.sparse_attn_fwd(q, k, v, sa.sparse_attn_plan(q, k, 0.9), None)
+    torch.cuda.synchronize()
+    qh, kh, vh = (x.cpu() for x in (q, k, v))
+    oh = torch.empty_like(qh)
+    s = _lib.SaShape(1, w.H, w.N, w.D, 64)
+    nbytes = int(lib.sparse_attn_host_workspace_size(s, 2, 0))
+    ws = torch.empty((nbytes,), dtype=torch.uint8, device=_dev())
+    stream = torch.cuda.current_stream(_dev())
+    st = lib.sparse_attn_host(ctypes.c_void_p(qh.data_ptr()), ctypes.c_void_p(kh.data_ptr()),
+                              ctypes.c_void_p(vh.data_ptr()), s, 0.9, None, _lib.SA_FILTER_LAMBDA,
+                              float("-inf"), w.D ** -0.5, 0, 0, ctypes.c_void_p(oh.data_ptr()),
+                              ctypes.c_void_p(ws.data_ptr()), nbytes, 2, ctypes.c_void_p(stream.cuda_stream),
+                              None, None)
+    assert st == 0, lib.sparse_attn_status_string(st)
+    stream.synchronize()
+    assert torch.equal(oh, ref.cpu())
+    st = lib.sparse_attn_host(ctypes.c_void_p(qh.data_ptr()), ctypes.c_void_p(kh.data_ptr()),
+                              ctypes.c_void_p(vh.data_ptr()), s, 0.9, None, _lib.SA_FILTER_LAMBDA,
+                              float("-inf"), w.D ** -0.5, 0, 0, ctypes.c_void_p(oh.data_ptr()),
+                              ctypes.c_void_p(ws.data_ptr()), nbytes - 256, 2,
+                              ctypes.c_void_p(stream.cuda_stream), None, None)
+    assert st == 3                        # SA_ERR_WORKSPACE: too small, nothing enqueued

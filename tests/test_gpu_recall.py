@@ -1,22 +1,18 @@
 """The cumulative-energy (recall) P.V filter on the GPU against the oracle's
 tiled-loop run of the same test (oracle.attention_recall), through the C ABI.
 
-The GPU takes each skip decision in fp32; it may differ from the oracle's fp64
-decision only where the oracle's margin ((1 - recall) l - sk alpha - e) / l is
-within rounding of zero (|margin| < 1e-4 here, far above fp32 rounding of the
-sums). A flip changes sk, so the later decisions of that query block may differ
-too: such a query block is excused from the strict comparison, and both outputs
-then lie within (1 - recall) max|V| of the unfiltered one, so they differ by at
-most twice that. Every other query block must match to the usual tolerance
-(max-abs 2e-2, relative Frobenius 1e-2), and the skip counts may differ by at
-most the number of decisions from the first borderline one on in the excused
-query blocks."""
+The GPU takes each skip decision in fp32 and records it
+(sparse_attn_fwd_decisions). The oracle replays those decisions, so every
+sampled output row is compared at the usual tolerance (max-abs 2e-2, relative
+Frobenius 1e-2), and at every visited pair the oracle's own fp64 test must
+agree with the GPU's decision unless its margin ((1 - recall) l - sk alpha - e)
+/ l lies within 1e-4 of zero. The skip counts equal the recorded skips."""
 import numpy as np
 import pytest
 import torch
 
 from oracle import sparse_attn_oracle as orc
-from tests.helpers import assert_output_close, to_np
+from tests.helpers import check_filter_replay, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -24,40 +20,40 @@ if torch.cuda.is_available():
     import free_block_sparse_mean_b200 as sa
     from free_block_sparse_mean_b200 import workloads as wl
 
-BORDER = 1e-4     # |margin| below this: the fp32 and fp64 decisions may differ
-
 
 def _dev():
     return torch.device("cuda:0")
 
 
-def _check_against_oracle(q, k, v, mask_np, recall, causal, o_gpu, stats_gpu, qblocks=None,
-                          max_excused_frac=0.25):
-    ref, st = orc.attention_recall(q.cpu(), k.cpu(), v.cpu(), mask_np, recall, None, causal,
-                                   qblocks=qblocks, return_stats=True)
-    got = to_np(o_gpu)
+def _run_checked(q, k, v, plan_or_mask, recall, causal, heads=None, qblocks=None, what=""):
+    """Forward with the recall filter, decisions recorded, checked head by head
+    (`heads`: sampled heads, default all; `qblocks`: sampled query blocks)."""
     B, H, N, _ = q.shape
-    excused, cascade = set(), 0
-    for b, h, i, j, skipped, margin in st["decisions"]:
-        if (b, h, i) in excused or abs(margin) < BORDER:
-            excused.add((b, h, i))
-            cascade += 1
-    vmax = float(np.abs(to_np(v)).max())
-    strict = np.isfinite(ref)
-    for b, h, i in excused:
-        rows = slice(i * 64, min(N, i * 64 + 64))
-        diff = np.abs(got[b, h, rows] - ref[b, h, rows]).max()
-        assert diff <= 2e-2 + 2 * (1 - recall) * vmax, (b, h, i, diff)
-        strict[b, h, rows] = False
-    assert_output_close(got, np.where(strict, ref, np.nan), f"recall={recall}")
-    n_q = len(list(qblocks)) * B * H if qblocks is not None else B * H * (-(-N // 64))
-    assert len(excused) <= max(2, int(n_q * max_excused_frac)), f"{len(excused)} of {n_q} query blocks excused"
-    if stats_gpu is not None:
-        s = to_np(stats_gpu)
-        assert s[0] == st["kept_pairs"]
-        assert abs(int(s[1]) - st["pv_skipped"]) <= cascade
-        return int(s[1]), st
-    return None, st
+    Nb = -(-N // 64)
+    stats = torch.zeros(4, dtype=torch.int64, device=_dev())
+    dec = torch.zeros((B, H, Nb, Nb), dtype=torch.uint8, device=_dev())
+    o = sa.sparse_attn_fwd(q, k, v, plan_or_mask, None, None, causal, recall=recall, stats=stats, decisions=dec)
+    torch.cuda.synchronize()
+    assert sa.sparse_attn_device_error() == 0
+    mask = to_np(plan_or_mask.mask if isinstance(plan_or_mask, sa.Plan) else plan_or_mask).astype(np.uint8)
+    dec_np, s = to_np(dec), to_np(stats)
+    assert s[1] == int(dec_np.sum())                    # the recorded skips are the counted ones
+    flips = 0
+    kept = 0
+    rec_min = 1.0
+    for h in (range(H) if heads is None else heads):
+        sl = slice(h, h + 1)
+        st, f = check_filter_replay(q[:, sl].cpu(), k[:, sl].cpu(), v[:, sl].cpu(), mask[:, sl], o[:, sl],
+                                    dec_np[:, sl], recall=recall, causal=causal, qblocks=qblocks,
+                                    what=f"{what} head {h}")
+        flips += f
+        kept += st["kept_pairs"]
+        rec_rows = st["recall_rows"]
+        if np.isfinite(rec_rows).any():
+            rec_min = min(rec_min, float(np.nanmin(rec_rows)))
+    if heads is None and qblocks is None:
+        assert s[0] == kept
+    return int(s[1]), flips, rec_min
 
 
 def _constructed(N, d, seed, aligned, a, spread):
@@ -86,13 +82,10 @@ def test_recall_constructed(recall, aligned, d):
     q, k, v = _constructed(N, d, 11 + aligned, aligned, a, spread)
     Nb = N // 64
     mask = torch.ones((1, 2, Nb, Nb), dtype=torch.uint8, device=_dev())
-    stats = torch.zeros(4, dtype=torch.int64, device=_dev())
-    o = sa.sparse_attn_fwd(q, k, v, mask, recall=recall, stats=stats)
-    torch.cuda.synchronize()
-    assert sa.sparse_attn_device_error() == 0
-    skipped, st = _check_against_oracle(q, k, v, to_np(mask).astype(np.uint8), recall, False, o, stats)
+    skipped, flips, rec_min = _run_checked(q, k, v, mask, recall, False, what=f"recall={recall}")
     assert skipped > 0
-    assert np.nanmin(st["recall_rows"]) >= recall - 1e-12
+    assert rec_min >= recall - 1e-12
+    print(f"recall {recall} d {d}: skipped {skipped}, decisions within the border that flipped: {flips}")
 
 
 @pytest.mark.parametrize("tau,recall", [(0.95, 0.99), (0.99, 0.95)])
@@ -101,26 +94,14 @@ def test_recall_small_workload_with_plan(tau, recall):
     w = wl.WORKLOADS["small"]
     q, k, v = wl.generate(w, seed=0, device=_dev())
     p = sa.sparse_attn_plan(q, k, tau)
-    stats = torch.zeros(4, dtype=torch.int64, device=_dev())
-    o = sa.sparse_attn_fwd(q, k, v, p, recall=recall, stats=stats)
-    torch.cuda.synchronize()
-    assert sa.sparse_attn_device_error() == 0
-    heads = [0, 5, 23]
-    mask = to_np(p.mask).astype(np.uint8)
-    for h in heads:
-        sl = slice(h, h + 1)
-        _check_against_oracle(q[:, sl], k[:, sl], v[:, sl], mask[:, sl], recall, False, o[:, sl], None)
+    _run_checked(q, k, v, p, recall, False, heads=[0, 5, 23], what=f"small tau={tau} recall={recall}")
 
 
 def test_recall_causal_ragged_two_batches():
     """B = 2, causal, N = 1000 (a tail of 40 rows), d = 64, plan with tau = 0.9."""
     q, k, v = wl.random_qkv(2, 2, 1000, 64, seed=3, device=_dev())
     p = sa.sparse_attn_plan(q, k, 0.9, None, True)
-    stats = torch.zeros(4, dtype=torch.int64, device=_dev())
-    o = sa.sparse_attn_fwd(q, k, v, p, recall=0.9, stats=stats)
-    torch.cuda.synchronize()
-    assert sa.sparse_attn_device_error() == 0
-    _check_against_oracle(q, k, v, to_np(p.mask).astype(np.uint8), 0.9, True, o, stats)
+    _run_checked(q, k, v, p, 0.9, True, what="causal ragged B=2")
 
 
 def test_recall_one_is_the_unfiltered_forward():
@@ -138,25 +119,18 @@ def test_recall_one_is_the_unfiltered_forward():
 @pytest.mark.slow
 def test_recall_full_size_sampled():
     """HunyuanVideo shape (H = 24, N = 118,800: a ragged tail), tau = 0.95, recall
-    0.99, in the benchmark's launch configuration; sampled query blocks of two
-    heads against the oracle. Rows this long fill their budget over hundreds of
-    small blocks, so most query blocks meet a decision within 1e-4 of the
-    threshold somewhere along the row: those are held to the 2 (1 - recall) max|V|
-    bound, the rest to the usual tolerance."""
+    0.99, in the benchmark's launch configuration: 64 seeded query blocks plus the
+    first and the ragged last of two heads, every row at the output tolerance
+    under the GPU's own decisions, and the decisions against the oracle's test."""
     w = wl.WORKLOADS["hunyuan"]
     q, k, v = wl.generate(w, seed=0, device=_dev())
     p = sa.sparse_attn_plan(q, k, 0.95, None, w.causal)
-    o = sa.sparse_attn_fwd(q, k, v, p, recall=0.99)
-    torch.cuda.synchronize()
-    assert sa.sparse_attn_device_error() == 0
     Nb = -(-w.N // 64)
-    mask = to_np(p.mask).astype(np.uint8)
     rng = np.random.default_rng(5)
-    for h in (0, 13):
-        qbs = sorted({0, Nb - 1, *rng.choice(Nb, size=6, replace=False).tolist()})
-        sl = slice(h, h + 1)
-        _check_against_oracle(q[:, sl].cpu(), k[:, sl].cpu(), v[:, sl].cpu(), mask[:, sl], 0.99, w.causal,
-                              o[:, sl], None, qblocks=qbs, max_excused_frac=1.0)
+    qbs = sorted({0, Nb - 1, *rng.choice(Nb, size=64, replace=False).tolist()})
+    skipped, flips, _ = _run_checked(q, k, v, p, 0.99, w.causal, heads=(0, 13), qblocks=qbs,
+                                     what="hunyuan recall 0.99")
+    print(f"hunyuan recall 0.99: {skipped} pairs skipped; {flips} sampled decisions flipped within the border")
 
 
 def test_recall_argument_errors():
