@@ -2,11 +2,18 @@
 """Benchmark of the block-sparse attention path (stage 1 plan + stage 2 forward).
 
 One step = sparse_attn_plan + sparse_attn_fwd over one batch of resident bf16
-Q/K/V of the chosen workload (default: the small DiT-layer shape, B=1 H=24 N=4096
-d=128, tau=0.95, lambda=-12). Prints ONE JSON line on rank 0.
+Q/K/V of the chosen workload (default: the largest configured shape, the
+HunyuanVideo-13B-shaped layer B=1 H=24 N=118,800 d=128 with centroid weight 1.5,
+tau=0.95, lambda=-12). Prints ONE JSON line on rank 0.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload small|tiny|wan|hunyuan|lm]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload hunyuan|wan|lm|small|tiny]
                     [--tau T] [--lam L|off] [--recall R] [--impl ours|reference]
+
+On rank 0 of a one-GPU run the line also carries the CPU oracle's timing
+(cpu_baseline) and, from the same oracle runs, the parity of the timed
+configuration (parity): mask rows differing from the oracle's plan and the
+blocks the 1e-4 tau band excuses, the output error against the oracle run on
+the GPU's mask and filter decisions, and the sparse-vs-dense error.
 
 Multi-GPU: the path has no exchange step; N ranks run N independent replicas of
 the same workload (weak scaling), timed on the device, max over ranks.
@@ -23,6 +30,7 @@ import subprocess
 import sys
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -44,7 +52,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="small", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--workload", default="hunyuan", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--tau", type=float, default=0.95)
     ap.add_argument("--lam", default="-12")
     ap.add_argument("--centroid-weight", type=float, default=None)
@@ -194,10 +202,30 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
-# --------------------------------------------------------------------------- CPU oracle timing
-def time_oracle(w, tau, lam, budget_s, seed, recall=None, cluster_iters=None):
-    """The oracle as it stands (fp64 NumPy) on a bounded sample of the workload:
-    whole heads (plan + forward) until the time budget is used, at least one."""
+# --------------------------------------------------------------------------- CPU oracle leg
+def oracle_qblocks(w):
+    """The query blocks the oracle's forward covers per head: all of them for
+    short heads, else 16 spread over the head (the first and the last included)."""
+    nb = -(-w.N // 64)
+    if w.N <= 8192:
+        return None
+    step = max(1, nb // 15)
+    return sorted(set(list(range(0, nb, step))[:15]) | {nb - 1})
+
+
+def time_oracle(w, tau, lam, budget_s, seed, recall=None, cluster_iters=None, gpu=None):
+    """The oracle as it stands (fp64 NumPy, host cores) on a bounded sample of the
+    workload: whole heads of plan + forward (the forward on oracle_qblocks for long
+    heads) until the time budget is used, at least one head.
+
+    gpu, if given, holds host copies of the timed configuration's device tensors
+    (q, k, v, out, mask, dec: inputs, output, mask and recorded filter decisions)
+    by head; the oracle then runs on those exact inputs, its forward on the GPU's
+    mask replaying the GPU's decisions, and the same runs give the parity fields
+    (returned as a dict, else None): the GPU mask against the oracle's plan (exact
+    outside the 1e-4 tau band), the GPU output against the oracle's, and the
+    sparse-vs-dense error (the oracle with every block kept, on up to 4 of the
+    sampled query blocks; not timed)."""
     from oracle import sparse_attn_oracle as orc
     try:
         import threadpoolctl
@@ -205,15 +233,22 @@ def time_oracle(w, tau, lam, budget_s, seed, recall=None, cluster_iters=None):
     except Exception:
         cores = os.cpu_count()
     per_head_dense = dense_flops(w) / (w.B * w.H)
-    if w.N > 8192:
-        qblocks = list(range(0, -(-w.N // 64), max(1, (-(-w.N // 64)) // 16)))[:16]
-    else:
-        qblocks = None
+    nb = -(-w.N // 64)
+    qblocks = oracle_qblocks(w)
     t_total = 0.0
     flops = 0.0
     heads = 0
+    par = None
+    if gpu is not None:
+        from tests.helpers import BAND, compare_masks, output_errors
+        par = {"heads": [], "mask_rows": 0, "mask_rows_differing": 0, "excused_blocks": 0, "max_abs": 0.0,
+               "rel_fro": 0.0, "dense_max_abs": 0.0, "dense_rel_fro": 0.0, "band": BAND,
+               "qblocks_per_head": nb if qblocks is None else len(qblocks)}
     for h in range(w.H):
-        q, k, v = wl.generate(w, seed=seed, device="cpu", heads=[h])
+        if gpu is not None:
+            q, k, v = gpu["q"][:, h:h + 1], gpu["k"][:, h:h + 1], gpu["v"][:, h:h + 1]
+        else:
+            q, k, v = wl.generate(w, seed=seed, device="cpu", heads=[h])
         t0 = time.perf_counter()
         if cluster_iters is not None:      # clustering, plan and forward of whole heads
             orc.clustered_attention(q, k, v, tau, lam, cluster_iters)
@@ -224,24 +259,47 @@ def time_oracle(w, tau, lam, budget_s, seed, recall=None, cluster_iters=None):
                 break
             continue
         p = orc.plan(q, k, tau, None, w.causal)
+        mask = p["mask"] if gpu is None else gpu["mask"][:, h:h + 1]
+        forced = None if gpu is None else gpu["dec"][:, h:h + 1]
         if recall is not None:
-            orc.attention_recall(q, k, v, p["mask"], recall, None, w.causal, qblocks=qblocks)
+            ref = orc.attention_recall(q, k, v, mask, recall, None, w.causal, qblocks=qblocks, forced=forced)
         else:
-            orc.fwd(q, k, v, p["mask"], lam, None, w.causal, qblocks=qblocks)
+            ref = orc.fwd(q, k, v, mask, lam, None, w.causal, qblocks=qblocks, forced=forced)
         dt = time.perf_counter() - t0
         t_total += dt
-        nb = -(-w.N // 64)
         frac = 1.0 if qblocks is None else len(qblocks) / nb
         # attention part scales with the sampled query blocks; plan is whole-head
         flops += per_head_dense * frac
         heads += 1
+        if par is not None:
+            rows, exc = compare_masks(mask, p, tau)
+            got = gpu["out"][:, h:h + 1].float().numpy()
+            ma, rel = output_errors(got, ref)
+            dq = (qblocks or list(range(nb)))
+            dq = [dq[i] for i in np.linspace(0, len(dq) - 1, min(4, len(dq))).round().astype(int)]
+            dense = orc.attention_masked(q, k, v, np.ones_like(mask), None, w.causal, qblocks=dq)
+            dma, drel = output_errors(got, dense)
+            par["heads"].append(h)
+            par["mask_rows"] += nb
+            par["mask_rows_differing"] += rows
+            par["excused_blocks"] += exc
+            par["max_abs"] = max(par["max_abs"], ma)
+            par["rel_fro"] = max(par["rel_fro"], rel)
+            par["dense_max_abs"] = max(par["dense_max_abs"], dma)
+            par["dense_rel_fro"] = max(par["dense_rel_fro"], drel)
         if t_total >= budget_s:
             break
     if cluster_iters is not None:
-        return flops / t_total / 1e12, t_total, cores, f"{heads} of {w.H} heads, clustering + plan + forward"
+        return flops / t_total / 1e12, t_total, cores, f"{heads} of {w.H} heads, clustering + plan + forward", None
     sample = (f"{heads} of {w.H} heads, full plan"
-              + ("" if qblocks is None else f", forward on {len(qblocks)} of {-(-w.N // 64)} query blocks"))
-    return flops / t_total / 1e12, t_total, cores, sample
+              + ("" if qblocks is None else f", forward on {len(qblocks)} of {nb} query blocks"))
+    if par is not None:
+        par["tolerance"] = {"max_abs": 2e-2, "rel_fro": 1e-2}
+        par["within_tolerance"] = par["max_abs"] <= 2e-2 and par["rel_fro"] <= 1e-2
+        par["note"] = ("per sampled head: mask against the oracle's plan; output against the oracle on the "
+                       "GPU's mask replaying its filter decisions (worst head); sparse-vs-dense: oracle with "
+                       "every block kept on up to 4 sampled query blocks")
+    return flops / t_total / 1e12, t_total, cores, sample, par
 
 
 # --------------------------------------------------------------------------- main arms
@@ -253,7 +311,7 @@ def run_reference(args, w, world, rank, pg):
     vals = []
     budget = max(2.0, min(args.cpu_seconds, 240.0 / max(1, args.steps + args.warmup)))
     for i in range(args.warmup + args.steps):
-        v, t, cores, sample = time_oracle(w, args.tau, lam, budget, args.seed, args.recall, args.cluster_iters)
+        v, t, cores, sample, _ = time_oracle(w, args.tau, lam, budget, args.seed, args.recall, args.cluster_iters)
         if i >= args.warmup:
             per_step.append(t)
             vals.append(v)
@@ -281,7 +339,8 @@ def config_dict(w, args, world):
             "global_batch": w.B * world, "parallelism": f"replicas{world}",
             "l2": "flushed between timed steps" if 3 * w.B * w.H * w.N * w.D * 2 < 2 * L2_BYTES
             else "inputs larger than L2 (flushed too)",
-            "centroid_weight": args.centroid_weight}
+            "centroid_weight": args.centroid_weight if args.centroid_weight is not None
+            else (w.centroid_weight if w.kind == "video" else None)}
 
 
 def check_device(sa, where):
@@ -351,10 +410,17 @@ def run_ours(args, w, world, rank, local, pg):
         run_plan()
         run_fwd()
 
-    # stats (outside timing): kept pairs, skipped P.V, algorithmic FLOPs of the forward
+    # stats (outside timing): kept pairs, skipped P.V, union tiles, algorithmic FLOPs
+    # of the forward; on the bf16 path the same launch also records the filter's
+    # decisions for the parity check of the oracle leg
     stats = torch.zeros(4, dtype=torch.int64, device=dev)
     run_plan()
-    run_fwd(stats)
+    dec = None
+    if not q8 and cl is None:
+        dec = torch.zeros((B, H, Nb, Nb), dtype=torch.uint8, device=dev)
+        sa.sparse_attn_fwd(q, k, v, plan, lam, out=out, stats=stats, recall=rec, decisions=dec)
+    else:
+        run_fwd(stats)
     torch.cuda.synchronize()
     check_device(sa, "the stats pass")
     st = [int(x) for x in stats.cpu()]
@@ -500,10 +566,22 @@ def run_ours(args, w, world, rank, local, pg):
                      "peak_source": peak_source},
         "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "cuda_graphs": not args.no_graph, "clocks": clocks,
     }
+    line["union"] = {"score_tiles": st[2], "pv_tiles": st[3], "kept_pairs": kept_pairs,
+                     "waste_pct": 100.0 * (st[2] - kept_pairs / 2) / max(kept_pairs / 2, 1),
+                     "note": "128x64 score tiles computed (one per union entry of a 128-row tile) against "
+                             "kept pairs / 2, the count with no union waste"}
     if rank == 0 and world == 1 and not args.no_cpu:
-        v_cpu, t_cpu, cores, sample = time_oracle(w, args.tau, lam, args.cpu_seconds, args.seed, rec, cl)
+        gpu = None
+        if dec is not None:
+            # the timed configuration's inputs, output (of the last timed step), mask and
+            # recorded decisions, copied to the host for the oracle leg
+            gpu = {"q": q.cpu(), "k": k.cpu(), "v": v.cpu(), "out": out.cpu(),
+                   "mask": plan.mask.cpu().numpy(), "dec": dec.cpu().numpy()}
+        v_cpu, t_cpu, cores, sample, par = time_oracle(w, args.tau, lam, args.cpu_seconds, args.seed, rec, cl,
+                                                        gpu=gpu)
         line["cpu_baseline"] = {"value": v_cpu, "unit": UNIT, "cores": cores, "kind": "oracle",
                                 "sample": sample, "seconds": t_cpu}
+        line["parity"] = par
     if rank == 0:
         print(json.dumps(line), flush=True)
 
