@@ -372,6 +372,8 @@ def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau,
     SA_ERR_DEVICE_CHECK, since O is then undefined for the affected rows."""
     lib = _lib.load()
     dev = torch.device(device)
+    if dev.type == "cuda" and dev.index is None:
+        dev = torch.device("cuda", torch.cuda.current_device())
     if q.shape != k.shape or q.shape != v.shape or q.dim() != 4:
         raise ValueError("q, k, v must share the shape [B, H, N, d]")
     for t in (q, k, v):
