@@ -118,10 +118,10 @@ sa_status launch_fwd(const sa_shape& s, const void* Q, const void* K, const void
   }
   if (!make_block_map(&mv, V, s)) return SA_ERR_CUDA;
   if (stats && cudaMemsetAsync(stats, 0, 4 * sizeof(int64_t), st) != cudaSuccess) return SA_ERR_CUDA;
-  auto kern = sa::fwd_kernel<D, kF8, kRecall>;
-  if (sa::set_smem(kern, Cfg::kSmemBytes) != SA_OK) return SA_ERR_CUDA;
   const float LOG2E = 1.4426950408889634f;
   const int lam_on = kRecall ? 1 : (std::isinf(lambda) && lambda < 0 ? 0 : 1);
+  auto kern = sa::fwd_kernel<D, kF8, kRecall>;
+  if (sa::set_smem(kern, Cfg::kSmemBytes) != SA_OK) return SA_ERR_CUDA;
   kern<<<static_cast<unsigned>(tiles), Cfg::kThreads, Cfg::kSmemBytes, st>>>(
       mq, mk, mv, mask, work, static_cast<__nv_bfloat16*>(O), s.N, Nb, Tq, tiles,
       static_cast<long long>(s.B) * s.H * Nb, scale * LOG2E,
