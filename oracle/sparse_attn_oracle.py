@@ -454,6 +454,48 @@ def quantize_blocks_e4m3(X, block: int = BLOCK):
     return codes, scales
 
 
+# ----------------------------------------------------------------------------
+# INT8 quantization of Q and K (symmetric, one scale per 64-token block)
+INT8_MAX = 127.0
+
+
+def quantize_blocks_int8(X, block: int = BLOCK):
+    """Per (batch, head, block of 64 tokens) symmetric INT8 quantization of X
+    [B, H, N, d]: amax = max |x| over the block, scale = amax / 127, and codes =
+    x * (127 / amax) rounded to the nearest integer (ties to even); the product
+    and the scale are formed in fp32 (scale 1 and codes 0 for an all-zero
+    block). |code| <= 127, so -128 never occurs. Returns (codes as fp64 values
+    [B, H, N, d], scales fp64 [B, H, Nb]); code * scale is the dequantized value."""
+    X32 = np.asarray(as_f64(X), dtype=np.float32)
+    B, H, N, d = X32.shape
+    nb = n_blocks(N, block)
+    codes = np.zeros((B, H, N, d))
+    scales = np.ones((B, H, nb))
+    for i in range(nb):
+        sl = slice(i * block, min(N, (i + 1) * block))
+        amax = np.abs(X32[:, :, sl, :]).max(axis=(2, 3))
+        pos = amax > 0
+        inv = np.where(pos, np.float32(INT8_MAX) / np.where(pos, amax, np.float32(1)), np.float32(0))
+        inv = inv.astype(np.float32)
+        y = (X32[:, :, sl, :] * inv[:, :, None, None]).astype(np.float32).astype(np.float64)
+        codes[:, :, sl, :] = np.clip(np.round(y), -INT8_MAX, INT8_MAX)   # np.round: half to even
+        scales[:, :, i] = np.where(pos, (amax / np.float32(INT8_MAX)).astype(np.float32), 1.0)
+    return codes, scales
+
+
+def fwd_int8qk(Q, K, V, mask, lam: Optional[float] = None, scale: Optional[float] = None,
+               causal: bool = False, block: int = BLOCK, qblocks=None, forced=None):
+    """Stage 2 with INT8 scores: fwd on the dequantized Q and K (codes times their
+    block scale), V as given. The mask comes from the unquantized plan."""
+    cq, sq = quantize_blocks_int8(Q, block)
+    ck, sk = quantize_blocks_int8(K, block)
+    N = cq.shape[2]
+    tok = np.minimum(np.arange(N) // block, sq.shape[2] - 1)
+    Qd = cq * sq[:, :, tok][..., None]
+    Kd = ck * sk[:, :, tok][..., None]
+    return fwd(Qd, Kd, V, mask, lam, scale, causal, block, qblocks, forced=forced)
+
+
 def fwd_fp8qk(Q, K, V, mask, lam: Optional[float] = None, scale: Optional[float] = None,
               causal: bool = False, block: int = BLOCK, qblocks=None):
     """Stage 2 with quantized scores: fwd on the dequantized Q and K (codes times

@@ -735,3 +735,57 @@ def test_forced_decisions_replay_brute_force(causal):
         np.testing.assert_array_equal(fn(Q, K, V, mask, arg, None, causal, forced=own), O)
         np.testing.assert_allclose(O, _brute_force_replay(Q, K, V, mask, own, causal), rtol=1e-10, atol=1e-12)
     assert Nb > 4
+
+
+# ---------------------------------------------------------------- INT8 quantization
+def test_quantize_blocks_int8_hand_values_and_ties():
+    """One block whose amax is 127 (scale exactly 1): the codes are x rounded to
+    the nearest integer with ties to even (0.5 -> 0, 1.5 -> 2, 2.5 -> 2, -3.5 -> -4),
+    and the amax element maps to +-127 exactly; an all-zero block gets scale 1 and
+    codes 0; a second block scaled by 2^-3 gets the same codes and scale 2^-3."""
+    row = np.array([127.0, 0.5, 1.5, 2.5, -3.5, -127.0, 0.49, 126.6])
+    X = np.zeros((1, 1, 192, 8))
+    X[0, 0, 0] = row
+    X[0, 0, 64] = row * 0.125
+    codes, scales = orc.quantize_blocks_int8(X)
+    np.testing.assert_array_equal(codes[0, 0, 0], [127, 0, 2, 2, -4, -127, 0, 127])
+    np.testing.assert_array_equal(codes[0, 0, 64], codes[0, 0, 0])
+    np.testing.assert_array_equal(scales[0, 0], [1.0, 0.125, 1.0])
+    assert np.all(codes[0, 0, 128:] == 0)
+
+
+def test_quantize_blocks_int8_error_bound_and_range():
+    """Random blocks: every code is an integer in [-127, 127], the block's amax
+    element reaches +-127, and the dequantized value is within half a step
+    (scale / 2, plus fp32 rounding) of x."""
+    r = _rng(31)
+    X = r.standard_normal((2, 3, 300, 16)) * np.exp(r.uniform(-4, 4, (2, 3, 300, 1)))
+    X = X.astype(np.float32).astype(np.float64)
+    codes, scales = orc.quantize_blocks_int8(X)
+    assert np.array_equal(codes, np.round(codes)) and np.abs(codes).max() <= 127
+    nb = orc.n_blocks(300)
+    for b in range(2):
+        for h in range(3):
+            for i in range(nb):
+                sl = slice(i * 64, min(300, i * 64 + 64))
+                c, x, sc = codes[b, h, sl], X[b, h, sl], scales[b, h, i]
+                assert np.abs(c).max() == 127
+                assert np.abs(c * sc - x).max() <= 0.5 * sc * (1 + 1e-5) + 1e-12
+
+
+def test_fwd_int8qk_is_fwd_when_q_and_k_are_representable():
+    """Inputs that are integers in [-127, 127] times a power of two, each block
+    holding a 127: quantization is exact, so fwd_int8qk equals fwd (with and
+    without lambda); on generic inputs the two differ."""
+    r = _rng(37)
+    Q = np.round(r.uniform(-127, 127, (1, 2, 192, 8))) * 2.0 ** -6
+    K = np.round(r.uniform(-127, 127, (1, 2, 192, 8))) * 2.0 ** -5
+    Q[:, :, ::64, 0] = 127 * 2.0 ** -6
+    K[:, :, ::64, 0] = 127 * 2.0 ** -5
+    V = r.standard_normal((1, 2, 192, 8))
+    mask = np.ones((1, 2, 3, 3), dtype=np.uint8)
+    for lam in (None, -2.0):
+        np.testing.assert_array_equal(orc.fwd_int8qk(Q, K, V, mask, lam), orc.fwd(Q, K, V, mask, lam))
+    Qg, Kg = r.standard_normal((1, 2, 192, 8)), r.standard_normal((1, 2, 192, 8))
+    a, b = orc.fwd_int8qk(Qg, Kg, V, mask), orc.fwd(Qg, Kg, V, mask)
+    assert 0 < np.abs(a - b).max() < 0.1
