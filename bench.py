@@ -65,8 +65,9 @@ def parse():
     ap.add_argument("--no-dense", action="store_true", help="skip the dense (full-mask) reference timing")
     ap.add_argument("--sweep", action="store_true",
                     help="one JSON line per configured (workload, tau, lambda, centroid weight); kernel timing only")
-    ap.add_argument("--qk", default="bf16", choices=["bf16", "fp8"],
-                    help="score operands: bf16 Q and K, or their FP8 E4M3 per-block codes (P.V stays bf16)")
+    ap.add_argument("--qk", default="bf16", choices=["bf16", "fp8", "int8"],
+                    help="score operands: bf16 Q and K, or their per-block FP8 E4M3 or INT8 codes "
+                         "(P.V stays bf16)")
     ap.add_argument("--recall", type=float, default=None,
                     help="P.V filter: the cumulative-energy test keeping this recall per row "
                          "(sparse_attn_fwd_recall) instead of the lambda test")
@@ -363,13 +364,14 @@ def run_ours(args, w, world, rank, local, pg):
     B, H, N, D = w.B, w.H, w.N, w.D
     Nb = -(-N // 64)
     # buffers reused by every step (resident, allocated once)
-    q8 = args.qk == "fp8"
+    q8 = args.qk in ("fp8", "int8")
+    i8 = args.qk == "int8"
     if q8 and rec is not None:
-        raise SystemExit("--recall runs on bf16 scores: drop --qk fp8")
+        raise SystemExit("--recall runs on bf16 scores: drop --qk")
     cl = args.cluster_iters
     if cl is not None and (q8 or w.causal):
         raise SystemExit("--cluster-iters needs bf16 scores and a non-causal workload")
-    plan = sa.sparse_attn_plan(q, k, args.tau, None, w.causal, with_idx=False, quantize=q8)
+    plan = sa.sparse_attn_plan(q, k, args.tau, None, w.causal, with_idx=False, quantize=args.qk if q8 else False)
     ws = torch.empty(sa.sparse_attn_plan_workspace_size(B, H, N, D), dtype=torch.uint8, device=dev)
     out = torch.empty_like(q)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -400,10 +402,11 @@ def run_ours(args, w, world, rank, local, pg):
     else:
         def run_plan():
             sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False,
-                                quantize=q8)
+                                quantize=args.qk if q8 else False)
 
         def run_fwd(stats=None):
-            sa.sparse_attn_fwd(q, k, v, plan, lam, out=out, stats=stats, qk_fp8=q8, recall=rec)
+            sa.sparse_attn_fwd(q, k, v, plan, lam, out=out, stats=stats, qk_fp8=q8 and not i8, qk_int8=i8,
+                               recall=rec)
         launches_per_step = 4
 
     def step():
@@ -444,11 +447,11 @@ def run_ours(args, w, world, rank, local, pg):
         if q8:   # the same score operands, every block kept
             full = dataclasses.replace(plan, mask=full, work=None)
         for _ in range(2):
-            sa.sparse_attn_fwd(q, k, v, full, None, out=out, causal=w.causal, qk_fp8=q8)
+            sa.sparse_attn_fwd(q, k, v, full, None, out=out, causal=w.causal, qk_fp8=q8 and not i8, qk_int8=i8)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         flush.zero_()
         e0.record(stream)
-        sa.sparse_attn_fwd(q, k, v, full, None, out=out, causal=w.causal, qk_fp8=q8)
+        sa.sparse_attn_fwd(q, k, v, full, None, out=out, causal=w.causal, qk_fp8=q8 and not i8, qk_int8=i8)
         e1.record(stream)
         torch.cuda.synchronize()
         dense_ms = e0.elapsed_time(e1)
@@ -506,8 +509,8 @@ def run_ours(args, w, world, rank, local, pg):
         # warm-up calls exactly like the timed ones, so that the caching pinned
         # allocator holds the output blocks the timed calls cycle through
         for _ in range(max(3, args.warmup)):
-            o_host = sa.sparse_attention(qh, kh, vh, args.tau, lam, None, w.causal, device=dev, qk_fp8=q8,
-                                             recall=rec)
+            o_host = sa.sparse_attention(qh, kh, vh, args.tau, lam, None, w.causal, device=dev,
+                                         qk_fp8=q8 and not i8, qk_int8=i8, recall=rec)
             torch.cuda.synchronize()
         barrier(pg, dev)
         t = []
@@ -515,8 +518,8 @@ def run_ours(args, w, world, rank, local, pg):
             flush.zero_()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            o_host = sa.sparse_attention(qh, kh, vh, args.tau, lam, None, w.causal, device=dev, qk_fp8=q8,
-                                             recall=rec)
+            o_host = sa.sparse_attention(qh, kh, vh, args.tau, lam, None, w.causal, device=dev,
+                                         qk_fp8=q8 and not i8, qk_int8=i8, recall=rec)
             b.record(stream)
             torch.cuda.synchronize()
             t.append(a.elapsed_time(b))
@@ -531,11 +534,11 @@ def run_ours(args, w, world, rank, local, pg):
     peak_t = float(pk["bf16_tflops"])
     peak_source = f"{pk_kind} bf16_tflops (burst)"
     if q8:
-        # QK^T on FP8 at twice the bf16 peak (the nominal fp8 : bf16 ratio), P.V at the
+        # QK^T on FP8 / INT8 at twice the bf16 peak (the nominal 8-bit : bf16 ratio), P.V at the
         # bf16 peak: the peak of this mix is the FLOPs over the time each part needs
         s_flops = 2.0 * D * pair_tokens
         peak_t = exec_flops / (s_flops / (2.0 * peak_t) + (exec_flops - s_flops) / peak_t)
-        peak_source = (f"{pk_kind} bf16_tflops (burst) for P.V, x2 (nominal fp8:bf16) for QK^T, "
+        peak_source = (f"{pk_kind} bf16_tflops (burst) for P.V, x2 (nominal {args.qk}:bf16) for QK^T, "
                        "combined over the executed FLOPs")
     achieved = exec_flops / (fwd_avg * 1e-3) / 1e12
     # predictor: compulsory bytes (Q and K read once; mask and counts written; with
@@ -548,7 +551,7 @@ def run_ours(args, w, world, rank, local, pg):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "fp8 e4m3 QK^T, bf16 P.V" if q8 else "bf16",
+        "vs_baseline": None, "dtype": (f"{'int8' if i8 else 'fp8 e4m3'} QK^T, bf16 P.V") if q8 else "bf16",
         "data": "synthetic (seeded cluster-centroid generator)",
         "config": config_dict(w, args, world),
         "plan_ms": plan_avg, "fwd_ms": fwd_avg, "dense_fwd_ms": dense_ms,
@@ -560,7 +563,8 @@ def run_ours(args, w, world, rank, local, pg):
                       "bytes": pred_bytes, "peak_source": f"{pk_kind} hbm_gbs"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": achieved / peak_t, "traffic": None if cl is not None else measured_traffic(w, args.tau, lam, args.qk, rec),
-                     "kernel": f"fwd_kernel<{D}, fp8 scores> (sparse_attn_fwd_q8)" if q8
+                     "kernel": (f"fwd_kernel<{D}, int8 scores> (sparse_attn_fwd_i8)" if i8
+                                else f"fwd_kernel<{D}, fp8 scores> (sparse_attn_fwd_q8)") if q8
                      else (f"fwd_kernel<{D}, recall filter> (sparse_attn_fwd_recall)" if rec is not None
                            else f"fwd_kernel<{D}> (sparse_attn_fwd)"),
                      "peak_source": peak_source},
@@ -590,8 +594,8 @@ def sweep(args):
     """Every configured point of every workload (one GPU, kernel timing only)."""
     base = dict(vars(args))
     for name, w in wl.WORKLOADS.items():
-        if args.qk == "fp8" and w.D != 128:
-            continue                                  # FP8 scores are for d = 128
+        if args.qk != "bf16" and w.D != 128:
+            continue                                  # 8-bit scores are for d = 128
         cws = w.centroid_weights or (None,)
         for tau in w.taus:
             for lam in w.lams:

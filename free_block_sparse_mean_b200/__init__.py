@@ -76,8 +76,10 @@ class Plan:
                                 of each row (rest of the row undefined), or None
     work  int32 [2*num_tiles]   query-block pairs in execution order for sparse_attn_fwd
                                 (global ids (b*H+h)*Nb+i, second -1 if absent), or None
-    q8, k8          uint8 [B, H, N, d]  FP8 E4M3 codes of q and k (quantize=True), else None
-    qscale, kscale  float32 [B, H, Nb]  their per-block scales (quantize=True), else None
+    q8, k8          uint8 [B, H, N, d]  8-bit codes of q and k (quantize="fp8": FP8 E4M3;
+                                        quantize="int8": int8 values), else None
+    qscale, kscale  float32 [B, H, Nb]  their per-block scales, else None
+    qfmt            "fp8", "int8" or None: the format of q8 and k8
     """
     mask: torch.Tensor
     count: torch.Tensor
@@ -85,6 +87,7 @@ class Plan:
     work: Optional[torch.Tensor]
     tau: Union[float, torch.Tensor]   # one threshold, or one per (batch, head)
     causal: bool
+    qfmt: Optional[str] = None
     q8: Optional[torch.Tensor] = None
     k8: Optional[torch.Tensor] = None
     qscale: Optional[torch.Tensor] = None
@@ -99,21 +102,23 @@ def sparse_attn_num_tiles(B: int, H: int, N: int, d: int) -> int:
     return int(_lib.load().sparse_attn_num_tiles(SaShape(B, H, N, d, BLOCK)))
 
 
-def sparse_attn_host_workspace_size(B: int, H: int, N: int, d: int, chunks: int = 4, qk_fp8: bool = False) -> int:
-    return int(_lib.load().sparse_attn_host_workspace_size(SaShape(B, H, N, d, BLOCK), int(chunks),
-                                                           _lib.SA_HOST_FP8_SCORES if qk_fp8 else 0))
+def sparse_attn_host_workspace_size(B: int, H: int, N: int, d: int, chunks: int = 4, qk_fp8: bool = False,
+                                    qk_int8: bool = False) -> int:
+    flags = (_lib.SA_HOST_FP8_SCORES if qk_fp8 else 0) | (_lib.SA_HOST_INT8_SCORES if qk_int8 else 0)
+    return int(_lib.load().sparse_attn_host_workspace_size(SaShape(B, H, N, d, BLOCK), int(chunks), flags))
 
 
 def sparse_attn_plan(q: torch.Tensor, k: torch.Tensor, tau, scale: Optional[float] = None,
                      causal: bool = False, *, with_idx: bool = False, with_work: bool = True,
                      out: Optional[Plan] = None, workspace: Optional[torch.Tensor] = None,
-                     quantize: bool = False) -> Plan:
+                     quantize=False) -> Plan:
     """Stage 1: cumulative-energy block mask from mean-pooled q and k.
 
     tau is one recall threshold for every head (a float), or one per head: a float32
     CUDA tensor of shape [B, H] or [H] on q's device (sparse_attn_plan_heads).
-    quantize=True (one tau, d = 128) also writes FP8 E4M3 copies of q and k with
-    per-block scales (sparse_attn_plan_q8) for sparse_attn_fwd(..., qk_fp8=True).
+    quantize="fp8" (or True; one tau, d = 128) also writes FP8 E4M3 copies of q and k
+    with per-block scales (sparse_attn_plan_q8) for sparse_attn_fwd(..., qk_fp8=True);
+    quantize="int8" writes INT8 copies (sparse_attn_plan_i8) for qk_int8=True.
     with_idx=True also writes the ascending kept lists (an int32 [B, H, Nb, Nb]
     tensor: 4 bytes per block pair, 331 MB on the 118,800-token video shape); the
     forward does not read them, so they are off by default."""
@@ -135,6 +140,10 @@ def sparse_attn_plan(q: torch.Tensor, k: torch.Tensor, tau, scale: Optional[floa
             tau=tau if isinstance(tau, torch.Tensor) else float(tau), causal=bool(causal))
     else:
         out.tau, out.causal = (tau if isinstance(tau, torch.Tensor) else float(tau)), bool(causal)
+    if quantize is True:
+        quantize = "fp8"
+    if quantize not in (False, None, "fp8", "int8"):
+        raise ValueError('quantize must be False, True, "fp8" or "int8"')
     if quantize and out.q8 is None:
         out.q8 = torch.empty((B, H, N, d), dtype=torch.uint8, device=dev)
         out.k8 = torch.empty((B, H, N, d), dtype=torch.uint8, device=dev)
@@ -145,12 +154,14 @@ def sparse_attn_plan(q: torch.Tensor, k: torch.Tensor, tau, scale: Optional[floa
         workspace = torch.empty((max(ws_bytes, 256),), dtype=torch.uint8, device=dev)
     if quantize:
         if isinstance(tau, torch.Tensor):
-            raise ValueError("quantize=True takes one tau for every head")
-        st = lib.sparse_attn_plan_q8(_ptr(q), _ptr(k), s, float(tau), float(scale), int(bool(causal)),
-                                     _ptr(out.mask), _ptr(out.count), _ptr(out.idx), _ptr(out.work),
-                                     _ptr(out.q8), _ptr(out.k8), _ptr(out.qscale), _ptr(out.kscale),
-                                     _ptr(workspace), ws_bytes, _stream(dev))
-        _call("sparse_attn_plan_q8", st)
+            raise ValueError("quantize takes one tau for every head")
+        fn = lib.sparse_attn_plan_i8 if quantize == "int8" else lib.sparse_attn_plan_q8
+        st = fn(_ptr(q), _ptr(k), s, float(tau), float(scale), int(bool(causal)),
+                _ptr(out.mask), _ptr(out.count), _ptr(out.idx), _ptr(out.work),
+                _ptr(out.q8), _ptr(out.k8), _ptr(out.qscale), _ptr(out.kscale),
+                _ptr(workspace), ws_bytes, _stream(dev))
+        out.qfmt = quantize
+        _call("sparse_attn_plan_i8" if quantize == "int8" else "sparse_attn_plan_q8", st)
         return out
     if isinstance(tau, torch.Tensor):
         if tau.dtype != torch.float32 or tau.device != dev:
@@ -176,13 +187,14 @@ def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan, lam
                     scale: Optional[float] = None, causal: Optional[bool] = None, *,
                     out: Optional[torch.Tensor] = None, stats: Optional[torch.Tensor] = None,
                     qk_fp8: bool = False, recall: Optional[float] = None,
-                    decisions: Optional[torch.Tensor] = None) -> torch.Tensor:
+                    decisions: Optional[torch.Tensor] = None, qk_int8: bool = False) -> torch.Tensor:
     """Stage 2: attention over the kept blocks with the lambda P.V filter.
 
     `plan` is a Plan or a uint8 mask [B, H, Nb, Nb]. lam=None turns the filter off.
     `stats`, if given, is an int64 CUDA tensor of 4 entries (see the C header).
     qk_fp8=True takes the scores on the plan's FP8 copies of q and k
-    (sparse_attn_fwd_q8; the plan must come from sparse_attn_plan(quantize=True)).
+    (sparse_attn_fwd_q8; the plan must come from sparse_attn_plan(quantize="fp8")),
+    qk_int8=True on its INT8 copies (sparse_attn_fwd_i8; quantize="int8").
     recall=rho (in (0, 1]) replaces the lambda test by the cumulative-energy test
     of sparse_attn_fwd_recall: every row keeps at least the fraction rho of the
     softmax energy of the blocks it visits; lam must then be None.
@@ -213,7 +225,7 @@ def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan, lam
     if stats is not None and (stats.dtype != torch.int64 or stats.numel() < 4 or stats.device != q.device):
         raise ValueError("stats must be an int64 tensor of >= 4 entries on q's device")
     if decisions is not None:
-        if qk_fp8:
+        if qk_fp8 or qk_int8:
             raise ValueError("decisions are recorded by the bf16-score forward")
         if decisions.dtype != torch.uint8 or tuple(decisions.shape) != (B, H, Nb, Nb) \
                 or not decisions.is_contiguous() or decisions.device != q.device:
@@ -227,7 +239,7 @@ def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan, lam
         _call("sparse_attn_fwd_decisions", st)
         return out
     if recall is not None:
-        if lam is not None or qk_fp8:
+        if lam is not None or qk_fp8 or qk_int8:
             raise ValueError("recall replaces the lambda filter and takes bf16 scores: "
                              "pass lam=None and qk_fp8=False with it")
         st = lib.sparse_attn_fwd_recall(_ptr(q), _ptr(k), _ptr(v), _shape(q), _ptr(mask), _ptr(work),
@@ -235,13 +247,17 @@ def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan, lam
                                         _stream(q.device))
         _call("sparse_attn_fwd_recall", st)
         return out
-    if qk_fp8:
-        if not isinstance(plan, Plan) or plan.q8 is None:
-            raise ValueError("qk_fp8=True needs a plan made with quantize=True")
-        st = lib.sparse_attn_fwd_q8(_ptr(plan.q8), _ptr(plan.k8), _ptr(plan.qscale), _ptr(plan.kscale), _ptr(v),
+    if qk_fp8 or qk_int8:
+        want = "int8" if qk_int8 else "fp8"
+        if qk_fp8 and qk_int8:
+            raise ValueError("qk_fp8 and qk_int8 exclude each other")
+        if not isinstance(plan, Plan) or plan.q8 is None or plan.qfmt != want:
+            raise ValueError(f'qk_{want}=True needs a plan made with quantize="{want}"')
+        fn = lib.sparse_attn_fwd_i8 if qk_int8 else lib.sparse_attn_fwd_q8
+        st = fn(_ptr(plan.q8), _ptr(plan.k8), _ptr(plan.qscale), _ptr(plan.kscale), _ptr(v),
                                     _shape(q), _ptr(mask), _ptr(work), lam_f, float(scale), int(causal),
                                     _ptr(out), _ptr(stats), _stream(q.device))
-        _call("sparse_attn_fwd_q8", st)
+        _call("sparse_attn_fwd_i8" if qk_int8 else "sparse_attn_fwd_q8", st)
         return out
     st = lib.sparse_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _shape(q), _ptr(mask), _ptr(work), lam_f,
                              float(scale), int(causal), _ptr(out), _ptr(stats), _stream(q.device))
@@ -350,7 +366,7 @@ def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau,
                      lam: Optional[float] = None, scale: Optional[float] = None, causal: bool = False,
                      device="cuda", out: Optional[torch.Tensor] = None, chunks: Optional[int] = None,
                      qk_fp8: bool = False, recall: Optional[float] = None,
-                     workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+                     workspace: Optional[torch.Tensor] = None, qk_int8: bool = False) -> torch.Tensor:
     """End to end from host tensors (the C call sparse_attn_host): copy q, k, v to
     the GPU, plan + forward, copy O back.
 
@@ -363,7 +379,7 @@ def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau,
     device-to-host copy run on three streams, so the copies of one group overlap
     the work of the others in both directions of the link. tau may be one value or
     a per-head float32 tensor ([B, H] or [H]) on `device`; qk_fp8=True takes the scores on FP8 copies of q and k (see
-    sparse_attn_plan's quantize); recall selects the cumulative-energy P.V filter
+    sparse_attn_plan's quantize), qk_int8=True on INT8 copies; recall selects the cumulative-energy P.V filter
     instead of lambda (see sparse_attn_fwd). The device workspace is allocated
     here unless given (sparse_attn_host_workspace_size bytes).
 
@@ -379,7 +395,7 @@ def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau,
     for t in (q, k, v):
         if t.device.type != "cpu" or t.dtype != torch.bfloat16 or not t.is_contiguous():
             raise ValueError("q, k, v must be contiguous host bf16 tensors")
-    if recall is not None and (lam is not None or qk_fp8):
+    if recall is not None and (lam is not None or qk_fp8 or qk_int8):
         raise ValueError("recall replaces the lambda filter and takes bf16 scores")
     B, H, N, d = q.shape
     if out is None:
@@ -389,7 +405,9 @@ def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau,
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     nch = max(1, min(B * H, chunks if chunks is not None else 4))
-    flags = _lib.SA_HOST_FP8_SCORES if qk_fp8 else 0
+    if qk_fp8 and qk_int8:
+        raise ValueError("qk_fp8 and qk_int8 exclude each other")
+    flags = (_lib.SA_HOST_FP8_SCORES if qk_fp8 else 0) | (_lib.SA_HOST_INT8_SCORES if qk_int8 else 0)
     s = _shape(q)
     ws_bytes = int(lib.sparse_attn_host_workspace_size(s, nch, flags))
     if ws_bytes == 0:

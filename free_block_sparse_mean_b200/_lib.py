@@ -14,6 +14,7 @@ SA_ERR_DEVICE_CHECK = 5
 SA_FILTER_LAMBDA = 0
 SA_FILTER_RECALL = 1
 SA_HOST_FP8_SCORES = 1
+SA_HOST_INT8_SCORES = 2
 STATUS_NAMES = {
     0: "SA_OK",
     1: "SA_ERR_INVALID_ARG",
@@ -35,6 +36,8 @@ EXPORTS = (
     "sparse_attn_plan_noalloc",
     "sparse_attn_plan_q8",
     "sparse_attn_fwd_q8",
+    "sparse_attn_plan_i8",
+    "sparse_attn_fwd_i8",
     "sparse_attn_fwd_recall",
     "sparse_attn_fwd_decisions",
     "sparse_attn_host_workspace_size",
@@ -97,6 +100,10 @@ def load(path: str = LIB_PATH):
     lib.sparse_attn_plan_q8.restype = i32
     lib.sparse_attn_fwd_q8.argtypes = [vp, vp, vp, vp, vp, SaShape, vp, vp, f32, f32, i32, vp, vp, vp]
     lib.sparse_attn_fwd_q8.restype = i32
+    lib.sparse_attn_plan_i8.argtypes = lib.sparse_attn_plan_q8.argtypes
+    lib.sparse_attn_plan_i8.restype = i32
+    lib.sparse_attn_fwd_i8.argtypes = lib.sparse_attn_fwd_q8.argtypes
+    lib.sparse_attn_fwd_i8.restype = i32
     lib.sparse_attn_fwd_recall.argtypes = [vp, vp, vp, SaShape, vp, vp, f32, f32, i32, vp, vp, vp]
     lib.sparse_attn_fwd_recall.restype = i32
     lib.sparse_attn_fwd_decisions.argtypes = [vp, vp, vp, SaShape, vp, vp, i32, f32, f32, i32, vp, vp, vp, vp]

@@ -61,12 +61,15 @@
 
 namespace sa {
 
-// kF8: Q and K arrive as FP8 E4M3 codes with one scale per 64-token block
-// (d = 128 only); S = Q K^T runs as tcgen05.mma kind::f8f6f4 and the two block
-// scales join the softmax scale. V, P and O are as in the bf16 kernel.
-template <int D, bool kF8 = false>
+// kQ: the score operands. kScoreBF16: bf16 Q and K. kScoreE4M3 / kScoreI8: Q and
+// K arrive as 8-bit codes (FP8 E4M3 or signed INT8) with one scale per 64-token
+// block (d = 128 only); S = Q K^T runs as tcgen05.mma kind::f8f6f4 (fp32
+// accumulate) or kind::i8 (s32 accumulate), and the two block scales join the
+// softmax scale. V, P and O are as in the bf16 kernel.
+template <int D, int kQ = kScoreBF16>
 struct FwdCfg {
-  static_assert(!kF8 || D == 128, "the FP8-score kernel is for d = 128");
+  static constexpr bool kF8 = kQ != kScoreBF16;        // 8-bit score codes
+  static_assert(!kF8 || D == 128, "the 8-bit-score kernel is for d = 128");
   static constexpr int kRows = 128;                    // query rows per tile
   static constexpr int kThreads = 192;                 // 2 role warps + 4 softmax warps
   static constexpr int kChunks = D / 64;               // 128-byte (64 x bf16) column chunks of V
@@ -92,7 +95,8 @@ struct FwdCfg {
   // TMEM columns: S, two P buffers (bf16 pairs), the O accumulator
   static constexpr uint32_t kColS = 0, kColP0 = 64, kColP1 = 96, kColO = 128;
   static constexpr uint32_t kTmemCols = 256;
-  static constexpr uint32_t kIdescS = kF8 ? idesc_e4m3_f32(128, 64) : idesc_bf16_f32(128, 64, false);
+  static constexpr uint32_t kIdescS = kQ == kScoreI8 ? idesc_s8_s32(128, 64)
+                                      : (kF8 ? idesc_e4m3_f32(128, 64) : idesc_bf16_f32(128, 64, false));
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
 };
 
@@ -134,7 +138,7 @@ __device__ __forceinline__ float softmax_exp64(const float (&s)[64], float scale
 // lambda vote's.
 // decisions (optional, [B,H,Nb,Nb] bytes): for every (query block, kept key
 // block) pair the tile visits, 1 if the filter skipped its P.V, else 0.
-template <int D, bool kF8, bool kRecall = false>
+template <int D, int kQ, bool kRecall = false>
 __global__ void __launch_bounds__(192, 2)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const uint8_t* __restrict__ mask,
@@ -143,7 +147,9 @@ __global__ void __launch_bounds__(192, 2)
                float budget, int causal, unsigned long long* __restrict__ stats,
                const float* __restrict__ qscale, const float* __restrict__ kscale,
                uint8_t* __restrict__ decisions) {
-  using C = FwdCfg<D, kF8>;
+  using C = FwdCfg<D, kQ>;
+  constexpr bool kF8 = C::kF8;                   // 8-bit score codes (E4M3 or INT8)
+  constexpr bool kI8 = kQ == kScoreI8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base + C::oQ;
@@ -347,7 +353,9 @@ __global__ void __launch_bounds__(192, 2)
           const uint32_t off = (kk & 3) * 32;  // 16 bf16 or 32 e4m3 = 32 bytes inside the swizzle atom
           const uint64_t ad = sdesc_sw128(sQa + (kk >> 2) * C::kQChunkBytes + off, 16, 1024);
           const uint64_t bd = sdesc_sw128(sKa + s * C::kKBytes + (kk >> 2) * C::kKVChunkBytes + off, 16, 1024);
-          if constexpr (kF8)
+          if constexpr (kI8)
+            tc_mma_ss_i8(dS, ad, bd, C::kIdescS, kk > 0 ? 1u : 0u);
+          else if constexpr (kF8)
             tc_mma_ss_f8(dS, ad, bd, C::kIdescS, kk > 0 ? 1u : 0u);
           else
             tc_mma_ss(dS, ad, bd, C::kIdescS, kk > 0 ? 1u : 0u);
@@ -419,6 +427,13 @@ __global__ void __launch_bounds__(192, 2)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free);         // S may now be overwritten by S(k+1)
+      if constexpr (kI8) {
+        // s32 scores (|S| < 2^22) to the exact floats 12582912 + S: the integer
+        // plus the bits of 1.5 * 2^23 (ordered like S); the offset is taken out
+        // of the row max below and folded into the exponentials' bias
+#pragma unroll
+        for (int c = 0; c < 64; ++c) s[c] = __int_as_float(__float_as_int(s[c]) + 0x4B400000);
+      }
       uint32_t pk[32];                            // P as packed bf16 pairs
       float rmax = -INFINITY, psum = 0.f;
       if (!warp_none) {
@@ -436,8 +451,9 @@ __global__ void __launch_bounds__(192, 2)
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) mx[u] = fmaxf(mx[u], s[56 + u]);
-        rmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
-               sc;                                // -inf stays -inf (sc > 0)
+        float mxv = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+        if constexpr (kI8) mxv -= 12582912.f;    // exact: back to the integer score
+        rmax = mxv * sc;                          // -inf stays -inf (sc > 0)
       }
       bool wpass = true;
       if (!kRecall && lam_on) {
@@ -461,7 +477,8 @@ __global__ void __launch_bounds__(192, 2)
 #pragma unroll
         for (int c = 0; c < 32; ++c) pk[c] = 0u;
       } else {
-        psum = softmax_exp64(s, sc, mref, pk);
+        // INT8: s holds 12582912 + S, so the bias also takes 12582912 * sc
+        psum = softmax_exp64(s, sc, kI8 ? mref + 12582912.f * sc : mref, pk);
       }
       m_true = m_new;
       l = l * alpha + psum;

@@ -52,10 +52,12 @@ static __device__ __forceinline__ uint32_t mix32(uint32_t x) {
 // thread loads 16-byte vectors (8 bf16) of a row; D/8 threads cover a row, so a
 // warp reads whole rows contiguously. Partial sums meet in shared memory.
 // HBM-bound: it is the one full pass over Q and K on the predictor side.
-// With Q8 (and K8, qs, ks) given, the same pass also quantizes the block to FP8
-// E4M3 for the quantized-score forward: scale = amax / 448 over the block, codes =
-// x * (448 / amax) rounded to nearest even and saturated (scale 1, codes 0 for an
-// all-zero block), [B,H,N,d] bytes and [B,H,Nb] fp32 scales.
+// With Q8 (and K8, qs, ks) given, the same pass also quantizes the block for the
+// quantized-score forward, [B,H,N,d] bytes and [B,H,Nb] fp32 scales (scale 1,
+// codes 0 for an all-zero block). qfmt = kScoreE4M3: FP8 E4M3, scale = amax / 448,
+// codes = x * (448 / amax) rounded to nearest even and saturated; qfmt =
+// kScoreI8: signed INT8, scale = amax / 127, codes = x * (127 / amax) rounded to
+// the nearest integer, ties to even (|code| <= 127).
 template <int D>
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ Q,
                                                    const __nv_bfloat16* __restrict__ K,
@@ -63,7 +65,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
                                                    int N, int Nb, uint8_t* __restrict__ Q8 = nullptr,
                                                    uint8_t* __restrict__ K8 = nullptr,
                                                    float* __restrict__ qs = nullptr,
-                                                   float* __restrict__ ks = nullptr) {
+                                                   float* __restrict__ ks = nullptr, int qfmt = kScoreE4M3) {
   constexpr int LPR = D / 8;          // threads per row
   constexpr int RPP = 256 / LPR;      // rows per pass
   __shared__ float part[RPP][D];
@@ -126,8 +128,9 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   }
   if (q8) {
     amax = fmax3(fmax3(wmax[0], wmax[1], wmax[2]), fmax3(wmax[3], wmax[4], wmax[5]), fmaxf(wmax[6], wmax[7]));
-    const float inv = amax > 0.f ? 448.f / amax : 0.f;
-    if (threadIdx.x == 0) (blockIdx.y == 0 ? qs : ks)[g] = amax > 0.f ? amax / 448.f : 1.f;
+    const float qmax = qfmt == kScoreI8 ? 127.f : 448.f;
+    const float inv = amax > 0.f ? qmax / amax : 0.f;
+    if (threadIdx.x == 0) (blockIdx.y == 0 ? qs : ks)[g] = amax > 0.f ? amax / qmax : 1.f;
     uint8_t* dst8 = q8 + (bh * N + static_cast<long long>(i) * kBlock) * D;
 #pragma unroll
     for (int p = 0; p < kPasses; ++p) {
@@ -138,9 +141,22 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const float2 f0 = __bfloat1622float2(h[2 * e]), f1 = __bfloat1622float2(h[2 * e + 1]);
-          const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(f0.x * inv, f0.y * inv), __NV_SATFINITE, __NV_E4M3);
-          const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(f1.x * inv, f1.y * inv), __NV_SATFINITE, __NV_E4M3);
-          w[e] = lo | (hi << 16);
+          if (qfmt == kScoreI8) {
+            const float y[4] = {f0.x * inv, f0.y * inv, f1.x * inv, f1.y * inv};
+            uint32_t b = 0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int c = max(-127, min(127, __float2int_rn(y[q])));   // nearest, ties to even
+              b |= (static_cast<uint32_t>(c) & 0xFFu) << (8 * q);
+            }
+            w[e] = b;
+          } else {
+            const uint32_t lo =
+                __nv_cvt_float2_to_fp8x2(make_float2(f0.x * inv, f0.y * inv), __NV_SATFINITE, __NV_E4M3);
+            const uint32_t hi =
+                __nv_cvt_float2_to_fp8x2(make_float2(f1.x * inv, f1.y * inv), __NV_SATFINITE, __NV_E4M3);
+            w[e] = lo | (hi << 16);
+          }
         }
         *reinterpret_cast<uint2*>(dst8 + static_cast<long long>(r) * D + c8) = make_uint2(w[0], w[1]);
       }

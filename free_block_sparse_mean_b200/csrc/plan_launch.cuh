@@ -22,8 +22,8 @@ inline sa_status set_smem(F* kernel, int bytes) {
   return SA_OK;
 }
 
-// Stage 1 on the stream: pool Q and K (and, with Q8 given, write their FP8 codes
-// and per-block scales), the pooled scores and the cumulative-energy selection
+// Stage 1 on the stream: pool Q and K (and, with Q8 given, write their 8-bit
+// codes in format qfmt and per-block scales), the pooled scores and the cumulative-energy selection
 // (mask, count, optional idx), then, with `work` given, the tile pairs and their
 // order. `scratch` holds plan_workspace(B*H, Nb, D).total bytes, 256-byte aligned.
 // tau_bh, when given, is a device array of one threshold per (b, h) that replaces tau.
@@ -31,7 +31,7 @@ template <int D>
 sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau, const float* tau_bh,
                       float scale, int causal, uint8_t* mask, int32_t* count, int32_t* idx, int32_t* work,
                       void* scratch, cudaStream_t st, uint8_t* Q8 = nullptr, uint8_t* K8 = nullptr,
-                      float* qscale = nullptr, float* kscale = nullptr) {
+                      float* qscale = nullptr, float* kscale = nullptr, int qfmt = kScoreE4M3) {
   const int Nb = static_cast<int>((static_cast<int64_t>(s.N) + 63) / 64);
   const long long BH = static_cast<long long>(s.B) * s.H;
   const PlanWorkspace L = plan_workspace(BH, Nb, D);
@@ -42,7 +42,7 @@ sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau
   uint32_t* bits = reinterpret_cast<uint32_t*>(wsb + L.bits);
   pool_kernel<D><<<dim3(static_cast<unsigned>(BH * Nb), 2), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Qp, Kp, s.N, Nb, Q8, K8, qscale,
-      kscale);
+      kscale, qfmt);
   if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
 
   // R query blocks per CTA: 4 for short heads so that the grid still fills the GPU.

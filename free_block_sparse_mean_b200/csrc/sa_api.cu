@@ -100,18 +100,18 @@ bool make_map8(CUtensorMap* map, const void* ptr, const sa_shape& s) {
 }
 
 // kRecall: the P.V filter is the recall test with budget = 1 - recall (lambda unused).
-template <int D, bool kF8 = false, bool kRecall = false>
+template <int D, int kQ = sa::kScoreBF16, bool kRecall = false>
 sa_status launch_fwd(const sa_shape& s, const void* Q, const void* K, const void* V, const uint8_t* mask,
                      const int32_t* work, float lambda, float scale, int causal, void* O, int64_t* stats,
                      cudaStream_t st, const float* qscale = nullptr, const float* kscale = nullptr,
                      float budget = 0.f, uint8_t* decisions = nullptr) {
-  using Cfg = sa::FwdCfg<D, kF8>;
+  using Cfg = sa::FwdCfg<D, kQ>;
   const int Nb = static_cast<int>(num_blocks(s));
   const int Tq = (Nb + 1) / 2;
   const long long tiles = static_cast<long long>(s.B) * s.H * Tq;
   if (tiles > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
   CUtensorMap mq, mk, mv;
-  if (kF8) {
+  if (Cfg::kF8) {
     if (!make_map8(&mq, Q, s) || !make_map8(&mk, K, s)) return SA_ERR_CUDA;
   } else {
     if (!make_map(&mq, Q, s, 64) || !make_block_map(&mk, K, s)) return SA_ERR_CUDA;
@@ -120,7 +120,7 @@ sa_status launch_fwd(const sa_shape& s, const void* Q, const void* K, const void
   if (stats && cudaMemsetAsync(stats, 0, 4 * sizeof(int64_t), st) != cudaSuccess) return SA_ERR_CUDA;
   const float LOG2E = 1.4426950408889634f;
   const int lam_on = kRecall ? 1 : (std::isinf(lambda) && lambda < 0 ? 0 : 1);
-  auto kern = sa::fwd_kernel<D, kF8, kRecall>;
+  auto kern = sa::fwd_kernel<D, kQ, kRecall>;
   if (sa::set_smem(kern, Cfg::kSmemBytes) != SA_OK) return SA_ERR_CUDA;
   kern<<<static_cast<unsigned>(tiles), Cfg::kThreads, Cfg::kSmemBytes, st>>>(
       mq, mk, mv, mask, work, static_cast<__nv_bfloat16*>(O), s.N, Nb, Tq, tiles,
@@ -280,9 +280,9 @@ sa_status sparse_attn_fwd_recall(const void* Q, const void* K, const void* V, sa
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float budget = 1.f - recall;
   if (s.d == 64)
-    return launch_fwd<64, false, true>(s, Q, K, V, mask, work, 0.f, scale, causal != 0, O, stats, st, nullptr,
+    return launch_fwd<64, sa::kScoreBF16, true>(s, Q, K, V, mask, work, 0.f, scale, causal != 0, O, stats, st, nullptr,
                                        nullptr, budget);
-  return launch_fwd<128, false, true>(s, Q, K, V, mask, work, 0.f, scale, causal != 0, O, stats, st, nullptr,
+  return launch_fwd<128, sa::kScoreBF16, true>(s, Q, K, V, mask, work, 0.f, scale, causal != 0, O, stats, st, nullptr,
                                       nullptr, budget);
 }
 
@@ -308,9 +308,9 @@ sa_status sparse_attn_fwd_decisions(const void* Q, const void* K, const void* V,
   if (filter == SA_FILTER_RECALL) {
     const float budget = 1.f - value;
     if (s.d == 64)
-      return launch_fwd<64, false, true>(s, Q, K, V, mask, work, 0.f, scale, c, O, stats, st, nullptr, nullptr,
+      return launch_fwd<64, sa::kScoreBF16, true>(s, Q, K, V, mask, work, 0.f, scale, c, O, stats, st, nullptr, nullptr,
                                          budget, decisions);
-    return launch_fwd<128, false, true>(s, Q, K, V, mask, work, 0.f, scale, c, O, stats, st, nullptr, nullptr,
+    return launch_fwd<128, sa::kScoreBF16, true>(s, Q, K, V, mask, work, 0.f, scale, c, O, stats, st, nullptr, nullptr,
                                         budget, decisions);
   }
   if (s.d == 64)
@@ -355,7 +355,8 @@ HostWorkspace host_workspace(const sa_shape& s, int chunks, bool fp8) {
 size_t sparse_attn_host_workspace_size(sa_shape s, int32_t chunks, int32_t flags) {
   if (check_shape(s) != SA_OK || chunks < 1) return 0;
   const long long BH = static_cast<long long>(s.B) * s.H;
-  return host_workspace(s, static_cast<int>(std::min<long long>(chunks, BH)), (flags & SA_HOST_FP8_SCORES) != 0)
+  return host_workspace(s, static_cast<int>(std::min<long long>(chunks, BH)),
+                        (flags & (SA_HOST_FP8_SCORES | SA_HOST_INT8_SCORES)) != 0)
       .total;
 }
 
@@ -367,22 +368,24 @@ sa_status sparse_attn_host(const void* Qh, const void* Kh, const void* Vh, sa_sh
   if (!Qh || !Kh || !Vh || !Oh) return SA_ERR_INVALID_ARG;
   const sa_status sh = check_shape(s);
   if (sh != SA_OK) return sh;
-  const bool fp8 = (flags & SA_HOST_FP8_SCORES) != 0;
-  if ((flags & ~SA_HOST_FP8_SCORES) != 0 || chunks < 1) return SA_ERR_INVALID_ARG;
+  const bool fp8 = (flags & SA_HOST_FP8_SCORES) != 0, i8 = (flags & SA_HOST_INT8_SCORES) != 0;
+  if ((flags & ~(SA_HOST_FP8_SCORES | SA_HOST_INT8_SCORES)) != 0 || (fp8 && i8) || chunks < 1)
+    return SA_ERR_INVALID_ARG;
+  const bool q8 = fp8 || i8;                       // 8-bit score codes
   if (tau_heads ? (reinterpret_cast<uintptr_t>(tau_heads) & 3u) != 0 : !(tau > 0.f && tau <= 1.f))
     return SA_ERR_INVALID_ARG;
   if (!(std::isfinite(scale) && scale > 0.f)) return SA_ERR_INVALID_ARG;
   if (filter == SA_FILTER_LAMBDA) {
     if (std::isnan(value) || (std::isinf(value) && value > 0)) return SA_ERR_INVALID_ARG;
   } else if (filter == SA_FILTER_RECALL) {
-    if (!(value > 0.f && value <= 1.f) || fp8) return SA_ERR_INVALID_ARG;
+    if (!(value > 0.f && value <= 1.f) || q8) return SA_ERR_INVALID_ARG;
   } else {
     return SA_ERR_INVALID_ARG;
   }
-  if (fp8 && s.d != 128) return SA_ERR_UNSUPPORTED;
+  if (q8 && s.d != 128) return SA_ERR_UNSUPPORTED;
   const long long BH = static_cast<long long>(s.B) * s.H;
   const int nch = static_cast<int>(std::min<long long>(chunks, BH));
-  const HostWorkspace L = host_workspace(s, nch, fp8);
+  const HostWorkspace L = host_workspace(s, nch, q8);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < L.total)
     return SA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -432,24 +435,27 @@ sa_status sparse_attn_host(const void* Qh, const void* Kh, const void* Vh, sa_sh
     void* pws = ws + L.plan;
     const float* tg = tau_heads ? tau_heads + lo : nullptr;   // this group's per-head thresholds
     sa_status r;
-    if (fp8) {
-      uint8_t* q8 = reinterpret_cast<uint8_t*>(ws + L.q8) + off / 2;
-      uint8_t* k8 = reinterpret_cast<uint8_t*>(ws + L.k8) + off / 2;
+    if (q8) {
+      uint8_t* c8q = reinterpret_cast<uint8_t*>(ws + L.q8) + off / 2;
+      uint8_t* c8k = reinterpret_cast<uint8_t*>(ws + L.k8) + off / 2;
       float* qs = reinterpret_cast<float*>(ws + L.qs) + static_cast<size_t>(lo) * Nb;
       float* ks = reinterpret_cast<float*>(ws + L.ks) + static_cast<size_t>(lo) * Nb;
-      r = sa::launch_plan<128>(g, q, k, tau, tg, scale, causal != 0, mask, count, nullptr, work, pws, st, q8, k8,
-                               qs, ks);
+      r = sa::launch_plan<128>(g, q, k, tau, tg, scale, causal != 0, mask, count, nullptr, work, pws, st, c8q, c8k,
+                               qs, ks, i8 ? sa::kScoreI8 : sa::kScoreE4M3);
       if (r == SA_OK)
-        r = launch_fwd<128, true>(g, q8, k8, v, mask, work, value, scale, causal != 0, o, nullptr, st, qs, ks);
+        r = i8 ? launch_fwd<128, sa::kScoreI8>(g, c8q, c8k, v, mask, work, value, scale, causal != 0, o, nullptr, st,
+                                               qs, ks)
+               : launch_fwd<128, sa::kScoreE4M3>(g, c8q, c8k, v, mask, work, value, scale, causal != 0, o, nullptr,
+                                                 st, qs, ks);
     } else {
       r = s.d == 64 ? sa::launch_plan<64>(g, q, k, tau, tg, scale, causal != 0, mask, count, nullptr, work, pws, st)
                     : sa::launch_plan<128>(g, q, k, tau, tg, scale, causal != 0, mask, count, nullptr, work, pws,
                                            st);
       if (r == SA_OK) {
         if (filter == SA_FILTER_RECALL)
-          r = s.d == 64 ? launch_fwd<64, false, true>(g, q, k, v, mask, work, 0.f, scale, causal != 0, o, nullptr,
+          r = s.d == 64 ? launch_fwd<64, sa::kScoreBF16, true>(g, q, k, v, mask, work, 0.f, scale, causal != 0, o, nullptr,
                                                       st, nullptr, nullptr, 1.f - value)
-                        : launch_fwd<128, false, true>(g, q, k, v, mask, work, 0.f, scale, causal != 0, o, nullptr,
+                        : launch_fwd<128, sa::kScoreBF16, true>(g, q, k, v, mask, work, 0.f, scale, causal != 0, o, nullptr,
                                                        st, nullptr, nullptr, 1.f - value);
         else
           r = s.d == 64 ? launch_fwd<64>(g, q, k, v, mask, work, value, scale, causal != 0, o, nullptr, st)
@@ -567,7 +573,45 @@ sa_status sparse_attn_fwd_q8(const void* Q8, const void* K8, const float* qscale
       (reinterpret_cast<uintptr_t>(qscale) & 3u) != 0 || (reinterpret_cast<uintptr_t>(kscale) & 3u) != 0)
     return SA_ERR_INVALID_ARG;
   if (stats && (reinterpret_cast<uintptr_t>(stats) & 7u) != 0) return SA_ERR_INVALID_ARG;
-  return launch_fwd<128, true>(s, Q8, K8, V, mask, work, lambda, scale, causal != 0, O, stats,
+  return launch_fwd<128, sa::kScoreE4M3>(s, Q8, K8, V, mask, work, lambda, scale, causal != 0, O, stats,
+                               static_cast<cudaStream_t>(stream), qscale, kscale);
+}
+
+sa_status sparse_attn_plan_i8(const void* Q, const void* K, sa_shape s, float tau, float scale, int32_t causal,
+                              uint8_t* mask, int32_t* count, int32_t* idx, int32_t* work, void* Q8, void* K8,
+                              float* qscale, float* kscale, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  if (!Q || !K || !mask || !count || !Q8 || !K8 || !qscale || !kscale) return SA_ERR_INVALID_ARG;
+  const sa_status sh = check_shape(s);
+  if (sh != SA_OK) return sh;
+  if (s.d != 128) return SA_ERR_UNSUPPORTED;
+  if (!(tau > 0.f && tau <= 1.f)) return SA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return SA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(Q8) || !aligned16(K8) ||
+      (reinterpret_cast<uintptr_t>(qscale) & 3u) != 0 || (reinterpret_cast<uintptr_t>(kscale) & 3u) != 0)
+    return SA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < sparse_attn_plan_workspace_size(s))
+    return SA_ERR_WORKSPACE;
+  return sa::launch_plan<128>(s, Q, K, tau, nullptr, scale, causal != 0, mask, count, idx, work, workspace,
+                          static_cast<cudaStream_t>(stream), static_cast<uint8_t*>(Q8), static_cast<uint8_t*>(K8),
+                          qscale, kscale, sa::kScoreI8);
+}
+
+sa_status sparse_attn_fwd_i8(const void* Q8, const void* K8, const float* qscale, const float* kscale,
+                             const void* V, sa_shape s, const uint8_t* mask, const int32_t* work, float lambda,
+                             float scale, int32_t causal, void* O, int64_t* stats, void* stream) {
+  if (!Q8 || !K8 || !qscale || !kscale || !V || !mask || !O) return SA_ERR_INVALID_ARG;
+  const sa_status sh = check_shape(s);
+  if (sh != SA_OK) return sh;
+  if (s.d != 128) return SA_ERR_UNSUPPORTED;
+  if (std::isnan(lambda) || (std::isinf(lambda) && lambda > 0)) return SA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return SA_ERR_INVALID_ARG;
+  if (!aligned16(Q8) || !aligned16(K8) || !aligned16(V) || !aligned16(O) ||
+      (reinterpret_cast<uintptr_t>(qscale) & 3u) != 0 || (reinterpret_cast<uintptr_t>(kscale) & 3u) != 0)
+    return SA_ERR_INVALID_ARG;
+  if (stats && (reinterpret_cast<uintptr_t>(stats) & 7u) != 0) return SA_ERR_INVALID_ARG;
+  return launch_fwd<128, sa::kScoreI8>(s, Q8, K8, V, mask, work, lambda, scale, causal != 0, O, stats,
                                static_cast<cudaStream_t>(stream), qscale, kscale);
 }
 

@@ -205,6 +205,18 @@ __device__ __forceinline__ void tc_mma_ss_f8(uint32_t d_tmem, uint64_t adesc, ui
       : "memory");
 }
 
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::i8 (both operands signed
+// 8-bit, s32 accumulate; K = 32 per instruction).
+__device__ __forceinline__ void tc_mma_ss_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16: A (M x K bf16, one row per
 // lane, two consecutive K elements per 32-bit column) is read from tensor memory.
 __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
@@ -258,6 +270,20 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
          | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }
+
+// Instruction descriptor for kind::i8 with signed 8-bit A and B, s32 D, both
+// K-major (D format 2 = s32, A and B format 1 = signed).
+__host__ __device__ constexpr uint32_t idesc_s8_s32(int M, int N) {
+  return (2u << 4)                                  // D format: s32
+         | (1u << 7)                                // A format: signed 8-bit
+         | (1u << 10)                               // B format: signed 8-bit
+         | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
+}
+
+// Score operand types of the forward kernel: bf16 Q and K, or 8-bit codes with
+// one scale per 64-token block (FP8 E4M3 or signed INT8).
+enum ScoreType : int { kScoreBF16 = 0, kScoreE4M3 = 1, kScoreI8 = 2 };
 
 // 32 consecutive 32-bit TMEM columns of this warp's 32 lanes (lane i -> row).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {

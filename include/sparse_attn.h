@@ -214,10 +214,12 @@ sa_status sparse_attn_fwd_decisions(const void* Q, const void* K, const void* V,
  *   tau_heads   NULL, or a DEVICE array of B*H thresholds (4-byte aligned) that
  *               replaces tau, as sparse_attn_plan_heads (tau is then ignored)
  *   filter, value  the P.V filter, as sparse_attn_fwd_decisions (SA_FILTER_RECALL
- *               cannot be combined with SA_HOST_FP8_SCORES)
+ *               takes bf16 scores: it cannot be combined with either score flag)
  *   scale, causal  as sparse_attn_fwd
- *   flags       0, or SA_HOST_FP8_SCORES: scores on FP8 codes of Q and K
- *               (sparse_attn_plan_q8 + sparse_attn_fwd_q8; d must be 128)
+ *   flags       0, SA_HOST_FP8_SCORES: scores on FP8 codes of Q and K
+ *               (sparse_attn_plan_q8 + sparse_attn_fwd_q8), or SA_HOST_INT8_SCORES:
+ *               on INT8 codes (sparse_attn_plan_i8 + sparse_attn_fwd_i8); d must be
+ *               128 for either, and the two flags cannot be combined
  *   Oh          out, host bf16 [B,H,N,d]; complete once `stream` is
  *   workspace   device memory of at least sparse_attn_host_workspace_size(s,
  *               chunks, flags) bytes, 256-byte aligned: the device copies of Q, K,
@@ -234,6 +236,7 @@ sa_status sparse_attn_fwd_decisions(const void* Q, const void* K, const void* V,
  * sparse_attn_fwd). Errors: those of sparse_attn_plan and sparse_attn_fwd, and
  * SA_ERR_WORKSPACE for a missing, misaligned or short workspace. */
 #define SA_HOST_FP8_SCORES 1
+#define SA_HOST_INT8_SCORES 2
 size_t sparse_attn_host_workspace_size(sa_shape s, int32_t chunks, int32_t flags);
 sa_status sparse_attn_host(const void* Qh, const void* Kh, const void* Vh, sa_shape s, float tau,
                            const float* tau_heads, int32_t filter, float value, float scale,
@@ -264,6 +267,25 @@ sa_status sparse_attn_plan_q8(const void* Q, const void* K, sa_shape s, float ta
  * V) and O are those of sparse_attn_fwd. d must be 128. Other arguments and
  * errors: as sparse_attn_fwd. */
 sa_status sparse_attn_fwd_q8(const void* Q8, const void* K8, const float* qscale, const float* kscale,
+                             const void* V, sa_shape s, const uint8_t* mask, const int32_t* work,
+                             float lambda, float scale, int32_t causal, void* O, int64_t* stats,
+                             void* stream);
+
+/* INT8 scores: the same two calls as sparse_attn_plan_q8 / sparse_attn_fwd_q8 with
+ * signed INT8 codes instead of FP8 E4M3 (this library's second quantization
+ * scheme; the pages give none). For each (b, h, 64-token block) of Q and of K:
+ * amax = max |x| over the block, scale = amax / 127 and code = x * (127 / amax)
+ * rounded to the nearest integer, ties to even (|code| <= 127, so -128 never
+ * occurs), both in fp32; an all-zero block gets scale 1 and codes 0. The forward
+ * takes S = (Q8 K8^T) * qscale[query block] * kscale[key block] by tcgen05.mma
+ * kind::i8 (exact s32 accumulation). INT8 keeps 7 significant bits per operand
+ * where E4M3 keeps 4, so the scores are about 16 times closer to the bf16 ones.
+ * Q8, K8 hold int8_t values; other arguments, outputs and errors: as the q8 calls. */
+sa_status sparse_attn_plan_i8(const void* Q, const void* K, sa_shape s, float tau, float scale,
+                              int32_t causal, uint8_t* mask, int32_t* count, int32_t* idx,
+                              int32_t* work, void* Q8, void* K8, float* qscale, float* kscale,
+                              void* workspace, size_t workspace_bytes, void* stream);
+sa_status sparse_attn_fwd_i8(const void* Q8, const void* K8, const float* qscale, const float* kscale,
                              const void* V, sa_shape s, const uint8_t* mask, const int32_t* work,
                              float lambda, float scale, int32_t causal, void* O, int64_t* stats,
                              void* stream);

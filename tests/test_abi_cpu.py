@@ -221,3 +221,28 @@ def test_host_call_rejects_bad_arguments(lib):
     assert call(flags=1, s=SaShape(1, 2, 128, 64, 64)) == 2           # FP8 scores: d = 128
     assert call(ws=None) == 3 and call(nbytes=need - 1) == 3
     assert call(ws=ctypes.c_void_p(0x100010)) == 3                   # workspace 256-byte aligned
+
+
+def test_int8_entry_points_reject_bad_arguments(lib):
+    s, s64 = SaShape(1, 2, 128, 128, 64), SaShape(1, 2, 128, 64, 64)
+    ws = ctypes.c_void_p(0x100000)
+
+    def plan(s=s, Q8=FAKE, qs=FAKE, tau=0.9):
+        return lib.sparse_attn_plan_i8(FAKE, FAKE, s, tau, 0.1, 0, FAKE, FAKE, None, None, Q8, FAKE, qs, FAKE,
+                                       ws, 1 << 30, None)
+
+    def fwd(s=s, K8=FAKE, ks=FAKE, lam=-math.inf):
+        return lib.sparse_attn_fwd_i8(FAKE, K8, FAKE, ks, FAKE, s, FAKE, None, lam, 0.1, 0, FAKE, None, None)
+
+    assert plan(Q8=None) == 1 and plan(qs=None) == 1
+    assert plan(qs=ctypes.c_void_p(0x10002)) == 1
+    assert plan(Q8=FAKE_ODD) == 1 and plan(tau=1.5) == 1
+    assert plan(s=s64) == 2
+    assert fwd(K8=None) == 1 and fwd(ks=None) == 1 and fwd(lam=float("nan")) == 1
+    assert fwd(s=s64) == 2
+    # the host call: the two score flags exclude each other, and INT8 needs d = 128
+    need = lib.sparse_attn_host_workspace_size(s, 2, 2)
+    assert need == lib.sparse_attn_host_workspace_size(s, 2, 1)
+    call = lambda flags, shape=s: lib.sparse_attn_host(FAKE, FAKE, FAKE, shape, 0.9, None, 0, -12.0, 0.1, 0,
+                                                       flags, FAKE, ws, need, 2, None, None, None)
+    assert call(3) == 1 and call(2, s64) == 2
