@@ -3,9 +3,13 @@ the oracle.
 
 The codes and scales are integer decisions taken in fp32 on both sides, so they
 must match bit for bit. The forward on the codes must match the oracle's forward
-on the dequantized Q and K within the output tolerance of the bf16 path, and,
-since INT8 keeps 7 significant bits per operand, its output must stay within the
-output tolerance of the bf16-score result as well."""
+on the dequantized Q and K within the output tolerance of the bf16 path.
+
+Against the bf16-score result the quantization itself moves the output: on these
+workloads the logits reach ~25 nats, and half an INT8 step per operand adds up to
+~0.02 nats per logit, about 2% of each probability. The tests hold INT8 to a
+relative Frobenius distance of 5e-2 from the bf16-score oracle, and to at least 3
+times less than FP8 E4M3 (whose 4 significant bits give ~11% on the same inputs)."""
 import numpy as np
 import pytest
 import torch
@@ -70,10 +74,13 @@ def test_int8_score_forward_matches_the_oracle(case, lam):
     ref = orc.fwd_int8qk(q.cpu(), k.cpu(), v.cpu(), mask, lam, None, causal)
     assert_output_close(to_np(o8), ref, f"int8 scores {case} lam={lam}")
     assert int(st8[0]) == int(st[0])                         # the same kept pairs
-    # 7 significant bits per operand: the output stays within the bf16 path's tolerance
+    # the quantization's own effect, against the bf16-score oracle and against E4M3
     ref16 = orc.fwd(q.cpu(), k.cpu(), v.cpu(), mask, lam, None, causal)
-    max_abs, rel = assert_output_close(to_np(o8), ref16, f"int8 scores vs bf16-score oracle, {case} lam={lam}")
-    print(f"{case} lam={lam}: int8-score output vs the bf16-score oracle max_abs={max_abs:.3e} rel_fro={rel:.3e}")
+    max_abs, rel = output_errors(to_np(o8), ref16)
+    _, rel8 = output_errors(orc.fwd_fp8qk(q.cpu(), k.cpu(), v.cpu(), mask, lam, None, causal), ref16)
+    print(f"{case} lam={lam}: int8-score output vs the bf16-score oracle max_abs={max_abs:.3e} rel_fro={rel:.3e}"
+          f" (fp8 scores: rel_fro={rel8:.3e})")
+    assert rel <= 5e-2 and rel * 3 <= rel8
 
 
 @pytest.mark.slow
@@ -81,8 +88,8 @@ def test_int8_score_forward_matches_the_oracle(case, lam):
 def test_int8_scores_full_size(name, tau, lam):
     """Full size: codes and scales of a sampled head byte for byte, and 16 sampled
     query blocks (first and ragged last included) against the oracle on the
-    dequantized Q and K and against the bf16-score oracle, both at the output
-    tolerance."""
+    dequantized Q and K at the output tolerance; against the bf16-score oracle
+    within 5e-2 and 3 times closer than FP8 scores."""
     w = wl.WORKLOADS[name]
     q, k, v = wl.generate(w, seed=0, device=_dev())
     p = sa.sparse_attn_plan(q, k, tau, None, w.causal, quantize="int8")
@@ -103,8 +110,11 @@ def test_int8_scores_full_size(name, tau, lam):
     ref = orc.fwd_int8qk(qh, kh, vh, mask[:, h:h + 1], lam, None, w.causal, qblocks=qbs)
     assert_output_close(got, ref, f"int8 {name} head {h} query blocks {qbs}")
     ref16 = orc.fwd(qh, kh, vh, mask[:, h:h + 1], lam, None, w.causal, qblocks=qbs)
-    ma, rel = assert_output_close(got, ref16, f"int8 vs bf16-score oracle {name} head {h}")
-    print(f"{name}: int8-score output vs the bf16-score oracle max_abs={ma:.3e} rel_fro={rel:.3e}")
+    ma, rel = output_errors(got, ref16)
+    _, rel8 = output_errors(orc.fwd_fp8qk(qh, kh, vh, mask[:, h:h + 1], lam, None, w.causal, qblocks=qbs), ref16)
+    print(f"{name}: int8-score output vs the bf16-score oracle max_abs={ma:.3e} rel_fro={rel:.3e}"
+          f" (fp8 scores: rel_fro={rel8:.3e})")
+    assert rel <= 5e-2 and rel * 3 <= rel8
 
 
 def test_int8_needs_an_int8_plan_and_d128():
