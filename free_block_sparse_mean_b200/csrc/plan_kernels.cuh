@@ -294,17 +294,11 @@ static __device__ __forceinline__ void select_row_sorted64(const float* row, int
 // bisection, or 8-way with kEightWay), then the mask row, the ascending kept list,
 // count[bh*Nb + i], the MinHash sort key of the kept set (*sig_out) and its bitset
 // (brow, ceil(Nb/32) words) for the pairing. sig_out and brow may be null.
-// kSelectCand: capacity of a warp's candidate buffer (the bisection path): once
-// the search range [lo, hi) holds at most this many values, they are copied to
-// `cand` and the remaining steps sum over them only, on top of the known sum of
-// the values at or above hi (S(>= hi), taken by the pass that set hi).
-constexpr int kSelectCand = 512;
-
 template <bool kEightWay>
 static __device__ __forceinline__ void select_row(float* row, int Nb, int i, long long bh, float tau, int lane,
                                                   uint8_t* __restrict__ mask, int* __restrict__ count,
                                                   int* __restrict__ idx, unsigned long long* sig_out,
-                                                  uint32_t* brow, float* cand) {
+                                                  uint32_t* brow) {
   const unsigned FULL = 0xffffffffu;
   const float LOG2E = 1.4426950408889634f;
   float m = -INFINITY;
@@ -334,8 +328,6 @@ static __device__ __forceinline__ void select_row(float* row, int Nb, int i, lon
   } else {
     const float T = tau * tot;
     uint32_t lo = 0u, hi = kmax + 1u;   // S(lo) >= T > S(hi)
-    float s_hi = 0.f;                   // bisection: S(>= hi) (nothing lies at or above kmax + 1)
-    int ncand = -1;                     // bisection: -1 = search the whole row, else cand[0..ncand)
     while (hi - lo > 1u) {
       if constexpr (kEightWay) {
         // 7 probes split [lo, hi) into 8 parts; the last one is above lo once hi - lo >= 2
@@ -369,61 +361,13 @@ static __device__ __forceinline__ void select_row(float* row, int Nb, int i, lon
       } else {
         const uint32_t mid = lo + ((hi - lo) >> 1);
         float s = 0.f;
-        if (ncand < 0) {
-          // full row; also count the values left in either half of the range
-          int cnt = 0;                               // (in [mid, hi)) << 16 | (in [lo, mid))
-          for (int j = lane; j < Nb; j += 32) {
-            const float e = row[j];
-            const uint32_t u = __float_as_uint(e);
-            s += (u >= mid) ? e : 0.f;
-            cnt += (u >= mid && u < hi) ? (1 << 16) : ((u >= lo && u < mid) ? 1 : 0);
-          }
-#pragma unroll
-          for (int o = 16; o; o >>= 1) {
-            s += __shfl_xor_sync(FULL, s, o);
-            cnt += __shfl_xor_sync(FULL, cnt, o);
-          }
-          int left;
-          if (s >= T) {
-            lo = mid;
-            left = cnt >> 16;
-          } else {
-            hi = mid;
-            s_hi = s;
-            left = cnt & 0xffff;
-          }
-          if (cand != nullptr && left <= kSelectCand && hi - lo > 1u) {
-            // copy the values in [lo, hi) to the candidate buffer, in row order
-            int nc = 0;
-            for (int jb = 0; jb < Nb; jb += 32) {
-              const int j = jb + lane;
-              const float e = (j < Nb) ? row[j] : 0.f;
-              const uint32_t u = __float_as_uint(e);
-              const bool in = j < Nb && u >= lo && u < hi;
-              const unsigned b = __ballot_sync(FULL, in);
-              if (in) cand[nc + __popc(b & ((1u << lane) - 1u))] = e;
-              nc += __popc(b);
-            }
-            __syncwarp();
-            ncand = nc;
-          }
-        } else {
-          // the candidates only: S(>= mid) = S(>= hi) + the candidates in [mid, hi)
-          for (int j = lane; j < ncand; j += 32) {
-            const float e = cand[j];
-            const uint32_t u = __float_as_uint(e);
-            s += (u >= mid && u < hi) ? e : 0.f;
-          }
-#pragma unroll
-          for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(FULL, s, o);
-          s += s_hi;
-          if (s >= T) {
-            lo = mid;
-          } else {
-            hi = mid;
-            s_hi = s;
-          }
+        for (int j = lane; j < Nb; j += 32) {
+          const float e = row[j];
+          s += (__float_as_uint(e) >= mid) ? e : 0.f;
         }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(FULL, s, o);
+        if (s >= T) lo = mid; else hi = mid;
       }
     }
     K = lo;
@@ -525,7 +469,6 @@ __global__ void __launch_bounds__(NT) score_select_kernel(const float* __restric
   static_assert(R % 4 == 0 && R <= 16 && NT % 32 == 0, "R rows per CTA, NT threads");
   constexpr bool kSmall = R == 4;   // staged phase 1, 8-way search in phase 2
   static_assert(!kSmall || NT == 128, "the staged phase 1 uses 128 threads");
-  static_assert(kSmall || NT == 256, "score_select_smem_bytes sizes 8 candidate buffers");
   constexpr int kCols = 2 * NT;  // key blocks per pass of phase 1
   constexpr int QS = R + 4;  // padded row stride of the transposed query tile
   extern __shared__ __align__(16) float sm[];
@@ -655,8 +598,6 @@ __global__ void __launch_bounds__(NT) score_select_kernel(const float* __restric
     }
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // the bisection path's candidate buffer of this warp (after the score rows)
-  float* cand = kSmall ? nullptr : L + R * ldL + warp * kSelectCand;
   for (int r = warp; r < R; r += NT / 32) {
     const int i = i0 + r;
     if (i >= Nb) break;
@@ -665,7 +606,7 @@ __global__ void __launch_bounds__(NT) score_select_kernel(const float* __restric
     if (kSmall && Nb <= 64)
       select_row_sorted64(L + r * ldL, Nb, i, bh, tau, lane, mask, count, idx, srow, brow);
     else
-      select_row<kSmall>(L + r * ldL, Nb, i, bh, tau, lane, mask, count, idx, srow, brow, cand);
+      select_row<kSmall>(L + r * ldL, Nb, i, bh, tau, lane, mask, count, idx, srow, brow);
   }
 }
 
@@ -674,10 +615,7 @@ template <int D, int R>
 inline int score_select_smem_bytes(int Nb) {
   const int ldL = (Nb + 3) & ~3;
   int floats = D * (R + 4) + R * ldL;
-  if (R == 4)
-    floats += 64 * (D + 1) + 2 * R * 64;
-  else
-    floats += (256 / 32) * kSelectCand;   // a candidate buffer per warp (256 threads)
+  if (R == 4) floats += 64 * (D + 1) + 2 * R * 64;
   return floats * static_cast<int>(sizeof(float));
 }
 
