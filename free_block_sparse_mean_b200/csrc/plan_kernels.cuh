@@ -294,6 +294,28 @@ static __device__ __forceinline__ void select_row_sorted64(const float* row, int
 // bisection, or 8-way with kEightWay), then the mask row, the ascending kept list,
 // count[bh*Nb + i], the MinHash sort key of the kept set (*sig_out) and its bitset
 // (brow, ceil(Nb/32) words) for the pairing. sig_out and brow may be null.
+// One lane's part of sum{e_j : bits(e_j) >= key} over a row of non-negative values:
+// the lane's elements j = lane + 32 t go to four partial sums by t mod 4 (so four
+// independent shared-memory loads and additions are in flight instead of one
+// chain), combined as (p0 + p1) + (p2 + p3). Every such sum of a row is formed in
+// this same order, with +0 for the elements below key, so sums over nested sets
+// are ordered like the sets (rounded addition of non-negative terms is monotone).
+static __device__ __forceinline__ float lane_sum_ge(const float* row, int Nb, int lane, uint32_t key) {
+  float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+  int j = lane;
+  for (; j + 96 < Nb; j += 128) {
+    const float e0 = row[j], e1 = row[j + 32], e2 = row[j + 64], e3 = row[j + 96];
+    p0 += (__float_as_uint(e0) >= key) ? e0 : 0.f;
+    p1 += (__float_as_uint(e1) >= key) ? e1 : 0.f;
+    p2 += (__float_as_uint(e2) >= key) ? e2 : 0.f;
+    p3 += (__float_as_uint(e3) >= key) ? e3 : 0.f;
+  }
+  if (j < Nb) p0 += (__float_as_uint(row[j]) >= key) ? row[j] : 0.f;
+  if (j + 32 < Nb) p1 += (__float_as_uint(row[j + 32]) >= key) ? row[j + 32] : 0.f;
+  if (j + 64 < Nb) p2 += (__float_as_uint(row[j + 64]) >= key) ? row[j + 64] : 0.f;
+  return (p0 + p1) + (p2 + p3);
+}
+
 template <bool kEightWay>
 static __device__ __forceinline__ void select_row(float* row, int Nb, int i, long long bh, float tau, int lane,
                                                   uint8_t* __restrict__ mask, int* __restrict__ count,
@@ -302,17 +324,53 @@ static __device__ __forceinline__ void select_row(float* row, int Nb, int i, lon
   const unsigned FULL = 0xffffffffu;
   const float LOG2E = 1.4426950408889634f;
   float m = -INFINITY;
-  for (int j = lane; j < Nb; j += 32) m = fmaxf(m, row[j]);
+  {
+    float m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+    int j = lane;
+    for (; j + 96 < Nb; j += 128) {
+      m = fmaxf(m, row[j]);
+      m1 = fmaxf(m1, row[j + 32]);
+      m2 = fmaxf(m2, row[j + 64]);
+      m3 = fmaxf(m3, row[j + 96]);
+    }
+    for (; j < Nb; j += 32) m = fmaxf(m, row[j]);
+    m = fmaxf(fmaxf(m, m1), fmaxf(m2, m3));
+  }
 #pragma unroll
   for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
   // e_j in place; the row max maps to exactly 1.
   float tot = 0.f;
   uint32_t kmax = 0;
-  for (int j = lane; j < Nb; j += 32) {
-    const float e = ex2((row[j] - m) * LOG2E);
-    row[j] = e;
-    tot += e;
-    kmax = max(kmax, __float_as_uint(e));
+  if constexpr (kEightWay) {
+    for (int j = lane; j < Nb; j += 32) {
+      const float e = ex2((row[j] - m) * LOG2E);
+      row[j] = e;
+      tot += e;
+      kmax = max(kmax, __float_as_uint(e));
+    }
+  } else {
+    uint32_t k1 = 0, k2 = 0, k3 = 0;
+    int j = lane;
+    for (; j + 96 < Nb; j += 128) {
+      const float e0 = ex2((row[j] - m) * LOG2E), e1 = ex2((row[j + 32] - m) * LOG2E);
+      const float e2 = ex2((row[j + 64] - m) * LOG2E), e3 = ex2((row[j + 96] - m) * LOG2E);
+      row[j] = e0;
+      row[j + 32] = e1;
+      row[j + 64] = e2;
+      row[j + 96] = e3;
+      kmax = max(kmax, __float_as_uint(e0));
+      k1 = max(k1, __float_as_uint(e1));
+      k2 = max(k2, __float_as_uint(e2));
+      k3 = max(k3, __float_as_uint(e3));
+    }
+    for (; j < Nb; j += 32) {
+      const float e = ex2((row[j] - m) * LOG2E);
+      row[j] = e;
+      kmax = max(kmax, __float_as_uint(e));
+    }
+    kmax = max(max(kmax, k1), max(k2, k3));
+    __syncwarp();
+    tot = lane_sum_ge(row, Nb, lane, 0u);          // the total, formed like every probe sum
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) {
@@ -360,11 +418,7 @@ static __device__ __forceinline__ void select_row(float* row, int Nb, int i, lon
         hi = nhi;
       } else {
         const uint32_t mid = lo + ((hi - lo) >> 1);
-        float s = 0.f;
-        for (int j = lane; j < Nb; j += 32) {
-          const float e = row[j];
-          s += (__float_as_uint(e) >= mid) ? e : 0.f;
-        }
+        float s = lane_sum_ge(row, Nb, lane, mid);
 #pragma unroll
         for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(FULL, s, o);
         if (s >= T) lo = mid; else hi = mid;
@@ -373,10 +427,24 @@ static __device__ __forceinline__ void select_row(float* row, int Nb, int i, lon
     K = lo;
     float sgt = 0.f;
     int nties = 0;
-    for (int j = lane; j < Nb; j += 32) {
-      const uint32_t kj = __float_as_uint(row[j]);
-      sgt += (kj > K) ? row[j] : 0.f;
-      nties += (kj == K);
+    if constexpr (kEightWay) {
+      for (int j = lane; j < Nb; j += 32) {
+        const uint32_t kj = __float_as_uint(row[j]);
+        sgt += (kj > K) ? row[j] : 0.f;
+        nties += (kj == K);
+      }
+    } else {
+      sgt = lane_sum_ge(row, Nb, lane, K + 1u);     // the values above e*, formed like the probes
+      int n1 = 0, n2 = 0, n3 = 0;
+      int j = lane;
+      for (; j + 96 < Nb; j += 128) {
+        nties += __float_as_uint(row[j]) == K;
+        n1 += __float_as_uint(row[j + 32]) == K;
+        n2 += __float_as_uint(row[j + 64]) == K;
+        n3 += __float_as_uint(row[j + 96]) == K;
+      }
+      for (; j < Nb; j += 32) nties += __float_as_uint(row[j]) == K;
+      nties += (n1 + n2) + n3;
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) {
