@@ -18,8 +18,29 @@ namespace sa {
 
 // Byte offsets of the plan workspace: pooled Q and K (fp32 [B,H,Nb,d]), then per
 // query block a 64-bit MinHash sort key and the kept set as a bitset of W words.
+// Shared memory of the pairing kernel for Nb blocks per head without the bitsets:
+// the sort keys of the blocks and of the tiles (powers of two), the pairs, the
+// order, the matching state and the scan scratch.
+__host__ __device__ inline int pair_base_smem_bytes(int Nb) {
+  int p = 2, p2 = 2;
+  while (p < Nb) p <<= 1;
+  const int Tq = (Nb + 1) / 2;
+  while (p2 < Tq) p2 <<= 1;
+  return (p + p2) * 8 + (2 * Tq + 4 * Nb + 34) * 4;
+}
+// The pairing keeps the kept-set bitsets, regrouped by sorted position, in shared
+// memory when they fit beside the rest (up to about 1,180 blocks per head), else in
+// global memory (the plan workspace's bitsT region).
+__host__ __device__ inline bool pair_bits_in_smem(int Nb) {
+  return pair_base_smem_bytes(Nb) + Nb * ((Nb + 31) / 32) * 4 <= 227 * 1024;
+}
+
+// Byte offsets of the plan workspace: pooled Q and K (fp32 [B,H,Nb,d]), then per
+// query block a 64-bit MinHash sort key and the kept set as a bitset of W words;
+// when the pairing's copy of the bitsets does not fit in shared memory, that copy,
+// word-major by sorted position ([B,H][W][Nb]).
 struct PlanWorkspace {
-  size_t qp, kp, sig, bits, total;
+  size_t qp, kp, sig, bits, bitsT, total;
   int W;
 };
 inline PlanWorkspace plan_workspace(long long BH, int Nb, int D) {
@@ -27,11 +48,13 @@ inline PlanWorkspace plan_workspace(long long BH, int Nb, int D) {
   PlanWorkspace w;
   w.W = (Nb + 31) / 32;
   const size_t pooled = al(static_cast<size_t>(BH) * Nb * D * sizeof(float));
+  const size_t bitset = al(static_cast<size_t>(BH) * Nb * w.W * sizeof(uint32_t));
   w.qp = 0;
   w.kp = pooled;
   w.sig = 2 * pooled;
   w.bits = w.sig + al(static_cast<size_t>(BH) * Nb * sizeof(unsigned long long));
-  w.total = w.bits + al(static_cast<size_t>(BH) * Nb * w.W * sizeof(uint32_t));
+  w.bitsT = w.bits + bitset;
+  w.total = w.bitsT + (pair_bits_in_smem(Nb) ? 0 : bitset);
   return w;
 }
 
@@ -700,11 +723,10 @@ inline int score_select_smem_bytes(int Nb) {
 // kPairRounds rounds, or a round without a new pair, the rest are paired in
 // order. Every block of a head is examined at once, so a round costs one pass.
 // The pairs of a head are then ordered by decreasing union size (longest first).
-// Above kPairMatchMaxNb blocks per head the bitsets no longer fit in shared
+// When the bitsets do not fit in shared
 // memory and consecutive blocks of the sorted order are paired directly.
 // Output: work[2*r], work[2*r+1] = global query-block ids (bh*Nb + i) of the r-th
 // tile (second -1 if the head has an odd block count).
-constexpr int kPairMatchMaxNb = 1024;
 constexpr int kPairWindow = 16;
 constexpr int kPairRounds = 6;
 // Heads per interleaved group of the tile order: as many as have their K and V
@@ -779,10 +801,14 @@ static __device__ int block_exclusive_scan(int v, int* sbuf, int* total) {
 // memory (pair_order_smem_bytes minus the keys). BH heads in all.
 static __device__ void pair_and_order(unsigned long long* keys, const uint32_t* bits_rows,
                                       const int* __restrict__ count, int Nb, int Tq, int G, long long bh,
-                                      long long BH, int* __restrict__ work, unsigned char* psm) {
+                                      long long BH, int* __restrict__ work, unsigned char* psm,
+                                      uint32_t* bits_by_pos) {
   const int P = 1 << (32 - __clz(max(Nb, 2) - 1));   // next power of two >= Nb
   const int P2 = 1 << (32 - __clz(max(Tq, 2) - 1));
-  const bool match = Nb <= kPairMatchMaxNb;
+  // bitsets by sorted position: in shared memory when they fit, else in the global
+  // bits_by_pos region ([W][Nb] of this head)
+  const bool in_smem = pair_bits_in_smem(Nb);
+  const bool match = in_smem || bits_by_pos != nullptr;
   const int W = (Nb + 31) / 32;                       // bitset words per row
   unsigned long long* keys2 = reinterpret_cast<unsigned long long*>(psm);      // [P2]
   int* pa = reinterpret_cast<int*>(keys2 + P2);                                  // [Tq]
@@ -792,7 +818,8 @@ static __device__ void pair_and_order(unsigned long long* keys, const uint32_t* 
   int* best = alive + Nb;                                                        // [Nb] pick of a position
   int* partner = best + Nb;                                                      // [Nb] -1 while unpaired
   int* sbuf = partner + Nb;                                                      // [34] scan scratch
-  uint32_t* bitsT = reinterpret_cast<uint32_t*>(sbuf + 34);                     // [W][Nb] by position (match only)
+  uint32_t* bitsT = in_smem ? reinterpret_cast<uint32_t*>(sbuf + 34)  // [W][Nb] by position
+                           : bits_by_pos;
   const int* cnt = count + bh * Nb;
 
   // 1. sort the MinHash keys
@@ -815,15 +842,15 @@ static __device__ void pair_and_order(unsigned long long* keys, const uint32_t* 
   //    sums without bitsets)
   if (match) {
     // kept-set bitsets, word-major by sorted position: neighbouring candidates are
-    // neighbouring addresses
+    // neighbouring addresses (shared memory, or this head's global region; the
+    // barrier makes the CTA's global writes visible to its own later reads)
     for (int x = threadIdx.x; x < Nb * W; x += blockDim.x) {
       const int p = x / W, w = x - p * W;
-      bitsT[w * Nb + p] = bits_rows[static_cast<long long>(order[p]) * W + w];
+      bitsT[static_cast<long long>(w) * Nb + p] = bits_rows[static_cast<long long>(order[p]) * W + w];
     }
     __syncthreads();
     // one warp per alive position, one lane per candidate (the 16 alive positions
-    // on each side); the launch gives at least Nb threads, so t < Nb covers the
-    // alive list in the mutual-pick step
+    // on each side)
     int na = Nb;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
     for (int round = 0; round < kPairRounds; ++round) {
@@ -837,8 +864,10 @@ static __device__ void pair_and_order(unsigned long long* keys, const uint32_t* 
         int sc = INT_MIN;
         if (ok) {
           sc = 0;
+#pragma unroll 4
           for (int w = 0; w < W; ++w) {
-            const uint32_t x = bitsT[w * Nb + me], y = bitsT[w * Nb + cpos];
+            const uint32_t x = bitsT[static_cast<long long>(w) * Nb + me];
+            const uint32_t y = bitsT[static_cast<long long>(w) * Nb + cpos];
             sc += __popc(x & y) - __popc(x ^ y);
           }
         }
@@ -855,17 +884,23 @@ static __device__ void pair_and_order(unsigned long long* keys, const uint32_t* 
         if (lane == 0) best[me] = kb ? static_cast<int>(kb & 0xffffu) : -1;
       }
       __syncthreads();
-      // mutual picks pair up; thread t alone reads and writes partner[alive[t]]
-      const int me = (t < na) ? alive[t] : -1;
-      if (me >= 0) {
-        const int c = best[me];
-        if (c >= 0 && best[c] == me) partner[me] = c;
-      }
-      const bool stay = me >= 0 && partner[me] < 0;
+      // mutual picks pair up, and the unpaired positions are compacted in place,
+      // blockDim.x positions at a time: thread t alone reads and writes
+      // partner[alive[base + t]], and an entry only ever moves to a lower index, so
+      // a chunk's writes never reach entries still to be read
       int nna = 0;
-      // no trailing barrier: sbuf is next written after this round's last barrier
-      const int at = block_exclusive_scan<false>(stay ? 1 : 0, sbuf, &nna);
-      if (stay) alive[at] = me;
+      for (int base = 0; base < na; base += blockDim.x) {
+        const int me = (base + t < na) ? alive[base + t] : -1;
+        if (me >= 0) {
+          const int c = best[me];
+          if (c >= 0 && best[c] == me) partner[me] = c;
+        }
+        const bool stay = me >= 0 && partner[me] < 0;
+        int tot = 0;
+        const int at = block_exclusive_scan(stay ? 1 : 0, sbuf, &tot);   // its barriers order reads and writes
+        if (stay) alive[nna + at] = me;
+        nna += tot;
+      }
       __syncthreads();
       if (nna == na) break;
       na = nna;
@@ -893,7 +928,9 @@ static __device__ void pair_and_order(unsigned long long* keys, const uint32_t* 
     for (int p = threadIdx.x; p < Tq; p += blockDim.x) {
       const int a = pa[p], b = pb[p];
       int c = 0;
-      for (int w = 0; w < W; ++w) c += __popc(bitsT[w * Nb + a] | (b >= 0 ? bitsT[w * Nb + b] : 0u));
+      for (int w = 0; w < W; ++w)
+        c += __popc(bitsT[static_cast<long long>(w) * Nb + a] |
+                    (b >= 0 ? bitsT[static_cast<long long>(w) * Nb + b] : 0u));
       keys2[p] = (static_cast<unsigned long long>(0xffffffu - static_cast<uint32_t>(c)) << 32) |
                  static_cast<unsigned long long>(p);
     }
@@ -929,26 +966,31 @@ static __device__ void pair_and_order(unsigned long long* keys, const uint32_t* 
   }
 }
 
-// One CTA per head: MinHash keys and bitsets from the selection kernel.
+// One CTA per head: MinHash keys and bitsets from the selection kernel. bitsT_g
+// (the plan workspace's bitsT region, [BH][W][Nb]) is needed above
+// blocks per head whose bitsets do not fit in shared memory; without it such heads
+// pair consecutive blocks
+// of the sorted order.
 static __global__ void __launch_bounds__(1024) pair_order_kernel(const unsigned long long* __restrict__ sig,
                                                                  const uint32_t* __restrict__ bits_g,
                                                                  const int* __restrict__ count, int Nb,
-                                                                 int Tq, int G, int* __restrict__ work) {
+                                                                 int Tq, int G, int* __restrict__ work,
+                                                                 uint32_t* __restrict__ bitsT_g) {
   extern __shared__ __align__(16) unsigned char psm[];
   const int P = 1 << (32 - __clz(max(Nb, 2) - 1));
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(psm);
   const long long bh = blockIdx.x;
+  const long long words = static_cast<long long>(Nb) * ((Nb + 31) / 32);
   for (int i = threadIdx.x; i < Nb; i += blockDim.x) keys[i] = sig[bh * Nb + i];
-  pair_and_order(keys, bits_g + bh * static_cast<long long>(Nb) * ((Nb + 31) / 32), count, Nb, Tq, G, bh,
-                 gridDim.x, work, psm + P * sizeof(unsigned long long));
+  pair_and_order(keys, bits_g + bh * words, count, Nb, Tq, G, bh, gridDim.x, work,
+                 psm + P * sizeof(unsigned long long),
+                 (!pair_bits_in_smem(Nb) && bitsT_g != nullptr) ? bitsT_g + bh * words : nullptr);
 }
 
 // Shared memory of pair_order_kernel for Nb blocks per head.
 inline int pair_order_smem_bytes(int Nb) {
-  auto p2 = [](int x) { int p = 2; while (p < x) p <<= 1; return p; };
-  const int Tq = (Nb + 1) / 2;
-  int bytes = (p2(Nb) + p2(Tq)) * 8 + (2 * Tq + 4 * Nb + 34) * 4;
-  if (Nb <= kPairMatchMaxNb) bytes += Nb * ((Nb + 31) / 32) * 4;
+  int bytes = pair_base_smem_bytes(Nb);
+  if (pair_bits_in_smem(Nb)) bytes += Nb * ((Nb + 31) / 32) * 4;
   return bytes;
 }
 

@@ -40,6 +40,7 @@ sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau
   float* Kp = reinterpret_cast<float*>(wsb + L.kp);
   unsigned long long* sig = reinterpret_cast<unsigned long long*>(wsb + L.sig);
   uint32_t* bits = reinterpret_cast<uint32_t*>(wsb + L.bits);
+  uint32_t* bitsT = pair_bits_in_smem(Nb) ? nullptr : reinterpret_cast<uint32_t*>(wsb + L.bitsT);
   pool_kernel<D><<<dim3(static_cast<unsigned>(BH * Nb), 2), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Qp, Kp, s.N, Nb, Q8, K8, qscale,
       kscale, qfmt);
@@ -57,8 +58,10 @@ sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau
   sa_status ls;
   if (Nb <= 256)
     ls = launch_ss(score_select_kernel<D, 4, 128>, 4, 128);
-  else if (Nb <= 3000)
+  else if (Nb <= 1536)
     ls = launch_ss(score_select_kernel<D, 16, 256>, 16, 256);
+  else if (Nb <= 3000)   // 16 warps: a row per warp in the selection, two-pass score rows
+    ls = launch_ss(score_select_kernel<D, 16, 512>, 16, 512);
   else
     ls = launch_ss(score_select_kernel<D, 8, 256>, 8, 256);
   if (ls != SA_OK) return ls;
@@ -70,7 +73,7 @@ sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau
     if (set_smem(pair_order_kernel, smem) != SA_OK) return SA_ERR_CUDA;
     const int G = order_group_heads(BH, s.N, D);
     pair_order_kernel<<<static_cast<unsigned>(BH), pair_order_threads(Nb), smem, st>>>(sig, bits, count, Nb, Tq,
-                                                                                     G, work);
+                                                                                     G, work, bitsT);
     if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   }
   return SA_OK;

@@ -13,8 +13,10 @@
 // GPU that loads the library holds it until the process exits. A call needs the
 // same bytes as sparse_attn_plan_workspace_size: the pooled Q and K
 // (2 * B*H*ceil(N/64)*d*4 bytes) plus, per query block, an 8-byte sort key and a
-// ceil(Nb/32)-word bitset of its kept set (for example H=24, d=128 fits up to
-// N = 75,776). Larger calls are rejected with SA_ERR_WORKSPACE before
+// ceil(Nb/32)-word bitset of its kept set, and, above about 1,200 blocks per
+// head (where the pairing's copy of the bitsets no longer fits in shared memory),
+// that copy (for example H=24, d=128 fits up to N = 75,776). Larger calls are
+// rejected with SA_ERR_WORKSPACE before
 // anything runs.
 //
 // Every call shares the one array, and the array keeps the last call's

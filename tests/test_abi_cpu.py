@@ -48,8 +48,15 @@ def test_workspace_and_tiles(lib):
     Nb = math.ceil(75600 / 64)
     al = lambda x: (x + 255) // 256 * 256
     W = (Nb + 31) // 32
+    # pooled Q and K, sort keys and bitsets (1182 blocks per head: the pairing keeps
+    # its copy of the bitsets in shared memory)
     expect = 2 * al(40 * Nb * 128 * 4) + al(40 * Nb * 8) + al(40 * Nb * W * 4)
     assert lib.sparse_attn_plan_workspace_size(s) == expect
+    big = SaShape(1, 24, 118800, 128, 64)                         # 1857 blocks: a global copy too
+    Nb2 = math.ceil(118800 / 64)
+    W2 = (Nb2 + 31) // 32
+    assert lib.sparse_attn_plan_workspace_size(big) == (2 * al(24 * Nb2 * 128 * 4) + al(24 * Nb2 * 8)
+                                                        + 2 * al(24 * Nb2 * W2 * 4))
     assert lib.sparse_attn_num_tiles(s) == 40 * ((Nb + 1) // 2)
     assert lib.sparse_attn_num_tiles(SaShape(2, 3, 1, 64, 64)) == 6
     for bad in (SaShape(1, 1, 64, 96, 64), SaShape(1, 1, 64, 128, 32), SaShape(0, 1, 64, 128, 64),
