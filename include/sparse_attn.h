@@ -88,9 +88,10 @@ int64_t sparse_attn_num_tiles(sa_shape s);
  *             ((b*H + h)*Nb + i; the second is -1 when a head has an odd block
  *             count). Every query block appears exactly once. Within a head,
  *             blocks are paired so that the two kept sets overlap (sorted by two
- *             MinHash signatures of the kept set, then each block takes the
- *             best-matching unused block among the next 32, for Nb <= 1024;
- *             consecutive blocks of that order above), and the head's tiles are
+ *             MinHash signatures of the kept set, then, in up to six rounds, blocks
+ *             that pick each other as the best match among the 32 unpaired blocks
+ *             within 16 places in that order are paired, the rest in order), and
+ *             the head's tiles are
  *             ranked by decreasing union size (longest first). Heads are taken in
  *             ascending (b,h) order in groups of G consecutive heads, G being the
  *             most heads whose K and V together fit in 64 MB (at least 1); within a
