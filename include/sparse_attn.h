@@ -62,7 +62,9 @@ typedef struct {
 
 /* Bytes of device workspace sparse_attn_plan needs for shape s: pooled Q and K
  * (fp32 [B,H,Nb,d] each), an 8-byte sort key and a ceil(Nb/32)-word kept-set
- * bitset per query block, each region 256-byte aligned. 0 if the shape is invalid. */
+ * bitset per query block, and, above about 1,200 blocks per head (where the
+ * pairing's copy of the bitsets no longer fits in shared memory), that copy; each
+ * region 256-byte aligned. 0 if the shape is invalid. */
 size_t sparse_attn_plan_workspace_size(sa_shape s);
 
 /* Number of 128-row query tiles, B*H*ceil(Nb/2); `work` holds two entries per
@@ -91,8 +93,8 @@ int64_t sparse_attn_num_tiles(sa_shape s);
  *             MinHash signatures of the kept set, then, in up to six rounds, blocks
  *             that pick each other as the best match among the 32 unpaired blocks
  *             within 16 places in that order are paired, the rest in order), and
- *             the head's tiles are
- *             ranked by decreasing union size (longest first). Heads are taken in
+ *             the head's tiles are ranked by decreasing union size (longest
+ *             first). Heads are taken in
  *             ascending (b,h) order in groups of G consecutive heads, G being the
  *             most heads whose K and V together fit in 64 MB (at least 1); within a
  *             group the tiles are interleaved by rank (rank 0 of every head of the
