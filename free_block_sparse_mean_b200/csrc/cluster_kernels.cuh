@@ -43,10 +43,12 @@ inline int gram_chunk(long long BH, int N) {
 }
 
 // Byte offsets of the clustering workspace: partial Gram matrices, the Gram
-// matrix, centroids, w_c = G c, b_c, cluster sizes, first positions, and the
-// assignment (when the caller does not want it back).
+// matrix, centroids, w_c = G c, b_c, cluster sizes, first positions, the
+// assignment (when the caller does not want it back), the tensor-core operand
+// rows of the centroids (bf16 [B*H][C][D + 64], see cluster_prep_kernel) and four
+// candidate clusters per token.
 struct ClusterWorkspace {
-  size_t gpart, gram, cent, w, b, cnt, off, assign, total;
+  size_t gpart, gram, cent, w, b, cnt, off, assign, w16, cand, total;
   int splits, chunk, C;
 };
 inline ClusterWorkspace cluster_workspace(long long BH, int N, int D) {
@@ -66,7 +68,9 @@ inline ClusterWorkspace cluster_workspace(long long BH, int N, int D) {
   w.cnt = w.b + al(c4);
   w.off = w.cnt + al(c4);
   w.assign = w.off + al(c4);
-  w.total = w.assign + al(static_cast<size_t>(BH) * N * sizeof(int));
+  w.w16 = w.assign + al(static_cast<size_t>(BH) * N * sizeof(int));
+  w.cand = w.w16 + al(static_cast<size_t>(BH) * w.C * (D + 64) * 2);
+  w.total = w.cand + al(static_cast<size_t>(BH) * N * 4 * sizeof(int));
   return w;
 }
 
@@ -152,13 +156,19 @@ __global__ void __launch_bounds__(256) cluster_init_assign_kernel(int* __restric
 // sizes cleared for the assignment to count. Grid
 // (ceil(C/16), B*H), D threads: thread i forms component i (G is symmetric, so
 // it reads column i of G as row i, and a warp reads G row by row).
+//
+// W16 (bf16 [B*H][C][D + 64]) receives each centroid's tensor-core operand row for
+// the assignment: -2 w_c in columns [0, D), then b_c as the sum of two bf16 values
+// (b_hi = bf16(b_c) in column D, b_lo = bf16(b_c - b_hi) in column D + 1) and zeros.
 template <int D>
 __global__ void __launch_bounds__(D) cluster_prep_kernel(const float* __restrict__ G, const float* __restrict__ cent,
                                                          float* __restrict__ W, float* __restrict__ bvec,
-                                                         int* __restrict__ cnt, int C) {
+                                                         int* __restrict__ cnt, int C,
+                                                         __nv_bfloat16* __restrict__ W16) {
   constexpr int kCl = 16;
   __shared__ float cs[kCl][D];
   __shared__ float red[kCl][D / 32];
+  __shared__ float bsh[kCl];
   const long long bh = blockIdx.y;
   const int c0 = blockIdx.x * kCl;
   const int ncl = min(kCl, C - c0);
@@ -177,7 +187,10 @@ __global__ void __launch_bounds__(D) cluster_prep_kernel(const float* __restrict
   }
 #pragma unroll
   for (int c = 0; c < kCl; ++c) {
-    if (c < ncl) W[(bh * C + c0 + c) * D + i] = acc[c];
+    if (c < ncl) {
+      W[(bh * C + c0 + c) * D + i] = acc[c];
+      W16[(bh * C + c0 + c) * (D + 64) + i] = __float2bfloat16_rn(-2.f * acc[c]);
+    }
     float v = cs[c][i] * acc[c];
 #pragma unroll
     for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -189,7 +202,19 @@ __global__ void __launch_bounds__(D) cluster_prep_kernel(const float* __restrict
 #pragma unroll
     for (int w = 0; w < D / 32; ++w) b += red[i][w];
     bvec[bh * C + c0 + i] = b;
+    bsh[i] = b;
     cnt[bh * C + c0 + i] = 0;   // counted again by the assignment
+  }
+  __syncthreads();
+  // the bias columns of the operand rows: b_hi, b_lo, then zeros
+  for (int x = i; x < ncl * 64; x += D) {
+    const int c = x >> 6, k = x & 63;
+    const float b = bsh[c];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(b);
+    __nv_bfloat16 v = __float2bfloat16_rn(0.f);
+    if (k == 0) v = hi;
+    if (k == 1) v = __float2bfloat16_rn(b - __bfloat162float(hi));
+    W16[(bh * C + c0 + c) * (D + 64) + D + k] = v;
   }
 }
 
@@ -313,6 +338,285 @@ __global__ void __launch_bounds__(256) cluster_assign_kernel(const __nv_bfloat16
     assign[bh * N + t0 + threadIdx.x] = bi;
     atomicAdd(&cnt[bh * C + bi], 1);
   }
+}
+
+// ----------------------------------------------------------------------------
+// Tensor-core assignment: the four nearest centroids of every token by a bf16
+// product on the tensor cores, then the exact argmin among those four in fp32
+// (cluster_rescore_kernel). One CTA = 128 tokens of one head:
+//   D[token][c] = x . (-2 w_c) + 1 . b_hi_c + 1 . b_lo_c
+// (tcgen05.mma kind::f16, fp32 accumulate in TMEM), over tiles of 128 centroids:
+// D / 16 K-steps of the token tile (TMA'd once) against the centroid tile's bf16
+// rows from cluster_prep_kernel, plus one K-step of a constant tile whose rows
+// start with two ones against the rows' bias columns. Warp 4 (one thread) loads
+// and issues; warps 0-3 (thread = token = TMEM lane) keep each token's four
+// smallest D values with their centroids (ties to the lower centroid) in
+// registers. Two TMEM buffers of 128 columns and three centroid-tile stages keep
+// the tensor cores and the epilogue overlapped.
+// The bf16 product moves the argmin for a fraction of a percent of the tokens;
+// the four best of the product contain the fp32 argmin (measured on the
+// workloads' inputs), and the re-score restores it exactly.
+template <int D>
+struct ClusterTcCfg {
+  static constexpr int kCh = D / 64;                   // 128-byte column chunks of a row
+  static constexpr int kTile = 128;                    // tokens per CTA, centroids per tile
+  static constexpr int kChunkBytes = kTile * 128;      // 16 KB: one column chunk of a tile
+  static constexpr int kStages = 3;
+  static constexpr int kWStage = (kCh + 1) * kChunkBytes;   // centroid rows + bias chunk
+  static constexpr int oX = 0;
+  static constexpr int oOnes = oX + kCh * kChunkBytes;
+  static constexpr int oW = oOnes + kChunkBytes;
+  static constexpr int oBar = oW + kStages * kWStage;
+  static constexpr int kSmemBytes = oBar + 128 + 1024;
+  static constexpr uint32_t kTmemCols = 256;
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128, false);
+};
+
+template <int D>
+__global__ void __launch_bounds__(160, 1)
+    cluster_assign_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                             int N, int C, int* __restrict__ cand) {
+  using Cf = ClusterTcCfg<D>;
+  extern __shared__ uint8_t tsm_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tsm_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sX = base + Cf::oX;
+  uint8_t* sOnes = base + Cf::oOnes;
+  uint8_t* sW = base + Cf::oW;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + Cf::oBar);
+  uint64_t* wfull = bars;                      // [3]
+  uint64_t* wempty = bars + 3;                 // [3]
+  uint64_t* dfull = bars + 6;                  // [2]
+  uint64_t* dempty = bars + 8;                 // [2], 4 arrivals
+  uint64_t* xfull = bars + 10;
+  uint64_t* drain = bars + 11;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 12);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 13);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long bh = blockIdx.y;
+  const int t0 = blockIdx.x * Cf::kTile;
+  const int ntiles = (C + Cf::kTile - 1) / Cf::kTile;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Cf::kStages; ++s) {
+      mbar_init(&wfull[s], 1);
+      mbar_init(&wempty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&dfull[b], 1);
+      mbar_init(&dempty[b], 4);
+    }
+    mbar_init(xfull, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // the constant tile: row r holds ones in columns 0 and 1 (16-byte chunk 0 of the
+  // row, which the 128-byte swizzle stores at chunk (r & 7)), zeros elsewhere
+  for (int x = threadIdx.x; x < Cf::kChunkBytes / 16; x += blockDim.x)
+    reinterpret_cast<uint4*>(sOnes)[x] = make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();
+  if (threadIdx.x < Cf::kTile) {
+    const int r = threadIdx.x;
+    const uint32_t one2 = 0x3F803F80u;         // two bf16 ones
+    *reinterpret_cast<uint32_t*>(sOnes + r * 128 + (r & 7) * 16) = one2;
+  }
+  fence_proxy_async_smem();                    // generic-proxy writes -> the tensor cores' reads
+  if (warp == 4) tmem_alloc(tmem_holder, Cf::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ loads and MMAs
+    if (lane == 0) {
+      tma_prefetch_desc(&tmX);
+      tma_prefetch_desc(&tmW);
+      mbar_expect_tx(xfull, Cf::kCh * Cf::kChunkBytes);
+      for (int c = 0; c < Cf::kCh; ++c)
+        tma_load_3d(sX + c * Cf::kChunkBytes, &tmX, c * 64, t0, static_cast<int>(bh), xfull);
+      auto load_w = [&](int t) {
+        const int s = t % Cf::kStages;
+        mbar_expect_tx(&wfull[s], Cf::kWStage);
+        for (int c = 0; c <= Cf::kCh; ++c)
+          tma_load_3d(sW + s * Cf::kWStage + c * Cf::kChunkBytes, &tmW, c * 64, t * Cf::kTile,
+                      static_cast<int>(bh), &wfull[s]);
+      };
+      int nw = 0;
+      for (; nw < Cf::kStages && nw < ntiles; ++nw) load_w(nw);
+      const uint32_t xa = smem_u32(sX), oa = smem_u32(sOnes), wa = smem_u32(sW);
+      bool ok = mbar_wait(xfull, 0u, abort_flag);
+      for (int t = 0; ok && t < ntiles; ++t) {
+        const int s = t % Cf::kStages, buf = t & 1;
+        if (!mbar_wait(&wfull[s], static_cast<uint32_t>(t / Cf::kStages) & 1u, abort_flag)) break;
+        if (t >= 2 && !mbar_wait(&dempty[buf], static_cast<uint32_t>((t >> 1) - 1) & 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t dD = tmem_base + buf * 128;
+        const uint32_t wb = wa + s * Cf::kWStage;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * Cf::kChunkBytes + (kk & 3) * 32;
+          tc_mma_ss(dD, sdesc_sw128(xa + off, 16, 1024), sdesc_sw128(wb + off, 16, 1024), Cf::kIdesc,
+                    kk > 0 ? 1u : 0u);
+        }
+        // the bias: the ones tile's first K-step against the rows' bias columns
+        tc_mma_ss(dD, sdesc_sw128(oa, 16, 1024), sdesc_sw128(wb + Cf::kCh * Cf::kChunkBytes, 16, 1024), Cf::kIdesc,
+                  1u);
+        tc_commit(&dfull[buf]);
+        tc_commit(&wempty[s]);
+        if (t + Cf::kStages < ntiles) {
+          if (!mbar_wait(&wempty[s], static_cast<uint32_t>(t / Cf::kStages) & 1u, abort_flag)) break;
+          load_w(t + Cf::kStages);
+          ++nw;
+        }
+      }
+      tc_commit(drain);
+      mbar_wait_drain(drain, 0u);
+      mbar_wait_drain(xfull, 0u);
+      for (int k = max(0, nw - Cf::kStages); k < nw; ++k)
+        mbar_wait_drain(&wfull[k % Cf::kStages], static_cast<uint32_t>(k / Cf::kStages) & 1u);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue: the four best
+    const int row = warp * 32 + lane;          // token of the tile == TMEM lane
+    const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
+    float b0 = INFINITY, b1 = INFINITY, b2 = INFINITY, b3 = INFINITY;
+    int i0 = 0x7fffffff, i1 = 0x7fffffff, i2 = 0x7fffffff, i3 = 0x7fffffff;
+    bool alive = true;
+    for (int t = 0; t < ntiles; ++t) {
+      const int buf = t & 1;
+      if (!warp_wait(&dfull[buf], static_cast<uint32_t>(t >> 1) & 1u, abort_flag)) {
+        alive = false;
+        break;
+      }
+      tc_fence_after();
+      float v[128];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        tmem_ld32(tmem_base + lane_bits + buf * 128 + q * 32, *reinterpret_cast<float(*)[32]>(&v[32 * q]));
+      tmem_wait_ld();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) pin32(*reinterpret_cast<float(*)[32]>(&v[32 * q]));
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&dempty[buf]);   // the buffer may take tile t + 2
+      const int c0 = t * Cf::kTile;
+      const int ncol = min(Cf::kTile, C - c0);
+#pragma unroll
+      for (int g = 0; g < Cf::kTile; g += 8) {
+        const float gm = fminf(fminf(fminf(v[g], v[g + 1]), fminf(v[g + 2], v[g + 3])),
+                               fminf(fminf(v[g + 4], v[g + 5]), fminf(v[g + 6], v[g + 7])));
+        if (g + 8 > ncol || gm < b3) {             // rare once the four best have settled
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float x = v[g + e];
+            const int c = c0 + g + e;
+            if (g + e < ncol && x < b3) {          // centroids in ascending order: ties keep the first
+              if (x < b2) {
+                b3 = b2;
+                i3 = i2;
+                if (x < b1) {
+                  b2 = b1;
+                  i2 = i1;
+                  if (x < b0) {
+                    b1 = b0;
+                    i1 = i0;
+                    b0 = x;
+                    i0 = c;
+                  } else {
+                    b1 = x;
+                    i1 = c;
+                  }
+                } else {
+                  b2 = x;
+                  i2 = c;
+                }
+              } else {
+                b3 = x;
+                i3 = c;
+              }
+            }
+          }
+        }
+      }
+    }
+    const int tok = t0 + row;
+    if (alive && tok < N) {
+      int4 o;
+      o.x = i0;
+      o.y = i1;
+      o.z = i2;
+      o.w = i3;
+      *reinterpret_cast<int4*>(cand + (bh * N + tok) * 4) = o;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cf::kTmemCols);
+  }
+}
+
+// The exact argmin among a token's four candidates: b_c - 2 x . w_c in fp32
+// (x the bf16 token, w_c and b_c from cluster_prep_kernel), ties to the lowest c;
+// the winner is counted into its cluster's size. A candidate outside [0, C) (a
+// head with fewer than four clusters) is skipped. One thread per token.
+template <int D>
+__global__ void __launch_bounds__(256) cluster_rescore_kernel(const __nv_bfloat16* __restrict__ X,
+                                                              const float* __restrict__ W,
+                                                              const float* __restrict__ bvec,
+                                                              const int* __restrict__ cand,
+                                                              int* __restrict__ assign, int* __restrict__ cnt, int N,
+                                                              int C) {
+  const long long bh = blockIdx.y;
+  const int tok = blockIdx.x * 256 + threadIdx.x;
+  if (tok >= N) return;
+  float x[D];
+  const uint4* src = reinterpret_cast<const uint4*>(X + (bh * N + tok) * static_cast<long long>(D));
+#pragma unroll
+  for (int q = 0; q < D / 8; ++q) {
+    const uint4 u = __ldg(src + q);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h[e]);
+      x[8 * q + 2 * e] = f.x;
+      x[8 * q + 2 * e + 1] = f.y;
+    }
+  }
+  const int4 cd = *reinterpret_cast<const int4*>(cand + (bh * N + tok) * 4);
+  const int cs[4] = {cd.x, cd.y, cd.z, cd.w};
+  float best = INFINITY;
+  int bi = 0x7fffffff;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int c = cs[q];
+    if (c < 0 || c >= C) continue;
+    const float4* w = reinterpret_cast<const float4*>(W + (bh * C + c) * static_cast<long long>(D));
+    float dot = 0.f;
+#pragma unroll
+    for (int k = 0; k < D / 4; ++k) {
+      const float4 wv = __ldg(w + k);
+      dot = fmaf(x[4 * k], wv.x, dot);
+      dot = fmaf(x[4 * k + 1], wv.y, dot);
+      dot = fmaf(x[4 * k + 2], wv.z, dot);
+      dot = fmaf(x[4 * k + 3], wv.w, dot);
+    }
+    const float sc = bvec[bh * C + c] - 2.f * dot;
+    if (sc < best || (sc == best && c < bi)) {
+      best = sc;
+      bi = c;
+    }
+  }
+  // a NaN score never compares smaller: a token whose every candidate scores NaN
+  // keeps no cluster, which the range check turns into cluster 0 and an error bit
+  if (bi < 0 || bi >= C) {
+    atomicOr(&g_dev_error, DEVERR_VALUE);
+    bi = 0;
+  }
+  assign[bh * N + tok] = bi;
+  atomicAdd(&cnt[bh * C + bi], 1);
 }
 
 // Clusters per CTA of cluster_order_kernel.

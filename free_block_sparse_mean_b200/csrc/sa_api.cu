@@ -131,6 +131,21 @@ sa_status launch_fwd(const sa_shape& s, const void* Q, const void* K, const void
   return SA_OK;
 }
 
+// The centroids' bf16 operand rows [B*H][C][D + 64] as a 3-D tensor {D + 64, C,
+// B*H}; box {64, 128 rows, 1}, 128B swizzle. Rows past C read as zero.
+bool make_w16_map(CUtensorMap* map, const void* ptr, long long BH, int C, int D) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D + 64), static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D + 64) * 2, static_cast<cuuint64_t>(C) * (D + 64) * 2};
+  cuuint32_t box[3] = {64u, 128u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Interaction clustering of X under the Gram metric of Y (see cluster_kernels.cuh).
 template <int D>
 sa_status launch_cluster(const sa_shape& s, const void* X, const void* Y, int iters, int32_t* assign_out,
@@ -148,6 +163,8 @@ sa_status launch_cluster(const sa_shape& s, const void* X, const void* Y, int it
   int* cnt = reinterpret_cast<int*>(wsb + L.cnt);
   int* off = reinterpret_cast<int*>(wsb + L.off);
   int* assign = assign_out ? assign_out : reinterpret_cast<int*>(wsb + L.assign);
+  auto* w16 = reinterpret_cast<__nv_bfloat16*>(wsb + L.w16);
+  int* cand = reinterpret_cast<int*>(wsb + L.cand);
   const auto* x = static_cast<const __nv_bfloat16*>(X);
   const auto* y = static_cast<const __nv_bfloat16*>(Y);
   const unsigned by = static_cast<unsigned>(BH);
@@ -159,13 +176,16 @@ sa_status launch_cluster(const sa_shape& s, const void* X, const void* Y, int it
   sa::cluster_init_assign_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(assign, cnt, N, C,
                                                                                                total);
   if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
-  constexpr int kAssignSmem = sa::cluster_assign_smem_bytes<D>();
-  if (sa::set_smem(sa::cluster_assign_kernel<D>, kAssignSmem) != SA_OK) return SA_ERR_CUDA;
+  using TC = sa::ClusterTcCfg<D>;
+  if (sa::set_smem(sa::cluster_assign_tc_kernel<D>, TC::kSmemBytes) != SA_OK) return SA_ERR_CUDA;
+  CUtensorMap mx, mw;
+  if (iters > 0 && (!make_map(&mx, X, s, 128) || !make_w16_map(&mw, w16, BH, C, D))) return SA_ERR_CUDA;
   const dim3 order_grid((C + sa::kOrderClusters - 1) / sa::kOrderClusters, by);
   const dim3 cent_grid((C + 7) / 8, by);
   for (int it = 0; it < iters; ++it) {
-    sa::cluster_prep_kernel<D><<<dim3((C + 15) / 16, by), D, 0, st>>>(G, cent, W, bvec, cnt, C);
-    sa::cluster_assign_kernel<D><<<dim3((N + 63) / 64, by), 256, kAssignSmem, st>>>(x, W, bvec, assign, cnt, N, C);
+    sa::cluster_prep_kernel<D><<<dim3((C + 15) / 16, by), D, 0, st>>>(G, cent, W, bvec, cnt, C, w16);
+    sa::cluster_assign_tc_kernel<D><<<dim3((N + 127) / 128, by), 160, TC::kSmemBytes, st>>>(mx, mw, N, C, cand);
+    sa::cluster_rescore_kernel<D><<<dim3((N + 255) / 256, by), 256, 0, st>>>(x, W, bvec, cand, assign, cnt, N, C);
     sa::cluster_offsets_kernel<<<by, 1024, 0, st>>>(cnt, off, C);
     sa::cluster_order_kernel<<<order_grid, 256, 0, st>>>(assign, off, perm, N, C);
     sa::cluster_centroid_kernel<D><<<cent_grid, 256, 0, st>>>(x, perm, off, cnt, cent, N, C);
