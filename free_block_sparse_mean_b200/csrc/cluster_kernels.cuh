@@ -8,9 +8,11 @@
 // (x - c)^T G (x - c) with G = sum_y y y^T. Dropping the term x^T G x, which is
 // the same for every centroid, the nearest centroid is the argmin over c of
 // c^T G c - 2 x . (G c). So each Lloyd iteration is: w_c = G c and b_c = c . w_c
-// per centroid (cluster_prep_kernel), an argmin over all centroids per token
-// (cluster_assign_kernel, a register-tiled fp32 product of the tokens with the
-// w_c), and the mean of each cluster's tokens (cluster_centroid_kernel). The
+// per centroid (cluster_prep_kernel), an argmin over all centroids per token (a
+// bf16 tensor-core product of the tokens with the w_c that keeps each token's four
+// best, cluster_assign_tc_kernel, then their exact fp32 scores,
+// cluster_rescore_kernel), and the mean of each cluster's tokens
+// (cluster_centroid_kernel). The
 // clusters start at the 64-token block means (the pooling kernel), so zero
 // iterations reproduce the plain blocks.
 //
@@ -20,8 +22,9 @@
 // so the tail of one shares a 64-token block with the head of the next (the
 // abstract's "tail merging", with no padding at all).
 //
-// Each iteration: cluster_prep_kernel (w_c, b_c; clears the sizes),
-// cluster_assign_kernel (argmin; counts the sizes), cluster_offsets_kernel (each
+// Each iteration: cluster_prep_kernel (w_c, b_c, their bf16 operand rows; clears
+// the sizes), cluster_assign_tc_kernel and cluster_rescore_kernel (argmin; counts
+// the sizes), cluster_offsets_kernel (each
 // cluster's first position), cluster_order_kernel (the stable order) and
 // cluster_centroid_kernel (each cluster's mean, summed over its tokens in token
 // order through the order just built). Everything is deterministic: every fp32
@@ -218,128 +221,6 @@ __global__ void __launch_bounds__(D) cluster_prep_kernel(const float* __restrict
   }
 }
 
-// Shared memory of cluster_assign_kernel: 64 tokens and 64 w_c, both D x 64 fp32.
-template <int D>
-constexpr int cluster_assign_smem_bytes() {
-  return 2 * D * 64 * static_cast<int>(sizeof(float));
-}
-
-// Nearest centroid of 64 tokens of one head: argmin over c of b_c - 2 x . w_c,
-// fp32, ties to the lowest c. Grid (ceil(N/64), B*H), 256 threads. Tokens and
-// w_c sit in shared memory dimension-major, so a thread's 4 tokens and 4
-// centroids are one 16-byte read each per dimension; thread (tg, cg) forms the
-// 4 x 4 products of tokens 4 tg .. and centroids 4 cg .. of each chunk of 64
-// centroids and keeps its 4 running minima; the 16 threads of a token group
-// then meet in shared memory, and the winner is counted into its cluster's size.
-template <int D>
-__global__ void __launch_bounds__(256) cluster_assign_kernel(const __nv_bfloat16* __restrict__ X,
-                                                             const float* __restrict__ W,
-                                                             const float* __restrict__ bvec, int* __restrict__ assign,
-                                                             int* __restrict__ cnt, int N, int C) {
-  extern __shared__ __align__(16) float csm[];
-  float* xs = csm;            // [D][64]: xs[k * 64 + token]
-  float* ws = csm + D * 64;   // [D][64]: ws[k * 64 + centroid of the chunk]
-  __shared__ float bs[64];
-  __shared__ float rsc[16][64];
-  __shared__ int ridx[16][64];
-  const long long bh = blockIdx.y;
-  const int t0 = blockIdx.x * 64;
-  const int nt = min(64, N - t0);
-  const __nv_bfloat16* src = X + (bh * N + t0) * static_cast<long long>(D);
-  for (int x = threadIdx.x; x < 64 * D / 8; x += 256) {
-    const int r = x & 63, c8 = (x >> 6) * 8;
-    uint4 u = make_uint4(0u, 0u, 0u, 0u);
-    if (r < nt) u = __ldg(reinterpret_cast<const uint4*>(src + static_cast<long long>(r) * D + c8));
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = __bfloat1622float2(h[e]);
-      xs[(c8 + 2 * e) * 64 + r] = f.x;
-      xs[(c8 + 2 * e + 1) * 64 + r] = f.y;
-    }
-  }
-  const int tg = threadIdx.x & 15, cg = threadIdx.x >> 4;
-  float best[4];
-  int bidx[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    best[i] = INFINITY;
-    bidx[i] = 0x7fffffff;
-  }
-  const float* wsrc = W + bh * static_cast<long long>(C) * D;
-  for (int cc = 0; cc < C; cc += 64) {
-    const int ncc = min(64, C - cc);
-    __syncthreads();   // the previous chunk is consumed (and, the first time, xs is written)
-    for (int x = threadIdx.x; x < 64 * D / 4; x += 256) {
-      const int c = x & 63, k4 = (x >> 6) * 4;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (c < ncc) v = __ldg(reinterpret_cast<const float4*>(wsrc + static_cast<long long>(cc + c) * D + k4));
-      ws[(k4 + 0) * 64 + c] = v.x;
-      ws[(k4 + 1) * 64 + c] = v.y;
-      ws[(k4 + 2) * 64 + c] = v.z;
-      ws[(k4 + 3) * 64 + c] = v.w;
-    }
-    if (threadIdx.x < 64) bs[threadIdx.x] = threadIdx.x < ncc ? bvec[bh * C + cc + threadIdx.x] : 0.f;
-    __syncthreads();
-    float acc[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-#pragma unroll 8
-    for (int k = 0; k < D; ++k) {
-      const float4 xv = *reinterpret_cast<const float4*>(&xs[k * 64 + 4 * tg]);
-      const float4 wv = *reinterpret_cast<const float4*>(&ws[k * 64 + 4 * cg]);
-      const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
-      const float wa[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(xa[i], wa[j], acc[i][j]);
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int cl = 4 * cg + j;
-      if (cl < ncc) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float sc = bs[cl] - 2.f * acc[i][j];
-          if (sc < best[i]) {       // centroids arrive in ascending order: ties keep the first
-            best[i] = sc;
-            bidx[i] = cc + cl;
-          }
-        }
-      }
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    rsc[cg][4 * tg + i] = best[i];
-    ridx[cg][4 * tg + i] = bidx[i];
-  }
-  __syncthreads();
-  if (threadIdx.x < nt) {
-    float b = rsc[0][threadIdx.x];
-    int bi = ridx[0][threadIdx.x];
-    for (int g = 1; g < 16; ++g) {
-      const float v = rsc[g][threadIdx.x];
-      const int vi = ridx[g][threadIdx.x];
-      if (v < b || (v == b && vi < bi)) {
-        b = v;
-        bi = vi;
-      }
-    }
-    // a NaN score never compares smaller: a token whose every score is NaN keeps
-    // no cluster, which the range check below turns into cluster 0 and an error bit
-    if (bi < 0 || bi >= C) {
-      atomicOr(&g_dev_error, DEVERR_VALUE);
-      bi = 0;
-    }
-    assign[bh * N + t0 + threadIdx.x] = bi;
-    atomicAdd(&cnt[bh * C + bi], 1);
-  }
-}
-
 // ----------------------------------------------------------------------------
 // Tensor-core assignment: the four nearest centroids of every token by a bf16
 // product on the tensor cores, then the exact argmin among those four in fp32
@@ -371,6 +252,37 @@ struct ClusterTcCfg {
   static constexpr uint32_t kTmemCols = 256;
   static constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128, false);
 };
+
+// A token's four smallest scores so far, ascending, with their centroids (the
+// epilogue's state, touched only when a score may enter).
+struct Top4 {
+  float b[4];
+  int i[4];
+};
+
+// Offers the scores x[e] of centroids c0 + e (e < lim) in ascending centroid order;
+// a score enters if it is smaller than the fourth best (so a tie keeps the earlier
+// centroid). Returns the new fourth best. Not inlined: the insertion code then
+// exists once, and the epilogue's hot path stays small.
+static __device__ __noinline__ float top4_offer8(Top4* st, float x0, float x1, float x2, float x3, float x4,
+                                                 float x5, float x6, float x7, int c0, int lim) {
+  const float xs[8] = {x0, x1, x2, x3, x4, x5, x6, x7};
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float x = xs[e];
+    if (e < lim && x < st->b[3]) {
+      int p = 3;
+      while (p > 0 && x < st->b[p - 1]) {
+        st->b[p] = st->b[p - 1];
+        st->i[p] = st->i[p - 1];
+        --p;
+      }
+      st->b[p] = x;
+      st->i[p] = c0 + e;
+    }
+  }
+  return st->b[3];
+}
 
 template <int D>
 __global__ void __launch_bounds__(160, 1)
@@ -480,8 +392,13 @@ __global__ void __launch_bounds__(160, 1)
     // ------------------------------------------------------------ epilogue: the four best
     const int row = warp * 32 + lane;          // token of the tile == TMEM lane
     const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
-    float b0 = INFINITY, b1 = INFINITY, b2 = INFINITY, b3 = INFINITY;
-    int i0 = 0x7fffffff, i1 = 0x7fffffff, i2 = 0x7fffffff, i3 = 0x7fffffff;
+    Top4 st;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      st.b[q] = INFINITY;
+      st.i[q] = 0x7fffffff;
+    }
+    float b3 = INFINITY;                       // st.b[3], in a register for the hot path
     bool alive = true;
     for (int t = 0; t < ntiles; ++t) {
       const int buf = t & 1;
@@ -502,40 +419,22 @@ __global__ void __launch_bounds__(160, 1)
       if (lane == 0) mbar_arrive(&dempty[buf]);   // the buffer may take tile t + 2
       const int c0 = t * Cf::kTile;
       const int ncol = min(Cf::kTile, C - c0);
+      const bool partial = ncol < Cf::kTile;   // the last tile: columns past C read zero rows
 #pragma unroll
-      for (int g = 0; g < Cf::kTile; g += 8) {
-        const float gm = fminf(fminf(fminf(v[g], v[g + 1]), fminf(v[g + 2], v[g + 3])),
-                               fminf(fminf(v[g + 4], v[g + 5]), fminf(v[g + 6], v[g + 7])));
-        if (g + 8 > ncol || gm < b3) {             // rare once the four best have settled
+      for (int q = 0; q < 4; ++q) {
+        const float* w = v + 32 * q;
+        float m8[4];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float x = v[g + e];
-            const int c = c0 + g + e;
-            if (g + e < ncol && x < b3) {          // centroids in ascending order: ties keep the first
-              if (x < b2) {
-                b3 = b2;
-                i3 = i2;
-                if (x < b1) {
-                  b2 = b1;
-                  i2 = i1;
-                  if (x < b0) {
-                    b1 = b0;
-                    i1 = i0;
-                    b0 = x;
-                    i0 = c;
-                  } else {
-                    b1 = x;
-                    i1 = c;
-                  }
-                } else {
-                  b2 = x;
-                  i2 = c;
-                }
-              } else {
-                b3 = x;
-                i3 = c;
-              }
-            }
+        for (int g = 0; g < 4; ++g)
+          m8[g] = fminf(fminf(fminf(w[8 * g], w[8 * g + 1]), fminf(w[8 * g + 2], w[8 * g + 3])),
+                        fminf(fminf(w[8 * g + 4], w[8 * g + 5]), fminf(w[8 * g + 6], w[8 * g + 7])));
+        if (partial || fminf(fminf(m8[0], m8[1]), fminf(m8[2], m8[3])) < b3) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int cb = 32 * q + 8 * g;
+            if (cb < ncol && (partial || m8[g] < b3))
+              b3 = top4_offer8(&st, w[8 * g], w[8 * g + 1], w[8 * g + 2], w[8 * g + 3], w[8 * g + 4],
+                               w[8 * g + 5], w[8 * g + 6], w[8 * g + 7], c0 + cb, ncol - cb);
           }
         }
       }
@@ -543,10 +442,10 @@ __global__ void __launch_bounds__(160, 1)
     const int tok = t0 + row;
     if (alive && tok < N) {
       int4 o;
-      o.x = i0;
-      o.y = i1;
-      o.z = i2;
-      o.w = i3;
+      o.x = st.i[0];
+      o.y = st.i[1];
+      o.z = st.i[2];
+      o.w = st.i[3];
       *reinterpret_cast<int4*>(cand + (bh * N + tok) * 4) = o;
     }
   }
