@@ -48,16 +48,18 @@ inline int gram_chunk(long long BH, int N) {
 // Byte offsets of the clustering workspace: partial Gram matrices, the Gram
 // matrix, centroids, w_c = G c, b_c, cluster sizes, first positions, the
 // assignment (when the caller does not want it back), the tensor-core operand
-// rows of the centroids (bf16 [B*H][C][D + 64], see cluster_prep_kernel) and four
-// candidate clusters per token.
+// rows of the centroids (bf16 [B*H][C][D], see cluster_prep_kernel), b_c again
+// padded to a multiple of 64 clusters per head, and four candidate clusters per
+// token.
 struct ClusterWorkspace {
-  size_t gpart, gram, cent, w, b, cnt, off, assign, w16, cand, total;
-  int splits, chunk, C;
+  size_t gpart, gram, cent, w, b, cnt, off, assign, w16, bpad, cand, total;
+  int splits, chunk, C, Cpad;
 };
 inline ClusterWorkspace cluster_workspace(long long BH, int N, int D) {
   auto al = [](size_t x) { return (x + 255) / 256 * 256; };
   ClusterWorkspace w;
   w.C = (N + kBlock - 1) / kBlock;
+  w.Cpad = (w.C + 63) / 64 * 64;
   w.chunk = gram_chunk(BH, N);
   w.splits = (N + w.chunk - 1) / w.chunk;
   const size_t dd = static_cast<size_t>(D) * D * sizeof(float);
@@ -72,64 +74,141 @@ inline ClusterWorkspace cluster_workspace(long long BH, int N, int D) {
   w.off = w.cnt + al(c4);
   w.assign = w.off + al(c4);
   w.w16 = w.assign + al(static_cast<size_t>(BH) * N * sizeof(int));
-  w.cand = w.w16 + al(static_cast<size_t>(BH) * w.C * (D + 64) * 2);
+  w.bpad = w.w16 + al(static_cast<size_t>(BH) * w.C * D * 2);
+  w.cand = w.bpad + al(static_cast<size_t>(BH) * w.Cpad * sizeof(float));
   w.total = w.cand + al(static_cast<size_t>(BH) * N * 4 * sizeof(int));
   return w;
 }
 
 // Partial Gram matrix sum_t y_t y_t^T over one chunk of `chunk` tokens of one
-// head, fp32, tokens in order. Grid (chunks, B*H), 256 threads; thread (r, c) of
-// a 16 x 16 grid owns the T x T entries rows T r .., columns T c .. (T = D/16).
+// head on the tensor cores. Grid (chunks, B*H), 128 threads. Per 64-token tile the
+// threads write Y^T (feature rows, token columns: the token is the contraction
+// index) into a 128-byte-swizzled K-major shared tile, 2 bytes at a time (lane =
+// token, so a warp's stores fall in 16 distinct banks); the one tile is both
+// operands of four K = 16 steps of tcgen05.mma (M = 128 feature rows, N = D
+// feature columns, fp32 accumulate in TMEM across the whole chunk). Rows D..127 of
+// the tile stay zero when D = 64. Two tiles alternate: a tile is rewritten once
+// the MMAs that read it two tiles earlier have completed. The accumulator goes
+// to part[bh][split] (fp32 D x D).
 template <int D>
-__global__ void __launch_bounds__(256) gram_partial_kernel(const __nv_bfloat16* __restrict__ Y,
-                                                           float* __restrict__ part, int N, int splits, int chunk) {
-  constexpr int T = D / 16;
-  constexpr int kTok = 32;
-  __shared__ __align__(16) float ys[kTok][D];
+struct GramTcCfg {
+  static constexpr int kTok = 64;                      // tokens per tile (one 128-byte row)
+  static constexpr int kTileBytes = 128 * 128;         // 128 feature rows x 64 tokens, bf16
+  static constexpr int kSmemBytes = 2 * kTileBytes + 1024 + 64;
+  static constexpr uint32_t kTmemCols = D;             // N = D fp32 columns
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(128, D, false);
+};
+
+template <int D>
+__global__ void __launch_bounds__(128) gram_tc_kernel(const __nv_bfloat16* __restrict__ Y, float* __restrict__ part,
+                                                      int N, int splits, int chunk) {
+  using Cf = GramTcCfg<D>;
+  constexpr int kOct = D / 8;                          // 16-byte feature groups of a token
+  constexpr int kUnits = 2 * kOct;                     // (32-token half, feature group) pairs per tile
+  extern __shared__ uint8_t gsm_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* done = reinterpret_cast<uint64_t*>(base + 2 * Cf::kTileBytes);   // [2]: MMAs of a tile completed
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(done + 2);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 3);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long bh = blockIdx.y;
   const int s = blockIdx.x;
   const int t0 = s * chunk, t1 = min(N, t0 + chunk);
-  const int ri = (threadIdx.x >> 4) * T, ci = (threadIdx.x & 15) * T;
-  float acc[T][T];
-#pragma unroll
-  for (int i = 0; i < T; ++i)
-#pragma unroll
-    for (int j = 0; j < T; ++j) acc[i][j] = 0.f;
+  const int ntile = t1 > t0 ? (t1 - t0 + Cf::kTok - 1) / Cf::kTok : 0;
+
+  for (int x = threadIdx.x; x < 2 * Cf::kTileBytes / 16; x += 128)
+    reinterpret_cast<uint4*>(base)[x] = make_uint4(0u, 0u, 0u, 0u);
+  if (threadIdx.x == 0) {
+    mbar_init(&done[0], 1);
+    mbar_init(&done[1], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(tmem_holder, Cf::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
   const __nv_bfloat16* src = Y + bh * static_cast<long long>(N) * D;
-  for (int t = t0; t < t1; t += kTok) {
-    const int n = min(kTok, t1 - t);
-    __syncthreads();   // the previous rows are consumed
-    for (int x = threadIdx.x; x < kTok * D / 8; x += 256) {
-      const int r = x / (D / 8), c8 = (x % (D / 8)) * 8;
-      uint4 u = make_uint4(0u, 0u, 0u, 0u);
-      if (r < n) u = __ldg(reinterpret_cast<const uint4*>(src + static_cast<long long>(t + r) * D + c8));
-      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+
+  bool ok = true;
+  for (int j = 0; j < ntile; ++j) {
+    const int buf = j & 1;
+    const int tt = t0 + j * Cf::kTok;
+    // this warp's units: 32 consecutive tokens (one per lane) x 8 features
+    uint4 u[kUnits / 4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(h[e]);
-        ys[r][c8 + 2 * e] = f.x;
-        ys[r][c8 + 2 * e + 1] = f.y;
+    for (int q = 0; q < kUnits / 4; ++q) {
+      const int unit = warp + 4 * q, half = unit / kOct, oct = unit % kOct;
+      const int t = tt + 32 * half + lane;
+      u[q] = t < t1 ? __ldg(reinterpret_cast<const uint4*>(src + static_cast<long long>(t) * D) + oct)
+                    : make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (j >= 2) {   // the MMAs of tile j - 2 (the last readers of this buffer) are done
+      const bool w = mbar_wait(&done[buf], static_cast<uint32_t>((j - 2) >> 1) & 1u, abort_flag);
+      if (!__syncthreads_and(w)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+    }
+    uint8_t* tile = base + buf * Cf::kTileBytes;
+#pragma unroll
+    for (int q = 0; q < kUnits / 4; ++q) {
+      const int unit = warp + 4 * q, half = unit / kOct, oct = unit % kOct;
+      const int kl = 32 * half + lane;                 // token within the tile = K index
+      const uint16_t* h = reinterpret_cast<const uint16_t*>(&u[q]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int row = 8 * oct + e;                   // feature = M (and N) index
+        *reinterpret_cast<uint16_t*>(tile + row * 128 + ((((kl >> 3) ^ (row & 7))) << 4) + (kl & 7) * 2) = h[e];
       }
     }
+    fence_proxy_async_smem();
+    tc_fence_before();
     __syncthreads();
-    for (int r = 0; r < n; ++r) {
-      float a[T], b[T];
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      const uint32_t ta = smem_u32(tile);
 #pragma unroll
-      for (int i = 0; i < T; ++i) {
-        a[i] = ys[r][ri + i];
-        b[i] = ys[r][ci + i];
+      for (int kk = 0; kk < Cf::kTok / 16; ++kk) {
+        const uint64_t d = sdesc_sw128(ta + kk * 32, 16, 1024);
+        tc_mma_ss(tmem_base, d, d, Cf::kIdesc, (j > 0 || kk > 0) ? 1u : 0u);
       }
-#pragma unroll
-      for (int i = 0; i < T; ++i)
-#pragma unroll
-        for (int j = 0; j < T; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+      tc_commit(&done[buf]);
     }
   }
+  // the last commit covers every MMA of the chunk
+  if (ok && ntile > 0) {
+    const int jl = ntile - 1;
+    ok = __syncthreads_and(mbar_wait(&done[jl & 1], static_cast<uint32_t>(jl >> 1) & 1u, abort_flag));
+  }
+  tc_fence_after();
   float* out = part + (bh * splits + s) * static_cast<long long>(D) * D;
+  const int row = warp * 32 + lane;                    // TMEM lane = feature row
 #pragma unroll
-  for (int i = 0; i < T; ++i)
+  for (int c = 0; c < D / 32; ++c) {
+    float v[32];
+    tmem_ld32(tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + c * 32, v);
+    tmem_wait_ld();
+    pin32(v);
+    if (row < D) {
 #pragma unroll
-    for (int j = 0; j < T; ++j) out[(ri + i) * D + ci + j] = acc[i][j];
+      for (int e = 0; e < 32; e += 4) {
+        // a chunk without tokens, or a wait that gave up, contributes zeros
+        const bool use = ok && ntile > 0;
+        *reinterpret_cast<float4*>(out + row * D + c * 32 + e) =
+            make_float4(use ? v[e] : 0.f, use ? v[e + 1] : 0.f, use ? v[e + 2] : 0.f, use ? v[e + 3] : 0.f);
+      }
+    }
+  }
+  if (!ok) atomicOr(&g_dev_error, DEVERR_TIMEOUT);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cf::kTmemCols);
+  }
 }
 
 // G[bh] = sum over the chunks, in chunk order. Grid (D*D/256, B*H), 256 threads.
@@ -160,18 +239,18 @@ __global__ void __launch_bounds__(256) cluster_init_assign_kernel(int* __restric
 // (ceil(C/16), B*H), D threads: thread i forms component i (G is symmetric, so
 // it reads column i of G as row i, and a warp reads G row by row).
 //
-// W16 (bf16 [B*H][C][D + 64]) receives each centroid's tensor-core operand row for
-// the assignment: -2 w_c in columns [0, D), then b_c as the sum of two bf16 values
-// (b_hi = bf16(b_c) in column D, b_lo = bf16(b_c - b_hi) in column D + 1) and zeros.
+// W16 (bf16 [B*H][C][D]) receives each centroid's tensor-core operand row for the
+// assignment, bf16(-2 w_c); bpad ([B*H][Cpad] fp32) receives b_c again, with zeros
+// in the padding columns [C, Cpad).
 template <int D>
 __global__ void __launch_bounds__(D) cluster_prep_kernel(const float* __restrict__ G, const float* __restrict__ cent,
                                                          float* __restrict__ W, float* __restrict__ bvec,
                                                          int* __restrict__ cnt, int C,
-                                                         __nv_bfloat16* __restrict__ W16) {
+                                                         __nv_bfloat16* __restrict__ W16, float* __restrict__ bpad,
+                                                         int Cpad) {
   constexpr int kCl = 16;
   __shared__ float cs[kCl][D];
   __shared__ float red[kCl][D / 32];
-  __shared__ float bsh[kCl];
   const long long bh = blockIdx.y;
   const int c0 = blockIdx.x * kCl;
   const int ncl = min(kCl, C - c0);
@@ -192,7 +271,7 @@ __global__ void __launch_bounds__(D) cluster_prep_kernel(const float* __restrict
   for (int c = 0; c < kCl; ++c) {
     if (c < ncl) {
       W[(bh * C + c0 + c) * D + i] = acc[c];
-      W16[(bh * C + c0 + c) * (D + 64) + i] = __float2bfloat16_rn(-2.f * acc[c]);
+      W16[(bh * C + c0 + c) * D + i] = __float2bfloat16_rn(-2.f * acc[c]);
     }
     float v = cs[c][i] * acc[c];
 #pragma unroll
@@ -205,108 +284,120 @@ __global__ void __launch_bounds__(D) cluster_prep_kernel(const float* __restrict
 #pragma unroll
     for (int w = 0; w < D / 32; ++w) b += red[i][w];
     bvec[bh * C + c0 + i] = b;
-    bsh[i] = b;
+    bpad[bh * Cpad + c0 + i] = b;
     cnt[bh * C + c0 + i] = 0;   // counted again by the assignment
   }
-  __syncthreads();
-  // the bias columns of the operand rows: b_hi, b_lo, then zeros
-  for (int x = i; x < ncl * 64; x += D) {
-    const int c = x >> 6, k = x & 63;
-    const float b = bsh[c];
-    const __nv_bfloat16 hi = __float2bfloat16_rn(b);
-    __nv_bfloat16 v = __float2bfloat16_rn(0.f);
-    if (k == 0) v = hi;
-    if (k == 1) v = __float2bfloat16_rn(b - __bfloat162float(hi));
-    W16[(bh * C + c0 + c) * (D + 64) + D + k] = v;
-  }
+  if (c0 + kCl >= C && C + i < Cpad) bpad[bh * Cpad + C + i] = 0.f;   // the last CTA: the padding
 }
 
 // ----------------------------------------------------------------------------
 // Tensor-core assignment: the four nearest centroids of every token by a bf16
 // product on the tensor cores, then the exact argmin among those four in fp32
-// (cluster_rescore_kernel). One CTA = 128 tokens of one head:
-//   D[token][c] = x . (-2 w_c) + 1 . b_hi_c + 1 . b_lo_c
-// (tcgen05.mma kind::f16, fp32 accumulate in TMEM), over tiles of 128 centroids:
-// D / 16 K-steps of the token tile (TMA'd once) against the centroid tile's bf16
-// rows from cluster_prep_kernel, plus one K-step of a constant tile whose rows
-// start with two ones against the rows' bias columns. Warp 4 (one thread) loads
-// and issues; warps 0-3 (thread = token = TMEM lane) keep each token's four
-// smallest D values with their centroids (ties to the lower centroid) in
-// registers. Two TMEM buffers of 128 columns and three centroid-tile stages keep
-// the tensor cores and the epilogue overlapped.
-// The bf16 product moves the argmin for a fraction of a percent of the tokens;
-// the four best of the product contain the fp32 argmin (measured on the
-// workloads' inputs), and the re-score restores it exactly.
+// (cluster_rescore_kernel). One CTA = 256 tokens of one head, two halves of 128
+// (the M = 128 of tcgen05.mma); per tile of 64 centroids
+//   D_h[token][c] = x . (-2 w_c)      (kind::f16, fp32 accumulate in TMEM)
+// with the tokens as the A operand in TMEM (written once from registers, so the
+// MMAs read only the centroid tile from shared memory) and the centroid tile's
+// bf16 rows from cluster_prep_kernel as B (TMA, one 4-D box per tile, six
+// stages). Both halves use each centroid tile, so a tile crosses L2 once per 256
+// tokens. Warp 16 (one thread) loads and issues. Warps 0-15 are the epilogue:
+// warp w reads TMEM lanes 32 (w % 4) .. (its 32 tokens) of half (w / 4) % 2 and
+// the 32 columns of column half w / 8 of each tile, adds b_c in fp32 and keeps
+// each token's four smallest values with their centroids in registers; the two
+// column halves merge at the end. A lane marks the values below its token's
+// current fourth best in a bit mask, parks the 32 values in its own shared-memory
+// row, and offers only the marked ones, so a warp pays for its busiest lane's
+// entries (after the first tile a few at most) rather than for every value that
+// any lane needs. Two TMEM buffers per half keep
+// the tensor cores and the epilogue overlapped; a CTA visits the centroid tiles
+// starting from the one that holds its tokens' first clusters (visit_tile), so
+// the four best settle in the first tile. The bf16 product moves the argmin for
+// a fraction of a percent of the tokens; the four best of the product contain
+// the fp32 argmin (measured on the workloads' inputs), and the re-score restores
+// it exactly.
 template <int D>
 struct ClusterTcCfg {
   static constexpr int kCh = D / 64;                   // 128-byte column chunks of a row
-  static constexpr int kTile = 128;                    // tokens per CTA, centroids per tile
-  static constexpr int kChunkBytes = kTile * 128;      // 16 KB: one column chunk of a tile
-  static constexpr int kStages = 3;
-  static constexpr int kWStage = (kCh + 1) * kChunkBytes;   // centroid rows + bias chunk
-  static constexpr int oX = 0;
-  static constexpr int oOnes = oX + kCh * kChunkBytes;
-  static constexpr int oW = oOnes + kChunkBytes;
-  static constexpr int oBar = oW + kStages * kWStage;
-  static constexpr int kSmemBytes = oBar + 128 + 1024;
-  static constexpr uint32_t kTmemCols = 256;
-  static constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128, false);
+  static constexpr int kTok = 256;                     // tokens per CTA: two halves of 128
+  static constexpr int kCt = 64;                       // centroids per tile (N of the MMA)
+  static constexpr int kChunkBytes = kCt * 128;        // 8 KB: one column chunk of a tile
+  static constexpr int kWStage = kCh * kChunkBytes;
+  static constexpr int kStages = 6;
+  static constexpr int kEpiWarps = 16;                 // 4 lane quadrants x 2 halves x 2 column halves
+  static constexpr int kThreads = (kEpiWarps + 1) * 32;  // + the issuing warp
+  static constexpr int oW = 0;
+  static constexpr int oMerge = oW + kStages * kWStage;     // [2 halves][128 tokens][4 values, 4 centroids]
+  static constexpr int kParkStride = 36;               // floats per lane row (144 B: 16-byte stores conflict-free)
+  static constexpr int oPark = oMerge + 2 * 128 * 8 * 4;    // [16 warps][32 lanes][36] fp32
+  static constexpr int oBar = oPark + kEpiWarps * 32 * kParkStride * 4;
+  static constexpr int kSmemBytes = oBar + 256 + 1024;
+  // TMEM columns: accumulator (buffer b, half h) at 64 (2 b + h); the tokens of
+  // half h (bf16 pairs, D / 2 columns) at kColX + (D / 2) h
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColX = 256;
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(128, kCt, false);
 };
 
-// A token's four smallest scores so far, ascending, with their centroids (the
-// epilogue's state, touched only when a score may enter).
+// A token's four smallest values so far, ascending, with their centroids.
 struct Top4 {
-  float b[4];
-  int i[4];
-};
-
-// Offers the scores x[e] of centroids c0 + e (e < lim) in ascending centroid order;
-// a score enters if it is smaller than the fourth best (so a tie keeps the earlier
-// centroid). Returns the new fourth best. Not inlined: the insertion code then
-// exists once, and the epilogue's hot path stays small.
-static __device__ __noinline__ float top4_offer8(Top4* st, float x0, float x1, float x2, float x3, float x4,
-                                                 float x5, float x6, float x7, int c0, int lim) {
-  const float xs[8] = {x0, x1, x2, x3, x4, x5, x6, x7};
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const float x = xs[e];
-    if (e < lim && x < st->b[3]) {
-      int p = 3;
-      while (p > 0 && x < st->b[p - 1]) {
-        st->b[p] = st->b[p - 1];
-        st->i[p] = st->i[p - 1];
-        --p;
-      }
-      st->b[p] = x;
-      st->i[p] = c0 + e;
+  float b0, b1, b2, b3;
+  int i0, i1, i2, i3;
+  __device__ __forceinline__ void init() {
+    b0 = b1 = b2 = b3 = INFINITY;
+    i0 = i1 = i2 = i3 = 0x7fffffff;
+  }
+  // x enters if it is smaller than the fourth best; it goes after the values it
+  // equals. Every new entry is a select of the old ones (no data-dependent
+  // branches beyond the entry test), so the state stays in registers.
+  __device__ __forceinline__ void offer(float x, int c) {
+    if (x < b3) {
+      const bool l2 = x < b2, l1 = x < b1, l0 = x < b0;
+      b3 = l2 ? b2 : x;
+      i3 = l2 ? i2 : c;
+      b2 = l1 ? b1 : (l2 ? x : b2);
+      i2 = l1 ? i1 : (l2 ? c : i2);
+      b1 = l0 ? b0 : (l1 ? x : b1);
+      i1 = l0 ? i0 : (l1 ? c : i1);
+      b0 = l0 ? x : b0;
+      i0 = l0 ? c : i0;
     }
   }
-  return st->b[3];
+};
+
+// The k-th centroid tile a CTA visits: its own tile tt0 first (the clusters its
+// tokens started in), then alternately the next one up and the next one down
+// (odd k up, even k down) while both sides last, then the rest of the longer
+// side, so a token's nearest clusters come early and the four best settle at once.
+static __device__ __forceinline__ int visit_tile(int k, int tt0, int nt) {
+  const int up = nt - 1 - tt0, m = min(up, tt0);
+  if (k <= 2 * m) return (k & 1) ? tt0 + (k + 1) / 2 : tt0 - k / 2;
+  return up > tt0 ? tt0 + k - m : tt0 - (k - m);
 }
 
 template <int D>
-__global__ void __launch_bounds__(160, 1)
-    cluster_assign_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                             int N, int C, int* __restrict__ cand) {
+__global__ void __launch_bounds__(ClusterTcCfg<D>::kThreads, 1)
+    cluster_assign_tc_kernel(const __nv_bfloat16* __restrict__ X, const __grid_constant__ CUtensorMap tmW,
+                             const float* __restrict__ bpad, int N, int C, int Cpad, int* __restrict__ cand) {
   using Cf = ClusterTcCfg<D>;
   extern __shared__ uint8_t tsm_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tsm_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sX = base + Cf::oX;
-  uint8_t* sOnes = base + Cf::oOnes;
   uint8_t* sW = base + Cf::oW;
+  float* sMerge = reinterpret_cast<float*>(base + Cf::oMerge);
+  float* sPark = reinterpret_cast<float*>(base + Cf::oPark);
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + Cf::oBar);
-  uint64_t* wfull = bars;                      // [3]
-  uint64_t* wempty = bars + 3;                 // [3]
-  uint64_t* dfull = bars + 6;                  // [2]
-  uint64_t* dempty = bars + 8;                 // [2], 4 arrivals
-  uint64_t* xfull = bars + 10;
-  uint64_t* drain = bars + 11;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 12);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* wfull = bars;                      // [6]
+  uint64_t* wempty = bars + 6;                 // [6]
+  uint64_t* dfull = bars + 12;                 // [2]
+  uint64_t* dempty = bars + 14;                // [2], one arrival per epilogue warp
+  uint64_t* drain = bars + 16;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 17);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 18);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long bh = blockIdx.y;
-  const int t0 = blockIdx.x * Cf::kTile;
-  const int ntiles = (C + Cf::kTile - 1) / Cf::kTile;
+  const int t0 = blockIdx.x * Cf::kTok;
+  const int ntiles = (C + Cf::kCt - 1) / Cf::kCt;
+  // the centroid tile holding the first cluster of this CTA's tokens (64 per cluster)
+  const int tt0 = min(ntiles - 1, t0 / (kBlock * Cf::kCt));
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < Cf::kStages; ++s) {
@@ -315,152 +406,201 @@ __global__ void __launch_bounds__(160, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&dfull[b], 1);
-      mbar_init(&dempty[b], 4);
+      mbar_init(&dempty[b], Cf::kEpiWarps);
     }
-    mbar_init(xfull, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  // the constant tile: row r holds ones in columns 0 and 1 (16-byte chunk 0 of the
-  // row, which the 128-byte swizzle stores at chunk (r & 7)), zeros elsewhere
-  for (int x = threadIdx.x; x < Cf::kChunkBytes / 16; x += blockDim.x)
-    reinterpret_cast<uint4*>(sOnes)[x] = make_uint4(0u, 0u, 0u, 0u);
-  __syncthreads();
-  if (threadIdx.x < Cf::kTile) {
-    const int r = threadIdx.x;
-    const uint32_t one2 = 0x3F803F80u;         // two bf16 ones
-    *reinterpret_cast<uint32_t*>(sOnes + r * 128 + (r & 7) * 16) = one2;
-  }
-  fence_proxy_async_smem();                    // generic-proxy writes -> the tensor cores' reads
-  if (warp == 4) tmem_alloc(tmem_holder, Cf::kTmemCols);
+  if (warp == Cf::kEpiWarps) tmem_alloc(tmem_holder, Cf::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // the tokens into TMEM: warp w < 8 writes lanes 32 (w % 4) .. of half w / 4, one
+  // token per lane, its bf16 row as D / 2 packed columns (zeros past N)
+  if (warp < 8) {
+    const int quad = warp & 3, h = warp >> 2;
+    const int tok = t0 + 128 * h + 32 * quad + lane;
+    const uint4* src = reinterpret_cast<const uint4*>(X + (bh * N + min(tok, N - 1)) * static_cast<long long>(D));
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      uint32_t r[32];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint4 u = tok < N ? __ldg(src + 8 * c + q) : make_uint4(0u, 0u, 0u, 0u);
+        r[4 * q] = u.x;
+        r[4 * q + 1] = u.y;
+        r[4 * q + 2] = u.z;
+        r[4 * q + 3] = u.w;
+      }
+      tmem_st32u(tmem_base + (static_cast<uint32_t>(32 * quad) << 16) + Cf::kColX + (D / 2) * h + 32 * c, r);
+    }
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
 
-  if (warp == 4) {
+  if (warp == Cf::kEpiWarps) {
     // ------------------------------------------------------------ loads and MMAs
     if (lane == 0) {
-      tma_prefetch_desc(&tmX);
       tma_prefetch_desc(&tmW);
-      mbar_expect_tx(xfull, Cf::kCh * Cf::kChunkBytes);
-      for (int c = 0; c < Cf::kCh; ++c)
-        tma_load_3d(sX + c * Cf::kChunkBytes, &tmX, c * 64, t0, static_cast<int>(bh), xfull);
-      auto load_w = [&](int t) {
+      auto load_w = [&](int t) {           // the t-th visited tile into stage t % kStages
         const int s = t % Cf::kStages;
         mbar_expect_tx(&wfull[s], Cf::kWStage);
-        for (int c = 0; c <= Cf::kCh; ++c)
-          tma_load_3d(sW + s * Cf::kWStage + c * Cf::kChunkBytes, &tmW, c * 64, t * Cf::kTile,
-                      static_cast<int>(bh), &wfull[s]);
+        tma_load_4d(sW + s * Cf::kWStage, &tmW, 0, visit_tile(t, tt0, ntiles) * Cf::kCt, 0, static_cast<int>(bh),
+                    &wfull[s]);
       };
       int nw = 0;
       for (; nw < Cf::kStages && nw < ntiles; ++nw) load_w(nw);
-      const uint32_t xa = smem_u32(sX), oa = smem_u32(sOnes), wa = smem_u32(sW);
-      bool ok = mbar_wait(xfull, 0u, abort_flag);
-      for (int t = 0; ok && t < ntiles; ++t) {
+      const uint32_t wa = smem_u32(sW);
+      for (int t = 0; t < ntiles; ++t) {
         const int s = t % Cf::kStages, buf = t & 1;
         if (!mbar_wait(&wfull[s], static_cast<uint32_t>(t / Cf::kStages) & 1u, abort_flag)) break;
         if (t >= 2 && !mbar_wait(&dempty[buf], static_cast<uint32_t>((t >> 1) - 1) & 1u, abort_flag)) break;
         tc_fence_after();
-        const uint32_t dD = tmem_base + buf * 128;
         const uint32_t wb = wa + s * Cf::kWStage;
+        // the two halves' K-steps alternate: consecutive MMAs write different
+        // accumulators, so an issue never waits on the previous one's result
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * Cf::kChunkBytes + (kk & 3) * 32;
-          tc_mma_ss(dD, sdesc_sw128(xa + off, 16, 1024), sdesc_sw128(wb + off, 16, 1024), Cf::kIdesc,
-                    kk > 0 ? 1u : 0u);
+          const uint64_t bd = sdesc_sw128(wb + (kk >> 2) * Cf::kChunkBytes + (kk & 3) * 32, 16, 1024);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            tc_mma_ts(tmem_base + Cf::kCt * (2 * buf + h), tmem_base + Cf::kColX + (D / 2) * h + kk * 8, bd,
+                      Cf::kIdesc, kk > 0 ? 1u : 0u);
         }
-        // the bias: the ones tile's first K-step against the rows' bias columns
-        tc_mma_ss(dD, sdesc_sw128(oa, 16, 1024), sdesc_sw128(wb + Cf::kCh * Cf::kChunkBytes, 16, 1024), Cf::kIdesc,
-                  1u);
         tc_commit(&dfull[buf]);
         tc_commit(&wempty[s]);
-        if (t + Cf::kStages < ntiles) {
-          if (!mbar_wait(&wempty[s], static_cast<uint32_t>(t / Cf::kStages) & 1u, abort_flag)) break;
-          load_w(t + Cf::kStages);
+        // refill the stage of the previous tile (its MMAs are older than the ones
+        // just issued, so the tensor pipe stays fed while this thread waits)
+        const int r = t - 1 + Cf::kStages;
+        if (t >= 1 && r < ntiles) {
+          const int sp = (t - 1) % Cf::kStages;
+          if (!mbar_wait(&wempty[sp], static_cast<uint32_t>((t - 1) / Cf::kStages) & 1u, abort_flag)) break;
+          load_w(r);
           ++nw;
         }
       }
       tc_commit(drain);
       mbar_wait_drain(drain, 0u);
-      mbar_wait_drain(xfull, 0u);
       for (int k = max(0, nw - Cf::kStages); k < nw; ++k)
         mbar_wait_drain(&wfull[k % Cf::kStages], static_cast<uint32_t>(k / Cf::kStages) & 1u);
     }
   } else {
     // ------------------------------------------------------------ epilogue: the four best
-    const int row = warp * 32 + lane;          // token of the tile == TMEM lane
-    const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
+    const int quad = warp & 3, h = (warp >> 2) & 1, cq = warp >> 3;
+    const int row = quad * 32 + lane;          // token of the half == TMEM lane
+    const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
+    const float* bhead = bpad + bh * Cpad;
+    float* park = sPark + (warp * 32 + lane) * Cf::kParkStride;
     Top4 st;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      st.b[q] = INFINITY;
-      st.i[q] = 0x7fffffff;
-    }
-    float b3 = INFINITY;                       // st.b[3], in a register for the hot path
+    st.init();
     bool alive = true;
     for (int t = 0; t < ntiles; ++t) {
       const int buf = t & 1;
+      const int c0 = visit_tile(t, tt0, ntiles) * Cf::kCt + cq * 32;
+      const int ncol = C - c0;                 // < 32 in the last tile: columns past C read zero rows
+      float bb[32];                            // b_c of the 32 columns (padded, so in bounds)
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 f = __ldg(reinterpret_cast<const float4*>(bhead + c0) + q);
+        bb[4 * q] = f.x;
+        bb[4 * q + 1] = f.y;
+        bb[4 * q + 2] = f.z;
+        bb[4 * q + 3] = f.w;
+      }
       if (!warp_wait(&dfull[buf], static_cast<uint32_t>(t >> 1) & 1u, abort_flag)) {
         alive = false;
         break;
       }
       tc_fence_after();
-      float v[128];
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        tmem_ld32(tmem_base + lane_bits + buf * 128 + q * 32, *reinterpret_cast<float(*)[32]>(&v[32 * q]));
+      float v[32];
+      tmem_ld32(tmem_base + lane_bits + Cf::kCt * (2 * buf + h) + cq * 32, v);
       tmem_wait_ld();
-#pragma unroll
-      for (int q = 0; q < 4; ++q) pin32(*reinterpret_cast<float(*)[32]>(&v[32 * q]));
+      pin32(v);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&dempty[buf]);   // the buffer may take tile t + 2
-      const int c0 = t * Cf::kTile;
-      const int ncol = min(Cf::kTile, C - c0);
-      const bool partial = ncol < Cf::kTile;   // the last tile: columns past C read zero rows
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float* w = v + 32 * q;
-        float m8[4];
+      for (int e = 0; e < 32; e += 2) f2unpack(fadd2(f2pack(v[e], v[e + 1]), f2pack(bb[e], bb[e + 1])), v[e], v[e + 1]);
+      if (ncol < 32) {
 #pragma unroll
-        for (int g = 0; g < 4; ++g)
-          m8[g] = fminf(fminf(fminf(w[8 * g], w[8 * g + 1]), fminf(w[8 * g + 2], w[8 * g + 3])),
-                        fminf(fminf(w[8 * g + 4], w[8 * g + 5]), fminf(w[8 * g + 6], w[8 * g + 7])));
-        if (partial || fminf(fminf(m8[0], m8[1]), fminf(m8[2], m8[3])) < b3) {
+        for (int e = 0; e < 32; ++e)
+          if (e >= ncol) v[e] = INFINITY;
+      }
+      // 8-column groups whose minimum is below the fourth best, then their values
+      uint32_t gm = 0;
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int cb = 32 * q + 8 * g;
-            if (cb < ncol && (partial || m8[g] < b3))
-              b3 = top4_offer8(&st, w[8 * g], w[8 * g + 1], w[8 * g + 2], w[8 * g + 3], w[8 * g + 4],
-                               w[8 * g + 5], w[8 * g + 6], w[8 * g + 7], c0 + cb, ncol - cb);
+      for (int g = 0; g < 4; ++g) {
+        const float* w = v + 8 * g;
+        const float m = fmin3(fmin3(w[0], w[1], w[2]), fmin3(w[3], w[4], w[5]), fminf(w[6], w[7]));
+        gm |= (m < st.b3 ? 1u : 0u) << g;
+      }
+      if (__any_sync(0xffffffffu, gm != 0u)) {
+        uint32_t pend = 0;                     // the values that may enter
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          if (gm & (1u << g)) {
+            const float* w = v + 8 * g;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) pend |= (w[e] < st.b3 ? 1u : 0u) << (8 * g + e);
+            reinterpret_cast<float4*>(park)[2 * g] = make_float4(w[0], w[1], w[2], w[3]);
+            reinterpret_cast<float4*>(park)[2 * g + 1] = make_float4(w[4], w[5], w[6], w[7]);
           }
+        }
+        while (pend) {                         // this lane's own row: no exchange between lanes
+          const int e = __ffs(pend) - 1;
+          pend &= pend - 1;
+          st.offer(park[e], c0 + e);
         }
       }
     }
-    const int tok = t0 + row;
-    if (alive && tok < N) {
-      int4 o;
-      o.x = st.i[0];
-      o.y = st.i[1];
-      o.z = st.i[2];
-      o.w = st.i[3];
-      *reinterpret_cast<int4*>(cand + (bh * N + tok) * 4) = o;
+    // the column halves of a token merge: half 1 hands its four to half 0
+    if (cq == 1) {
+      float* m = sMerge + (h * 128 + row) * 8;
+      m[0] = st.b0;
+      m[1] = st.b1;
+      m[2] = st.b2;
+      m[3] = st.b3;
+      m[4] = __int_as_float(st.i0);
+      m[5] = __int_as_float(st.i1);
+      m[6] = __int_as_float(st.i2);
+      m[7] = __int_as_float(st.i3);
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(Cf::kEpiWarps * 32) : "memory");   // the epilogue warps
+    const int tok = t0 + 128 * h + row;
+    if (cq == 0 && tok < N) {
+      const float* m = sMerge + (h * 128 + row) * 8;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) st.offer(m[q], __float_as_int(m[4 + q]));
+      // a wait that gave up anywhere leaves this token's candidates unwritten
+      if (alive && !*abort_flag) {
+        int4 o;
+        o.x = st.i0;
+        o.y = st.i1;
+        o.z = st.i2;
+        o.w = st.i3;
+        *reinterpret_cast<int4*>(cand + (bh * N + tok) * 4) = o;
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == Cf::kEpiWarps) {
     tc_fence_after();
     tmem_dealloc(tmem_base, Cf::kTmemCols);
   }
 }
 
 // The exact argmin among a token's four candidates: b_c - 2 x . w_c in fp32
-// (x the bf16 token, w_c and b_c from cluster_prep_kernel), ties to the lowest c;
-// the winner is counted into its cluster's size. A candidate outside [0, C) (a
-// head with fewer than four clusters) is skipped. One thread per token.
+// (x the bf16 token, w_c and b_c from cluster_prep_kernel), ties to the lowest
+// c; the winner is counted into its cluster's size. A candidate outside [0, C)
+// (a head with fewer than four clusters) is skipped. A warp per token: lane l
+// holds components [D/32 l, D/32 (l+1)) of x and of the four rows (coalesced
+// loads, all issued before the arithmetic), and the four partial dot products are
+// summed across the warp. Grid (ceil(N / 64), B*H), 256 threads, 8 tokens per warp.
 template <int D>
 __global__ void __launch_bounds__(256) cluster_rescore_kernel(const __nv_bfloat16* __restrict__ X,
                                                               const float* __restrict__ W,
@@ -468,54 +608,73 @@ __global__ void __launch_bounds__(256) cluster_rescore_kernel(const __nv_bfloat1
                                                               const int* __restrict__ cand,
                                                               int* __restrict__ assign, int* __restrict__ cnt, int N,
                                                               int C) {
+  constexpr int E = D / 32;                    // components per lane: 4 or 2
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long bh = blockIdx.y;
-  const int tok = blockIdx.x * 256 + threadIdx.x;
-  if (tok >= N) return;
-  float x[D];
-  const uint4* src = reinterpret_cast<const uint4*>(X + (bh * N + tok) * static_cast<long long>(D));
+  for (int k = 0; k < 8; ++k) {
+    const int tok = blockIdx.x * 64 + warp * 8 + k;
+    if (tok >= N) return;
+    const long long r = bh * N + tok;
+    const int4 cd = *reinterpret_cast<const int4*>(cand + r * 4);
+    const int cs[4] = {cd.x, cd.y, cd.z, cd.w};
+    float x[E];
+    if constexpr (E == 4) {
+      const uint2 u = __ldg(reinterpret_cast<const uint2*>(X + r * D) + lane);
+      x[0] = __uint_as_float(u.x << 16);
+      x[1] = __uint_as_float(u.x & 0xffff0000u);
+      x[2] = __uint_as_float(u.y << 16);
+      x[3] = __uint_as_float(u.y & 0xffff0000u);
+    } else {
+      const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(X + r * D) + lane);
+      x[0] = __uint_as_float(u << 16);
+      x[1] = __uint_as_float(u & 0xffff0000u);
+    }
+    float wv[4][E];
+    float bq[4];
 #pragma unroll
-  for (int q = 0; q < D / 8; ++q) {
-    const uint4 u = __ldg(src + q);
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+    for (int q = 0; q < 4; ++q) {
+      const bool ok = cs[q] >= 0 && cs[q] < C;
+      const long long row = bh * C + (ok ? cs[q] : 0);
+      if constexpr (E == 4) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(W + row * D) + lane);
+        wv[q][0] = v.x;
+        wv[q][1] = v.y;
+        wv[q][2] = v.z;
+        wv[q][3] = v.w;
+      } else {
+        const float2 v = __ldg(reinterpret_cast<const float2*>(W + row * D) + lane);
+        wv[q][0] = v.x;
+        wv[q][1] = v.y;
+      }
+      bq[q] = __ldg(bvec + row);
+    }
+    float best = INFINITY;
+    int bi = 0x7fffffff;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = __bfloat1622float2(h[e]);
-      x[8 * q + 2 * e] = f.x;
-      x[8 * q + 2 * e + 1] = f.y;
+    for (int q = 0; q < 4; ++q) {
+      float dot = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) dot = fmaf(x[e], wv[q][e], dot);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      const float sc = bq[q] - 2.f * dot;
+      const int c = cs[q];
+      if (c >= 0 && c < C && (sc < best || (sc == best && c < bi))) {
+        best = sc;
+        bi = c;
+      }
+    }
+    // a NaN score never compares smaller: a token whose every candidate scores NaN
+    // keeps no cluster, which the range check turns into cluster 0 and an error bit
+    if (lane == 0) {
+      if (bi < 0 || bi >= C) {
+        atomicOr(&g_dev_error, DEVERR_VALUE);
+        bi = 0;
+      }
+      assign[r] = bi;
+      atomicAdd(&cnt[bh * C + bi], 1);
     }
   }
-  const int4 cd = *reinterpret_cast<const int4*>(cand + (bh * N + tok) * 4);
-  const int cs[4] = {cd.x, cd.y, cd.z, cd.w};
-  float best = INFINITY;
-  int bi = 0x7fffffff;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int c = cs[q];
-    if (c < 0 || c >= C) continue;
-    const float4* w = reinterpret_cast<const float4*>(W + (bh * C + c) * static_cast<long long>(D));
-    float dot = 0.f;
-#pragma unroll
-    for (int k = 0; k < D / 4; ++k) {
-      const float4 wv = __ldg(w + k);
-      dot = fmaf(x[4 * k], wv.x, dot);
-      dot = fmaf(x[4 * k + 1], wv.y, dot);
-      dot = fmaf(x[4 * k + 2], wv.z, dot);
-      dot = fmaf(x[4 * k + 3], wv.w, dot);
-    }
-    const float sc = bvec[bh * C + c] - 2.f * dot;
-    if (sc < best || (sc == best && c < bi)) {
-      best = sc;
-      bi = c;
-    }
-  }
-  // a NaN score never compares smaller: a token whose every candidate scores NaN
-  // keeps no cluster, which the range check turns into cluster 0 and an error bit
-  if (bi < 0 || bi >= C) {
-    atomicOr(&g_dev_error, DEVERR_VALUE);
-    bi = 0;
-  }
-  assign[bh * N + tok] = bi;
-  atomicAdd(&cnt[bh * C + bi], 1);
 }
 
 // Clusters per CTA of cluster_order_kernel.
@@ -664,26 +823,38 @@ __global__ void __launch_bounds__(1024) cluster_offsets_kernel(const int* __rest
 
 // Row moves of [B,H,N,D] bf16 tensors by a per-head permutation: gather
 // dst[bh, p] = src[bh, perm[bh, p]], or (inverse) scatter dst[bh, perm[bh, p]] =
-// src[bh, p]. One thread per 16 bytes. A perm entry outside [0, N) moves
-// nothing and sets the range bit of the device error word.
+// src[bh, p]. Grid (ceil(N * D / 8 / 1024), B*H), four 16-byte vectors per
+// thread (the index within a head fits 32 bits). A perm entry outside [0, N) moves nothing
+// and sets the range bit of the device error word.
 template <int D>
 __global__ void __launch_bounds__(256) permute_rows_kernel(const __nv_bfloat16* __restrict__ src,
                                                            const int* __restrict__ perm, __nv_bfloat16* __restrict__ dst,
-                                                           int N, long long rows, int inverse) {
+                                                           int N, int inverse) {
   constexpr int V = D / 8;   // 16-byte vectors per row
-  const long long x = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
-  if (x >= rows * V) return;
-  const long long r = x / V;
-  const int v = static_cast<int>(x - r * V);
-  const long long bh = r / N;
-  const int p = perm[r];
-  if (p < 0 || p >= N) {
-    if (v == 0) atomicOr(&g_dev_error, DEVERR_RANGE);
-    return;
+  constexpr int kU = 4;      // vectors per thread, 256 apart: all loads issue before the stores
+  const long long bh = blockIdx.y;
+  const int base = blockIdx.x * 256 * kU + threadIdx.x;
+  uint4 val[kU];
+  long long to[kU];
+#pragma unroll
+  for (int u = 0; u < kU; ++u) {
+    const int x = base + u * 256;
+    to[u] = -1;
+    if (x < N * V) {
+      const int r = x / V, v = x % V;
+      const int p = __ldg(perm + bh * N + r);
+      if (p < 0 || p >= N) {
+        if (v == 0) atomicOr(&g_dev_error, DEVERR_RANGE);
+      } else {
+        const long long from = bh * N + (inverse ? r : p);
+        to[u] = (bh * N + (inverse ? p : r)) * V + v;
+        val[u] = __ldg(reinterpret_cast<const uint4*>(src + from * D) + v);
+      }
+    }
   }
-  const long long other = bh * N + p;
-  const long long from = inverse ? r : other, to = inverse ? other : r;
-  reinterpret_cast<uint4*>(dst + to * D)[v] = __ldg(reinterpret_cast<const uint4*>(src + from * D) + v);
+#pragma unroll
+  for (int u = 0; u < kU; ++u)
+    if (to[u] >= 0) reinterpret_cast<uint4*>(dst)[to[u]] = val[u];
 }
 
 }  // namespace sa

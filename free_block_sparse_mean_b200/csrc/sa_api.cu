@@ -131,16 +131,18 @@ sa_status launch_fwd(const sa_shape& s, const void* Q, const void* K, const void
   return SA_OK;
 }
 
-// The centroids' bf16 operand rows [B*H][C][D + 64] as a 3-D tensor {D + 64, C,
-// B*H}; box {64, 128 rows, 1}, 128B swizzle. Rows past C read as zero.
+// The centroids' bf16 operand rows [B*H][C][D] as a 4-D tensor {64 elements, C
+// rows, D/64 chunks, B*H} (row stride 2D bytes, chunk stride 128 bytes): one box
+// {64, 64, D/64, 1} is a 64-centroid tile, landing as [chunk][row][128 B] with the
+// 128B swizzle. Rows past C read as zero.
 bool make_w16_map(CUtensorMap* map, const void* ptr, long long BH, int C, int D) {
   auto enc = get_encode();
   if (!enc) return false;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D + 64), static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D + 64) * 2, static_cast<cuuint64_t>(C) * (D + 64) * 2};
-  cuuint32_t box[3] = {64u, 128u, 1u};
-  cuuint32_t estr[3] = {1u, 1u, 1u};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+  cuuint64_t dims[4] = {64u, static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(D / 64), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, 128u, static_cast<cuuint64_t>(C) * D * 2};
+  cuuint32_t box[4] = {64u, 64u, static_cast<cuuint32_t>(D / 64), 1u};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -165,10 +167,12 @@ sa_status launch_cluster(const sa_shape& s, const void* X, const void* Y, int it
   int* assign = assign_out ? assign_out : reinterpret_cast<int*>(wsb + L.assign);
   auto* w16 = reinterpret_cast<__nv_bfloat16*>(wsb + L.w16);
   int* cand = reinterpret_cast<int*>(wsb + L.cand);
+  float* bpad = reinterpret_cast<float*>(wsb + L.bpad);
   const auto* x = static_cast<const __nv_bfloat16*>(X);
   const auto* y = static_cast<const __nv_bfloat16*>(Y);
   const unsigned by = static_cast<unsigned>(BH);
-  sa::gram_partial_kernel<D><<<dim3(L.splits, by), 256, 0, st>>>(y, gpart, N, L.splits, L.chunk);
+  if (sa::set_smem(sa::gram_tc_kernel<D>, sa::GramTcCfg<D>::kSmemBytes) != SA_OK) return SA_ERR_CUDA;
+  sa::gram_tc_kernel<D><<<dim3(L.splits, by), 128, sa::GramTcCfg<D>::kSmemBytes, st>>>(y, gpart, N, L.splits, L.chunk);
   sa::gram_reduce_kernel<D><<<dim3(D * D / 256, by), 256, 0, st>>>(gpart, G, L.splits);
   // the block means (the pooling kernel, queries half only) and every token in its block
   sa::pool_kernel<D><<<dim3(static_cast<unsigned>(BH * C), 1), 256, 0, st>>>(x, x, cent, nullptr, N, C);
@@ -178,17 +182,20 @@ sa_status launch_cluster(const sa_shape& s, const void* X, const void* Y, int it
   if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   using TC = sa::ClusterTcCfg<D>;
   if (sa::set_smem(sa::cluster_assign_tc_kernel<D>, TC::kSmemBytes) != SA_OK) return SA_ERR_CUDA;
-  CUtensorMap mx, mw;
-  if (iters > 0 && (!make_map(&mx, X, s, 128) || !make_w16_map(&mw, w16, BH, C, D))) return SA_ERR_CUDA;
+  CUtensorMap mw;
+  if (iters > 0 && !make_w16_map(&mw, w16, BH, C, D)) return SA_ERR_CUDA;
   const dim3 order_grid((C + sa::kOrderClusters - 1) / sa::kOrderClusters, by);
   const dim3 cent_grid((C + 7) / 8, by);
   for (int it = 0; it < iters; ++it) {
-    sa::cluster_prep_kernel<D><<<dim3((C + 15) / 16, by), D, 0, st>>>(G, cent, W, bvec, cnt, C, w16);
-    sa::cluster_assign_tc_kernel<D><<<dim3((N + 127) / 128, by), 160, TC::kSmemBytes, st>>>(mx, mw, N, C, cand);
-    sa::cluster_rescore_kernel<D><<<dim3((N + 255) / 256, by), 256, 0, st>>>(x, W, bvec, cand, assign, cnt, N, C);
+    sa::cluster_prep_kernel<D><<<dim3((C + 15) / 16, by), D, 0, st>>>(G, cent, W, bvec, cnt, C, w16, bpad, L.Cpad);
+    sa::cluster_assign_tc_kernel<D><<<dim3((N + TC::kTok - 1) / TC::kTok, by), TC::kThreads, TC::kSmemBytes, st>>>(
+        x, mw, bpad, N, C, L.Cpad, cand);
+    sa::cluster_rescore_kernel<D><<<dim3((N + 63) / 64, by), 256, 0, st>>>(x, W, bvec, cand, assign, cnt, N, C);
     sa::cluster_offsets_kernel<<<by, 1024, 0, st>>>(cnt, off, C);
     sa::cluster_order_kernel<<<order_grid, 256, 0, st>>>(assign, off, perm, N, C);
-    sa::cluster_centroid_kernel<D><<<cent_grid, 256, 0, st>>>(x, perm, off, cnt, cent, N, C);
+    // the means of the new clusters: the next iteration's centroids, or the output
+    if (it + 1 < iters || cent_out)
+      sa::cluster_centroid_kernel<D><<<cent_grid, 256, 0, st>>>(x, perm, off, cnt, cent, N, C);
     if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   }
   if (iters == 0) {   // the plain blocks: identity order, block means from the pooling kernel
@@ -533,16 +540,15 @@ sa_status sparse_attn_permute_rows(const void* src, const int32_t* perm, sa_shap
   if (sh != SA_OK) return sh;
   if (!aligned16(src) || !aligned16(dst) || (reinterpret_cast<uintptr_t>(perm) & 3u) != 0)
     return SA_ERR_INVALID_ARG;
-  const long long rows = static_cast<long long>(s.B) * s.H * s.N;
-  const long long threads = rows * (s.d / 8);
-  const unsigned grid = static_cast<unsigned>((threads + 255) / 256);
+  const dim3 grid(static_cast<unsigned>((static_cast<long long>(s.N) * (s.d / 8) + 1023) / 1024),
+                  static_cast<unsigned>(static_cast<long long>(s.B) * s.H));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const auto* x = static_cast<const __nv_bfloat16*>(src);
   auto* y = static_cast<__nv_bfloat16*>(dst);
   if (s.d == 64)
-    sa::permute_rows_kernel<64><<<grid, 256, 0, st>>>(x, perm, y, s.N, rows, inverse != 0);
+    sa::permute_rows_kernel<64><<<grid, 256, 0, st>>>(x, perm, y, s.N, inverse != 0);
   else
-    sa::permute_rows_kernel<128><<<grid, 256, 0, st>>>(x, perm, y, s.N, rows, inverse != 0);
+    sa::permute_rows_kernel<128><<<grid, 256, 0, st>>>(x, perm, y, s.N, inverse != 0);
   if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   return SA_OK;
 }
