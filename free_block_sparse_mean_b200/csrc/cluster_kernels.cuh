@@ -48,18 +48,16 @@ inline int gram_chunk(long long BH, int N) {
 // Byte offsets of the clustering workspace: partial Gram matrices, the Gram
 // matrix, centroids, w_c = G c, b_c, cluster sizes, first positions, the
 // assignment (when the caller does not want it back), the tensor-core operand
-// rows of the centroids (bf16 [B*H][C][D], see cluster_prep_kernel), b_c again
-// padded to a multiple of 64 clusters per head, and four candidate clusters per
-// token.
+// rows of the centroids (bf16 [B*H][C][D + 64], see cluster_prep_kernel) and four
+// candidate clusters per token.
 struct ClusterWorkspace {
-  size_t gpart, gram, cent, w, b, cnt, off, assign, w16, bpad, cand, total;
-  int splits, chunk, C, Cpad;
+  size_t gpart, gram, cent, w, b, cnt, off, assign, w16, cand, total;
+  int splits, chunk, C;
 };
 inline ClusterWorkspace cluster_workspace(long long BH, int N, int D) {
   auto al = [](size_t x) { return (x + 255) / 256 * 256; };
   ClusterWorkspace w;
   w.C = (N + kBlock - 1) / kBlock;
-  w.Cpad = (w.C + 63) / 64 * 64;
   w.chunk = gram_chunk(BH, N);
   w.splits = (N + w.chunk - 1) / w.chunk;
   const size_t dd = static_cast<size_t>(D) * D * sizeof(float);
@@ -74,8 +72,7 @@ inline ClusterWorkspace cluster_workspace(long long BH, int N, int D) {
   w.off = w.cnt + al(c4);
   w.assign = w.off + al(c4);
   w.w16 = w.assign + al(static_cast<size_t>(BH) * N * sizeof(int));
-  w.bpad = w.w16 + al(static_cast<size_t>(BH) * w.C * D * 2);
-  w.cand = w.bpad + al(static_cast<size_t>(BH) * w.Cpad * sizeof(float));
+  w.cand = w.w16 + al(static_cast<size_t>(BH) * w.C * (D + 64) * 2);
   w.total = w.cand + al(static_cast<size_t>(BH) * N * 4 * sizeof(int));
   return w;
 }
@@ -239,18 +236,19 @@ __global__ void __launch_bounds__(256) cluster_init_assign_kernel(int* __restric
 // (ceil(C/16), B*H), D threads: thread i forms component i (G is symmetric, so
 // it reads column i of G as row i, and a warp reads G row by row).
 //
-// W16 (bf16 [B*H][C][D]) receives each centroid's tensor-core operand row for the
-// assignment, bf16(-2 w_c); bpad ([B*H][Cpad] fp32) receives b_c again, with zeros
-// in the padding columns [C, Cpad).
+// W16 (bf16 [B*H][C][D + 64]) receives each centroid's tensor-core operand row for
+// the assignment: bf16(-2 w_c) in columns [0, D), then b_c as the sum of two bf16
+// values (b_hi = bf16(b_c) in column D, b_lo = bf16(b_c - b_hi) in column D + 1)
+// and zeros.
 template <int D>
 __global__ void __launch_bounds__(D) cluster_prep_kernel(const float* __restrict__ G, const float* __restrict__ cent,
                                                          float* __restrict__ W, float* __restrict__ bvec,
                                                          int* __restrict__ cnt, int C,
-                                                         __nv_bfloat16* __restrict__ W16, float* __restrict__ bpad,
-                                                         int Cpad) {
+                                                         __nv_bfloat16* __restrict__ W16) {
   constexpr int kCl = 16;
   __shared__ float cs[kCl][D];
   __shared__ float red[kCl][D / 32];
+  __shared__ float bsh[kCl];
   const long long bh = blockIdx.y;
   const int c0 = blockIdx.x * kCl;
   const int ncl = min(kCl, C - c0);
@@ -271,7 +269,7 @@ __global__ void __launch_bounds__(D) cluster_prep_kernel(const float* __restrict
   for (int c = 0; c < kCl; ++c) {
     if (c < ncl) {
       W[(bh * C + c0 + c) * D + i] = acc[c];
-      W16[(bh * C + c0 + c) * D + i] = __float2bfloat16_rn(-2.f * acc[c]);
+      W16[(bh * C + c0 + c) * (D + 64) + i] = __float2bfloat16_rn(-2.f * acc[c]);
     }
     float v = cs[c][i] * acc[c];
 #pragma unroll
@@ -284,10 +282,20 @@ __global__ void __launch_bounds__(D) cluster_prep_kernel(const float* __restrict
 #pragma unroll
     for (int w = 0; w < D / 32; ++w) b += red[i][w];
     bvec[bh * C + c0 + i] = b;
-    bpad[bh * Cpad + c0 + i] = b;
+    bsh[i] = b;
     cnt[bh * C + c0 + i] = 0;   // counted again by the assignment
   }
-  if (c0 + kCl >= C && C + i < Cpad) bpad[bh * Cpad + C + i] = 0.f;   // the last CTA: the padding
+  __syncthreads();
+  // the bias columns of the operand rows: b_hi, b_lo, then zeros
+  for (int x = i; x < ncl * 64; x += D) {
+    const int c = x >> 6, k = x & 63;
+    const float b = bsh[c];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(b);
+    __nv_bfloat16 v = __float2bfloat16_rn(0.f);
+    if (k == 0) v = hi;
+    if (k == 1) v = __float2bfloat16_rn(b - __bfloat162float(hi));
+    W16[(bh * C + c0 + c) * (D + 64) + D + k] = v;
+  }
 }
 
 // ----------------------------------------------------------------------------
@@ -295,15 +303,20 @@ __global__ void __launch_bounds__(D) cluster_prep_kernel(const float* __restrict
 // product on the tensor cores, then the exact argmin among those four in fp32
 // (cluster_rescore_kernel). One CTA = 256 tokens of one head, two halves of 128
 // (the M = 128 of tcgen05.mma); per tile of 64 centroids
-//   D_h[token][c] = x . (-2 w_c)      (kind::f16, fp32 accumulate in TMEM)
-// with the tokens as the A operand in TMEM (written once from registers, so the
-// MMAs read only the centroid tile from shared memory) and the centroid tile's
-// bf16 rows from cluster_prep_kernel as B (TMA, one 4-D box per tile, six
-// stages). Both halves use each centroid tile, so a tile crosses L2 once per 256
-// tokens. Warp 16 (one thread) loads and issues. Warps 0-15 are the epilogue:
+//   D_h[token][c] = x . (-2 w_c) + 1 . b_hi_c + 1 . b_lo_c
+// (kind::f16, fp32 accumulate in TMEM) with the tokens as the A operand in TMEM
+// (written once from registers, so the MMAs read only the centroid tile from
+// shared memory) and the centroid tile's bf16 rows from cluster_prep_kernel as B
+// (TMA, one 4-D box per tile with the bias chunk, five stages): D / 16 K-steps
+// of the tokens, then one K-step of a block of TMEM columns whose rows start with
+// two ones against the rows' bias columns. Both halves use each centroid tile, so a tile crosses L2 once per 256
+// tokens. Warp 16 (one thread) issues the loads; warps 17 and 18 (one thread
+// each) issue the MMAs of half 0 and half 1: a single issuing thread waits about
+// as long per MMA as a 128 x 64 x 16 product takes at half the math rate, two keep
+// the tensor pipe busy. Warps 0-15 are the epilogue:
 // warp w reads TMEM lanes 32 (w % 4) .. (its 32 tokens) of half (w / 4) % 2 and
-// the 32 columns of column half w / 8 of each tile, adds b_c in fp32 and keeps
-// each token's four smallest values with their centroids in registers; the two
+// the 32 columns of column half w / 8 of each tile and keeps each token's four
+// smallest values with their centroids in registers; the two
 // column halves merge at the end. A lane marks the values below its token's
 // current fourth best in a bit mask, parks the 32 values in its own shared-memory
 // row, and offers only the marked ones, so a warp pays for its busiest lane's
@@ -321,10 +334,12 @@ struct ClusterTcCfg {
   static constexpr int kTok = 256;                     // tokens per CTA: two halves of 128
   static constexpr int kCt = 64;                       // centroids per tile (N of the MMA)
   static constexpr int kChunkBytes = kCt * 128;        // 8 KB: one column chunk of a tile
-  static constexpr int kWStage = kCh * kChunkBytes;
-  static constexpr int kStages = 6;
+  static constexpr int kWStage = (kCh + 1) * kChunkBytes;   // centroid rows + bias chunk
+  static constexpr int kStages = 5;
   static constexpr int kEpiWarps = 16;                 // 4 lane quadrants x 2 halves x 2 column halves
-  static constexpr int kThreads = (kEpiWarps + 1) * 32;  // + the issuing warp
+  static constexpr int kLoadWarp = kEpiWarps;          // TMA
+  static constexpr int kMmaWarp = kEpiWarps + 1;       // + h: the MMAs of half h; warp kMmaWarp owns TMEM
+  static constexpr int kThreads = (kEpiWarps + 3) * 32;
   static constexpr int oW = 0;
   static constexpr int oMerge = oW + kStages * kWStage;     // [2 halves][128 tokens][4 values, 4 centroids]
   static constexpr int kParkStride = 36;               // floats per lane row (144 B: 16-byte stores conflict-free)
@@ -332,9 +347,11 @@ struct ClusterTcCfg {
   static constexpr int oBar = oPark + kEpiWarps * 32 * kParkStride * 4;
   static constexpr int kSmemBytes = oBar + 256 + 1024;
   // TMEM columns: accumulator (buffer b, half h) at 64 (2 b + h); the tokens of
-  // half h (bf16 pairs, D / 2 columns) at kColX + (D / 2) h
+  // half h (bf16 pairs, D / 2 columns) at kColX + (D / 2) h; the ones block (its
+  // first column two bf16 ones, then zeros) at kColOnes
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColX = 256;
+  static constexpr uint32_t kColOnes = 384;
   static constexpr uint32_t kIdesc = idesc_bf16_f32(128, kCt, false);
 };
 
@@ -376,8 +393,8 @@ static __device__ __forceinline__ int visit_tile(int k, int tt0, int nt) {
 
 template <int D>
 __global__ void __launch_bounds__(ClusterTcCfg<D>::kThreads, 1)
-    cluster_assign_tc_kernel(const __nv_bfloat16* __restrict__ X, const __grid_constant__ CUtensorMap tmW,
-                             const float* __restrict__ bpad, int N, int C, int Cpad, int* __restrict__ cand) {
+    cluster_assign_tc_kernel(const __nv_bfloat16* __restrict__ X, const __grid_constant__ CUtensorMap tmW, int N,
+                             int C, int* __restrict__ cand) {
   using Cf = ClusterTcCfg<D>;
   extern __shared__ uint8_t tsm_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tsm_raw) + 1023) & ~uintptr_t(1023));
@@ -385,13 +402,13 @@ __global__ void __launch_bounds__(ClusterTcCfg<D>::kThreads, 1)
   float* sMerge = reinterpret_cast<float*>(base + Cf::oMerge);
   float* sPark = reinterpret_cast<float*>(base + Cf::oPark);
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + Cf::oBar);
-  uint64_t* wfull = bars;                      // [6]
-  uint64_t* wempty = bars + 6;                 // [6]
-  uint64_t* dfull = bars + 12;                 // [2]
-  uint64_t* dempty = bars + 14;                // [2], one arrival per epilogue warp
-  uint64_t* drain = bars + 16;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 17);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 18);
+  uint64_t* wfull = bars;                      // [kStages]
+  uint64_t* wempty = bars + 6;                 // [kStages], one arrival per half's MMAs
+  uint64_t* dfull = bars + 12;                 // [half][buffer]
+  uint64_t* dempty = bars + 16;                // [half][buffer], one arrival per epilogue warp of the half
+  uint64_t* drain = bars + 20;                 // [half]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 22);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 23);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long bh = blockIdx.y;
   const int t0 = blockIdx.x * Cf::kTok;
@@ -402,17 +419,18 @@ __global__ void __launch_bounds__(ClusterTcCfg<D>::kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < Cf::kStages; ++s) {
       mbar_init(&wfull[s], 1);
-      mbar_init(&wempty[s], 1);
+      mbar_init(&wempty[s], 2);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < 4; ++b) {
       mbar_init(&dfull[b], 1);
-      mbar_init(&dempty[b], Cf::kEpiWarps);
+      mbar_init(&dempty[b], Cf::kEpiWarps / 2);
     }
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == Cf::kEpiWarps) tmem_alloc(tmem_holder, Cf::kTmemCols);
+  if (warp == Cf::kMmaWarp) tmem_alloc(tmem_holder, Cf::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -436,64 +454,69 @@ __global__ void __launch_bounds__(ClusterTcCfg<D>::kThreads, 1)
       }
       tmem_st32u(tmem_base + (static_cast<uint32_t>(32 * quad) << 16) + Cf::kColX + (D / 2) * h + 32 * c, r);
     }
+    if (h == 0) {   // the ones block, for this warp's lanes
+      uint32_t r[32];
+#pragma unroll
+      for (int q = 0; q < 32; ++q) r[q] = q == 0 ? 0x3F803F80u : 0u;   // two bf16 ones
+      tmem_st32u(tmem_base + (static_cast<uint32_t>(32 * quad) << 16) + Cf::kColOnes, r);
+    }
     tmem_wait_st();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
 
-  if (warp == Cf::kEpiWarps) {
-    // ------------------------------------------------------------ loads and MMAs
+  if (warp == Cf::kLoadWarp) {
+    // ------------------------------------------------------------ loads
     if (lane == 0) {
       tma_prefetch_desc(&tmW);
-      auto load_w = [&](int t) {           // the t-th visited tile into stage t % kStages
+      int nw = 0;
+      for (int t = 0; t < ntiles; ++t) {
         const int s = t % Cf::kStages;
+        // the stage's previous tile (t - kStages) is read by both halves' MMAs
+        if (t >= Cf::kStages &&
+            !mbar_wait(&wempty[s], static_cast<uint32_t>((t - Cf::kStages) / Cf::kStages) & 1u, abort_flag))
+          break;
         mbar_expect_tx(&wfull[s], Cf::kWStage);
         tma_load_4d(sW + s * Cf::kWStage, &tmW, 0, visit_tile(t, tt0, ntiles) * Cf::kCt, 0, static_cast<int>(bh),
                     &wfull[s]);
-      };
-      int nw = 0;
-      for (; nw < Cf::kStages && nw < ntiles; ++nw) load_w(nw);
+        ++nw;
+      }
+      for (int k = max(0, nw - Cf::kStages); k < nw; ++k)   // no copy outlives the CTA
+        mbar_wait_drain(&wfull[k % Cf::kStages], static_cast<uint32_t>(k / Cf::kStages) & 1u);
+    }
+  } else if (warp > Cf::kLoadWarp) {
+    // ------------------------------------------------------------ the MMAs of half h
+    const int h = warp - Cf::kMmaWarp;
+    if (lane == 0) {
       const uint32_t wa = smem_u32(sW);
+      const uint32_t aX = tmem_base + Cf::kColX + (D / 2) * h;
       for (int t = 0; t < ntiles; ++t) {
         const int s = t % Cf::kStages, buf = t & 1;
         if (!mbar_wait(&wfull[s], static_cast<uint32_t>(t / Cf::kStages) & 1u, abort_flag)) break;
-        if (t >= 2 && !mbar_wait(&dempty[buf], static_cast<uint32_t>((t >> 1) - 1) & 1u, abort_flag)) break;
+        if (t >= 2 && !mbar_wait(&dempty[2 * h + buf], static_cast<uint32_t>((t >> 1) - 1) & 1u, abort_flag))
+          break;
         tc_fence_after();
         const uint32_t wb = wa + s * Cf::kWStage;
-        // the two halves' K-steps alternate: consecutive MMAs write different
-        // accumulators, so an issue never waits on the previous one's result
+        const uint32_t dD = tmem_base + Cf::kCt * (2 * buf + h);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t bd = sdesc_sw128(wb + (kk >> 2) * Cf::kChunkBytes + (kk & 3) * 32, 16, 1024);
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-            tc_mma_ts(tmem_base + Cf::kCt * (2 * buf + h), tmem_base + Cf::kColX + (D / 2) * h + kk * 8, bd,
-                      Cf::kIdesc, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&dfull[buf]);
+        for (int kk = 0; kk < D / 16; ++kk)
+          tc_mma_ts(dD, aX + kk * 8, sdesc_sw128(wb + (kk >> 2) * Cf::kChunkBytes + (kk & 3) * 32, 16, 1024),
+                    Cf::kIdesc, kk > 0 ? 1u : 0u);
+        // the bias: the ones block against the first K-step of the rows' bias chunk
+        tc_mma_ts(dD, tmem_base + Cf::kColOnes, sdesc_sw128(wb + Cf::kCh * Cf::kChunkBytes, 16, 1024), Cf::kIdesc,
+                  1u);
+        tc_commit(&dfull[2 * h + buf]);
         tc_commit(&wempty[s]);
-        // refill the stage of the previous tile (its MMAs are older than the ones
-        // just issued, so the tensor pipe stays fed while this thread waits)
-        const int r = t - 1 + Cf::kStages;
-        if (t >= 1 && r < ntiles) {
-          const int sp = (t - 1) % Cf::kStages;
-          if (!mbar_wait(&wempty[sp], static_cast<uint32_t>((t - 1) / Cf::kStages) & 1u, abort_flag)) break;
-          load_w(r);
-          ++nw;
-        }
       }
-      tc_commit(drain);
-      mbar_wait_drain(drain, 0u);
-      for (int k = max(0, nw - Cf::kStages); k < nw; ++k)
-        mbar_wait_drain(&wfull[k % Cf::kStages], static_cast<uint32_t>(k / Cf::kStages) & 1u);
+      tc_commit(&drain[h]);
+      mbar_wait_drain(&drain[h], 0u);
     }
   } else {
     // ------------------------------------------------------------ epilogue: the four best
     const int quad = warp & 3, h = (warp >> 2) & 1, cq = warp >> 3;
     const int row = quad * 32 + lane;          // token of the half == TMEM lane
     const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
-    const float* bhead = bpad + bh * Cpad;
     float* park = sPark + (warp * 32 + lane) * Cf::kParkStride;
     Top4 st;
     st.init();
@@ -502,16 +525,7 @@ __global__ void __launch_bounds__(ClusterTcCfg<D>::kThreads, 1)
       const int buf = t & 1;
       const int c0 = visit_tile(t, tt0, ntiles) * Cf::kCt + cq * 32;
       const int ncol = C - c0;                 // < 32 in the last tile: columns past C read zero rows
-      float bb[32];                            // b_c of the 32 columns (padded, so in bounds)
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const float4 f = __ldg(reinterpret_cast<const float4*>(bhead + c0) + q);
-        bb[4 * q] = f.x;
-        bb[4 * q + 1] = f.y;
-        bb[4 * q + 2] = f.z;
-        bb[4 * q + 3] = f.w;
-      }
-      if (!warp_wait(&dfull[buf], static_cast<uint32_t>(t >> 1) & 1u, abort_flag)) {
+      if (!warp_wait(&dfull[2 * h + buf], static_cast<uint32_t>(t >> 1) & 1u, abort_flag)) {
         alive = false;
         break;
       }
@@ -522,9 +536,7 @@ __global__ void __launch_bounds__(ClusterTcCfg<D>::kThreads, 1)
       pin32(v);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&dempty[buf]);   // the buffer may take tile t + 2
-#pragma unroll
-      for (int e = 0; e < 32; e += 2) f2unpack(fadd2(f2pack(v[e], v[e + 1]), f2pack(bb[e], bb[e + 1])), v[e], v[e + 1]);
+      if (lane == 0) mbar_arrive(&dempty[2 * h + buf]);   // the buffer may take tile t + 2
       if (ncol < 32) {
 #pragma unroll
         for (int e = 0; e < 32; ++e)
@@ -551,9 +563,13 @@ __global__ void __launch_bounds__(ClusterTcCfg<D>::kThreads, 1)
           }
         }
         while (pend) {                         // this lane's own row: no exchange between lanes
-          const int e = __ffs(pend) - 1;
+          const int e0 = __ffs(pend) - 1;      // two entries per pass: their loads overlap
           pend &= pend - 1;
-          st.offer(park[e], c0 + e);
+          const int e1 = pend ? __ffs(pend) - 1 : e0;
+          pend &= pend - 1;
+          const float x0 = park[e0], x1 = park[e1];
+          st.offer(x0, c0 + e0);
+          if (e1 != e0) st.offer(x1, c0 + e1);
         }
       }
     }
@@ -588,7 +604,7 @@ __global__ void __launch_bounds__(ClusterTcCfg<D>::kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == Cf::kEpiWarps) {
+  if (warp == Cf::kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_base, Cf::kTmemCols);
   }

@@ -131,16 +131,18 @@ sa_status launch_fwd(const sa_shape& s, const void* Q, const void* K, const void
   return SA_OK;
 }
 
-// The centroids' bf16 operand rows [B*H][C][D] as a 4-D tensor {64 elements, C
-// rows, D/64 chunks, B*H} (row stride 2D bytes, chunk stride 128 bytes): one box
-// {64, 64, D/64, 1} is a 64-centroid tile, landing as [chunk][row][128 B] with the
-// 128B swizzle. Rows past C read as zero.
+// The centroids' bf16 operand rows [B*H][C][D + 64] as a 4-D tensor {64
+// elements, C rows, D/64 + 1 chunks, B*H} (row stride 2(D + 64) bytes, chunk
+// stride 128 bytes): one box {64, 64, D/64 + 1, 1} is a 64-centroid tile with its
+// bias chunk, landing as [chunk][row][128 B] with the 128B swizzle. Rows past C
+// read as zero.
 bool make_w16_map(CUtensorMap* map, const void* ptr, long long BH, int C, int D) {
   auto enc = get_encode();
   if (!enc) return false;
-  cuuint64_t dims[4] = {64u, static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(D / 64), static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, 128u, static_cast<cuuint64_t>(C) * D * 2};
-  cuuint32_t box[4] = {64u, 64u, static_cast<cuuint32_t>(D / 64), 1u};
+  cuuint64_t dims[4] = {64u, static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(D / 64 + 1),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D + 64) * 2, 128u, static_cast<cuuint64_t>(C) * (D + 64) * 2};
+  cuuint32_t box[4] = {64u, 64u, static_cast<cuuint32_t>(D / 64 + 1), 1u};
   cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -167,7 +169,6 @@ sa_status launch_cluster(const sa_shape& s, const void* X, const void* Y, int it
   int* assign = assign_out ? assign_out : reinterpret_cast<int*>(wsb + L.assign);
   auto* w16 = reinterpret_cast<__nv_bfloat16*>(wsb + L.w16);
   int* cand = reinterpret_cast<int*>(wsb + L.cand);
-  float* bpad = reinterpret_cast<float*>(wsb + L.bpad);
   const auto* x = static_cast<const __nv_bfloat16*>(X);
   const auto* y = static_cast<const __nv_bfloat16*>(Y);
   const unsigned by = static_cast<unsigned>(BH);
@@ -187,9 +188,9 @@ sa_status launch_cluster(const sa_shape& s, const void* X, const void* Y, int it
   const dim3 order_grid((C + sa::kOrderClusters - 1) / sa::kOrderClusters, by);
   const dim3 cent_grid((C + 7) / 8, by);
   for (int it = 0; it < iters; ++it) {
-    sa::cluster_prep_kernel<D><<<dim3((C + 15) / 16, by), D, 0, st>>>(G, cent, W, bvec, cnt, C, w16, bpad, L.Cpad);
+    sa::cluster_prep_kernel<D><<<dim3((C + 15) / 16, by), D, 0, st>>>(G, cent, W, bvec, cnt, C, w16);
     sa::cluster_assign_tc_kernel<D><<<dim3((N + TC::kTok - 1) / TC::kTok, by), TC::kThreads, TC::kSmemBytes, st>>>(
-        x, mw, bpad, N, C, L.Cpad, cand);
+        x, mw, N, C, cand);
     sa::cluster_rescore_kernel<D><<<dim3((N + 63) / 64, by), 256, 0, st>>>(x, W, bvec, cand, assign, cnt, N, C);
     sa::cluster_offsets_kernel<<<by, 1024, 0, st>>>(cnt, off, C);
     sa::cluster_order_kernel<<<order_grid, 256, 0, st>>>(assign, off, perm, N, C);
