@@ -396,9 +396,10 @@ def run_ours(args, w, world, rank, local, pg):
         def run_fwd(stats=None):
             sa.sparse_attn_fwd(qs, ks, vs, plan, lam, out=os_, stats=stats, recall=rec)
             sa.sparse_attn_permute_rows(os_, cq.perm, inverse=True, out=out)
-        # kernels per step: per clustering 4 + 6 per iteration less the last iteration's
-        # centroid pass (+2 with none), 3 row moves, 3 plan kernels, the forward, the move back
-        launches_per_step = 2 * (4 + (6 * cl - 1 if cl > 0 else 2)) + 3 + 3 + 1 + 1
+        # kernels per step: per clustering 4, then 8 per iteration less the last
+        # iteration's centroid pass (with none, the 4 kernels of the order), 3 row moves,
+        # 3 plan kernels, the forward, the move back
+        launches_per_step = 2 * (4 + (8 * cl - 1 if cl > 0 else 4)) + 3 + 3 + 1 + 1
     else:
         def run_plan():
             sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False,

@@ -25,7 +25,8 @@
 // Each iteration: cluster_prep_kernel (w_c, b_c, their bf16 operand rows; clears
 // the sizes), cluster_assign_tc_kernel and cluster_rescore_kernel (argmin; counts
 // the sizes), cluster_offsets_kernel (each
-// cluster's first position), cluster_order_kernel (the stable order) and
+// cluster's first position), the stable order (cluster_chunk_count_kernel,
+// cluster_chunk_scan_kernel, cluster_order_kernel) and
 // cluster_centroid_kernel (each cluster's mean, summed over its tokens in token
 // order through the order just built). Everything is deterministic: every fp32
 // sum runs in a fixed order, the sizes are integer counts, and argmin ties go to
@@ -36,23 +37,33 @@
 
 namespace sa {
 
-// Tokens per partial Gram matrix: about 600 CTAs over all heads, at least 512
-// tokens each, a multiple of 32.
+// Tokens per partial Gram matrix: at most 592 CTAs over all heads (four per SM,
+// one wave), at least 512 tokens each, a multiple of 32.
 inline int gram_chunk(long long BH, int N) {
-  const long long want_splits = (600 + BH - 1) / BH;
+  const long long want_splits = BH >= 592 ? 1 : 592 / BH;
   long long chunk = (N + want_splits - 1) / want_splits;
   chunk = chunk < 512 ? 512 : chunk;
   return static_cast<int>((chunk + 31) / 32 * 32);
 }
 
+// Tokens per chunk of the stable order: at most 64 chunks per head, at least
+// 1024 tokens each, a multiple of 32.
+inline int order_chunk(int N) {
+  int n = (N + 1023) / 1024;
+  n = n > 64 ? 64 : n;
+  const int L = (N + n - 1) / n;
+  return (L + 31) / 32 * 32;
+}
+
 // Byte offsets of the clustering workspace: partial Gram matrices, the Gram
 // matrix, centroids, w_c = G c, b_c, cluster sizes, first positions, the
 // assignment (when the caller does not want it back), the tensor-core operand
-// rows of the centroids (bf16 [B*H][C][D + 64], see cluster_prep_kernel) and four
-// candidate clusters per token.
+// rows of the centroids (bf16 [B*H][C][D + 64], see cluster_prep_kernel), four
+// candidate clusters per token, and per (chunk, cluster) token counts, then
+// first positions, of the stable order.
 struct ClusterWorkspace {
-  size_t gpart, gram, cent, w, b, cnt, off, assign, w16, cand, total;
-  int splits, chunk, C;
+  size_t gpart, gram, cent, w, b, cnt, off, assign, w16, cand, chunks, total;
+  int splits, chunk, C, order_len, order_chunks;
 };
 inline ClusterWorkspace cluster_workspace(long long BH, int N, int D) {
   auto al = [](size_t x) { return (x + 255) / 256 * 256; };
@@ -60,6 +71,8 @@ inline ClusterWorkspace cluster_workspace(long long BH, int N, int D) {
   w.C = (N + kBlock - 1) / kBlock;
   w.chunk = gram_chunk(BH, N);
   w.splits = (N + w.chunk - 1) / w.chunk;
+  w.order_len = order_chunk(N);
+  w.order_chunks = (N + w.order_len - 1) / w.order_len;
   const size_t dd = static_cast<size_t>(D) * D * sizeof(float);
   const size_t cd = static_cast<size_t>(BH) * w.C * D * sizeof(float);
   const size_t c4 = static_cast<size_t>(BH) * w.C * sizeof(int);
@@ -73,7 +86,8 @@ inline ClusterWorkspace cluster_workspace(long long BH, int N, int D) {
   w.assign = w.off + al(c4);
   w.w16 = w.assign + al(static_cast<size_t>(BH) * N * sizeof(int));
   w.cand = w.w16 + al(static_cast<size_t>(BH) * w.C * (D + 64) * 2);
-  w.total = w.cand + al(static_cast<size_t>(BH) * N * 4 * sizeof(int));
+  w.chunks = w.cand + al(static_cast<size_t>(BH) * N * 4 * sizeof(int));
+  w.total = w.chunks + al(static_cast<size_t>(BH) * w.order_chunks * w.C * sizeof(int));
   return w;
 }
 
@@ -85,8 +99,9 @@ inline ClusterWorkspace cluster_workspace(long long BH, int N, int D) {
 // operands of four K = 16 steps of tcgen05.mma (M = 128 feature rows, N = D
 // feature columns, fp32 accumulate in TMEM across the whole chunk). Rows D..127 of
 // the tile stay zero when D = 64. Two tiles alternate: a tile is rewritten once
-// the MMAs that read it two tiles earlier have completed. The accumulator goes
-// to part[bh][split] (fp32 D x D).
+// the MMAs that read it two tiles earlier have completed, and the next tile's
+// loads are in flight while the current one is written. The accumulator goes to
+// part[bh][split] (fp32 D x D).
 template <int D>
 struct GramTcCfg {
   static constexpr int kTok = 64;                      // tokens per tile (one 128-byte row)
@@ -97,7 +112,7 @@ struct GramTcCfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(128) gram_tc_kernel(const __nv_bfloat16* __restrict__ Y, float* __restrict__ part,
+__global__ void __launch_bounds__(128, 4) gram_tc_kernel(const __nv_bfloat16* __restrict__ Y, float* __restrict__ part,
                                                       int N, int splits, int chunk) {
   using Cf = GramTcCfg<D>;
   constexpr int kOct = D / 8;                          // 16-byte feature groups of a token
@@ -128,19 +143,24 @@ __global__ void __launch_bounds__(128) gram_tc_kernel(const __nv_bfloat16* __res
   const uint32_t tmem_base = *tmem_holder;
   const __nv_bfloat16* src = Y + bh * static_cast<long long>(N) * D;
 
-  bool ok = true;
-  for (int j = 0; j < ntile; ++j) {
-    const int buf = j & 1;
+  // this warp's units of a tile: 32 consecutive tokens (one per lane) x 8 features
+  auto load_tile = [&](int j, uint4 (&u)[kUnits / 4]) {
     const int tt = t0 + j * Cf::kTok;
-    // this warp's units: 32 consecutive tokens (one per lane) x 8 features
-    uint4 u[kUnits / 4];
 #pragma unroll
     for (int q = 0; q < kUnits / 4; ++q) {
       const int unit = warp + 4 * q, half = unit / kOct, oct = unit % kOct;
       const int t = tt + 32 * half + lane;
-      u[q] = t < t1 ? __ldg(reinterpret_cast<const uint4*>(src + static_cast<long long>(t) * D) + oct)
-                    : make_uint4(0u, 0u, 0u, 0u);
+      u[q] = (j < ntile && t < t1) ? __ldg(reinterpret_cast<const uint4*>(src + static_cast<long long>(t) * D) + oct)
+                                    : make_uint4(0u, 0u, 0u, 0u);
     }
+  };
+  bool ok = true;
+  uint4 u[kUnits / 4];
+  load_tile(0, u);
+  for (int j = 0; j < ntile; ++j) {
+    const int buf = j & 1;
+    uint4 un[kUnits / 4];
+    load_tile(j + 1, un);                            // in flight while tile j is written
     if (j >= 2) {   // the MMAs of tile j - 2 (the last readers of this buffer) are done
       const bool w = mbar_wait(&done[buf], static_cast<uint32_t>((j - 2) >> 1) & 1u, abort_flag);
       if (!__syncthreads_and(w)) {
@@ -174,6 +194,8 @@ __global__ void __launch_bounds__(128) gram_tc_kernel(const __nv_bfloat16* __res
       }
       tc_commit(&done[buf]);
     }
+#pragma unroll
+    for (int q = 0; q < kUnits / 4; ++q) u[q] = un[q];
   }
   // the last commit covers every MMA of the chunk
   if (ok && ntile > 0) {
@@ -693,50 +715,89 @@ __global__ void __launch_bounds__(256) cluster_rescore_kernel(const __nv_bfloat1
   }
 }
 
-// Clusters per CTA of cluster_order_kernel.
-constexpr int kOrderClusters = 64;
-
-// The stable order: the tokens of cluster c go to perm[off[c] ..] in token
-// order. One CTA per 64 clusters of a head scans the head's assignment 256
-// tokens at a time; a token's place among its cluster's tokens of those 256 is
-// its rank among the lanes of its warp with the same cluster (match_any) plus
-// the counts of the earlier warps. Grid (ceil(C/64), B*H), 256 threads.
-__global__ void __launch_bounds__(256) cluster_order_kernel(const int* __restrict__ assign,
-                                                            const int* __restrict__ off, int* __restrict__ perm,
-                                                            int N, int C) {
-  __shared__ int scnt[kOrderClusters];          // tokens placed so far per cluster
-  __shared__ int wcnt[8][kOrderClusters];       // per warp, current 256 tokens
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// The stable order, a counting sort in three steps over chunks of L tokens of a
+// head (order_chunk): the tokens of cluster c go to perm[off[c] ..] in token order.
+//
+// Step 1: part[bh][j][c] = the number of chunk j's tokens in cluster c. Grid
+// (chunks, B*H), 256 threads, a shared-memory histogram of C counts (a warp's
+// lanes with the same cluster add once, through match_any). A cluster index
+// outside [0, C) is not counted; it sets the range bit of the device error word.
+__global__ void __launch_bounds__(256) cluster_chunk_count_kernel(const int* __restrict__ assign,
+                                                                  int* __restrict__ part, int N, int C, int L) {
+  extern __shared__ int hist[];
   const long long bh = blockIdx.y;
-  const int c0 = blockIdx.x * kOrderClusters;
-  const int ncl = min(kOrderClusters, C - c0);
-  const int* a = assign + bh * N;
-  if (threadIdx.x < kOrderClusters) scnt[threadIdx.x] = 0;
-  for (int t0 = 0; t0 < N; t0 += 256) {
-    const int t = t0 + threadIdx.x;
-    const int c = (t < N) ? a[t] - c0 : -1;
-    const bool mine = c >= 0 && c < ncl;
-    for (int e = threadIdx.x; e < 8 * kOrderClusters; e += 256) (&wcnt[0][0])[e] = 0;
-    __syncthreads();
-    const unsigned in = __ballot_sync(0xffffffffu, mine);
-    unsigned peers = 0u;
-    if (mine) {
-      peers = __match_any_sync(in, c);
-      if ((peers & ((1u << lane) - 1u)) == 0u) wcnt[warp][c] = __popc(peers);   // lowest lane of the group
+  const int j = blockIdx.x, lane = threadIdx.x & 31;
+  const int t0 = j * L, t1 = min(N, t0 + L);
+  for (int c = threadIdx.x; c < C; c += 256) hist[c] = 0;
+  __syncthreads();
+  for (int tb = t0; tb < t1; tb += 256) {
+    const int t = tb + threadIdx.x;
+    int c = t < t1 ? assign[bh * N + t] : -1;
+    if (t < t1 && (c < 0 || c >= C)) {
+      atomicOr(&g_dev_error, DEVERR_RANGE);
+      c = -1;
     }
-    __syncthreads();
-    if (mine) {
-      int rank = scnt[c] + __popc(peers & ((1u << lane) - 1u));
-      for (int w = 0; w < warp; ++w) rank += wcnt[w][c];
-      perm[bh * N + off[bh * C + c0 + c] + rank] = t;
+    const unsigned peers = __match_any_sync(0xffffffffu, c);
+    if (c >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[c], __popc(peers));
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < C; c += 256) part[(bh * gridDim.x + j) * C + c] = hist[c];
+}
+
+// Step 2: part[bh][j][c] becomes the first position of chunk j's tokens of
+// cluster c: off[c] plus the counts of the earlier chunks. Grid (ceil(C/256),
+// B*H), a thread per cluster walking the chunks in order.
+__global__ void __launch_bounds__(256) cluster_chunk_scan_kernel(const int* __restrict__ off, int* __restrict__ part,
+                                                                 int C, int chunks) {
+  const long long bh = blockIdx.y;
+  const int c = blockIdx.x * 256 + threadIdx.x;
+  if (c >= C) return;
+  int run = off[bh * C + c];
+  int* col = part + bh * chunks * static_cast<long long>(C) + c;
+  for (int j0 = 0; j0 < chunks; j0 += 16) {   // 16 loads in flight, then their stores
+    int v[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) v[q] = j0 + q < chunks ? col[static_cast<long long>(j0 + q) * C] : 0;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      if (j0 + q < chunks) col[static_cast<long long>(j0 + q) * C] = run;
+      run += v[q];
     }
-    __syncthreads();
-    if (threadIdx.x < kOrderClusters) {
-      int add = 0;
-      for (int w = 0; w < 8; ++w) add += wcnt[w][threadIdx.x];
-      scnt[threadIdx.x] += add;
+  }
+}
+
+// Step 3: one warp per chunk places its tokens 32 at a time, in token order: a
+// token's position is its cluster's next free position in the chunk (a
+// shared-memory copy of step 2's column) plus its rank among the lanes with the
+// same cluster (match_any); the group's highest lane then advances the position.
+// Grid (chunks, B*H), 32 threads, C ints of shared memory. A position outside
+// [0, N) (inconsistent sizes) is not written; it sets the range bit.
+__global__ void __launch_bounds__(32) cluster_order_kernel(const int* __restrict__ assign,
+                                                           const int* __restrict__ part, int* __restrict__ perm,
+                                                           int N, int C, int L) {
+  extern __shared__ int next[];
+  const long long bh = blockIdx.y;
+  const int j = blockIdx.x, lane = threadIdx.x;
+  const int t0 = j * L, t1 = min(N, t0 + L);
+  const int* col = part + (bh * gridDim.x + j) * C;
+  for (int c = lane; c < C; c += 32) next[c] = col[c];
+  __syncwarp();
+  const unsigned below = (1u << lane) - 1u;
+  for (int tb = t0; tb < t1; tb += 32) {
+    const int t = tb + lane;
+    int c = t < t1 ? assign[bh * N + t] : -1;
+    if (c >= C) c = -1;                        // counted as an error in step 1
+    const unsigned peers = __match_any_sync(0xffffffffu, c);
+    if (c >= 0) {
+      const int pos = next[c] + __popc(peers & below);
+      if (pos >= 0 && pos < N)
+        perm[bh * N + pos] = t;
+      else
+        atomicOr(&g_dev_error, DEVERR_RANGE);
     }
-    __syncthreads();   // wcnt is read above before the next 256 clear it
+    __syncwarp();
+    if (c >= 0 && lane == 31 - __clz(peers)) next[c] += __popc(peers);
+    __syncwarp();
   }
 }
 

@@ -185,24 +185,29 @@ sa_status launch_cluster(const sa_shape& s, const void* X, const void* Y, int it
   if (sa::set_smem(sa::cluster_assign_tc_kernel<D>, TC::kSmemBytes) != SA_OK) return SA_ERR_CUDA;
   CUtensorMap mw;
   if (iters > 0 && !make_w16_map(&mw, w16, BH, C, D)) return SA_ERR_CUDA;
-  const dim3 order_grid((C + sa::kOrderClusters - 1) / sa::kOrderClusters, by);
+  int* part = reinterpret_cast<int*>(wsb + L.chunks);
+  const dim3 chunk_grid(static_cast<unsigned>(L.order_chunks), by);
+  const size_t hist_bytes = static_cast<size_t>(C) * sizeof(int);
+  // the stable order of the current assignment (cnt holds the sizes)
+  auto order = [&]() {
+    sa::cluster_chunk_count_kernel<<<chunk_grid, 256, hist_bytes, st>>>(assign, part, N, C, L.order_len);
+    sa::cluster_offsets_kernel<<<by, 1024, 0, st>>>(cnt, off, C);
+    sa::cluster_chunk_scan_kernel<<<dim3((C + 255) / 256, by), 256, 0, st>>>(off, part, C, L.order_chunks);
+    sa::cluster_order_kernel<<<chunk_grid, 32, hist_bytes, st>>>(assign, part, perm, N, C, L.order_len);
+  };
   const dim3 cent_grid((C + 7) / 8, by);
   for (int it = 0; it < iters; ++it) {
     sa::cluster_prep_kernel<D><<<dim3((C + 15) / 16, by), D, 0, st>>>(G, cent, W, bvec, cnt, C, w16);
     sa::cluster_assign_tc_kernel<D><<<dim3((N + TC::kTok - 1) / TC::kTok, by), TC::kThreads, TC::kSmemBytes, st>>>(
         x, mw, N, C, cand);
     sa::cluster_rescore_kernel<D><<<dim3((N + 63) / 64, by), 256, 0, st>>>(x, W, bvec, cand, assign, cnt, N, C);
-    sa::cluster_offsets_kernel<<<by, 1024, 0, st>>>(cnt, off, C);
-    sa::cluster_order_kernel<<<order_grid, 256, 0, st>>>(assign, off, perm, N, C);
+    order();
     // the means of the new clusters: the next iteration's centroids, or the output
     if (it + 1 < iters || cent_out)
       sa::cluster_centroid_kernel<D><<<cent_grid, 256, 0, st>>>(x, perm, off, cnt, cent, N, C);
     if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   }
-  if (iters == 0) {   // the plain blocks: identity order, block means from the pooling kernel
-    sa::cluster_offsets_kernel<<<by, 1024, 0, st>>>(cnt, off, C);
-    sa::cluster_order_kernel<<<order_grid, 256, 0, st>>>(assign, off, perm, N, C);
-  }
+  if (iters == 0) order();   // the plain blocks: identity order, block means from the pooling kernel
   if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   if (cent_out && cudaMemcpyAsync(cent_out, cent, static_cast<size_t>(BH) * C * D * sizeof(float),
                                   cudaMemcpyDeviceToDevice, st) != cudaSuccess)
