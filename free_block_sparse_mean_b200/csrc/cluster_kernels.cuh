@@ -9,9 +9,9 @@
 // the same for every centroid, the nearest centroid is the argmin over c of
 // c^T G c - 2 x . (G c). So each Lloyd iteration is: w_c = G c and b_c = c . w_c
 // per centroid (cluster_prep_kernel), an argmin over all centroids per token (a
-// bf16 tensor-core product of the tokens with the w_c that keeps each token's four
-// best, cluster_assign_tc_kernel, then their exact fp32 scores,
-// cluster_rescore_kernel), and the mean of each cluster's tokens
+// tensor-core product of the bf16 tokens with the w_c split into bf16 high and
+// low parts that keeps each token's four best, cluster_assign_tc_kernel, then
+// their exact fp32 scores, cluster_rescore_kernel), and the mean of each cluster's tokens
 // (cluster_centroid_kernel). The
 // clusters start at the 64-token block means (the pooling kernel), so zero
 // iterations reproduce the plain blocks.
@@ -58,7 +58,7 @@ inline int order_chunk(int N) {
 // Byte offsets of the clustering workspace: partial Gram matrices, the Gram
 // matrix, centroids, w_c = G c, b_c, cluster sizes, first positions, the
 // assignment (when the caller does not want it back), the tensor-core operand
-// rows of the centroids (bf16 [B*H][C][D + 64], see cluster_prep_kernel), four
+// rows of the centroids (bf16 [B*H][C][2D + 64], see cluster_prep_kernel), four
 // candidate clusters per token, and per (chunk, cluster) token counts, then
 // first positions, of the stable order.
 struct ClusterWorkspace {
@@ -85,7 +85,7 @@ inline ClusterWorkspace cluster_workspace(long long BH, int N, int D) {
   w.off = w.cnt + al(c4);
   w.assign = w.off + al(c4);
   w.w16 = w.assign + al(static_cast<size_t>(BH) * N * sizeof(int));
-  w.cand = w.w16 + al(static_cast<size_t>(BH) * w.C * (D + 64) * 2);
+  w.cand = w.w16 + al(static_cast<size_t>(BH) * w.C * (2 * D + 64) * 2);
   w.chunks = w.cand + al(static_cast<size_t>(BH) * N * 4 * sizeof(int));
   w.total = w.chunks + al(static_cast<size_t>(BH) * w.order_chunks * w.C * sizeof(int));
   return w;
@@ -258,10 +258,10 @@ __global__ void __launch_bounds__(256) cluster_init_assign_kernel(int* __restric
 // (ceil(C/16), B*H), D threads: thread i forms component i (G is symmetric, so
 // it reads column i of G as row i, and a warp reads G row by row).
 //
-// W16 (bf16 [B*H][C][D + 64]) receives each centroid's tensor-core operand row for
-// the assignment: bf16(-2 w_c) in columns [0, D), then b_c as the sum of two bf16
-// values (b_hi = bf16(b_c) in column D, b_lo = bf16(b_c - b_hi) in column D + 1)
-// and zeros.
+// W16 (bf16 [B*H][C][2D + 64]) receives each centroid's tensor-core operand row
+// for the assignment: v = -2 w_c as two bf16 parts, hi = bf16(v) in columns
+// [0, D) and lo = bf16(v - hi) in [D, 2D) (together 16 significant bits), then
+// b_c the same way (b_hi in column 2D, b_lo in 2D + 1) and zeros.
 template <int D>
 __global__ void __launch_bounds__(D) cluster_prep_kernel(const float* __restrict__ G, const float* __restrict__ cent,
                                                          float* __restrict__ W, float* __restrict__ bvec,
@@ -291,7 +291,10 @@ __global__ void __launch_bounds__(D) cluster_prep_kernel(const float* __restrict
   for (int c = 0; c < kCl; ++c) {
     if (c < ncl) {
       W[(bh * C + c0 + c) * D + i] = acc[c];
-      W16[(bh * C + c0 + c) * (D + 64) + i] = __float2bfloat16_rn(-2.f * acc[c]);
+      const float v = -2.f * acc[c];
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+      W16[(bh * C + c0 + c) * (2 * D + 64) + i] = hi;
+      W16[(bh * C + c0 + c) * (2 * D + 64) + D + i] = __float2bfloat16_rn(v - __bfloat162float(hi));
     }
     float v = cs[c][i] * acc[c];
 #pragma unroll
@@ -316,7 +319,7 @@ __global__ void __launch_bounds__(D) cluster_prep_kernel(const float* __restrict
     __nv_bfloat16 v = __float2bfloat16_rn(0.f);
     if (k == 0) v = hi;
     if (k == 1) v = __float2bfloat16_rn(b - __bfloat162float(hi));
-    W16[(bh * C + c0 + c) * (D + 64) + D + k] = v;
+    W16[(bh * C + c0 + c) * (2 * D + 64) + 2 * D + k] = v;
   }
 }
 
@@ -325,13 +328,15 @@ __global__ void __launch_bounds__(D) cluster_prep_kernel(const float* __restrict
 // product on the tensor cores, then the exact argmin among those four in fp32
 // (cluster_rescore_kernel). One CTA = 256 tokens of one head, two halves of 128
 // (the M = 128 of tcgen05.mma); per tile of 64 centroids
-//   D_h[token][c] = x . (-2 w_c) + 1 . b_hi_c + 1 . b_lo_c
-// (kind::f16, fp32 accumulate in TMEM) with the tokens as the A operand in TMEM
-// (written once from registers, so the MMAs read only the centroid tile from
-// shared memory) and the centroid tile's bf16 rows from cluster_prep_kernel as B
-// (TMA, one 4-D box per tile with the bias chunk, five stages): D / 16 K-steps
-// of the tokens, then one K-step of a block of TMEM columns whose rows start with
-// two ones against the rows' bias columns. Both halves use each centroid tile, so a tile crosses L2 once per 256
+//   D_h[token][c] = x . hi_c + x . lo_c + 1 . b_hi_c + 1 . b_lo_c
+// (kind::f16, fp32 accumulate in TMEM; hi + lo = -2 w_c to 16 significant bits,
+// so the product is off by about 2^-17 of |x| |w_c| rather than bf16's 2^-9) with
+// the tokens as the A operand in TMEM (written once from registers, so the MMAs
+// read only the centroid tile from shared memory) and the centroid tile's rows
+// from cluster_prep_kernel as B (TMA, one 4-D box per tile with the low part and
+// the bias chunk): D / 16 K-steps of the tokens against the high part, D / 16
+// against the low part, then one K-step of a block of TMEM columns whose rows
+// start with two ones against the rows' bias columns. Both halves use each centroid tile, so a tile crosses L2 once per 256
 // tokens. Warp 16 (one thread) issues the loads; warps 17 and 18 (one thread
 // each) issue the MMAs of half 0 and half 1: a single issuing thread waits about
 // as long per MMA as a 128 x 64 x 16 product takes at half the math rate, two keep
@@ -346,18 +351,19 @@ __global__ void __launch_bounds__(D) cluster_prep_kernel(const float* __restrict
 // any lane needs. Two TMEM buffers per half keep
 // the tensor cores and the epilogue overlapped; a CTA visits the centroid tiles
 // starting from the one that holds its tokens' first clusters (visit_tile), so
-// the four best settle in the first tile. The bf16 product moves the argmin for
-// a fraction of a percent of the tokens; the four best of the product contain
-// the fp32 argmin (measured on the workloads' inputs), and the re-score restores
-// it exactly.
+// the four best settle in the first tile. The split product still moves the
+// argmin where two distances agree to about 1e-5; its four best contained the
+// fp32 argmin for every token measured (inputs whose distances crowd within 1e-4
+// of each other included, where bf16 alone needed sixteen), and the re-score
+// restores it exactly.
 template <int D>
 struct ClusterTcCfg {
   static constexpr int kCh = D / 64;                   // 128-byte column chunks of a row
   static constexpr int kTok = 256;                     // tokens per CTA: two halves of 128
   static constexpr int kCt = 64;                       // centroids per tile (N of the MMA)
   static constexpr int kChunkBytes = kCt * 128;        // 8 KB: one column chunk of a tile
-  static constexpr int kWStage = (kCh + 1) * kChunkBytes;   // centroid rows + bias chunk
-  static constexpr int kStages = 5;
+  static constexpr int kWStage = (2 * kCh + 1) * kChunkBytes;   // high, low and bias chunks
+  static constexpr int kStages = D == 128 ? 3 : 5;
   static constexpr int kEpiWarps = 16;                 // 4 lane quadrants x 2 halves x 2 column halves
   static constexpr int kLoadWarp = kEpiWarps;          // TMA
   static constexpr int kMmaWarp = kEpiWarps + 1;       // + h: the MMAs of half h; warp kMmaWarp owns TMEM
@@ -522,12 +528,15 @@ __global__ void __launch_bounds__(ClusterTcCfg<D>::kThreads, 1)
         const uint32_t wb = wa + s * Cf::kWStage;
         const uint32_t dD = tmem_base + Cf::kCt * (2 * buf + h);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          tc_mma_ts(dD, aX + kk * 8, sdesc_sw128(wb + (kk >> 2) * Cf::kChunkBytes + (kk & 3) * 32, 16, 1024),
-                    Cf::kIdesc, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < 2 * (D / 16); ++kk) {   // the high part, then the low part
+          const int k = kk % (D / 16);
+          tc_mma_ts(dD, aX + k * 8,
+                    sdesc_sw128(wb + (kk >> 2) * Cf::kChunkBytes + (kk & 3) * 32, 16, 1024), Cf::kIdesc,
+                    kk > 0 ? 1u : 0u);
+        }
         // the bias: the ones block against the first K-step of the rows' bias chunk
-        tc_mma_ts(dD, tmem_base + Cf::kColOnes, sdesc_sw128(wb + Cf::kCh * Cf::kChunkBytes, 16, 1024), Cf::kIdesc,
-                  1u);
+        tc_mma_ts(dD, tmem_base + Cf::kColOnes, sdesc_sw128(wb + 2 * Cf::kCh * Cf::kChunkBytes, 16, 1024),
+                  Cf::kIdesc, 1u);
         tc_commit(&dfull[2 * h + buf]);
         tc_commit(&wempty[s]);
       }

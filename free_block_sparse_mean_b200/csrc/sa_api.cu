@@ -131,18 +131,19 @@ sa_status launch_fwd(const sa_shape& s, const void* Q, const void* K, const void
   return SA_OK;
 }
 
-// The centroids' bf16 operand rows [B*H][C][D + 64] as a 4-D tensor {64
-// elements, C rows, D/64 + 1 chunks, B*H} (row stride 2(D + 64) bytes, chunk
-// stride 128 bytes): one box {64, 64, D/64 + 1, 1} is a 64-centroid tile with its
-// bias chunk, landing as [chunk][row][128 B] with the 128B swizzle. Rows past C
-// read as zero.
+// The centroids' bf16 operand rows [B*H][C][2D + 64] as a 4-D tensor {64
+// elements, C rows, D/32 + 1 chunks, B*H} (row stride 2(2D + 64) bytes, chunk
+// stride 128 bytes): one box {64, 64, D/32 + 1, 1} is a 64-centroid tile with its
+// high, low and bias chunks, landing as [chunk][row][128 B] with the 128B
+// swizzle. Rows past C read as zero.
 bool make_w16_map(CUtensorMap* map, const void* ptr, long long BH, int C, int D) {
   auto enc = get_encode();
   if (!enc) return false;
-  cuuint64_t dims[4] = {64u, static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(D / 64 + 1),
+  cuuint64_t dims[4] = {64u, static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(D / 32 + 1),
                         static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D + 64) * 2, 128u, static_cast<cuuint64_t>(C) * (D + 64) * 2};
-  cuuint32_t box[4] = {64u, 64u, static_cast<cuuint32_t>(D / 64 + 1), 1u};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(2 * D + 64) * 2, 128u,
+                           static_cast<cuuint64_t>(C) * (2 * D + 64) * 2};
+  cuuint32_t box[4] = {64u, 64u, static_cast<cuuint32_t>(D / 32 + 1), 1u};
   cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

@@ -37,6 +37,18 @@ def _inputs(case):
         q, k, v = wl.random_qkv(2, 2, 1000, 64, seed=4, device=_dev())
         drift = torch.sin(torch.arange(1000, device=_dev()) / 40.0)[None, None, :, None]
         return (q.float() * 0.5 + drift).to(torch.bfloat16), k, v
+    if case in ("tiles128", "tiles64"):
+        # more clusters than one centroid tile of the tensor-core assignment (64):
+        # 301 clusters (five tiles, the last one partial) with d = 128, and 141
+        # clusters (three tiles) over B = 2 with d = 64; CTAs of 256 tokens start in
+        # every tile, so every visiting order occurs
+        B, H, N, d = (1, 2, 19217, 128) if case == "tiles128" else (2, 1, 9000, 64)
+        q, k, v = wl.random_qkv(B, H, N, d, seed=11, device=_dev())
+        pos = torch.arange(N, device=_dev(), dtype=torch.float32)
+        drift = (torch.sin(pos / 300.0)[:, None] * torch.linspace(-1.0, 1.0, d, device=_dev())[None, :]
+                 + torch.cos(pos / 97.0)[:, None] * torch.linspace(1.0, -0.5, d, device=_dev())[None, :])
+        drift = drift[None, None]
+        return (q.float() * 0.5 + drift).to(torch.bfloat16), (k.float() * 0.5 - drift).to(torch.bfloat16), v
     raise ValueError(case)
 
 
@@ -57,7 +69,7 @@ def _check_order_and_centroids(x, res, C):
                 np.testing.assert_allclose(cent[b, h, c], m, rtol=1e-5, atol=1e-5)
 
 
-@pytest.mark.parametrize("case", ["small", "ragged64"])
+@pytest.mark.parametrize("case", ["small", "ragged64", "tiles128", "tiles64"])
 @pytest.mark.parametrize("side", ["q", "k"])
 def test_one_iteration_matches_the_oracle(case, side):
     q, k, _ = _inputs(case)
@@ -80,20 +92,22 @@ def test_one_iteration_matches_the_oracle(case, side):
     _check_order_and_centroids(x, res, C)
 
 
+@pytest.mark.parametrize("case,iters", [("small", 4), ("tiles128", 3)])
 @pytest.mark.parametrize("side", ["q", "k"])
-def test_every_iteration_matches_an_oracle_step(side):
+def test_every_iteration_matches_an_oracle_step(case, iters, side):
     """Each Lloyd iteration on its own: from the GPU's centroids after t
     iterations, one oracle assignment step (argmin of the interaction distance,
     ties to the lowest index) must give the GPU's assignment after t + 1
     iterations, except tokens whose two distances lie within 1e-5 (relative) of
     each other; the GPU's centroids after t + 1 are the means of that assignment.
     Deterministic kernels: the first t iterations of the (t + 1)-run are the t-run."""
-    q, k, _ = _inputs("small")
+    q, k, _ = _inputs(case)
     x, y = (q, k) if side == "q" else (k, q)
     X, Y = orc.as_f64(x.cpu()), orc.as_f64(y.cpu())
     G = orc.gram(Y)
+    C = -(-x.shape[2] // 64)
     prev = sa.sparse_attn_cluster(x, y, 1, with_centroids=True)
-    for t in range(1, 4):
+    for t in range(1, iters):
         nxt = sa.sparse_attn_cluster(x, y, t + 1, with_centroids=True)
         torch.cuda.synchronize()
         assert sa.sparse_attn_device_error() == 0
@@ -107,7 +121,7 @@ def test_every_iteration_matches_an_oracle_step(side):
             gap = d[a_g[b, h, tok]] - d[a_o[b, h, tok]]
             assert gap <= 1e-5 * (abs(d).max() + 1.0), (t, b, h, tok, gap)
         print(f"iteration {t + 1} ({side}): {len(diff[0])} of {a_g.size} tokens on near-ties")
-        _check_order_and_centroids(x, nxt, 64)
+        _check_order_and_centroids(x, nxt, C)
         prev = nxt
 
 
