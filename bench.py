@@ -92,9 +92,10 @@ def peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def measured_traffic(w, tau, lam, qk="bf16", recall=None):
+def measured_traffic(w, tau, lam, qk="bf16", recall=None, centroid_weight=None):
     """DRAM bytes per launch of the forward kernel from the committed ncu capture,
-    or None if the kernel source changed since (or the workload differs)."""
+    or None if the kernel source changed since (or the workload differs: for the
+    video workloads the key names the centroid weight, which sets the sparsity)."""
     import hashlib
     p = os.path.join(ROOT, "profiles", "fwd_kernel_traffic.json")
     if not os.path.exists(p):
@@ -111,6 +112,9 @@ def measured_traffic(w, tau, lam, qk="bf16", recall=None):
     key = key.replace("lambda=-12.0", "lambda=-12") + ("" if qk == "bf16" else f" qk={qk}")
     if recall is not None:
         key = key.split(" lambda=")[0] + f" recall={recall:g}"
+    if w.kind == "video":
+        cw = w.centroid_weight if centroid_weight is None else centroid_weight
+        key += f" centroid_weight={cw:g}"
     ent = d.get("traffic_bytes_per_launch", {}).get(key)
     return None if ent is None else float(ent["total"])
 
@@ -563,7 +567,7 @@ def run_ours(args, w, world, rank, local, pg):
         "predictor": {"bound": "hbm", "achieved": pred_gbs, "peak": hbm, "unit": "GB/s", "frac": pred_gbs / hbm,
                       "bytes": pred_bytes, "peak_source": f"{pk_kind} hbm_gbs"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
-                     "frac": achieved / peak_t, "traffic": None if cl is not None else measured_traffic(w, args.tau, lam, args.qk, rec),
+                     "frac": achieved / peak_t, "traffic": None if cl is not None else measured_traffic(w, args.tau, lam, args.qk, rec, args.centroid_weight),
                      "kernel": (f"fwd_kernel<{D}, int8 scores> (sparse_attn_fwd_i8)" if i8
                                 else f"fwd_kernel<{D}, fp8 scores> (sparse_attn_fwd_q8)") if q8
                      else (f"fwd_kernel<{D}, recall filter> (sparse_attn_fwd_recall)" if rec is not None
