@@ -339,6 +339,40 @@ static __device__ __forceinline__ float lane_sum_ge(const float* row, int Nb, in
   return (p0 + p1) + (p2 + p3);
 }
 
+// lane_sum_ge, plus how many of the lane's elements have bits >= key.
+static __device__ __forceinline__ float lane_sum_count_ge(const float* row, int Nb, int lane, uint32_t key, int& n) {
+  float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+  int n0 = 0, n1 = 0, n2 = 0, n3 = 0;
+  int j = lane;
+  for (; j + 96 < Nb; j += 128) {
+    const float e0 = row[j], e1 = row[j + 32], e2 = row[j + 64], e3 = row[j + 96];
+    const bool g0 = __float_as_uint(e0) >= key, g1 = __float_as_uint(e1) >= key;
+    const bool g2 = __float_as_uint(e2) >= key, g3 = __float_as_uint(e3) >= key;
+    p0 += g0 ? e0 : 0.f;
+    p1 += g1 ? e1 : 0.f;
+    p2 += g2 ? e2 : 0.f;
+    p3 += g3 ? e3 : 0.f;
+    n0 += g0;
+    n1 += g1;
+    n2 += g2;
+    n3 += g3;
+  }
+  if (j < Nb && __float_as_uint(row[j]) >= key) {
+    p0 += row[j];
+    ++n0;
+  }
+  if (j + 32 < Nb && __float_as_uint(row[j + 32]) >= key) {
+    p1 += row[j + 32];
+    ++n1;
+  }
+  if (j + 64 < Nb && __float_as_uint(row[j + 64]) >= key) {
+    p2 += row[j + 64];
+    ++n2;
+  }
+  n = (n0 + n1) + (n2 + n3);
+  return (p0 + p1) + (p2 + p3);
+}
+
 template <bool kEightWay>
 static __device__ __forceinline__ void select_row(float* row, int Nb, int i, long long bh, float tau, int lane,
                                                   uint8_t* __restrict__ mask, int* __restrict__ count,
@@ -409,6 +443,13 @@ static __device__ __forceinline__ void select_row(float* row, int Nb, int i, lon
   } else {
     const float T = tau * tot;
     uint32_t lo = 0u, hi = kmax + 1u;   // S(lo) >= T > S(hi)
+    // bisection only: the numbers of elements with bits >= lo and >= hi, and S(hi).
+    // Once exactly one element lies in [lo, hi), S is constant on [lo, its bits]
+    // and on (its bits, hi], so its bits are the largest key with S >= T, the key
+    // the search would end on: it stops there.
+    int c_lo = Nb, c_hi = 0;
+    float s_hi = 0.f;
+    bool single = false;
     while (hi - lo > 1u) {
       if constexpr (kEightWay) {
         // 7 probes split [lo, hi) into 8 parts; the last one is above lo once hi - lo >= 2
@@ -440,17 +481,41 @@ static __device__ __forceinline__ void select_row(float* row, int Nb, int i, lon
         lo = nlo;
         hi = nhi;
       } else {
+        if (c_lo - c_hi == 1) {
+          single = true;
+          break;
+        }
         const uint32_t mid = lo + ((hi - lo) >> 1);
-        float s = lane_sum_ge(row, Nb, lane, mid);
+        int c;
+        float s = lane_sum_count_ge(row, Nb, lane, mid, c);
 #pragma unroll
         for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(FULL, s, o);
-        if (s >= T) lo = mid; else hi = mid;
+        c = __reduce_add_sync(FULL, c);
+        if (s >= T) {
+          lo = mid;
+          c_lo = c;
+        } else {
+          hi = mid;
+          c_hi = c;
+          s_hi = s;
+        }
       }
     }
     K = lo;
     float sgt = 0.f;
     int nties = 0;
-    if constexpr (kEightWay) {
+    if (single) {
+      // the one element in [lo, hi): its bits are the cut-off; S(hi) was formed like
+      // every probe, over the elements above it
+      uint32_t u = 0u;
+      for (int j = lane; j < Nb; j += 32) {
+        const uint32_t kj = __float_as_uint(row[j]);
+        if (kj >= lo && kj < hi) u = kj;
+      }
+      K = __reduce_max_sync(FULL, u);
+      sgt = s_hi;
+      nties = 1;
+    } else if constexpr (kEightWay) {
       for (int j = lane; j < Nb; j += 32) {
         const uint32_t kj = __float_as_uint(row[j]);
         sgt += (kj > K) ? row[j] : 0.f;
@@ -469,10 +534,12 @@ static __device__ __forceinline__ void select_row(float* row, int Nb, int i, lon
       for (; j < Nb; j += 32) nties += __float_as_uint(row[j]) == K;
       nties += (n1 + n2) + n3;
     }
+    if (!single) {   // the lanes' parts (the single case has the totals already)
 #pragma unroll
-    for (int o = 16; o; o >>= 1) {
-      sgt += __shfl_xor_sync(FULL, sgt, o);
-      nties += __shfl_xor_sync(FULL, nties, o);
+      for (int o = 16; o; o >>= 1) {
+        sgt += __shfl_xor_sync(FULL, sgt, o);
+        nties += __shfl_xor_sync(FULL, nties, o);
+      }
     }
     const float eK = __uint_as_float(K);
     float acc = sgt;
