@@ -16,8 +16,6 @@
 
 namespace sa {
 
-// Byte offsets of the plan workspace: pooled Q and K (fp32 [B,H,Nb,d]), then per
-// query block a 64-bit MinHash sort key and the kept set as a bitset of W words.
 // Shared memory of the pairing kernel for Nb blocks per head without the bitsets:
 // the sort keys of the blocks and of the tiles (powers of two), the pairs, the
 // order, the matching state and the scan scratch.
@@ -35,15 +33,27 @@ __host__ __device__ inline bool pair_bits_in_smem(int Nb) {
   return pair_base_smem_bytes(Nb) + Nb * ((Nb + 31) / 32) * 4 <= 227 * 1024;
 }
 
+// The pooled scores are computed in strips of 128 query blocks of one head
+// (pooled_scores_tc_kernel) into a buffer of whole strips, then selected
+// (select_kernel); the plan runs strip batches until every strip is done. The
+// buffer holds at most kPlanScoreBytes (or, in a fixed scratch, what is left),
+// and at least one strip.
+constexpr size_t kPlanScoreBytes = 64ull << 20;
+constexpr int kStripRows = 128;
+__host__ __device__ inline int score_ld(int Nb) { return (Nb + 31) & ~31; }   // floats per score row
+inline size_t score_strip_bytes(int Nb) { return static_cast<size_t>(kStripRows) * score_ld(Nb) * sizeof(float); }
+
 // Byte offsets of the plan workspace: pooled Q and K (fp32 [B,H,Nb,d]), then per
 // query block a 64-bit MinHash sort key and the kept set as a bitset of W words;
 // when the pairing's copy of the bitsets does not fit in shared memory, that copy,
-// word-major by sorted position ([B,H][W][Nb]).
+// word-major by sorted position ([B,H][W][Nb]); last the score strips (fp32
+// [strips][128][score_ld(Nb)]). score_cap bounds the strips' bytes (at least one
+// strip is always counted).
 struct PlanWorkspace {
-  size_t qp, kp, sig, bits, bitsT, total;
-  int W;
+  size_t qp, kp, sig, bits, bitsT, scores, total;
+  int W, strips, strips_per_batch;
 };
-inline PlanWorkspace plan_workspace(long long BH, int Nb, int D) {
+inline PlanWorkspace plan_workspace(long long BH, int Nb, int D, size_t score_cap = kPlanScoreBytes) {
   auto al = [](size_t x) { return (x + 255) / 256 * 256; };
   PlanWorkspace w;
   w.W = (Nb + 31) / 32;
@@ -54,7 +64,14 @@ inline PlanWorkspace plan_workspace(long long BH, int Nb, int D) {
   w.sig = 2 * pooled;
   w.bits = w.sig + al(static_cast<size_t>(BH) * Nb * sizeof(unsigned long long));
   w.bitsT = w.bits + bitset;
-  w.total = w.bitsT + (pair_bits_in_smem(Nb) ? 0 : bitset);
+  w.scores = w.bitsT + (pair_bits_in_smem(Nb) ? 0 : bitset);
+  const long long strips = BH * ((Nb + kStripRows - 1) / kStripRows);
+  const size_t sb = score_strip_bytes(Nb);
+  long long fit = static_cast<long long>(score_cap / sb);
+  fit = fit < 1 ? 1 : (fit > strips ? strips : fit);
+  w.strips = static_cast<int>(strips);
+  w.strips_per_batch = static_cast<int>(fit);
+  w.total = w.scores + al(static_cast<size_t>(fit) * sb);
   return w;
 }
 
@@ -589,163 +606,144 @@ static __device__ __forceinline__ void select_row(float* row, int Nb, int i, lon
 }
 
 // ----------------------------------------------------------------------------
-// Pooled scores + selection. One CTA = R query blocks of one head. tau is the
-// recall threshold of every head, or tau_bh[b*H + h] per head when tau_bh is given.
+// Pooled scores. One CTA = a 128 x 128 tile of
+//   L[i][j] = scale * <Qp_i, Kp_j>   (-inf for causal j > i)
+// of one head: query blocks 128 rt .. of strip (bh, rt), key blocks 128 ct ...
+// Every L[i][j] is one fp32 FMA chain over k = 0 .. D-1 in order, then the scale:
+// fp32 accumulation matters here, since the kept set near tau moves with the
+// scores' rounding (tcgen05 kind::tf32 with an exact three-way split of the
+// operands was measured at about ten times the error of these chains: its fp32
+// accumulation is coarser). Thread t (of 256) owns the 8 x 8 outputs rows
+// 8 (t / 16) .., columns 8 (t % 16) ..; the operands pass through shared memory
+// transposed (k-major) in 16-k slices, the next slice loading into registers while
+// the current one is used. The tile is stored into the strip buffer
+// scores[blockIdx.y][row][j] (row stride score_ld(Nb)). Grid (ceil(Nb/128) column
+// tiles, strips of the batch), 256 threads.
+template <int D>
+__global__ void __launch_bounds__(256, 2) pooled_scores_kernel(const float* __restrict__ Qp,
+                                                               const float* __restrict__ Kp, int Nb, float scale,
+                                                               int causal, int strip0, float* __restrict__ scores) {
+  constexpr int kK = 16;                       // k per slice
+  __shared__ __align__(16) float As[2][kK][128];
+  __shared__ __align__(16) float Bs[2][kK][128];
+  const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
+  const int nrt = (Nb + 127) / 128;
+  const int strip = strip0 + static_cast<int>(blockIdx.y);
+  const int bh = strip / nrt, rt = strip - bh * nrt, ct = static_cast<int>(blockIdx.x);
+  const float* qa = Qp + (static_cast<long long>(bh) * Nb + 128 * rt) * D;
+  const float* kb = Kp + (static_cast<long long>(bh) * Nb + 128 * ct) * D;
+  const int nq = min(128, Nb - 128 * rt), nk = min(128, Nb - 128 * ct);
+  // loads of a slice: thread t reads row t / 2 (0..127), k 8 (t % 2) .. +7 of both
+  // operands (two float4 each); zeros past the head's last block
+  const int lr = t >> 1, lk = (t & 1) * 8;
+  float4 ra[2], rb[2];
+  auto fetch = [&](int k0) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      ra[u] = lr < nq ? __ldg(reinterpret_cast<const float4*>(qa + static_cast<long long>(lr) * D + k0 + lk) + u)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+      rb[u] = lr < nk ? __ldg(reinterpret_cast<const float4*>(kb + static_cast<long long>(lr) * D + k0 + lk) + u)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  auto stash = [&](int buf) {                  // transposed: [k][row]
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float a4[4] = {ra[u].x, ra[u].y, ra[u].z, ra[u].w};
+      const float b4[4] = {rb[u].x, rb[u].y, rb[u].z, rb[u].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        As[buf][lk + 4 * u + e][lr] = a4[e];
+        Bs[buf][lk + 4 * u + e][lr] = b4[e];
+      }
+    }
+  };
+  float acc[8][8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
+  fetch(0);
+  stash(0);
+  __syncthreads();
+  for (int s = 0; s < D / kK; ++s) {
+    const int buf = s & 1;
+    if (s + 1 < D / kK) fetch((s + 1) * kK);   // in flight during this slice's FMAs
+#pragma unroll
+    for (int kk = 0; kk < kK; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][8 * ty]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][8 * ty + 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][8 * tx]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][8 * tx + 4]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
+    }
+    if (s + 1 < D / kK) {
+      stash(buf ^ 1);                          // the other buffer was last read a slice ago
+      __syncthreads();
+    }
+  }
+  const int ld = score_ld(Nb);
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int row = 8 * ty + r, i = 128 * rt + row;
+    if (i >= Nb) break;
+    float* dst = scores + (static_cast<long long>(blockIdx.y) * 128 + row) * ld + 128 * ct + 8 * tx;
+    const int j0 = 128 * ct + 8 * tx;
+    float v[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      v[c] = acc[r][c] * scale;
+      if (causal && j0 + c > i) v[c] = -INFINITY;
+    }
+    if (j0 + 8 <= Nb) {
+      reinterpret_cast<float4*>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
+      reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
+    } else {
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        if (j0 + c < Nb) dst[c] = v[c];
+    }
+  }
+}
+
+// Selection of 4 query blocks per CTA from the score strips, one warp per row
+// (phase 2 below): rows 4 blockIdx.x .. of strip strip0 + blockIdx.y, copied from
+// the strip buffer into shared memory (the search reads a row many times). Rows
+// of up to 256 blocks take the 8-way search, up to 64 the sorted prefix. Grid
+// (32, strips of the batch), 128 threads, 16 score_ld(Nb) bytes of shared memory.
+// tau is the recall threshold of every head, or tau_bh[b*H + h] per head when
+// tau_bh is given.
 //
-// Phase 1 (CUDA-core fp32 GEMM, the pooled scores must stay fp32 to keep the
-// kept set stable near tau): thread t owns key blocks c = 2t, 2t+1 of each
-// 2*NT-wide pass and all R rows; the R pooled query rows sit in shared memory
-// (transposed, read as broadcast float4), Kp rows stream from L2 in 32-byte
-// pieces. Scores go to shared memory: L[r][j] = scale * <Qp_r, Kp_j>, -inf for
-// causal j > i.
-//
-// With R = 4 (heads of up to 256 blocks) phase 1 instead stages 64 pooled key
-// rows at a time in shared memory with one coalesced round of loads and splits d
-// between two threads per key block, so all threads work and the L2 latency is
-// paid once per 64 key blocks rather than once per 8 dimensions.
-//
-// Phase 2 (one warp per row): e_j = exp(L_j - max), T = tau * sum e. The kept set
-// is {j : e_j > e*} plus the lowest-index ties at e* needed to reach T, where
+// Selection (one warp per row): e_j = exp(L_j - max), T = tau * sum e. The kept
+// set is {j : e_j > e*} plus the lowest-index ties at e* needed to reach T, where
 // e* is the largest value with sum_{e_j >= e*} e_j >= T. e* is found by searching
-// the IEEE bit pattern of e (monotone for non-negative floats): a bisection, or
-// with R = 4 an 8-way search (7 probes per step, about 10 steps instead of 30,
-// for short rows where the steps' shuffle latency dominates). Every probe sums in
-// the same order as the total, so the probe at 0 equals the total exactly, and
-// a probe's sum can only grow as the probe falls (rounded addition of non-negative
-// terms is monotone), so both searches find the same e*. This is the
-// sorted-prefix rule without sorting.
-template <int D, int R, int NT>
-__global__ void __launch_bounds__(NT) score_select_kernel(const float* __restrict__ Qp,
-                                                           const float* __restrict__ Kp, int Nb,
-                                                           float scale, int causal, float tau,
-                                                           const float* __restrict__ tau_bh,
-                                                           uint8_t* __restrict__ mask,
-                                                           int* __restrict__ count,
-                                                           int* __restrict__ idx,
-                                                           unsigned long long* __restrict__ sig,
-                                                           uint32_t* __restrict__ bits) {
-  static_assert(R % 4 == 0 && R <= 16 && NT % 32 == 0, "R rows per CTA, NT threads");
-  constexpr bool kSmall = R == 4;   // staged phase 1, 8-way search in phase 2
-  static_assert(!kSmall || NT == 128, "the staged phase 1 uses 128 threads");
-  constexpr int kCols = 2 * NT;  // key blocks per pass of phase 1
-  constexpr int QS = R + 4;  // padded row stride of the transposed query tile
-  extern __shared__ __align__(16) float sm[];
-  float* qT = sm;                          // [D][QS]
-  float* L = sm + D * QS;                  // [R][ldL]
-  const int ldL = (Nb + 3) & ~3;
-  const long long bh = blockIdx.y;
-  const int i0 = blockIdx.x * R;
-  const float* qp = Qp + bh * Nb * D;
-  const float* kp = Kp + bh * Nb * D;
-
-  for (int e = threadIdx.x; e < R * D; e += blockDim.x) {
-    const int r = e / D, k = e % D;
-    qT[k * QS + r] = (i0 + r < Nb) ? qp[static_cast<long long>(i0 + r) * D + k] : 0.f;
-  }
+// the IEEE bit pattern of e (monotone for non-negative floats): a bisection that
+// stops once one element lies between its bounds, or for short rows an 8-way
+// search (7 probes per step, about 10 steps instead of 30, where the steps'
+// shuffle latency dominates). Every probe sums in the same fixed order, so the
+// kept set does not depend on the search path.
+template <bool kShort>
+__global__ void __launch_bounds__(128) select_kernel(const float* __restrict__ scores, int Nb, int strip0, float tau,
+                                                     const float* __restrict__ tau_bh, uint8_t* __restrict__ mask,
+                                                     int* __restrict__ count, int* __restrict__ idx,
+                                                     unsigned long long* __restrict__ sig,
+                                                     uint32_t* __restrict__ bits) {
+  extern __shared__ __align__(16) float Lrows[];   // [4][ld]
+  const int ld = score_ld(Nb);
+  const int nrt = (Nb + 127) / 128;
+  const int strip = strip0 + static_cast<int>(blockIdx.y);
+  const long long bh = strip / nrt;
+  const int rt = strip - static_cast<int>(bh) * nrt;
+  const int r0 = 4 * static_cast<int>(blockIdx.x);          // first row within the strip
+  if (128 * rt + r0 >= Nb) return;
+  const float4* src = reinterpret_cast<const float4*>(scores + (static_cast<long long>(blockIdx.y) * 128 + r0) * ld);
+  for (int x = threadIdx.x; x < ld; x += 128) reinterpret_cast<float4*>(Lrows)[x] = src[x];   // 4 rows
   __syncthreads();
-
-  // ---------------- phase 1: scores
-  if constexpr (kSmall) {
-    float* kS = L + R * ldL;                    // [64][D + 1] staged key rows
-    float* red = kS + 64 * (D + 1);             // [2][R][64] half-d partial dots
-    const int c = threadIdx.x & 63, h = threadIdx.x >> 6;
-    for (int cb = 0; cb < Nb; cb += 64) {
-      const int ncols = min(64, Nb - cb);
-      for (int e = threadIdx.x; e < ncols * (D / 4); e += NT) {
-        const int r = e / (D / 4), c4 = e - r * (D / 4);
-        const float4 v = __ldg(reinterpret_cast<const float4*>(kp + static_cast<long long>(cb + r) * D) + c4);
-        float* dst = kS + r * (D + 1) + 4 * c4;
-        dst[0] = v.x;
-        dst[1] = v.y;
-        dst[2] = v.z;
-        dst[3] = v.w;
-      }
-      __syncthreads();
-      float acc[R];
-#pragma unroll
-      for (int r = 0; r < R; ++r) acc[r] = 0.f;
-      if (c < ncols) {
-        const float* kr = kS + c * (D + 1) + h * (D / 2);
-        const float* qh = qT + h * (D / 2) * QS;
-#pragma unroll 8
-        for (int d = 0; d < D / 2; ++d) {
-          const float kv = kr[d];
-          const float4 q = *reinterpret_cast<const float4*>(qh + d * QS);
-          acc[0] = fmaf(q.x, kv, acc[0]);
-          acc[1] = fmaf(q.y, kv, acc[1]);
-          acc[2] = fmaf(q.z, kv, acc[2]);
-          acc[3] = fmaf(q.w, kv, acc[3]);
-        }
-      }
-#pragma unroll
-      for (int r = 0; r < R; ++r) red[(h * R + r) * 64 + c] = acc[r];
-      __syncthreads();
-      if (h == 0 && c < ncols) {
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-          float v = (red[r * 64 + c] + red[(R + r) * 64 + c]) * scale;
-          if (causal && cb + c > i0 + r) v = -INFINITY;
-          L[r * ldL + cb + c] = v;
-        }
-      }
-      __syncthreads();                          // kS and red are reused by the next pass
-    }
-  } else {
-  for (int cb = 0; cb < Nb; cb += kCols) {
-    const int c0 = cb + 2 * threadIdx.x;
-    float acc0[R], acc1[R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) acc0[r] = acc1[r] = 0.f;
-    if (c0 < Nb) {
-      const bool has1 = c0 + 1 < Nb;
-      const float4* k0 = reinterpret_cast<const float4*>(kp + static_cast<long long>(c0) * D);
-      const float4* k1 = reinterpret_cast<const float4*>(kp + static_cast<long long>(has1 ? c0 + 1 : c0) * D);
-#pragma unroll 2
-      for (int k = 0; k < D; k += 8) {
-        float4 a[2], b[2];
-        a[0] = __ldg(k0 + k / 4);
-        a[1] = __ldg(k0 + k / 4 + 1);
-        b[0] = __ldg(k1 + k / 4);
-        b[1] = __ldg(k1 + k / 4 + 1);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const float av = reinterpret_cast<const float*>(a)[kk];
-          const float bv = reinterpret_cast<const float*>(b)[kk];
-          const float4* qrow = reinterpret_cast<const float4*>(qT + (k + kk) * QS);
-#pragma unroll
-          for (int r4 = 0; r4 < R / 4; ++r4) {
-            const float4 q = qrow[r4];
-            acc0[4 * r4 + 0] = fmaf(q.x, av, acc0[4 * r4 + 0]);
-            acc0[4 * r4 + 1] = fmaf(q.y, av, acc0[4 * r4 + 1]);
-            acc0[4 * r4 + 2] = fmaf(q.z, av, acc0[4 * r4 + 2]);
-            acc0[4 * r4 + 3] = fmaf(q.w, av, acc0[4 * r4 + 3]);
-            acc1[4 * r4 + 0] = fmaf(q.x, bv, acc1[4 * r4 + 0]);
-            acc1[4 * r4 + 1] = fmaf(q.y, bv, acc1[4 * r4 + 1]);
-            acc1[4 * r4 + 2] = fmaf(q.z, bv, acc1[4 * r4 + 2]);
-            acc1[4 * r4 + 3] = fmaf(q.w, bv, acc1[4 * r4 + 3]);
-          }
-        }
-      }
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const int i = i0 + r;
-        float v0 = acc0[r] * scale, v1 = acc1[r] * scale;
-        if (causal) {
-          if (c0 > i) v0 = -INFINITY;
-          if (c0 + 1 > i) v1 = -INFINITY;
-        }
-        if (has1) {
-          *reinterpret_cast<float2*>(L + r * ldL + c0) = make_float2(v0, v1);
-        } else {
-          L[r * ldL + c0] = v0;
-        }
-      }
-    }
-  }
-  }
-  __syncthreads();
-
-  // ---------------- phase 2: selection, one warp per row
   // the head's own tau when one is given per (b, h); an invalid one (not in (0, 1])
   // is recorded in the device error word and the head keeps every block
   if (tau_bh) {
@@ -756,26 +754,19 @@ __global__ void __launch_bounds__(NT) score_select_kernel(const float* __restric
     }
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int r = warp; r < R; r += NT / 32) {
-    const int i = i0 + r;
-    if (i >= Nb) break;
-    uint32_t* brow = bits ? bits + (bh * Nb + i) * static_cast<long long>((Nb + 31) / 32) : nullptr;
-    unsigned long long* srow = sig ? sig + bh * Nb + i : nullptr;
-    if (kSmall && Nb <= 64)
-      select_row_sorted64(L + r * ldL, Nb, i, bh, tau, lane, mask, count, idx, srow, brow);
-    else
-      select_row<kSmall>(L + r * ldL, Nb, i, bh, tau, lane, mask, count, idx, srow, brow);
-  }
+  const int i = 128 * rt + r0 + warp;
+  if (i >= Nb) return;
+  uint32_t* brow = bits ? bits + (bh * Nb + i) * static_cast<long long>((Nb + 31) / 32) : nullptr;
+  unsigned long long* srow = sig ? sig + bh * Nb + i : nullptr;
+  if (kShort && Nb <= 64)
+    select_row_sorted64(Lrows + warp * ld, Nb, i, bh, tau, lane, mask, count, idx, srow, brow);
+  else
+    select_row<kShort>(Lrows + warp * ld, Nb, i, bh, tau, lane, mask, count, idx, srow, brow);
 }
 
-// Dynamic shared memory of score_select_kernel<D, R, ...> for Nb blocks per head.
-template <int D, int R>
-inline int score_select_smem_bytes(int Nb) {
-  const int ldL = (Nb + 3) & ~3;
-  int floats = D * (R + 4) + R * ldL;
-  if (R == 4) floats += 64 * (D + 1) + 2 * R * 64;
-  return floats * static_cast<int>(sizeof(float));
-}
+// Dynamic shared memory of select_kernel for Nb blocks per head.
+inline int select_smem_bytes(int Nb) { return 4 * score_ld(Nb) * static_cast<int>(sizeof(float)); }
+
 
 // ----------------------------------------------------------------------------
 // Query-tile pairing and order. A 128-row query tile holds two 64-row query

@@ -1,7 +1,8 @@
-// Host-side launch sequence of stage 1 (pool -> pooled scores + selection ->
+// Host-side launch sequence of stage 1 (pool -> pooled scores -> selection ->
 // tile order), shared by the workspace entry points (sa_api.cu) and the
 // allocation-free one (sa_noalloc.cu): both pass a scratch region laid out by
-// plan_workspace and get the same kernels, grid shapes and shared-memory sizes.
+// plan_workspace and get the same kernels and arithmetic (only the number of
+// score strips per batch may differ, which changes no result).
 #pragma once
 
 #include <mutex>
@@ -23,49 +24,47 @@ inline sa_status set_smem(F* kernel, int bytes) {
 }
 
 // Stage 1 on the stream: pool Q and K (and, with Q8 given, write their 8-bit
-// codes in format qfmt and per-block scales), the pooled scores and the cumulative-energy selection
+// codes in format qfmt and per-block scales), the pooled scores in batches of
+// 128-block strips (pooled_scores_kernel) each followed by their selection
 // (mask, count, optional idx), then, with `work` given, the tile pairs and their
-// order. `scratch` holds plan_workspace(B*H, Nb, D).total bytes, 256-byte aligned.
-// tau_bh, when given, is a device array of one threshold per (b, h) that replaces tau.
+// order. `scratch` holds plan_workspace(B*H, Nb, D, score_cap).total bytes,
+// 256-byte aligned. tau_bh, when given, is a device array of one threshold per
+// (b, h) that replaces tau.
 template <int D>
 sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau, const float* tau_bh,
                       float scale, int causal, uint8_t* mask, int32_t* count, int32_t* idx, int32_t* work,
                       void* scratch, cudaStream_t st, uint8_t* Q8 = nullptr, uint8_t* K8 = nullptr,
-                      float* qscale = nullptr, float* kscale = nullptr, int qfmt = kScoreE4M3) {
+                      float* qscale = nullptr, float* kscale = nullptr, int qfmt = kScoreE4M3,
+                      size_t score_cap = kPlanScoreBytes) {
   const int Nb = static_cast<int>((static_cast<int64_t>(s.N) + 63) / 64);
   const long long BH = static_cast<long long>(s.B) * s.H;
-  const PlanWorkspace L = plan_workspace(BH, Nb, D);
+  const PlanWorkspace L = plan_workspace(BH, Nb, D, score_cap);
   char* wsb = static_cast<char*>(scratch);
   float* Qp = reinterpret_cast<float*>(wsb + L.qp);
   float* Kp = reinterpret_cast<float*>(wsb + L.kp);
   unsigned long long* sig = reinterpret_cast<unsigned long long*>(wsb + L.sig);
   uint32_t* bits = reinterpret_cast<uint32_t*>(wsb + L.bits);
   uint32_t* bitsT = pair_bits_in_smem(Nb) ? nullptr : reinterpret_cast<uint32_t*>(wsb + L.bitsT);
+  float* scores = reinterpret_cast<float*>(wsb + L.scores);
   pool_kernel<D><<<dim3(static_cast<unsigned>(BH * Nb), 2), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), Qp, Kp, s.N, Nb, Q8, K8, qscale,
       kscale, qfmt);
   if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
 
-  // R query blocks per CTA: 4 for short heads so that the grid still fills the GPU.
-  auto launch_ss = [&](auto kern, int R, int NT) -> sa_status {
-    const int smem = R == 4 ? score_select_smem_bytes<D, 4>(Nb)
-                            : (R == 8 ? score_select_smem_bytes<D, 8>(Nb) : score_select_smem_bytes<D, 16>(Nb));
-    if (set_smem(kern, smem) != SA_OK) return SA_ERR_CUDA;
-    kern<<<dim3((Nb + R - 1) / R, static_cast<unsigned>(BH)), NT, smem, st>>>(Qp, Kp, Nb, scale, causal, tau,
-                                                                               tau_bh, mask, count, idx, sig, bits);
-    return SA_OK;
-  };
-  sa_status ls;
-  if (Nb <= 256)
-    ls = launch_ss(score_select_kernel<D, 4, 128>, 4, 128);
-  else if (Nb <= 1536)
-    ls = launch_ss(score_select_kernel<D, 16, 256>, 16, 256);
-  else if (Nb <= 3000)   // 16 warps: a row per warp in the selection, two-pass score rows
-    ls = launch_ss(score_select_kernel<D, 16, 512>, 16, 512);
-  else
-    ls = launch_ss(score_select_kernel<D, 8, 256>, 8, 256);
-  if (ls != SA_OK) return ls;
-  if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+  const bool shortrows = Nb <= 256;
+  const int ssm = select_smem_bytes(Nb);
+  if (set_smem(shortrows ? select_kernel<true> : select_kernel<false>, ssm) != SA_OK) return SA_ERR_CUDA;
+  const unsigned nct = static_cast<unsigned>((Nb + 127) / 128);
+  for (int s0 = 0; s0 < L.strips; s0 += L.strips_per_batch) {
+    const unsigned ns = static_cast<unsigned>(min(L.strips_per_batch, L.strips - s0));
+    pooled_scores_kernel<D><<<dim3(nct, ns), 256, 0, st>>>(Qp, Kp, Nb, scale, causal, s0, scores);
+    if (shortrows)
+      select_kernel<true><<<dim3(32, ns), 128, ssm, st>>>(scores, Nb, s0, tau, tau_bh, mask, count, idx, sig, bits);
+    else
+      select_kernel<false><<<dim3(32, ns), 128, ssm, st>>>(scores, Nb, s0, tau, tau_bh, mask, count, idx, sig,
+                                                           bits);
+    if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+  }
 
   if (work) {
     const int Tq = (Nb + 1) / 2;

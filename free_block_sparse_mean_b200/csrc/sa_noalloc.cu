@@ -11,13 +11,13 @@
 //
 // Scratch: kNoAllocScratchBytes = 32 MiB, a file-scope __device__ array. Every
 // GPU that loads the library holds it until the process exits. A call needs the
-// same bytes as sparse_attn_plan_workspace_size: the pooled Q and K
-// (2 * B*H*ceil(N/64)*d*4 bytes) plus, per query block, an 8-byte sort key and a
+// fixed regions of sparse_attn_plan_workspace_size (the pooled Q and K,
+// 2 * B*H*ceil(N/64)*d*4 bytes, plus, per query block, an 8-byte sort key and a
 // ceil(Nb/32)-word bitset of its kept set, and, above about 1,200 blocks per
-// head (where the pairing's copy of the bitsets no longer fits in shared memory),
-// that copy (for example H=24, d=128 fits up to N = 75,776). Larger calls are
-// rejected with SA_ERR_WORKSPACE before
-// anything runs.
+// head, the pairing's copy of the bitsets) and room for at least one strip of
+// pooled scores (128 rows of ceil(Nb/32)*32 floats); the strips take whatever is
+// left (for example H=24, d=128 fits up to N = 74,432). Larger calls are rejected
+// with SA_ERR_WORKSPACE before anything runs.
 //
 // Every call shares the one array, and the array keeps the last call's
 // contents. The kernels write every scratch byte they later read, so nothing
@@ -98,14 +98,19 @@ extern "C" sa_status sparse_attn_plan_noalloc(const void* Q, const void* K, sa_s
   if (!(tau > 0.f && tau <= 1.f)) return SA_ERR_INVALID_ARG;
   if (!(std::isfinite(scale) && scale > 0.f)) return SA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(Q) & 15u) || (reinterpret_cast<uintptr_t>(K) & 15u)) return SA_ERR_INVALID_ARG;
-  const sa::PlanWorkspace need = sa::plan_workspace(static_cast<long long>(s.B) * s.H,
-                                                    static_cast<int>((static_cast<int64_t>(s.N) + 63) / 64), s.d);
-  if (need.total > kNoAllocScratchBytes) return SA_ERR_WORKSPACE;  // beyond the fixed scratch
+  // the fixed regions and one score strip must fit; the strips then take the rest
+  const long long BH = static_cast<long long>(s.B) * s.H;
+  const int Nb = static_cast<int>((static_cast<int64_t>(s.N) + 63) / 64);
+  const sa::PlanWorkspace least = sa::plan_workspace(BH, Nb, s.d, 0);
+  if (least.total > kNoAllocScratchBytes) return SA_ERR_WORKSPACE;  // beyond the fixed scratch
+  const size_t score_cap = kNoAllocScratchBytes - least.scores;
   void* scratch = nullptr;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const sa_status got = scratch_for_current_device(st, &scratch);
   if (got != SA_OK) return got;
   if (s.d == 64)
-    return sa::launch_plan<64>(s, Q, K, tau, nullptr, scale, causal != 0, mask, count, idx, work, scratch, st);
-  return sa::launch_plan<128>(s, Q, K, tau, nullptr, scale, causal != 0, mask, count, idx, work, scratch, st);
+    return sa::launch_plan<64>(s, Q, K, tau, nullptr, scale, causal != 0, mask, count, idx, work, scratch, st,
+                               nullptr, nullptr, nullptr, nullptr, sa::kScoreE4M3, score_cap);
+  return sa::launch_plan<128>(s, Q, K, tau, nullptr, scale, causal != 0, mask, count, idx, work, scratch, st,
+                              nullptr, nullptr, nullptr, nullptr, sa::kScoreE4M3, score_cap);
 }

@@ -47,16 +47,25 @@ def test_workspace_and_tiles(lib):
     s = SaShape(1, 40, 75600, 128, 64)
     Nb = math.ceil(75600 / 64)
     al = lambda x: (x + 255) // 256 * 256
+
+    def strips(BH, Nb):   # score strips of 128 rows of ceil(Nb/32)*32 floats, at most 64 MiB of them
+        sb = 128 * ((Nb + 31) // 32 * 32) * 4
+        return al(max(1, min(BH * math.ceil(Nb / 128), (64 << 20) // sb)) * sb)
+
     W = (Nb + 31) // 32
     # pooled Q and K, sort keys and bitsets (1182 blocks per head: the pairing keeps
-    # its copy of the bitsets in shared memory)
-    expect = 2 * al(40 * Nb * 128 * 4) + al(40 * Nb * 8) + al(40 * Nb * W * 4)
+    # its copy of the bitsets in shared memory), then the score strips
+    expect = 2 * al(40 * Nb * 128 * 4) + al(40 * Nb * 8) + al(40 * Nb * W * 4) + strips(40, Nb)
     assert lib.sparse_attn_plan_workspace_size(s) == expect
     big = SaShape(1, 24, 118800, 128, 64)                         # 1857 blocks: a global copy too
     Nb2 = math.ceil(118800 / 64)
     W2 = (Nb2 + 31) // 32
     assert lib.sparse_attn_plan_workspace_size(big) == (2 * al(24 * Nb2 * 128 * 4) + al(24 * Nb2 * 8)
-                                                        + 2 * al(24 * Nb2 * W2 * 4))
+                                                        + 2 * al(24 * Nb2 * W2 * 4) + strips(24, Nb2))
+    tiny = SaShape(1, 1, 1000, 64, 64)                            # one strip of one head
+    Nb3 = math.ceil(1000 / 64)
+    assert lib.sparse_attn_plan_workspace_size(tiny) == (2 * al(Nb3 * 64 * 4) + al(Nb3 * 8) + al(Nb3 * 4)
+                                                         + al(128 * 32 * 4))
     assert lib.sparse_attn_num_tiles(s) == 40 * ((Nb + 1) // 2)
     assert lib.sparse_attn_num_tiles(SaShape(2, 3, 1, 64, 64)) == 6
     for bad in (SaShape(1, 1, 64, 96, 64), SaShape(1, 1, 64, 128, 32), SaShape(0, 1, 64, 128, 64),
