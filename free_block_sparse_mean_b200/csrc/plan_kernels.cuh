@@ -613,33 +613,38 @@ static __device__ __forceinline__ void select_row(float* row, int Nb, int i, lon
 // fp32 accumulation matters here, since the kept set near tau moves with the
 // scores' rounding (tcgen05 kind::tf32 with an exact three-way split of the
 // operands was measured at about ten times the error of these chains: its fp32
-// accumulation is coarser). Thread t (of 256) owns the 8 x 8 outputs rows
-// 8 (t / 16) .., columns 8 (t % 16) ..; the operands pass through shared memory
-// transposed (k-major) in 16-k slices, the next slice loading into registers while
-// the current one is used. The tile is stored into the strip buffer
-// scores[blockIdx.y][row][j] (row stride score_ld(Nb)). Grid (ceil(Nb/128) column
-// tiles, strips of the batch), 256 threads.
-template <int D>
+// accumulation is coarser). With kT = 128, thread t (of 256) owns the 8 x 8
+// outputs rows 8 (t / 16) .., columns 8 (t % 16) ..; heads of at most 64 blocks take
+// kT = 64 tiles (4 x 4 outputs per thread), which gives the same chains. The
+// operands pass through shared memory transposed (k-major) in 16-k slices, the next
+// slice loading into registers while the current one is used. The tile is stored
+// into the strip buffer scores[blockIdx.y][row][j] (row stride score_ld(Nb)). Grid
+// (ceil(Nb/kT) column tiles, strips of the batch), 256 threads.
+template <int D, int kT = 128>
 __global__ void __launch_bounds__(256, 2) pooled_scores_kernel(const float* __restrict__ Qp,
                                                                const float* __restrict__ Kp, int Nb, float scale,
                                                                int causal, int strip0, float* __restrict__ scores) {
+  static_assert(kT == 128 || kT == 64, "tile of 128 or 64 blocks");
   constexpr int kK = 16;                       // k per slice
-  __shared__ __align__(16) float As[2][kK][128];
-  __shared__ __align__(16) float Bs[2][kK][128];
+  constexpr int kO = kT / 16;                  // outputs per thread along each side
+  constexpr int kV = kT / 64;                  // float4 loads per operand and slice per thread
+  __shared__ __align__(16) float As[2][kK][kT];
+  __shared__ __align__(16) float Bs[2][kK][kT];
   const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
   const int nrt = (Nb + 127) / 128;
   const int strip = strip0 + static_cast<int>(blockIdx.y);
   const int bh = strip / nrt, rt = strip - bh * nrt, ct = static_cast<int>(blockIdx.x);
+  // kT = 64 serves heads of at most 64 blocks: one row tile (rt = 0) and one column tile
   const float* qa = Qp + (static_cast<long long>(bh) * Nb + 128 * rt) * D;
-  const float* kb = Kp + (static_cast<long long>(bh) * Nb + 128 * ct) * D;
-  const int nq = min(128, Nb - 128 * rt), nk = min(128, Nb - 128 * ct);
-  // loads of a slice: thread t reads row t / 2 (0..127), k 8 (t % 2) .. +7 of both
-  // operands (two float4 each); zeros past the head's last block
-  const int lr = t >> 1, lk = (t & 1) * 8;
-  float4 ra[2], rb[2];
+  const float* kb = Kp + (static_cast<long long>(bh) * Nb + kT * ct) * D;
+  const int nq = min(kT, Nb - 128 * rt), nk = min(kT, Nb - kT * ct);
+  // loads of a slice: thread t reads row t / (256 / kT) of both operands, kV float4s
+  // of k from 4 kV (t % (256 / kT)); zeros past the head's last block
+  const int lr = t / (256 / kT), lk = (t % (256 / kT)) * 4 * kV;
+  float4 ra[kV], rb[kV];
   auto fetch = [&](int k0) {
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < kV; ++u) {
       ra[u] = lr < nq ? __ldg(reinterpret_cast<const float4*>(qa + static_cast<long long>(lr) * D + k0 + lk) + u)
                       : make_float4(0.f, 0.f, 0.f, 0.f);
       rb[u] = lr < nk ? __ldg(reinterpret_cast<const float4*>(kb + static_cast<long long>(lr) * D + k0 + lk) + u)
@@ -648,7 +653,7 @@ __global__ void __launch_bounds__(256, 2) pooled_scores_kernel(const float* __re
   };
   auto stash = [&](int buf) {                  // transposed: [k][row]
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < kV; ++u) {
       const float a4[4] = {ra[u].x, ra[u].y, ra[u].z, ra[u].w};
       const float b4[4] = {rb[u].x, rb[u].y, rb[u].z, rb[u].w};
 #pragma unroll
@@ -658,11 +663,11 @@ __global__ void __launch_bounds__(256, 2) pooled_scores_kernel(const float* __re
       }
     }
   };
-  float acc[8][8];
+  float acc[kO][kO];
 #pragma unroll
-  for (int r = 0; r < 8; ++r)
+  for (int r = 0; r < kO; ++r)
 #pragma unroll
-    for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
+    for (int c = 0; c < kO; ++c) acc[r][c] = 0.f;
   fetch(0);
   stash(0);
   __syncthreads();
@@ -671,16 +676,24 @@ __global__ void __launch_bounds__(256, 2) pooled_scores_kernel(const float* __re
     if (s + 1 < D / kK) fetch((s + 1) * kK);   // in flight during this slice's FMAs
 #pragma unroll
     for (int kk = 0; kk < kK; ++kk) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][8 * ty]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][8 * ty + 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][8 * tx]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][8 * tx + 4]);
-      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      float av[kO], bv[kO];
 #pragma unroll
-      for (int r = 0; r < 8; ++r)
+      for (int h = 0; h < kO / 4; ++h) {
+        const float4 a = *reinterpret_cast<const float4*>(&As[buf][kk][kO * ty + 4 * h]);
+        const float4 b = *reinterpret_cast<const float4*>(&Bs[buf][kk][kO * tx + 4 * h]);
+        av[4 * h] = a.x;
+        av[4 * h + 1] = a.y;
+        av[4 * h + 2] = a.z;
+        av[4 * h + 3] = a.w;
+        bv[4 * h] = b.x;
+        bv[4 * h + 1] = b.y;
+        bv[4 * h + 2] = b.z;
+        bv[4 * h + 3] = b.w;
+      }
 #pragma unroll
-        for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
+      for (int r = 0; r < kO; ++r)
+#pragma unroll
+        for (int c = 0; c < kO; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
     }
     if (s + 1 < D / kK) {
       stash(buf ^ 1);                          // the other buffer was last read a slice ago
@@ -689,23 +702,24 @@ __global__ void __launch_bounds__(256, 2) pooled_scores_kernel(const float* __re
   }
   const int ld = score_ld(Nb);
 #pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    const int row = 8 * ty + r, i = 128 * rt + row;
+  for (int r = 0; r < kO; ++r) {
+    const int row = kO * ty + r, i = 128 * rt + row;
     if (i >= Nb) break;
-    float* dst = scores + (static_cast<long long>(blockIdx.y) * 128 + row) * ld + 128 * ct + 8 * tx;
-    const int j0 = 128 * ct + 8 * tx;
-    float v[8];
+    const int j0 = kT * ct + kO * tx;
+    float* dst = scores + (static_cast<long long>(blockIdx.y) * 128 + row) * ld + j0;
+    float v[kO];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < kO; ++c) {
       v[c] = acc[r][c] * scale;
       if (causal && j0 + c > i) v[c] = -INFINITY;
     }
-    if (j0 + 8 <= Nb) {
-      reinterpret_cast<float4*>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
-      reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
+    if (j0 + kO <= Nb) {
+#pragma unroll
+      for (int h = 0; h < kO / 4; ++h)
+        reinterpret_cast<float4*>(dst)[h] = make_float4(v[4 * h], v[4 * h + 1], v[4 * h + 2], v[4 * h + 3]);
     } else {
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
+      for (int c = 0; c < kO; ++c)
         if (j0 + c < Nb) dst[c] = v[c];
     }
   }

@@ -57,7 +57,10 @@ sa_status launch_plan(const sa_shape& s, const void* Q, const void* K, float tau
   const unsigned nct = static_cast<unsigned>((Nb + 127) / 128);
   for (int s0 = 0; s0 < L.strips; s0 += L.strips_per_batch) {
     const unsigned ns = static_cast<unsigned>(min(L.strips_per_batch, L.strips - s0));
-    pooled_scores_kernel<D><<<dim3(nct, ns), 256, 0, st>>>(Qp, Kp, Nb, scale, causal, s0, scores);
+    if (Nb <= 64)   // one 64-block tile per head
+      pooled_scores_kernel<D, 64><<<dim3(1, ns), 256, 0, st>>>(Qp, Kp, Nb, scale, causal, s0, scores);
+    else
+      pooled_scores_kernel<D, 128><<<dim3(nct, ns), 256, 0, st>>>(Qp, Kp, Nb, scale, causal, s0, scores);
     if (shortrows)
       select_kernel<true><<<dim3(32, ns), 128, ssm, st>>>(scores, Nb, s0, tau, tau_bh, mask, count, idx, sig, bits);
     else
