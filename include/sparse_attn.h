@@ -62,9 +62,11 @@ typedef struct {
 
 /* Bytes of device workspace sparse_attn_plan needs for shape s: pooled Q and K
  * (fp32 [B,H,Nb,d] each), an 8-byte sort key and a ceil(Nb/32)-word kept-set
- * bitset per query block, and, above about 1,200 blocks per head (where the
- * pairing's copy of the bitsets no longer fits in shared memory), that copy; each
- * region 256-byte aligned. 0 if the shape is invalid. */
+ * bitset per query block, above about 1,200 blocks per head (where the pairing's
+ * copy of the bitsets no longer fits in shared memory) that copy, and the pooled
+ * scores of as many 128-query-block strips (128 rows of ceil(Nb/32)*32 floats) as
+ * fit in 64 MiB, at least one (the plan computes and selects the strips batch by
+ * batch); each region 256-byte aligned. 0 if the shape is invalid. */
 size_t sparse_attn_plan_workspace_size(sa_shape s);
 
 /* Number of 128-row query tiles, B*H*ceil(Nb/2); `work` holds two entries per
@@ -336,12 +338,13 @@ sa_status sparse_attn_permute_rows(const void* src, const int32_t* perm, sa_shap
  * whose host owns the allocator, a latency-critical path that must not call
  * cudaMalloc). The paper has no counterpart: this is a deployment variant.
  *
- * Same arguments, outputs and errors as sparse_attn_plan, minus the workspace.
- * Its scratch (the same bytes sparse_attn_plan_workspace_size reports) goes to a
- * fixed 32 MiB device array inside the library, held by every GPU that loads the
- * library until the process exits; the call fits when that size is <= 32 MiB
- * (e.g. H=24, d=128 up to N = 75,776) and returns SA_ERR_WORKSPACE (nothing
- * launched) otherwise. It calls no allocator. The first call on a device looks up the
+ * Same arguments, outputs and errors as sparse_attn_plan, minus the workspace,
+ * and the same results. Its scratch goes to a fixed 32 MiB device array inside
+ * the library, held by every GPU that loads the library until the process exits:
+ * the regions sparse_attn_plan_workspace_size counts, with as many score strips as
+ * the array leaves room for. The call fits when the other regions and one strip
+ * fit in 32 MiB (e.g. H=24, d=128 up to N = 74,432) and returns SA_ERR_WORKSPACE
+ * (nothing launched) otherwise. It calls no allocator. The first call on a device looks up the
  * array's device address and caches it; make that first call before any stream
  * capture on the device. All calls share the array (it keeps the last call's
  * contents, and nothing in it needs to start at zero), so calls that overlap on
