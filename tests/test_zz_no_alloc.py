@@ -36,8 +36,10 @@ def test_noalloc_plan_matches_workspace_plan_twice():
     lib = _lib.load()
     dev = torch.device("cuda:0")
     stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
-    # Nb = 47 and 18 (the 4-row selection CTA), 313 (16 rows) and 3125 (8 rows, and
-    # pairing by consecutive blocks above 1024), all within the fixed scratch
+    # Nb = 47 and 18 (64-block score tiles), 313 and 3125 blocks, all within the fixed
+    # scratch; at Nb = 3125 the two calls compute and select the score strips in
+    # different batch counts (the workspace holds 40 strips, the fixed scratch about
+    # 14), which must not change any output
     cases = [(1, 4, 3000, 128, False, 0.95, 1), (2, 3, 1100, 64, True, 0.9, 2),
              (1, 2, 20000, 64, False, 0.9, 3), (1, 2, 200000, 64, False, 0.95, 4)]
     for B, H, N, d, causal, tau, seed in cases:
