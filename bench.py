@@ -119,6 +119,16 @@ def measured_traffic(w, tau, lam, qk="bf16", recall=None, centroid_weight=None):
     return None if ent is None else float(ent["total"])
 
 
+def plan_batches(BH, Nb):
+    """Strip batches of one plan call: the pooled scores are computed and selected in
+    strips of 128 query blocks, as many per batch as fit in 64 MiB (at least one),
+    as the library lays out its workspace."""
+    strips = BH * ((Nb + 127) // 128)
+    strip_bytes = 128 * ((Nb + 31) // 32 * 32) * 4
+    per = max(1, min(strips, (64 << 20) // strip_bytes))
+    return (strips + per - 1) // per
+
+
 def dense_flops(w):
     if w.causal:
         return 2.0 * w.B * w.H * w.N * (w.N + 1) * w.D
@@ -402,8 +412,10 @@ def run_ours(args, w, world, rank, local, pg):
             sa.sparse_attn_permute_rows(os_, cq.perm, inverse=True, out=out)
         # kernels per step: per clustering 4, then 8 per iteration less the last
         # iteration's centroid pass (with none, the 4 kernels of the order), 3 row moves,
-        # 3 plan kernels, the forward, the move back
-        launches_per_step = 2 * (4 + (8 * cl - 1 if cl > 0 else 4)) + 3 + 3 + 1 + 1
+        # the plan (pool, a score and a selection kernel per strip batch, the pairing),
+        # the forward, the move back
+        plan_launches = 2 + 2 * plan_batches(w.B * w.H, -(-w.N // 64))
+        launches_per_step = 2 * (4 + (8 * cl - 1 if cl > 0 else 4)) + 3 + plan_launches + 1 + 1
     else:
         def run_plan():
             sa.sparse_attn_plan(q, k, args.tau, None, w.causal, out=plan, workspace=ws, with_idx=False,
@@ -412,7 +424,9 @@ def run_ours(args, w, world, rank, local, pg):
         def run_fwd(stats=None):
             sa.sparse_attn_fwd(q, k, v, plan, lam, out=out, stats=stats, qk_fp8=q8 and not i8, qk_int8=i8,
                                recall=rec)
-        launches_per_step = 4
+        # the plan (pool, a score and a selection kernel per strip batch, the pairing)
+        # and the forward
+        launches_per_step = 2 + 2 * plan_batches(w.B * w.H, -(-w.N // 64)) + 1
 
     def step():
         run_plan()
