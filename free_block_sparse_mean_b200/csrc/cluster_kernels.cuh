@@ -5,32 +5,32 @@
 // interaction rather than by feature similarity, and reduces the objective to a
 // quadratic form. Replacing a token x by a centroid c changes its score with
 // every token y of the other side by (x - c).y; the sum of the squares is
-// (x - c)^T G (x - c) with G = sum_y y y^T. Dropping the term x^T G x, which is
+// (x - c)^T G (x - c) with G = sum_y y y^T (gram_tc_kernel and gram_reduce_kernel,
+// on the tensor cores with fp32 accumulation). Dropping the term x^T G x, which is
 // the same for every centroid, the nearest centroid is the argmin over c of
 // c^T G c - 2 x . (G c). So each Lloyd iteration is: w_c = G c and b_c = c . w_c
 // per centroid (cluster_prep_kernel), an argmin over all centroids per token (a
 // tensor-core product of the bf16 tokens with the w_c split into bf16 high and
 // low parts that keeps each token's four best, cluster_assign_tc_kernel, then
-// their exact fp32 scores, cluster_rescore_kernel), and the mean of each cluster's tokens
-// (cluster_centroid_kernel). The
-// clusters start at the 64-token block means (the pooling kernel), so zero
-// iterations reproduce the plain blocks.
+// their exact fp32 scores, cluster_rescore_kernel), and the mean of each
+// cluster's tokens (cluster_centroid_kernel). The clusters start at the 64-token
+// block means (the pooling kernel), so zero iterations reproduce the plain blocks.
 //
 // The reordering is a stable sort of the tokens by cluster: a per-head
 // exclusive scan of the cluster sizes gives each cluster's first position, and
 // each cluster's tokens follow in token order. Clusters are packed back to back,
 // so the tail of one shares a 64-token block with the head of the next (the
-// abstract's "tail merging", with no padding at all).
+// abstract's tail merging, with no padding at all).
 //
 // Each iteration: cluster_prep_kernel (w_c, b_c, their bf16 operand rows; clears
 // the sizes), cluster_assign_tc_kernel and cluster_rescore_kernel (argmin; counts
-// the sizes), cluster_offsets_kernel (each
-// cluster's first position), the stable order (cluster_chunk_count_kernel,
-// cluster_chunk_scan_kernel, cluster_order_kernel) and
-// cluster_centroid_kernel (each cluster's mean, summed over its tokens in token
-// order through the order just built). Everything is deterministic: every fp32
-// sum runs in a fixed order, the sizes are integer counts, and argmin ties go to
-// the lowest cluster index.
+// the sizes), cluster_offsets_kernel (each cluster's first position), the stable
+// order (cluster_chunk_count_kernel, cluster_chunk_scan_kernel,
+// cluster_order_kernel) and cluster_centroid_kernel (each cluster's mean, summed
+// over its tokens in token order through the order just built; the last
+// iteration skips it unless the centroids are returned). Everything is
+// deterministic: every fp32 sum runs in a fixed order, the sizes are integer
+// counts, and argmin ties go to the lowest cluster index.
 #pragma once
 
 #include "sa_device.cuh"
